@@ -1,0 +1,82 @@
+"""The oracle's pins must be able to fail.  Each case plants one plausible
+mistake (a transposed operand, a wrong sign or index, a dropped term) in a
+copy of ``oracle.c``, compiles it on the CPU, swaps it in, and checks that at
+least one pin from ``test_oracle_pins`` now fails.  CPU only."""
+import ctypes
+import os
+import subprocess
+
+import pytest
+
+import oracle
+from tests import test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
+
+# (name, original text, mutated text)
+MUTATIONS = [
+    ("B_for_C_in_update", "h[n] = a * h[n] + delta * Brow[n * L + t] * u[t];",
+     "h[n] = a * h[n] + delta * Crow[n * L + t] * u[t];"),
+    ("decay_sign", "double a = exp(delta * A[d * N + n]);", "double a = exp(-delta * A[d * N + n]);"),
+    ("drop_skip_term", "y += (Dv ? Dv[d] : 0.0) * u[t];", "(void)Dv;"),
+    ("history_index", "xin[k] = hist_w ? hist_w[k + 1] : 0.0;", "xin[k] = hist_w ? hist_w[k] : 0.0;"),
+    ("flipped_taps", "acc += w[k] * xin[t + k];", "acc += w[W - 1 - k] * xin[t + k];"),
+    ("softplus_formula", "return log1p(exp(v));", "return exp(v);"),
+    ("gate_added", "if (z) y *= o_silu(z[row * L + t]);", "if (z) y += o_silu(z[row * L + t]);"),
+    ("dt_bias_dropped_scan", "double v = dt[row * L + t] + (dt_bias ? dt_bias[d] : 0.0);",
+     "double v = dt[row * L + t];"),
+    ("h0_ignored", "for (n = 0; n < N; ++n) h[n] = h0 ? h0[row * N + n] : 0.0;",
+     "for (n = 0; n < N; ++n) h[n] = 0.0;"),
+    ("group_index_scan", "const int64_t g = d / (D / G);", "const int64_t g = d % G;"),
+    ("ssu_roll_direction", "for (k = 0; k < W - 1; ++k) cs[k] = cs[k + 1];",
+     "for (k = W - 2; k >= 0; --k) cs[k + 1] = cs[k];"),
+    ("ssu_decay_sign", "double a = exp(delta * A[hp * N + n]);", "double a = exp(delta * A[hp * N + n] * 0.5);"),
+    ("ssu_skip_dropped", "y += (Dv ? Dv[hp] : 0.0) * u;", "(void)Dv;"),
+    ("ssu_state_written_late", "s[n] = a * s[n] + delta * Bv[n] * u;\n                    y += Cv[n] * s[n];",
+     "y += Cv[n] * s[n];\n                    s[n] = a * s[n] + delta * Bv[n] * u;"),
+    ("mamba2_group_index", "const double* Bv = Bm + (b * G + hh / heads_per_group) * N;",
+     "const double* Bv = Bm + (b * G + hh % G) * N;"),
+    ("mamba2_skip_uses_state", "if (D_head) y += D_head[hh] * xv;", "if (D_head) y += D_head[hh] * s[0];"),
+    ("conv_state_out_shift", "for (k = 0; k < W; ++k) hist_out[k] = all[L + k];",
+     "for (k = 0; k < W; ++k) hist_out[k] = all[L + k - (k > 0)];"),
+]
+
+# pins exercised against each mutant (all cheap)
+PIN_CALLS = [
+    lambda: pins.test_scan_matches_brute_force(2, 2, 3, 8, 4, 1, 4),
+    lambda: pins.test_scan_matches_brute_force(3, 1, 3, 7, 2, 3, 3),
+    lambda: pins.test_scan_matches_brute_force(4, 2, 2, 3, 4, 2, 4),
+    lambda: pins.test_scan_matches_brute_force(6, 1, 4, 5, 2, 2, 4),
+    lambda: pins.test_scan_closed_form_constant_inputs(-0.7),
+    lambda: pins.test_prefill_then_decode_equals_full_prefill(3),
+    lambda: pins.test_ssu_single_step_matches_scan_brute_force_with_groups(),
+    lambda: pins.test_mamba2_notation_matches_general_form(2),
+    lambda: pins.test_mamba2_groups_map_consecutive_heads(),
+    lambda: pins.test_conv_matches_numpy_convolve_and_state(7),
+    lambda: pins.test_conv_matches_numpy_convolve_and_state(2),
+    lambda: pins.test_conv_impulse_response(4),
+    lambda: pins.test_activation_special_values(),
+]
+
+
+@pytest.mark.parametrize("name,orig,mut", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_planted_mistake_is_caught(name, orig, mut, tmp_path):
+    src = open(SRC).read()
+    assert src.count(orig) == 1, f"mutation anchor for {name} not found exactly once"
+    path = tmp_path / f"{name}.c"
+    path.write_text(src.replace(orig, mut))
+    lib_path = tmp_path / f"lib{name}.so"
+    subprocess.check_call(["gcc", "-O2", "-std=c99", "-shared", "-fPIC", str(path), "-o",
+                           str(lib_path), "-lm"])
+    saved = oracle._load()
+    oracle._lib = oracle.configure(ctypes.CDLL(str(lib_path)))
+    failures = 0
+    try:
+        for call in PIN_CALLS:
+            try:
+                call()
+            except AssertionError:
+                failures += 1
+    finally:
+        oracle._lib = saved
+    assert failures > 0, f"no pin caught the planted mistake {name}"

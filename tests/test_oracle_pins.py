@@ -1,0 +1,340 @@
+"""Pins for the fp64 oracle: each check ties the oracle to something other than
+itself -- a brute-force direct sum, a closed form, a library routine, or an
+invariant of the method -- so that a dropped term, a wrong sign or index, or a
+transposed operand in ``oracle.c`` fails at least one test.  CPU only.
+"""
+import math
+
+import numpy as np
+import pytest
+from scipy.special import expit
+
+import oracle
+from state_space_model_causal_b200 import inputs as gen
+
+
+def _silu_ref(v):
+    # logistic from scipy, not the oracle's 1/(1+exp(-v))
+    return v * expit(v)
+
+
+def _softplus_ref(v):
+    return np.logaddexp(0.0, v)
+
+
+def _conv_ref(x_row, w, bias, hist):
+    """Causal cross-correlation through numpy.convolve: w[W-1] multiplies the
+    current token, history (last W raw values, oldest first) pads the left."""
+    W = len(w)
+    if len(x_row) == 0:
+        return np.zeros(0)
+    padded = np.concatenate([hist[1:] if W > 1 else hist[:0], x_row])
+    return np.convolve(padded, w[::-1], mode="valid") + bias
+
+
+def _brute_force_scan(x, dt, A, Bm, Cm, Dv, z, dt_bias, softplus, cw, cb, cs, h0):
+    """Direct, recurrence-free evaluation of the scan on tiny inputs:
+
+    h_t[n] = exp(A_n * sum_{r<=t} delta_r) h0[n]
+             + sum_{s<=t} exp(A_n * sum_{s<r<=t} delta_r) delta_s B_s[n] u_s
+    y_t    = (sum_n C_t[n] h_t[n] + D u_t) * silu(z_t)
+    """
+    Bt, Dd, L = x.shape
+    N = A.shape[1]
+    G = Bm.shape[1]
+    out = np.zeros((Bt, Dd, L))
+    hT = np.zeros((Bt, Dd, N))
+    for b in range(Bt):
+        for d in range(Dd):
+            g = d // (Dd // G)
+            if cw is not None:
+                W = cw.shape[1]
+                hist = cs[b, d] if cs is not None else np.zeros(W)
+                u = _silu_ref(_conv_ref(x[b, d], cw[d], cb[d] if cb is not None else 0.0, hist))
+            else:
+                u = x[b, d].copy()
+            v = dt[b, d] + (dt_bias[d] if dt_bias is not None else 0.0)
+            delta = _softplus_ref(v) if softplus else v
+            for t in range(L):
+                y = 0.0
+                for n in range(N):
+                    h = math.exp(A[d, n] * delta[: t + 1].sum()) * (h0[b, d, n] if h0 is not None else 0.0)
+                    for s in range(t + 1):
+                        h += math.exp(A[d, n] * delta[s + 1: t + 1].sum()) * delta[s] * Bm[b, g, n, s] * u[s]
+                    y += Cm[b, g, n, t] * h
+                    if t == L - 1:
+                        hT[b, d, n] = h
+                y += (Dv[d] if Dv is not None else 0.0) * u[t]
+                if z is not None:
+                    y *= _silu_ref(z[b, d, t])
+                out[b, d, t] = y
+    return out, hT
+
+
+def _rand(shape, seed, name, scale=1.0):
+    return gen.normal(shape, "pins", seed, name) * scale
+
+
+@pytest.mark.parametrize("seed,Bt,Dd,L,N,G,W", [
+    (0, 1, 1, 1, 1, 1, 0),
+    (1, 1, 2, 5, 3, 1, 0),
+    (2, 2, 3, 8, 4, 1, 4),
+    (3, 1, 3, 7, 2, 3, 3),
+    (4, 2, 2, 3, 4, 2, 4),   # L < W
+    (5, 1, 2, 6, 3, 1, 1),   # W = 1
+    (6, 1, 4, 5, 2, 2, 4),   # two channels per group
+])
+def test_scan_matches_brute_force(seed, Bt, Dd, L, N, G, W):
+    x = _rand((Bt, Dd, L), seed, "x")
+    dt = gen.uniform((Bt, Dd, L), -2.0, 1.0, "pins", seed, "dt")
+    A = -np.abs(_rand((Dd, N), seed, "A")) - 0.1
+    Bm = _rand((Bt, G, N, L), seed, "B")
+    Cm = _rand((Bt, G, N, L), seed, "C")
+    Dv = _rand((Dd,), seed, "D")
+    z = _rand((Bt, Dd, L), seed, "z")
+    db = _rand((Dd,), seed, "db", 0.5)
+    h0 = _rand((Bt, Dd, N), seed, "h0")
+    cw = _rand((Dd, W), seed, "cw", 0.5) if W else None
+    cb = _rand((Dd,), seed, "cb") if W else None
+    cs = _rand((Bt, Dd, W), seed, "cs") if W else None
+    for softplus in (True, False):
+        out, hf, _ = oracle.scan(x, dt, A, Bm, Cm, D=Dv, z=z, dt_bias=db, dt_softplus=softplus,
+                                 conv_weight=cw, conv_bias=cb, conv_state=cs, h0=h0)
+        ref, hT = _brute_force_scan(x, dt, A, Bm, Cm, Dv, z, db, softplus, cw, cb, cs, h0)
+        np.testing.assert_allclose(out, ref, rtol=1e-11, atol=1e-12)
+        np.testing.assert_allclose(hf, hT, rtol=1e-11, atol=1e-12)
+
+
+def test_scan_optional_inputs_absent_match_brute_force():
+    Bt, Dd, L, N = 1, 2, 6, 3
+    x = _rand((Bt, Dd, L), 9, "x")
+    dt = gen.uniform((Bt, Dd, L), -3.0, 0.0, "pins", 9, "dt")
+    A = -np.abs(_rand((Dd, N), 9, "A"))
+    Bm = _rand((Bt, 1, N, L), 9, "B")
+    Cm = _rand((Bt, 1, N, L), 9, "C")
+    out, hf, _ = oracle.scan(x, dt, A, Bm, Cm)
+    ref, hT = _brute_force_scan(x, dt, A, Bm, Cm, None, None, None, True, None, None, None, None)
+    np.testing.assert_allclose(out, ref, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(hf, hT, rtol=1e-11, atol=1e-12)
+
+
+@pytest.mark.parametrize("A_val", [-0.7, -3.0, -0.01])
+def test_scan_closed_form_constant_inputs(A_val):
+    """Constant delta, A, B, C, x and h0 = 0: a = exp(delta A),
+    h_t = delta B x (1 - a^(t+1)) / (1 - a), y_t = C h_t + D x."""
+    L, N = 50, 2
+    delta, Bv, Cv, xv, Dval = 0.3, 1.7, -0.4, 0.9, 0.25
+    x = np.full((1, 1, L), xv)
+    dt = np.full((1, 1, L), delta)
+    A = np.full((1, N), A_val)
+    Bm = np.full((1, 1, N, L), Bv)
+    Cm = np.full((1, 1, N, L), Cv)
+    out, hf, _ = oracle.scan(x, dt, A, Bm, Cm, D=np.array([Dval]), dt_softplus=False)
+    a = math.exp(delta * A_val)
+    t = np.arange(L)
+    h = delta * Bv * xv * (1 - a ** (t + 1)) / (1 - a)
+    np.testing.assert_allclose(out[0, 0], N * Cv * h + Dval * xv, rtol=1e-12)
+    np.testing.assert_allclose(hf[0, 0], np.full(N, h[-1]), rtol=1e-12)
+
+
+def test_scan_A_zero_is_prefix_sum():
+    L, N = 40, 3
+    x = _rand((1, 1, L), 11, "x")
+    dt = np.abs(_rand((1, 1, L), 11, "dt"))
+    Bm = _rand((1, 1, N, L), 11, "B")
+    Cm = _rand((1, 1, N, L), 11, "C")
+    out, _, _ = oracle.scan(x, dt, np.zeros((1, N)), Bm, Cm, dt_softplus=False)
+    h = np.cumsum(dt[0, 0] * Bm[0, 0] * x[0, 0], axis=1)  # (N, L)
+    np.testing.assert_allclose(out[0, 0], (Cm[0, 0] * h).sum(0), rtol=1e-11, atol=1e-12)
+
+
+def test_scan_very_negative_A_has_no_memory():
+    L, N = 20, 2
+    x = _rand((1, 1, L), 12, "x")
+    dt = np.full((1, 1, L), 1.0)
+    Bm = _rand((1, 1, N, L), 12, "B")
+    Cm = _rand((1, 1, N, L), 12, "C")
+    out, _, _ = oracle.scan(x, dt, np.full((1, N), -1e4), Bm, Cm, dt_softplus=False)
+    ref = (Cm[0, 0] * Bm[0, 0] * x[0, 0]).sum(0)
+    np.testing.assert_allclose(out[0, 0], ref, rtol=1e-12)
+
+
+def test_scan_B_zero_gives_skip_times_gate():
+    s = gen.scan_inputs(2, 16, 3, 4, W=4, io="f32", seed=3, tag="pins")
+    Bz = np.zeros_like(s.B)
+    out, hf, _ = oracle.scan(s.x, s.dt, s.A, Bz, s.C, D=s.D, z=s.z, dt_bias=s.dt_bias,
+                             conv_weight=s.conv_weight, conv_bias=s.conv_bias)
+    u = np.stack([[_silu_ref(_conv_ref(s.x[b, d], s.conv_weight[d], 0.0, np.zeros(4)))
+                   for d in range(3)] for b in range(2)])
+    np.testing.assert_allclose(out, s.D[None, :, None] * u * _silu_ref(s.z), rtol=1e-12, atol=1e-14)
+    assert np.all(hf == 0.0)
+
+
+def test_scan_linear_in_x_without_conv():
+    s = gen.scan_inputs(1, 24, 3, 4, io="f32", seed=4, tag="pins")
+    x2 = _rand(s.x.shape, 4, "x2")
+    alpha, beta = 0.6, -1.3
+    kw = dict(D=s.D, z=s.z, dt_bias=s.dt_bias)
+    y1, _, _ = oracle.scan(s.x, s.dt, s.A, s.B, s.C, **kw)
+    y2, _, _ = oracle.scan(x2, s.dt, s.A, s.B, s.C, **kw)
+    y12, _, _ = oracle.scan(alpha * s.x + beta * x2, s.dt, s.A, s.B, s.C, **kw)
+    np.testing.assert_allclose(y12, alpha * y1 + beta * y2, rtol=1e-10, atol=1e-12)
+
+
+@pytest.mark.parametrize("split", [1, 2, 3, 17, 39])
+def test_scan_chunked_equals_sequential(split):
+    s = gen.scan_inputs(2, 40, 3, 4, W=4, io="f32", seed=5, tag="pins", conv_state=True, h0=True)
+    kw = dict(D=s.D, dt_bias=s.dt_bias, conv_weight=s.conv_weight, conv_bias=s.conv_bias)
+    full, hf, csf = oracle.scan(s.x, s.dt, s.A, s.B, s.C, z=s.z, conv_state=s.conv_state,
+                                h0=s.h0, **kw)
+    a, h1, cs1 = oracle.scan(s.x[..., :split], s.dt[..., :split], s.A, s.B[..., :split],
+                             s.C[..., :split], z=s.z[..., :split], conv_state=s.conv_state,
+                             h0=s.h0, **kw)
+    b, h2, cs2 = oracle.scan(s.x[..., split:], s.dt[..., split:], s.A, s.B[..., split:],
+                             s.C[..., split:], z=s.z[..., split:], conv_state=cs1, h0=h1, **kw)
+    np.testing.assert_allclose(np.concatenate([a, b], -1), full, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(h2, hf, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(cs2, csf, rtol=0, atol=0)
+
+
+def _decode_steps_via_ssu(s, h, cs, t0, t1):
+    """Run tokens t0..t1-1 through the single-token oracle (Mamba-1 layout
+    mapped onto (B, H=1, P=D, N))."""
+    Bt, Dd, _ = s.x.shape
+    N = s.A.shape[1]
+    outs = []
+    st = h.reshape(Bt, 1, Dd, N)
+    for t in range(t0, t1):
+        o, st, cs = oracle.ssu(st, s.x[:, None, :, t], s.dt[:, None, :, t], s.A[None], s.B[..., t],
+                               s.C[..., t], D=s.D[None], z=s.z[:, None, :, t],
+                               dt_bias=s.dt_bias[None], conv_weight=s.conv_weight,
+                               conv_bias=s.conv_bias, conv_state=cs)
+        outs.append(o[:, 0])
+    return np.stack(outs, -1), st.reshape(Bt, Dd, N), cs
+
+
+@pytest.mark.parametrize("k", [1, 3, 6])
+def test_prefill_then_decode_equals_full_prefill(k):
+    L = 12
+    s = gen.scan_inputs(2, L, 3, 4, W=4, io="f32", seed=6, tag="pins", conv_state=True, h0=True)
+    kw = dict(D=s.D, dt_bias=s.dt_bias, conv_weight=s.conv_weight, conv_bias=s.conv_bias)
+    full, hf, csf = oracle.scan(s.x, s.dt, s.A, s.B, s.C, z=s.z, conv_state=s.conv_state,
+                                h0=s.h0, **kw)
+    _, hp, csp = oracle.scan(s.x[..., :L - k], s.dt[..., :L - k], s.A, s.B[..., :L - k],
+                             s.C[..., :L - k], z=s.z[..., :L - k], conv_state=s.conv_state,
+                             h0=s.h0, **kw)
+    dec, hd, csd = _decode_steps_via_ssu(s, hp, csp, L - k, L)
+    np.testing.assert_allclose(dec, full[..., L - k:], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(hd, hf, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(csd.reshape(csf.shape), csf, rtol=0, atol=0)
+
+
+def test_single_token_prefill_equals_one_update_without_conv():
+    s = gen.scan_inputs(2, 1, 4, 5, io="f32", seed=7, tag="pins", h0=True)
+    out, hf, _ = oracle.scan(s.x, s.dt, s.A, s.B, s.C, D=s.D, z=s.z, dt_bias=s.dt_bias, h0=s.h0)
+    o, st, _ = oracle.ssu(s.h0[:, None], s.x[:, None, :, 0], s.dt[:, None, :, 0], s.A[None],
+                          s.B[..., 0], s.C[..., 0], D=s.D[None], z=s.z[:, None, :, 0],
+                          dt_bias=s.dt_bias[None])
+    np.testing.assert_allclose(o[:, 0], out[..., 0], rtol=1e-13)
+    np.testing.assert_allclose(st[:, 0], hf, rtol=1e-13)
+
+
+@pytest.mark.parametrize("G", [1, 2, 4])
+def test_mamba2_notation_matches_general_form(G):
+    Bt, H, P, N = 3, 4, 5, 6
+    s = gen.ssu_mamba2_inputs(Bt, H, P, N, G=G, io="f32", state="f32", seed=8, tag="pins",
+                              with_z=True)
+    o2, st2 = oracle.ssu_mamba2(s.state, s.x, s.dt, s.A, s.B, s.C, D=s.D, z=s.z,
+                                dt_bias=s.dt_bias)
+    og, stg, _ = oracle.ssu(s.state, s.x, s.dt[:, :, None], s.A[:, None, None], s.B, s.C,
+                            D=s.D[:, None], z=s.z, dt_bias=s.dt_bias[:, None])
+    np.testing.assert_allclose(o2, og, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(st2, stg, rtol=1e-13, atol=1e-14)
+
+
+def test_mamba2_groups_map_consecutive_heads():
+    """G groups: heads [g*H/G, (g+1)*H/G) read group g.  Equal to G separate
+    calls with one group each on those head ranges."""
+    Bt, H, P, N, G = 2, 6, 3, 4, 3
+    s = gen.ssu_mamba2_inputs(Bt, H, P, N, G=G, io="f32", state="f32", seed=9, tag="pins",
+                              with_z=True)
+    o, st = oracle.ssu_mamba2(s.state, s.x, s.dt, s.A, s.B, s.C, D=s.D, z=s.z, dt_bias=s.dt_bias)
+    hpg = H // G
+    for g in range(G):
+        hs = slice(g * hpg, (g + 1) * hpg)
+        og, stg = oracle.ssu_mamba2(s.state[:, hs], s.x[:, hs], s.dt[:, hs], s.A[hs],
+                                    s.B[:, g:g + 1], s.C[:, g:g + 1], D=s.D[hs], z=s.z[:, hs],
+                                    dt_bias=s.dt_bias[hs])
+        np.testing.assert_allclose(o[:, hs], og, rtol=1e-14)
+        np.testing.assert_allclose(st[:, hs], stg, rtol=1e-14)
+
+
+def test_ssu_single_step_matches_scan_brute_force_with_groups():
+    """One decode step with state, conv and groups equals the brute-force scan
+    of a single token whose conv history is the incoming conv state."""
+    Bt, Dd, N, W, G = 2, 4, 3, 4, 2
+    s = gen.scan_inputs(Bt, 1, Dd, N, G=G, W=W, io="f32", seed=10, tag="pins", conv_state=True,
+                        h0=True)
+    ref, hT = _brute_force_scan(s.x, s.dt, s.A, s.B, s.C, s.D, s.z, s.dt_bias, True,
+                                s.conv_weight, s.conv_bias, s.conv_state, s.h0)
+    # Mamba-1 channels as heads with headdim 1, so the group maps per channel.
+    o, st, cs = oracle.ssu(s.h0[:, :, None, :], s.x[:, :, None, 0], s.dt[:, :, None, 0],
+                           s.A[:, None, :], s.B[..., 0], s.C[..., 0], D=s.D[:, None],
+                           z=s.z[:, :, None, 0], dt_bias=s.dt_bias[:, None],
+                           conv_weight=s.conv_weight, conv_bias=s.conv_bias,
+                           conv_state=s.conv_state)
+    np.testing.assert_allclose(o[:, :, 0], ref[..., 0], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(st[:, :, 0], hT, rtol=1e-12, atol=1e-13)
+    expect_cs = np.concatenate([s.conv_state[..., 1:], s.x[..., :1]], -1)
+    np.testing.assert_array_equal(cs.reshape(Bt, Dd, W), expect_cs)
+
+
+@pytest.mark.parametrize("W", [1, 2, 3, 4, 6])
+def test_conv_impulse_response(W):
+    L = 10
+    w = _rand((1, W), 13, "w")
+    x = np.zeros((1, 1, L))
+    x[0, 0, 0] = 1.0
+    out, _ = oracle.conv1d(x, w, bias=np.array([0.5]))
+    expect = np.full(L, 0.5)
+    for t in range(min(W, L)):
+        expect[t] += w[0, W - 1 - t]
+    np.testing.assert_allclose(out[0, 0], expect, rtol=0, atol=1e-15)
+
+
+def test_conv_width_one_is_scaling():
+    x = _rand((2, 3, 9), 14, "x")
+    w = _rand((3, 1), 14, "w")
+    b = _rand((3,), 14, "b")
+    out, cs = oracle.conv1d(x, w, bias=b)
+    np.testing.assert_allclose(out, w[None, :, :1] * x + b[None, :, None], rtol=1e-15)
+    np.testing.assert_array_equal(cs[..., 0], x[..., -1])
+
+
+@pytest.mark.parametrize("L", [0, 1, 2, 3, 4, 7])
+def test_conv_matches_numpy_convolve_and_state(L):
+    Bt, Dd, W = 2, 3, 4
+    x = _rand((Bt, Dd, L), 15, "x")
+    w = _rand((Dd, W), 15, "w")
+    b = _rand((Dd,), 15, "b")
+    cs = _rand((Bt, Dd, W), 15, "cs")
+    for silu in (False, True):
+        out, cso = oracle.conv1d(x, w, bias=b, conv_state=cs, silu=silu)
+        for bb in range(Bt):
+            for d in range(Dd):
+                ref = _conv_ref(x[bb, d], w[d], b[d], cs[bb, d])
+                if silu:
+                    ref = _silu_ref(ref)
+                np.testing.assert_allclose(out[bb, d], ref, rtol=1e-13, atol=1e-14)
+                np.testing.assert_array_equal(cso[bb, d], np.concatenate([cs[bb, d], x[bb, d]])[-W:])
+
+
+def test_activation_special_values():
+    assert oracle.softplus(0.0) == pytest.approx(math.log(2.0), rel=1e-15)
+    assert oracle.softplus(800.0) == pytest.approx(800.0, rel=1e-15)
+    assert oracle.softplus(-800.0) == 0.0
+    assert oracle.silu(0.0) == 0.0
+    for v in (-3.0, -0.5, 0.25, 2.0, 30.0):
+        # silu(v) - silu(-v) = v and softplus(v) - softplus(-v) = v
+        assert oracle.silu(v) - oracle.silu(-v) == pytest.approx(v, rel=1e-14)
+        assert oracle.softplus(v) - oracle.softplus(-v) == pytest.approx(v, rel=1e-14)
