@@ -1,0 +1,538 @@
+"""Benchmark of the Mamba hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+                    [--sweep] [--no-decode]
+
+Headline (one JSON line on rank 0): the fused prefill -- causal conv1d (W=4)
++ SiLU + selective scan + D skip + SiLU(z) gate -- of a Mamba-2.8B-shaped
+layer, batch 4, L=2048, d_inner=5120, d_state=16, fp16 I/O, fp32 parameters
+and state; value = scan elements B*L*D*N per second (Gelem/s).  One step is
+one call of ssm_selective_scan_fwd on inputs already resident in HBM; L2 is
+flushed before every step and only the kernel is inside each step's event
+pair.  The same line carries the decode updates (ssm_selective_state_update)
+measured in the same run: HBM GB/s and fraction of the measured copy peak for
+the Mamba-1 2.8B-shaped decode step (64 layer slabs) and the Mamba-2 layouts at
+their largest effective batch.
+
+Multi-GPU: the work does not need an exchange between GPUs (every (b, d)
+recurrence is independent), so N ranks run independent replicas (weak
+scaling, no data-path collective); value = all ranks' elements / the slowest
+rank's time.  --impl reference times the fp64 CPU oracle on a bounded sample of
+the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "scan Gelem/s (B·L·D·N) prefill; SSU decode HBM GB/s vs B200 peak, per batch"
+WORKLOAD = "mamba1-2.8b-prefill: conv1d(W=4)+SiLU+selective-scan+gate, B=4 L=2048 D=5120 N=16, fp16 I/O"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+SFU_EX2_PER_CLK_PER_SM = 16  # MUFU ex2 throughput per SM per clock
+NUM_SMS = 148
+SM_MAX_MHZ = 1965.0
+
+
+# --------------------------------------------------------------- helpers --
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p.get("sm_max_mhz", SM_MAX_MHZ)), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, SM_MAX_MHZ, "fallback"
+
+
+def src_hash(*names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "state_space_model_causal_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(summary_name, source_files):
+    """DRAM bytes per launch recorded in a committed ncu summary, if that
+    summary was taken on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", summary_name)
+    try:
+        rec = {}
+        for line in open(path):
+            if ":" in line and not line.startswith("#"):
+                k, v = line.split(":", 1)
+                rec[k.strip()] = v.strip()
+        if rec.get("source_sha256_16") != src_hash(*source_files):
+            return None
+        return float(rec["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi samples of this GPU's clocks while the timed region runs."""
+
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in getattr(self, "lines", []):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8 or (self.uuid and self.uuid not in parts[0]):
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def device_uuid(dev):
+    import torch
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return None
+
+
+# --------------------------------------------------------------- prefill --
+class Prefill:
+    """Device-resident inputs and the call of the 2.8B-shaped prefill."""
+
+    def __init__(self, dev, seed=0):
+        import torch
+        from state_space_model_causal_b200 import inputs as gen
+        self.gen = gen
+        s = gen.prefill_2p8b(seed=seed)
+        self.s = s
+        self.Bt, self.D, self.L = s.x.shape
+        self.N = s.A.shape[1]
+        self.W = s.conv_weight.shape[1]
+        t = lambda a, dt: gen.to_torch(np.ascontiguousarray(a), dt, dev)  # noqa: E731
+        self.x, self.dt, self.z = t(s.x, "f16"), t(s.dt, "f16"), t(s.z, "f16")
+        self.B, self.C = t(s.B, "f16"), t(s.C, "f16")
+        self.A, self.Dv = t(s.A, "f32"), t(s.D, "f32")
+        self.db, self.cw, self.cb = t(s.dt_bias, "f32"), t(s.conv_weight, "f32"), t(s.conv_bias, "f32")
+        self.h = torch.zeros(self.Bt, self.D, self.N, device=dev)
+        self.cs = torch.zeros(self.Bt, self.D, self.W, device=dev)
+        self.out = torch.empty_like(self.x)
+        self.elems = self.Bt * self.L * self.D * self.N
+
+    def algorithmic_bytes(self):
+        BLD = self.Bt * self.L * self.D
+        io = 4 * BLD * 2                                  # x, dt, z in + out, fp16
+        bc = 2 * self.Bt * self.N * self.L * 2            # B, C
+        params = self.D * self.N * 4 + self.D * 4 * 3 + self.D * self.W * 4
+        states = self.Bt * self.D * (self.N + self.W) * 4  # final ssm/conv state written
+        return io + bc + params + states
+
+    def run(self, stream=None):
+        from state_space_model_causal_b200 import ssm_selective_scan_fwd
+        ssm_selective_scan_fwd(self.x, self.dt, self.A, self.B, self.C, D=self.Dv, z=self.z,
+                               dt_bias=self.db, conv_weight=self.cw, conv_bias=self.cb,
+                               conv_state=self.cs, ssm_state=self.h, out=self.out, stream=stream)
+
+
+def time_prefill(pf, steps, warmup, dev, flush):
+    """Per-step CUDA events around the kernel only, L2 flushed before each step."""
+    import torch
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(warmup):
+        flush.zero_()
+        pf.run()
+    torch.cuda.synchronize(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for a, b in ev:
+        flush.zero_()
+        a.record(stream)
+        pf.run()
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def time_prefill_e2e(pf, steps, warmup, dev):
+    """Same metric end to end: pinned host inputs -> device, the C-ABI call,
+    result back to pinned host memory, all inside each step's event pair."""
+    import torch
+    host = {k: getattr(pf, k).cpu().pin_memory() for k in ("x", "dt", "z", "B", "C")}
+    back = {k: torch.empty_like(getattr(pf, k), device="cpu").pin_memory()
+            for k in ("out", "h", "cs")}
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = sum(v.numel() * v.element_size() for v in back.values())
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        for k, v in host.items():
+            getattr(pf, k).copy_(v, non_blocking=True)
+        pf.h.zero_()
+        pf.cs.zero_()
+        pf.run()
+        for k, v in back.items():
+            v.copy_(getattr(pf, k), non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for a, b in ev:
+        a.record(stream)
+        step()
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = [a.elapsed_time(b) for a, b in ev]
+    return ms, h2d, d2h
+
+
+# ---------------------------------------------------------------- decode --
+def graph_time(calls, replays, dev, warm_eager=3):
+    """Per-call microseconds: `calls` (a list of closures) captured in one
+    CUDA graph, 5 warm replays, `replays` timed replays (events per replay)."""
+    import torch
+    for _ in range(warm_eager):
+        for c in calls:
+            c()
+    torch.cuda.synchronize(dev)
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream(dev)
+    s.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            for c in calls:
+                c()
+    torch.cuda.current_stream(dev).wait_stream(s)
+    for _ in range(5):
+        g.replay()
+    torch.cuda.synchronize(dev)
+    lat = []
+    for _ in range(replays):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        b.synchronize()
+        lat.append(a.elapsed_time(b))
+    del g
+    per_call = [1000.0 * l / len(calls) for l in lat]
+    return statistics.mean(per_call), statistics.median(per_call)
+
+
+def decode_mamba1_2p8b(dev, hbm_peak, slabs=64, replays=20):
+    """Mamba-1 2.8B-shaped decode: B=245, D=5120, N=16, W=4; fp32 ssm and conv
+    state ~ N(0,1), fp16 x/dt/z/B/C; one independent slab per layer, each call
+    of the graph on the next slab (13.2 GB per replay, far above L2)."""
+    import torch
+    from state_space_model_causal_b200 import inputs as gen, ssm_selective_state_update
+    Bt, D, N, W = 245, 5120, 16, 4
+    tag = ("bench", "decode_2p8b")
+    calls, bufs = [], []
+    for k in range(slabs):
+        st = gen.device_normal((Bt, D, N), "f32", *tag, k, "state", device=dev)
+        cs = gen.device_normal((Bt, D, W), "f32", *tag, k, "cs", device=dev)
+        x = gen.device_normal((Bt, D), "f16", *tag, k, "x", device=dev)
+        dt = gen.device_uniform((Bt, D), -4.0, -1.0, "f16", *tag, k, "dt", device=dev)
+        z = gen.device_normal((Bt, D), "f16", *tag, k, "z", device=dev)
+        Bm = gen.device_normal((Bt, 1, N), "f16", *tag, k, "B", device=dev)
+        Cm = gen.device_normal((Bt, 1, N), "f16", *tag, k, "C", device=dev)
+        A = -torch.arange(1, N + 1, device=dev, dtype=torch.float32).repeat(D, 1)
+        Dv = torch.ones(D, device=dev)
+        db = torch.from_numpy(gen.dt_bias_draw((D,), *tag, k, "db").astype(np.float32)).to(dev)
+        cw = gen.device_normal((D, W), "f32", *tag, k, "cw", std=0.2, device=dev)
+        cb = torch.zeros(D, device=dev)
+        out = torch.empty_like(x)
+        b = (st, x, dt, A, Bm, Cm, Dv, z, db, cw, cb, cs, out)
+        bufs.append(b)
+        calls.append(lambda b=b: ssm_selective_state_update(
+            b[0], b[1], b[2], b[3], b[4], b[5], D=b[6], z=b[7], dt_bias=b[8], conv_weight=b[9],
+            conv_bias=b[10], conv_state=b[11], out=b[12]))
+    us, med = graph_time(calls, replays, dev)
+    BD = Bt * D
+    nbytes = (BD * N * 4 * 2 + BD * ((W - 1) + W) * 4 + BD * 2 * 3 + BD * 2
+              + Bt * N * 2 * 2 + D * N * 4 + D * 4 * 3 + D * W * 4)
+    gbs = nbytes / (us * 1e-6) / 1e9
+    del bufs, calls
+    torch.cuda.empty_cache()
+    return {"workload": "mamba1-2.8b-decode: B=245 D=5120 N=16 W=4, fp32 ssm/conv state, fp16 io, 64 slabs",
+            "us_per_call": round(us, 3), "us_median": round(med, 3), "bytes_per_call": nbytes,
+            "GBps": round(gbs, 1), "frac_of_hbm_peak": round(gbs / hbm_peak, 4),
+            "l2": "each call on a different 100 MB slab", "gpu_launches_per_replay": slabs}
+
+
+def decode_mamba2(dev, hbm_peak, H, P, N, R, cache, io, replays=10, calls_per_graph=5):
+    """Mamba-2 SSU at effective batch R; slabs rotate so every call of the
+    graph touches state that is not resident in L2."""
+    import torch
+    from state_space_model_causal_b200 import inputs as gen, ssm_selective_state_update
+    Bt, Hr = gen.effective_batch_shape(R, H)
+    es = 4 if cache == "f32" else 2
+    state_bytes = Bt * Hr * P * N * es
+    nslab = max(1, min(calls_per_graph, math.ceil(2 * L2_BYTES / state_bytes)))
+    tag = ("bench", "mamba2", H, P, N, R, cache)
+    A = -torch.from_numpy(gen.uniform((Hr,), 1.0, 16.0, *tag, "A").astype(np.float32)).to(dev)
+    db = torch.from_numpy(gen.dt_bias_draw((Hr,), *tag, "db").astype(np.float32)).to(dev)
+    Dv = torch.ones(Hr, device=dev)
+    calls, bufs = [], []
+    for k in range(nslab):
+        st = gen.device_normal((Bt, Hr, P, N), cache, *tag, k, "state", device=dev)
+        x = gen.device_normal((Bt, Hr, P), io, *tag, k, "x", device=dev)
+        dt = gen.device_uniform((Bt, Hr), -4.0, -1.0, io, *tag, k, "dt", device=dev)
+        Bm = gen.device_normal((Bt, 1, N), io, *tag, k, "B", device=dev)
+        Cm = gen.device_normal((Bt, 1, N), io, *tag, k, "C", device=dev)
+        out = torch.empty_like(x)
+        b = (st, x, dt, Bm, Cm, out)
+        bufs.append(b)
+    for i in range(calls_per_graph):
+        b = bufs[i % nslab]
+        calls.append(lambda b=b: ssm_selective_state_update(
+            b[0], b[1], b[2], A, b[3], b[4], D=Dv, dt_bias=db, out=b[5]))
+    us, med = graph_time(calls, replays, dev)
+    rows = Bt * Hr * P
+    nbytes = rows * N * es * 2 + rows * 2 * 2 + Bt * Hr * 2 + Bt * N * 2 * 2 + Hr * 4 * 3
+    gbs = nbytes / (us * 1e-6) / 1e9
+    del bufs, calls
+    torch.cuda.empty_cache()
+    return {"workload": f"mamba2-ssu: H={H} P={P} N={N} G=1, {io} io, {cache} cache",
+            "effective_batch": R, "batch": Bt, "heads": Hr, "us_per_call": round(us, 3),
+            "us_median": round(med, 3), "bytes_per_call": nbytes, "GBps": round(gbs, 1),
+            "frac_of_hbm_peak": round(gbs / hbm_peak, 4),
+            "l2": f"{nslab} state slabs rotated ({nslab * state_bytes / 2**20:.0f} MiB)"}
+
+
+# ------------------------------------------------------------- reference --
+def oracle_prefill_sample(channels, seed=0):
+    """Time the fp64 oracle on `channels` full-length (b, d) channels of the
+    2.8B-shaped prefill recipe (at most the workload's 4 x 5120); returns
+    (seconds, elements)."""
+    import oracle
+    from state_space_model_causal_b200 import inputs as gen
+    channels = max(1, min(4 * 5120, channels))
+    Bt = -(-channels // 5120)
+    s = gen.prefill_2p8b(seed=seed, Bt=Bt, D=-(-channels // Bt))
+    t0 = time.perf_counter()
+    oracle.scan(s.x, s.dt, s.A, s.B, s.C, D=s.D, z=s.z, dt_bias=s.dt_bias,
+                conv_weight=s.conv_weight, conv_bias=s.conv_bias)
+    dt = time.perf_counter() - t0
+    return dt, s.x.shape[0] * s.x.shape[1] * s.x.shape[2] * s.A.shape[1]
+
+
+def cpu_baseline(target_s=10.0):
+    import oracle
+    oracle.build()
+    t, e = oracle_prefill_sample(64)
+    ch = int(64 * target_s / max(t, 1e-3))
+    t, e = oracle_prefill_sample(ch)
+    ch = e // (2048 * 16)
+    return {"value": round(e / t / 1e9, 6), "unit": "Gelem/s", "cores": 1, "kind": "oracle",
+            "sample": f"{ch} of the 20480 (b,d) channels of the 2.8B-shaped prefill, full "
+                      f"L=2048, fp64 sequential C on one thread, {t:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    t, _ = oracle_prefill_sample(64)
+    ch = max(64, min(5120, int(64 * 5.0 / max(t, 1e-3))))  # ~5 s of CPU work per step
+    for _ in range(args.warmup):
+        oracle_prefill_sample(ch)
+    times, elems = [], 0
+    for _ in range(args.steps):
+        t, e = oracle_prefill_sample(ch)
+        times.append(t)
+        elems = e
+    ms = 1000.0 * statistics.mean(times)
+    value = elems / (ms / 1000.0) / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "Gelem/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "sample": f"{ch} channels x L=2048 per step",
+                       "l2": "n/a (host)"},
+            "cpu_baseline": {"value": round(value, 6), "unit": "Gelem/s", "cores": 1,
+                             "kind": "oracle", "sample": f"{ch} (b,d) channels per step"},
+            "e2e": {"value": round(value, 6), "unit": "Gelem/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- sweep --
+def run_sweep(dev, hbm_peak):
+    out = []
+    for cache in ("f16", "f32"):
+        for R in (8, 16, 32, 64, 128, 256, 512, 1024, 2048, 4096, 8192, 16384, 32768, 65536, 131072):
+            r = decode_mamba2(dev, hbm_peak, 80, 64, 128, R, cache, "f16", replays=20)
+            print(json.dumps(r), flush=True)
+            out.append(r)
+    for cache in ("bf16", "f32"):
+        for R in (8, 16, 32, 64, 128, 256, 512, 1024, 2048, 4096, 8192, 16384, 32768, 65536):
+            r = decode_mamba2(dev, hbm_peak, 32, 128, 256, R, cache, "bf16", replays=20)
+            print(json.dumps(r), flush=True)
+            out.append(r)
+    return out
+
+
+# ----------------------------------------------------------------- main --
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--sweep", action="store_true", help="per-effective-batch decode sweep lines")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+        pg = dist
+
+    import state_space_model_causal_b200 as pkg
+    pkg.library()  # fails loudly when the extension is missing
+    hbm_peak, sm_max, peak_src = peaks()
+    if args.sweep:
+        if rank == 0:
+            run_sweep(dev, hbm_peak)
+        return 0
+
+    pf = Prefill(dev)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(device_uuid(dev)) as clk:
+        ms = time_prefill(pf, args.steps, args.warmup, dev, flush)
+    torch.cuda.synchronize(dev)
+    if pg:
+        pg.barrier()
+    ms_step = statistics.mean(ms)
+    if pg:
+        t = torch.tensor([ms_step], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms_step = float(t.item())
+    value = world * pf.elems / (ms_step * 1e-3) / 1e9
+
+    # roofline of the prefill kernel: one exp(delta*A) per element on the SFU
+    sfu_peak = NUM_SMS * SFU_EX2_PER_CLK_PER_SM * sm_max * 1e6 / 1e9  # Gelem/s
+    alg_bytes = pf.algorithmic_bytes()
+    hbm_gbs = alg_bytes / (ms_step * 1e-3) / 1e9
+    traffic = profiled_traffic("scan_chunked_prefill_2p8b.txt", ["scan.cu", "common.cuh"])
+    roofline = {"bound": "alu", "achieved": round(pf.elems / (ms_step * 1e-3) / 1e9, 2),
+                "peak": round(sfu_peak, 1), "unit": "Gelem/s",
+                "frac": round(pf.elems / (ms_step * 1e-3) / 1e9 / sfu_peak, 4),
+                "traffic": traffic, "peak_kind": "SFU ex2 16/clk/SM x 148 SMs x max SM clock",
+                "hbm_achieved_gbs": round(hbm_gbs, 1), "hbm_peak_gbs": hbm_peak,
+                "hbm_frac": round(hbm_gbs / hbm_peak, 4), "hbm_peak_kind": peak_src,
+                "algorithmic_bytes_per_launch": alg_bytes}
+
+    e2e_ms, h2d, d2h = time_prefill_e2e(pf, max(3, args.steps // 4), 3, dev)
+    e2e_val = world * pf.elems / (statistics.mean(e2e_ms) * 1e-3) / 1e9
+
+    decode = []
+    if not args.no_decode:
+        decode.append(decode_mamba1_2p8b(dev, hbm_peak))
+        decode.append(decode_mamba2(dev, hbm_peak, 80, 64, 128, 131072, "f16", "f16"))
+        decode.append(decode_mamba2(dev, hbm_peak, 80, 64, 128, 131072, "f32", "f16"))
+        decode.append(decode_mamba2(dev, hbm_peak, 32, 128, 256, 65536, "bf16", "bf16"))
+        decode.append(decode_mamba2(dev, hbm_peak, 32, 128, 256, 65536, "f32", "bf16"))
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline()
+
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {"metric": METRIC, "value": round(value, 2), "unit": "Gelem/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "global_batch": 4 * world, "seq_len": 2048,
+                       "d_inner": 5120, "d_state": 16, "conv_width": 4, "io_dtype": "f16",
+                       "parallelism": f"replicas x{world}",
+                       "l2": "flushed (256 MiB write) before every step; inputs 338 MB > 126 MB L2"},
+            "roofline": roofline, "cpu_baseline": cpu,
+            "e2e": {"value": round(e2e_val, 3), "unit": "Gelem/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": args.steps, "clocks": clk.summary(), "decode": decode}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

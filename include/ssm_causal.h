@@ -1,0 +1,274 @@
+/*
+ * ssm_causal.h -- C ABI of libssm_causal.so, the B200 (sm_100a) Mamba hot path.
+ *
+ * Three operations, each one call:
+ *
+ *   ssm_causal_conv1d_fwd       depthwise causal conv1d (+ optional SiLU) over a
+ *                               sequence, reading and writing the conv-state cache.
+ *   ssm_selective_scan_fwd      fused prefill: causal conv1d -> SiLU ->
+ *                               Delta = softplus(dt + dt_bias) -> selective scan
+ *                               -> D skip -> SiLU(z) gate, state caches in/out.
+ *   ssm_selective_state_update  single-token decode update of the state caches,
+ *                               Mamba-1 layout (d_inner x d_state, optional fused
+ *                               conv-state roll) and Mamba-2 layout (nheads x
+ *                               headdim x dstate, scalar A per head, ngroups).
+ *
+ * Sources.  The operators "causal-conv1d, selective-scan, silu, element-mul"
+ * and the Mamba state cache that is read and updated by capturing the conv and
+ * scan operators come from "feat(llama.cu): 适配 mamba 模型" (InfiniLM-Rust PR
+ * #48), sections 2.1 and 3.1.  The update's argument list and order
+ * (state, x, dt, A, B, C, D, z, dt_bias, dt_softplus, out), the Mamba-2 shape
+ * (batch, nheads, headdim, dstate, ngroups) and the effective batch
+ * batch x nheads come from "[XPU] Add tuned Mamba SSU configs for Intel Arc Pro
+ * B70" (vLLM PR #50534 report), sections 实现拆解 (item 2) and 关键源码片段.
+ * The pages do not print the equations.  The definitions used are:
+ *
+ *   conv    xc[t] = bias + sum_{k<W} w[k] * x[t-(W-1)+k]   (x[t<0] from conv_state)
+ *   SiLU    silu(v) = v * sigmoid(v)
+ *   Delta   delta = softplus(dt + dt_bias)  (dt + dt_bias when dt_softplus == 0)
+ *   scan    h[n] = exp(delta * A[n]) * h[n] + delta * B[n] * u
+ *   output  y = (sum_n C[n] * h[n] + D * u) * silu(z)   (no gate without z)
+ *
+ * where u is silu(xc) when the conv is fused and x otherwise.  The conv state
+ * of a channel holds its last W raw inputs, oldest first; a decode step rolls
+ * it left by one and appends the new input before the dot product.
+ *
+ * Tensors.  Every tensor is an ssm_tensor: a DEVICE pointer, a dtype, a rank
+ * and per-dimension sizes and strides counted in ELEMENTS.  Strides must be
+ * >= 0; a stride of 0 broadcasts an input along that dimension (never allowed
+ * for outputs or in/out caches).  An optional tensor is absent when its data
+ * pointer is NULL (its other fields are then ignored).  Parameters (A, D,
+ * dt_bias, conv weight and bias) are float32.  Arithmetic is float32 in every
+ * kernel; 16-bit inputs are widened on load and 16-bit outputs and caches are
+ * rounded to nearest even on store.
+ *
+ * Ownership and threading.  The caller owns every buffer.  The library never
+ * allocates or frees device memory, keeps no pointer after a call returns,
+ * never synchronises the stream and holds no mutable global state: every entry
+ * point is reentrant.  Work is enqueued on `stream` (a cudaStream_t; NULL is
+ * the legacy default stream) and runs asynchronously.
+ *
+ * Errors.  Every argument is checked before anything is launched; on an error
+ * nothing is launched and nothing is written, and the status says which check
+ * failed.  SSM_ERR_CUDA means the launch itself reported an error.  No entry
+ * point aborts, throws or traps on the device.  Outputs must not overlap any
+ * input (SSM_ERR_ALIAS); the in/out caches are updated in place.
+ */
+#ifndef SSM_CAUSAL_H
+#define SSM_CAUSAL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SSM_CAUSAL_ABI_VERSION 1
+#define SSM_MAX_DIMS 5
+
+typedef enum ssm_dtype {
+    SSM_F32 = 0,
+    SSM_F16 = 1,
+    SSM_BF16 = 2,
+    SSM_I32 = 3 /* index tensors only */
+} ssm_dtype;
+
+typedef enum ssm_status {
+    SSM_OK = 0,
+    SSM_ERR_NULL = 1,        /* a required pointer (args, tensor data) is NULL */
+    SSM_ERR_SHAPE = 2,       /* rank or sizes inconsistent with the others */
+    SSM_ERR_DTYPE = 3,       /* unsupported dtype or dtype combination */
+    SSM_ERR_STRIDE = 4,      /* negative stride, zero stride on an output, or a
+                                layout the kernels cannot address */
+    SSM_ERR_UNSUPPORTED = 5, /* valid but outside the implemented range (e.g.
+                                d_state > 256, conv width > 8) */
+    SSM_ERR_CUDA = 6,        /* the CUDA launch returned an error */
+    SSM_ERR_INTERNAL = 7,    /* a library invariant failed */
+    SSM_ERR_VERSION = 8,     /* struct_size does not match this library */
+    SSM_ERR_ALIAS = 9        /* an output overlaps an input */
+} ssm_status;
+
+/* Flags for the `flags` field of every args struct. */
+#define SSM_FLAG_DRY_RUN 0x1u /* check arguments and choose the launch, but launch nothing */
+
+typedef struct ssm_tensor {
+    void* data;                    /* device pointer; NULL = absent (optional tensors) */
+    int32_t dtype;                 /* ssm_dtype */
+    int32_t ndim;                  /* rank, 1..SSM_MAX_DIMS */
+    int64_t shape[SSM_MAX_DIMS];   /* sizes, >= 0 */
+    int64_t stride[SSM_MAX_DIMS];  /* in elements, >= 0 */
+} ssm_tensor;
+
+/* Optional report of the launch an entry point chose (filled on SSM_OK, also
+ * in dry-run mode).  Set struct_size = sizeof(ssm_launch_info). */
+typedef struct ssm_launch_info {
+    uint32_t struct_size;
+    int32_t kernel;          /* ssm_kernel_id */
+    int32_t grid;            /* CTAs launched (0 when there is no work) */
+    int32_t block;           /* threads per CTA */
+    int32_t smem_bytes;      /* dynamic shared memory per CTA */
+    int32_t rows_per_item;   /* state rows (or channels) one work item covers */
+    int64_t work_items;      /* independent work items in the problem */
+} ssm_launch_info;
+
+typedef enum ssm_kernel_id {
+    SSM_KERNEL_NONE = 0,            /* empty problem: nothing launched */
+    SSM_KERNEL_CONV1D = 1,          /* vectorised conv1d, L contiguous */
+    SSM_KERNEL_CONV1D_GENERIC = 2,  /* any strides */
+    SSM_KERNEL_SCAN_CHUNKED = 3,    /* fused prefill, smem-staged chunks of L */
+    SSM_KERNEL_SCAN_GENERIC = 4,    /* fused prefill, any strides / group layout */
+    SSM_KERNEL_SSU_VEC = 5,         /* 128-bit streaming state update */
+    SSM_KERNEL_SSU_GENERIC = 6      /* state update, any strides / dstate */
+} ssm_kernel_id;
+
+/* ------------------------------------------------------------------------ *
+ * ssm_causal_conv1d_fwd
+ *
+ *   x          (B, D, L)  f32 | f16 | bf16                       input
+ *   weight     (D, W)     f32, 1 <= W <= 8                        required
+ *   bias       (D)        f32                                     optional
+ *   conv_state (B, D, W)  f32 or x's dtype, in/out                optional:
+ *              read as the W raw inputs preceding x[:, :, 0] (oldest first),
+ *              then overwritten with the last W raw inputs of (state ++ x).
+ *              Absent: zeros are used and nothing is written.
+ *   silu       nonzero: apply SiLU to the conv output
+ *   out        (B, D, L)  x's dtype                               output
+ *
+ * out[b,d,t] = act(bias[d] + sum_k weight[d,k] * x[b,d,t-(W-1)+k]).
+ * L = 0 leaves conv_state unchanged.
+ * ------------------------------------------------------------------------ */
+typedef struct ssm_conv1d_args {
+    uint32_t struct_size; /* = sizeof(ssm_conv1d_args) */
+    uint32_t flags;       /* SSM_FLAG_* */
+    ssm_tensor x;
+    ssm_tensor weight;
+    ssm_tensor bias;
+    ssm_tensor conv_state;
+    int32_t silu;
+    ssm_tensor out;
+    ssm_launch_info* info; /* optional */
+} ssm_conv1d_args;
+
+ssm_status ssm_causal_conv1d_fwd(const ssm_conv1d_args* args, void* stream);
+
+/* ------------------------------------------------------------------------ *
+ * ssm_selective_scan_fwd -- fused prefill over L tokens (Mamba-1 layout).
+ *
+ *   x           (B, D, L)            f32 | f16 | bf16    input (raw when the conv is fused)
+ *   dt          (B, D, L)            x's dtype
+ *   A           (D, N)               f32, 1 <= N <= 256
+ *   B, C        (B, G, N, L) or (B, N, L)  x's dtype; channel d reads group d / (D/G)
+ *   D           (D)                  f32                 optional (absent = 0)
+ *   z           (B, D, L)            x's dtype           optional (absent = no gate)
+ *   dt_bias     (D)                  f32                 optional (absent = 0)
+ *   dt_softplus nonzero: delta = softplus(dt + dt_bias)
+ *   conv_weight (D, W)               f32, 1 <= W <= 8    optional: fuses conv + SiLU
+ *   conv_bias   (D)                  f32                 optional
+ *   conv_state  (B, D, W)            f32 or x's dtype    optional in/out, only with
+ *               conv_weight (as in ssm_causal_conv1d_fwd)
+ *   ssm_state   (B, D, N)            f32                 optional in/out: read as h0
+ *               and overwritten with the state after the last token.  Absent:
+ *               h0 = 0 and the final state is not written.
+ *   out         (B, D, L)            x's dtype           output
+ *
+ * The time dimension (last) of x, dt, z, B, C and out may have any stride; the
+ * fast kernel needs it to be 1.  L = 0 leaves every cache unchanged.
+ * ------------------------------------------------------------------------ */
+typedef struct ssm_scan_args {
+    uint32_t struct_size; /* = sizeof(ssm_scan_args) */
+    uint32_t flags;
+    ssm_tensor x;
+    ssm_tensor dt;
+    ssm_tensor A;
+    ssm_tensor B;
+    ssm_tensor C;
+    ssm_tensor D;
+    ssm_tensor z;
+    ssm_tensor dt_bias;
+    int32_t dt_softplus;
+    ssm_tensor conv_weight;
+    ssm_tensor conv_bias;
+    ssm_tensor conv_state;
+    ssm_tensor ssm_state;
+    ssm_tensor out;
+    ssm_launch_info* info; /* optional */
+} ssm_scan_args;
+
+ssm_status ssm_selective_scan_fwd(const ssm_scan_args* args, void* stream);
+
+/* ------------------------------------------------------------------------ *
+ * ssm_selective_state_update -- one decode token, caches updated in place.
+ *
+ * Mamba-1 layout (state rank 3):
+ *   state   (B, D, N)        f32 | f16 | bf16   in/out
+ *   x, z, out (B, D)         f32 | f16 | bf16   (z optional)
+ *   dt      (B, D)
+ *   A       (D, N)           f32
+ *   B, C    (B, G, N) or (B, N); channel d reads group d / (D/G)
+ *   D, dt_bias (D)           f32, optional
+ *   conv_weight (D, W), conv_bias (D), conv_state (B, D, W) in/out: optional
+ *           fused conv update.  When given, x is the raw input: the channel's
+ *           conv state is rolled left by one, x appended, and
+ *           u = silu(conv_bias + sum_k conv_weight[k] * conv_state[k]) replaces x.
+ *
+ * Mamba-2 layout (state rank 4):
+ *   state   (B, H, P, N)     f32 | f16 | bf16   in/out
+ *   x, z, out (B, H, P)
+ *   dt      (B, H) per head, or (B, H, P)
+ *   A       (H) scalar per head, or (H, P, N)   f32
+ *   B, C    (B, G, N); head h reads group h / (H/G)
+ *   D, dt_bias (H) or (H, P) f32, optional
+ *   conv_*  as above with D = H*P channels, channel c = h*P + p
+ *
+ * For every row r = (b, h, p): delta = softplus(dt + dt_bias);
+ * state[r, n] = exp(delta * A) * state[r, n] + delta * B[n] * u;
+ * out[r] = (sum_n C[n] * state[r, n] + D * u) * silu(z).  The readout uses the
+ * float32 updated state before it is rounded into a 16-bit cache.
+ *
+ * state_batch_indices (B) int32, optional: row b reads and writes cache slot
+ * state_batch_indices[b]; state and conv_state then both hold the pool's slot
+ * count in dim 0, which may differ from B.  A negative index marks a padding
+ * row, which is skipped entirely (its out row is left untouched); an index at
+ * or past the slot count is skipped the same way.  Without
+ * indices, dim 0 of the caches must equal B.
+ * ------------------------------------------------------------------------ */
+typedef struct ssm_ssu_args {
+    uint32_t struct_size; /* = sizeof(ssm_ssu_args) */
+    uint32_t flags;
+    ssm_tensor state;
+    ssm_tensor x;
+    ssm_tensor dt;
+    ssm_tensor A;
+    ssm_tensor B;
+    ssm_tensor C;
+    ssm_tensor D;
+    ssm_tensor z;
+    ssm_tensor dt_bias;
+    int32_t dt_softplus;
+    ssm_tensor conv_weight;
+    ssm_tensor conv_bias;
+    ssm_tensor conv_state;
+    ssm_tensor state_batch_indices;
+    ssm_tensor out;
+    ssm_launch_info* info; /* optional */
+} ssm_ssu_args;
+
+ssm_status ssm_selective_state_update(const ssm_ssu_args* args, void* stream);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char* ssm_status_string(int status);
+
+/* SSM_CAUSAL_ABI_VERSION of the loaded library. */
+int ssm_abi_version(void);
+
+/* sizeof() of the three args structs and of ssm_tensor / ssm_launch_info as
+ * compiled into the library, so that bindings can check their layouts:
+ * which = 0 tensor, 1 conv1d args, 2 scan args, 3 ssu args, 4 launch info. */
+size_t ssm_struct_size(int which);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSM_CAUSAL_H */

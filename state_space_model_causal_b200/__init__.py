@@ -1,3 +1,9 @@
 """B200-native Mamba hot path: causal conv1d, fused prefill selective scan and
 single-token selective_state_update, behind the C-ABI library
-``libssm_causal.so`` (declared in ``include/ssm_causal.h``)."""
+``libssm_causal.so`` (declared in ``include/ssm_causal.h``).
+
+The functions below are the thin ctypes binding of the three C entry points;
+they raise if the library has not been built (there is no fallback path).
+"""
+from .binding import (LaunchInfo, SsmError, library, ssm_causal_conv1d_fwd,  # noqa: F401
+                      ssm_selective_scan_fwd, ssm_selective_state_update)

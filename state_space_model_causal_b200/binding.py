@@ -1,0 +1,235 @@
+"""Thin ctypes binding of libssm_causal.so (declared in include/ssm_causal.h).
+
+Argument marshalling only: torch tensors are described by (device pointer,
+dtype, shape, strides) and handed to the C entry points together with the
+current CUDA stream.  Every step of the computation runs in the library's
+CUDA kernels; there is no CPU or PyTorch fallback.  If the shared library is
+missing, importing the functions raises instead of degrading silently.
+
+The three entry points keep the C names:
+
+* :func:`ssm_causal_conv1d_fwd`
+* :func:`ssm_selective_scan_fwd`
+* :func:`ssm_selective_state_update`
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional, Sequence
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libssm_causal.so")
+MAX_DIMS = 5
+
+SSM_F32, SSM_F16, SSM_BF16, SSM_I32 = 0, 1, 2, 3
+SSM_FLAG_DRY_RUN = 0x1
+
+STATUS = {
+    0: "SSM_OK", 1: "SSM_ERR_NULL", 2: "SSM_ERR_SHAPE", 3: "SSM_ERR_DTYPE", 4: "SSM_ERR_STRIDE",
+    5: "SSM_ERR_UNSUPPORTED", 6: "SSM_ERR_CUDA", 7: "SSM_ERR_INTERNAL", 8: "SSM_ERR_VERSION",
+    9: "SSM_ERR_ALIAS",
+}
+KERNELS = {
+    0: "none", 1: "conv1d", 2: "conv1d_generic", 3: "scan_chunked", 4: "scan_generic",
+    5: "ssu_vec", 6: "ssu_generic",
+}
+
+
+class SsmError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(msg)
+        self.status = status
+        self.name = STATUS.get(status, str(status))
+
+
+class Tensor(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("dtype", ctypes.c_int32), ("ndim", ctypes.c_int32),
+                ("shape", ctypes.c_int64 * MAX_DIMS), ("stride", ctypes.c_int64 * MAX_DIMS)]
+
+
+class LaunchInfo(ctypes.Structure):
+    _fields_ = [("struct_size", ctypes.c_uint32), ("kernel", ctypes.c_int32),
+                ("grid", ctypes.c_int32), ("block", ctypes.c_int32),
+                ("smem_bytes", ctypes.c_int32), ("rows_per_item", ctypes.c_int32),
+                ("work_items", ctypes.c_int64)]
+
+    def as_dict(self):
+        return {"kernel": KERNELS.get(self.kernel, self.kernel), "grid": self.grid,
+                "block": self.block, "smem_bytes": self.smem_bytes,
+                "rows_per_item": self.rows_per_item, "work_items": self.work_items}
+
+
+class Conv1dArgs(ctypes.Structure):
+    _fields_ = [("struct_size", ctypes.c_uint32), ("flags", ctypes.c_uint32),
+                ("x", Tensor), ("weight", Tensor), ("bias", Tensor), ("conv_state", Tensor),
+                ("silu", ctypes.c_int32), ("out", Tensor),
+                ("info", ctypes.POINTER(LaunchInfo))]
+
+
+class ScanArgs(ctypes.Structure):
+    _fields_ = [("struct_size", ctypes.c_uint32), ("flags", ctypes.c_uint32),
+                ("x", Tensor), ("dt", Tensor), ("A", Tensor), ("B", Tensor), ("C", Tensor),
+                ("D", Tensor), ("z", Tensor), ("dt_bias", Tensor), ("dt_softplus", ctypes.c_int32),
+                ("conv_weight", Tensor), ("conv_bias", Tensor), ("conv_state", Tensor),
+                ("ssm_state", Tensor), ("out", Tensor), ("info", ctypes.POINTER(LaunchInfo))]
+
+
+class SsuArgs(ctypes.Structure):
+    _fields_ = [("struct_size", ctypes.c_uint32), ("flags", ctypes.c_uint32),
+                ("state", Tensor), ("x", Tensor), ("dt", Tensor), ("A", Tensor), ("B", Tensor),
+                ("C", Tensor), ("D", Tensor), ("z", Tensor), ("dt_bias", Tensor),
+                ("dt_softplus", ctypes.c_int32), ("conv_weight", Tensor), ("conv_bias", Tensor),
+                ("conv_state", Tensor), ("state_batch_indices", Tensor), ("out", Tensor),
+                ("info", ctypes.POINTER(LaunchInfo))]
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def library():
+    """Load libssm_causal.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise ImportError(
+                    f"{LIB_PATH} is missing: build it with "
+                    "`python -m state_space_model_causal_b200.build` (there is no fallback)")
+            lib = ctypes.CDLL(LIB_PATH)
+            for name, argt in (("ssm_causal_conv1d_fwd", Conv1dArgs),
+                               ("ssm_selective_scan_fwd", ScanArgs),
+                               ("ssm_selective_state_update", SsuArgs)):
+                fn = getattr(lib, name)
+                fn.restype = ctypes.c_int
+                fn.argtypes = [ctypes.POINTER(argt), ctypes.c_void_p]
+            lib.ssm_status_string.restype = ctypes.c_char_p
+            lib.ssm_status_string.argtypes = [ctypes.c_int]
+            lib.ssm_abi_version.restype = ctypes.c_int
+            lib.ssm_struct_size.restype = ctypes.c_size_t
+            lib.ssm_struct_size.argtypes = [ctypes.c_int]
+            for which, st in enumerate((Tensor, Conv1dArgs, ScanArgs, SsuArgs, LaunchInfo)):
+                if lib.ssm_struct_size(which) != ctypes.sizeof(st):
+                    raise ImportError(f"struct layout mismatch for {st.__name__}")
+            _lib = lib
+    return _lib
+
+
+# ------------------------------------------------------------ descriptors --
+def raw_tensor(ptr: int, dtype: int, shape: Sequence[int], stride: Optional[Sequence[int]] = None):
+    """Descriptor from a raw pointer (used for host-side argument checks)."""
+    t = Tensor()
+    t.data = ptr
+    t.dtype = dtype
+    t.ndim = len(shape)
+    if stride is None:
+        stride, acc = [], 1
+        for s in reversed(shape):
+            stride.insert(0, acc)
+            acc *= max(int(s), 1)
+    for i, (s, st) in enumerate(zip(shape, stride)):
+        t.shape[i] = int(s)
+        t.stride[i] = int(st)
+    return t
+
+
+def _dtype_code(t) -> int:
+    import torch
+    codes = {torch.float32: SSM_F32, torch.float16: SSM_F16, torch.bfloat16: SSM_BF16,
+             torch.int32: SSM_I32}
+    if t.dtype not in codes:
+        raise TypeError(f"unsupported dtype {t.dtype}")
+    return codes[t.dtype]
+
+
+def describe(t) -> Tensor:
+    """torch.Tensor (CUDA) or None -> ssm_tensor."""
+    if t is None:
+        return Tensor()
+    if not t.is_cuda:
+        raise ValueError("libssm_causal takes CUDA tensors only (no CPU fallback)")
+    if t.dim() == 0 or t.dim() > MAX_DIMS:
+        raise ValueError(f"rank {t.dim()} is outside 1..{MAX_DIMS}")
+    return raw_tensor(t.data_ptr() if t.numel() > 0 else max(t.data_ptr(), 16), _dtype_code(t),
+                      tuple(t.shape), tuple(t.stride()))
+
+
+def _stream_of(tensors, stream):
+    if stream is not None:
+        return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    import torch
+    dev = next(t.device for t in tensors if t is not None)
+    return torch.cuda.current_stream(dev).cuda_stream
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        msg = library().ssm_status_string(status).decode()
+        raise SsmError(status, f"{what}: {msg}")
+
+
+def _info_ptr(info: Optional[LaunchInfo]):
+    if info is None:
+        return None
+    info.struct_size = ctypes.sizeof(LaunchInfo)
+    return ctypes.pointer(info)
+
+
+# ------------------------------------------------------------ entry points --
+def ssm_causal_conv1d_fwd(x, weight, bias=None, conv_state=None, silu=False, out=None,
+                          stream=None, info: Optional[LaunchInfo] = None):
+    """Causal depthwise conv1d.  x (B, D, L); weight (D, W) f32; bias (D);
+    conv_state (B, D, W) in/out.  Returns out (B, D, L)."""
+    import torch
+    if out is None:
+        out = torch.empty_like(x)
+    a = Conv1dArgs()
+    a.struct_size = ctypes.sizeof(Conv1dArgs)
+    a.x, a.weight, a.bias, a.conv_state, a.out = map(describe, (x, weight, bias, conv_state, out))
+    a.silu = int(bool(silu))
+    a.info = _info_ptr(info)
+    _check(library().ssm_causal_conv1d_fwd(ctypes.byref(a), _stream_of([x], stream)),
+           "ssm_causal_conv1d_fwd")
+    return out
+
+
+def ssm_selective_scan_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, dt_softplus=True,
+                           conv_weight=None, conv_bias=None, conv_state=None, ssm_state=None,
+                           out=None, stream=None, info: Optional[LaunchInfo] = None):
+    """Fused prefill (see include/ssm_causal.h).  Returns out (B, D, L)."""
+    import torch
+    if out is None:
+        out = torch.empty_like(x)
+    a = ScanArgs()
+    a.struct_size = ctypes.sizeof(ScanArgs)
+    (a.x, a.dt, a.A, a.B, a.C, a.D, a.z, a.dt_bias, a.conv_weight, a.conv_bias, a.conv_state,
+     a.ssm_state, a.out) = map(describe, (x, dt, A, B, C, D, z, dt_bias, conv_weight, conv_bias,
+                                          conv_state, ssm_state, out))
+    a.dt_softplus = int(bool(dt_softplus))
+    a.info = _info_ptr(info)
+    _check(library().ssm_selective_scan_fwd(ctypes.byref(a), _stream_of([x], stream)),
+           "ssm_selective_scan_fwd")
+    return out
+
+
+def ssm_selective_state_update(state, x, dt, A, B, C, D=None, z=None, dt_bias=None,
+                               dt_softplus=True, conv_weight=None, conv_bias=None,
+                               conv_state=None, state_batch_indices=None, out=None, stream=None,
+                               info: Optional[LaunchInfo] = None):
+    """One decode step; state (and conv_state) updated in place.  Returns out."""
+    import torch
+    if out is None:
+        out = torch.empty_like(x)
+    a = SsuArgs()
+    a.struct_size = ctypes.sizeof(SsuArgs)
+    (a.state, a.x, a.dt, a.A, a.B, a.C, a.D, a.z, a.dt_bias, a.conv_weight, a.conv_bias,
+     a.conv_state, a.state_batch_indices, a.out) = map(
+        describe, (state, x, dt, A, B, C, D, z, dt_bias, conv_weight, conv_bias, conv_state,
+                   state_batch_indices, out))
+    a.dt_softplus = int(bool(dt_softplus))
+    a.info = _info_ptr(info)
+    _check(library().ssm_selective_state_update(ctypes.byref(a), _stream_of([x], stream)),
+           "ssm_selective_state_update")
+    return out

@@ -1,0 +1,676 @@
+// api.cpp -- the C ABI of libssm_causal.so: argument validation, layout
+// normalisation, launch planning and dispatch to the sm_100a kernels.
+//
+// Everything here runs on the host before any CUDA call: a rejected call
+// launches nothing and writes nothing.  The only CUDA calls are the SM-count
+// query used for grid sizing (skipped in dry-run mode) and the launches.
+#include "../../include/ssm_causal.h"
+
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+
+#include "problem.h"
+
+namespace ssm {
+int scan_chunked_smem_bytes(int ns);
+}
+
+namespace {
+
+using namespace ssm;
+
+constexpr int kDefaultSms = 148;  // B200
+constexpr int kMaxN = 256;
+constexpr int kMaxConvW = 8;
+
+// ------------------------------------------------------------ tensor checks --
+bool present(const ssm_tensor& t) { return t.data != nullptr; }
+
+int esize(int dt) {
+    switch (dt) {
+        case SSM_F32: return 4;
+        case SSM_F16: return 2;
+        case SSM_BF16: return 2;
+        case SSM_I32: return 4;
+        default: return 0;
+    }
+}
+
+bool is_float(int dt) { return dt == SSM_F32 || dt == SSM_F16 || dt == SSM_BF16; }
+
+// rank, non-negative sizes and strides, element-aligned pointer
+ssm_status basic(const ssm_tensor& t) {
+    if (!t.data) return SSM_ERR_NULL;
+    if (t.ndim < 1 || t.ndim > SSM_MAX_DIMS) return SSM_ERR_SHAPE;
+    if (esize(t.dtype) == 0) return SSM_ERR_DTYPE;
+    for (int i = 0; i < t.ndim; ++i) {
+        if (t.shape[i] < 0) return SSM_ERR_SHAPE;
+        if (t.stride[i] < 0) return SSM_ERR_STRIDE;
+    }
+    if (reinterpret_cast<uintptr_t>(t.data) % esize(t.dtype) != 0) return SSM_ERR_STRIDE;
+    return SSM_OK;
+}
+
+ssm_status want_shape(const ssm_tensor& t, int nd, const int64_t* dims) {
+    if (t.ndim != nd) return SSM_ERR_SHAPE;
+    for (int i = 0; i < nd; ++i)
+        if (t.shape[i] != dims[i]) return SSM_ERR_SHAPE;
+    return SSM_OK;
+}
+
+ssm_status want(const ssm_tensor& t, std::initializer_list<int64_t> dims) {
+    return want_shape(t, (int)dims.size(), dims.begin());
+}
+
+int64_t numel(const ssm_tensor& t) {
+    int64_t n = 1;
+    for (int i = 0; i < t.ndim; ++i) n *= t.shape[i];
+    return n;
+}
+
+// Byte range [lo, hi) the tensor touches (empty tensors touch nothing).
+void extent(const ssm_tensor& t, uintptr_t* lo, uintptr_t* hi) {
+    const uintptr_t base = reinterpret_cast<uintptr_t>(t.data);
+    if (!t.data || numel(t) == 0) {
+        *lo = *hi = base;
+        return;
+    }
+    int64_t last = 0;
+    for (int i = 0; i < t.ndim; ++i) last += (t.shape[i] - 1) * t.stride[i];
+    *lo = base;
+    *hi = base + (uintptr_t)((last + 1) * esize(t.dtype));
+}
+
+bool overlap(const ssm_tensor& a, const ssm_tensor& b) {
+    uintptr_t al, ah, bl, bh;
+    extent(a, &al, &ah);
+    extent(b, &bl, &bh);
+    if (al == ah || bl == bh) return false;
+    return al < bh && bl < ah;
+}
+
+// An output must not write one address twice: sort the non-trivial dims by
+// stride and require each stride to clear the span of the smaller ones.
+bool non_overlapping(const ssm_tensor& t) {
+    int64_t st[SSM_MAX_DIMS], sh[SSM_MAX_DIMS];
+    int n = 0;
+    for (int i = 0; i < t.ndim; ++i) {
+        if (t.shape[i] <= 1) continue;
+        st[n] = t.stride[i];
+        sh[n] = t.shape[i];
+        ++n;
+    }
+    for (int i = 0; i < n; ++i)
+        for (int j = i + 1; j < n; ++j)
+            if (st[j] < st[i]) {
+                std::swap(st[i], st[j]);
+                std::swap(sh[i], sh[j]);
+            }
+    int64_t span = 1;
+    for (int i = 0; i < n; ++i) {
+        if (st[i] < span) return false;
+        span = st[i] * (sh[i] - 1) + span;
+    }
+    return true;
+}
+
+// stride of dim i, with size-1 dims reading as 0 (never stepped)
+int64_t sd(const ssm_tensor& t, int i) { return t.shape[i] == 1 ? 0 : t.stride[i]; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int sm_count(bool dry_run) {
+    if (dry_run) return kDefaultSms;
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return kDefaultSms;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        return kDefaultSms;
+    return n;
+}
+
+void fill_info(ssm_launch_info* info, int kernel, int grid, int block, int smem, int64_t rows,
+               int64_t items) {
+    if (!info) return;
+    info->kernel = kernel;
+    info->grid = grid;
+    info->block = block;
+    info->smem_bytes = smem;
+    info->rows_per_item = (int32_t)rows;
+    info->work_items = items;
+}
+
+ssm_status info_ok(const ssm_launch_info* info) {
+    if (info && info->struct_size != sizeof(ssm_launch_info)) return SSM_ERR_VERSION;
+    return SSM_OK;
+}
+
+#define SSM_TRY(expr)                  \
+    do {                               \
+        ssm_status _s = (expr);        \
+        if (_s != SSM_OK) return _s;   \
+    } while (0)
+
+// ------------------------------------------------------------------ conv1d --
+ssm_status conv1d_impl(const ssm_conv1d_args* a, cudaStream_t stream) {
+    if (!a) return SSM_ERR_NULL;
+    if (a->struct_size != sizeof(ssm_conv1d_args)) return SSM_ERR_VERSION;
+    SSM_TRY(info_ok(a->info));
+    SSM_TRY(basic(a->x));
+    SSM_TRY(basic(a->weight));
+    SSM_TRY(basic(a->out));
+    if (a->x.ndim != 3) return SSM_ERR_SHAPE;
+    const int64_t B = a->x.shape[0], D = a->x.shape[1], L = a->x.shape[2];
+    if (a->weight.ndim != 2 || a->weight.shape[0] != D) return SSM_ERR_SHAPE;
+    const int64_t W = a->weight.shape[1];
+    if (!is_float(a->x.dtype)) return SSM_ERR_DTYPE;
+    if (a->weight.dtype != SSM_F32 || a->out.dtype != a->x.dtype) return SSM_ERR_DTYPE;
+    SSM_TRY(want(a->out, {B, D, L}));
+    if (W < 1) return SSM_ERR_SHAPE;
+    if (W > kMaxConvW) return SSM_ERR_UNSUPPORTED;
+    if (present(a->bias)) {
+        SSM_TRY(basic(a->bias));
+        SSM_TRY(want(a->bias, {D}));
+        if (a->bias.dtype != SSM_F32) return SSM_ERR_DTYPE;
+    }
+    if (present(a->conv_state)) {
+        SSM_TRY(basic(a->conv_state));
+        SSM_TRY(want(a->conv_state, {B, D, W}));
+        if (a->conv_state.dtype != SSM_F32 && a->conv_state.dtype != a->x.dtype) return SSM_ERR_DTYPE;
+        if (!non_overlapping(a->conv_state)) return SSM_ERR_STRIDE;
+    }
+    if (!non_overlapping(a->out)) return SSM_ERR_STRIDE;
+    const ssm_tensor* ins[] = {&a->x, &a->weight, &a->bias};
+    for (const ssm_tensor* t : ins) {
+        if (overlap(a->out, *t)) return SSM_ERR_ALIAS;
+        if (present(a->conv_state) && overlap(a->conv_state, *t)) return SSM_ERR_ALIAS;
+    }
+    if (present(a->conv_state) && overlap(a->out, a->conv_state)) return SSM_ERR_ALIAS;
+
+    Conv1dProblem p{};
+    p.Bn = B; p.D = D; p.L = L; p.W = W; p.io_dt = a->x.dtype;
+    p.x = a->x.data; p.x_b = sd(a->x, 0); p.x_d = sd(a->x, 1); p.x_t = sd(a->x, 2);
+    p.w = static_cast<const float*>(a->weight.data); p.w_d = sd(a->weight, 0); p.w_k = sd(a->weight, 1);
+    p.bias = static_cast<const float*>(a->bias.data);
+    p.b_d = present(a->bias) ? sd(a->bias, 0) : 0;
+    p.conv_state = a->conv_state.data;
+    if (present(a->conv_state)) {
+        p.cs_dt = a->conv_state.dtype;
+        p.cs_b = sd(a->conv_state, 0); p.cs_d = sd(a->conv_state, 1); p.cs_k = sd(a->conv_state, 2);
+    }
+    p.silu = a->silu != 0;
+    p.out = a->out.data; p.o_b = sd(a->out, 0); p.o_d = sd(a->out, 1); p.o_t = sd(a->out, 2);
+
+    Conv1dPlan plan{};
+    const int64_t rows = B * D;
+    const bool empty = rows == 0 || (L == 0 && !present(a->conv_state));
+    // L == 0 with a conv state: the state is unchanged, nothing to do
+    if (empty || L == 0) {
+        fill_info(a->info, SSM_KERNEL_NONE, 0, 0, 0, 0, 0);
+        return SSM_OK;
+    }
+    plan.kernel = SSM_KERNEL_CONV1D;
+    plan.block = 128;
+    const int64_t grid = (rows + 3) / 4;
+    if (grid > INT32_MAX) return SSM_ERR_UNSUPPORTED;
+    plan.grid = (int)grid;
+    fill_info(a->info, plan.kernel, plan.grid, plan.block, 0, 1, rows);
+    if (a->flags & SSM_FLAG_DRY_RUN) return SSM_OK;
+    return launch_conv1d(p, plan, stream) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+// -------------------------------------------------------------------- scan --
+ssm_status scan_impl(const ssm_scan_args* a, cudaStream_t stream) {
+    if (!a) return SSM_ERR_NULL;
+    if (a->struct_size != sizeof(ssm_scan_args)) return SSM_ERR_VERSION;
+    SSM_TRY(info_ok(a->info));
+    SSM_TRY(basic(a->x));
+    SSM_TRY(basic(a->dt));
+    SSM_TRY(basic(a->A));
+    SSM_TRY(basic(a->B));
+    SSM_TRY(basic(a->C));
+    SSM_TRY(basic(a->out));
+    if (a->x.ndim != 3) return SSM_ERR_SHAPE;
+    const int64_t Bn = a->x.shape[0], D = a->x.shape[1], L = a->x.shape[2];
+    if (a->A.ndim != 2 || a->A.shape[0] != D) return SSM_ERR_SHAPE;
+    const int64_t N = a->A.shape[1];
+    const int io = a->x.dtype;
+    if (!is_float(io)) return SSM_ERR_DTYPE;
+    if (a->A.dtype != SSM_F32) return SSM_ERR_DTYPE;
+    for (const ssm_tensor* t : {&a->dt, &a->B, &a->C, &a->out})
+        if (t->dtype != io) return SSM_ERR_DTYPE;
+    SSM_TRY(want(a->dt, {Bn, D, L}));
+    SSM_TRY(want(a->out, {Bn, D, L}));
+    int64_t G = 1;
+    int64_t bs[4], cs[4];  // strides of B, C as (b, g, n, t)
+    if (a->B.ndim == 4) {
+        G = a->B.shape[1];
+        SSM_TRY(want(a->B, {Bn, G, N, L}));
+        SSM_TRY(want(a->C, {Bn, G, N, L}));
+        for (int i = 0; i < 4; ++i) { bs[i] = sd(a->B, i); cs[i] = sd(a->C, i); }
+    } else if (a->B.ndim == 3) {
+        SSM_TRY(want(a->B, {Bn, N, L}));
+        SSM_TRY(want(a->C, {Bn, N, L}));
+        bs[0] = sd(a->B, 0); bs[1] = 0; bs[2] = sd(a->B, 1); bs[3] = sd(a->B, 2);
+        cs[0] = sd(a->C, 0); cs[1] = 0; cs[2] = sd(a->C, 1); cs[3] = sd(a->C, 2);
+    } else {
+        return SSM_ERR_SHAPE;
+    }
+    if (G < 1 || (D > 0 && D % G != 0)) return SSM_ERR_SHAPE;
+    if (N < 1) return SSM_ERR_SHAPE;
+    if (N > kMaxN) return SSM_ERR_UNSUPPORTED;
+    const ssm_tensor* opt1[] = {&a->D, &a->dt_bias, &a->conv_bias};
+    for (const ssm_tensor* t : opt1) {
+        if (!present(*t)) continue;
+        SSM_TRY(basic(*t));
+        SSM_TRY(want(*t, {D}));
+        if (t->dtype != SSM_F32) return SSM_ERR_DTYPE;
+    }
+    if (present(a->z)) {
+        SSM_TRY(basic(a->z));
+        SSM_TRY(want(a->z, {Bn, D, L}));
+        if (a->z.dtype != io) return SSM_ERR_DTYPE;
+    }
+    int64_t W = 0;
+    if (present(a->conv_weight)) {
+        SSM_TRY(basic(a->conv_weight));
+        if (a->conv_weight.ndim != 2 || a->conv_weight.shape[0] != D) return SSM_ERR_SHAPE;
+        if (a->conv_weight.dtype != SSM_F32) return SSM_ERR_DTYPE;
+        W = a->conv_weight.shape[1];
+        if (W < 1) return SSM_ERR_SHAPE;
+        if (W > kMaxConvW) return SSM_ERR_UNSUPPORTED;
+    } else if (present(a->conv_bias) || present(a->conv_state)) {
+        return SSM_ERR_NULL;  // conv bias / state without conv weight
+    }
+    if (present(a->conv_state)) {
+        SSM_TRY(basic(a->conv_state));
+        SSM_TRY(want(a->conv_state, {Bn, D, W}));
+        if (a->conv_state.dtype != SSM_F32 && a->conv_state.dtype != io) return SSM_ERR_DTYPE;
+        if (!non_overlapping(a->conv_state)) return SSM_ERR_STRIDE;
+    }
+    if (present(a->ssm_state)) {
+        SSM_TRY(basic(a->ssm_state));
+        SSM_TRY(want(a->ssm_state, {Bn, D, N}));
+        if (a->ssm_state.dtype != SSM_F32) return SSM_ERR_DTYPE;
+        if (!non_overlapping(a->ssm_state)) return SSM_ERR_STRIDE;
+    }
+    if (!non_overlapping(a->out)) return SSM_ERR_STRIDE;
+    const ssm_tensor* ins[] = {&a->x, &a->dt, &a->A, &a->B, &a->C, &a->D, &a->z, &a->dt_bias,
+                               &a->conv_weight, &a->conv_bias};
+    const ssm_tensor* outs[] = {&a->out, &a->conv_state, &a->ssm_state};
+    for (const ssm_tensor* o : outs) {
+        if (!present(*o)) continue;
+        for (const ssm_tensor* t : ins)
+            if (present(*t) && overlap(*o, *t)) return SSM_ERR_ALIAS;
+    }
+    if (overlap(a->out, a->conv_state) || overlap(a->out, a->ssm_state) ||
+        overlap(a->conv_state, a->ssm_state))
+        return SSM_ERR_ALIAS;
+
+    ScanProblem p{};
+    p.Bn = Bn; p.D = D; p.L = L; p.N = N; p.G = G; p.W = W;
+    p.ch_per_group = G > 0 && D > 0 ? D / G : 1;
+    p.io_dt = io;
+    p.x = a->x.data; p.x_b = sd(a->x, 0); p.x_d = sd(a->x, 1); p.x_t = sd(a->x, 2);
+    p.dt = a->dt.data; p.dt_b = sd(a->dt, 0); p.dt_d = sd(a->dt, 1); p.dt_t = sd(a->dt, 2);
+    p.A = static_cast<const float*>(a->A.data); p.A_d = sd(a->A, 0); p.A_n = sd(a->A, 1);
+    p.Bm = a->B.data; p.B_b = bs[0]; p.B_g = bs[1]; p.B_n = bs[2]; p.B_t = bs[3];
+    p.Cm = a->C.data; p.C_b = cs[0]; p.C_g = cs[1]; p.C_n = cs[2]; p.C_t = cs[3];
+    p.Dp = static_cast<const float*>(a->D.data); p.D_d = present(a->D) ? sd(a->D, 0) : 0;
+    p.z = a->z.data;
+    if (present(a->z)) { p.z_b = sd(a->z, 0); p.z_d = sd(a->z, 1); p.z_t = sd(a->z, 2); }
+    p.dt_bias = static_cast<const float*>(a->dt_bias.data);
+    p.db_d = present(a->dt_bias) ? sd(a->dt_bias, 0) : 0;
+    p.softplus = a->dt_softplus != 0;
+    if (W > 0) {
+        p.conv_w = static_cast<const float*>(a->conv_weight.data);
+        p.cw_d = sd(a->conv_weight, 0); p.cw_k = sd(a->conv_weight, 1);
+        p.conv_b = static_cast<const float*>(a->conv_bias.data);
+        p.cb_d = present(a->conv_bias) ? sd(a->conv_bias, 0) : 0;
+        p.conv_state = a->conv_state.data;
+        if (present(a->conv_state)) {
+            p.cs_dt = a->conv_state.dtype;
+            p.cs_b = sd(a->conv_state, 0); p.cs_d = sd(a->conv_state, 1); p.cs_k = sd(a->conv_state, 2);
+        }
+    }
+    p.ssm_state = static_cast<float*>(a->ssm_state.data);
+    if (present(a->ssm_state)) {
+        p.ss_b = sd(a->ssm_state, 0); p.ss_d = sd(a->ssm_state, 1); p.ss_n = sd(a->ssm_state, 2);
+    }
+    p.out = a->out.data; p.o_b = sd(a->out, 0); p.o_d = sd(a->out, 1); p.o_t = sd(a->out, 2);
+
+    if (Bn == 0 || D == 0 || L == 0) {  // nothing to compute, caches unchanged
+        fill_info(a->info, SSM_KERNEL_NONE, 0, 0, 0, 0, 0);
+        return SSM_OK;
+    }
+    ScanPlan plan{};
+    int ns = 1;
+    while (ns * 4 < N) ns *= 2;
+    const int dtile = 64 / (ns <= 16 ? ns : 16);
+    const bool groups_fit = G == 1 || (p.ch_per_group % dtile == 0);
+    if (ns <= 16 && groups_fit && Bn <= 65535) {
+        plan.kernel = SSM_KERNEL_SCAN_CHUNKED;
+        plan.ns = ns;
+        plan.dt_tile = dtile;
+        plan.t_chunk = 32;
+        plan.block = dtile * ns;
+        const int64_t grid = ((D + dtile - 1) / dtile) * Bn;
+        if (grid > INT32_MAX) return SSM_ERR_UNSUPPORTED;
+        plan.grid = (int)grid;
+        plan.smem = scan_chunked_smem_bytes(ns);
+        fill_info(a->info, plan.kernel, plan.grid, plan.block, plan.smem, dtile,
+                  ((D + dtile - 1) / dtile) * Bn);
+    } else {
+        plan.kernel = SSM_KERNEL_SCAN_GENERIC;
+        plan.block = 128;
+        const int64_t rows = Bn * D;
+        plan.grid = (int)std::min<int64_t>((rows + 127) / 128, (int64_t)sm_count(a->flags & SSM_FLAG_DRY_RUN) * 16);
+        fill_info(a->info, plan.kernel, plan.grid, plan.block, 0, 1, rows);
+    }
+    if (a->flags & SSM_FLAG_DRY_RUN) return SSM_OK;
+    return launch_scan(p, plan, stream) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+// --------------------------------------------------------------------- ssu --
+// Per-head parameter (D, dt_bias): (Hm) or, in the Mamba-2 layout, (H, P).
+ssm_status head_param(const ssm_tensor& t, bool m2, int64_t H, int64_t P, int64_t* sh, int64_t* sp) {
+    SSM_TRY(basic(t));
+    if (t.dtype != SSM_F32) return SSM_ERR_DTYPE;
+    if (t.ndim == 1) {
+        SSM_TRY(want(t, {H}));
+        *sh = sd(t, 0);
+        *sp = 0;
+        return SSM_OK;
+    }
+    if (m2 && t.ndim == 2) {
+        SSM_TRY(want(t, {H, P}));
+        *sh = sd(t, 0);
+        *sp = sd(t, 1);
+        return SSM_OK;
+    }
+    return SSM_ERR_SHAPE;
+}
+
+ssm_status ssu_impl(const ssm_ssu_args* a, cudaStream_t stream) {
+    if (!a) return SSM_ERR_NULL;
+    if (a->struct_size != sizeof(ssm_ssu_args)) return SSM_ERR_VERSION;
+    SSM_TRY(info_ok(a->info));
+    for (const ssm_tensor* t : {&a->state, &a->x, &a->dt, &a->A, &a->B, &a->C, &a->out})
+        SSM_TRY(basic(*t));
+    const bool m2 = a->state.ndim == 4;
+    if (a->state.ndim != 3 && !m2) return SSM_ERR_SHAPE;
+    const int64_t slots = a->state.shape[0];
+    int64_t H, P, N;
+    if (m2) {
+        H = a->state.shape[1]; P = a->state.shape[2]; N = a->state.shape[3];
+    } else {
+        H = a->state.shape[1]; P = 1; N = a->state.shape[2];  // channel = head, headdim 1
+    }
+    const int64_t Bn = a->x.shape[0];
+    if (!is_float(a->state.dtype)) return SSM_ERR_DTYPE;
+    for (const ssm_tensor* t : {&a->x, &a->dt, &a->B, &a->C, &a->out})
+        if (!is_float(t->dtype)) return SSM_ERR_DTYPE;
+    if (a->A.dtype != SSM_F32) return SSM_ERR_DTYPE;
+
+    SsuProblem p{};
+    p.Bn = Bn; p.H = H; p.P = P; p.N = N;
+    p.n_slots = slots;
+    // x / out / z
+    auto row3 = [&](const ssm_tensor& t, int64_t* b, int64_t* h, int64_t* pp) -> ssm_status {
+        if (m2) {
+            SSM_TRY(want(t, {Bn, H, P}));
+            *b = sd(t, 0); *h = sd(t, 1); *pp = sd(t, 2);
+        } else {
+            SSM_TRY(want(t, {Bn, H}));
+            *b = sd(t, 0); *h = sd(t, 1); *pp = 0;
+        }
+        return SSM_OK;
+    };
+    SSM_TRY(row3(a->x, &p.x_b, &p.x_h, &p.x_p));
+    SSM_TRY(row3(a->out, &p.o_b, &p.o_h, &p.o_p));
+    if (present(a->z)) {
+        SSM_TRY(basic(a->z));
+        if (!is_float(a->z.dtype)) return SSM_ERR_DTYPE;
+        SSM_TRY(row3(a->z, &p.z_b, &p.z_h, &p.z_p));
+        p.z = a->z.data; p.z_dt = a->z.dtype;
+    }
+    // dt: (B, H) per head/channel, or (B, H, P) per row in the Mamba-2 layout
+    if (a->dt.ndim == 2) {
+        SSM_TRY(want(a->dt, {Bn, H}));
+        p.dt_b = sd(a->dt, 0); p.dt_h = sd(a->dt, 1); p.dt_p = 0;
+    } else if (m2 && a->dt.ndim == 3) {
+        SSM_TRY(want(a->dt, {Bn, H, P}));
+        p.dt_b = sd(a->dt, 0); p.dt_h = sd(a->dt, 1); p.dt_p = sd(a->dt, 2);
+    } else {
+        return SSM_ERR_SHAPE;
+    }
+    // A: Mamba-1 (D, N); Mamba-2 (H) or (H, P, N)
+    if (!m2) {
+        SSM_TRY(want(a->A, {H, N}));
+        p.A_full = 1; p.A_h = sd(a->A, 0); p.A_p = 0; p.A_n = sd(a->A, 1);
+    } else if (a->A.ndim == 1) {
+        SSM_TRY(want(a->A, {H}));
+        p.A_full = 0; p.A_h = sd(a->A, 0);
+    } else if (a->A.ndim == 3) {
+        SSM_TRY(want(a->A, {H, P, N}));
+        p.A_h = sd(a->A, 0); p.A_p = sd(a->A, 1); p.A_n = sd(a->A, 2);
+        p.A_full = (p.A_p != 0 || p.A_n != 0) ? 1 : 0;  // fully broadcast = one scalar per head
+    } else {
+        return SSM_ERR_SHAPE;
+    }
+    // B, C: (B, G, N) or (B, N)
+    int64_t G = 1;
+    if (a->B.ndim == 3) {
+        G = a->B.shape[1];
+        SSM_TRY(want(a->B, {Bn, G, N}));
+        SSM_TRY(want(a->C, {Bn, G, N}));
+        p.B_b = sd(a->B, 0); p.B_g = sd(a->B, 1); p.B_n = sd(a->B, 2);
+        p.C_b = sd(a->C, 0); p.C_g = sd(a->C, 1); p.C_n = sd(a->C, 2);
+    } else if (a->B.ndim == 2) {
+        SSM_TRY(want(a->B, {Bn, N}));
+        SSM_TRY(want(a->C, {Bn, N}));
+        p.B_b = sd(a->B, 0); p.B_g = 0; p.B_n = sd(a->B, 1);
+        p.C_b = sd(a->C, 0); p.C_g = 0; p.C_n = sd(a->C, 1);
+    } else {
+        return SSM_ERR_SHAPE;
+    }
+    if (N < 1 || H < 1 || P < 1) return SSM_ERR_SHAPE;
+    if (G < 1 || H % G != 0) return SSM_ERR_SHAPE;
+    if (N > kMaxN) return SSM_ERR_UNSUPPORTED;
+    p.G = G;
+    p.heads_per_group = H / G;
+    if (present(a->D)) {
+        SSM_TRY(head_param(a->D, m2, H, P, &p.D_h, &p.D_p));
+        p.Dp = static_cast<const float*>(a->D.data);
+    }
+    if (present(a->dt_bias)) {
+        SSM_TRY(head_param(a->dt_bias, m2, H, P, &p.db_h, &p.db_p));
+        p.dt_bias = static_cast<const float*>(a->dt_bias.data);
+    }
+    // state: (slots, H, P, N) / (slots, D, N)
+    p.state = a->state.data; p.state_dt = a->state.dtype;
+    p.st_b = sd(a->state, 0);
+    if (m2) {
+        p.st_h = sd(a->state, 1); p.st_p = sd(a->state, 2); p.st_n = sd(a->state, 3);
+    } else {
+        p.st_h = sd(a->state, 1); p.st_p = 0; p.st_n = sd(a->state, 2);
+    }
+    if (!non_overlapping(a->state)) return SSM_ERR_STRIDE;
+    // slot indices
+    if (present(a->state_batch_indices)) {
+        SSM_TRY(basic(a->state_batch_indices));
+        if (a->state_batch_indices.dtype != SSM_I32) return SSM_ERR_DTYPE;
+        SSM_TRY(want(a->state_batch_indices, {Bn}));
+        p.slot_idx = static_cast<const int32_t*>(a->state_batch_indices.data);
+        p.si_b = sd(a->state_batch_indices, 0);
+    } else if (slots != Bn) {
+        return SSM_ERR_SHAPE;
+    }
+    // conv
+    const int64_t Cch = H * P;
+    if (present(a->conv_weight)) {
+        SSM_TRY(basic(a->conv_weight));
+        if (a->conv_weight.ndim != 2 || a->conv_weight.shape[0] != Cch) return SSM_ERR_SHAPE;
+        if (a->conv_weight.dtype != SSM_F32) return SSM_ERR_DTYPE;
+        const int64_t W = a->conv_weight.shape[1];
+        if (W < 1) return SSM_ERR_SHAPE;
+        if (W > kMaxConvW) return SSM_ERR_UNSUPPORTED;
+        if (!present(a->conv_state)) return SSM_ERR_NULL;
+        SSM_TRY(basic(a->conv_state));
+        SSM_TRY(want(a->conv_state, {slots, Cch, W}));
+        if (!is_float(a->conv_state.dtype)) return SSM_ERR_DTYPE;
+        if (!non_overlapping(a->conv_state)) return SSM_ERR_STRIDE;
+        p.W = W;
+        p.conv_w = static_cast<const float*>(a->conv_weight.data);
+        p.cw_c = sd(a->conv_weight, 0); p.cw_w = sd(a->conv_weight, 1);
+        p.conv_state = a->conv_state.data; p.cs_dt = a->conv_state.dtype;
+        p.cs_b = sd(a->conv_state, 0); p.cs_c = sd(a->conv_state, 1); p.cs_w = sd(a->conv_state, 2);
+        if (present(a->conv_bias)) {
+            SSM_TRY(basic(a->conv_bias));
+            SSM_TRY(want(a->conv_bias, {Cch}));
+            if (a->conv_bias.dtype != SSM_F32) return SSM_ERR_DTYPE;
+            p.conv_b = static_cast<const float*>(a->conv_bias.data);
+            p.cb_c = sd(a->conv_bias, 0);
+        }
+    } else if (present(a->conv_state) || present(a->conv_bias)) {
+        return SSM_ERR_NULL;
+    }
+    if (!non_overlapping(a->out)) return SSM_ERR_STRIDE;
+    // aliasing: outputs vs inputs and vs each other
+    const ssm_tensor* ins[] = {&a->x, &a->dt, &a->A, &a->B, &a->C, &a->D, &a->z, &a->dt_bias,
+                               &a->conv_weight, &a->conv_bias, &a->state_batch_indices};
+    const ssm_tensor* outs[] = {&a->out, &a->state, &a->conv_state};
+    for (const ssm_tensor* o : outs) {
+        if (!present(*o)) continue;
+        for (const ssm_tensor* t : ins)
+            if (present(*t) && overlap(*o, *t)) return SSM_ERR_ALIAS;
+    }
+    if (overlap(a->out, a->state) || overlap(a->out, a->conv_state) ||
+        overlap(a->state, a->conv_state))
+        return SSM_ERR_ALIAS;
+    p.x = a->x.data; p.x_dt = a->x.dtype;
+    p.dt = a->dt.data; p.dt_dt = a->dt.dtype;
+    p.A = static_cast<const float*>(a->A.data);
+    p.Bm = a->B.data; p.B_dt = a->B.dtype;
+    p.Cm = a->C.data; p.C_dt = a->C.dtype;
+    p.softplus = a->dt_softplus != 0;
+    p.out = a->out.data; p.out_dt = a->out.dtype;
+
+    const bool dry = (a->flags & SSM_FLAG_DRY_RUN) != 0;
+    const int64_t HP = H * P;
+    if (Bn == 0) {
+        fill_info(a->info, SSM_KERNEL_NONE, 0, 0, 0, 0, 0);
+        return SSM_OK;
+    }
+    if (HP > INT32_MAX) return SSM_ERR_UNSUPPORTED;
+
+    // ---- plan: vector kernel when the state rows are 16-byte addressable
+    SsuPlan plan{};
+    const int es = esize(p.state_dt);
+    bool vec = p.st_n == 1 && (N * es) % 16 == 0 && aligned16(p.state) &&
+               (p.st_b * es) % 16 == 0 && (p.st_h * es) % 16 == 0 && (p.st_p * es) % 16 == 0;
+    if (vec && p.A_full) {
+        const int ve = 16 / es;
+        vec = p.A_n == 1 && aligned16(p.A) && (p.A_h * 4) % 16 == 0 && (p.A_p * 4) % 16 == 0 &&
+              ve % 4 == 0;
+    }
+    int lpr = 0, cpl = 0;
+    if (vec) {
+        const int64_t cpr = N * es / 16;  // 16-byte chunks per row
+        lpr = 1;
+        while (lpr < 32 && cpr % (2 * lpr) == 0) lpr *= 2;
+        cpl = (int)(cpr / lpr);
+        if (cpl > 2) vec = false;
+    }
+    const int sms = sm_count(dry);
+    if (vec) {
+        plan.kernel = SSM_KERNEL_SSU_VEC;
+        plan.block = 256;
+        plan.lpr = lpr;
+        plan.cpl = cpl;
+        const int64_t rows_per_pass = plan.block / lpr;
+        const int64_t row_bytes = N * es;
+        // target ~32 KB of state per work item, but at least one item per CTA slot
+        const int64_t total_rows = Bn * HP;
+        const int64_t ctas = (int64_t)sms * 8;
+        int64_t rpi = std::max<int64_t>(rows_per_pass, (32 * 1024) / row_bytes);
+        rpi = std::min<int64_t>(rpi, std::max<int64_t>(rows_per_pass, (total_rows + ctas - 1) / ctas));
+        rpi = (rpi + rows_per_pass - 1) / rows_per_pass * rows_per_pass;
+        rpi = std::min<int64_t>(rpi, HP);
+        if (G > 1) {
+            // an item must not straddle a group: take the largest divisor of the
+            // group's row count not above the target
+            const int64_t rg = p.heads_per_group * P;
+            int64_t best = 1;
+            for (int64_t dv = 1; dv * dv <= rg; ++dv) {
+                if (rg % dv) continue;
+                if (dv <= rpi) best = std::max(best, dv);
+                if (rg / dv <= rpi) best = std::max(best, rg / dv);
+            }
+            rpi = best;
+        }
+        plan.rows_per_item = rpi;
+        plan.items_per_b = (HP + rpi - 1) / rpi;
+        plan.n_items = Bn * plan.items_per_b;
+        plan.grid = (int)std::min<int64_t>(plan.n_items, ctas);
+    } else {
+        plan.kernel = SSM_KERNEL_SSU_GENERIC;
+        plan.block = 128;
+        const int64_t rows = Bn * HP;
+        plan.rows_per_item = 1;
+        plan.n_items = rows;
+        plan.grid = (int)std::min<int64_t>((rows + 127) / 128, (int64_t)sms * 16);
+    }
+    fill_info(a->info, plan.kernel, plan.grid, plan.block, 0, plan.rows_per_item, plan.n_items);
+    if (dry) return SSM_OK;
+    return launch_ssu(p, plan, stream) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+ssm_status ssm_causal_conv1d_fwd(const ssm_conv1d_args* args, void* stream) {
+    return conv1d_impl(args, static_cast<cudaStream_t>(stream));
+}
+
+ssm_status ssm_selective_scan_fwd(const ssm_scan_args* args, void* stream) {
+    return scan_impl(args, static_cast<cudaStream_t>(stream));
+}
+
+ssm_status ssm_selective_state_update(const ssm_ssu_args* args, void* stream) {
+    return ssu_impl(args, static_cast<cudaStream_t>(stream));
+}
+
+const char* ssm_status_string(int status) {
+    switch (status) {
+        case SSM_OK: return "SSM_OK";
+        case SSM_ERR_NULL: return "SSM_ERR_NULL: a required pointer is NULL";
+        case SSM_ERR_SHAPE: return "SSM_ERR_SHAPE: rank or sizes inconsistent";
+        case SSM_ERR_DTYPE: return "SSM_ERR_DTYPE: unsupported dtype or dtype combination";
+        case SSM_ERR_STRIDE: return "SSM_ERR_STRIDE: negative, overlapping or unaddressable layout";
+        case SSM_ERR_UNSUPPORTED: return "SSM_ERR_UNSUPPORTED: outside the implemented range";
+        case SSM_ERR_CUDA: return "SSM_ERR_CUDA: the CUDA launch failed";
+        case SSM_ERR_INTERNAL: return "SSM_ERR_INTERNAL: library invariant failed";
+        case SSM_ERR_VERSION: return "SSM_ERR_VERSION: struct_size does not match the library";
+        case SSM_ERR_ALIAS: return "SSM_ERR_ALIAS: an output overlaps an input";
+        default: return "unknown ssm_status";
+    }
+}
+
+int ssm_abi_version(void) { return SSM_CAUSAL_ABI_VERSION; }
+
+size_t ssm_struct_size(int which) {
+    switch (which) {
+        case 0: return sizeof(ssm_tensor);
+        case 1: return sizeof(ssm_conv1d_args);
+        case 2: return sizeof(ssm_scan_args);
+        case 3: return sizeof(ssm_ssu_args);
+        case 4: return sizeof(ssm_launch_info);
+        default: return 0;
+    }
+}
+
+}  // extern "C"

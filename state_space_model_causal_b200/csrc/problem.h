@@ -1,0 +1,98 @@
+// problem.h -- normalised problem descriptors passed from the C-ABI layer
+// (api.cpp) to the kernel launchers.  Host and device share these PODs; all
+// strides are in elements, all offsets are 64-bit.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ssm {
+
+// Single-token state update in the normalised (B, H, P, N) form.  A Mamba-1
+// problem (d_inner channels) is mapped to H = d_inner heads of headdim P = 1,
+// so that channel c = h * P + p and group g = h / (H / G) hold in both layouts.
+struct SsuProblem {
+    int64_t Bn, H, P, N, G, W;  // W = 0: no fused conv
+    int64_t heads_per_group;    // H / G
+    void* state;  int state_dt;  int64_t st_b, st_h, st_p, st_n;
+    const void* x;  int x_dt;  int64_t x_b, x_h, x_p;
+    const void* dt; int dt_dt; int64_t dt_b, dt_h, dt_p;
+    const float* A; int64_t A_h, A_p, A_n; int A_full;  // A_full = 0: A[h * A_h] per head
+    const void* Bm; int B_dt; int64_t B_b, B_g, B_n;
+    const void* Cm; int C_dt; int64_t C_b, C_g, C_n;
+    const float* Dp; int64_t D_h, D_p;
+    const void* z;  int z_dt;  int64_t z_b, z_h, z_p;
+    const float* dt_bias; int64_t db_h, db_p;
+    int softplus;
+    void* conv_state; int cs_dt; int64_t cs_b, cs_c, cs_w;
+    const float* conv_w; int64_t cw_c, cw_w;
+    const float* conv_b; int64_t cb_c;
+    const int32_t* slot_idx; int64_t si_b;  // NULL: batch row b uses cache slot b
+    int64_t n_slots;                        // dim 0 of the caches; other indices are padding
+    void* out; int out_dt; int64_t o_b, o_h, o_p;
+};
+
+struct SsuPlan {
+    int kernel;          // ssm_kernel_id
+    int block;           // threads per CTA
+    int grid;            // CTAs
+    int lpr;             // lanes per state row (vector kernel)
+    int cpl;             // 16-byte chunks per lane per row (vector kernel)
+    int64_t rows_per_item;
+    int64_t items_per_b;
+    int64_t n_items;
+};
+
+// Fused prefill (Mamba-1 layout): x, dt, z, out (B, D, L); B, C (B, G, N, L).
+struct ScanProblem {
+    int64_t Bn, D, L, N, G, W;  // W = 0: no fused conv (u = x)
+    int64_t ch_per_group;       // D / G
+    int io_dt;
+    const void* x;  int64_t x_b, x_d, x_t;
+    const void* dt; int64_t dt_b, dt_d, dt_t;
+    const float* A; int64_t A_d, A_n;
+    const void* Bm; int64_t B_b, B_g, B_n, B_t;
+    const void* Cm; int64_t C_b, C_g, C_n, C_t;
+    const float* Dp; int64_t D_d;
+    const void* z;  int64_t z_b, z_d, z_t;
+    const float* dt_bias; int64_t db_d;
+    int softplus;
+    const float* conv_w; int64_t cw_d, cw_k;
+    const float* conv_b; int64_t cb_d;
+    void* conv_state; int cs_dt; int64_t cs_b, cs_d, cs_k;
+    float* ssm_state; int64_t ss_b, ss_d, ss_n;
+    void* out; int64_t o_b, o_d, o_t;
+};
+
+struct ScanPlan {
+    int kernel;
+    int block;
+    int grid;
+    int ns;         // threads per channel (chunked kernel)
+    int dt_tile;    // channels per CTA
+    int t_chunk;    // time steps per smem chunk
+    int smem;       // dynamic shared memory bytes
+};
+
+struct Conv1dProblem {
+    int64_t Bn, D, L, W;
+    int io_dt;
+    const void* x; int64_t x_b, x_d, x_t;
+    const float* w; int64_t w_d, w_k;
+    const float* bias; int64_t b_d;
+    void* conv_state; int cs_dt; int64_t cs_b, cs_d, cs_k;
+    int silu;
+    void* out; int64_t o_b, o_d, o_t;
+};
+
+struct Conv1dPlan {
+    int kernel;
+    int block;
+    int grid;
+};
+
+cudaError_t launch_ssu(const SsuProblem& p, const SsuPlan& plan, cudaStream_t s);
+cudaError_t launch_scan(const ScanProblem& p, const ScanPlan& plan, cudaStream_t s);
+cudaError_t launch_conv1d(const Conv1dProblem& p, const Conv1dPlan& plan, cudaStream_t s);
+
+}  // namespace ssm

@@ -1,0 +1,337 @@
+"""Host-side checks of the C ABI (no GPU needed, nothing is launched).
+
+The library must load, export every function that include/ssm_causal.h
+declares, agree with the binding on struct layouts, and reject every invalid
+argument with its documented status before any CUDA call.  Valid calls are
+made in dry-run mode (SSM_FLAG_DRY_RUN), which checks and plans but launches
+nothing, so the chosen kernel and launch shape can be inspected on the CPU.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from state_space_model_causal_b200 import binding as bd
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ssm_causal.h")
+
+F32, F16, BF16, I32 = bd.SSM_F32, bd.SSM_F16, bd.SSM_BF16, bd.SSM_I32
+OK, ENULL, ESHAPE, EDTYPE, ESTRIDE, EUNSUP, ECUDA, EINT, EVER, EALIAS = range(10)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return bd.library()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*[A-Za-z_][\w\s\*]*?\b(ssm_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_header_declares_the_three_entry_points():
+    fns = declared_functions()
+    for name in ("ssm_causal_conv1d_fwd", "ssm_selective_scan_fwd", "ssm_selective_state_update",
+                 "ssm_status_string", "ssm_abi_version", "ssm_struct_size"):
+        assert name in fns
+
+
+def test_library_exports_every_declared_symbol(lib):
+    missing = [f for f in declared_functions() if not hasattr(lib, f)]
+    assert not missing, f"declared but not exported: {missing}"
+
+
+def test_abi_version_and_struct_layouts(lib):
+    assert lib.ssm_abi_version() == 1
+    for which, st in enumerate((bd.Tensor, bd.Conv1dArgs, bd.ScanArgs, bd.SsuArgs, bd.LaunchInfo)):
+        assert lib.ssm_struct_size(which) == ctypes.sizeof(st)
+    assert lib.ssm_struct_size(99) == 0
+
+
+def test_status_strings(lib):
+    for code, name in bd.STATUS.items():
+        assert lib.ssm_status_string(code).decode().startswith(name)
+    assert lib.ssm_status_string(1234).decode() == "unknown ssm_status"
+
+
+# ---------------------------------------------------------------- helpers --
+class FakeMem:
+    """Hands out distinct, 256-byte-aligned fake device addresses far apart."""
+
+    def __init__(self):
+        self.next = 1 << 40
+
+    def __call__(self, dtype, shape, stride=None):
+        ptr = self.next
+        self.next += 1 << 36
+        return bd.raw_tensor(ptr, dtype, shape, stride)
+
+
+def scan_args(mem, Bn=4, D=5120, L=2048, N=16, G=None, W=4, io=F16, **over):
+    a = bd.ScanArgs()
+    a.struct_size = ctypes.sizeof(bd.ScanArgs)
+    a.flags = bd.SSM_FLAG_DRY_RUN
+    a.x = mem(io, (Bn, D, L))
+    a.dt = mem(io, (Bn, D, L))
+    a.A = mem(F32, (D, N))
+    bshape = (Bn, N, L) if G is None else (Bn, G, N, L)
+    a.B = mem(io, bshape)
+    a.C = mem(io, bshape)
+    a.D = mem(F32, (D,))
+    a.z = mem(io, (Bn, D, L))
+    a.dt_bias = mem(F32, (D,))
+    a.dt_softplus = 1
+    if W:
+        a.conv_weight = mem(F32, (D, W))
+        a.conv_bias = mem(F32, (D,))
+        a.conv_state = mem(F32, (Bn, D, W))
+    a.ssm_state = mem(F32, (Bn, D, N))
+    a.out = mem(io, (Bn, D, L))
+    for k, v in over.items():
+        setattr(a, k, v)
+    return a
+
+
+def ssu_m1_args(mem, Bn=245, D=5120, N=16, W=4, io=F16, st=F32, **over):
+    a = bd.SsuArgs()
+    a.struct_size = ctypes.sizeof(bd.SsuArgs)
+    a.flags = bd.SSM_FLAG_DRY_RUN
+    a.state = mem(st, (Bn, D, N))
+    a.x = mem(io, (Bn, D))
+    a.dt = mem(io, (Bn, D))
+    a.A = mem(F32, (D, N))
+    a.B = mem(io, (Bn, 1, N))
+    a.C = mem(io, (Bn, 1, N))
+    a.D = mem(F32, (D,))
+    a.z = mem(io, (Bn, D))
+    a.dt_bias = mem(F32, (D,))
+    a.dt_softplus = 1
+    if W:
+        a.conv_weight = mem(F32, (D, W))
+        a.conv_bias = mem(F32, (D,))
+        a.conv_state = mem(F32, (Bn, D, W))
+    a.out = mem(io, (Bn, D))
+    for k, v in over.items():
+        setattr(a, k, v)
+    return a
+
+
+def ssu_m2_args(mem, Bn=8, H=80, P=64, N=128, G=1, io=F16, st=F16, **over):
+    a = bd.SsuArgs()
+    a.struct_size = ctypes.sizeof(bd.SsuArgs)
+    a.flags = bd.SSM_FLAG_DRY_RUN
+    a.state = mem(st, (Bn, H, P, N))
+    a.x = mem(io, (Bn, H, P))
+    a.dt = mem(io, (Bn, H))
+    a.A = mem(F32, (H,))
+    a.B = mem(io, (Bn, G, N))
+    a.C = mem(io, (Bn, G, N))
+    a.D = mem(F32, (H,))
+    a.dt_bias = mem(F32, (H,))
+    a.dt_softplus = 1
+    a.out = mem(io, (Bn, H, P))
+    for k, v in over.items():
+        setattr(a, k, v)
+    return a
+
+
+def conv_args(mem, Bn=2, D=64, L=100, W=4, io=F16, **over):
+    a = bd.Conv1dArgs()
+    a.struct_size = ctypes.sizeof(bd.Conv1dArgs)
+    a.flags = bd.SSM_FLAG_DRY_RUN
+    a.x = mem(io, (Bn, D, L))
+    a.weight = mem(F32, (D, W))
+    a.bias = mem(F32, (D,))
+    a.conv_state = mem(F32, (Bn, D, W))
+    a.silu = 1
+    a.out = mem(io, (Bn, D, L))
+    for k, v in over.items():
+        setattr(a, k, v)
+    return a
+
+
+def call(lib, fn, args):
+    info = bd.LaunchInfo()
+    info.struct_size = ctypes.sizeof(bd.LaunchInfo)
+    args.info = ctypes.pointer(info)
+    st = getattr(lib, fn)(ctypes.byref(args), None)
+    return st, info
+
+
+# ------------------------------------------------------------- valid plans --
+def test_prefill_2p8b_plan(lib):
+    st, info = call(lib, "ssm_selective_scan_fwd", scan_args(FakeMem()))
+    assert st == OK
+    assert bd.KERNELS[info.kernel] == "scan_chunked"
+    assert info.block == 64 and info.rows_per_item == 16
+    assert info.grid == 4 * 5120 // 16
+
+
+def test_small_scan_plan_and_generic_for_large_state(lib):
+    mem = FakeMem()
+    st, info = call(lib, "ssm_selective_scan_fwd", scan_args(mem, Bn=1, D=64, L=128, W=0, io=F32))
+    assert st == OK and bd.KERNELS[info.kernel] == "scan_chunked"
+    st, info = call(lib, "ssm_selective_scan_fwd", scan_args(mem, Bn=1, D=8, L=16, N=128, W=0))
+    assert st == OK and bd.KERNELS[info.kernel] == "scan_generic"
+
+
+def test_scan_groups_choose_generic_when_tile_straddles_groups(lib):
+    mem = FakeMem()
+    st, info = call(lib, "ssm_selective_scan_fwd", scan_args(mem, Bn=1, D=64, L=8, G=4))
+    assert st == OK and bd.KERNELS[info.kernel] == "scan_chunked"  # 16 channels per group
+    st, info = call(lib, "ssm_selective_scan_fwd", scan_args(mem, Bn=1, D=24, L=8, G=3))
+    assert st == OK and bd.KERNELS[info.kernel] == "scan_generic"  # 8 channels per group
+
+
+def test_decode_2p8b_plan(lib):
+    st, info = call(lib, "ssm_selective_state_update", ssu_m1_args(FakeMem()))
+    assert st == OK and bd.KERNELS[info.kernel] == "ssu_vec"
+    assert info.block == 256 and info.grid == 148 * 8
+
+
+@pytest.mark.parametrize("P,N,st_dt,io", [(64, 128, F16, F16), (64, 128, F32, F16),
+                                          (128, 256, BF16, BF16), (128, 256, F32, BF16)])
+@pytest.mark.parametrize("R", [8, 128, 4096, 131072])
+def test_mamba2_plans_use_vector_kernel(lib, P, N, st_dt, io, R):
+    H = 80 if N == 128 else 32
+    Bn, Hr = (-(-R // H), H) if R >= H else (1, R)
+    st, info = call(lib, "ssm_selective_state_update",
+                    ssu_m2_args(FakeMem(), Bn=Bn, H=Hr, P=P, N=N, io=io, st=st_dt))
+    assert st == OK and bd.KERNELS[info.kernel] == "ssu_vec"
+    assert 0 < info.grid <= 148 * 8
+    assert info.work_items * info.rows_per_item >= Bn * Hr * P
+
+
+def test_mamba2_groups_items_do_not_straddle_groups(lib):
+    st, info = call(lib, "ssm_selective_state_update", ssu_m2_args(FakeMem(), Bn=3, H=12, P=6, N=128, G=4))
+    assert st == OK and bd.KERNELS[info.kernel] == "ssu_vec"
+    assert (12 // 4 * 6) % info.rows_per_item == 0
+
+
+def test_ssu_generic_for_unaligned_rows(lib):
+    mem = FakeMem()
+    st, info = call(lib, "ssm_selective_state_update", ssu_m2_args(mem, N=3, st=F32))
+    assert st == OK and bd.KERNELS[info.kernel] == "ssu_generic"
+    # dstate not contiguous
+    a = ssu_m2_args(mem, Bn=2, H=4, P=8, N=16, st=F32)
+    a.state = mem(F32, (2, 4, 8, 16), (4 * 8 * 16 * 2, 8 * 16 * 2, 16 * 2, 2))
+    st, info = call(lib, "ssm_selective_state_update", a)
+    assert st == OK and bd.KERNELS[info.kernel] == "ssu_generic"
+
+
+def test_empty_problems_launch_nothing(lib):
+    mem = FakeMem()
+    st, info = call(lib, "ssm_selective_scan_fwd", scan_args(mem, Bn=2, D=16, L=0))
+    assert st == OK and info.kernel == 0 and info.grid == 0
+    st, info = call(lib, "ssm_selective_state_update", ssu_m2_args(mem, Bn=0))
+    assert st == OK and info.kernel == 0
+    st, info = call(lib, "ssm_causal_conv1d_fwd", conv_args(mem, L=0))
+    assert st == OK and info.kernel == 0
+
+
+def test_conv_plan(lib):
+    st, info = call(lib, "ssm_causal_conv1d_fwd", conv_args(FakeMem()))
+    assert st == OK and bd.KERNELS[info.kernel] == "conv1d" and info.grid == 2 * 64 // 4
+
+
+# ------------------------------------------------------------ error paths --
+def test_null_args_and_version(lib):
+    for fn in ("ssm_causal_conv1d_fwd", "ssm_selective_scan_fwd", "ssm_selective_state_update"):
+        assert getattr(lib, fn)(None, None) == ENULL
+    a = scan_args(FakeMem())
+    a.struct_size -= 8
+    assert lib.ssm_selective_scan_fwd(ctypes.byref(a), None) == EVER
+    a = scan_args(FakeMem())
+    info = bd.LaunchInfo()
+    info.struct_size = 3
+    a.info = ctypes.pointer(info)
+    assert lib.ssm_selective_scan_fwd(ctypes.byref(a), None) == EVER
+
+
+def _expect(lib, fn, args, status):
+    st, _ = call(lib, fn, args)
+    assert st == status, f"{fn}: expected {bd.STATUS[status]}, got {bd.STATUS.get(st, st)}"
+
+
+def test_scan_error_paths(lib):
+    fn = "ssm_selective_scan_fwd"
+    m = FakeMem()
+    _expect(lib, fn, scan_args(m, x=bd.Tensor()), ENULL)                       # missing x
+    _expect(lib, fn, scan_args(m, dt=m(F16, (4, 5120, 2047))), ESHAPE)         # dt length
+    _expect(lib, fn, scan_args(m, A=m(F16, (5120, 16))), EDTYPE)               # A not f32
+    _expect(lib, fn, scan_args(m, dt=m(F32, (4, 5120, 2048))), EDTYPE)         # mixed io
+    _expect(lib, fn, scan_args(m, x=m(F16, (4, 5120, 2048), (5120 * 2048, 2048, -1))), ESTRIDE)
+    _expect(lib, fn, scan_args(m, out=m(F16, (4, 5120, 2048), (5120 * 2048, 2048, 0))), ESTRIDE)
+    _expect(lib, fn, scan_args(m, Bn=1, D=10, L=4, G=3), ESHAPE)               # G does not divide D
+    _expect(lib, fn, scan_args(m, Bn=1, D=8, L=4, N=300), EUNSUP)              # N > 256
+    _expect(lib, fn, scan_args(m, Bn=1, D=8, L=4, W=9), EUNSUP)                # W > 8
+    a = scan_args(m, Bn=1, D=8, L=4, W=0)
+    a.conv_state = m(F32, (1, 8, 4))
+    _expect(lib, fn, a, ENULL)                                                 # state without weight
+    a = scan_args(m, Bn=1, D=8, L=4)
+    a.out = a.x                                                                # in-place out
+    _expect(lib, fn, a, EALIAS)
+    a = scan_args(m, Bn=1, D=8, L=4)
+    a.ssm_state = a.conv_state
+    _expect(lib, fn, a, ESHAPE)
+    a = scan_args(m, Bn=1, D=8, L=4)
+    a.x.data += 1                                                              # misaligned element
+    _expect(lib, fn, a, ESTRIDE)
+    a = scan_args(m, Bn=1, D=8, L=4)
+    a.x.dtype = 7
+    _expect(lib, fn, a, EDTYPE)
+    a = scan_args(m, Bn=1, D=8, L=4)
+    a.x.ndim = 0
+    _expect(lib, fn, a, ESHAPE)
+
+
+def test_ssu_error_paths(lib):
+    fn = "ssm_selective_state_update"
+    m = FakeMem()
+    _expect(lib, fn, ssu_m2_args(m, state=bd.Tensor()), ENULL)
+    _expect(lib, fn, ssu_m2_args(m, x=m(F16, (8, 80, 63))), ESHAPE)
+    _expect(lib, fn, ssu_m2_args(m, A=m(F16, (80,))), EDTYPE)
+    _expect(lib, fn, ssu_m2_args(m, H=80, G=3), ESHAPE)                        # G does not divide H
+    _expect(lib, fn, ssu_m2_args(m, N=512, st=F32), EUNSUP)
+    _expect(lib, fn, ssu_m2_args(m, state=m(F16, (8, 80, 64, 128), (0, 8192, 128, 1))), ESTRIDE)
+    _expect(lib, fn, ssu_m1_args(m, W=9), EUNSUP)
+    a = ssu_m1_args(m)
+    a.conv_state = bd.Tensor()
+    _expect(lib, fn, a, ENULL)                                                 # conv weight without state
+    a = ssu_m1_args(m)
+    a.out = a.x
+    _expect(lib, fn, a, EALIAS)
+    a = ssu_m1_args(m, Bn=4, D=8)
+    a.state = m(F32, (6, 8, 16))                                               # slots != batch
+    a.conv_state = m(F32, (6, 8, 4))
+    _expect(lib, fn, a, ESHAPE)
+    a.state_batch_indices = m(I32, (4,))
+    _expect(lib, fn, a, OK)                                                    # ... unless indexed
+    a.state_batch_indices = m(F32, (4,))
+    _expect(lib, fn, a, EDTYPE)
+    a = ssu_m1_args(m, Bn=4, D=8)
+    a.dt = m(F16, (4, 8, 1))                                                   # rank-3 dt is Mamba-2 only
+    _expect(lib, fn, a, ESHAPE)
+
+
+def test_conv_error_paths(lib):
+    fn = "ssm_causal_conv1d_fwd"
+    m = FakeMem()
+    _expect(lib, fn, conv_args(m, weight=bd.Tensor()), ENULL)
+    _expect(lib, fn, conv_args(m, out=m(F32, (2, 64, 100))), EDTYPE)
+    _expect(lib, fn, conv_args(m, weight=m(F32, (64, 9))), EUNSUP)
+    _expect(lib, fn, conv_args(m, weight=m(F32, (64, 0))), ESHAPE)
+    _expect(lib, fn, conv_args(m, conv_state=m(F32, (2, 64, 3))), ESHAPE)
+    a = conv_args(m)
+    a.out = a.x
+    _expect(lib, fn, a, EALIAS)
+
+
+def test_binding_rejects_cpu_tensors():
+    torch = pytest.importorskip("torch")
+    x = torch.zeros(1, 2, 3)
+    with pytest.raises(ValueError, match="CUDA tensors only"):
+        bd.describe(x)

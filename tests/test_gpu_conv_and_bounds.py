@@ -1,0 +1,129 @@
+"""GPU parity of the standalone causal conv1d, and out-of-bounds guards: every
+output and cache is placed inside a larger buffer whose surrounding bands
+hold a fixed bit pattern, which must survive every kernel unchanged."""
+import numpy as np
+import pytest
+
+import oracle
+from state_space_model_causal_b200 import inputs as gen
+from tests.parity import TOL, N, T, assert_close
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("io", ["f32", "f16", "bf16"])
+@pytest.mark.parametrize("L,W", [(1, 4), (3, 4), (4, 4), (255, 4), (256, 4), (257, 4), (700, 4),
+                                 (50, 1), (50, 2), (50, 8)])
+@pytest.mark.parametrize("silu", [False, True])
+def test_conv1d_matches_oracle(io, L, W, silu):
+    import torch
+    from state_space_model_causal_b200 import ssm_causal_conv1d_fwd
+    Bt, D = 2, 6
+    x = gen.round_to(gen.normal((Bt, D, L), "conv", L, W, "x"), io)
+    w = gen.round_to(gen.normal((D, W), "conv", L, W, "w", std=0.2), "f32")
+    b = gen.round_to(gen.normal((D,), "conv", L, W, "b"), "f32")
+    cs = gen.round_to(gen.normal((Bt, D, W), "conv", L, W, "cs"), "f32")
+    csg = T(cs, "f32")
+    out = ssm_causal_conv1d_fwd(T(x, io), T(w, "f32"), bias=T(b, "f32"), conv_state=csg, silu=silu)
+    torch.cuda.synchronize()
+    ref, csref = oracle.conv1d(x, w, bias=b, conv_state=cs, silu=silu)
+    assert_close(N(out), ref, TOL[io], "out")
+    np.testing.assert_array_equal(N(csg), csref)
+
+
+def test_conv1d_without_state_and_full_size():
+    import torch
+    from state_space_model_causal_b200 import ssm_causal_conv1d_fwd
+    s = gen.prefill_2p8b(seed=0)
+    out = ssm_causal_conv1d_fwd(T(s.x, "f16"), T(s.conv_weight, "f32"),
+                                bias=T(s.conv_bias, "f32"), silu=True)
+    torch.cuda.synchronize()
+    got = N(out)
+    rng = np.random.default_rng(3)
+    for b, d in zip(rng.integers(0, 4, 16), rng.integers(0, 5120, 16)):
+        ref, _ = oracle.conv1d(s.x[b:b + 1, d:d + 1], s.conv_weight[d:d + 1],
+                               bias=s.conv_bias[d:d + 1], silu=True)
+        assert_close(got[b:b + 1, d:d + 1], ref, TOL["f16"], f"row ({b},{d})")
+
+
+# ------------------------------------------------------------ canary bands --
+CANARY_WORDS = 4096  # 16 KiB of pattern on each side
+
+
+def _banded(shape, dtype):
+    """Tensor of `shape`/`dtype` carved out of a uint8 buffer with canary
+    bands of 0xA5 bytes before and after it."""
+    import torch
+    es = {torch.float32: 4, torch.float16: 2, torch.bfloat16: 2}[dtype]
+    n = int(np.prod(shape)) * es
+    pad = CANARY_WORDS * 4
+    buf = torch.full((pad + n + pad,), 0xA5, dtype=torch.uint8, device="cuda")
+    t = buf[pad:pad + n].view(dtype).view(*shape)
+    return buf, t, pad, n
+
+
+def _bands_intact(buf, pad, n):
+    import torch
+    return bool(torch.all(buf[:pad] == 0xA5)) and bool(torch.all(buf[pad + n:] == 0xA5))
+
+
+def test_prefill_writes_stay_inside_outputs():
+    import torch
+    from state_space_model_causal_b200 import ssm_selective_scan_fwd
+    s = gen.scan_inputs(3, 77, 40, 16, W=4, io="f16", seed=20, tag="canary", conv_state=True,
+                        h0=True)
+    bo, out, po, no = _banded((3, 40, 77), torch.float16)
+    bh, h, ph, nh = _banded((3, 40, 16), torch.float32)
+    bc, cs, pc, nc = _banded((3, 40, 4), torch.float32)
+    h.copy_(T(s.h0, "f32"))
+    cs.copy_(T(s.conv_state, "f32"))
+    ssm_selective_scan_fwd(T(s.x, "f16"), T(s.dt, "f16"), T(s.A, "f32"), T(s.B, "f16"),
+                           T(s.C, "f16"), D=T(s.D, "f32"), z=T(s.z, "f16"),
+                           dt_bias=T(s.dt_bias, "f32"), conv_weight=T(s.conv_weight, "f32"),
+                           conv_bias=T(s.conv_bias, "f32"), conv_state=cs, ssm_state=h, out=out)
+    torch.cuda.synchronize()
+    for buf, pad, n in ((bo, po, no), (bh, ph, nh), (bc, pc, nc)):
+        assert _bands_intact(buf, pad, n)
+
+
+@pytest.mark.parametrize("layout", ["mamba1", "mamba2"])
+def test_ssu_writes_stay_inside_caches(layout):
+    import torch
+    from state_space_model_causal_b200 import ssm_selective_state_update
+    if layout == "mamba1":
+        s = gen.ssu_mamba1_inputs(5, 72, 16, W=4, io="f16", state="f32", seed=21, tag="canary1")
+        bst, st, pst, nst = _banded(s.state.shape, torch.float32)
+        bcs, cs, pcs, ncs = _banded(s.conv_state.shape, torch.float32)
+        st.copy_(T(s.state, "f32"))
+        cs.copy_(T(s.conv_state, "f32"))
+        bo, out, po, no = _banded(s.x.shape, torch.float16)
+        ssm_selective_state_update(st, T(s.x, "f16"), T(s.dt, "f16"), T(s.A, "f32"), T(s.B, "f16"),
+                                   T(s.C, "f16"), D=T(s.D, "f32"), z=T(s.z, "f16"),
+                                   dt_bias=T(s.dt_bias, "f32"), conv_weight=T(s.conv_weight, "f32"),
+                                   conv_bias=T(s.conv_bias, "f32"), conv_state=cs, out=out)
+        bands = [(bst, pst, nst), (bcs, pcs, ncs), (bo, po, no)]
+    else:
+        s = gen.ssu_mamba2_inputs(3, 5, 24, 128, io="bf16", state="bf16", seed=22, tag="canary2")
+        bst, st, pst, nst = _banded(s.state.shape, torch.bfloat16)
+        st.copy_(T(s.state, "bf16"))
+        bo, out, po, no = _banded(s.x.shape, torch.bfloat16)
+        ssm_selective_state_update(st, T(s.x, "bf16"), T(s.dt, "bf16"), T(s.A, "f32"),
+                                   T(s.B, "bf16"), T(s.C, "bf16"), D=T(s.D, "f32"),
+                                   dt_bias=T(s.dt_bias, "f32"), out=out)
+        bands = [(bst, pst, nst), (bo, po, no)]
+    torch.cuda.synchronize()
+    for buf, pad, n in bands:
+        assert _bands_intact(buf, pad, n)
+
+
+def test_conv1d_writes_stay_inside_outputs():
+    import torch
+    from state_space_model_causal_b200 import ssm_causal_conv1d_fwd
+    x = gen.round_to(gen.normal((2, 9, 301), "cc", "x"), "f16")
+    w = gen.round_to(gen.normal((9, 4), "cc", "w"), "f32")
+    bo, out, po, no = _banded((2, 9, 301), torch.float16)
+    bc, cs, pc, nc = _banded((2, 9, 4), torch.float32)
+    cs.zero_()
+    ssm_causal_conv1d_fwd(T(x, "f16"), T(w, "f32"), conv_state=cs, silu=True, out=out)
+    torch.cuda.synchronize()
+    assert _bands_intact(bo, po, no) and _bands_intact(bc, pc, nc)

@@ -1,0 +1,173 @@
+"""GPU parity of the fused prefill (ssm_selective_scan_fwd) against the fp64
+oracle, on the same seeded inputs, through the C ABI."""
+import numpy as np
+import pytest
+
+from state_space_model_causal_b200 import inputs as gen
+from tests.parity import TOL, N, T, assert_close, run_scan_gpu, run_scan_oracle
+
+pytestmark = pytest.mark.gpu
+
+
+def _check(s, tol=None, softplus=True, conv_state_dtype="f32", with_state=True):
+    tol = tol or TOL[s.io]
+    out, h, cs = run_scan_gpu(s, softplus=softplus, conv_state_dtype=conv_state_dtype,
+                              with_state=with_state)
+    ref, href, csref = run_scan_oracle(s, softplus=softplus)
+    assert_close(out, ref, tol, "out")
+    if with_state:
+        assert_close(h, href, tol, "ssm_state")
+        if csref is not None:
+            # the final conv state is a copy of raw inputs: exact
+            np.testing.assert_array_equal(cs, gen.round_to(csref, conv_state_dtype))
+
+
+def test_scan_small_fp32_seed0():
+    """B=1, L=128, D=64, N=16, fp32, no conv, h0 = 0, seed 0."""
+    s = gen.scan_small(seed=0)
+    _check(s, tol=1e-5)
+
+
+def test_prefill_2p8b_shape_reduced_spans_tiles_and_ragged_tail():
+    """2.8B-shaped layer (N=16, W=4, fp16 I/O) at reduced D/L: several channel
+    tiles and a ragged last time chunk, incoming conv and ssm state."""
+    s = gen.scan_inputs(2, 100, 48, 16, W=4, io="f16", seed=1, tag="prefill_reduced",
+                        conv_state=True, h0=True)
+    _check(s)
+
+
+@pytest.mark.parametrize("io", ["f32", "f16", "bf16"])
+@pytest.mark.parametrize("N_", [1, 4, 8, 16, 33, 64])
+def test_scan_dstate_and_dtype_variants(io, N_):
+    s = gen.scan_inputs(2, 70, 40, N_, W=4, io=io, seed=2, tag=f"var{N_}{io}", conv_state=True,
+                        h0=True)
+    _check(s)
+
+
+@pytest.mark.parametrize("N_", [65, 128, 256])
+def test_scan_large_dstate_generic_kernel(N_):
+    s = gen.scan_inputs(1, 40, 6, N_, W=4, io="f32", seed=3, tag=f"big{N_}", h0=True)
+    _check(s)
+
+
+@pytest.mark.parametrize("W", [1, 2, 3, 4, 8])
+def test_scan_conv_widths(W):
+    s = gen.scan_inputs(2, 45, 20, 16, W=W, io="f32", seed=4, tag=f"w{W}", conv_state=True)
+    _check(s)
+
+
+@pytest.mark.parametrize("L", [1, 2, 3, 5, 31, 32, 33])
+def test_scan_short_sequences(L):
+    s = gen.scan_inputs(2, L, 24, 16, W=4, io="f32", seed=5, tag=f"L{L}", conv_state=True, h0=True)
+    _check(s)
+
+
+def test_scan_optional_inputs_absent_and_no_softplus():
+    s = gen.scan_inputs(2, 50, 32, 16, io="f32", seed=6, tag="noopt", with_z=False, with_D=False,
+                        with_dt_bias=False)
+    _check(s, with_state=False)
+    s = gen.scan_inputs(2, 50, 32, 16, io="f32", seed=7, tag="nosp", W=4)
+    s.dt = np.abs(s.dt) * 0.01  # keep delta positive without the softplus
+    _check(s, softplus=False)
+
+
+@pytest.mark.parametrize("G,D", [(2, 64), (4, 64), (3, 24)])
+def test_scan_groups(G, D):
+    s = gen.scan_inputs(2, 40, D, 16, G=G, W=4, io="f16", seed=8, tag=f"g{G}", h0=True)
+    _check(s)
+
+
+def test_scan_fp16_conv_state():
+    s = gen.scan_inputs(2, 37, 16, 16, W=4, io="f16", seed=9, tag="cs16", conv_state=True)
+    _check(s, conv_state_dtype="f16")
+
+
+def test_scan_strided_views_from_packed_projection():
+    """x and z as halves of one (B, 2D, L) projection output, B/C as slices of
+    a (B, 2N + R, L) tensor, and a non-unit time stride for dt."""
+    import torch
+    from state_space_model_causal_b200 import ssm_selective_scan_fwd
+    Bt, D, L, N_ = 2, 32, 60, 16
+    s = gen.scan_inputs(Bt, L, D, N_, W=4, io="f16", seed=10, tag="strided", h0=True)
+    xz = T(np.concatenate([s.x, s.z], axis=1), "f16")
+    x, z = xz[:, :D], xz[:, D:]
+    bc = T(np.concatenate([s.B[:, 0], s.C[:, 0], np.zeros((Bt, 3, L))], axis=1), "f16")
+    Bm, Cm = bc[:, :N_], bc[:, N_:2 * N_]
+    dt_wide = T(np.repeat(s.dt, 2, axis=-1), "f16")
+    dt = dt_wide[..., ::2]
+    h = T(s.h0, "f32")
+    out = ssm_selective_scan_fwd(x, dt, T(s.A, "f32"), Bm, Cm, D=T(s.D, "f32"), z=z,
+                                 dt_bias=T(s.dt_bias, "f32"), conv_weight=T(s.conv_weight, "f32"),
+                                 conv_bias=T(s.conv_bias, "f32"), ssm_state=h)
+    torch.cuda.synchronize()
+    ref, href, _ = run_scan_oracle(s)
+    assert_close(N(out), ref, TOL["f16"], "out")
+    assert_close(N(h), href, TOL["f16"], "ssm_state")
+
+
+def test_scan_empty_sequence_leaves_caches_unchanged():
+    import torch
+    from state_space_model_causal_b200 import ssm_selective_scan_fwd
+    s = gen.scan_inputs(2, 1, 8, 16, W=4, io="f32", seed=11, tag="empty", conv_state=True, h0=True)
+    z0 = torch.zeros(2, 8, 0, device="cuda")
+    bc = torch.zeros(2, 16, 0, device="cuda")
+    h = T(s.h0, "f32")
+    cs = T(s.conv_state, "f32")
+    ssm_selective_scan_fwd(z0, z0.clone(), T(s.A, "f32"), bc, bc.clone(), conv_weight=T(s.conv_weight, "f32"),
+                           conv_state=cs, ssm_state=h)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(N(h), s.h0)
+    np.testing.assert_array_equal(N(cs), s.conv_state)
+
+
+def test_prefill_2p8b_full_size_sampled_channels():
+    """Full 2.8B-shaped prefill (B=4, L=2048, D=5120, N=16, W=4, fp16) in the
+    launch configuration the benchmark times; 48 sampled channels are checked
+    against the oracle one by one."""
+    import torch
+    s = gen.prefill_2p8b(seed=0)
+    out, h, cs = run_scan_gpu(s)
+    rng = np.random.default_rng(123)
+    picks = [(int(b), int(d)) for b, d in zip(rng.integers(0, 4, 48), rng.integers(0, 5120, 48))]
+    picks += [(0, 0), (3, 5119)]
+    for b, d in picks:
+        sub = gen.ScanInputs(s.x[b:b + 1, d:d + 1], s.dt[b:b + 1, d:d + 1], s.A[d:d + 1],
+                             s.B[b:b + 1], s.C[b:b + 1], s.D[d:d + 1], s.z[b:b + 1, d:d + 1],
+                             s.dt_bias[d:d + 1], s.conv_weight[d:d + 1], s.conv_bias[d:d + 1],
+                             None, None, io="f16")
+        ref, href, csref = run_scan_oracle(sub)
+        assert_close(out[b:b + 1, d:d + 1], ref, TOL["f16"], f"out[{b},{d}]")
+        assert_close(h[b:b + 1, d:d + 1], href, TOL["f16"], f"state[{b},{d}]")
+        np.testing.assert_array_equal(cs[b, d], csref[0, 0])
+    assert np.isfinite(out).all()
+    torch.cuda.empty_cache()
+
+
+def test_prefill_then_decode_on_gpu_matches_full_prefill():
+    """GPU prefill of L-k tokens followed by k GPU decode steps (Mamba-1 layout
+    with the fused conv update) equals the oracle's full prefill."""
+    import torch
+    from state_space_model_causal_b200 import ssm_selective_scan_fwd, ssm_selective_state_update
+    L, k = 40, 5
+    s = gen.scan_inputs(2, L, 32, 16, W=4, io="f32", seed=12, tag="pd", conv_state=True, h0=True)
+    h = T(s.h0, "f32")
+    cs = T(s.conv_state, "f32")
+    cut = lambda a: T(np.ascontiguousarray(a[..., :L - k]), "f32")  # noqa: E731
+    ssm_selective_scan_fwd(cut(s.x), cut(s.dt), T(s.A, "f32"), cut(s.B), cut(s.C),
+                           D=T(s.D, "f32"), z=cut(s.z), dt_bias=T(s.dt_bias, "f32"),
+                           conv_weight=T(s.conv_weight, "f32"), conv_bias=T(s.conv_bias, "f32"),
+                           conv_state=cs, ssm_state=h)
+    outs = []
+    for t in range(L - k, L):
+        o = ssm_selective_state_update(h, T(s.x[..., t], "f32"), T(s.dt[..., t], "f32"),
+                                       T(s.A, "f32"), T(s.B[..., t], "f32"), T(s.C[..., t], "f32"),
+                                       D=T(s.D, "f32"), z=T(s.z[..., t], "f32"),
+                                       dt_bias=T(s.dt_bias, "f32"),
+                                       conv_weight=T(s.conv_weight, "f32"),
+                                       conv_bias=T(s.conv_bias, "f32"), conv_state=cs)
+        outs.append(N(o))
+    torch.cuda.synchronize()
+    ref, href, csref = run_scan_oracle(s)
+    assert_close(np.stack(outs, -1), ref[..., L - k:], 1e-5, "decoded outputs")
+    assert_close(N(h), href, 1e-5, "final ssm_state")
+    np.testing.assert_array_equal(N(cs), csref)
