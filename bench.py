@@ -84,55 +84,64 @@ def profiled_traffic(summary_name, source_files):
 
 
 class ClockSampler:
-    """nvidia-smi samples of this GPU's clocks while the timed region runs."""
+    """Samples this GPU's SM clock and clock-event reasons through NVML every
+    few milliseconds while the timed region runs (read-only queries)."""
 
-    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
 
-    def __init__(self, uuid):
+    def __init__(self, uuid, period_s=0.005):
         self.uuid = uuid
-        self.proc = None
+        self.period = period_s
+        self.samples = []
+        self.max_mhz = None
+        self._stop = None
+        self._thread = None
+        self.error = None
 
     def __enter__(self):
+        import threading
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except Exception:
-            self.proc = None
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByUUID(self.uuid)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+            masks = [(n, getattr(pynvml, attr)) for n, attr in self.REASONS]
+        except Exception as e:  # no NVML: record why, keep running
+            self.error = f"nvml unavailable: {e}"
+            return self
+        self._stop = threading.Event()
+
+        def run():
+            while not self._stop.is_set():
+                try:
+                    mhz = float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM))
+                    r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    self.samples.append((mhz, [n for n, m in masks if r & m]))
+                except Exception as e:
+                    self.error = str(e)
+                    return
+                self._stop.wait(self.period)
+
+        self._thread = threading.Thread(target=run, daemon=True)
+        self._thread.start()
         return self
 
     def __exit__(self, *exc):
-        self.lines = []
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                out, _ = self.proc.communicate(timeout=5)
-            except Exception:
-                self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [l for l in out.splitlines() if l.strip()]
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=2)
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in getattr(self, "lines", []):
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 8 or (self.uuid and self.uuid not in parts[0]):
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
-            except ValueError:
-                continue
-            for name, v in zip(names, parts[4:8]):
-                if v.lower().startswith("active"):
-                    reasons.add(name)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "note": self.error or "no samples"}
+        reasons = sorted({r for _, rs in self.samples for r in rs})
+        return {"sm_mhz": statistics.median(m for m, _ in self.samples),
+                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(self.samples),
+                "source": "NVML, 5 ms period, during the timed steps"}
 
 
 def device_uuid(dev):
@@ -426,16 +435,74 @@ def run_sweep(dev, hbm_peak):
     return out
 
 
+# ------------------------------------------------------ single cases --
+def run_only(args, dev):
+    """Warm-up then timed launches of one case, nothing else (profiling)."""
+    import torch
+    from state_space_model_causal_b200 import inputs as gen, ssm_selective_state_update
+    if args.only == "prefill":
+        pf = Prefill(dev)
+        fn = pf.run
+    elif args.only == "decode_m1":
+        Bt, D, N, W = 490, 5120, 16, 4  # two layers' worth of rows, 200 MB of state
+        tag = ("only", "decode_m1")
+        st = gen.device_normal((Bt, D, N), "f32", *tag, "state", device=dev)
+        cs = gen.device_normal((Bt, D, W), "f32", *tag, "cs", device=dev)
+        x = gen.device_normal((Bt, D), "f16", *tag, "x", device=dev)
+        dt = gen.device_uniform((Bt, D), -4.0, -1.0, "f16", *tag, "dt", device=dev)
+        z = gen.device_normal((Bt, D), "f16", *tag, "z", device=dev)
+        Bm = gen.device_normal((Bt, 1, N), "f16", *tag, "B", device=dev)
+        Cm = gen.device_normal((Bt, 1, N), "f16", *tag, "C", device=dev)
+        A = -torch.arange(1, N + 1, device=dev, dtype=torch.float32).repeat(D, 1)
+        Dv, db = torch.ones(D, device=dev), torch.full((D,), -3.0, device=dev)
+        cw = gen.device_normal((D, W), "f32", *tag, "cw", std=0.2, device=dev)
+        out = torch.empty_like(x)
+        fn = lambda: ssm_selective_state_update(st, x, dt, A, Bm, Cm, D=Dv, z=z, dt_bias=db,  # noqa
+                                                conv_weight=cw, conv_state=cs, out=out)
+    else:
+        H, P, N, cache, io = {"m2_f16": (80, 64, 128, "f16", "f16"),
+                              "m2_f32": (80, 64, 128, "f32", "f16"),
+                              "m2_bf16": (32, 128, 256, "bf16", "bf16"),
+                              "m2_f32_256": (32, 128, 256, "f32", "bf16")}[args.only]
+        Bt, Hr = gen.effective_batch_shape(args.R, H)
+        tag = ("only", args.only, args.R)
+        st = gen.device_normal((Bt, Hr, P, N), cache, *tag, "state", device=dev)
+        x = gen.device_normal((Bt, Hr, P), io, *tag, "x", device=dev)
+        dt = gen.device_uniform((Bt, Hr), -4.0, -1.0, io, *tag, "dt", device=dev)
+        Bm = gen.device_normal((Bt, 1, N), io, *tag, "B", device=dev)
+        Cm = gen.device_normal((Bt, 1, N), io, *tag, "C", device=dev)
+        A = -torch.linspace(1.0, 16.0, Hr, device=dev)
+        Dv, db = torch.ones(Hr, device=dev), torch.full((Hr,), -3.0, device=dev)
+        out = torch.empty_like(x)
+        fn = lambda: ssm_selective_state_update(st, x, dt, A, Bm, Cm, D=Dv, dt_bias=db, out=out)  # noqa
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        fn()
+    b.record()
+    torch.cuda.synchronize(dev)
+    print(f"{args.only}: {a.elapsed_time(b) * 1000 / args.steps:.1f} us per launch", flush=True)
+    return 0
+
+
 # ----------------------------------------------------------------- main --
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--sweep", action="store_true", help="per-effective-batch decode sweep lines")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--only", choices=["prefill", "decode_m1", "m2_f16", "m2_f32", "m2_bf16",
+                                       "m2_f32_256"],
+                    help="run --warmup then --steps launches of one case and exit "
+                         "(for profiler captures; prints no JSON line)")
+    ap.add_argument("--R", type=int, default=16384, help="effective batch for --only m2_*")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -466,6 +533,9 @@ def main():
         if rank == 0:
             run_sweep(dev, hbm_peak)
         return 0
+
+    if args.only:
+        return run_only(args, dev)
 
     pf = Prefill(dev)
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)

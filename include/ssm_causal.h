@@ -118,8 +118,17 @@ typedef enum ssm_kernel_id {
     SSM_KERNEL_CONV1D_GENERIC = 2,  /* any strides */
     SSM_KERNEL_SCAN_CHUNKED = 3,    /* fused prefill, smem-staged chunks of L */
     SSM_KERNEL_SCAN_GENERIC = 4,    /* fused prefill, any strides / group layout */
-    SSM_KERNEL_SSU_VEC = 5,         /* 128-bit streaming state update */
-    SSM_KERNEL_SSU_GENERIC = 6      /* state update, any strides / dstate */
+    SSM_KERNEL_SSU_VEC = 5,         /* 128-bit streaming state update, one decay per
+                                       head (Mamba-2 layout, scalar A, no conv) */
+    SSM_KERNEL_SSU_GENERIC = 6,     /* state update, any strides / dstate */
+    SSM_KERNEL_SCAN_VEC = 7,        /* fused prefill, 16-byte prefetched loads, packed
+                                       f32x2 scan; d_state <= 16, conv width 0 or 4,
+                                       time contiguous, L % 8 == 0, 16-byte aligned rows */
+    SSM_KERNEL_SSU_ROW = 8,         /* 128-bit state update with a decay per element
+                                       (Mamba-1 layout or full A), fused conv roll */
+    SSM_KERNEL_SSU_TMA = 9          /* state update fed by bulk copies (TMA) into
+                                       shared-memory stages: one decay per head, dense
+                                       rows (Mamba-2 layout, scalar A, no conv) */
 } ssm_kernel_id;
 
 /* ------------------------------------------------------------------------ *
@@ -255,6 +264,14 @@ typedef struct ssm_ssu_args {
 } ssm_ssu_args;
 
 ssm_status ssm_selective_state_update(const ssm_ssu_args* args, void* stream);
+
+/* Waits for the work enqueued on `stream` so far, then reports in *code the
+ * device-side error word of the library's kernels and clears it: 0 = none,
+ * 1 = a kernel gave up a bounded wait on one of its bulk copies and exited
+ * early (its outputs for that call are incomplete).  No kernel ever traps or
+ * hangs instead.  Returns SSM_ERR_NULL for a NULL code, SSM_ERR_CUDA if the
+ * stream or the copy fails. */
+ssm_status ssm_device_error(int* code, void* stream);
 
 /* Human-readable name of a status code (static storage, never NULL). */
 const char* ssm_status_string(int status);

@@ -33,7 +33,7 @@ STATUS = {
 }
 KERNELS = {
     0: "none", 1: "conv1d", 2: "conv1d_generic", 3: "scan_chunked", 4: "scan_generic",
-    5: "ssu_vec", 6: "ssu_generic",
+    5: "ssu_vec", 6: "ssu_generic", 7: "scan_vec", 8: "ssu_row", 9: "ssu_tma",
 }
 
 
@@ -108,6 +108,8 @@ def library():
             lib.ssm_status_string.restype = ctypes.c_char_p
             lib.ssm_status_string.argtypes = [ctypes.c_int]
             lib.ssm_abi_version.restype = ctypes.c_int
+            lib.ssm_device_error.restype = ctypes.c_int
+            lib.ssm_device_error.argtypes = [ctypes.POINTER(ctypes.c_int), ctypes.c_void_p]
             lib.ssm_struct_size.restype = ctypes.c_size_t
             lib.ssm_struct_size.argtypes = [ctypes.c_int]
             for which, st in enumerate((Tensor, Conv1dArgs, ScanArgs, SsuArgs, LaunchInfo)):
@@ -233,3 +235,13 @@ def ssm_selective_state_update(state, x, dt, A, B, C, D=None, z=None, dt_bias=No
     _check(library().ssm_selective_state_update(ctypes.byref(a), _stream_of([x], stream)),
            "ssm_selective_state_update")
     return out
+
+
+def ssm_device_error(stream=None) -> int:
+    """Wait for the current stream and return (and clear) the library's device
+    error word: 0 = none, 1 = a kernel gave up a bounded wait and exited early."""
+    import torch
+    code = ctypes.c_int(0)
+    st = stream.cuda_stream if stream is not None else torch.cuda.current_stream().cuda_stream
+    _check(library().ssm_device_error(ctypes.byref(code), st), "ssm_device_error")
+    return code.value

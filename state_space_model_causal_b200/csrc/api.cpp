@@ -10,6 +10,7 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 
 #include "problem.h"
@@ -346,6 +347,31 @@ ssm_status scan_impl(const ssm_scan_args* a, cudaStream_t stream) {
         return SSM_OK;
     }
     ScanPlan plan{};
+    const int es = esize(io);
+    auto al16 = [](const void* ptr) { return ptr == nullptr || aligned16(ptr); };
+    auto m16 = [es](int64_t st) { return (st * es) % 16 == 0; };
+    const bool vec_layout =
+        p.x_t == 1 && p.dt_t == 1 && p.o_t == 1 && p.B_t == 1 && p.C_t == 1 &&
+        (!p.z || p.z_t == 1) && al16(p.x) && al16(p.dt) && al16(p.out) && al16(p.Bm) &&
+        al16(p.Cm) && al16(p.z) && m16(p.x_b) && m16(p.x_d) && m16(p.dt_b) && m16(p.dt_d) &&
+        m16(p.o_b) && m16(p.o_d) && m16(p.B_b) && m16(p.B_g) && m16(p.B_n) && m16(p.C_b) &&
+        m16(p.C_g) && m16(p.C_n) && (!p.z || (m16(p.z_b) && m16(p.z_d)));
+    if (vec_layout && scan_vec_supported(p)) {
+        plan.kernel = SSM_KERNEL_SCAN_VEC;
+        plan.block = scan_vec_threads();
+        const int64_t tiles = (D + scan_vec_channels_per_cta() - 1) / scan_vec_channels_per_cta();
+        if (tiles * Bn > INT32_MAX) return SSM_ERR_UNSUPPORTED;
+        plan.grid = (int)(tiles * Bn);
+        plan.sw_pairs = 0;
+        if (const char* e = std::getenv("SSM_SCAN_SW_PAIRS")) {
+            const int v = std::atoi(e);
+            if (v >= 0 && v <= 2) plan.sw_pairs = v;
+        }
+        fill_info(a->info, plan.kernel, plan.grid, plan.block, 0, scan_vec_channels_per_cta(),
+                  tiles * Bn);
+        if (a->flags & SSM_FLAG_DRY_RUN) return SSM_OK;
+        return launch_scan(p, plan, stream) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+    }
     int ns = 1;
     while (ns * 4 < N) ns *= 2;
     const int dtile = 64 / (ns <= 16 ? ns : 16);
@@ -566,56 +592,111 @@ ssm_status ssu_impl(const ssm_ssu_args* a, cudaStream_t stream) {
     }
     if (HP > INT32_MAX) return SSM_ERR_UNSUPPORTED;
 
-    // ---- plan: vector kernel when the state rows are 16-byte addressable
+    // ---- plan: streaming kernels when the state rows are 16-byte addressable
     SsuPlan plan{};
     const int es = esize(p.state_dt);
-    bool vec = p.st_n == 1 && (N * es) % 16 == 0 && aligned16(p.state) &&
-               (p.st_b * es) % 16 == 0 && (p.st_h * es) % 16 == 0 && (p.st_p * es) % 16 == 0;
-    if (vec && p.A_full) {
-        const int ve = 16 / es;
-        vec = p.A_n == 1 && aligned16(p.A) && (p.A_h * 4) % 16 == 0 && (p.A_p * 4) % 16 == 0 &&
-              ve % 4 == 0;
-    }
-    int lpr = 0, cpl = 0;
-    if (vec) {
-        const int64_t cpr = N * es / 16;  // 16-byte chunks per row
-        lpr = 1;
-        while (lpr < 32 && cpr % (2 * lpr) == 0) lpr *= 2;
-        cpl = (int)(cpr / lpr);
-        if (cpl > 2) vec = false;
-    }
+    const bool vec_rows = p.st_n == 1 && (N * es) % 16 == 0 && aligned16(p.state) &&
+                          (p.st_b * es) % 16 == 0 && (p.st_h * es) % 16 == 0 &&
+                          (p.st_p * es) % 16 == 0;
+    const int64_t cpr = vec_rows ? N * es / 16 : 0;  // 16-byte chunks per row
     const int sms = sm_count(dry);
-    if (vec) {
-        plan.kernel = SSM_KERNEL_SSU_VEC;
-        plan.block = 256;
-        plan.lpr = lpr;
-        plan.cpl = cpl;
-        const int64_t rows_per_pass = plan.block / lpr;
-        const int64_t row_bytes = N * es;
-        // target ~32 KB of state per work item, but at least one item per CTA slot
-        const int64_t total_rows = Bn * HP;
-        const int64_t ctas = (int64_t)sms * 8;
-        int64_t rpi = std::max<int64_t>(rows_per_pass, (32 * 1024) / row_bytes);
-        rpi = std::min<int64_t>(rpi, std::max<int64_t>(rows_per_pass, (total_rows + ctas - 1) / ctas));
-        rpi = (rpi + rows_per_pass - 1) / rows_per_pass * rows_per_pass;
-        rpi = std::min<int64_t>(rpi, HP);
-        if (G > 1) {
-            // an item must not straddle a group: take the largest divisor of the
-            // group's row count not above the target
-            const int64_t rg = p.heads_per_group * P;
-            int64_t best = 1;
-            for (int64_t dv = 1; dv * dv <= rg; ++dv) {
-                if (rg % dv) continue;
-                if (dv <= rpi) best = std::max(best, dv);
-                if (rg / dv <= rpi) best = std::max(best, rg / dv);
+    const int64_t ctas = (int64_t)sms * (p.A_full || p.W ? 4 : 3);  // resident CTAs of 256 threads
+    const int64_t row_bytes = N * es;
+    auto pow2 = [](int64_t v) { return v > 0 && (v & (v - 1)) == 0; };
+    const bool dense_rows = p.st_p == N || P == 1;
+    if (vec_rows && dense_rows && !p.A_full && p.W == 0) {
+        // bulk-copy pipeline: items are contiguous row blocks of one head; one
+        // 16-byte chunk per lane for 16-bit states keeps B/C in 16 registers
+        int cpl = 0;
+        int64_t lpr = 0;
+        const int order[2] = {es == 2 ? 1 : 2, es == 2 ? 2 : 1};
+        for (int c : order) {
+            if (cpr % c) continue;
+            if (cpr / c <= 32 && pow2(cpr / c)) {
+                cpl = c;
+                lpr = cpr / c;
+                break;
             }
-            rpi = best;
         }
-        plan.rows_per_item = rpi;
-        plan.items_per_b = (HP + rpi - 1) / rpi;
-        plan.n_items = Bn * plan.items_per_b;
+        const int64_t rows_per_pass = 256 / std::max<int64_t>(lpr, 1);
+        const int64_t max_rows = rows_per_pass * ssu_tma_max_rows_per_thread();
+        if (cpl && row_bytes <= 16 * 1024) {
+            const int64_t ctas_tma = (int64_t)sms * 3;
+            int64_t rb = std::max<int64_t>(1, std::min<int64_t>({P, (16 * 1024) / row_bytes, max_rows}));
+            while (rb > 8 && Bn * H * ((P + rb - 1) / rb) < 2 * ctas_tma) rb = (rb + 1) / 2;
+            plan.kernel = SSM_KERNEL_SSU_TMA;
+            plan.block = 256;
+            plan.lpr = (int)lpr;
+            plan.cpl = cpl;
+            plan.rows_per_item = rb;
+            plan.items_per_b = H * ((P + rb - 1) / rb);
+            plan.n_items = Bn * plan.items_per_b;
+            plan.stage_bytes = (int)((rb * row_bytes + 127) / 128 * 128);
+        }
+    }
+    if (plan.kernel == 0 && vec_rows && !p.A_full && p.W == 0) {
+        // one decay per head: lanes split each row, per-head work once per item
+        int cpl = 0;
+        int64_t lpr = 0;
+        for (int c : {2, 4, 1}) {
+            if (cpr % c) continue;
+            if (cpr / c <= 32 && pow2(cpr / c)) {
+                cpl = c;
+                lpr = cpr / c;
+                break;
+            }
+        }
+        if (cpl) {
+            plan.kernel = SSM_KERNEL_SSU_VEC;
+            plan.block = 256;
+            plan.lpr = (int)lpr;
+            plan.cpl = cpl;
+            // ~32 KB of state per item, halved while the items cannot fill the GPU
+            int64_t rb = std::max<int64_t>(1, std::min<int64_t>(P, (32 * 1024) / row_bytes));
+            while (rb > 8 && Bn * H * ((P + rb - 1) / rb) < 2 * ctas) rb = (rb + 1) / 2;
+            plan.rows_per_item = rb;
+            plan.items_per_b = H * ((P + rb - 1) / rb);
+            plan.n_items = Bn * plan.items_per_b;
+        }
+    } else if (vec_rows && cpr <= 16 && N <= 64) {
+        // a decay per element (and the conv): whole rows per thread when small
+        const int cpt = cpr % 4 == 0 ? 4 : (cpr % 2 == 0 ? 2 : 1);
+        const int64_t lpr = cpr / cpt;
+        const int ve = 16 / es;
+        const bool a_vec = p.A_n == 1 && aligned16(p.A) && (p.A_h * 4) % 16 == 0 &&
+                           (p.A_p * 4) % 16 == 0 && ve % 4 == 0;
+        if (a_vec && pow2(lpr) && lpr <= 32) {
+            plan.kernel = SSM_KERNEL_SSU_ROW;
+            plan.block = 256;
+            plan.lpr = (int)lpr;
+            plan.cpl = cpt;
+            const int64_t rows_per_pass = plan.block / lpr;
+            int64_t rb = std::max<int64_t>(rows_per_pass, (16 * 1024) / row_bytes);
+            rb = (rb + rows_per_pass - 1) / rows_per_pass * rows_per_pass;
+            while (rb > rows_per_pass && Bn * ((HP + rb - 1) / rb) < 2 * ctas) rb -= rows_per_pass;
+            if (G > 1) {
+                // an item must not straddle a group: largest divisor of the
+                // group's row count not above rb
+                const int64_t rg = p.heads_per_group * P;
+                int64_t best = 1;
+                for (int64_t dv = 1; dv * dv <= rg; ++dv) {
+                    if (rg % dv) continue;
+                    if (dv <= rb) best = std::max(best, dv);
+                    if (rg / dv <= rb) best = std::max(best, rg / dv);
+                }
+                rb = best;
+            }
+            plan.rows_per_item = std::min<int64_t>(rb, HP);
+            plan.items_per_b = (HP + plan.rows_per_item - 1) / plan.rows_per_item;
+            plan.n_items = Bn * plan.items_per_b;
+        }
+    }
+    if (plan.kernel == SSM_KERNEL_SSU_TMA && plan.n_items < (int64_t)1 << 31) {
+        plan.grid = (int)std::min<int64_t>(plan.n_items, (int64_t)sms * 3);
+    } else if (plan.kernel != 0 && plan.n_items < (int64_t)1 << 31) {
         plan.grid = (int)std::min<int64_t>(plan.n_items, ctas);
     } else {
+        plan = SsuPlan{};
         plan.kernel = SSM_KERNEL_SSU_GENERIC;
         plan.block = 128;
         const int64_t rows = Bn * HP;
@@ -623,7 +704,9 @@ ssm_status ssu_impl(const ssm_ssu_args* a, cudaStream_t stream) {
         plan.n_items = rows;
         plan.grid = (int)std::min<int64_t>((rows + 127) / 128, (int64_t)sms * 16);
     }
-    fill_info(a->info, plan.kernel, plan.grid, plan.block, 0, plan.rows_per_item, plan.n_items);
+    fill_info(a->info, plan.kernel, plan.grid, plan.block,
+              plan.kernel == SSM_KERNEL_SSU_TMA ? ssu_tma_stages() * plan.stage_bytes : 0,
+              plan.rows_per_item, plan.n_items);
     if (dry) return SSM_OK;
     return launch_ssu(p, plan, stream) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
@@ -658,6 +741,13 @@ const char* ssm_status_string(int status) {
         case SSM_ERR_ALIAS: return "SSM_ERR_ALIAS: an output overlaps an input";
         default: return "unknown ssm_status";
     }
+}
+
+ssm_status ssm_device_error(int* code, void* stream) {
+    if (!code) return SSM_ERR_NULL;
+    return read_and_clear_device_error(code, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? SSM_OK
+               : SSM_ERR_CUDA;
 }
 
 int ssm_abi_version(void) { return SSM_CAUSAL_ABI_VERSION; }

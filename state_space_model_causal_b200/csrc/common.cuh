@@ -117,6 +117,40 @@ __device__ __forceinline__ void st_stream16(void* p, const uint4& v) {
     __stcs(static_cast<uint4*>(p), v);
 }
 
+// ------------------------------------------------------- packed f32x2 math --
+// Two fp32 lanes in one 64-bit register pair; sm_100 executes add/mul/fma on
+// both halves with one instruction.
+typedef unsigned long long u64;
+
+__device__ __forceinline__ u64 pk(float lo, float hi) {
+    u64 r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void upk(u64 v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ u64 fmul2(u64 a, u64 b) {
+    u64 d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ u64 ffma2(u64 a, u64 b, u64 c) {
+    u64 d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ u64 fadd2(u64 a, u64 b) {
+    u64 d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ u64 fsub2(u64 a, u64 b) {
+    u64 d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
 // ------------------------------------------------------------ activations --
 // 2^x on the SFU (ex2.approx, flush-to-zero): relative error ~2 ulp.
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -133,9 +167,25 @@ __device__ __forceinline__ float silu_f(float v) {
     return __fdividef(v, 1.0f + exp_fast(-v));
 }
 
-// softplus(v) = log(1 + e^v); above 20 the correction e^-v is below 2^-28 * v.
+// softplus(v) = log(1 + e^v).  Above v = 20 the correction e^-v is below
+// 2^-28 * v, so v is returned.  With e = e^v <= 1/16 (v <= -2.77, where the
+// discretisation step of a selective SSM usually lives) log(1 + e) is the
+// alternating series e - e^2/2 + e^3/3 - ... cut after e^7/7: the remainder
+// is below e^8/8 <= 2^-35, i.e. < 2^-31 relative to the result.  In between,
+// log1pf.
 __device__ __forceinline__ float softplus_f(float v) {
-    return v > 20.0f ? v : log1pf(exp_fast(v));
+    if (v > 20.0f) return v;
+    const float e = exp_fast(v);
+    if (e <= 0.0625f) {
+        float s = fmaf(e, 1.0f / 7.0f, -1.0f / 6.0f);
+        s = fmaf(s, e, 0.2f);
+        s = fmaf(s, e, -0.25f);
+        s = fmaf(s, e, 1.0f / 3.0f);
+        s = fmaf(s, e, -0.5f);
+        s = fmaf(s, e, 1.0f);
+        return e * s;
+    }
+    return log1pf(e);
 }
 
 }  // namespace ssm

@@ -41,6 +41,7 @@ struct SsuPlan {
     int64_t rows_per_item;
     int64_t items_per_b;
     int64_t n_items;
+    int stage_bytes;     // bulk-copy kernel: bytes of one shared-memory stage
 };
 
 // Fused prefill (Mamba-1 layout): x, dt, z, out (B, D, L); B, C (B, G, N, L).
@@ -72,6 +73,7 @@ struct ScanPlan {
     int dt_tile;    // channels per CTA
     int t_chunk;    // time steps per smem chunk
     int smem;       // dynamic shared memory bytes
+    int sw_pairs;   // vector kernel: state-entry pairs per thread whose exp runs on the FMA pipe
 };
 
 struct Conv1dProblem {
@@ -92,7 +94,14 @@ struct Conv1dPlan {
 };
 
 cudaError_t launch_ssu(const SsuProblem& p, const SsuPlan& plan, cudaStream_t s);
+int ssu_tma_stages();
+int ssu_tma_max_rows_per_thread();
+cudaError_t read_and_clear_device_error(int* code, cudaStream_t s);
 cudaError_t launch_scan(const ScanProblem& p, const ScanPlan& plan, cudaStream_t s);
+bool scan_vec_supported(const ScanProblem& p);
+int scan_vec_threads();
+int scan_vec_channels_per_cta();
+cudaError_t launch_scan_vec(const ScanProblem& p, int sw_pairs, cudaStream_t s);
 cudaError_t launch_conv1d(const Conv1dProblem& p, const Conv1dPlan& plan, cudaStream_t s);
 
 }  // namespace ssm

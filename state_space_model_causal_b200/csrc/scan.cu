@@ -314,6 +314,7 @@ int scan_chunked_smem_bytes(int ns) {
 }
 
 cudaError_t launch_scan(const ScanProblem& p, const ScanPlan& plan, cudaStream_t s) {
+    if (plan.kernel == SSM_KERNEL_SCAN_VEC) return launch_scan_vec(p, plan.sw_pairs, s);
     if (plan.kernel == SSM_KERNEL_SCAN_CHUNKED) {
         switch (p.io_dt) {
             case kF32: return launch_chunked<float>(p, plan, s);

@@ -165,15 +165,29 @@ def call(lib, fn, args):
 def test_prefill_2p8b_plan(lib):
     st, info = call(lib, "ssm_selective_scan_fwd", scan_args(FakeMem()))
     assert st == OK
-    assert bd.KERNELS[info.kernel] == "scan_chunked"
+    assert bd.KERNELS[info.kernel] == "scan_vec"
     assert info.block == 64 and info.rows_per_item == 16
     assert info.grid == 4 * 5120 // 16
+
+
+def test_unaligned_or_odd_prefill_layouts_use_the_chunked_kernel(lib):
+    mem = FakeMem()
+    st, info = call(lib, "ssm_selective_scan_fwd", scan_args(mem, Bn=2, D=64, L=100))
+    assert st == OK and bd.KERNELS[info.kernel] == "scan_chunked"  # L % 8 != 0
+    st, info = call(lib, "ssm_selective_scan_fwd", scan_args(mem, Bn=2, D=64, L=64, N=32))
+    assert st == OK and bd.KERNELS[info.kernel] == "scan_chunked"  # d_state > 16
+    st, info = call(lib, "ssm_selective_scan_fwd", scan_args(mem, Bn=2, D=64, L=64, W=3))
+    assert st == OK and bd.KERNELS[info.kernel] == "scan_chunked"  # conv width 3
+    a = scan_args(mem, Bn=2, D=64, L=64)
+    a.x.data += 2                                                  # 2-byte aligned rows
+    st, info = call(lib, "ssm_selective_scan_fwd", a)
+    assert st == OK and bd.KERNELS[info.kernel] == "scan_chunked"
 
 
 def test_small_scan_plan_and_generic_for_large_state(lib):
     mem = FakeMem()
     st, info = call(lib, "ssm_selective_scan_fwd", scan_args(mem, Bn=1, D=64, L=128, W=0, io=F32))
-    assert st == OK and bd.KERNELS[info.kernel] == "scan_chunked"
+    assert st == OK and bd.KERNELS[info.kernel] == "scan_vec"
     st, info = call(lib, "ssm_selective_scan_fwd", scan_args(mem, Bn=1, D=8, L=16, N=128, W=0))
     assert st == OK and bd.KERNELS[info.kernel] == "scan_generic"
 
@@ -181,33 +195,46 @@ def test_small_scan_plan_and_generic_for_large_state(lib):
 def test_scan_groups_choose_generic_when_tile_straddles_groups(lib):
     mem = FakeMem()
     st, info = call(lib, "ssm_selective_scan_fwd", scan_args(mem, Bn=1, D=64, L=8, G=4))
-    assert st == OK and bd.KERNELS[info.kernel] == "scan_chunked"  # 16 channels per group
+    assert st == OK and bd.KERNELS[info.kernel] == "scan_vec"  # 16 channels per group
     st, info = call(lib, "ssm_selective_scan_fwd", scan_args(mem, Bn=1, D=24, L=8, G=3))
     assert st == OK and bd.KERNELS[info.kernel] == "scan_generic"  # 8 channels per group
 
 
 def test_decode_2p8b_plan(lib):
     st, info = call(lib, "ssm_selective_state_update", ssu_m1_args(FakeMem()))
-    assert st == OK and bd.KERNELS[info.kernel] == "ssu_vec"
-    assert info.block == 256 and info.grid == 148 * 8
+    assert st == OK and bd.KERNELS[info.kernel] == "ssu_row"
+    assert info.block == 256 and info.grid == 148 * 4
 
 
 @pytest.mark.parametrize("P,N,st_dt,io", [(64, 128, F16, F16), (64, 128, F32, F16),
                                           (128, 256, BF16, BF16), (128, 256, F32, BF16)])
 @pytest.mark.parametrize("R", [8, 128, 4096, 131072])
-def test_mamba2_plans_use_vector_kernel(lib, P, N, st_dt, io, R):
+def test_mamba2_plans_use_bulk_copy_kernel(lib, P, N, st_dt, io, R):
     H = 80 if N == 128 else 32
     Bn, Hr = (-(-R // H), H) if R >= H else (1, R)
     st, info = call(lib, "ssm_selective_state_update",
                     ssu_m2_args(FakeMem(), Bn=Bn, H=Hr, P=P, N=N, io=io, st=st_dt))
-    assert st == OK and bd.KERNELS[info.kernel] == "ssu_vec"
-    assert 0 < info.grid <= 148 * 8
+    assert st == OK and bd.KERNELS[info.kernel] == "ssu_tma"
+    assert 0 < info.grid <= 148 * 3
+    assert info.smem_bytes <= 4 * 16 * 1024 and info.smem_bytes % 128 == 0
     assert info.work_items * info.rows_per_item >= Bn * Hr * P
 
 
 def test_mamba2_groups_items_do_not_straddle_groups(lib):
     st, info = call(lib, "ssm_selective_state_update", ssu_m2_args(FakeMem(), Bn=3, H=12, P=6, N=128, G=4))
+    assert st == OK and bd.KERNELS[info.kernel] == "ssu_tma"
+    # rows that are not dense (row stride > row size) take the register-streaming kernel
+    m = FakeMem()
+    a = ssu_m2_args(m, Bn=3, H=12, P=6, N=128, G=4)
+    a.state = m(F16, (3, 12, 6, 128), (12 * 6 * 256, 6 * 256, 256, 1))
+    st, info = call(lib, "ssm_selective_state_update", a)
     assert st == OK and bd.KERNELS[info.kernel] == "ssu_vec"
+    # full A per element takes the per-row kernel; its items must not straddle a group
+    m = FakeMem()
+    a = ssu_m2_args(m, Bn=3, H=12, P=6, N=16, G=4, st=F32)
+    a.A = m(F32, (12, 6, 16))
+    st, info = call(lib, "ssm_selective_state_update", a)
+    assert st == OK and bd.KERNELS[info.kernel] == "ssu_row"
     assert (12 // 4 * 6) % info.rows_per_item == 0
 
 

@@ -66,8 +66,8 @@ def test_scan_optional_inputs_absent_and_no_softplus():
     s = gen.scan_inputs(2, 50, 32, 16, io="f32", seed=6, tag="noopt", with_z=False, with_D=False,
                         with_dt_bias=False)
     _check(s, with_state=False)
-    s = gen.scan_inputs(2, 50, 32, 16, io="f32", seed=7, tag="nosp", W=4)
-    s.dt = np.abs(s.dt) * 0.01  # keep delta positive without the softplus
+    s = gen.scan_inputs(2, 50, 32, 16, io="f32", seed=7, tag="nosp", W=4, with_dt_bias=False)
+    s.dt = np.abs(s.dt) * 0.01  # delta = dt must stay positive without the softplus
     _check(s, softplus=False)
 
 

@@ -270,3 +270,30 @@ def test_empty_batch_is_a_no_op():
                B=torch.zeros(0, 1, 16, device="cuda"), C=torch.zeros(0, 1, 16, device="cuda"))
     torch.cuda.synchronize()
     assert out.shape == (0, 4, 8)
+
+
+def test_mamba2_dt_per_row_with_scalar_A():
+    """dt given per (head, headdim) row with one A per head: the bulk-copy
+    kernel's per-row discretisation branch."""
+    import torch
+    s = gen.ssu_mamba2_inputs(5, 6, 32, 128, io="f16", state="f16", seed=11, tag="dtrow",
+                              dt_per_head=False, with_z=True)
+    out, st = _m2_gpu(s)
+    torch.cuda.synchronize()
+    o, sref = _m2_oracle(s)
+    assert_close(N(out), o, TOL["f16"], "out")
+    assert_close(N(st), sref, TOL["f16"], "state")
+
+
+def test_bulk_copy_kernels_leave_the_device_error_word_clear():
+    import torch
+    from state_space_model_causal_b200 import LaunchInfo, ssm_device_error
+    s = gen.mamba2_64x128(4096, cache="f16")
+    info = LaunchInfo()
+    st = T(s.state, "f16")
+    from state_space_model_causal_b200 import ssm_selective_state_update
+    ssm_selective_state_update(st, T(s.x, "f16"), T(s.dt, "f16"), T(s.A, "f32"), T(s.B, "f16"),
+                               T(s.C, "f16"), D=T(s.D, "f32"), dt_bias=T(s.dt_bias, "f32"), info=info)
+    assert info.as_dict()["kernel"] == "ssu_tma"
+    assert ssm_device_error() == 0
+    torch.cuda.synchronize()
