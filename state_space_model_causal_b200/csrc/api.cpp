@@ -365,7 +365,7 @@ ssm_status scan_impl(const ssm_scan_args* a, cudaStream_t stream) {
         plan.sw_pairs = 0;
         if (const char* e = std::getenv("SSM_SCAN_SW_PAIRS")) {
             const int v = std::atoi(e);
-            if (v >= 0 && v <= 2) plan.sw_pairs = v;
+            if (v >= 0 && v <= 3) plan.sw_pairs = v;
         }
         fill_info(a->info, plan.kernel, plan.grid, plan.block, 0, scan_vec_channels_per_cta(),
                   tiles * Bn);
@@ -691,12 +691,15 @@ ssm_status ssu_impl(const ssm_ssu_args* a, cudaStream_t stream) {
             plan.n_items = Bn * plan.items_per_b;
         }
     }
+    plan.sms = sms;
     if (plan.kernel == SSM_KERNEL_SSU_TMA && plan.n_items < (int64_t)1 << 31) {
+        // the launcher caps it at the CTAs that fit at once (occupancy query)
         plan.grid = (int)std::min<int64_t>(plan.n_items, (int64_t)sms * 3);
     } else if (plan.kernel != 0 && plan.n_items < (int64_t)1 << 31) {
         plan.grid = (int)std::min<int64_t>(plan.n_items, ctas);
     } else {
         plan = SsuPlan{};
+        plan.sms = sms;
         plan.kernel = SSM_KERNEL_SSU_GENERIC;
         plan.block = 128;
         const int64_t rows = Bn * HP;

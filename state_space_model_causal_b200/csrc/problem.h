@@ -42,6 +42,7 @@ struct SsuPlan {
     int64_t items_per_b;
     int64_t n_items;
     int stage_bytes;     // bulk-copy kernel: bytes of one shared-memory stage
+    int sms;             // SMs of the device (persistent grids)
 };
 
 // Fused prefill (Mamba-1 layout): x, dt, z, out (B, D, L); B, C (B, G, N, L).

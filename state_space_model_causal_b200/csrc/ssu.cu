@@ -538,13 +538,29 @@ cudaError_t launch_head(const SsuProblem& p, const SsuPlan& plan, cudaStream_t s
     return cudaGetLastError();
 }
 
+// Opt the kernel into its dynamic shared memory and the largest shared-memory
+// carveout, and return how many of its CTAs fit on one SM.
+template <typename K>
+cudaError_t prepare_tma_kernel(K kern, int block, int smem, int* per_sm) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(per_sm, kern, block, smem);
+}
+
 template <typename ST>
 cudaError_t launch_head_tma(const SsuProblem& p, const SsuPlan& plan, cudaStream_t s) {
     const int smem = kTmaStages * plan.stage_bytes;
     auto run = [&](auto kern) -> cudaError_t {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        int per_sm = 0;
+        cudaError_t e = prepare_tma_kernel(kern, plan.block, smem, &per_sm);
         if (e != cudaSuccess) return e;
-        kern<<<plan.grid, plan.block, smem, s>>>(p, plan);
+        // persistent grid: every CTA resident at once (the item ranges are static)
+        const int64_t cap = (int64_t)plan.sms * (per_sm > 0 ? per_sm : 1);
+        const int grid = (int)(plan.n_items < cap ? plan.n_items : cap);
+        kern<<<grid, plan.block, smem, s>>>(p, plan);
         return cudaGetLastError();
     };
     switch (plan.cpl) {

@@ -166,7 +166,7 @@ def test_prefill_2p8b_plan(lib):
     st, info = call(lib, "ssm_selective_scan_fwd", scan_args(FakeMem()))
     assert st == OK
     assert bd.KERNELS[info.kernel] == "scan_vec"
-    assert info.block == 64 and info.rows_per_item == 16
+    assert info.block == 32 and info.rows_per_item == 16
     assert info.grid == 4 * 5120 // 16
 
 
