@@ -126,9 +126,11 @@ typedef enum ssm_kernel_id {
                                        time contiguous, L % 8 == 0, 16-byte aligned rows */
     SSM_KERNEL_SSU_ROW = 8,         /* 128-bit state update with a decay per element
                                        (Mamba-1 layout or full A), fused conv roll */
-    SSM_KERNEL_SSU_TMA = 9          /* state update fed by bulk copies (TMA) into
+    SSM_KERNEL_SSU_TMA = 9,         /* state update fed by bulk copies (TMA) into
                                        shared-memory stages: one decay per head, dense
                                        rows (Mamba-2 layout, scalar A, no conv) */
+    SSM_KERNEL_SSU_ROW_TMA = 10     /* state update fed by bulk copies: a decay per
+                                       element, fused conv roll (Mamba-1 layout) */
 } ssm_kernel_id;
 
 /* ------------------------------------------------------------------------ *

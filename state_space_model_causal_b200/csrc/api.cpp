@@ -604,7 +604,14 @@ ssm_status ssu_impl(const ssm_ssu_args* a, cudaStream_t stream) {
     const int64_t row_bytes = N * es;
     auto pow2 = [](int64_t v) { return v > 0 && (v & (v - 1)) == 0; };
     const bool dense_rows = p.st_p == N || P == 1;
-    if (vec_rows && dense_rows && !p.A_full && p.W == 0) {
+    // one I/O dtype for x, dt, B, C, z, out lets the bulk-copy kernel use typed access
+    const int io = p.x_dt;
+    const bool one_io = p.dt_dt == io && p.B_dt == io && p.C_dt == io && p.out_dt == io &&
+                        (!p.z || p.z_dt == io);
+    const int es_io = esize(io);
+    const bool x_rows = p.x_p == 1 && aligned16(p.x) && (p.x_b * es_io) % 16 == 0 &&
+                        (p.x_h * es_io) % 16 == 0;
+    if (vec_rows && dense_rows && !p.A_full && p.W == 0 && one_io && x_rows && P >= 2) {
         // bulk-copy pipeline: items are contiguous row blocks of one head; one
         // 16-byte chunk per lane for 16-bit states keeps B/C in 16 registers
         int cpl = 0;
@@ -618,20 +625,69 @@ ssm_status ssu_impl(const ssm_ssu_args* a, cudaStream_t stream) {
                 break;
             }
         }
-        const int64_t rows_per_pass = 256 / std::max<int64_t>(lpr, 1);
-        const int64_t max_rows = rows_per_pass * ssu_tma_max_rows_per_thread();
-        if (cpl && row_bytes <= 16 * 1024) {
+        if (cpl) {
+            const int64_t rows_per_pass = 256 / lpr;
+            // rows per thread: up to 4 (reduce-scatter needs rpt <= lpr), stage <= 24 KB
+            int rpt = 4;
+            while (rpt > 1 && (rpt > lpr || rpt * rows_per_pass * row_bytes > 24 * 1024)) rpt /= 2;
+            if (cpl == 2 && rpt > 2) rpt = 2;
+            const int64_t xalign = 16 / es_io;  // rows per item keep x 16-byte aligned
+            int64_t rb = std::min<int64_t>(rpt * rows_per_pass, P);
+            rb = std::max<int64_t>(xalign, rb / xalign * xalign);
             const int64_t ctas_tma = (int64_t)sms * 3;
-            int64_t rb = std::max<int64_t>(1, std::min<int64_t>({P, (16 * 1024) / row_bytes, max_rows}));
-            while (rb > 8 && Bn * H * ((P + rb - 1) / rb) < 2 * ctas_tma) rb = (rb + 1) / 2;
-            plan.kernel = SSM_KERNEL_SSU_TMA;
+            while (rb > xalign && Bn * H * ((P + rb - 1) / rb) < 2 * ctas_tma)
+                rb = std::max<int64_t>(xalign, (rb / 2) / xalign * xalign);
+            if (rb <= rpt * rows_per_pass && P % xalign == 0) {
+                plan.kernel = SSM_KERNEL_SSU_TMA;
+                plan.block = 256;
+                plan.lpr = (int)lpr;
+                plan.cpl = cpl;
+                plan.rpt = rpt;
+                plan.rows_per_item = rb;
+                plan.items_per_b = H * ((P + rb - 1) / rb);
+                plan.n_items = Bn * plan.items_per_b;
+                plan.stage_bytes = (int)((rb * row_bytes + rb * es_io + 127) / 128 * 128);
+                plan.stages = (int)std::max<int64_t>(
+                    2, std::min<int64_t>(ssu_tma_max_stages(), (72 * 1024) / plan.stage_bytes));
+            }
+        }
+    }
+    // Mamba-1 layout through bulk copies: channel rows, their conv rows, the
+    // x/dt/z slices and the batch row's B/C are contiguous and 16-byte aligned;
+    // one thread per row (d_state of at most 4 chunks of 16 bytes)
+    if (plan.kernel == 0 && vec_rows && P == 1 && p.A_full && one_io && cpr <= 4 && pow2(cpr) &&
+        (p.W == 0 || p.W == 4) && p.st_h == N && p.A_n == 1 && p.A_p == 0 && aligned16(p.A) &&
+        (p.A_h * 4) % 16 == 0 && (16 / es) % 4 == 0 && p.G == 1) {
+        const int cs_es = p.W ? esize(p.cs_dt) : 4;
+        const bool io_ok = p.x_h == 1 && p.dt_h == 1 && (!p.z || p.z_h == 1) && aligned16(p.x) &&
+                           aligned16(p.dt) && (!p.z || aligned16(p.z)) && (p.x_b * es_io) % 16 == 0 &&
+                           (p.dt_b * es_io) % 16 == 0 && (!p.z || (p.z_b * es_io) % 16 == 0);
+        const bool bc_ok = p.B_n == 1 && p.C_n == 1 && aligned16(p.Bm) && aligned16(p.Cm) &&
+                           (p.B_b * es_io) % 16 == 0 && (p.C_b * es_io) % 16 == 0 &&
+                           (N * es_io) % 16 == 0 && (cpr * 16 / es) % (16 / es_io) == 0;
+        const bool cs_ok = p.W == 0 || (p.cs_w == 1 && p.cs_c == p.W && aligned16(p.conv_state) &&
+                                        (p.cs_b * cs_es) % 16 == 0);
+        // channels % 8 == 0: every copy of a (possibly ragged) last block is a
+        // whole number of 16-byte units, so no copy reads past its tensor
+        if (io_ok && bc_ok && cs_ok && H % 8 == 0) {
+            int64_t rb = 256;
+            const int64_t ctas_tma = (int64_t)sms * 3;
+            while (rb > 64 && Bn * ((H + rb - 1) / rb) < 2 * ctas_tma) rb /= 2;
+            plan.kernel = SSM_KERNEL_SSU_ROW_TMA;
             plan.block = 256;
-            plan.lpr = (int)lpr;
-            plan.cpl = cpl;
+            plan.lpr = 1;
+            plan.cpl = (int)cpr;
+            plan.rpt = 1;
             plan.rows_per_item = rb;
-            plan.items_per_b = H * ((P + rb - 1) / rb);
+            plan.items_per_b = (H + rb - 1) / rb;
             plan.n_items = Bn * plan.items_per_b;
-            plan.stage_bytes = (int)((rb * row_bytes + 127) / 128 * 128);
+            const int64_t io_bytes = (rb * es_io + 15) / 16 * 16;
+            const int64_t cs_bytes = (rb * p.W * cs_es + 15) / 16 * 16;
+            const int64_t bc_bytes = (N * es_io + 15) / 16 * 16;
+            plan.stage_bytes =
+                (int)((rb * row_bytes + cs_bytes + 3 * io_bytes + 2 * bc_bytes + 127) / 128 * 128);
+            plan.stages = (int)std::max<int64_t>(
+                2, std::min<int64_t>(ssu_tma_max_stages(), (72 * 1024) / plan.stage_bytes));
         }
     }
     if (plan.kernel == 0 && vec_rows && !p.A_full && p.W == 0) {
@@ -658,7 +714,7 @@ ssm_status ssu_impl(const ssm_ssu_args* a, cudaStream_t stream) {
             plan.items_per_b = H * ((P + rb - 1) / rb);
             plan.n_items = Bn * plan.items_per_b;
         }
-    } else if (vec_rows && cpr <= 16 && N <= 64) {
+    } else if (plan.kernel == 0 && vec_rows && cpr <= 16 && N <= 64) {
         // a decay per element (and the conv): whole rows per thread when small
         const int cpt = cpr % 4 == 0 ? 4 : (cpr % 2 == 0 ? 2 : 1);
         const int64_t lpr = cpr / cpt;
@@ -692,7 +748,8 @@ ssm_status ssu_impl(const ssm_ssu_args* a, cudaStream_t stream) {
         }
     }
     plan.sms = sms;
-    if (plan.kernel == SSM_KERNEL_SSU_TMA && plan.n_items < (int64_t)1 << 31) {
+    if ((plan.kernel == SSM_KERNEL_SSU_TMA || plan.kernel == SSM_KERNEL_SSU_ROW_TMA) &&
+        plan.n_items < (int64_t)1 << 31) {
         // the launcher caps it at the CTAs that fit at once (occupancy query)
         plan.grid = (int)std::min<int64_t>(plan.n_items, (int64_t)sms * 3);
     } else if (plan.kernel != 0 && plan.n_items < (int64_t)1 << 31) {
@@ -708,7 +765,8 @@ ssm_status ssu_impl(const ssm_ssu_args* a, cudaStream_t stream) {
         plan.grid = (int)std::min<int64_t>((rows + 127) / 128, (int64_t)sms * 16);
     }
     fill_info(a->info, plan.kernel, plan.grid, plan.block,
-              plan.kernel == SSM_KERNEL_SSU_TMA ? ssu_tma_stages() * plan.stage_bytes : 0,
+              (plan.kernel == SSM_KERNEL_SSU_TMA || plan.kernel == SSM_KERNEL_SSU_ROW_TMA)
+                  ? plan.stages * plan.stage_bytes : 0,
               plan.rows_per_item, plan.n_items);
     if (dry) return SSM_OK;
     return launch_ssu(p, plan, stream) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;

@@ -42,6 +42,8 @@ struct SsuPlan {
     int64_t items_per_b;
     int64_t n_items;
     int stage_bytes;     // bulk-copy kernel: bytes of one shared-memory stage
+    int stages;          // bulk-copy kernel: stages in flight per CTA
+    int rpt;             // bulk-copy kernel: rows per thread per item
     int sms;             // SMs of the device (persistent grids)
 };
 
@@ -95,8 +97,7 @@ struct Conv1dPlan {
 };
 
 cudaError_t launch_ssu(const SsuProblem& p, const SsuPlan& plan, cudaStream_t s);
-int ssu_tma_stages();
-int ssu_tma_max_rows_per_thread();
+int ssu_tma_max_stages();
 cudaError_t read_and_clear_device_error(int* code, cudaStream_t s);
 cudaError_t launch_scan(const ScanProblem& p, const ScanPlan& plan, cudaStream_t s);
 bool scan_vec_supported(const ScanProblem& p);

@@ -212,30 +212,49 @@ __global__ void __launch_bounds__(256, 3) ssu_head_kernel(const SsuProblem p, co
 
 // ------------------------------------------------------------------------
 // Per-head decay kernel fed by bulk copies (TMA) -- the main Mamba-2 decode
-// path.  A work item is a block of rows of one (b, h); with dense rows it is
-// one contiguous range of the cache, which one thread copies into a shared
-// memory stage with cp.async.bulk (completion counted on an mbarrier).  Each
-// CTA walks a contiguous range of items and keeps kTmaStages copies in flight,
-// so the bytes in flight per SM no longer depend on registers; the threads
-// update from shared memory and stream the new state back with 16-byte
-// stores.  B/C are reloaded only when (b, group) changes, Delta and
-// exp(Delta*A) once per item, x before the wait so its latency overlaps the
-// copy.
+// path.  A work item is a block of rb rows of one (b, h); with dense rows it
+// is one contiguous range of the cache, and its rb x values are contiguous
+// too, so one thread copies both into a shared-memory stage with
+// cp.async.bulk (completion counted in bytes on an mbarrier).  Each CTA walks
+// a contiguous range of items (decoded incrementally), keeps plan.stages
+// copies in flight, and its threads update from shared memory and stream the
+// new state back with 16-byte stores.  `lpr` lanes share a row, each owning
+// CPL 16-byte chunks; a thread owns RPT rows of an item, and the RPT partial
+// readouts of a thread are summed over the row's lanes by a butterfly
+// reduce-scatter.  I/O dtype IoT is a template parameter.
 // ------------------------------------------------------------------------
-constexpr int kTmaStages = 4;
-constexpr int kTmaMaxRows = 8;                 // rows per thread per item
+constexpr int kTmaStagesMax = 4;
 constexpr long long kWaitBudget = 4000000000LL;  // cycles before a wait gives up (~2 s)
 
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-template <typename ST, int CPL>
+// Sum v[0..R) over the lpr lanes of a row.  Afterwards lane r of the row holds
+// the total of row k = r / (lpr / R) in v[0].  Needs R <= lpr.
+template <int R>
+__device__ __forceinline__ void row_reduce_scatter(float* v, unsigned lane_r, unsigned lpr) {
+    unsigned off = lpr >> 1;
+#pragma unroll
+    for (int w = R; w > 1; w >>= 1) {
+        const bool upper = (lane_r & off) != 0;
+#pragma unroll
+        for (int i = 0; i < w / 2; ++i) {
+            const float send = upper ? v[i] : v[i + w / 2];
+            const float keep = upper ? v[i + w / 2] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+        off >>= 1;
+    }
+    for (; off >= 1; off >>= 1) v[0] += __shfl_xor_sync(0xffffffffu, v[0], off);
+}
+
+template <typename ST, typename IoT, int CPL, int RPT>
 __global__ void __launch_bounds__(256, 3) ssu_head_tma_kernel(const SsuProblem p, const SsuPlan plan) {
     using V = Vec16<ST>;
     constexpr int VE = V::VE;
     extern __shared__ __align__(128) unsigned char tma_stage[];
-    __shared__ __align__(8) uint64_t full[kTmaStages];
+    __shared__ __align__(8) uint64_t full[kTmaStagesMax];
 
     const unsigned tid = threadIdx.x;
     const unsigned lpr = (unsigned)plan.lpr;
@@ -243,70 +262,101 @@ __global__ void __launch_bounds__(256, 3) ssu_head_tma_kernel(const SsuProblem p
     const unsigned row_slot = tid / lpr;
     const unsigned rows_per_pass = blockDim.x / lpr;
     const unsigned P = (unsigned)p.P;
+    const unsigned H = (unsigned)p.H;
     const unsigned rb = (unsigned)plan.rows_per_item;
     const unsigned iph = (P + rb - 1) / rb;
-    const unsigned items_per_b = (unsigned)p.H * iph;
     const unsigned n_items = (unsigned)plan.n_items;
     const unsigned per = (n_items + gridDim.x - 1) / gridDim.x;
     const unsigned i0 = blockIdx.x * per;
     const unsigned i1 = min(i0 + per, n_items);
     if (i0 >= i1) return;  // uniform
     const unsigned cnt = i1 - i0;
+    const unsigned S = (unsigned)plan.stages;
     const unsigned stage_bytes = (unsigned)plan.stage_bytes;
-    const int64_t es = sizeof(ST);
-    const unsigned row_bytes = (unsigned)(p.N * es);
+    const unsigned row_bytes = (unsigned)(p.N * (int64_t)sizeof(ST));
+    const unsigned x_off = rb * row_bytes;  // x values follow the rows in a stage
     const bool dt_row = p.dt_p != 0;
+    const IoT* __restrict__ xg = static_cast<const IoT*>(p.x);
+    const IoT* __restrict__ dtg = static_cast<const IoT*>(p.dt);
+    const IoT* __restrict__ Bg = static_cast<const IoT*>(p.Bm);
+    const IoT* __restrict__ Cg = static_cast<const IoT*>(p.Cm);
+    const IoT* __restrict__ zg = static_cast<const IoT*>(p.z);
+    IoT* __restrict__ og = static_cast<IoT*>(p.out);
 
-    auto decode = [&](unsigned item, unsigned& b, unsigned& h, unsigned& p0, unsigned& p1) {
-        b = item / items_per_b;
-        const unsigned rem = item - b * items_per_b;
-        h = rem / iph;
-        p0 = (rem - h * iph) * rb;
-        p1 = min(p0 + rb, P);
+    // item index -> (b, h, first row); advanced incrementally
+    struct Pos { unsigned b, h, pb; };
+    auto first = [&](unsigned item) {
+        Pos q;
+        q.b = item / (H * iph);
+        const unsigned rem = item - q.b * H * iph;
+        q.h = rem / iph;
+        q.pb = rem - q.h * iph;
+        return q;
+    };
+    auto next = [&](Pos& q) {
+        if (++q.pb == iph) {
+            q.pb = 0;
+            if (++q.h == H) {
+                q.h = 0;
+                ++q.b;
+            }
+        }
     };
     auto slot_of = [&](unsigned b) -> int64_t {
         if (!p.slot_idx) return b;
         const int64_t sl = p.slot_idx[b * p.si_b];
         return (sl < 0 || sl >= p.n_slots) ? -1 : sl;
     };
-    // thread 0: start the copy of local item k into stage k % kTmaStages; a
+    // thread 0: start the copies of the item at `q` into stage k % S; a
     // padding row completes the stage's phase without data
-    auto issue = [&](unsigned k) {
-        unsigned b, h, p0, p1;
-        decode(i0 + k, b, h, p0, p1);
-        uint64_t* bar = &full[k % kTmaStages];
-        const int64_t slot = slot_of(b);
+    auto issue = [&](unsigned k, const Pos& q) {
+        uint64_t* bar = &full[k % S];
+        const int64_t slot = slot_of(q.b);
         if (slot < 0) {
             mbar_arrive(bar);
             return;
         }
+        const unsigned p0 = q.pb * rb;
+        const unsigned nr = min(rb, P - p0);
         const char* src = static_cast<const char*>(p.state) +
-                          (slot * p.st_b + (int64_t)h * p.st_h + (int64_t)p0 * p.st_p) * es;
-        const uint32_t bytes = (p1 - p0) * row_bytes;
-        mbar_arrive_expect_tx(bar, bytes);
-        tma_load_1d(tma_stage + (k % kTmaStages) * stage_bytes, src, bytes, bar);
+                          (slot * p.st_b + (int64_t)q.h * p.st_h + (int64_t)p0 * p.st_p) * (int64_t)sizeof(ST);
+        const IoT* xs = xg + q.b * p.x_b + (int64_t)q.h * p.x_h + p0;
+        const uint32_t sbytes = nr * row_bytes;
+        const uint32_t xbytes = (nr * (unsigned)sizeof(IoT) + 15u) & ~15u;
+        unsigned char* dst = tma_stage + (k % S) * stage_bytes;
+        mbar_arrive_expect_tx(bar, sbytes + xbytes);
+        tma_load_1d(dst, src, sbytes, bar);
+        tma_load_1d(dst + x_off, xs, xbytes, bar);
     };
 
     if (tid == 0) {
-        for (int s = 0; s < kTmaStages; ++s) mbar_init(&full[s], 1);
+        for (unsigned s2 = 0; s2 < S; ++s2) mbar_init(&full[s2], 1);
         mbar_fence_init();
     }
     __syncthreads();
-    if (tid == 0)
-        for (unsigned k = 0; k < min(cnt, (unsigned)kTmaStages); ++k) issue(k);
+    Pos cur = first(i0);
+    if (tid == 0) {
+        Pos q = cur;
+        for (unsigned k = 0; k < min(cnt, S); ++k) {
+            issue(k, q);
+            next(q);
+        }
+    }
+    Pos ahead = cur;  // position of item k + S (thread 0's refill cursor)
+    for (unsigned k = 0; k < S; ++k) next(ahead);
 
     int64_t cached_key = -1;
     float Bv[CPL][VE], Cv[CPL][VE];
-    for (unsigned k = 0; k < cnt; ++k) {
-        unsigned b, h, p0, p1;
-        decode(i0 + k, b, h, p0, p1);
+    for (unsigned k = 0; k < cnt; ++k, next(cur)) {
+        const unsigned b = cur.b, h = cur.h;
+        const unsigned p0 = cur.pb * rb;
+        const unsigned p1 = min(p0 + rb, P);
         const int64_t slot = slot_of(b);
-        const unsigned stage = k % kTmaStages;
-        const uint32_t parity = (k / kTmaStages) & 1u;
-        const unsigned g = h / (unsigned)p.heads_per_group;
-        float delta = 0.0f, dA = 0.0f, a2 = 0.0f;
-        float xv[kTmaMaxRows];
+        const unsigned stage = k % S;
+        const uint32_t parity = (k / S) & 1u;
+        float delta = 0.0f, dA = 0.0f, a2 = 0.0f, dskip = 0.0f;
         if (slot >= 0) {
+            const unsigned g = h / (unsigned)p.heads_per_group;
             const int64_t key = (int64_t)b * p.G + g;
             if (key != cached_key) {
                 cached_key = key;
@@ -315,58 +365,58 @@ __global__ void __launch_bounds__(256, 3) ssu_head_tma_kernel(const SsuProblem p
 #pragma unroll
                     for (int e = 0; e < VE; ++e) {
                         const int64_t n = (int64_t)(lane_r + lpr * j) * VE + e;
-                        Bv[j][e] = ld_f(p.Bm, b * p.B_b + g * p.B_g + n * p.B_n, p.B_dt);
-                        Cv[j][e] = ld_f(p.Cm, b * p.C_b + g * p.C_g + n * p.C_n, p.C_dt);
+                        Bv[j][e] = to_f(Bg[b * p.B_b + g * p.B_g + n * p.B_n]);
+                        Cv[j][e] = to_f(Cg[b * p.C_b + g * p.C_g + n * p.C_n]);
                     }
                 }
             }
             a2 = p.A[h * p.A_h] * kLog2e;
+            dskip = p.Dp ? p.Dp[h * p.D_h] : 0.0f;
             if (!dt_row) {
-                float v = ld_f(p.dt, b * p.dt_b + h * p.dt_h, p.dt_dt);
+                float v = to_f(dtg[b * p.dt_b + h * p.dt_h]);
                 if (p.dt_bias) v += p.dt_bias[h * p.db_h];
                 delta = p.softplus ? softplus_f(v) : v;
                 dA = ex2_approx(delta * a2);
-            }
-#pragma unroll
-            for (int r = 0; r < kTmaMaxRows; ++r) {
-                const unsigned pp = p0 + row_slot + r * rows_per_pass;
-                xv[r] = pp < p1 ? ld_f(p.x, b * p.x_b + h * p.x_h + pp * p.x_p, p.x_dt) : 0.0f;
             }
         }
         const bool ok = mbar_wait_bounded(&full[stage], parity, kWaitBudget);
         if (__syncthreads_or(!ok)) {
             // give up: wait (bounded) for this CTA's copies still in flight, flag, exit
             if (tid == 0) {
-                for (unsigned kk = k; kk < min(cnt, k + kTmaStages); ++kk)
-                    mbar_wait_bounded(&full[kk % kTmaStages], (kk / kTmaStages) & 1u, kWaitBudget);
+                for (unsigned kk = k; kk < min(cnt, k + S); ++kk)
+                    mbar_wait_bounded(&full[kk % S], (kk / S) & 1u, kWaitBudget);
                 atomicExch(&g_ssm_device_error, 1);
             }
             return;
         }
         if (slot >= 0) {
             const unsigned char* st = tma_stage + stage * stage_bytes;
-            char* gbase = static_cast<char*>(p.state) + (slot * p.st_b + (int64_t)h * p.st_h) * es;
+            const IoT* xsm = reinterpret_cast<const IoT*>(st + x_off);
+            char* gbase = static_cast<char*>(p.state) +
+                          (slot * p.st_b + (int64_t)h * p.st_h) * (int64_t)sizeof(ST);
+            float acc[RPT], xr[RPT];
 #pragma unroll
-            for (int r = 0; r < kTmaMaxRows; ++r) {
-                if (r * rows_per_pass >= rb) break;  // uniform
-                const unsigned pp = p0 + row_slot + r * rows_per_pass;
+            for (int r = 0; r < RPT; ++r) {
+                const unsigned pl = row_slot + r * rows_per_pass;  // row within the item
+                const unsigned pp = p0 + pl;
                 const bool rok = pp < p1;
+                xr[r] = rok ? to_f(xsm[pl]) : 0.0f;
                 float dl = delta, da = dA;
                 if (dt_row && rok) {
-                    float v = ld_f(p.dt, b * p.dt_b + h * p.dt_h + pp * p.dt_p, p.dt_dt);
+                    float v = to_f(dtg[b * p.dt_b + h * p.dt_h + pp * p.dt_p]);
                     if (p.dt_bias) v += p.dt_bias[h * p.db_h + pp * p.db_p];
                     dl = p.softplus ? softplus_f(v) : v;
                     da = ex2_approx(dl * a2);
                 }
-                const float du = dl * xv[r];
+                const float du = dl * xr[r];
                 const u64 da2 = pk(da, da), du2 = pk(du, du);
                 u64 acc2 = pk(0.0f, 0.0f);
-                const unsigned char* srow = st + (pp - p0) * row_bytes;
-                char* grow = gbase + (int64_t)pp * p.st_p * es;
+                const unsigned char* srow = st + pl * row_bytes;
+                char* grow = gbase + (int64_t)pp * p.st_p * (int64_t)sizeof(ST);
 #pragma unroll
                 for (int j = 0; j < CPL; ++j) {
                     const unsigned off = (lane_r + lpr * j) * 16;
-                    uint4 raw = rok ? *reinterpret_cast<const uint4*>(srow + off) : make_uint4(0, 0, 0, 0);
+                    const uint4 raw = rok ? *reinterpret_cast<const uint4*>(srow + off) : make_uint4(0, 0, 0, 0);
                     float sv[VE];
                     V::unpack(raw, sv);
 #pragma unroll
@@ -380,15 +430,233 @@ __global__ void __launch_bounds__(256, 3) ssu_head_tma_kernel(const SsuProblem p
                 }
                 float a0, a1;
                 upk(acc2, a0, a1);
-                float acc = a0 + a1;
-                for (unsigned o = lpr >> 1; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-                if (rok && lane_r == 0) row_epilogue(p, b, h, pp, acc, xv[r]);
+                acc[r] = a0 + a1;
+            }
+            row_reduce_scatter<RPT>(acc, lane_r, lpr);
+            const unsigned group = lpr / RPT;
+            if (lane_r % group == 0) {
+                const unsigned r = lane_r / group;
+                const unsigned pl = row_slot + r * rows_per_pass;
+                const unsigned pp = p0 + pl;
+                if (pp < p1) {
+                    float xv = 0.0f;
+#pragma unroll
+                    for (int rr = 0; rr < RPT; ++rr)
+                        if (rr == (int)r) xv = xr[rr];
+                    float y = fmaf(dskip, xv, acc[0]);
+                    if (zg) y *= silu_f(to_f(zg[b * p.z_b + h * p.z_h + pp * p.z_p]));
+                    og[b * p.o_b + h * p.o_h + pp * p.o_p] = from_f<IoT>(y);
+                }
             }
         }
         __syncthreads();  // every thread is done reading this stage
-        if (tid == 0 && k + kTmaStages < cnt) {
+        if (tid == 0 && k + S < cnt) {
             fence_proxy_async_smem();
-            issue(k + kTmaStages);
+            issue(k + S, ahead);
+        }
+        next(ahead);
+    }
+}
+
+// ------------------------------------------------------------------------
+// Per-row decay kernel fed by bulk copies -- the Mamba-1 decode path (A per
+// (channel, state entry), fused conv-state roll).  A work item is (block of
+// rb channels, batch row b); items are ordered channel-block-major, so the
+// consecutive items of a CTA reuse A, the conv weights and the per-channel
+// parameters from L1.  The item's state rows, conv-state rows, x, dt and z
+// slices and the batch row's B and C are each contiguous and arrive by bulk
+// copy in one stage.  A thread owns whole rows (CPT 16-byte chunks = the
+// full d_state): the conv, SiLU, softplus and gate are computed once per row
+// and the readout needs no cross-lane reduction.
+// ------------------------------------------------------------------------
+template <typename ST, typename IoT, int W, int CPT>
+__global__ void __launch_bounds__(256, 3) ssu_row_tma_kernel(const SsuProblem p, const SsuPlan plan) {
+    using V = Vec16<ST>;
+    constexpr int VE = V::VE;
+    extern __shared__ __align__(128) unsigned char tma_stage[];
+    __shared__ __align__(8) uint64_t full[kTmaStagesMax];
+
+    const unsigned tid = threadIdx.x;
+    const unsigned Dch = (unsigned)p.H;  // channels (rows)
+    const unsigned Bn = (unsigned)p.Bn;
+    const unsigned rb = (unsigned)plan.rows_per_item;  // <= blockDim.x: one row per thread
+    const unsigned n_items = (unsigned)plan.n_items;
+    const unsigned per = (n_items + gridDim.x - 1) / gridDim.x;
+    const unsigned i0 = blockIdx.x * per;
+    const unsigned i1 = min(i0 + per, n_items);
+    if (i0 >= i1) return;  // uniform
+    const unsigned cnt = i1 - i0;
+    const unsigned S = (unsigned)plan.stages;
+    const unsigned stage_bytes = (unsigned)plan.stage_bytes;
+    const unsigned row_bytes = (unsigned)(p.N * (int64_t)sizeof(ST));
+    const unsigned cs_es = p.cs_dt == kF32 ? 4u : 2u;
+    const unsigned pad16 = 15u;
+    const unsigned N = (unsigned)p.N;
+    // stage layout: state rows | conv rows | x | dt | z | B | C
+    const unsigned off_cs = rb * row_bytes;
+    const unsigned off_x = off_cs + ((rb * (unsigned)W * cs_es + pad16) & ~pad16);
+    const unsigned io_bytes = (rb * (unsigned)sizeof(IoT) + pad16) & ~pad16;
+    const unsigned off_dt = off_x + io_bytes;
+    const unsigned off_z = off_dt + io_bytes;
+    const unsigned off_B = off_z + io_bytes;
+    const unsigned bc_bytes = (N * (unsigned)sizeof(IoT) + pad16) & ~pad16;
+    const unsigned off_C = off_B + bc_bytes;
+    const IoT* __restrict__ xg = static_cast<const IoT*>(p.x);
+    const IoT* __restrict__ dtg = static_cast<const IoT*>(p.dt);
+    const IoT* __restrict__ zg = static_cast<const IoT*>(p.z);
+    const IoT* __restrict__ Bg = static_cast<const IoT*>(p.Bm);
+    const IoT* __restrict__ Cg = static_cast<const IoT*>(p.Cm);
+    IoT* __restrict__ og = static_cast<IoT*>(p.out);
+
+    auto slot_of = [&](unsigned b) -> int64_t {
+        if (!p.slot_idx) return b;
+        const int64_t sl = p.slot_idx[b * p.si_b];
+        return (sl < 0 || sl >= p.n_slots) ? -1 : sl;
+    };
+    // item -> (channel block, batch row); channel-block-major order
+    auto issue = [&](unsigned k) {
+        const unsigned item = i0 + k;
+        const unsigned cb = item / Bn, b = item - cb * Bn;
+        uint64_t* bar = &full[k % S];
+        const int64_t slot = slot_of(b);
+        if (slot < 0) {
+            mbar_arrive(bar);
+            return;
+        }
+        const unsigned c0 = cb * rb;
+        const unsigned nr = min(rb, Dch - c0);
+        unsigned char* dst = tma_stage + (k % S) * stage_bytes;
+        const uint32_t sbytes = nr * row_bytes;
+        const uint32_t cbytes = W > 0 ? nr * (unsigned)W * cs_es : 0u;
+        const uint32_t ibytes = nr * (unsigned)sizeof(IoT);
+        mbar_arrive_expect_tx(bar, sbytes + cbytes + ibytes * (zg ? 3u : 2u) + 2u * bc_bytes);
+        tma_load_1d(dst, static_cast<const char*>(p.state) +
+                             (slot * p.st_b + (int64_t)c0 * p.st_h) * (int64_t)sizeof(ST), sbytes, bar);
+        if (W > 0)
+            tma_load_1d(dst + off_cs, static_cast<const char*>(p.conv_state) +
+                                          (slot * p.cs_b + (int64_t)c0 * p.cs_c) * (int64_t)cs_es, cbytes, bar);
+        tma_load_1d(dst + off_x, xg + b * p.x_b + c0, ibytes, bar);
+        tma_load_1d(dst + off_dt, dtg + b * p.dt_b + c0, ibytes, bar);
+        if (zg) tma_load_1d(dst + off_z, zg + b * p.z_b + c0, ibytes, bar);
+        tma_load_1d(dst + off_B, Bg + b * p.B_b, bc_bytes, bar);
+        tma_load_1d(dst + off_C, Cg + b * p.C_b, bc_bytes, bar);
+    };
+
+    if (tid == 0) {
+        for (unsigned s2 = 0; s2 < S; ++s2) mbar_init(&full[s2], 1);
+        mbar_fence_init();
+    }
+    __syncthreads();
+    if (tid == 0)
+        for (unsigned k = 0; k < min(cnt, S); ++k) issue(k);
+
+    for (unsigned k = 0; k < cnt; ++k) {
+        const unsigned item = i0 + k;
+        const unsigned cb = item / Bn, b = item - cb * Bn;
+        const unsigned c0 = cb * rb;
+        const unsigned c1 = min(c0 + rb, Dch);
+        const int64_t slot = slot_of(b);
+        const unsigned stage = k % S;
+        const uint32_t parity = (k / S) & 1u;
+        // this thread's channel and its parameters (L1-resident across items),
+        // loaded before the stage wait so their latency overlaps the copy
+        const unsigned c = c0 + tid;
+        const bool rok = slot >= 0 && tid < rb && c < c1;
+        const unsigned cc = rok ? c : 0;
+        float wv[W > 0 ? W : 1];
+        float cbias = 0.0f, dbias = 0.0f, dskip = 0.0f;
+        float4 a4[CPT * VE / 4];
+        if (rok) {
+#pragma unroll
+            for (int kk = 0; kk < W; ++kk) wv[kk] = p.conv_w[cc * p.cw_c + kk * p.cw_w];
+            cbias = (W > 0 && p.conv_b) ? p.conv_b[cc * p.cb_c] : 0.0f;
+            dbias = p.dt_bias ? p.dt_bias[cc * p.db_h] : 0.0f;
+            dskip = p.Dp ? p.Dp[cc * p.D_h] : 0.0f;
+            const float4* ap = reinterpret_cast<const float4*>(p.A + cc * p.A_h);
+#pragma unroll
+            for (int i = 0; i < CPT * VE / 4; ++i) a4[i] = __ldg(ap + i);
+        }
+        const bool ok = mbar_wait_bounded(&full[stage], parity, kWaitBudget);
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) {
+                for (unsigned kk = k; kk < min(cnt, k + S); ++kk)
+                    mbar_wait_bounded(&full[kk % S], (kk / S) & 1u, kWaitBudget);
+                atomicExch(&g_ssm_device_error, 1);
+            }
+            return;
+        }
+        if (rok) {
+            const unsigned char* st = tma_stage + stage * stage_bytes;
+            const unsigned cl = tid;
+            const float xv = to_f(reinterpret_cast<const IoT*>(st + off_x)[cl]);
+            float u = xv;
+            float win[W > 0 ? W : 1];
+            if constexpr (W > 0) {
+                const unsigned char* crow = st + off_cs + cl * (unsigned)W * cs_es;
+#pragma unroll
+                for (int kk = 0; kk < W - 1; ++kk)
+                    win[kk] = cs_es == 4 ? reinterpret_cast<const float*>(crow)[kk + 1]
+                                         : ld_f(crow, kk + 1, p.cs_dt);
+                win[W - 1] = xv;
+                float acc_c = cbias;
+#pragma unroll
+                for (int kk = 0; kk < W; ++kk) acc_c = fmaf(wv[kk], win[kk], acc_c);
+                u = silu_f(acc_c);
+            }
+            const float v = to_f(reinterpret_cast<const IoT*>(st + off_dt)[cl]) + dbias;
+            const float dl = p.softplus ? softplus_f(v) : v;
+            const float dl2 = dl * kLog2e;
+            const float du = dl * u;
+            // B and C of the batch row: 16-byte vector reads (broadcast), widened once
+            constexpr int NS = CPT * VE;             // d_state
+            constexpr int IV = 16 / sizeof(IoT);     // I/O values per 16 bytes
+            float bv[NS], cv[NS];
+#pragma unroll
+            for (int i = 0; i < NS; i += IV) {
+                const uint4 rbv = *reinterpret_cast<const uint4*>(st + off_B + i * sizeof(IoT));
+                const uint4 rcv = *reinterpret_cast<const uint4*>(st + off_C + i * sizeof(IoT));
+                Vec16<IoT>::unpack(rbv, bv + i);
+                Vec16<IoT>::unpack(rcv, cv + i);
+            }
+            const unsigned char* srow = st + cl * row_bytes;
+            char* grow = static_cast<char*>(p.state) + (slot * p.st_b + (int64_t)c * p.st_h) * (int64_t)sizeof(ST);
+            float acc = 0.0f;
+#pragma unroll
+            for (int j = 0; j < CPT; ++j) {
+                float sv[VE];
+                V::unpack(*reinterpret_cast<const uint4*>(srow + j * 16), sv);
+#pragma unroll
+                for (int e = 0; e < VE; e += 4) {
+                    const int n = j * VE + e;
+                    const float4 a = a4[n / 4];
+                    const float av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        sv[e + i] = fmaf(ex2_approx(dl2 * av[i]), sv[e + i], du * bv[n + i]);
+                        acc = fmaf(cv[n + i], sv[e + i], acc);
+                    }
+                }
+                st_stream16(grow + j * 16, V::pack(sv));
+            }
+            float y = fmaf(dskip, u, acc);
+            if (zg) y *= silu_f(to_f(reinterpret_cast<const IoT*>(st + off_z)[cl]));
+            og[b * p.o_b + (int64_t)c * p.o_h] = from_f<IoT>(y);
+            if constexpr (W > 0) {
+                // rolled conv state: old entries 1..W-1, then x
+                const int64_t cso = slot * p.cs_b + (int64_t)c * p.cs_c;
+                if (cs_es == 4 && W == 4) {
+                    *reinterpret_cast<float4*>(static_cast<float*>(p.conv_state) + cso) =
+                        make_float4(win[0], win[1], win[2], win[3]);
+                } else {
+#pragma unroll
+                    for (int kk = 0; kk < W; ++kk) st_f(p.conv_state, cso + kk * p.cs_w, p.cs_dt, win[kk]);
+                }
+            }
+        }
+        __syncthreads();  // every thread is done reading this stage
+        if (tid == 0 && k + S < cnt) {
+            fence_proxy_async_smem();
+            issue(k + S);
         }
     }
 }
@@ -550,9 +818,9 @@ cudaError_t prepare_tma_kernel(K kern, int block, int smem, int* per_sm) {
     return cudaOccupancyMaxActiveBlocksPerMultiprocessor(per_sm, kern, block, smem);
 }
 
-template <typename ST>
-cudaError_t launch_head_tma(const SsuProblem& p, const SsuPlan& plan, cudaStream_t s) {
-    const int smem = kTmaStages * plan.stage_bytes;
+template <typename ST, typename IoT>
+cudaError_t launch_head_tma_io(const SsuProblem& p, const SsuPlan& plan, cudaStream_t s) {
+    const int smem = plan.stages * plan.stage_bytes;
     auto run = [&](auto kern) -> cudaError_t {
         int per_sm = 0;
         cudaError_t e = prepare_tma_kernel(kern, plan.block, smem, &per_sm);
@@ -563,9 +831,57 @@ cudaError_t launch_head_tma(const SsuProblem& p, const SsuPlan& plan, cudaStream
         kern<<<grid, plan.block, smem, s>>>(p, plan);
         return cudaGetLastError();
     };
-    switch (plan.cpl) {
-        case 1: return run(ssu_head_tma_kernel<ST, 1>);
-        case 2: return run(ssu_head_tma_kernel<ST, 2>);
+    const int key = plan.cpl * 10 + plan.rpt;
+    switch (key) {
+        case 11: return run(ssu_head_tma_kernel<ST, IoT, 1, 1>);
+        case 12: return run(ssu_head_tma_kernel<ST, IoT, 1, 2>);
+        case 14: return run(ssu_head_tma_kernel<ST, IoT, 1, 4>);
+        case 21: return run(ssu_head_tma_kernel<ST, IoT, 2, 1>);
+        case 22: return run(ssu_head_tma_kernel<ST, IoT, 2, 2>);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+template <typename ST, typename IoT>
+cudaError_t launch_row_tma_io(const SsuProblem& p, const SsuPlan& plan, cudaStream_t s) {
+    const int smem = plan.stages * plan.stage_bytes;
+    auto run = [&](auto kern) -> cudaError_t {
+        int per_sm = 0;
+        cudaError_t e = prepare_tma_kernel(kern, plan.block, smem, &per_sm);
+        if (e != cudaSuccess) return e;
+        const int64_t cap = (int64_t)plan.sms * (per_sm > 0 ? per_sm : 1);
+        const int grid = (int)(plan.n_items < cap ? plan.n_items : cap);
+        kern<<<grid, plan.block, smem, s>>>(p, plan);
+        return cudaGetLastError();
+    };
+    const int key = (int)p.W * 10 + plan.cpl;
+    switch (key) {
+        case 1: return run(ssu_row_tma_kernel<ST, IoT, 0, 1>);
+        case 2: return run(ssu_row_tma_kernel<ST, IoT, 0, 2>);
+        case 4: return run(ssu_row_tma_kernel<ST, IoT, 0, 4>);
+        case 41: return run(ssu_row_tma_kernel<ST, IoT, 4, 1>);
+        case 42: return run(ssu_row_tma_kernel<ST, IoT, 4, 2>);
+        case 44: return run(ssu_row_tma_kernel<ST, IoT, 4, 4>);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+template <typename ST>
+cudaError_t launch_row_tma(const SsuProblem& p, const SsuPlan& plan, cudaStream_t s) {
+    switch (p.x_dt) {
+        case kF32: return launch_row_tma_io<ST, float>(p, plan, s);
+        case kF16: return launch_row_tma_io<ST, __half>(p, plan, s);
+        case kBF16: return launch_row_tma_io<ST, __nv_bfloat16>(p, plan, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+template <typename ST>
+cudaError_t launch_head_tma(const SsuProblem& p, const SsuPlan& plan, cudaStream_t s) {
+    switch (p.x_dt) {
+        case kF32: return launch_head_tma_io<ST, float>(p, plan, s);
+        case kF16: return launch_head_tma_io<ST, __half>(p, plan, s);
+        case kBF16: return launch_head_tma_io<ST, __nv_bfloat16>(p, plan, s);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -584,6 +900,14 @@ cudaError_t launch_row(const SsuProblem& p, const SsuPlan& plan, cudaStream_t s)
 }  // namespace
 
 cudaError_t launch_ssu(const SsuProblem& p, const SsuPlan& plan, cudaStream_t s) {
+    if (plan.kernel == SSM_KERNEL_SSU_ROW_TMA) {
+        switch (p.state_dt) {
+            case kF32: return launch_row_tma<float>(p, plan, s);
+            case kF16: return launch_row_tma<__half>(p, plan, s);
+            case kBF16: return launch_row_tma<__nv_bfloat16>(p, plan, s);
+            default: return cudaErrorInvalidValue;
+        }
+    }
     if (plan.kernel == SSM_KERNEL_SSU_TMA) {
         switch (p.state_dt) {
             case kF32: return launch_head_tma<float>(p, plan, s);
@@ -610,8 +934,7 @@ cudaError_t launch_ssu(const SsuProblem& p, const SsuPlan& plan, cudaStream_t s)
     return cudaErrorInvalidValue;
 }
 
-int ssu_tma_stages() { return kTmaStages; }
-int ssu_tma_max_rows_per_thread() { return kTmaMaxRows; }
+int ssu_tma_max_stages() { return kTmaStagesMax; }
 
 // Read the device error word into *code (after the stream's work so far) and
 // clear it.

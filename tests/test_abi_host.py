@@ -202,8 +202,11 @@ def test_scan_groups_choose_generic_when_tile_straddles_groups(lib):
 
 def test_decode_2p8b_plan(lib):
     st, info = call(lib, "ssm_selective_state_update", ssu_m1_args(FakeMem()))
+    assert st == OK and bd.KERNELS[info.kernel] == "ssu_row_tma"
+    assert info.block == 256 and info.grid == 148 * 3 and info.rows_per_item == 256
+    # a channel count that is not a multiple of 8 takes the register-streaming row kernel
+    st, info = call(lib, "ssm_selective_state_update", ssu_m1_args(FakeMem(), D=100))
     assert st == OK and bd.KERNELS[info.kernel] == "ssu_row"
-    assert info.block == 256 and info.grid == 148 * 4
 
 
 @pytest.mark.parametrize("P,N,st_dt,io", [(64, 128, F16, F16), (64, 128, F32, F16),
@@ -216,13 +219,16 @@ def test_mamba2_plans_use_bulk_copy_kernel(lib, P, N, st_dt, io, R):
                     ssu_m2_args(FakeMem(), Bn=Bn, H=Hr, P=P, N=N, io=io, st=st_dt))
     assert st == OK and bd.KERNELS[info.kernel] == "ssu_tma"
     assert 0 < info.grid <= 148 * 3
-    assert info.smem_bytes <= 4 * 16 * 1024 and info.smem_bytes % 128 == 0
+    assert 0 < info.smem_bytes <= 76 * 1024 and info.smem_bytes % 128 == 0
     assert info.work_items * info.rows_per_item >= Bn * Hr * P
 
 
 def test_mamba2_groups_items_do_not_straddle_groups(lib):
-    st, info = call(lib, "ssm_selective_state_update", ssu_m2_args(FakeMem(), Bn=3, H=12, P=6, N=128, G=4))
+    st, info = call(lib, "ssm_selective_state_update", ssu_m2_args(FakeMem(), Bn=3, H=12, P=8, N=128, G=4))
     assert st == OK and bd.KERNELS[info.kernel] == "ssu_tma"
+    # headdim 6: an item's fp16 x values cannot start 16-byte aligned -> streaming kernel
+    st, info = call(lib, "ssm_selective_state_update", ssu_m2_args(FakeMem(), Bn=3, H=12, P=6, N=128, G=4))
+    assert st == OK and bd.KERNELS[info.kernel] == "ssu_vec"
     # rows that are not dense (row stride > row size) take the register-streaming kernel
     m = FakeMem()
     a = ssu_m2_args(m, Bn=3, H=12, P=6, N=128, G=4)

@@ -297,3 +297,39 @@ def test_bulk_copy_kernels_leave_the_device_error_word_clear():
     assert info.as_dict()["kernel"] == "ssu_tma"
     assert ssm_device_error() == 0
     torch.cuda.synchronize()
+
+
+def test_mamba1_slot_indices_with_padding_rows():
+    """Mamba-1 decode over a pool of 6 cache slots (state and conv state) for 4
+    requests, one of them a padding row; the bulk-copy kernel must leave the
+    padding row's output and every unused slot untouched."""
+    import torch
+    pool = gen.ssu_mamba1_inputs(6, 64, 16, W=4, io="f16", state="f32", seed=12, tag="pool1")
+    s = gen.ssu_mamba1_inputs(4, 64, 16, W=4, io="f16", state="f32", seed=13, tag="req1")
+    idx = np.array([5, -1, 0, 3], dtype=np.int32)
+    st = T(pool.state, "f32")
+    cs = T(pool.conv_state, "f32")
+    out = torch.full((4, 64), 3.0, dtype=torch.float16, device="cuda")
+    from state_space_model_causal_b200 import LaunchInfo
+    info = LaunchInfo()
+    _ssu(state=st, x=T(s.x, "f16"), dt=T(s.dt, "f16"), A=T(s.A, "f32"), B=T(s.B, "f16"),
+         C=T(s.C, "f16"), D=T(s.D, "f32"), z=T(s.z, "f16"), dt_bias=T(s.dt_bias, "f32"),
+         conv_weight=T(s.conv_weight, "f32"), conv_bias=T(s.conv_bias, "f32"), conv_state=cs,
+         state_batch_indices=torch.from_numpy(idx).cuda(), out=out, info=info)
+    torch.cuda.synchronize()
+    assert info.as_dict()["kernel"] == "ssu_row_tma"
+    got_st, got_cs, got_out = N(st), N(cs), N(out)
+    for b, slot in enumerate(idx):
+        if slot < 0:
+            assert np.all(got_out[b] == 3.0)
+            continue
+        one = gen.SsuInputs(pool.state[slot:slot + 1], s.x[b:b + 1], s.dt[b:b + 1], s.A,
+                            s.B[b:b + 1], s.C[b:b + 1], s.D, s.z[b:b + 1], s.dt_bias,
+                            s.conv_weight, s.conv_bias, pool.conv_state[slot:slot + 1])
+        o, sref, csref = _m1_oracle(one)
+        assert_close(got_out[b], o[0], TOL["f16"], f"out[{b}]")
+        assert_close(got_st[slot], sref[0], TOL["f16"], f"state[{slot}]")
+        np.testing.assert_array_equal(got_cs[slot], csref[0])
+    for slot in (1, 2, 4):
+        np.testing.assert_array_equal(got_st[slot], pool.state[slot])
+        np.testing.assert_array_equal(got_cs[slot], pool.conv_state[slot])
