@@ -313,9 +313,12 @@ def decode_mamba1_2p8b(dev, hbm_peak, slabs=64, replays=20):
     gbs = nbytes / (us * 1e-6) / 1e9
     del bufs, calls
     torch.cuda.empty_cache()
+    traffic = profiled_traffic("ssu_row_tma_decode_2p8b.txt", ["ssu.cu", "common.cuh", "tma.cuh"])
     return {"workload": "mamba1-2.8b-decode: B=245 D=5120 N=16 W=4, fp32 ssm/conv state, fp16 io, 64 slabs",
             "us_per_call": round(us, 3), "us_median": round(med, 3), "bytes_per_call": nbytes,
             "GBps": round(gbs, 1), "frac_of_hbm_peak": round(gbs / hbm_peak, 4),
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+                         "frac": round(gbs / hbm_peak, 4), "traffic": traffic},
             "l2": "each call on a different 100 MB slab", "gpu_launches_per_replay": slabs}
 
 
@@ -352,7 +355,11 @@ def decode_mamba2(dev, hbm_peak, H, P, N, R, cache, io, replays=10, calls_per_gr
     gbs = nbytes / (us * 1e-6) / 1e9
     del bufs, calls
     torch.cuda.empty_cache()
+    traffic = profiled_traffic(f"ssu_head_tma_mamba2_{P}x{N}_{cache}_R{R}.txt",
+                               ["ssu.cu", "common.cuh", "tma.cuh"])
     return {"workload": f"mamba2-ssu: H={H} P={P} N={N} G=1, {io} io, {cache} cache",
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+                         "frac": round(gbs / hbm_peak, 4), "traffic": traffic},
             "effective_batch": R, "batch": Bt, "heads": Hr, "us_per_call": round(us, 3),
             "us_median": round(med, 3), "bytes_per_call": nbytes, "GBps": round(gbs, 1),
             "frac_of_hbm_peak": round(gbs / hbm_peak, 4),
@@ -444,7 +451,7 @@ def run_only(args, dev):
         pf = Prefill(dev)
         fn = pf.run
     elif args.only == "decode_m1":
-        Bt, D, N, W = 490, 5120, 16, 4  # two layers' worth of rows, 200 MB of state
+        Bt, D, N, W = args.B, 5120, 16, 4  # default: two layers' worth of rows, 200 MB of state
         tag = ("only", "decode_m1")
         st = gen.device_normal((Bt, D, N), "f32", *tag, "state", device=dev)
         cs = gen.device_normal((Bt, D, W), "f32", *tag, "cs", device=dev)
@@ -503,6 +510,7 @@ def main():
                     help="run --warmup then --steps launches of one case and exit "
                          "(for profiler captures; prints no JSON line)")
     ap.add_argument("--R", type=int, default=16384, help="effective batch for --only m2_*")
+    ap.add_argument("--B", type=int, default=490, help="batch for --only decode_m1")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -559,7 +567,7 @@ def main():
     sfu_peak = NUM_SMS * SFU_EX2_PER_CLK_PER_SM * sm_max * 1e6 / 1e9  # Gelem/s
     alg_bytes = pf.algorithmic_bytes()
     hbm_gbs = alg_bytes / (ms_step * 1e-3) / 1e9
-    traffic = profiled_traffic("scan_chunked_prefill_2p8b.txt", ["scan.cu", "common.cuh"])
+    traffic = profiled_traffic("scan_vec_prefill_2p8b.txt", ["scan_vec.cu", "common.cuh"])
     roofline = {"bound": "alu", "achieved": round(pf.elems / (ms_step * 1e-3) / 1e9, 2),
                 "peak": round(sfu_peak, 1), "unit": "Gelem/s",
                 "frac": round(pf.elems / (ms_step * 1e-3) / 1e9 / sfu_peak, 4),
