@@ -670,11 +670,10 @@ ssm_status ssu_impl(const ssm_ssu_args* a, cudaStream_t stream) {
         // channels % 8 == 0: every copy of a (possibly ragged) last block is a
         // whole number of 16-byte units, so no copy reads past its tensor
         if (io_ok && bc_ok && cs_ok && H % 8 == 0) {
-            int64_t rb = 256;
-            const int64_t ctas_tma = (int64_t)sms * 3;
-            while (rb > 64 && Bn * ((H + rb - 1) / rb) < 2 * ctas_tma) rb /= 2;
+            // items of 32 channels (one per lane), one pipeline per warp
+            const int64_t rb = 32;
             plan.kernel = SSM_KERNEL_SSU_ROW_TMA;
-            plan.block = 256;
+            plan.block = 32 * ssu_row_tma_warps();
             plan.lpr = 1;
             plan.cpl = (int)cpr;
             plan.rpt = 1;
@@ -686,8 +685,7 @@ ssm_status ssu_impl(const ssm_ssu_args* a, cudaStream_t stream) {
             const int64_t bc_bytes = (N * es_io + 15) / 16 * 16;
             plan.stage_bytes =
                 (int)((rb * row_bytes + cs_bytes + 3 * io_bytes + 2 * bc_bytes + 127) / 128 * 128);
-            plan.stages = (int)std::max<int64_t>(
-                2, std::min<int64_t>(ssu_tma_max_stages(), (72 * 1024) / plan.stage_bytes));
+            plan.stages = ssu_row_tma_stages();
         }
     }
     if (plan.kernel == 0 && vec_rows && !p.A_full && p.W == 0) {
@@ -748,8 +746,11 @@ ssm_status ssu_impl(const ssm_ssu_args* a, cudaStream_t stream) {
         }
     }
     plan.sms = sms;
-    if ((plan.kernel == SSM_KERNEL_SSU_TMA || plan.kernel == SSM_KERNEL_SSU_ROW_TMA) &&
-        plan.n_items < (int64_t)1 << 31) {
+    if (plan.kernel == SSM_KERNEL_SSU_ROW_TMA && plan.n_items < (int64_t)1 << 31) {
+        // one pipeline per warp; the launcher caps the CTAs at what fits at once
+        plan.grid = (int)std::min<int64_t>((plan.n_items + ssu_row_tma_warps() - 1) / ssu_row_tma_warps(),
+                                           (int64_t)sms * 5);
+    } else if (plan.kernel == SSM_KERNEL_SSU_TMA && plan.n_items < (int64_t)1 << 31) {
         // the launcher caps it at the CTAs that fit at once (occupancy query)
         plan.grid = (int)std::min<int64_t>(plan.n_items, (int64_t)sms * 3);
     } else if (plan.kernel != 0 && plan.n_items < (int64_t)1 << 31) {
@@ -765,8 +766,9 @@ ssm_status ssu_impl(const ssm_ssu_args* a, cudaStream_t stream) {
         plan.grid = (int)std::min<int64_t>((rows + 127) / 128, (int64_t)sms * 16);
     }
     fill_info(a->info, plan.kernel, plan.grid, plan.block,
-              (plan.kernel == SSM_KERNEL_SSU_TMA || plan.kernel == SSM_KERNEL_SSU_ROW_TMA)
-                  ? plan.stages * plan.stage_bytes : 0,
+              plan.kernel == SSM_KERNEL_SSU_TMA ? plan.stages * plan.stage_bytes
+              : plan.kernel == SSM_KERNEL_SSU_ROW_TMA ? ssu_row_tma_warps() * plan.stages * plan.stage_bytes
+                                                      : 0,
               plan.rows_per_item, plan.n_items);
     if (dry) return SSM_OK;
     return launch_ssu(p, plan, stream) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;

@@ -98,6 +98,8 @@ struct Conv1dPlan {
 
 cudaError_t launch_ssu(const SsuProblem& p, const SsuPlan& plan, cudaStream_t s);
 int ssu_tma_max_stages();
+int ssu_row_tma_warps();
+int ssu_row_tma_stages();
 cudaError_t read_and_clear_device_error(int* code, cudaStream_t s);
 cudaError_t launch_scan(const ScanProblem& p, const ScanPlan& plan, cudaStream_t s);
 bool scan_vec_supported(const ScanProblem& p);

@@ -460,38 +460,59 @@ __global__ void __launch_bounds__(256, 3) ssu_head_tma_kernel(const SsuProblem p
 
 // ------------------------------------------------------------------------
 // Per-row decay kernel fed by bulk copies -- the Mamba-1 decode path (A per
-// (channel, state entry), fused conv-state roll).  A work item is (block of
-// rb channels, batch row b); items are ordered channel-block-major, so the
-// consecutive items of a CTA reuse A, the conv weights and the per-channel
-// parameters from L1.  The item's state rows, conv-state rows, x, dt and z
-// slices and the batch row's B and C are each contiguous and arrive by bulk
-// copy in one stage.  A thread owns whole rows (CPT 16-byte chunks = the
-// full d_state): the conv, SiLU, softplus and gate are computed once per row
-// and the readout needs no cross-lane reduction.
+// (channel, state entry), fused conv-state roll).  Every warp runs its own
+// pipeline over a contiguous range of work items, an item being (32 channels,
+// batch row b).  The warp's lane 0 moves each item through a ring of
+// kWarpStages shared-memory stages with 1-D bulk copies: state rows, conv
+// rows, x/dt/z slices and the row's B and C in (completion counted on the
+// stage's mbarrier); the updated state and conv rows, written back into the
+// stage in place, out again as bulk stores.  A stage is refilled once its
+// store has read it, one step later, so kWarpStages - 1 loads run ahead of
+// the compute.  No CTA-wide barrier sits in the loop: warps never wait for
+// each other.  Items are ordered channel-block-major, so a warp's
+// consecutive items reuse A and the conv weights from L1.  A lane owns one
+// whole row (CPT 16-byte chunks = the full d_state): conv, SiLU, softplus
+// and gate once per row, no cross-lane reduction.  Lane l walks its chunks
+// starting at chunk (l / (8/CPT)) mod CPT so that the 16-byte shared-memory
+// accesses of neighbouring rows hit distinct banks; A, B and C are taken in
+// the same rotated order.
 // ------------------------------------------------------------------------
+#ifndef SSM_ROW_TMA_STAGES
+#define SSM_ROW_TMA_STAGES 3
+#endif
+#ifndef SSM_ROW_TMA_WARPS
+#define SSM_ROW_TMA_WARPS 4
+#endif
+constexpr int kWarpStages = SSM_ROW_TMA_STAGES;  // items in flight per warp
+constexpr int kRowWarps = SSM_ROW_TMA_WARPS;     // warps per CTA
+// register cap: enough for 20 resident warps per SM
+constexpr int kRowMinBlocks = 20 / kRowWarps > 0 ? 20 / kRowWarps : 1;
+
 template <typename ST, typename IoT, int W, int CPT>
-__global__ void __launch_bounds__(256, 3) ssu_row_tma_kernel(const SsuProblem p, const SsuPlan plan) {
+__global__ void __launch_bounds__(32 * kRowWarps, kRowMinBlocks) ssu_row_tma_kernel(const SsuProblem p, const SsuPlan plan) {
     using V = Vec16<ST>;
     constexpr int VE = V::VE;
+    constexpr int NS = CPT * VE;  // d_state
     extern __shared__ __align__(128) unsigned char tma_stage[];
-    __shared__ __align__(8) uint64_t full[kTmaStagesMax];
+    __shared__ __align__(8) uint64_t full[kRowWarps][kWarpStages];
 
-    const unsigned tid = threadIdx.x;
+    const unsigned lane = threadIdx.x & 31u;
+    const unsigned warp = threadIdx.x >> 5;
     const unsigned Dch = (unsigned)p.H;  // channels (rows)
     const unsigned Bn = (unsigned)p.Bn;
-    const unsigned rb = (unsigned)plan.rows_per_item;  // <= blockDim.x: one row per thread
+    constexpr unsigned rb = 32;          // rows per item: one per lane
     const unsigned n_items = (unsigned)plan.n_items;
-    const unsigned per = (n_items + gridDim.x - 1) / gridDim.x;
-    const unsigned i0 = blockIdx.x * per;
+    const unsigned nw = gridDim.x * kRowWarps;
+    const unsigned per = (n_items + nw - 1) / nw;
+    const unsigned i0 = (blockIdx.x * kRowWarps + warp) * per;
     const unsigned i1 = min(i0 + per, n_items);
-    if (i0 >= i1) return;  // uniform
-    const unsigned cnt = i1 - i0;
-    const unsigned S = (unsigned)plan.stages;
+    const unsigned cnt = i0 < i1 ? i1 - i0 : 0u;
     const unsigned stage_bytes = (unsigned)plan.stage_bytes;
-    const unsigned row_bytes = (unsigned)(p.N * (int64_t)sizeof(ST));
+    unsigned char* ring = tma_stage + warp * kWarpStages * stage_bytes;
+    uint64_t* bars = full[warp];
+    const unsigned row_bytes = (unsigned)(NS * sizeof(ST));
     const unsigned cs_es = p.cs_dt == kF32 ? 4u : 2u;
     const unsigned pad16 = 15u;
-    const unsigned N = (unsigned)p.N;
     // stage layout: state rows | conv rows | x | dt | z | B | C
     const unsigned off_cs = rb * row_bytes;
     const unsigned off_x = off_cs + ((rb * (unsigned)W * cs_es + pad16) & ~pad16);
@@ -499,7 +520,7 @@ __global__ void __launch_bounds__(256, 3) ssu_row_tma_kernel(const SsuProblem p,
     const unsigned off_dt = off_x + io_bytes;
     const unsigned off_z = off_dt + io_bytes;
     const unsigned off_B = off_z + io_bytes;
-    const unsigned bc_bytes = (N * (unsigned)sizeof(IoT) + pad16) & ~pad16;
+    const unsigned bc_bytes = (NS * (unsigned)sizeof(IoT) + pad16) & ~pad16;
     const unsigned off_C = off_B + bc_bytes;
     const IoT* __restrict__ xg = static_cast<const IoT*>(p.x);
     const IoT* __restrict__ dtg = static_cast<const IoT*>(p.dt);
@@ -507,17 +528,19 @@ __global__ void __launch_bounds__(256, 3) ssu_row_tma_kernel(const SsuProblem p,
     const IoT* __restrict__ Bg = static_cast<const IoT*>(p.Bm);
     const IoT* __restrict__ Cg = static_cast<const IoT*>(p.Cm);
     IoT* __restrict__ og = static_cast<IoT*>(p.out);
+    const unsigned rot = (lane / (8u / CPT)) & (CPT - 1u);
 
     auto slot_of = [&](unsigned b) -> int64_t {
         if (!p.slot_idx) return b;
         const int64_t sl = p.slot_idx[b * p.si_b];
         return (sl < 0 || sl >= p.n_slots) ? -1 : sl;
     };
-    // item -> (channel block, batch row); channel-block-major order
+    // lane 0: start the copies of local item k; a padding row completes the
+    // stage's phase without data
     auto issue = [&](unsigned k) {
         const unsigned item = i0 + k;
         const unsigned cb = item / Bn, b = item - cb * Bn;
-        uint64_t* bar = &full[k % S];
+        uint64_t* bar = &bars[k % kWarpStages];
         const int64_t slot = slot_of(b);
         if (slot < 0) {
             mbar_arrive(bar);
@@ -525,7 +548,7 @@ __global__ void __launch_bounds__(256, 3) ssu_row_tma_kernel(const SsuProblem p,
         }
         const unsigned c0 = cb * rb;
         const unsigned nr = min(rb, Dch - c0);
-        unsigned char* dst = tma_stage + (k % S) * stage_bytes;
+        unsigned char* dst = ring + (k % kWarpStages) * stage_bytes;
         const uint32_t sbytes = nr * row_bytes;
         const uint32_t cbytes = W > 0 ? nr * (unsigned)W * cs_es : 0u;
         const uint32_t ibytes = nr * (unsigned)sizeof(IoT);
@@ -542,61 +565,74 @@ __global__ void __launch_bounds__(256, 3) ssu_row_tma_kernel(const SsuProblem p,
         tma_load_1d(dst + off_C, Cg + b * p.C_b, bc_bytes, bar);
     };
 
-    if (tid == 0) {
-        for (unsigned s2 = 0; s2 < S; ++s2) mbar_init(&full[s2], 1);
+    if (lane == 0) {
+        for (unsigned s2 = 0; s2 < kWarpStages; ++s2) mbar_init(&bars[s2], 1);
         mbar_fence_init();
     }
-    __syncthreads();
-    if (tid == 0)
-        for (unsigned k = 0; k < min(cnt, S); ++k) issue(k);
+    __syncwarp();
+    if (lane == 0)
+        for (unsigned k = 0; k < min(cnt, (unsigned)kWarpStages); ++k) issue(k);
 
     for (unsigned k = 0; k < cnt; ++k) {
         const unsigned item = i0 + k;
         const unsigned cb = item / Bn, b = item - cb * Bn;
         const unsigned c0 = cb * rb;
-        const unsigned c1 = min(c0 + rb, Dch);
+        const unsigned c = c0 + lane;
         const int64_t slot = slot_of(b);
-        const unsigned stage = k % S;
-        const uint32_t parity = (k / S) & 1u;
-        // this thread's channel and its parameters (L1-resident across items),
-        // loaded before the stage wait so their latency overlaps the copy
-        const unsigned c = c0 + tid;
-        const bool rok = slot >= 0 && tid < rb && c < c1;
-        const unsigned cc = rok ? c : 0;
+        const bool rok = slot >= 0 && c < Dch;
+        const unsigned cc = rok ? c : 0u;
+        // this lane's channel parameters, loaded before the stage wait so their
+        // latency overlaps the copy; A in the lane's rotated chunk order
         float wv[W > 0 ? W : 1];
         float cbias = 0.0f, dbias = 0.0f, dskip = 0.0f;
-        float4 a4[CPT * VE / 4];
+        float4 a4[NS / 4];
         if (rok) {
 #pragma unroll
             for (int kk = 0; kk < W; ++kk) wv[kk] = p.conv_w[cc * p.cw_c + kk * p.cw_w];
             cbias = (W > 0 && p.conv_b) ? p.conv_b[cc * p.cb_c] : 0.0f;
             dbias = p.dt_bias ? p.dt_bias[cc * p.db_h] : 0.0f;
             dskip = p.Dp ? p.Dp[cc * p.D_h] : 0.0f;
-            const float4* ap = reinterpret_cast<const float4*>(p.A + cc * p.A_h);
+            const float* ap = p.A + cc * p.A_h;
 #pragma unroll
-            for (int i = 0; i < CPT * VE / 4; ++i) a4[i] = __ldg(ap + i);
+            for (int j = 0; j < CPT; ++j) {
+                const unsigned cj = (j + rot) & (CPT - 1u);
+#pragma unroll
+                for (int e = 0; e < VE; e += 4) a4[(j * VE + e) / 4] = __ldg(reinterpret_cast<const float4*>(ap + cj * VE + e));
+            }
         }
-        const bool ok = mbar_wait_bounded(&full[stage], parity, kWaitBudget);
-        if (__syncthreads_or(!ok)) {
-            if (tid == 0) {
-                for (unsigned kk = k; kk < min(cnt, k + S); ++kk)
-                    mbar_wait_bounded(&full[kk % S], (kk / S) & 1u, kWaitBudget);
+        const unsigned stage = k % kWarpStages;
+        const bool ok = mbar_wait_bounded(&bars[stage], (k / kWarpStages) & 1u, kWaitBudget);
+        if (__any_sync(0xffffffffu, !ok)) {
+            // give up: wait (bounded) for this warp's copies still in flight, flag, exit
+            if (lane == 0) {
+                // items issued so far: up to k + kWarpStages - 2 (the first
+                // kWarpStages before the loop, one refill per later step)
+                const unsigned hi = min(cnt, k == 0 ? (unsigned)kWarpStages : k + kWarpStages - 1);
+                for (unsigned kk = k; kk < hi; ++kk)
+                    mbar_wait_bounded(&bars[kk % kWarpStages], (kk / kWarpStages) & 1u, kWaitBudget);
+                bulk_wait_all();
                 atomicExch(&g_ssm_device_error, 1);
             }
             return;
         }
         if (rok) {
-            const unsigned char* st = tma_stage + stage * stage_bytes;
-            const unsigned cl = tid;
+            unsigned char* st = ring + stage * stage_bytes;
+            const unsigned cl = lane;
             const float xv = to_f(reinterpret_cast<const IoT*>(st + off_x)[cl]);
             float u = xv;
             float win[W > 0 ? W : 1];
             if constexpr (W > 0) {
                 const unsigned char* crow = st + off_cs + cl * (unsigned)W * cs_es;
+                if (cs_es == 4 && W == 4) {
+                    // one 16-byte read per row: conflict-free across the warp
+                    const float4 q = *reinterpret_cast<const float4*>(crow);
+                    win[0] = q.y;
+                    win[1] = q.z;
+                    win[2] = q.w;
+                } else {
 #pragma unroll
-                for (int kk = 0; kk < W - 1; ++kk)
-                    win[kk] = cs_es == 4 ? reinterpret_cast<const float*>(crow)[kk + 1]
-                                         : ld_f(crow, kk + 1, p.cs_dt);
+                    for (int kk = 0; kk < W - 1; ++kk) win[kk] = ld_f(crow, kk + 1, p.cs_dt);
+                }
                 win[W - 1] = xv;
                 float acc_c = cbias;
 #pragma unroll
@@ -607,58 +643,79 @@ __global__ void __launch_bounds__(256, 3) ssu_row_tma_kernel(const SsuProblem p,
             const float dl = p.softplus ? softplus_f(v) : v;
             const float dl2 = dl * kLog2e;
             const float du = dl * u;
-            // B and C of the batch row: 16-byte vector reads (broadcast), widened once
-            constexpr int NS = CPT * VE;             // d_state
-            constexpr int IV = 16 / sizeof(IoT);     // I/O values per 16 bytes
-            float bv[NS], cv[NS];
-#pragma unroll
-            for (int i = 0; i < NS; i += IV) {
-                const uint4 rbv = *reinterpret_cast<const uint4*>(st + off_B + i * sizeof(IoT));
-                const uint4 rcv = *reinterpret_cast<const uint4*>(st + off_C + i * sizeof(IoT));
-                Vec16<IoT>::unpack(rbv, bv + i);
-                Vec16<IoT>::unpack(rcv, cv + i);
-            }
-            const unsigned char* srow = st + cl * row_bytes;
-            char* grow = static_cast<char*>(p.state) + (slot * p.st_b + (int64_t)c * p.st_h) * (int64_t)sizeof(ST);
+            unsigned char* srow = st + cl * row_bytes;
             float acc = 0.0f;
 #pragma unroll
             for (int j = 0; j < CPT; ++j) {
-                float sv[VE];
-                V::unpack(*reinterpret_cast<const uint4*>(srow + j * 16), sv);
+                const unsigned cj = (j + rot) & (CPT - 1u);
+                float sv[VE], bv[VE], cv[VE];
+                V::unpack(*reinterpret_cast<const uint4*>(srow + cj * 16), sv);
+                // B/C of this chunk (VE I/O values: 8 or 16 bytes, broadcast)
+                if constexpr (VE * sizeof(IoT) == 16) {
+                    Vec16<IoT>::unpack(*reinterpret_cast<const uint4*>(st + off_B + cj * VE * sizeof(IoT)), bv);
+                    Vec16<IoT>::unpack(*reinterpret_cast<const uint4*>(st + off_C + cj * VE * sizeof(IoT)), cv);
+                } else {
+                    float t8[8];
+                    const uint2 rbv = *reinterpret_cast<const uint2*>(st + off_B + cj * VE * sizeof(IoT));
+                    const uint2 rcv = *reinterpret_cast<const uint2*>(st + off_C + cj * VE * sizeof(IoT));
+                    Vec16<IoT>::unpack(make_uint4(rbv.x, rbv.y, 0u, 0u), t8);
+#pragma unroll
+                    for (int e = 0; e < VE; ++e) bv[e] = t8[e];
+                    Vec16<IoT>::unpack(make_uint4(rcv.x, rcv.y, 0u, 0u), t8);
+#pragma unroll
+                    for (int e = 0; e < VE; ++e) cv[e] = t8[e];
+                }
 #pragma unroll
                 for (int e = 0; e < VE; e += 4) {
-                    const int n = j * VE + e;
-                    const float4 a = a4[n / 4];
+                    const float4 a = a4[(j * VE + e) / 4];
                     const float av[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
-                        sv[e + i] = fmaf(ex2_approx(dl2 * av[i]), sv[e + i], du * bv[n + i]);
-                        acc = fmaf(cv[n + i], sv[e + i], acc);
+                        sv[e + i] = fmaf(ex2_approx(dl2 * av[i]), sv[e + i], du * bv[e + i]);
+                        acc = fmaf(cv[e + i], sv[e + i], acc);
                     }
                 }
-                st_stream16(grow + j * 16, V::pack(sv));
+                // new state back into the stage, in place; bulk-stored below
+                *reinterpret_cast<uint4*>(srow + cj * 16) = V::pack(sv);
             }
             float y = fmaf(dskip, u, acc);
             if (zg) y *= silu_f(to_f(reinterpret_cast<const IoT*>(st + off_z)[cl]));
             og[b * p.o_b + (int64_t)c * p.o_h] = from_f<IoT>(y);
             if constexpr (W > 0) {
-                // rolled conv state: old entries 1..W-1, then x
-                const int64_t cso = slot * p.cs_b + (int64_t)c * p.cs_c;
+                // rolled conv state (old entries 1..W-1, then x), in place
+                unsigned char* crow = st + off_cs + cl * (unsigned)W * cs_es;
                 if (cs_es == 4 && W == 4) {
-                    *reinterpret_cast<float4*>(static_cast<float*>(p.conv_state) + cso) =
-                        make_float4(win[0], win[1], win[2], win[3]);
+                    *reinterpret_cast<float4*>(crow) = make_float4(win[0], win[1], win[2], win[3]);
                 } else {
 #pragma unroll
-                    for (int kk = 0; kk < W; ++kk) st_f(p.conv_state, cso + kk * p.cs_w, p.cs_dt, win[kk]);
+                    for (int kk = 0; kk < W; ++kk) st_f(crow, kk, p.cs_dt, win[kk]);
                 }
             }
         }
-        __syncthreads();  // every thread is done reading this stage
-        if (tid == 0 && k + S < cnt) {
-            fence_proxy_async_smem();
-            issue(k + S);
+        // each lane orders its shared-memory accesses of this stage before the
+        // bulk copies that read (store) and later overwrite (refill) it
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            // stream the item's state and conv rows out of the stage, then refill
+            // the stage of the previous item once its own store has read it
+            if (slot >= 0) {
+                const unsigned nr = min(rb, Dch - c0);
+                const unsigned char* st = ring + stage * stage_bytes;
+                tma_store_1d(static_cast<char*>(p.state) + (slot * p.st_b + (int64_t)c0 * p.st_h) * (int64_t)sizeof(ST),
+                             st, nr * row_bytes);
+                if (W > 0)
+                    tma_store_1d(static_cast<char*>(p.conv_state) + (slot * p.cs_b + (int64_t)c0 * p.cs_c) * (int64_t)cs_es,
+                                 st + off_cs, nr * (unsigned)W * cs_es);
+            }
+            bulk_commit();
+            if (k >= 1 && k - 1 + kWarpStages < cnt) {
+                bulk_wait_read<1>();
+                issue(k - 1 + kWarpStages);
+            }
         }
     }
+    if (lane == 0) bulk_wait_all();
 }
 
 // ------------------------------------------------------------------------
@@ -844,13 +901,15 @@ cudaError_t launch_head_tma_io(const SsuProblem& p, const SsuPlan& plan, cudaStr
 
 template <typename ST, typename IoT>
 cudaError_t launch_row_tma_io(const SsuProblem& p, const SsuPlan& plan, cudaStream_t s) {
-    const int smem = plan.stages * plan.stage_bytes;
+    const int smem = kRowWarps * kWarpStages * plan.stage_bytes;
     auto run = [&](auto kern) -> cudaError_t {
         int per_sm = 0;
         cudaError_t e = prepare_tma_kernel(kern, plan.block, smem, &per_sm);
         if (e != cudaSuccess) return e;
+        // every CTA resident at once; each warp takes a contiguous item range
         const int64_t cap = (int64_t)plan.sms * (per_sm > 0 ? per_sm : 1);
-        const int grid = (int)(plan.n_items < cap ? plan.n_items : cap);
+        const int64_t want = (plan.n_items + kRowWarps - 1) / kRowWarps;
+        const int grid = (int)(want < cap ? want : cap);
         kern<<<grid, plan.block, smem, s>>>(p, plan);
         return cudaGetLastError();
     };
@@ -935,6 +994,8 @@ cudaError_t launch_ssu(const SsuProblem& p, const SsuPlan& plan, cudaStream_t s)
 }
 
 int ssu_tma_max_stages() { return kTmaStagesMax; }
+int ssu_row_tma_warps() { return kRowWarps; }
+int ssu_row_tma_stages() { return kWarpStages; }
 
 // Read the device error word into *code (after the stream's work so far) and
 // clear it.

@@ -65,6 +65,21 @@ __device__ __forceinline__ void tma_load_1d(void* dst, const void* src, uint32_t
         : "memory");
 }
 
+// 1-D bulk copy this CTA's shared memory -> global, tracked in bulk groups of
+// the issuing thread.  Addresses 16-byte aligned, size a multiple of 16.
+__device__ __forceinline__ void tma_store_1d(void* dst, const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+                 "r"(smem_u32(src)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// wait until at most N of this thread's bulk groups still read shared memory
+template <int N> __device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// wait until every bulk group of this thread has completed (writes done)
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // order this thread's earlier generic-proxy shared-memory accesses before
 // later async-proxy (TMA) accesses to the same buffer
 __device__ __forceinline__ void fence_proxy_async_smem() {

@@ -203,7 +203,10 @@ def test_scan_groups_choose_generic_when_tile_straddles_groups(lib):
 def test_decode_2p8b_plan(lib):
     st, info = call(lib, "ssm_selective_state_update", ssu_m1_args(FakeMem()))
     assert st == OK and bd.KERNELS[info.kernel] == "ssu_row_tma"
-    assert info.block == 256 and info.grid == 148 * 3 and info.rows_per_item == 256
+    # one bulk-copy pipeline per warp, 32 channels (one per lane) per work item
+    assert info.block == 128 and info.rows_per_item == 32
+    assert 0 < info.grid <= 148 * 5 and info.work_items == 245 * (5120 // 32)
+    assert 0 < info.smem_bytes <= 48 * 1024 and info.smem_bytes % 128 == 0
     # a channel count that is not a multiple of 8 takes the register-streaming row kernel
     st, info = call(lib, "ssm_selective_state_update", ssu_m1_args(FakeMem(), D=100))
     assert st == OK and bd.KERNELS[info.kernel] == "ssu_row"
