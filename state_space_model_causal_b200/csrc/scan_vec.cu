@@ -102,24 +102,45 @@ __device__ __forceinline__ void store8(IoT* p, const float* f) {
     }
 }
 
-// raw I/O of one chunk as staged by cp.async: x, dt, z of the 16 channels and
-// B, C of the 16 state entries, each [row][32 steps]
-template <typename IoT> struct __align__(16) RawStage {
+// x, dt, z of one chunk as staged by cp.async: [channel][32 steps].  Each
+// thread copies, and later reads back, only its own 8-step vectors.
+template <typename IoT> struct __align__(16) RawXZ {
     IoT x[kDT][kT];
     IoT dt[kDT][kT];
     IoT z[kDT][kT];
+};
+
+// B, C of one chunk: [state entry n][32 steps], read by every thread of the
+// CTA during the scan (so double-buffered).  The 16-byte pieces of row n are
+// stored XOR-swizzled by (n / 4) mod 4, so the four rows 4q + j that the four
+// q-groups read at once fall in distinct banks.
+template <typename IoT> struct __align__(16) RawBC {
     IoT B[16][kT];
     IoT C[16][kT];
 };
+template <typename IoT> constexpr int kCE = 16 / (int)sizeof(IoT);  // elements per 16-byte piece
+__device__ __forceinline__ int bc_swz(int n, int piece) { return piece ^ ((n >> 2) & 3); }
 
 template <typename IoT> struct __align__(16) VecSmem {
-    RawStage<IoT> raw;          // the chunk's inputs, refilled for the next chunk once read
+    RawXZ<IoT> xz;
+    RawBC<IoT> bc[2];
     float4 dd[kPairs][kT + 1];  // (delta_c0, delta_c1, delta*u_c0, delta*u_c1) per channel pair
-    float y[kDT][kYStride];     // D*u, then + sum_n C h
-    float g[kDT][kYStride];     // silu(z)
-    float B[kT][16];
-    float C[kT][16];
+    float y[kDT][kYStride];     // sum_n C h per (channel, step)
 };
+
+// 8 bytes of a B or C row (4 steps of 16-bit I/O, 2 of fp32), widened on use
+template <typename IoT> __device__ __forceinline__ float elt8(const uint2& w, int k);
+template <> __device__ __forceinline__ float elt8<float>(const uint2& w, int k) {
+    return __uint_as_float(k == 0 ? w.x : w.y);
+}
+template <> __device__ __forceinline__ float elt8<__half>(const uint2& w, int k) {
+    const uint32_t h = k < 2 ? w.x : w.y;
+    return __half2float(__ushort_as_half((unsigned short)((k & 1) ? (h >> 16) : (h & 0xffffu))));
+}
+template <> __device__ __forceinline__ float elt8<__nv_bfloat16>(const uint2& w, int k) {
+    const uint32_t h = k < 2 ? w.x : w.y;
+    return __uint_as_float((k & 1) ? (h & 0xffff0000u) : (h << 16));
+}
 
 // per-channel state of the prologue: conv weights, biases, conv history
 template <int W> struct ChanParams {
@@ -128,7 +149,8 @@ template <int W> struct ChanParams {
     float hist[W > 1 ? W - 1 : 1];  // raw inputs at (chunk start) - (W-1) + i
 };
 
-// conv + SiLU, softplus and gate for 8 steps of one channel, in registers
+// conv + SiLU, softplus and gate for 8 steps of one channel, in registers;
+// the softplus and the gate run on packed step pairs
 template <int W>
 __device__ __forceinline__ void prologue8(const ScanProblem& p, ChanParams<W>& cp, const float* xs,
                                           const float* dts, const float* zs, bool has_z, bool v_ok,
@@ -159,11 +181,48 @@ __device__ __forceinline__ void prologue8(const ScanProblem& p, ChanParams<W>& c
         for (int i = 0; i < kV; ++i) u[i] = xs[i];
     }
 #pragma unroll
-    for (int i = 0; i < kV; ++i) {
-        const float v = dts[i] + cp.dbias;
-        dl[i] = v_ok ? (p.softplus ? softplus_f(v) : v) : 0.0f;
-        du[i] = v_ok ? dl[i] * u[i] : 0.0f;
-        gate[i] = has_z ? silu_f(zs[i]) : 1.0f;
+    for (int i = 0; i < kV; i += 2) {
+        const u64 v2 = fadd2(pk(dts[i], dts[i + 1]), pk(cp.dbias, cp.dbias));
+        float v0, v1;
+        upk(v2, v0, v1);
+        if (p.softplus) {
+            // softplus as in softplus_f, on a pair: log1p series for e^v <= 1/16
+            const u64 l2 = fmul2(v2, pk(kLog2e, kLog2e));
+            float l0, l1;
+            upk(l2, l0, l1);
+            const u64 e2 = pk(ex2_approx(l0), ex2_approx(l1));
+            u64 s2 = ffma2(e2, pk(1.0f / 7.0f, 1.0f / 7.0f), pk(-1.0f / 6.0f, -1.0f / 6.0f));
+            s2 = ffma2(s2, e2, pk(0.2f, 0.2f));
+            s2 = ffma2(s2, e2, pk(-0.25f, -0.25f));
+            s2 = ffma2(s2, e2, pk(1.0f / 3.0f, 1.0f / 3.0f));
+            s2 = ffma2(s2, e2, pk(-0.5f, -0.5f));
+            s2 = ffma2(s2, e2, pk(1.0f, 1.0f));
+            s2 = fmul2(s2, e2);
+            float e0, e1, r0, r1;
+            upk(e2, e0, e1);
+            upk(s2, r0, r1);
+            if (e0 > 0.0625f) r0 = v0 > 20.0f ? v0 : log1pf(e0);
+            if (e1 > 0.0625f) r1 = v1 > 20.0f ? v1 : log1pf(e1);
+            v0 = r0;
+            v1 = r1;
+        }
+        dl[i] = v_ok ? v0 : 0.0f;
+        dl[i + 1] = v_ok ? v1 : 0.0f;
+        const u64 du2 = fmul2(pk(dl[i], dl[i + 1]), pk(u[i], u[i + 1]));
+        upk(du2, du[i], du[i + 1]);
+        if (has_z) {
+            // SiLU(z) = z / (1 + 2^(-z log2 e)) on a pair
+            const u64 zn = fmul2(pk(zs[i], zs[i + 1]), pk(-kLog2e, -kLog2e));
+            float a0, a1;
+            upk(zn, a0, a1);
+            const u64 den = fadd2(pk(ex2_approx(a0), ex2_approx(a1)), pk(1.0f, 1.0f));
+            float d0, d1;
+            upk(den, d0, d1);
+            const u64 g2 = fmul2(pk(zs[i], zs[i + 1]), pk(__fdividef(1.0f, d0), __fdividef(1.0f, d1)));
+            upk(g2, gate[i], gate[i + 1]);
+        } else {
+            gate[i] = gate[i + 1] = 1.0f;
+        }
     }
 }
 
@@ -171,9 +230,11 @@ __device__ __forceinline__ void prologue8(const ScanProblem& p, ChanParams<W>& c
 // tid / 4 the channel pair (channels 2pr, 2pr+1) and q = tid % 4.  In the
 // prologue and epilogue q selects the 8-step vector [8q, 8q+8) of the chunk;
 // in the scan it selects the state entries n = 4q .. 4q+3 of both channels.
-// The same thread also loads B/C rows n = pr and pr + 8 (vector q).
+// The same thread stages B/C rows n = pr and pr + 8 (vector q).  Gate and
+// D*u of a thread's prologue vectors stay in its registers until its
+// epilogue, which covers the same (channel, step) vectors.
 template <typename IoT, int W, int SW>
-__global__ void __launch_bounds__(kThreads, 12) scan_vec_kernel(const ScanProblem p) {
+__global__ void __launch_bounds__(kThreads, 9) scan_vec_kernel(const ScanProblem p) {
     __shared__ VecSmem<IoT> sm;
     const int tid = threadIdx.x;
     const int pr = tid >> 2;
@@ -211,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 12) scan_vec_kernel(const ScanProble
                                 ? ld_f(p.conv_state, b * p.cs_b + dch[c] * p.cs_d + (1 + i) * p.cs_k, p.cs_dt)
                                 : 0.0f;
     }
-    // B/C rows this thread loads
+    // B/C rows this thread stages
     const IoT* brow[2];
     const IoT* crow[2];
     bool nok[2];
@@ -242,26 +303,27 @@ __global__ void __launch_bounds__(kThreads, 12) scan_vec_kernel(const ScanProble
 
     const int64_t L = p.L;
     const int nchunks = (int)((L + kT - 1) / kT);
-    constexpr int kVB = kV * (int)sizeof(IoT) / 16;  // 16-byte copies per 8-step vector
-    // each thread stages exactly the vectors it reads back in the prologue
+    constexpr int kE = kCE<IoT>;
+    constexpr int kVB = kV / kE;  // 16-byte copies per 8-step vector
     auto fetch = [&](int ci) {
-        RawStage<IoT>& st = sm.raw;
         const int64_t t = (int64_t)ci * kT + kV * q;
         const bool v_ok = t < L;  // L is a multiple of 8: a vector is all in or all out
         const int64_t ts = v_ok ? t : 0;
+        RawXZ<IoT>& xz = sm.xz;
+        RawBC<IoT>& bc = sm.bc[ci & 1];
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
             const int ch = 2 * pr + c;
+            const int n = pr + 8 * c;
 #pragma unroll
             for (int k = 0; k < kVB; ++k) {
-                cp_async16(&st.x[ch][kV * q] + k * 16 / sizeof(IoT), xrow[c] + ts + k * 16 / sizeof(IoT), v_ok);
-                cp_async16(&st.dt[ch][kV * q] + k * 16 / sizeof(IoT), dtrow[c] + ts + k * 16 / sizeof(IoT), v_ok);
-                cp_async16(&st.z[ch][kV * q] + k * 16 / sizeof(IoT),
-                           (has_z ? zrow[c] : xrow[c]) + ts + k * 16 / sizeof(IoT), v_ok && has_z);
-                cp_async16(&st.B[pr + 8 * c][kV * q] + k * 16 / sizeof(IoT), brow[c] + ts + k * 16 / sizeof(IoT),
-                           v_ok && nok[c]);
-                cp_async16(&st.C[pr + 8 * c][kV * q] + k * 16 / sizeof(IoT), crow[c] + ts + k * 16 / sizeof(IoT),
-                           v_ok && nok[c]);
+                const int e = kV * q + k * kE;  // first step of the piece
+                cp_async16(&xz.x[ch][e], xrow[c] + ts + k * kE, v_ok);
+                cp_async16(&xz.dt[ch][e], dtrow[c] + ts + k * kE, v_ok);
+                cp_async16(&xz.z[ch][e], (has_z ? zrow[c] : xrow[c]) + ts + k * kE, v_ok && has_z);
+                const int sp = bc_swz(n, e / kE) * kE;
+                cp_async16(&bc.B[n][sp], brow[c] + ts + k * kE, v_ok && nok[c]);
+                cp_async16(&bc.C[n][sp], crow[c] + ts + k * kE, v_ok && nok[c]);
             }
         }
         cp_async_commit();
@@ -276,47 +338,38 @@ __global__ void __launch_bounds__(kThreads, 12) scan_vec_kernel(const ScanProble
     };
     fetch(0);
 
+    constexpr int kQ = 8 / (int)sizeof(IoT);  // steps per 8-byte B/C read
     for (int ci = 0; ci < nchunks; ++ci) {
         const int64_t t0 = (int64_t)ci * kT;
         const bool vec_ok = t0 + kV * q < L;
         // ---- this chunk's staged inputs (copied during the previous scan)
         cp_async_wait<0>();
-        const RawStage<IoT>& st = sm.raw;
-        // ---- prologue in registers for both channels, results to shared memory
-        float dlc[2][kV], duc[2][kV];
+        // ---- prologue in registers for both channels; (delta, delta*u) to
+        // shared memory, gate and D*u kept for the epilogue
+        float gk[2][kV], duk[2][kV];
+        {
+            float dlc[2][kV], duc[2][kV];
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-            float xs[kV], dts[kV], zs[kV], u[kV], gate[kV];
-            unpack8(&st.x[2 * pr + c][kV * q], xs);
-            unpack8(&st.dt[2 * pr + c][kV * q], dts);
-            unpack8(&st.z[2 * pr + c][kV * q], zs);
-            prologue8<W>(p, cp[c], xs, dts, zs, has_z, vec_ok && ok[c], q, lane, dlc[c], duc[c], u, gate);
-            const int ch = 2 * pr + c;
-            float4* yp = reinterpret_cast<float4*>(&sm.y[ch][kV * q]);
-            yp[0] = make_float4(cp[c].dskip * u[0], cp[c].dskip * u[1], cp[c].dskip * u[2], cp[c].dskip * u[3]);
-            yp[1] = make_float4(cp[c].dskip * u[4], cp[c].dskip * u[5], cp[c].dskip * u[6], cp[c].dskip * u[7]);
-            float4* gp = reinterpret_cast<float4*>(&sm.g[ch][kV * q]);
-            gp[0] = make_float4(gate[0], gate[1], gate[2], gate[3]);
-            gp[1] = make_float4(gate[4], gate[5], gate[6], gate[7]);
-        }
+            for (int c = 0; c < 2; ++c) {
+                float xs[kV], dts[kV], zs[kV], u[kV];
+                unpack8(&sm.xz.x[2 * pr + c][kV * q], xs);
+                unpack8(&sm.xz.dt[2 * pr + c][kV * q], dts);
+                unpack8(&sm.xz.z[2 * pr + c][kV * q], zs);
+                prologue8<W>(p, cp[c], xs, dts, zs, has_z, vec_ok && ok[c], q, lane, dlc[c], duc[c], u, gk[c]);
 #pragma unroll
-        for (int i = 0; i < kV; ++i)
-            sm.dd[pr][kV * q + i] = make_float4(dlc[0][i], dlc[1][i], duc[0][i], duc[1][i]);
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-            float bv[kV], cv[kV];
-            unpack8(&st.B[pr + 8 * r][kV * q], bv);
-            unpack8(&st.C[pr + 8 * r][kV * q], cv);
-#pragma unroll
-            for (int i = 0; i < kV; ++i) {
-                sm.B[kV * q + i][pr + 8 * r] = bv[i];
-                sm.C[kV * q + i][pr + 8 * r] = cv[i];
+                for (int i = 0; i < kV; ++i) duk[c][i] = cp[c].dskip * u[i];
             }
+#pragma unroll
+            for (int i = 0; i < kV; ++i)
+                sm.dd[pr][kV * q + i] = make_float4(dlc[0][i], dlc[1][i], duc[0][i], duc[1][i]);
         }
-        // each thread re-fills only the staging words it has just read, so the
-        // next chunk's copies can start now and fly during the scan
-        if (ci + 1 < nchunks) fetch(ci + 1);
+        // every thread has waited for its own copies of this chunk: after the
+        // barrier all B/C rows are visible.  x/dt/z words were read back by
+        // their own thread, so the next chunk's copies can start now and fly
+        // during the scan (B/C into the other buffer).
         __syncwarp();
+        if (ci + 1 < nchunks) fetch(ci + 1);
+        const RawBC<IoT>& bc = sm.bc[ci & 1];
 
         // ---- scan: thread (pr, q) updates state entries 4q..4q+3 of both
         // channels; packed pairs run across the two channels
@@ -324,23 +377,35 @@ __global__ void __launch_bounds__(kThreads, 12) scan_vec_kernel(const ScanProble
         for (int tt = 0; tt < kT; tt += 4) {
             float v[8];  // v[2k + c]: partial readout of step tt+k, channel c
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float4 dd = sm.dd[pr][tt + k];
-                const float4 b4 = *reinterpret_cast<const float4*>(&sm.B[tt + k][4 * q]);
-                const float4 c4 = *reinterpret_cast<const float4*>(&sm.C[tt + k][4 * q]);
-                const u64 dl2 = pk(dd.x, dd.y);
-                const u64 du2 = pk(dd.z, dd.w);
-                const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
-                const float cc[4] = {c4.x, c4.y, c4.z, c4.w};
-                u64 y2 = 0;
+            for (int s0 = 0; s0 < 4; s0 += kQ) {
+                // B/C of rows 4q + j for steps tt+s0 .. tt+s0+kQ-1
+                uint2 wb[4], wc[4];
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    const u64 x2 = fmul2(dl2, Ap[j]);
-                    const u64 a2 = j < SW ? exp2_pair_fma(x2) : exp2_pair_sfu(x2);
-                    hp[j] = ffma2(a2, hp[j], fmul2(du2, pk(bb[j], bb[j])));
-                    y2 = j == 0 ? fmul2(pk(cc[j], cc[j]), hp[j]) : ffma2(pk(cc[j], cc[j]), hp[j], y2);
+                    const int n = 4 * q + j;
+                    const int e = tt + s0;
+                    const int off = bc_swz(n, e / kE) * kE + e % kE;
+                    wb[j] = *reinterpret_cast<const uint2*>(&bc.B[n][off]);
+                    wc[j] = *reinterpret_cast<const uint2*>(&bc.C[n][off]);
                 }
-                upk(y2, v[2 * k], v[2 * k + 1]);
+#pragma unroll
+                for (int kk = 0; kk < kQ; ++kk) {
+                    const int k = s0 + kk;
+                    const float4 dd = sm.dd[pr][tt + k];
+                    const u64 dl2 = pk(dd.x, dd.y);
+                    const u64 du2 = pk(dd.z, dd.w);
+                    u64 y2 = 0;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const float bj = elt8<IoT>(wb[j], kk);
+                        const float cj = elt8<IoT>(wc[j], kk);
+                        const u64 x2 = fmul2(dl2, Ap[j]);
+                        const u64 a2 = j < SW ? exp2_pair_fma(x2) : exp2_pair_sfu(x2);
+                        hp[j] = ffma2(a2, hp[j], fmul2(du2, pk(bj, bj)));
+                        y2 = j == 0 ? fmul2(pk(cj, cj), hp[j]) : ffma2(pk(cj, cj), hp[j], y2);
+                    }
+                    upk(y2, v[2 * k], v[2 * k + 1]);
+                }
             }
             // butterfly reduce-scatter of the 8 partials over the 4 threads of
             // the pair: thread q ends with both channels' totals for step tt+q
@@ -359,13 +424,13 @@ __global__ void __launch_bounds__(kThreads, 12) scan_vec_kernel(const ScanProble
                     const float keep = up1 ? v[i + 2] : v[i];
                     v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
                 }
-                sm.y[2 * pr][tt + q] += v[0];
-                sm.y[2 * pr + 1][tt + q] += v[1];
+                sm.y[2 * pr][tt + q] = v[0];
+                sm.y[2 * pr + 1][tt + q] = v[1];
             }
         }
         __syncwarp();
 
-        // ---- epilogue: gate and store 8 steps of both channels
+        // ---- epilogue: D skip, gate and store 8 steps of both channels
         if (vec_ok) {
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
@@ -373,14 +438,13 @@ __global__ void __launch_bounds__(kThreads, 12) scan_vec_kernel(const ScanProble
                 const int ch = 2 * pr + c;
                 const float4 y0 = *reinterpret_cast<const float4*>(&sm.y[ch][kV * q]);
                 const float4 y1 = *reinterpret_cast<const float4*>(&sm.y[ch][kV * q + 4]);
-                const float4 g0 = *reinterpret_cast<const float4*>(&sm.g[ch][kV * q]);
-                const float4 g1 = *reinterpret_cast<const float4*>(&sm.g[ch][kV * q + 4]);
-                const float o[kV] = {y0.x * g0.x, y0.y * g0.y, y0.z * g0.z, y0.w * g0.w,
-                                     y1.x * g1.x, y1.y * g1.y, y1.z * g1.z, y1.w * g1.w};
+                const float ys[kV] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
+                float o[kV];
+#pragma unroll
+                for (int i = 0; i < kV; ++i) o[i] = (ys[i] + duk[c][i]) * gk[c][i];
                 store8<IoT>(orow[c] + t0 + kV * q, o);
             }
         }
-        __syncwarp();
     }
 
     // ---- final caches
