@@ -66,6 +66,8 @@ def configure(lib):
     lib.oracle_ssu.argtypes = [_i64] * 6 + [_dp] * 9 + [ctypes.c_int] + [_dp] * 3 + [_dp]
     lib.oracle_ssu_mamba2.restype = ctypes.c_int
     lib.oracle_ssu_mamba2.argtypes = [_i64] * 5 + [_dp] * 8 + [_dp] + [ctypes.c_int] + [_dp]
+    lib.oracle_scan_mamba2.restype = ctypes.c_int
+    lib.oracle_scan_mamba2.argtypes = [_i64] * 6 + [_dp] * 8 + [ctypes.c_int] + [_dp] * 3
     return lib
 
 
@@ -234,3 +236,33 @@ def ssu_mamba2(state, x, dt, A, B, C, D=None, z=None, dt_bias=None, dt_softplus=
     if rc != 0:
         raise ValueError("oracle_ssu_mamba2 rejected its arguments")
     return out, st
+
+
+def scan_mamba2(x, dt, A, B, C, D=None, z=None, dt_bias=None, dt_softplus=True, h0=None):
+    """Prefill, Mamba-2 layout.  x, z (Bt, H, P, L); dt (Bt, H, L); A, D, dt_bias (H);
+    B, C (Bt, G, N, L) or (Bt, N, L); h0 (Bt, H, P, N).  Returns (out, h_final)."""
+    lib = _load()
+    xa, px = _in(x)
+    Bt, H, P, L = xa.shape
+    _, pdt = _in(dt, (Bt, H, L))
+    _, pA = _in(A, (H,))
+    Bm = np.asarray(B, dtype=np.float64)
+    Cm = np.asarray(C, dtype=np.float64)
+    if Bm.ndim == 3:
+        Bm = Bm[:, None]
+    if Cm.ndim == 3:
+        Cm = Cm[:, None]
+    G, N = Bm.shape[1], Bm.shape[2]
+    _, pB = _in(Bm, (Bt, G, N, L))
+    _, pC = _in(Cm, (Bt, G, N, L))
+    _, pD = _in(D, (H,)) if D is not None else (None, None)
+    _, pz = _in(z, (Bt, H, P, L)) if z is not None else (None, None)
+    _, pdb = _in(dt_bias, (H,)) if dt_bias is not None else (None, None)
+    _, ph0 = _in(h0, (Bt, H, P, N)) if h0 is not None else (None, None)
+    out, po = _out((Bt, H, P, L))
+    hf, phf = _out((Bt, H, P, N))
+    rc = lib.oracle_scan_mamba2(Bt, H, P, N, G, L, px, pdt, pA, pB, pC, pD, pz, pdb,
+                                int(bool(dt_softplus)), ph0, po, phf)
+    if rc != 0:
+        raise ValueError("oracle_scan_mamba2 rejected its arguments")
+    return out, hf

@@ -36,6 +36,9 @@
  *   scan:  x, dt, z, out (B, D, L);  A (D, N);  Bm, Cm (B, G, N, L);
  *          D, dt_bias, conv_bias (D);  conv_w (D, W);  conv_state (B, D, W);
  *          h (B, D, N).   Channel d reads group g = d / (D / G).
+ *   scan, Mamba-2 layout:  x, z, out (B, H, P, L);  dt (B, H, L);  A (H);
+ *          Bm, Cm (B, G, N, L);  D, dt_bias (H);  h (B, H, P, N).
+ *          Head h reads group g = h / (H / G).
  *   ssu:   state (B, H, P, N);  x, z, out (B, H, P);  dt (B, H, P);
  *          A (H, P, N);  Bm, Cm (B, G, N);  D, dt_bias (H, P);
  *          conv_w (H*P, W); conv_bias (H*P); conv_state (B, H*P, W).
@@ -245,6 +248,57 @@ int oracle_ssu_mamba2(int64_t B, int64_t H, int64_t P, int64_t N, int64_t G,
                 if (D_head) y += D_head[hh] * xv;
                 if (z) y *= o_silu(z[row]);
                 out[row] = y;
+            }
+        }
+    }
+    return 0;
+}
+
+/* ---------------------------------------------------------------------------
+ * Prefill in the Mamba-2 layout: per batch entry and head, sequentially over
+ * t, one Delta and one decay per head and step, then every (p, n) state entry
+ * of the head takes the same update as in the scan above with u = x (no conv):
+ *   delta   = softplus(dt[b,h,t] + dt_bias[h])
+ *   s[p,n]  = exp(delta * A[h]) * s[p,n] + delta * B[b,g,n,t] * x[b,h,p,t]
+ *   out     = (sum_n C[b,g,n,t] * s[p,n] + D[h] * x[b,h,p,t]) * silu(z[b,h,p,t])
+ * with g = h / (H / G).  The per-head scalar A and the group sharing are the
+ * Mamba-2 shape (batch, nheads, headdim, dstate, ngroups) of "[XPU] Add tuned
+ * Mamba SSU configs for Intel Arc Pro B70", section 实现拆解.  h0 (B,H,P,N) or
+ * NULL (zeros); the state after the last step goes to h_final (B,H,P,N).
+ * ------------------------------------------------------------------------- */
+int oracle_scan_mamba2(int64_t B, int64_t H, int64_t P, int64_t N, int64_t G, int64_t L,
+                       const double* x, const double* dt, const double* A_head, const double* Bm,
+                       const double* Cm, const double* D_head, const double* z,
+                       const double* dt_bias_head, int dt_softplus, const double* h0,
+                       double* out, double* h_final) {
+    int64_t b, hh, p, n, t;
+    if (B < 0 || H < 1 || P < 1 || N < 1 || G < 1 || L < 0 || H % G != 0) return -1;
+    const int64_t per_group = H / G;
+    for (b = 0; b < B; ++b) {
+        for (hh = 0; hh < H; ++hh) {
+            double* S = h_final + (b * H + hh) * P * N;  /* the head's P x N state */
+            for (p = 0; p < P; ++p)
+                for (n = 0; n < N; ++n)
+                    S[p * N + n] = h0 ? h0[((b * H + hh) * P + p) * N + n] : 0.0;
+            const int64_t grp = hh / per_group;
+            const double* Bg = Bm + (b * G + grp) * N * L;
+            const double* Cg = Cm + (b * G + grp) * N * L;
+            for (t = 0; t < L; ++t) {
+                double v = dt[(b * H + hh) * L + t] + (dt_bias_head ? dt_bias_head[hh] : 0.0);
+                double delta = dt_softplus ? o_softplus(v) : v;
+                double decay = exp(delta * A_head[hh]);
+                for (p = 0; p < P; ++p) {
+                    const int64_t at = ((b * H + hh) * P + p) * L + t;
+                    double xv = x[at];
+                    double acc = 0.0;
+                    for (n = 0; n < N; ++n) {
+                        S[p * N + n] = decay * S[p * N + n] + delta * Bg[n * L + t] * xv;
+                        acc += Cg[n * L + t] * S[p * N + n];
+                    }
+                    if (D_head) acc += D_head[hh] * xv;
+                    if (z) acc *= o_silu(z[at]);
+                    out[at] = acc;
+                }
             }
         }
     }

@@ -39,6 +39,13 @@ MUTATIONS = [
     ("mamba2_skip_uses_state", "if (D_head) y += D_head[hh] * xv;", "if (D_head) y += D_head[hh] * s[0];"),
     ("conv_state_out_shift", "for (k = 0; k < W; ++k) hist_out[k] = all[L + k];",
      "for (k = 0; k < W; ++k) hist_out[k] = all[L + k - (k > 0)];"),
+    ("m2_prefill_group_index", "const int64_t grp = hh / per_group;", "const int64_t grp = hh % G;"),
+    ("m2_prefill_readout_before_update",
+     "S[p * N + n] = decay * S[p * N + n] + delta * Bg[n * L + t] * xv;\n                        acc += Cg[n * L + t] * S[p * N + n];",
+     "acc += Cg[n * L + t] * S[p * N + n];\n                        S[p * N + n] = decay * S[p * N + n] + delta * Bg[n * L + t] * xv;"),
+    ("m2_prefill_bias_dropped", "double v = dt[(b * H + hh) * L + t] + (dt_bias_head ? dt_bias_head[hh] : 0.0);",
+     "double v = dt[(b * H + hh) * L + t];"),
+    ("m2_prefill_skip_dropped", "if (D_head) acc += D_head[hh] * xv;", "(void)D_head;"),
 ]
 
 # pins exercised against each mutant (all cheap)
@@ -56,6 +63,9 @@ PIN_CALLS = [
     lambda: pins.test_conv_matches_numpy_convolve_and_state(2),
     lambda: pins.test_conv_impulse_response(4),
     lambda: pins.test_activation_special_values(),
+    lambda: pins.test_mamba2_prefill_matches_mamba1_scan_with_heads_expanded(2),
+    lambda: pins.test_mamba2_prefill_equals_repeated_decode(),
+    lambda: pins.test_mamba2_prefill_two_steps_by_hand(),
 ]
 
 

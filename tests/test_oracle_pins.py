@@ -269,6 +269,70 @@ def test_mamba2_groups_map_consecutive_heads():
         np.testing.assert_allclose(st[:, hs], stg, rtol=1e-14)
 
 
+def _m2_prefill_inputs(seed, Bt, H, P, N, G, L):
+    x = _rand((Bt, H, P, L), seed, "m2x")
+    dt = gen.uniform((Bt, H, L), -3.0, 0.5, "pins", seed, "m2dt")
+    A = -gen.uniform((H,), 0.2, 3.0, "pins", seed, "m2A")
+    Bm = _rand((Bt, G, N, L), seed, "m2B")
+    Cm = _rand((Bt, G, N, L), seed, "m2C")
+    Dv = _rand((H,), seed, "m2D")
+    z = _rand((Bt, H, P, L), seed, "m2z")
+    db = _rand((H,), seed, "m2db", 0.5)
+    h0 = _rand((Bt, H, P, N), seed, "m2h0")
+    return x, dt, A, Bm, Cm, Dv, z, db, h0
+
+
+@pytest.mark.parametrize("G", [1, 2])
+def test_mamba2_prefill_matches_mamba1_scan_with_heads_expanded(G):
+    """The Mamba-2-layout prefill equals the (separately pinned) Mamba-1 scan
+    with one channel per (head, headdim) row: A, dt, dt_bias and D repeated
+    over the head's rows and over n, no conv."""
+    Bt, H, P, N, L = 2, 4, 3, 5, 9
+    x, dt, A, Bm, Cm, Dv, z, db, h0 = _m2_prefill_inputs(11, Bt, H, P, N, G, L)
+    out, hf = oracle.scan_mamba2(x, dt, A, Bm, Cm, D=Dv, z=z, dt_bias=db, h0=h0)
+    D1 = H * P
+    out1, hf1, _ = oracle.scan(x.reshape(Bt, D1, L), np.repeat(dt, P, axis=1),
+                               np.repeat(A, P)[:, None] * np.ones((1, N)), Bm, Cm,
+                               D=np.repeat(Dv, P), z=z.reshape(Bt, D1, L),
+                               dt_bias=np.repeat(db, P), h0=h0.reshape(Bt, D1, N))
+    np.testing.assert_allclose(out, out1.reshape(Bt, H, P, L), rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(hf, hf1.reshape(Bt, H, P, N), rtol=1e-12, atol=1e-13)
+
+
+def test_mamba2_prefill_equals_repeated_decode():
+    """L prefill steps equal L single-token updates of the (separately pinned)
+    Mamba-2 decode oracle, state carried from one to the next."""
+    Bt, H, P, N, G, L = 2, 6, 3, 4, 3, 7
+    x, dt, A, Bm, Cm, Dv, z, db, h0 = _m2_prefill_inputs(12, Bt, H, P, N, G, L)
+    out, hf = oracle.scan_mamba2(x, dt, A, Bm, Cm, D=Dv, z=z, dt_bias=db, h0=h0)
+    st = h0
+    for t in range(L):
+        o, st = oracle.ssu_mamba2(st, x[..., t], dt[..., t], A, Bm[..., t], Cm[..., t], D=Dv,
+                                  z=z[..., t], dt_bias=db)
+        np.testing.assert_allclose(out[..., t], o, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(hf, st, rtol=1e-13, atol=1e-14)
+
+
+def test_mamba2_prefill_two_steps_by_hand():
+    """One head, headdim 2, d_state 1, two steps, written out."""
+    import math
+    x = np.array([[[[0.5, -1.0], [2.0, 0.25]]]])      # (1, 1, 2, 2)
+    dt = np.array([[[0.3, -0.2]]])
+    A, Dv, db = np.array([-1.5]), np.array([0.7]), np.array([0.1])
+    Bm = np.array([[[[1.2, -0.4]]]])                  # (1, 1, 1, 2)
+    Cm = np.array([[[[0.9, 2.0]]]])
+    out, hf = oracle.scan_mamba2(x, dt, A, Bm, Cm, D=Dv, dt_bias=db)
+    sp = lambda v: math.log1p(math.exp(v))  # noqa: E731
+    for p in range(2):
+        h = 0.0
+        for t in range(2):
+            d = sp(dt[0, 0, t] + db[0])
+            h = math.exp(d * A[0]) * h + d * Bm[0, 0, 0, t] * x[0, 0, p, t]
+            assert out[0, 0, p, t] == pytest.approx(Cm[0, 0, 0, t] * h + Dv[0] * x[0, 0, p, t],
+                                                    rel=1e-14, abs=1e-15)
+        assert hf[0, 0, p, 0] == pytest.approx(h, rel=1e-14)
+
+
 def test_ssu_single_step_matches_scan_brute_force_with_groups():
     """One decode step with state, conv and groups equals the brute-force scan
     of a single token whose conv history is the incoming conv state."""
