@@ -191,6 +191,69 @@ class Prefill:
                                conv_state=self.cs, ssm_state=self.h, out=self.out, stream=stream)
 
 
+class PrefillM2:
+    """Mamba-2-layout prefill, Mamba-2 2.7B-shaped layer (d_inner 5120 = 80 heads x
+    headdim 64, dstate 128, one group), B=8, L=2048, fp16 I/O, fp32 state.  Inputs
+    are drawn on the device and stored time-major as the model holds them (x as
+    (B, L, H, P)), passed as their (B, H, P, L) views."""
+
+    def __init__(self, dev, Bt=8, L=2048, H=80, P=64, N=128):
+        import torch
+        from state_space_model_causal_b200 import inputs as gen
+        tag = ("bench", "prefill_m2")
+        self.Bt, self.L, self.H, self.P, self.N = Bt, L, H, P, N
+        view = lambda t: t.permute(0, 2, 3, 1)  # noqa: E731
+        self.x = view(gen.device_normal((Bt, L, H, P), "f16", *tag, "x", device=dev))
+        self.z = view(gen.device_normal((Bt, L, H, P), "f16", *tag, "z", device=dev))
+        self.dt = gen.device_uniform((Bt, L, H), -4.0, -1.0, "f16", *tag, "dt", device=dev).permute(0, 2, 1)
+        self.B = view(gen.device_normal((Bt, L, 1, N), "f16", *tag, "B", device=dev))
+        self.C = view(gen.device_normal((Bt, L, 1, N), "f16", *tag, "C", device=dev))
+        self.A = -torch.from_numpy(gen.uniform((H,), 1.0, 16.0, *tag, "A").astype(np.float32)).to(dev)
+        self.db = torch.from_numpy(gen.dt_bias_draw((H,), *tag, "db").astype(np.float32)).to(dev)
+        self.Dv = torch.ones(H, device=dev)
+        self.h = gen.device_normal((Bt, H, P, N), "f32", *tag, "h0", device=dev)
+        self.out = view(torch.empty(Bt, L, H, P, dtype=torch.float16, device=dev))
+        self.elems = Bt * L * H * P * N
+
+    def algorithmic_bytes(self):
+        io = 3 * self.Bt * self.L * self.H * self.P * 2 + self.Bt * self.L * self.H * 2  # x, z, out; dt
+        bc = 2 * self.Bt * self.L * self.N * 2
+        state = 2 * self.Bt * self.H * self.P * self.N * 4  # read and written
+        return io + bc + state + 3 * self.H * 4
+
+    def run(self):
+        from state_space_model_causal_b200 import ssm_selective_scan_fwd
+        ssm_selective_scan_fwd(self.x, self.dt, self.A, self.B, self.C, D=self.Dv, z=self.z,
+                               dt_bias=self.db, ssm_state=self.h, out=self.out)
+
+
+def prefill_mamba2(dev, hbm_peak, sm_max, steps=20, warmup=3):
+    """Mamba-2-layout prefill: CUDA events per step, L2 flushed before each."""
+    import torch
+    pm = PrefillM2(dev)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    ms = time_prefill(pm, steps, warmup, dev, flush)
+    mean = statistics.mean(ms)
+    gel = pm.elems / (mean * 1e-3) / 1e9
+    # FP32 pipe: 128 lanes per SM; per state element and step the method needs
+    # delta*x*B (1 mul), the decay FMA and the readout FMA: 3 FP32 operations
+    fp32_peak = NUM_SMS * 128 * sm_max * 1e6 / 3 / 1e9  # Gelem/s
+    alg = pm.algorithmic_bytes()
+    gbs = alg / (mean * 1e-3) / 1e9
+    traffic = profiled_traffic("scan_m2_prefill_2p7b.txt", ["scan_m2.cu", "common.cuh"])
+    del pm
+    torch.cuda.empty_cache()
+    return {"workload": "mamba2-2.7b-prefill: B=8 L=2048 H=80 P=64 N=128 G=1, fp16 I/O, fp32 state, "
+                        "time-major rows",
+            "us_per_call": round(mean * 1e3, 2), "Gelem_s": round(gel, 1),
+            "roofline": {"bound": "alu", "achieved": round(gel, 1), "peak": round(fp32_peak, 1),
+                         "unit": "Gelem/s", "frac": round(gel / fp32_peak, 4), "traffic": traffic,
+                         "peak_kind": "FP32 pipe 128 lanes/SM x 148 SMs x max SM clock / 3 ops per element",
+                         "hbm_achieved_gbs": round(gbs, 1), "hbm_peak_gbs": hbm_peak,
+                         "hbm_frac": round(gbs / hbm_peak, 4), "algorithmic_bytes_per_launch": alg},
+            "l2": "flushed (256 MiB write) before every step", "gpu_launches": steps}
+
+
 def time_prefill(pf, steps, warmup, dev, flush):
     """Per-step CUDA events around the kernel only, L2 flushed before each step."""
     import torch
@@ -450,6 +513,9 @@ def run_only(args, dev):
     if args.only == "prefill":
         pf = Prefill(dev)
         fn = pf.run
+    elif args.only == "prefill_m2":
+        pm = PrefillM2(dev)
+        fn = pm.run
     elif args.only == "decode_m1":
         Bt, D, N, W = args.B, 5120, 16, 4  # default: two layers' worth of rows, 200 MB of state
         tag = ("only", "decode_m1")
@@ -505,8 +571,8 @@ def main():
     ap.add_argument("--sweep", action="store_true", help="per-effective-batch decode sweep lines")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--only", choices=["prefill", "decode_m1", "m2_f16", "m2_f32", "m2_bf16",
-                                       "m2_f32_256"],
+    ap.add_argument("--only", choices=["prefill", "prefill_m2", "decode_m1", "m2_f16", "m2_f32",
+                                       "m2_bf16", "m2_f32_256"],
                     help="run --warmup then --steps launches of one case and exit "
                          "(for profiler captures; prints no JSON line)")
     ap.add_argument("--R", type=int, default=16384, help="effective batch for --only m2_*")
@@ -579,6 +645,8 @@ def main():
     e2e_ms, h2d, d2h = time_prefill_e2e(pf, max(3, args.steps // 4), 3, dev)
     e2e_val = world * pf.elems / (statistics.mean(e2e_ms) * 1e-3) / 1e9
 
+    prefill_m2 = prefill_mamba2(dev, hbm_peak, sm_max) if not args.no_decode else None
+
     decode = []
     if not args.no_decode:
         decode.append(decode_mamba1_2p8b(dev, hbm_peak))
@@ -607,7 +675,8 @@ def main():
             "roofline": roofline, "cpu_baseline": cpu,
             "e2e": {"value": round(e2e_val, 3), "unit": "Gelem/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
-            "gpu_launches": args.steps, "clocks": clk.summary(), "decode": decode}
+            "gpu_launches": args.steps, "clocks": clk.summary(), "prefill_mamba2": prefill_m2,
+            "decode": decode}
     print(json.dumps(line), flush=True)
     return 0
 

@@ -129,8 +129,13 @@ typedef enum ssm_kernel_id {
     SSM_KERNEL_SSU_TMA = 9,         /* state update fed by bulk copies (TMA) into
                                        shared-memory stages: one decay per head, dense
                                        rows (Mamba-2 layout, scalar A, no conv) */
-    SSM_KERNEL_SSU_ROW_TMA = 10     /* state update fed by bulk copies: a decay per
+    SSM_KERNEL_SSU_ROW_TMA = 10,    /* state update fed by bulk copies: a decay per
                                        element, fused conv roll (Mamba-1 layout) */
+    SSM_KERNEL_SCAN_M2 = 11,        /* Mamba-2-layout prefill: register tiles of the
+                                       (headdim x dstate) state per head, staged
+                                       16-step chunks; headdim and dstate contiguous,
+                                       dstate 64, 128 or 256, headdim % 8 == 0 */
+    SSM_KERNEL_SCAN_M2_GENERIC = 12 /* Mamba-2-layout prefill, any strides, warp per row */
 } ssm_kernel_id;
 
 /* ------------------------------------------------------------------------ *
@@ -185,6 +190,24 @@ ssm_status ssm_causal_conv1d_fwd(const ssm_conv1d_args* args, void* stream);
  *
  * The time dimension (last) of x, dt, z, B, C and out may have any stride; the
  * fast kernel needs it to be 1.  L = 0 leaves every cache unchanged.
+ *
+ * Mamba-2 layout (x of rank 4): one Delta and one scalar A per head,
+ *   x, z, out   (B, H, P, L)         f32 | f16 | bf16    (z optional)
+ *   dt          (B, H, L)            x's dtype
+ *   A           (H)                  f32
+ *   B, C        (B, G, N, L) or (B, N, L)  x's dtype; head h reads group h / (H/G)
+ *   D, dt_bias  (H)                  f32, optional
+ *   ssm_state   (B, H, P, N)         f32, optional in/out as above
+ *   conv_*      must be absent (SSM_ERR_UNSUPPORTED): the Mamba-2 conv runs
+ *               over the concatenated x/B/C channels before they are split, as
+ *               its own ssm_causal_conv1d_fwd call.
+ * For every (b, h, p, t): delta = softplus(dt[b,h,t] + dt_bias[h]);
+ * s[n] = exp(delta * A[h]) * s[n] + delta * B[b,g,n,t] * x[b,h,p,t];
+ * out = (sum_n C[b,g,n,t] * s[n] + D[h] * x[b,h,p,t]) * silu(z[b,h,p,t]).
+ * The fast kernel wants the time-major memory of the Mamba-2 model: P
+ * contiguous in x, z and out, N contiguous in B and C (e.g. x stored as
+ * (B, L, H, P) and described with the strides of its (B, H, P, L) view),
+ * 16-byte aligned rows, P a multiple of 8 and N = 64, 128 or 256.
  * ------------------------------------------------------------------------ */
 typedef struct ssm_scan_args {
     uint32_t struct_size; /* = sizeof(ssm_scan_args) */

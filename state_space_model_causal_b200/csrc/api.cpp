@@ -96,6 +96,7 @@ bool overlap(const ssm_tensor& a, const ssm_tensor& b) {
 // An output must not write one address twice: sort the non-trivial dims by
 // stride and require each stride to clear the span of the smaller ones.
 bool non_overlapping(const ssm_tensor& t) {
+    if (numel(t) == 0) return true;  // writes nothing
     int64_t st[SSM_MAX_DIMS], sh[SSM_MAX_DIMS];
     int n = 0;
     for (int i = 0; i < t.ndim; ++i) {
@@ -223,6 +224,123 @@ ssm_status conv1d_impl(const ssm_conv1d_args* a, cudaStream_t stream) {
 }
 
 // -------------------------------------------------------------------- scan --
+// Prefill in the Mamba-2 layout (x of rank 4); arguments past the common
+// checks of scan_impl.
+ssm_status scan_m2_impl(const ssm_scan_args* a, cudaStream_t stream) {
+    const int64_t Bn = a->x.shape[0], H = a->x.shape[1], P = a->x.shape[2], L = a->x.shape[3];
+    const int io = a->x.dtype;
+    if (!is_float(io)) return SSM_ERR_DTYPE;
+    if (present(a->conv_weight) || present(a->conv_bias) || present(a->conv_state)) return SSM_ERR_UNSUPPORTED;
+    if (a->A.dtype != SSM_F32) return SSM_ERR_DTYPE;
+    SSM_TRY(want(a->A, {H}));
+    for (const ssm_tensor* t : {&a->dt, &a->B, &a->C, &a->out})
+        if (t->dtype != io) return SSM_ERR_DTYPE;
+    SSM_TRY(want(a->dt, {Bn, H, L}));
+    SSM_TRY(want(a->out, {Bn, H, P, L}));
+    int64_t G = 1, N = 0;
+    int64_t bs[4], cs[4];  // strides of B, C as (b, g, n, t)
+    if (a->B.ndim == 4) {
+        G = a->B.shape[1];
+        N = a->B.shape[2];
+        SSM_TRY(want(a->B, {Bn, G, N, L}));
+        SSM_TRY(want(a->C, {Bn, G, N, L}));
+        for (int i = 0; i < 4; ++i) { bs[i] = sd(a->B, i); cs[i] = sd(a->C, i); }
+    } else if (a->B.ndim == 3) {
+        N = a->B.shape[1];
+        SSM_TRY(want(a->B, {Bn, N, L}));
+        SSM_TRY(want(a->C, {Bn, N, L}));
+        bs[0] = sd(a->B, 0); bs[1] = 0; bs[2] = sd(a->B, 1); bs[3] = sd(a->B, 2);
+        cs[0] = sd(a->C, 0); cs[1] = 0; cs[2] = sd(a->C, 1); cs[3] = sd(a->C, 2);
+    } else {
+        return SSM_ERR_SHAPE;
+    }
+    if (G < 1 || (H > 0 && H % G != 0)) return SSM_ERR_SHAPE;
+    if (N < 1) return SSM_ERR_SHAPE;
+    if (N > kMaxN) return SSM_ERR_UNSUPPORTED;
+    for (const ssm_tensor* t : {&a->D, &a->dt_bias}) {
+        if (!present(*t)) continue;
+        SSM_TRY(basic(*t));
+        SSM_TRY(want(*t, {H}));
+        if (t->dtype != SSM_F32) return SSM_ERR_DTYPE;
+    }
+    if (present(a->z)) {
+        SSM_TRY(basic(a->z));
+        SSM_TRY(want(a->z, {Bn, H, P, L}));
+        if (a->z.dtype != io) return SSM_ERR_DTYPE;
+    }
+    if (present(a->ssm_state)) {
+        SSM_TRY(basic(a->ssm_state));
+        SSM_TRY(want(a->ssm_state, {Bn, H, P, N}));
+        if (a->ssm_state.dtype != SSM_F32) return SSM_ERR_DTYPE;
+        if (!non_overlapping(a->ssm_state)) return SSM_ERR_STRIDE;
+    }
+    if (!non_overlapping(a->out)) return SSM_ERR_STRIDE;
+    const ssm_tensor* ins[] = {&a->x, &a->dt, &a->A, &a->B, &a->C, &a->D, &a->z, &a->dt_bias};
+    for (const ssm_tensor* o : {&a->out, &a->ssm_state}) {
+        if (!present(*o)) continue;
+        for (const ssm_tensor* t : ins)
+            if (present(*t) && overlap(*o, *t)) return SSM_ERR_ALIAS;
+    }
+    if (overlap(a->out, a->ssm_state)) return SSM_ERR_ALIAS;
+
+    ScanM2Problem p{};
+    p.Bn = Bn; p.H = H; p.P = P; p.N = N; p.G = G; p.L = L;
+    p.io_dt = io;
+    p.x = a->x.data; p.x_b = sd(a->x, 0); p.x_h = sd(a->x, 1); p.x_p = sd(a->x, 2); p.x_t = sd(a->x, 3);
+    p.dt = a->dt.data; p.dt_b = sd(a->dt, 0); p.dt_h = sd(a->dt, 1); p.dt_t = sd(a->dt, 2);
+    p.A = static_cast<const float*>(a->A.data); p.A_h = sd(a->A, 0);
+    p.Bm = a->B.data; p.B_b = bs[0]; p.B_g = bs[1]; p.B_n = bs[2]; p.B_t = bs[3];
+    p.Cm = a->C.data; p.C_b = cs[0]; p.C_g = cs[1]; p.C_n = cs[2]; p.C_t = cs[3];
+    p.Dp = static_cast<const float*>(a->D.data); p.D_h = present(a->D) ? sd(a->D, 0) : 0;
+    p.z = a->z.data;
+    if (present(a->z)) { p.z_b = sd(a->z, 0); p.z_h = sd(a->z, 1); p.z_p = sd(a->z, 2); p.z_t = sd(a->z, 3); }
+    p.dt_bias = static_cast<const float*>(a->dt_bias.data); p.db_h = present(a->dt_bias) ? sd(a->dt_bias, 0) : 0;
+    p.softplus = a->dt_softplus != 0;
+    p.ssm_state = static_cast<float*>(a->ssm_state.data);
+    if (present(a->ssm_state)) {
+        p.ss_b = sd(a->ssm_state, 0); p.ss_h = sd(a->ssm_state, 1); p.ss_p = sd(a->ssm_state, 2);
+        p.ss_n = sd(a->ssm_state, 3);
+    }
+    p.out = a->out.data; p.o_b = sd(a->out, 0); p.o_h = sd(a->out, 1); p.o_p = sd(a->out, 2); p.o_t = sd(a->out, 3);
+    if (Bn == 0 || H == 0 || P == 0 || L == 0) {  // nothing to compute, caches unchanged
+        fill_info(a->info, SSM_KERNEL_NONE, 0, 0, 0, 0, 0);
+        return SSM_OK;
+    }
+    // fast kernel: headdim / dstate contiguous, 16-byte aligned rows and steps
+    const int es = esize(io);
+    const int64_t rpc = scan_m2_rows_per_cta(N);
+    auto al16 = [](const void* ptr) { return ptr == nullptr || aligned16(ptr); };
+    auto m16 = [es](int64_t st) { return (st * es) % 16 == 0; };
+    const bool fast = rpc > 0 && P % 8 == 0 && p.x_p == 1 && p.o_p == 1 &&
+                      (!p.z || p.z_p == 1) && p.B_n == 1 && p.C_n == 1 &&
+                      al16(p.x) && al16(p.out) && al16(p.z) && al16(p.Bm) && al16(p.Cm) &&
+                      m16(p.x_b) && m16(p.x_h) && m16(p.x_t) && m16(p.o_b) && m16(p.o_h) && m16(p.o_t) &&
+                      (!p.z || (m16(p.z_b) && m16(p.z_h) && m16(p.z_t))) && m16(p.B_b) && m16(p.B_g) &&
+                      m16(p.B_t) && m16(p.C_b) && m16(p.C_g) && m16(p.C_t) && H <= 65535 && Bn <= 65535;
+    int kernel, grid, block, smem;
+    int64_t items;
+    if (fast) {
+        kernel = SSM_KERNEL_SCAN_M2;
+        const int64_t blocks = (P + rpc - 1) / rpc;
+        if (blocks * H * Bn > INT32_MAX) return SSM_ERR_UNSUPPORTED;
+        grid = (int)(blocks * H * Bn);
+        block = 128;
+        smem = scan_m2_smem_bytes(io, N);
+        items = blocks * H * Bn;
+    } else {
+        kernel = SSM_KERNEL_SCAN_M2_GENERIC;
+        const int64_t rows = Bn * H * P;
+        if ((rows + 3) / 4 > INT32_MAX) return SSM_ERR_UNSUPPORTED;
+        grid = (int)((rows + 3) / 4);
+        block = 128;
+        smem = 0;
+        items = rows;
+    }
+    fill_info(a->info, kernel, grid, block, smem, fast ? rpc : 1, items);
+    if (a->flags & SSM_FLAG_DRY_RUN) return SSM_OK;
+    return launch_scan_m2(p, kernel, stream) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
 ssm_status scan_impl(const ssm_scan_args* a, cudaStream_t stream) {
     if (!a) return SSM_ERR_NULL;
     if (a->struct_size != sizeof(ssm_scan_args)) return SSM_ERR_VERSION;
@@ -233,6 +351,7 @@ ssm_status scan_impl(const ssm_scan_args* a, cudaStream_t stream) {
     SSM_TRY(basic(a->B));
     SSM_TRY(basic(a->C));
     SSM_TRY(basic(a->out));
+    if (a->x.ndim == 4) return scan_m2_impl(a, stream);
     if (a->x.ndim != 3) return SSM_ERR_SHAPE;
     const int64_t Bn = a->x.shape[0], D = a->x.shape[1], L = a->x.shape[2];
     if (a->A.ndim != 2 || a->A.shape[0] != D) return SSM_ERR_SHAPE;

@@ -79,6 +79,25 @@ struct ScanPlan {
     int sw_pairs;   // vector kernel: state-entry pairs per thread whose exp runs on the FMA pipe
 };
 
+// Prefill in the Mamba-2 layout: x, z, out (Bn, H, P, L); dt (Bn, H, L);
+// A, D, dt_bias (H); B, C (Bn, G, N, L); ssm_state (Bn, H, P, N).  Strides in
+// elements; head h reads group h / (H / G).
+struct ScanM2Problem {
+    int64_t Bn, H, P, N, G, L;
+    int io_dt;
+    const void* x;  int64_t x_b, x_h, x_p, x_t;
+    const void* dt; int64_t dt_b, dt_h, dt_t;
+    const float* A; int64_t A_h;
+    const void* Bm; int64_t B_b, B_g, B_n, B_t;
+    const void* Cm; int64_t C_b, C_g, C_n, C_t;
+    const float* Dp; int64_t D_h;
+    const void* z;  int64_t z_b, z_h, z_p, z_t;
+    const float* dt_bias; int64_t db_h;
+    int softplus;
+    float* ssm_state; int64_t ss_b, ss_h, ss_p, ss_n;
+    void* out; int64_t o_b, o_h, o_p, o_t;
+};
+
 struct Conv1dProblem {
     int64_t Bn, D, L, W;
     int io_dt;
@@ -107,5 +126,8 @@ int scan_vec_threads();
 int scan_vec_channels_per_cta();
 cudaError_t launch_scan_vec(const ScanProblem& p, int sw_pairs, cudaStream_t s);
 cudaError_t launch_conv1d(const Conv1dProblem& p, const Conv1dPlan& plan, cudaStream_t s);
+int scan_m2_rows_per_cta(int64_t N);
+int scan_m2_smem_bytes(int io_dt, int64_t N);
+cudaError_t launch_scan_m2(const ScanM2Problem& p, int kernel, cudaStream_t s);
 
 }  // namespace ssm

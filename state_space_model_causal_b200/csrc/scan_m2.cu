@@ -1,0 +1,431 @@
+// scan_m2.cu -- prefill in the Mamba-2 layout for sm_100a: the selective scan
+// over (nheads, headdim, dstate) with one scalar A and one Delta per head and
+// step, B and C shared by the heads of a group, then the D skip and the SiLU(z)
+// gate.  The Mamba-2 shape (batch, nheads, headdim, dstate, ngroups) is the one
+// of "[XPU] Add tuned Mamba SSU configs for Intel Arc Pro B70" (vLLM PR #50534
+// report), section 实现拆解; per (b, h), sequentially over t:
+//
+//   delta   = softplus(dt[b,h,t] + dt_bias[h])          (dt + dt_bias without softplus)
+//   s[p,n]  = exp(delta * A[h]) * s[p,n] + delta * x[b,h,p,t] * B[b,g,n,t]
+//   out     = (sum_n C[b,g,n,t] * s[p,n] + D[h] * x[b,h,p,t]) * silu(z[b,h,p,t])
+//
+// with g = h / (H / G).  The decay is one exponential per (b, h, t), so the
+// work is two FMAs per state element and step: the kernel is FMA-bound, not
+// SFU-bound like the Mamba-1 prefill.
+//
+// Fast kernel (time-major rows: headdim contiguous in x, z, out, and a
+// multiple of 8; dstate 64, 128 or 256, contiguous in B, C; 16-byte aligned
+// rows):
+//   * a CTA is 128 threads on one (b, h) and a block of RPC = 512 / NG
+//     headdim rows, NG = dstate / 16.  Thread (pg, ng) owns rows 4pg..4pg+3 of
+//     the block and state entries 16ng..16ng+15: a 4 x 16 register tile of the
+//     state, updated with packed f32x2 operations across n;
+//   * 16-step chunks of x, z, B, C are staged by 16-byte cp.async copies into a
+//     double buffer while the previous chunk is scanned; dt is prefetched into a
+//     register one chunk ahead;
+//   * per chunk the CTA computes once (delta, decay) per step, delta * x per
+//     (step, row) and the fp32 B, C rows (16-byte pieces XOR-swizzled so the NG
+//     groups of a quarter-warp read distinct banks);
+//   * the readout partials of 4 steps x 4 rows are summed over the NG threads
+//     of a row block by a butterfly reduce-scatter; the epilogue applies the D
+//     skip and the gate to 8 consecutive rows per thread and stores 16 bytes.
+// Generic kernel: one warp per (b, h, p) row, any strides, dstate <= 256.
+#include "../../include/ssm_causal.h"
+#include "common.cuh"
+#include "problem.h"
+
+namespace ssm {
+namespace {
+
+constexpr int kM2Threads = 128;
+constexpr int kM2T = 16;  // steps per chunk
+
+// (16-byte piece u of a B/C row) -> stored piece: the pieces a quarter-warp's
+// NG groups read at once (u = 4 ng + k) land in distinct banks
+__device__ __forceinline__ int m2_swz(int u) { return u ^ ((u >> 3) & 7); }
+
+template <typename IoT, int NG> struct M2Smem {
+    static constexpr int RPC = 512 / NG;  // headdim rows per CTA
+    static constexpr int N = 16 * NG;
+    struct Raw {
+        IoT x[kM2T][RPC];
+        IoT z[kM2T][RPC];
+        IoT B[kM2T][N];
+        IoT C[kM2T][N];
+    };
+    Raw raw[2];
+    float2 dd[kM2T];           // (decay, delta) per step
+    float dx[kM2T][RPC];       // delta * x
+    float B[kM2T][N];          // swizzled fp32 rows
+    float C[kM2T][N];
+    float y[kM2T][RPC];        // sum_n C s
+};
+
+__device__ __forceinline__ void cp_async16_m2(void* dst, const void* src, bool valid) {
+    const unsigned d = static_cast<unsigned>(__cvta_generic_to_shared(dst));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src), "r"(valid ? 16 : 0)
+                 : "memory");
+}
+
+template <typename IoT, int NG>
+__global__ void __launch_bounds__(kM2Threads) scan_m2_kernel(const ScanM2Problem p) {
+    using S = M2Smem<IoT, NG>;
+    constexpr int RPC = S::RPC;
+    constexpr int N = S::N;
+    constexpr int E = 16 / (int)sizeof(IoT);  // elements per 16-byte copy
+    constexpr int PG = kM2Threads / NG;       // row groups of 4
+    extern __shared__ __align__(16) unsigned char m2_smem[];
+    S& sm = *reinterpret_cast<S*>(m2_smem);
+
+    const int tid = threadIdx.x;
+    const int ng = tid % NG;
+    const int pg = tid / NG;
+    const int64_t b = blockIdx.z;
+    const int64_t h = blockIdx.y;
+    const int64_t p0 = (int64_t)blockIdx.x * RPC;  // first headdim row of the CTA
+    const int64_t g = h / (p.H / p.G);
+    const int64_t L = p.L;
+    const IoT* xg = static_cast<const IoT*>(p.x) + b * p.x_b + h * p.x_h + p0;
+    const IoT* zg = p.z ? static_cast<const IoT*>(p.z) + b * p.z_b + h * p.z_h + p0 : nullptr;
+    const IoT* Bg = static_cast<const IoT*>(p.Bm) + b * p.B_b + g * p.B_g;
+    const IoT* Cg = static_cast<const IoT*>(p.Cm) + b * p.C_b + g * p.C_g;
+    const IoT* dtg = static_cast<const IoT*>(p.dt) + b * p.dt_b + h * p.dt_h;
+    IoT* og = static_cast<IoT*>(p.out) + b * p.o_b + h * p.o_h + p0;
+    const float A2 = p.A[h * p.A_h] * kLog2e;
+    const float dbias = p.dt_bias ? p.dt_bias[h * p.db_h] : 0.0f;
+    const float dskip = p.Dp ? p.Dp[h * p.D_h] : 0.0f;
+    const int rows = (int)(p.P - p0 < RPC ? p.P - p0 : RPC);  // valid rows of the block
+
+    // state tile: rows 4pg + r, entries 16ng + 2j, 16ng + 2j + 1 as pairs
+    u64 hs[4][8];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const int row = 4 * pg + r;
+        const bool v = row < rows;
+        const float* src = p.ssm_state
+                               ? p.ssm_state + b * p.ss_b + h * p.ss_h + (p0 + (v ? row : 0)) * p.ss_p +
+                                     16 * ng * p.ss_n
+                               : nullptr;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            float a = 0.0f, c = 0.0f;
+            if (src && v) {
+                a = src[(2 * j) * p.ss_n];
+                c = src[(2 * j + 1) * p.ss_n];
+            }
+            hs[r][j] = pk(a, c);
+        }
+    }
+    // this thread's B/C pieces: u = 4ng + k, stored at m2_swz(u)
+    int boff[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) boff[k] = m2_swz(4 * ng + k) * 4;
+
+    const int nchunks = (int)((L + kM2T - 1) / kM2T);
+    auto fetch = [&](int ci) {
+        typename S::Raw& rw = sm.raw[ci & 1];
+        const int64_t t0 = (int64_t)ci * kM2T;
+        // x, z: kM2T x RPC elements; B, C: kM2T x N
+        constexpr int XC = kM2T * RPC / E;
+        constexpr int BC = kM2T * N / E;
+        for (int i = tid; i < XC; i += kM2Threads) {
+            const int t = i / (RPC / E), e = (i % (RPC / E)) * E;
+            const bool v = t0 + t < L && e < rows;
+            const int64_t ts = v ? t0 + t : 0;
+            cp_async16_m2(&rw.x[t][e], xg + ts * p.x_t + (v ? e : 0), v);
+            cp_async16_m2(&rw.z[t][e], (zg ? zg : xg) + ts * (zg ? p.z_t : p.x_t) + (v ? e : 0), v && zg);
+        }
+        for (int i = tid; i < BC; i += kM2Threads) {
+            const int t = i / (N / E), e = (i % (N / E)) * E;
+            const bool v = t0 + t < L;
+            const int64_t ts = v ? t0 + t : 0;
+            cp_async16_m2(&rw.B[t][e], Bg + ts * p.B_t + e, v);
+            cp_async16_m2(&rw.C[t][e], Cg + ts * p.C_t + e, v);
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    // dt of the next chunk, one step per thread of the first warp
+    float dt_next = 0.0f;
+    auto load_dt = [&](int ci) {
+        const int64_t t = (int64_t)ci * kM2T + tid;
+        dt_next = (tid < kM2T && t < L) ? to_f(dtg[t * p.dt_t]) : 0.0f;
+    };
+    fetch(0);
+    load_dt(0);
+
+    for (int ci = 0; ci < nchunks; ++ci) {
+        const int64_t t0 = (int64_t)ci * kM2T;
+        const int steps = (int)(L - t0 < kM2T ? L - t0 : kM2T);
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+        // ---- per step: delta and the decay (steps past L keep the state)
+        if (tid < kM2T) {
+            float delta = 0.0f, decay = 1.0f;
+            if (tid < steps) {
+                const float v = dt_next + dbias;
+                delta = p.softplus ? softplus_f(v) : v;
+                decay = ex2_approx(delta * A2);
+            }
+            sm.dd[tid] = make_float2(decay, delta);
+        }
+        __syncthreads();  // dd and this chunk's staged rows visible to all
+        if (ci + 1 < nchunks) {
+            fetch(ci + 1);
+            load_dt(ci + 1);
+        }
+        const typename S::Raw& rw = sm.raw[ci & 1];
+        // ---- widen: delta * x per (step, row), fp32 B / C rows (swizzled)
+        for (int i = tid; i < kM2T * RPC / 8; i += kM2Threads) {
+            const int t = i / (RPC / 8), e = (i % (RPC / 8)) * 8;
+            float xv[8];
+            if constexpr (sizeof(IoT) == 2) {
+                Vec16<IoT>::unpack(*reinterpret_cast<const uint4*>(&rw.x[t][e]), xv);
+            } else {
+                Vec16<float>::unpack(*reinterpret_cast<const uint4*>(&rw.x[t][e]), xv);
+                Vec16<float>::unpack(*reinterpret_cast<const uint4*>(&rw.x[t][e + 4]), xv + 4);
+            }
+            const float dl = sm.dd[t].y;
+            *reinterpret_cast<float4*>(&sm.dx[t][e]) = make_float4(dl * xv[0], dl * xv[1], dl * xv[2], dl * xv[3]);
+            *reinterpret_cast<float4*>(&sm.dx[t][e + 4]) = make_float4(dl * xv[4], dl * xv[5], dl * xv[6], dl * xv[7]);
+        }
+        for (int i = tid; i < kM2T * N / 4; i += kM2Threads) {
+            const int t = i / (N / 4), u = i % (N / 4);  // 16-byte fp32 piece u of row t
+            float bv[4], cv[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                bv[k] = to_f(rw.B[t][4 * u + k]);
+                cv[k] = to_f(rw.C[t][4 * u + k]);
+            }
+            const int su = m2_swz(u) * 4;
+            *reinterpret_cast<float4*>(&sm.B[t][su]) = make_float4(bv[0], bv[1], bv[2], bv[3]);
+            *reinterpret_cast<float4*>(&sm.C[t][su]) = make_float4(cv[0], cv[1], cv[2], cv[3]);
+        }
+        __syncthreads();
+
+        // ---- scan: 4 groups of 4 steps
+#pragma unroll 1
+        for (int tt = 0; tt < kM2T; tt += 4) {
+            float v[16];  // v[4r + k]: partial readout of row r at step tt + k
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int t = tt + k;
+                const float decay = sm.dd[t].x;
+                const u64 dA2 = pk(decay, decay);
+                const float4 dx4 = *reinterpret_cast<const float4*>(&sm.dx[t][4 * pg]);
+                const float dxr[4] = {dx4.x, dx4.y, dx4.z, dx4.w};
+                u64 b2[8], c2[8];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float4 bq = *reinterpret_cast<const float4*>(&sm.B[t][boff[q]]);
+                    const float4 cq = *reinterpret_cast<const float4*>(&sm.C[t][boff[q]]);
+                    b2[2 * q] = pk(bq.x, bq.y);
+                    b2[2 * q + 1] = pk(bq.z, bq.w);
+                    c2[2 * q] = pk(cq.x, cq.y);
+                    c2[2 * q + 1] = pk(cq.z, cq.w);
+                }
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    const u64 dx2 = pk(dxr[r], dxr[r]);
+                    u64 y2 = 0;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        hs[r][j] = ffma2(dA2, hs[r][j], fmul2(dx2, b2[j]));
+                        y2 = j == 0 ? fmul2(c2[j], hs[r][j]) : ffma2(c2[j], hs[r][j], y2);
+                    }
+                    float lo, hi;
+                    upk(y2, lo, hi);
+                    v[4 * r + k] = lo + hi;
+                }
+            }
+            // butterfly reduce-scatter over the NG threads of the row group:
+            // thread ng ends with v[i], i = ng * (16 / NG) + local
+#pragma unroll
+            for (int m = NG / 2, S2 = 8; m >= 1; m >>= 1, S2 >>= 1) {
+                const bool up = (ng & m) != 0;
+#pragma unroll
+                for (int i = 0; i < S2; ++i) {
+                    const float send = up ? v[i] : v[i + S2];
+                    const float keep = up ? v[i + S2] : v[i];
+                    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+                }
+            }
+#pragma unroll
+            for (int l = 0; l < 16 / NG; ++l) {
+                const int i = ng * (16 / NG) + l;
+                sm.y[tt + (i & 3)][4 * pg + (i >> 2)] = v[l];
+            }
+        }
+        __syncthreads();
+
+        // ---- epilogue: D skip and gate on 8 consecutive rows, 16-byte stores
+        for (int i = tid; i < kM2T * RPC / 8; i += kM2Threads) {
+            const int t = i / (RPC / 8), e = (i % (RPC / 8)) * 8;
+            if (t >= steps || e >= rows) continue;
+            float xv[8], zv[8], o[8];
+            if constexpr (sizeof(IoT) == 2) {
+                Vec16<IoT>::unpack(*reinterpret_cast<const uint4*>(&rw.x[t][e]), xv);
+                Vec16<IoT>::unpack(*reinterpret_cast<const uint4*>(&rw.z[t][e]), zv);
+            } else {
+                Vec16<float>::unpack(*reinterpret_cast<const uint4*>(&rw.x[t][e]), xv);
+                Vec16<float>::unpack(*reinterpret_cast<const uint4*>(&rw.x[t][e + 4]), xv + 4);
+                Vec16<float>::unpack(*reinterpret_cast<const uint4*>(&rw.z[t][e]), zv);
+                Vec16<float>::unpack(*reinterpret_cast<const uint4*>(&rw.z[t][e + 4]), zv + 4);
+            }
+            const float4 y0 = *reinterpret_cast<const float4*>(&sm.y[t][e]);
+            const float4 y1 = *reinterpret_cast<const float4*>(&sm.y[t][e + 4]);
+            const float ys[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                o[k] = fmaf(dskip, xv[k], ys[k]);
+                if (zg) o[k] *= silu_f(zv[k]);
+            }
+            IoT* dst = og + (t0 + t) * p.o_t + e;
+            if constexpr (sizeof(IoT) == 2) {
+                __stcs(reinterpret_cast<uint4*>(dst), Vec16<IoT>::pack(o));
+            } else {
+                __stcs(reinterpret_cast<uint4*>(dst), Vec16<float>::pack(o));
+                __stcs(reinterpret_cast<uint4*>(dst) + 1, Vec16<float>::pack(o + 4));
+            }
+        }
+        // the next chunk overwrites dd / dx / B / C / y only after its own
+        // first barrier, which every thread reaches after this epilogue
+    }
+
+    // ---- final state
+    if (p.ssm_state) {
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const int row = 4 * pg + r;
+            if (row >= rows) continue;
+            float* dst = p.ssm_state + b * p.ss_b + h * p.ss_h + (p0 + row) * p.ss_p + 16 * ng * p.ss_n;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                float a, c;
+                upk(hs[r][j], a, c);
+                dst[(2 * j) * p.ss_n] = a;
+                dst[(2 * j + 1) * p.ss_n] = c;
+            }
+        }
+    }
+}
+
+// One warp per (b, h, p) row, any strides, dstate <= 256: lane l owns entries
+// n = l + 32 i.
+template <typename IoT>
+__global__ void __launch_bounds__(128) scan_m2_generic_kernel(const ScanM2Problem p) {
+    const int lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
+    if (row >= p.Bn * p.H * p.P) return;
+    const int64_t pp = row % p.P, h = (row / p.P) % p.H, b = row / (p.P * p.H);
+    const int64_t g = h / (p.H / p.G);
+    const float A = p.A[h * p.A_h];
+    const float dbias = p.dt_bias ? p.dt_bias[h * p.db_h] : 0.0f;
+    const float dskip = p.Dp ? p.Dp[h * p.D_h] : 0.0f;
+    float s[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int64_t n = lane + 32 * i;
+        s[i] = (n < p.N && p.ssm_state) ? p.ssm_state[b * p.ss_b + h * p.ss_h + pp * p.ss_p + n * p.ss_n] : 0.0f;
+    }
+    for (int64_t t = 0; t < p.L; ++t) {
+        const float v = ld_f(p.dt, b * p.dt_b + h * p.dt_h + t * p.dt_t, p.io_dt) + dbias;
+        const float delta = p.softplus ? softplus_f(v) : v;
+        const float decay = exp_fast(delta * A);
+        const float xv = ld_f(p.x, b * p.x_b + h * p.x_h + pp * p.x_p + t * p.x_t, p.io_dt);
+        const float dx = delta * xv;
+        float acc = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int64_t n = lane + 32 * i;
+            if (n < p.N) {
+                const float bv = ld_f(p.Bm, b * p.B_b + g * p.B_g + n * p.B_n + t * p.B_t, p.io_dt);
+                const float cv = ld_f(p.Cm, b * p.C_b + g * p.C_g + n * p.C_n + t * p.C_t, p.io_dt);
+                s[i] = fmaf(decay, s[i], dx * bv);
+                acc = fmaf(cv, s[i], acc);
+            }
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) {
+            float y = fmaf(dskip, xv, acc);
+            if (p.z) y *= silu_f(ld_f(p.z, b * p.z_b + h * p.z_h + pp * p.z_p + t * p.z_t, p.io_dt));
+            st_f(p.out, b * p.o_b + h * p.o_h + pp * p.o_p + t * p.o_t, p.io_dt, y);
+        }
+    }
+    if (p.ssm_state) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int64_t n = lane + 32 * i;
+            if (n < p.N) p.ssm_state[b * p.ss_b + h * p.ss_h + pp * p.ss_p + n * p.ss_n] = s[i];
+        }
+    }
+}
+
+template <typename IoT, int NG>
+cudaError_t launch_m2_ng(const ScanM2Problem& p, cudaStream_t s) {
+    using Sm = M2Smem<IoT, NG>;
+    auto kern = scan_m2_kernel<IoT, NG>;
+    const int smem = (int)sizeof(Sm);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)((p.P + Sm::RPC - 1) / Sm::RPC), (unsigned)p.H, (unsigned)p.Bn);
+    kern<<<grid, kM2Threads, smem, s>>>(p);
+    return cudaGetLastError();
+}
+
+template <typename IoT>
+cudaError_t launch_m2_io(const ScanM2Problem& p, cudaStream_t s) {
+    switch (p.N / 16) {
+        case 1: return launch_m2_ng<IoT, 1>(p, s);
+        case 2: return launch_m2_ng<IoT, 2>(p, s);
+        case 4: return launch_m2_ng<IoT, 4>(p, s);
+        case 8: return launch_m2_ng<IoT, 8>(p, s);
+        case 16: return launch_m2_ng<IoT, 16>(p, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace
+
+// the fast kernel's dstate values (NG = 4, 8, 16): 0 for any other dstate
+int scan_m2_rows_per_cta(int64_t N) { return N == 64 || N == 128 || N == 256 ? (int)(512 / (N / 16)) : 0; }
+
+int scan_m2_smem_bytes(int io_dt, int64_t N) {
+    auto pick = [&](auto tag) -> int {
+        using T = decltype(tag);
+        switch (N / 16) {
+            case 1: return (int)sizeof(M2Smem<T, 1>);
+            case 2: return (int)sizeof(M2Smem<T, 2>);
+            case 4: return (int)sizeof(M2Smem<T, 4>);
+            case 8: return (int)sizeof(M2Smem<T, 8>);
+            case 16: return (int)sizeof(M2Smem<T, 16>);
+            default: return 0;
+        }
+    };
+    if (io_dt == kF32) return pick(float{});
+    if (io_dt == kF16) return pick(__half{});
+    return pick(__nv_bfloat16{});
+}
+
+cudaError_t launch_scan_m2(const ScanM2Problem& p, int kernel, cudaStream_t s) {
+    if (kernel == SSM_KERNEL_SCAN_M2) {
+        switch (p.io_dt) {
+            case kF32: return launch_m2_io<float>(p, s);
+            case kF16: return launch_m2_io<__half>(p, s);
+            case kBF16: return launch_m2_io<__nv_bfloat16>(p, s);
+            default: return cudaErrorInvalidValue;
+        }
+    }
+    const int64_t rows = p.Bn * p.H * p.P;
+    const unsigned grid = (unsigned)((rows + 3) / 4);
+    switch (p.io_dt) {
+        case kF32: scan_m2_generic_kernel<float><<<grid, 128, 0, s>>>(p); break;
+        case kF16: scan_m2_generic_kernel<__half><<<grid, 128, 0, s>>>(p); break;
+        case kBF16: scan_m2_generic_kernel<__nv_bfloat16><<<grid, 128, 0, s>>>(p); break;
+        default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace ssm

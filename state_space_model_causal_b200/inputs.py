@@ -175,6 +175,40 @@ def prefill_2p8b(seed=0, Bt=4, L=2048, D=5120, N=16, W=4) -> ScanInputs:
 # --------------------------------------------------------------------------
 # decode (single-token state update)
 # --------------------------------------------------------------------------
+# prefill (Mamba-2 layout)
+# --------------------------------------------------------------------------
+@dataclasses.dataclass
+class ScanM2Inputs:
+    x: np.ndarray            # (B, H, P, L)
+    dt: np.ndarray           # (B, H, L)
+    A: np.ndarray            # (H,) fp32 values
+    B: np.ndarray            # (B, G, N, L)
+    C: np.ndarray            # (B, G, N, L)
+    D: Optional[np.ndarray]  # (H,)
+    z: Optional[np.ndarray]  # (B, H, P, L)
+    dt_bias: Optional[np.ndarray]  # (H,)
+    h0: Optional[np.ndarray]       # (B, H, P, N) fp32 values
+    io: str = "f32"
+
+
+def scan_m2_inputs(Bt, H, P, N, L, *, G=1, io="f32", seed=0, tag="scan_m2", with_z=True,
+                   with_D=True, with_dt_bias=True, h0=False) -> ScanM2Inputs:
+    """Seeded Mamba-2-layout prefill inputs, distributions of the Mamba-2 SSU
+    configs: x, z, B, C ~ N(0,1); dt ~ U(-4,-1); A = -U(1,16) per head; D = 1."""
+    t = (seed, tag)
+    x = round_to(normal((Bt, H, P, L), *t, "x"), io)
+    dt = round_to(uniform((Bt, H, L), -4.0, -1.0, *t, "dt"), io)
+    A = round_to(-uniform((H,), 1.0, 16.0, *t, "A"), "f32")
+    Bm = round_to(normal((Bt, G, N, L), *t, "B"), io)
+    Cm = round_to(normal((Bt, G, N, L), *t, "C"), io)
+    Dv = np.ones(H) if with_D else None
+    z = round_to(normal((Bt, H, P, L), *t, "z"), io) if with_z else None
+    db = round_to(dt_bias_draw((H,), *t, "dt_bias"), "f32") if with_dt_bias else None
+    hh = round_to(normal((Bt, H, P, N), *t, "h0"), "f32") if h0 else None
+    return ScanM2Inputs(x, dt, A, Bm, Cm, Dv, z, db, hh, io)
+
+
+# --------------------------------------------------------------------------
 @dataclasses.dataclass
 class SsuInputs:
     state: np.ndarray        # Mamba-1: (B, D, N); Mamba-2: (B, H, P, N)

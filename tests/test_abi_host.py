@@ -371,3 +371,74 @@ def test_binding_rejects_cpu_tensors():
     x = torch.zeros(1, 2, 3)
     with pytest.raises(ValueError, match="CUDA tensors only"):
         bd.describe(x)
+
+
+# ------------------------------------------------- Mamba-2-layout prefill --
+def scan_m2_args(mem, Bn=8, H=80, P=64, N=128, L=2048, G=1, io=F16, time_major=True, **over):
+    """x (B, H, P, L) as the view of (B, L, H, P) storage when time_major."""
+    a = bd.ScanArgs()
+    a.struct_size = ctypes.sizeof(bd.ScanArgs)
+    a.flags = bd.SSM_FLAG_DRY_RUN
+    if time_major:
+        a.x = mem(io, (Bn, H, P, L), (L * H * P, P, 1, H * P))
+        a.z = mem(io, (Bn, H, P, L), (L * H * P, P, 1, H * P))
+        a.out = mem(io, (Bn, H, P, L), (L * H * P, P, 1, H * P))
+        a.dt = mem(io, (Bn, H, L), (L * H, 1, H))
+        a.B = mem(io, (Bn, G, N, L), (L * G * N, N, 1, G * N))
+        a.C = mem(io, (Bn, G, N, L), (L * G * N, N, 1, G * N))
+    else:
+        a.x = mem(io, (Bn, H, P, L))
+        a.z = mem(io, (Bn, H, P, L))
+        a.out = mem(io, (Bn, H, P, L))
+        a.dt = mem(io, (Bn, H, L))
+        a.B = mem(io, (Bn, G, N, L))
+        a.C = mem(io, (Bn, G, N, L))
+    a.A = mem(F32, (H,))
+    a.D = mem(F32, (H,))
+    a.dt_bias = mem(F32, (H,))
+    a.dt_softplus = 1
+    a.ssm_state = mem(F32, (Bn, H, P, N))
+    for k, v in over.items():
+        setattr(a, k, v)
+    return a
+
+
+def test_m2_prefill_plan_fast_kernel(lib):
+    st, info = call(lib, "ssm_selective_scan_fwd", scan_m2_args(FakeMem()))
+    assert st == OK and bd.KERNELS[info.kernel] == "scan_m2"
+    # one CTA of 128 threads per (batch, head): 64 headdim rows x 128 state entries
+    assert info.block == 128 and info.rows_per_item == 64 and info.grid == 8 * 80
+    assert 0 < info.smem_bytes <= 227 * 1024
+    st, info = call(lib, "ssm_selective_scan_fwd", scan_m2_args(FakeMem(), H=32, P=128, N=256, io=BF16))
+    assert st == OK and bd.KERNELS[info.kernel] == "scan_m2"
+    assert info.rows_per_item == 32 and info.grid == 8 * 32 * 4 and info.smem_bytes <= 227 * 1024
+
+
+@pytest.mark.parametrize("over,why", [
+    (dict(time_major=False), "time-last rows"),
+    (dict(N=96), "dstate not 64/128/256"),
+    (dict(P=12), "headdim not a multiple of 8"),
+])
+def test_m2_prefill_plan_generic_kernel(lib, over, why):
+    st, info = call(lib, "ssm_selective_scan_fwd", scan_m2_args(FakeMem(), **over))
+    assert st == OK and bd.KERNELS[info.kernel] == "scan_m2_generic", why
+
+
+def test_m2_prefill_errors(lib):
+    mem = FakeMem()
+    a = scan_m2_args(mem)
+    a.conv_weight = mem(F32, (80 * 64, 4))
+    assert call(lib, "ssm_selective_scan_fwd", a)[0] == EUNSUP  # conv is its own call
+    assert call(lib, "ssm_selective_scan_fwd", scan_m2_args(mem, A=mem(F32, (80, 128))))[0] == ESHAPE
+    assert call(lib, "ssm_selective_scan_fwd", scan_m2_args(mem, G=3))[0] == ESHAPE  # H % G
+    assert call(lib, "ssm_selective_scan_fwd", scan_m2_args(mem, N=300))[0] == EUNSUP
+    assert call(lib, "ssm_selective_scan_fwd", scan_m2_args(mem, D=mem(F32, (64,))))[0] == ESHAPE
+    assert call(lib, "ssm_selective_scan_fwd", scan_m2_args(mem, z=mem(F32, (8, 80, 64, 2048))))[0] == EDTYPE
+    assert call(lib, "ssm_selective_scan_fwd",
+                scan_m2_args(mem, ssm_state=mem(F16, (8, 80, 64, 128))))[0] == EDTYPE
+    a = scan_m2_args(mem)
+    a.out = a.x
+    assert call(lib, "ssm_selective_scan_fwd", a)[0] == EALIAS
+    a = scan_m2_args(mem, L=0)
+    st, info = call(lib, "ssm_selective_scan_fwd", a)
+    assert st == OK and bd.KERNELS[info.kernel] == "none"
