@@ -324,7 +324,7 @@ ssm_status scan_m2_impl(const ssm_scan_args* a, cudaStream_t stream) {
         const int64_t blocks = (P + rpc - 1) / rpc;
         if (blocks * H * Bn > INT32_MAX) return SSM_ERR_UNSUPPORTED;
         grid = (int)(blocks * H * Bn);
-        block = 128;
+        block = scan_m2_threads();
         smem = scan_m2_smem_bytes(io, N);
         items = blocks * H * Bn;
     } else {

@@ -127,6 +127,7 @@ int scan_vec_channels_per_cta();
 cudaError_t launch_scan_vec(const ScanProblem& p, int sw_pairs, cudaStream_t s);
 cudaError_t launch_conv1d(const Conv1dProblem& p, const Conv1dPlan& plan, cudaStream_t s);
 int scan_m2_rows_per_cta(int64_t N);
+int scan_m2_threads();
 int scan_m2_smem_bytes(int io_dt, int64_t N);
 cudaError_t launch_scan_m2(const ScanM2Problem& p, int kernel, cudaStream_t s);
 

@@ -17,11 +17,14 @@
 // multiple of 8; dstate 64, 128 or 256, contiguous in B, C; 16-byte aligned
 // rows):
 //   * a CTA is 128 threads on one (b, h) and a block of RPC = 512 / NG
-//     headdim rows, NG = dstate / 16.  Thread (pg, ng) owns rows 4pg..4pg+3 of
+//     headdim rows, NG = dstate / 16 (thread count, chunk length and the
+//     register budget are build-time parameters; the defaults measured best).  Thread (pg, ng) owns rows 4pg..4pg+3 of
 //     the block and state entries 16ng..16ng+15: a 4 x 16 register tile of the
-//     state, updated with packed f32x2 operations across n;
-//   * 16-step chunks of x, z, B, C are staged by 16-byte cp.async copies into a
-//     double buffer while the previous chunk is scanned; dt is prefetched into a
+//     state, updated with packed f32x2 operations across n, one 16-byte piece
+//     of B and C at a time so that the tile fits with room to schedule;
+//   * 16-step chunks of x, z, B, C are staged by 16-byte cp.async copies while
+//     the previous chunk is scanned (x, z double-buffered for the epilogue;
+//     B, C single-buffered, refilled once widened); dt is prefetched into a
 //     register one chunk ahead;
 //   * per chunk the CTA computes once (delta, decay) per step, delta * x per
 //     (step, row) and the fp32 B, C rows (16-byte pieces XOR-swizzled so the NG
@@ -37,23 +40,33 @@
 namespace ssm {
 namespace {
 
-constexpr int kM2Threads = 128;
-constexpr int kM2T = 16;  // steps per chunk
+#ifndef SSM_M2_THREADS
+#define SSM_M2_THREADS 128
+#endif
+#ifndef SSM_M2_STEPS
+#define SSM_M2_STEPS 16
+#endif
+#ifndef SSM_M2_MIN_CTAS
+#define SSM_M2_MIN_CTAS 3
+#endif
+constexpr int kM2Threads = SSM_M2_THREADS;  // threads per CTA
+constexpr int kM2T = SSM_M2_STEPS;          // steps per chunk
+constexpr int kM2MinCtas = SSM_M2_MIN_CTAS; // register budget: CTAs resident per SM
 
 // (16-byte piece u of a B/C row) -> stored piece: the pieces a quarter-warp's
 // NG groups read at once (u = 4 ng + k) land in distinct banks
 __device__ __forceinline__ int m2_swz(int u) { return u ^ ((u >> 3) & 7); }
 
 template <typename IoT, int NG> struct M2Smem {
-    static constexpr int RPC = 512 / NG;  // headdim rows per CTA
+    static constexpr int RPC = 4 * kM2Threads / NG;  // headdim rows per CTA
     static constexpr int N = 16 * NG;
-    struct Raw {
+    struct RawXZ {
         IoT x[kM2T][RPC];
         IoT z[kM2T][RPC];
-        IoT B[kM2T][N];
-        IoT C[kM2T][N];
     };
-    Raw raw[2];
+    RawXZ raw[2];      // x, z: read again by the epilogue, so double-buffered
+    IoT rawB[kM2T][N];  // B, C: widened right after arrival, single buffer
+    IoT rawC[kM2T][N];
     float2 dd[kM2T];           // (decay, delta) per step
     float dx[kM2T][RPC];       // delta * x
     float B[kM2T][N];          // swizzled fp32 rows
@@ -68,7 +81,7 @@ __device__ __forceinline__ void cp_async16_m2(void* dst, const void* src, bool v
 }
 
 template <typename IoT, int NG>
-__global__ void __launch_bounds__(kM2Threads) scan_m2_kernel(const ScanM2Problem p) {
+__global__ void __launch_bounds__(kM2Threads, kM2MinCtas) scan_m2_kernel(const ScanM2Problem p) {
     using S = M2Smem<IoT, NG>;
     constexpr int RPC = S::RPC;
     constexpr int N = S::N;
@@ -122,12 +135,11 @@ __global__ void __launch_bounds__(kM2Threads) scan_m2_kernel(const ScanM2Problem
     for (int k = 0; k < 4; ++k) boff[k] = m2_swz(4 * ng + k) * 4;
 
     const int nchunks = (int)((L + kM2T - 1) / kM2T);
-    auto fetch = [&](int ci) {
-        typename S::Raw& rw = sm.raw[ci & 1];
+    // x, z of chunk ci: kM2T x RPC elements each, into raw[ci & 1]
+    auto fetch_xz = [&](int ci) {
+        typename S::RawXZ& rw = sm.raw[ci & 1];
         const int64_t t0 = (int64_t)ci * kM2T;
-        // x, z: kM2T x RPC elements; B, C: kM2T x N
         constexpr int XC = kM2T * RPC / E;
-        constexpr int BC = kM2T * N / E;
         for (int i = tid; i < XC; i += kM2Threads) {
             const int t = i / (RPC / E), e = (i % (RPC / E)) * E;
             const bool v = t0 + t < L && e < rows;
@@ -135,22 +147,29 @@ __global__ void __launch_bounds__(kM2Threads) scan_m2_kernel(const ScanM2Problem
             cp_async16_m2(&rw.x[t][e], xg + ts * p.x_t + (v ? e : 0), v);
             cp_async16_m2(&rw.z[t][e], (zg ? zg : xg) + ts * (zg ? p.z_t : p.x_t) + (v ? e : 0), v && zg);
         }
+    };
+    // B, C of chunk ci: kM2T x N elements each
+    auto fetch_bc = [&](int ci) {
+        const int64_t t0 = (int64_t)ci * kM2T;
+        constexpr int BC = kM2T * N / E;
         for (int i = tid; i < BC; i += kM2Threads) {
             const int t = i / (N / E), e = (i % (N / E)) * E;
             const bool v = t0 + t < L;
             const int64_t ts = v ? t0 + t : 0;
-            cp_async16_m2(&rw.B[t][e], Bg + ts * p.B_t + e, v);
-            cp_async16_m2(&rw.C[t][e], Cg + ts * p.C_t + e, v);
+            cp_async16_m2(&sm.rawB[t][e], Bg + ts * p.B_t + e, v);
+            cp_async16_m2(&sm.rawC[t][e], Cg + ts * p.C_t + e, v);
         }
-        asm volatile("cp.async.commit_group;" ::: "memory");
     };
+    auto commit = []() { asm volatile("cp.async.commit_group;" ::: "memory"); };
     // dt of the next chunk, one step per thread of the first warp
     float dt_next = 0.0f;
     auto load_dt = [&](int ci) {
         const int64_t t = (int64_t)ci * kM2T + tid;
         dt_next = (tid < kM2T && t < L) ? to_f(dtg[t * p.dt_t]) : 0.0f;
     };
-    fetch(0);
+    fetch_xz(0);
+    fetch_bc(0);
+    commit();
     load_dt(0);
 
     for (int ci = 0; ci < nchunks; ++ci) {
@@ -169,10 +188,10 @@ __global__ void __launch_bounds__(kM2Threads) scan_m2_kernel(const ScanM2Problem
         }
         __syncthreads();  // dd and this chunk's staged rows visible to all
         if (ci + 1 < nchunks) {
-            fetch(ci + 1);
+            fetch_xz(ci + 1);
             load_dt(ci + 1);
         }
-        const typename S::Raw& rw = sm.raw[ci & 1];
+        const typename S::RawXZ& rw = sm.raw[ci & 1];
         // ---- widen: delta * x per (step, row), fp32 B / C rows (swizzled)
         for (int i = tid; i < kM2T * RPC / 8; i += kM2Threads) {
             const int t = i / (RPC / 8), e = (i % (RPC / 8)) * 8;
@@ -192,14 +211,17 @@ __global__ void __launch_bounds__(kM2Threads) scan_m2_kernel(const ScanM2Problem
             float bv[4], cv[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-                bv[k] = to_f(rw.B[t][4 * u + k]);
-                cv[k] = to_f(rw.C[t][4 * u + k]);
+                bv[k] = to_f(sm.rawB[t][4 * u + k]);
+                cv[k] = to_f(sm.rawC[t][4 * u + k]);
             }
             const int su = m2_swz(u) * 4;
             *reinterpret_cast<float4*>(&sm.B[t][su]) = make_float4(bv[0], bv[1], bv[2], bv[3]);
             *reinterpret_cast<float4*>(&sm.C[t][su]) = make_float4(cv[0], cv[1], cv[2], cv[3]);
         }
         __syncthreads();
+        // the raw B/C rows are widened: the next chunk's may land now
+        if (ci + 1 < nchunks) fetch_bc(ci + 1);
+        commit();
 
         // ---- scan: 4 groups of 4 steps
 #pragma unroll 1
@@ -211,28 +233,29 @@ __global__ void __launch_bounds__(kM2Threads) scan_m2_kernel(const ScanM2Problem
                 const float decay = sm.dd[t].x;
                 const u64 dA2 = pk(decay, decay);
                 const float4 dx4 = *reinterpret_cast<const float4*>(&sm.dx[t][4 * pg]);
-                const float dxr[4] = {dx4.x, dx4.y, dx4.z, dx4.w};
-                u64 b2[8], c2[8];
+                const u64 dx2[4] = {pk(dx4.x, dx4.x), pk(dx4.y, dx4.y), pk(dx4.z, dx4.z), pk(dx4.w, dx4.w)};
+                u64 y2[4];
+                // one 16-byte piece of B and C at a time (short live ranges)
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     const float4 bq = *reinterpret_cast<const float4*>(&sm.B[t][boff[q]]);
                     const float4 cq = *reinterpret_cast<const float4*>(&sm.C[t][boff[q]]);
-                    b2[2 * q] = pk(bq.x, bq.y);
-                    b2[2 * q + 1] = pk(bq.z, bq.w);
-                    c2[2 * q] = pk(cq.x, cq.y);
-                    c2[2 * q + 1] = pk(cq.z, cq.w);
+                    const u64 b2[2] = {pk(bq.x, bq.y), pk(bq.z, bq.w)};
+                    const u64 c2[2] = {pk(cq.x, cq.y), pk(cq.z, cq.w)};
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+#pragma unroll
+                        for (int jj = 0; jj < 2; ++jj) {
+                            const int j = 2 * q + jj;
+                            hs[r][j] = ffma2(dA2, hs[r][j], fmul2(dx2[r], b2[jj]));
+                            y2[r] = j == 0 ? fmul2(c2[jj], hs[r][j]) : ffma2(c2[jj], hs[r][j], y2[r]);
+                        }
+                    }
                 }
 #pragma unroll
                 for (int r = 0; r < 4; ++r) {
-                    const u64 dx2 = pk(dxr[r], dxr[r]);
-                    u64 y2 = 0;
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        hs[r][j] = ffma2(dA2, hs[r][j], fmul2(dx2, b2[j]));
-                        y2 = j == 0 ? fmul2(c2[j], hs[r][j]) : ffma2(c2[j], hs[r][j], y2);
-                    }
                     float lo, hi;
-                    upk(y2, lo, hi);
+                    upk(y2[r], lo, hi);
                     v[4 * r + k] = lo + hi;
                 }
             }
@@ -389,7 +412,10 @@ cudaError_t launch_m2_io(const ScanM2Problem& p, cudaStream_t s) {
 }  // namespace
 
 // the fast kernel's dstate values (NG = 4, 8, 16): 0 for any other dstate
-int scan_m2_rows_per_cta(int64_t N) { return N == 64 || N == 128 || N == 256 ? (int)(512 / (N / 16)) : 0; }
+int scan_m2_rows_per_cta(int64_t N) {
+    return N == 64 || N == 128 || N == 256 ? (int)(4 * kM2Threads / (N / 16)) : 0;
+}
+int scan_m2_threads() { return kM2Threads; }
 
 int scan_m2_smem_bytes(int io_dt, int64_t N) {
     auto pick = [&](auto tag) -> int {
@@ -418,7 +444,7 @@ cudaError_t launch_scan_m2(const ScanM2Problem& p, int kernel, cudaStream_t s) {
         }
     }
     const int64_t rows = p.Bn * p.H * p.P;
-    const unsigned grid = (unsigned)((rows + 3) / 4);
+    const unsigned grid = (unsigned)((rows + 3) / 4);  // generic kernel: 4 warps of 32
     switch (p.io_dt) {
         case kF32: scan_m2_generic_kernel<float><<<grid, 128, 0, s>>>(p); break;
         case kF16: scan_m2_generic_kernel<__half><<<grid, 128, 0, s>>>(p); break;
