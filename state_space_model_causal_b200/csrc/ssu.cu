@@ -495,6 +495,7 @@ __global__ void __launch_bounds__(32 * kRowWarps, kRowMinBlocks) ssu_row_tma_ker
     constexpr int NS = CPT * VE;  // d_state
     extern __shared__ __align__(128) unsigned char tma_stage[];
     __shared__ __align__(8) uint64_t full[kRowWarps][kWarpStages];
+    __shared__ __align__(16) float bcw[kRowWarps][2 * NS];  // the item's B, C widened once
 
     const unsigned lane = threadIdx.x & 31u;
     const unsigned warp = threadIdx.x >> 5;
@@ -615,6 +616,13 @@ __global__ void __launch_bounds__(32 * kRowWarps, kRowMinBlocks) ssu_row_tma_ker
             }
             return;
         }
+        {
+            // widen the item's B and C once for the warp (every lane reads all of them)
+            const unsigned char* st0 = ring + stage * stage_bytes;
+            for (int i = (int)lane; i < 2 * NS; i += 32)
+                bcw[warp][i] = to_f(reinterpret_cast<const IoT*>(st0 + (i < NS ? off_B : off_C))[i < NS ? i : i - NS]);
+            __syncwarp();
+        }
         if (rok) {
             unsigned char* st = ring + stage * stage_bytes;
             const unsigned cl = lane;
@@ -644,41 +652,38 @@ __global__ void __launch_bounds__(32 * kRowWarps, kRowMinBlocks) ssu_row_tma_ker
             const float dl2 = dl * kLog2e;
             const float du = dl * u;
             unsigned char* srow = st + cl * row_bytes;
-            float acc = 0.0f;
+            const float* bw = bcw[warp];
+            const u64 dl2d = pk(dl2, dl2), dud = pk(du, du);
+            u64 acc2 = 0;
 #pragma unroll
             for (int j = 0; j < CPT; ++j) {
                 const unsigned cj = (j + rot) & (CPT - 1u);
-                float sv[VE], bv[VE], cv[VE];
+                float sv[VE];
                 V::unpack(*reinterpret_cast<const uint4*>(srow + cj * 16), sv);
-                // B/C of this chunk (VE I/O values: 8 or 16 bytes, broadcast)
-                if constexpr (VE * sizeof(IoT) == 16) {
-                    Vec16<IoT>::unpack(*reinterpret_cast<const uint4*>(st + off_B + cj * VE * sizeof(IoT)), bv);
-                    Vec16<IoT>::unpack(*reinterpret_cast<const uint4*>(st + off_C + cj * VE * sizeof(IoT)), cv);
-                } else {
-                    float t8[8];
-                    const uint2 rbv = *reinterpret_cast<const uint2*>(st + off_B + cj * VE * sizeof(IoT));
-                    const uint2 rcv = *reinterpret_cast<const uint2*>(st + off_C + cj * VE * sizeof(IoT));
-                    Vec16<IoT>::unpack(make_uint4(rbv.x, rbv.y, 0u, 0u), t8);
-#pragma unroll
-                    for (int e = 0; e < VE; ++e) bv[e] = t8[e];
-                    Vec16<IoT>::unpack(make_uint4(rcv.x, rcv.y, 0u, 0u), t8);
-#pragma unroll
-                    for (int e = 0; e < VE; ++e) cv[e] = t8[e];
-                }
+                // packed pairs: decay exp on the SFU per element, the rest f32x2
 #pragma unroll
                 for (int e = 0; e < VE; e += 4) {
                     const float4 a = a4[(j * VE + e) / 4];
-                    const float av[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        sv[e + i] = fmaf(ex2_approx(dl2 * av[i]), sv[e + i], du * bv[e + i]);
-                        acc = fmaf(cv[e + i], sv[e + i], acc);
-                    }
+                    const float4 b4 = *reinterpret_cast<const float4*>(bw + cj * VE + e);
+                    const float4 c4 = *reinterpret_cast<const float4*>(bw + NS + cj * VE + e);
+                    float e0, e1, e2, e3;
+                    upk(fmul2(dl2d, pk(a.x, a.y)), e0, e1);
+                    upk(fmul2(dl2d, pk(a.z, a.w)), e2, e3);
+                    const u64 s01 = ffma2(pk(ex2_approx(e0), ex2_approx(e1)), pk(sv[e], sv[e + 1]),
+                                          fmul2(dud, pk(b4.x, b4.y)));
+                    const u64 s23 = ffma2(pk(ex2_approx(e2), ex2_approx(e3)), pk(sv[e + 2], sv[e + 3]),
+                                          fmul2(dud, pk(b4.z, b4.w)));
+                    acc2 = ffma2(pk(c4.x, c4.y), s01, acc2);
+                    acc2 = ffma2(pk(c4.z, c4.w), s23, acc2);
+                    upk(s01, sv[e], sv[e + 1]);
+                    upk(s23, sv[e + 2], sv[e + 3]);
                 }
                 // new state back into the stage, in place; bulk-stored below
                 *reinterpret_cast<uint4*>(srow + cj * 16) = V::pack(sv);
             }
-            float y = fmaf(dskip, u, acc);
+            float acc_lo, acc_hi;
+            upk(acc2, acc_lo, acc_hi);
+            float y = fmaf(dskip, u, acc_lo + acc_hi);
             if (zg) y *= silu_f(to_f(reinterpret_cast<const IoT*>(st + off_z)[cl]));
             og[b * p.o_b + (int64_t)c * p.o_h] = from_f<IoT>(y);
             if constexpr (W > 0) {
