@@ -458,6 +458,24 @@ def cpu_baseline(target_s=10.0):
                       f"L=2048, fp64 sequential C on one thread, {t:.1f} s"}
 
 
+# ------------------------------------------------------- multi-rank host --
+def max_over_ranks(ms_step, pg, device):
+    """The step time of the job: the slowest rank's (every rank calls this
+    once, in the same order).  pg is torch.distributed or None."""
+    if pg is None:
+        return float(ms_step)
+    import torch
+    t = torch.tensor([float(ms_step)], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, units_per_rank, ms_step):
+    """Whole-job units per second (Gunits/s): every rank processes the same
+    fixed work (weak scaling), the job is as slow as its slowest rank."""
+    return world * units_per_rank / (ms_step * 1e-3) / 1e9
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -622,12 +640,8 @@ def main():
     torch.cuda.synchronize(dev)
     if pg:
         pg.barrier()
-    ms_step = statistics.mean(ms)
-    if pg:
-        t = torch.tensor([ms_step], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms_step = float(t.item())
-    value = world * pf.elems / (ms_step * 1e-3) / 1e9
+    ms_step = max_over_ranks(statistics.mean(ms), pg, dev)
+    value = job_throughput(world, pf.elems, ms_step)
 
     # roofline of the prefill kernel: one exp(delta*A) per element on the SFU
     sfu_peak = NUM_SMS * SFU_EX2_PER_CLK_PER_SM * sm_max * 1e6 / 1e9  # Gelem/s
