@@ -713,6 +713,16 @@ ssm_status ssu_impl(const ssm_ssu_args* a, cudaStream_t stream) {
 
     // ---- plan: streaming kernels when the state rows are 16-byte addressable
     SsuPlan plan{};
+    // bulk-copy waits give up after ~2 s of cycles.  Failure tests can shorten
+    // that and name one work item whose copies are never started, so that its
+    // wait runs out (SSM_TEST_WAIT_CYCLES, SSM_TEST_DROP_ITEM).
+    plan.wait_budget = 4000000000LL;
+    plan.drop_item = -1;
+    if (const char* e = std::getenv("SSM_TEST_WAIT_CYCLES")) {
+        const long long v = std::atoll(e);
+        if (v > 0) plan.wait_budget = v;
+    }
+    if (const char* e = std::getenv("SSM_TEST_DROP_ITEM")) plan.drop_item = std::atoll(e);
     const int es = esize(p.state_dt);
     const bool vec_rows = p.st_n == 1 && (N * es) % 16 == 0 && aligned16(p.state) &&
                           (p.st_b * es) % 16 == 0 && (p.st_h * es) % 16 == 0 &&

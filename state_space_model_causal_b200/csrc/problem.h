@@ -45,6 +45,9 @@ struct SsuPlan {
     int stages;          // bulk-copy kernel: stages in flight per CTA
     int rpt;             // bulk-copy kernel: rows per thread per item
     int sms;             // SMs of the device (persistent grids)
+    long long wait_budget;  // bulk-copy kernels: cycles before a wait gives up
+    int64_t drop_item;      // failure tests only: work item whose copies are never
+                            // started, so its wait runs out (-1: none)
 };
 
 // Fused prefill (Mamba-1 layout): x, dt, z, out (B, D, L); B, C (B, G, N, L).

@@ -224,7 +224,6 @@ __global__ void __launch_bounds__(256, 3) ssu_head_kernel(const SsuProblem p, co
 // reduce-scatter.  I/O dtype IoT is a template parameter.
 // ------------------------------------------------------------------------
 constexpr int kTmaStagesMax = 4;
-constexpr long long kWaitBudget = 4000000000LL;  // cycles before a wait gives up (~2 s)
 
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
@@ -311,6 +310,7 @@ __global__ void __launch_bounds__(256, 3) ssu_head_tma_kernel(const SsuProblem p
     // padding row completes the stage's phase without data
     auto issue = [&](unsigned k, const Pos& q) {
         uint64_t* bar = &full[k % S];
+        if ((int64_t)(i0 + k) == plan.drop_item) return;  // failure test: never completes
         const int64_t slot = slot_of(q.b);
         if (slot < 0) {
             mbar_arrive(bar);
@@ -379,12 +379,12 @@ __global__ void __launch_bounds__(256, 3) ssu_head_tma_kernel(const SsuProblem p
                 dA = ex2_approx(delta * a2);
             }
         }
-        const bool ok = mbar_wait_bounded(&full[stage], parity, kWaitBudget);
+        const bool ok = mbar_wait_bounded(&full[stage], parity, plan.wait_budget);
         if (__syncthreads_or(!ok)) {
             // give up: wait (bounded) for this CTA's copies still in flight, flag, exit
             if (tid == 0) {
                 for (unsigned kk = k; kk < min(cnt, k + S); ++kk)
-                    mbar_wait_bounded(&full[kk % S], (kk / S) & 1u, kWaitBudget);
+                    mbar_wait_bounded(&full[kk % S], (kk / S) & 1u, plan.wait_budget);
                 atomicExch(&g_ssm_device_error, 1);
             }
             return;
@@ -540,6 +540,7 @@ __global__ void __launch_bounds__(32 * kRowWarps, kRowMinBlocks) ssu_row_tma_ker
     // stage's phase without data
     auto issue = [&](unsigned k) {
         const unsigned item = i0 + k;
+        if ((int64_t)item == plan.drop_item) return;  // failure test: never completes
         const unsigned cb = item / Bn, b = item - cb * Bn;
         uint64_t* bar = &bars[k % kWarpStages];
         const int64_t slot = slot_of(b);
@@ -602,7 +603,7 @@ __global__ void __launch_bounds__(32 * kRowWarps, kRowMinBlocks) ssu_row_tma_ker
             }
         }
         const unsigned stage = k % kWarpStages;
-        const bool ok = mbar_wait_bounded(&bars[stage], (k / kWarpStages) & 1u, kWaitBudget);
+        const bool ok = mbar_wait_bounded(&bars[stage], (k / kWarpStages) & 1u, plan.wait_budget);
         if (__any_sync(0xffffffffu, !ok)) {
             // give up: wait (bounded) for this warp's copies still in flight, flag, exit
             if (lane == 0) {
@@ -610,7 +611,7 @@ __global__ void __launch_bounds__(32 * kRowWarps, kRowMinBlocks) ssu_row_tma_ker
                 // kWarpStages before the loop, one refill per later step)
                 const unsigned hi = min(cnt, k == 0 ? (unsigned)kWarpStages : k + kWarpStages - 1);
                 for (unsigned kk = k; kk < hi; ++kk)
-                    mbar_wait_bounded(&bars[kk % kWarpStages], (kk / kWarpStages) & 1u, kWaitBudget);
+                    mbar_wait_bounded(&bars[kk % kWarpStages], (kk / kWarpStages) & 1u, plan.wait_budget);
                 bulk_wait_all();
                 atomicExch(&g_ssm_device_error, 1);
             }
