@@ -442,3 +442,18 @@ def test_m2_prefill_errors(lib):
     a = scan_m2_args(mem, L=0)
     st, info = call(lib, "ssm_selective_scan_fwd", a)
     assert st == OK and bd.KERNELS[info.kernel] == "none"
+
+
+def test_plain_c_client_links_and_runs(tmp_path, lib):
+    """A C program built against include/ssm_causal.h and linked to the .so
+    (no Python, no torch types) plans a prefill and a decode and gets every
+    documented error status."""
+    import subprocess
+    src = os.path.join(ROOT, "tests", "c_abi_client.c")
+    exe = tmp_path / "c_abi_client"
+    libdir = os.path.dirname(bd.LIB_PATH)
+    subprocess.check_call(["gcc", "-std=c99", "-O1", "-I", os.path.join(ROOT, "include"), src, "-o", str(exe),
+                           "-L", libdir, "-lssm_causal", f"-Wl,-rpath,{libdir}"])
+    res = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert res.returncode == 0, res.stdout + res.stderr
+    assert "fails 0" in res.stdout
