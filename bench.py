@@ -423,7 +423,7 @@ def decode_mamba2(dev, hbm_peak, H, P, N, R, cache, io, replays=10, calls_per_gr
     return {"workload": f"mamba2-ssu: H={H} P={P} N={N} G=1, {io} io, {cache} cache",
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
                          "frac": round(gbs / hbm_peak, 4), "traffic": traffic},
-            "effective_batch": R, "batch": Bt, "heads": Hr, "us_per_call": round(us, 3),
+            "effective_batch": R, "batch": Bt, "heads": Hr, "P": P, "N": N, "us_per_call": round(us, 3),
             "us_median": round(med, 3), "bytes_per_call": nbytes, "GBps": round(gbs, 1),
             "frac_of_hbm_peak": round(gbs / hbm_peak, 4),
             "l2": f"{nslab} state slabs rotated ({nslab * state_bytes / 2**20:.0f} MiB)"}
@@ -444,6 +444,48 @@ def oracle_prefill_sample(channels, seed=0):
                 conv_weight=s.conv_weight, conv_bias=s.conv_bias)
     dt = time.perf_counter() - t0
     return dt, s.x.shape[0] * s.x.shape[1] * s.x.shape[2] * s.A.shape[1]
+
+
+def oracle_beside(entry, kind, rows=None):
+    """Time the fp64 oracle (one host thread) on a bounded sample of a sub-line's
+    workload and express it in that line's unit, so that every measured kernel
+    has the oracle timed beside it.  kind: "m1_decode", "m2_decode" or
+    "m2_prefill"; rows overrides the sample size (tests)."""
+    import oracle
+    from state_space_model_causal_b200 import inputs as gen
+    if kind == "m1_decode":
+        Bt = rows or 64
+        s = gen.ssu_mamba1_inputs(Bt, 5120, 16, W=4, io="f16", state="f32", seed=0, tag="oracle_beside")
+        t0 = time.perf_counter()
+        oracle.ssu(s.state[:, :, None, :], s.x[:, :, None], s.dt[:, :, None], s.A[:, None, :], s.B, s.C,
+                   D=s.D[:, None], z=s.z[:, :, None], dt_bias=s.dt_bias[:, None],
+                   conv_weight=s.conv_weight, conv_bias=s.conv_bias, conv_state=s.conv_state)
+        dt = time.perf_counter() - t0
+        per_row = entry["bytes_per_call"] / (245 * 5120)
+        value, unit = Bt * 5120 * per_row / dt / 1e9, "GB/s"
+        sample = f"{Bt} of the 245 batch rows (all 5120 channels), one decode step"
+    elif kind == "m2_decode":
+        H, P, N = entry["heads"], entry["P"], entry["N"]
+        Bt = rows or 8
+        s = gen.ssu_mamba2_inputs(Bt, H, P, N, io="f32", state="f32", seed=0, tag="oracle_beside")
+        t0 = time.perf_counter()
+        oracle.ssu_mamba2(s.state, s.x, s.dt, s.A, s.B, s.C, D=s.D, dt_bias=s.dt_bias)
+        dt = time.perf_counter() - t0
+        per_b = entry["bytes_per_call"] / entry["batch"]
+        value, unit = Bt * per_b / dt / 1e9, "GB/s"
+        sample = f"{Bt} batch rows x {H} heads, one decode step"
+    elif kind == "m2_prefill":
+        heads = rows or 4
+        s = gen.scan_m2_inputs(1, heads, 64, 128, 2048, io="f16", seed=0, tag="oracle_beside")
+        t0 = time.perf_counter()
+        oracle.scan_mamba2(s.x, s.dt, s.A, s.B, s.C, D=s.D, z=s.z, dt_bias=s.dt_bias)
+        dt = time.perf_counter() - t0
+        value, unit = heads * 64 * 128 * 2048 / dt / 1e9, "Gelem/s"
+        sample = f"{heads} of the 640 (b, h) heads, full L=2048"
+    else:
+        raise ValueError(kind)
+    return {"value": round(value, 6), "unit": unit, "cores": 1, "kind": "oracle",
+            "sample": f"{sample}; fp64 sequential C on one host thread, {dt:.2f} s"}
 
 
 def cpu_baseline(target_s=10.0):
@@ -672,6 +714,11 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         cpu = cpu_baseline()
+        # the oracle timed beside every other measured kernel, in its line's unit
+        if prefill_m2:
+            prefill_m2["oracle"] = oracle_beside(prefill_m2, "m2_prefill")
+        for i, entry in enumerate(decode):
+            entry["oracle"] = oracle_beside(entry, "m1_decode" if i == 0 else "m2_decode")
 
     if pg:
         pg.barrier()

@@ -68,3 +68,18 @@ def test_reference_arm_runs_on_rank_zero_only():
                           "--warmup", "3"], capture_output=True, text=True, timeout=120, cwd=ROOT, env=env)
     assert res.returncode == 0, res.stderr[-2000:]
     assert res.stdout.strip() == ""
+
+
+@pytest.mark.parametrize("kind,entry,rows", [
+    ("m1_decode", {"bytes_per_call": 206208320}, 1),
+    ("m2_decode", {"bytes_per_call": 4331209248, "batch": 1639, "heads": 80, "P": 64, "N": 128}, 1),
+    ("m2_prefill", {}, 1),
+])
+def test_oracle_beside_each_sub_line_runs_on_the_host(kind, entry, rows):
+    """The oracle timings attached to the bench's sub-lines run on the host
+    (no GPU) and report a positive rate in the line's unit."""
+    sys.path.insert(0, ROOT)
+    import bench
+    r = bench.oracle_beside(entry, kind, rows=rows)
+    assert r["value"] > 0 and r["kind"] == "oracle" and r["cores"] == 1
+    assert r["unit"] == ("Gelem/s" if kind == "m2_prefill" else "GB/s")
