@@ -718,11 +718,19 @@ ssm_status ssu_impl(const ssm_ssu_args* a, cudaStream_t stream) {
     // wait runs out (SSM_TEST_WAIT_CYCLES, SSM_TEST_DROP_ITEM).
     plan.wait_budget = 4000000000LL;
     plan.drop_item = -1;
-    if (const char* e = std::getenv("SSM_TEST_WAIT_CYCLES")) {
-        const long long v = std::atoll(e);
-        if (v > 0) plan.wait_budget = v;
-    }
-    if (const char* e = std::getenv("SSM_TEST_DROP_ITEM")) plan.drop_item = std::atoll(e);
+    // only a whole decimal number counts; anything else leaves the defaults
+    auto env_int = [](const char* name, long long* v) {
+        const char* e = std::getenv(name);
+        if (!e || !*e) return false;
+        char* end = nullptr;
+        const long long x = std::strtoll(e, &end, 10);
+        if (!end || *end != '\0') return false;
+        *v = x;
+        return true;
+    };
+    long long v = 0;
+    if (env_int("SSM_TEST_WAIT_CYCLES", &v) && v > 0) plan.wait_budget = v;
+    if (env_int("SSM_TEST_DROP_ITEM", &v) && v >= 0) plan.drop_item = v;
     const int es = esize(p.state_dt);
     const bool vec_rows = p.st_n == 1 && (N * es) % 16 == 0 && aligned16(p.state) &&
                           (p.st_b * es) % 16 == 0 && (p.st_h * es) % 16 == 0 &&
