@@ -454,7 +454,7 @@ def oracle_beside(entry, kind, rows=None):
     import oracle
     from state_space_model_causal_b200 import inputs as gen
     if kind == "m1_decode":
-        Bt = rows or 64
+        Bt = rows or 245
         s = gen.ssu_mamba1_inputs(Bt, 5120, 16, W=4, io="f16", state="f32", seed=0, tag="oracle_beside")
         t0 = time.perf_counter()
         oracle.ssu(s.state[:, :, None, :], s.x[:, :, None], s.dt[:, :, None], s.A[:, None, :], s.B, s.C,
@@ -466,7 +466,7 @@ def oracle_beside(entry, kind, rows=None):
         sample = f"{Bt} of the 245 batch rows (all 5120 channels), one decode step"
     elif kind == "m2_decode":
         H, P, N = entry["heads"], entry["P"], entry["N"]
-        Bt = rows or 8
+        Bt = rows or 64
         s = gen.ssu_mamba2_inputs(Bt, H, P, N, io="f32", state="f32", seed=0, tag="oracle_beside")
         t0 = time.perf_counter()
         oracle.ssu_mamba2(s.state, s.x, s.dt, s.A, s.B, s.C, D=s.D, dt_bias=s.dt_bias)
@@ -475,7 +475,7 @@ def oracle_beside(entry, kind, rows=None):
         value, unit = Bt * per_b / dt / 1e9, "GB/s"
         sample = f"{Bt} batch rows x {H} heads, one decode step"
     elif kind == "m2_prefill":
-        heads = rows or 4
+        heads = rows or 8
         s = gen.scan_m2_inputs(1, heads, 64, 128, 2048, io="f16", seed=0, tag="oracle_beside")
         t0 = time.perf_counter()
         oracle.scan_mamba2(s.x, s.dt, s.A, s.B, s.C, D=s.D, z=s.z, dt_bias=s.dt_bias)
