@@ -47,10 +47,10 @@
  * never synchronises the stream (except ssm_device_error) and holds no mutable
  * host-side state: every entry point is reentrant.  The only state it keeps is
  * on the device, one error word that the kernels set when they give up a bounded
- * wait (see ssm_device_error).  Environment variables SSM_SCAN_SW_PAIRS (a
- * prefill tuning knob), SSM_TEST_DROP_ITEM and SSM_TEST_WAIT_CYCLES (failure
- * tests of the bounded waits) are read at each call and are never needed in
- * normal use.  Work is enqueued on `stream` (a cudaStream_t; NULL is
+ * wait (see ssm_device_error).  Environment variables SSM_SCAN_SW_PAIRS,
+ * SSM_SSU_ROWS_PER_ITEM, SSM_SSU_CTAS_PER_SM (tuning sweeps), SSM_TEST_DROP_ITEM
+ * and SSM_TEST_WAIT_CYCLES (failure tests of the bounded waits) are read at
+ * each call and are never needed in normal use.  Work is enqueued on `stream` (a cudaStream_t; NULL is
  * the legacy default stream) and runs asynchronously.
  *
  * Errors.  Every argument is checked before anything is launched; on an error

@@ -124,6 +124,18 @@ int64_t sd(const ssm_tensor& t, int i) { return t.shape[i] == 1 ? 0 : t.stride[i
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// An integer environment switch: only a whole decimal number counts; anything
+// else (unset, empty, trailing characters) leaves the caller's default.
+bool env_int(const char* name, long long* v) {
+    const char* e = std::getenv(name);
+    if (!e || !*e) return false;
+    char* end = nullptr;
+    const long long x = std::strtoll(e, &end, 10);
+    if (!end || *end != '\0') return false;
+    *v = x;
+    return true;
+}
+
 int sm_count(bool dry_run) {
     if (dry_run) return kDefaultSms;
     int dev = 0, n = 0;
@@ -718,16 +730,6 @@ ssm_status ssu_impl(const ssm_ssu_args* a, cudaStream_t stream) {
     // wait runs out (SSM_TEST_WAIT_CYCLES, SSM_TEST_DROP_ITEM).
     plan.wait_budget = 4000000000LL;
     plan.drop_item = -1;
-    // only a whole decimal number counts; anything else leaves the defaults
-    auto env_int = [](const char* name, long long* v) {
-        const char* e = std::getenv(name);
-        if (!e || !*e) return false;
-        char* end = nullptr;
-        const long long x = std::strtoll(e, &end, 10);
-        if (!end || *end != '\0') return false;
-        *v = x;
-        return true;
-    };
     long long v = 0;
     if (env_int("SSM_TEST_WAIT_CYCLES", &v) && v > 0) plan.wait_budget = v;
     if (env_int("SSM_TEST_DROP_ITEM", &v) && v >= 0) plan.drop_item = v;
@@ -771,9 +773,17 @@ ssm_status ssu_impl(const ssm_ssu_args* a, cudaStream_t stream) {
             const int64_t xalign = 16 / es_io;  // rows per item keep x 16-byte aligned
             int64_t rb = std::min<int64_t>(rpt * rows_per_pass, P);
             rb = std::max<int64_t>(xalign, rb / xalign * xalign);
-            const int64_t ctas_tma = (int64_t)sms * 3;
-            while (rb > xalign && Bn * H * ((P + rb - 1) / rb) < 2 * ctas_tma)
+            // the largest items measured fastest at every effective batch
+            // (per-item work dominates; smaller items only add items), so
+            // items are split only while there are fewer of them than SMs
+            while (rb > xalign && Bn * H * ((P + rb - 1) / rb) < sms)
                 rb = std::max<int64_t>(xalign, (rb / 2) / xalign * xalign);
+            // tuning switches (sweeps): rows per item, CTAs per SM
+            long long t = 0;
+            if (env_int("SSM_SSU_ROWS_PER_ITEM", &t) && t >= xalign && t % xalign == 0 &&
+                t <= rpt * rows_per_pass)
+                rb = std::min<int64_t>(t, P / xalign * xalign);
+            if (env_int("SSM_SSU_CTAS_PER_SM", &t) && t > 0 && t <= 32) plan.ctas_per_sm = (int)t;
             if (rb <= rpt * rows_per_pass && P % xalign == 0) {
                 plan.kernel = SSM_KERNEL_SSU_TMA;
                 plan.block = 256;

@@ -45,6 +45,7 @@ struct SsuPlan {
     int stages;          // bulk-copy kernel: stages in flight per CTA
     int rpt;             // bulk-copy kernel: rows per thread per item
     int sms;             // SMs of the device (persistent grids)
+    int ctas_per_sm;        // bulk-copy head kernel: CTAs per SM (0: as many as fit)
     long long wait_budget;  // bulk-copy kernels: cycles before a wait gives up
     int64_t drop_item;      // failure tests only: work item whose copies are never
                             // started, so its wait runs out (-1: none)

@@ -888,9 +888,12 @@ cudaError_t launch_head_tma_io(const SsuProblem& p, const SsuPlan& plan, cudaStr
         int per_sm = 0;
         cudaError_t e = prepare_tma_kernel(kern, plan.block, smem, &per_sm);
         if (e != cudaSuccess) return e;
-        // persistent grid: every CTA resident at once (the item ranges are static)
+        if (plan.ctas_per_sm > 0 && plan.ctas_per_sm < per_sm) per_sm = plan.ctas_per_sm;
+        // persistent grid: every CTA resident at once (the item ranges are
+        // static), and every CTA given the same number of items
         const int64_t cap = (int64_t)plan.sms * (per_sm > 0 ? per_sm : 1);
-        const int grid = (int)(plan.n_items < cap ? plan.n_items : cap);
+        const int64_t per_cta = (plan.n_items + cap - 1) / cap;
+        const int grid = (int)((plan.n_items + per_cta - 1) / per_cta);
         kern<<<grid, plan.block, smem, s>>>(p, plan);
         return cudaGetLastError();
     };
