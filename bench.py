@@ -466,7 +466,7 @@ def oracle_beside(entry, kind, rows=None):
         sample = f"{Bt} of the 245 batch rows (all 5120 channels), one decode step"
     elif kind == "m2_decode":
         H, P, N = entry["heads"], entry["P"], entry["N"]
-        Bt = rows or 64
+        Bt = rows or 16
         s = gen.ssu_mamba2_inputs(Bt, H, P, N, io="f32", state="f32", seed=0, tag="oracle_beside")
         t0 = time.perf_counter()
         oracle.ssu_mamba2(s.state, s.x, s.dt, s.A, s.B, s.C, D=s.D, dt_bias=s.dt_bias)
