@@ -1,0 +1,110 @@
+"""Randomised invariants of the fp64 oracle (CPU, hypothesis).
+
+The fixed-shape pins in test_oracle_pins.py tie the oracle to brute-force
+sums, closed forms and invariants.  These tests draw shapes, split points
+and seeds at random to show the same invariants hold away from the pinned
+shapes:
+  * a prefill split anywhere, state and conv state carried across, equals
+    the whole prefill (Mamba-1 and Mamba-2 layouts);
+  * without the conv and with h0 = 0, the output is linear in x (z fixed);
+  * a prefill of the first tokens followed by single-token updates equals
+    the whole prefill (Mamba-1 layout with the fused conv);
+  * the Mamba-2-layout prefill equals the Mamba-1 scan with its per-head
+    values repeated over the head's rows.
+"""
+import numpy as np
+from hypothesis import given, settings
+from hypothesis import strategies as st
+
+import oracle
+from state_space_model_causal_b200 import inputs as gen
+
+SETTINGS = dict(max_examples=25, deadline=None)
+
+
+@settings(**SETTINGS)
+@given(Bt=st.integers(1, 2), D=st.integers(1, 6), L=st.integers(2, 24), N=st.integers(1, 6),
+       W=st.sampled_from([0, 1, 3, 4]), frac=st.floats(0.05, 0.95), seed=st.integers(0, 10**6))
+def test_mamba1_prefill_split_anywhere(Bt, D, L, N, W, frac, seed):
+    split = max(1, min(L - 1, int(L * frac)))
+    s = gen.scan_inputs(Bt, L, D, N, W=W, io="f32", seed=seed, tag="prop", conv_state=W > 0, h0=True)
+    kw = dict(D=s.D, dt_bias=s.dt_bias, conv_weight=s.conv_weight, conv_bias=s.conv_bias)
+    full, hf, csf = oracle.scan(s.x, s.dt, s.A, s.B, s.C, z=s.z, conv_state=s.conv_state, h0=s.h0, **kw)
+    cut = lambda a, sl: a[..., sl]  # noqa: E731
+    a, h1, cs1 = oracle.scan(cut(s.x, slice(0, split)), cut(s.dt, slice(0, split)), s.A,
+                             cut(s.B, slice(0, split)), cut(s.C, slice(0, split)),
+                             z=cut(s.z, slice(0, split)), conv_state=s.conv_state, h0=s.h0, **kw)
+    b, h2, cs2 = oracle.scan(cut(s.x, slice(split, L)), cut(s.dt, slice(split, L)), s.A,
+                             cut(s.B, slice(split, L)), cut(s.C, slice(split, L)),
+                             z=cut(s.z, slice(split, L)), conv_state=cs1, h0=h1, **kw)
+    np.testing.assert_allclose(np.concatenate([a, b], -1), full, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(h2, hf, rtol=1e-11, atol=1e-12)
+    if W > 0:
+        np.testing.assert_array_equal(cs2, csf)
+
+
+@settings(**SETTINGS)
+@given(Bt=st.integers(1, 2), H=st.integers(1, 4), P=st.integers(1, 5), N=st.integers(1, 8),
+       L=st.integers(2, 20), G=st.sampled_from([1, 2]), frac=st.floats(0.05, 0.95),
+       seed=st.integers(0, 10**6))
+def test_mamba2_prefill_split_anywhere(Bt, H, P, N, L, G, frac, seed):
+    H = H * G  # heads divisible by groups
+    split = max(1, min(L - 1, int(L * frac)))
+    s = gen.scan_m2_inputs(Bt, H, P, N, L, G=G, io="f32", seed=seed, tag="prop", h0=True)
+    full, hf = oracle.scan_mamba2(s.x, s.dt, s.A, s.B, s.C, D=s.D, z=s.z, dt_bias=s.dt_bias, h0=s.h0)
+    sl1, sl2 = slice(0, split), slice(split, L)
+    a, h1 = oracle.scan_mamba2(s.x[..., sl1], s.dt[..., sl1], s.A, s.B[..., sl1], s.C[..., sl1], D=s.D,
+                               z=s.z[..., sl1], dt_bias=s.dt_bias, h0=s.h0)
+    b, h2 = oracle.scan_mamba2(s.x[..., sl2], s.dt[..., sl2], s.A, s.B[..., sl2], s.C[..., sl2], D=s.D,
+                               z=s.z[..., sl2], dt_bias=s.dt_bias, h0=h1)
+    np.testing.assert_allclose(np.concatenate([a, b], -1), full, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(h2, hf, rtol=1e-11, atol=1e-12)
+
+
+@settings(**SETTINGS)
+@given(D=st.integers(1, 5), L=st.integers(1, 16), N=st.integers(1, 5), alpha=st.floats(-3, 3),
+       seed=st.integers(0, 10**6))
+def test_mamba1_output_linear_in_x_without_conv(D, L, N, alpha, seed):
+    s = gen.scan_inputs(1, L, D, N, W=0, io="f32", seed=seed, tag="prop_lin")
+    x2 = gen.normal(s.x.shape, "prop_lin", seed, "x2")
+    kw = dict(D=s.D, z=s.z, dt_bias=s.dt_bias)
+    y1, _, _ = oracle.scan(s.x, s.dt, s.A, s.B, s.C, **kw)
+    y2, _, _ = oracle.scan(x2, s.dt, s.A, s.B, s.C, **kw)
+    y12, _, _ = oracle.scan(s.x + alpha * x2, s.dt, s.A, s.B, s.C, **kw)
+    np.testing.assert_allclose(y12, y1 + alpha * y2, rtol=1e-10, atol=1e-11)
+
+
+@settings(**SETTINGS)
+@given(Bt=st.integers(1, 2), D=st.integers(1, 4), N=st.integers(1, 4), L=st.integers(2, 10),
+       k=st.integers(1, 4), seed=st.integers(0, 10**6))
+def test_mamba1_prefill_then_single_token_updates(Bt, D, N, L, k, seed):
+    k = min(k, L - 1)
+    s = gen.scan_inputs(Bt, L, D, N, W=4, io="f32", seed=seed, tag="prop_pd", conv_state=True, h0=True)
+    kw = dict(D=s.D, dt_bias=s.dt_bias, conv_weight=s.conv_weight, conv_bias=s.conv_bias)
+    full, hf, csf = oracle.scan(s.x, s.dt, s.A, s.B, s.C, z=s.z, conv_state=s.conv_state, h0=s.h0, **kw)
+    head = slice(0, L - k)
+    _, h, cs = oracle.scan(s.x[..., head], s.dt[..., head], s.A, s.B[..., head], s.C[..., head],
+                           z=s.z[..., head], conv_state=s.conv_state, h0=s.h0, **kw)
+    st_ = h.reshape(Bt, 1, D, N)
+    for t in range(L - k, L):
+        o, st_, cs = oracle.ssu(st_, s.x[:, None, :, t], s.dt[:, None, :, t], s.A[None], s.B[..., t],
+                                s.C[..., t], D=s.D[None], z=s.z[:, None, :, t], dt_bias=s.dt_bias[None],
+                                conv_weight=s.conv_weight, conv_bias=s.conv_bias, conv_state=cs)
+        np.testing.assert_allclose(o[:, 0], full[..., t], rtol=1e-11, atol=1e-12)
+        cs = cs.reshape(Bt, D, -1)
+    np.testing.assert_allclose(st_.reshape(Bt, D, N), hf, rtol=1e-11, atol=1e-12)
+
+
+@settings(**SETTINGS)
+@given(Bt=st.integers(1, 2), H=st.integers(1, 3), P=st.integers(1, 4), N=st.integers(1, 6),
+       L=st.integers(1, 12), seed=st.integers(0, 10**6))
+def test_mamba2_prefill_equals_mamba1_scan_with_heads_repeated(Bt, H, P, N, L, seed):
+    s = gen.scan_m2_inputs(Bt, H, P, N, L, io="f32", seed=seed, tag="prop_x", h0=True)
+    y2, h2 = oracle.scan_mamba2(s.x, s.dt, s.A, s.B, s.C, D=s.D, z=s.z, dt_bias=s.dt_bias, h0=s.h0)
+    D1 = H * P
+    y1, h1, _ = oracle.scan(s.x.reshape(Bt, D1, L), np.repeat(s.dt, P, axis=1),
+                            np.repeat(s.A, P)[:, None] * np.ones((1, N)), s.B, s.C, D=np.repeat(s.D, P),
+                            z=s.z.reshape(Bt, D1, L), dt_bias=np.repeat(s.dt_bias, P),
+                            h0=s.h0.reshape(Bt, D1, N))
+    np.testing.assert_allclose(y2, y1.reshape(Bt, H, P, L), rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(h2, h1.reshape(Bt, H, P, N), rtol=1e-12, atol=1e-13)
