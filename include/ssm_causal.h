@@ -37,7 +37,9 @@
  * and per-dimension sizes and strides counted in ELEMENTS.  Strides must be
  * >= 0; a stride of 0 broadcasts an input along that dimension (never allowed
  * for outputs or in/out caches).  An optional tensor is absent when its data
- * pointer is NULL (its other fields are then ignored).  Parameters (A, D,
+ * pointer is NULL (its other fields are then ignored).  A non-empty tensor
+ * whose element count or byte span (from its first to its last element)
+ * exceeds 2^56 is rejected with SSM_ERR_UNSUPPORTED.  Parameters (A, D,
  * dt_bias, conv weight and bias) are float32.  Arithmetic is float32 in every
  * kernel; 16-bit inputs are widened on load and 16-bit outputs and caches are
  * rounded to nearest even on store.
@@ -269,7 +271,9 @@ ssm_status ssm_selective_scan_fwd(const ssm_scan_args* args, void* stream);
  * state_batch_indices[b]; state and conv_state then both hold the pool's slot
  * count in dim 0, which may differ from B.  A negative index marks a padding
  * row, which is skipped entirely (its out row is left untouched); an index at
- * or past the slot count is skipped the same way.  Without
+ * or past the slot count is skipped the same way.  Two rows that name the
+ * same slot race: that slot's caches and both rows' outputs are then
+ * undefined, so a batch names each slot at most once.  Without
  * indices, dim 0 of the caches must equal B.
  * ------------------------------------------------------------------------ */
 typedef struct ssm_ssu_args {

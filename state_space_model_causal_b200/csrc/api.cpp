@@ -42,7 +42,13 @@ int esize(int dt) {
 
 bool is_float(int dt) { return dt == SSM_F32 || dt == SSM_F16 || dt == SSM_BF16; }
 
-// rank, non-negative sizes and strides, element-aligned pointer
+// Largest element count and byte span a tensor may describe: far above any
+// device memory, low enough that no size, offset or extent computed from the
+// tensor overflows int64.
+constexpr int64_t kMaxSpan = (int64_t)1 << 56;
+
+// rank, non-negative sizes and strides, element-aligned pointer, element
+// count and byte span within kMaxSpan
 ssm_status basic(const ssm_tensor& t) {
     if (!t.data) return SSM_ERR_NULL;
     if (t.ndim < 1 || t.ndim > SSM_MAX_DIMS) return SSM_ERR_SHAPE;
@@ -52,6 +58,19 @@ ssm_status basic(const ssm_tensor& t) {
         if (t.stride[i] < 0) return SSM_ERR_STRIDE;
     }
     if (reinterpret_cast<uintptr_t>(t.data) % esize(t.dtype) != 0) return SSM_ERR_STRIDE;
+    for (int i = 0; i < t.ndim; ++i)
+        if (t.shape[i] == 0) return SSM_OK;  // empty: touches no memory
+    int64_t count = 1, last = 0;
+    for (int i = 0; i < t.ndim; ++i)
+        if (__builtin_mul_overflow(count, t.shape[i], &count) || count > kMaxSpan)
+            return SSM_ERR_UNSUPPORTED;
+    for (int i = 0; i < t.ndim; ++i) {
+        int64_t step = 0;
+        if (__builtin_mul_overflow(t.shape[i] - 1, t.stride[i], &step) ||
+            __builtin_add_overflow(last, step, &last) || last > kMaxSpan)
+            return SSM_ERR_UNSUPPORTED;
+    }
+    if ((last + 1) * esize(t.dtype) > kMaxSpan) return SSM_ERR_UNSUPPORTED;
     return SSM_OK;
 }
 
@@ -494,10 +513,8 @@ ssm_status scan_impl(const ssm_scan_args* a, cudaStream_t stream) {
         if (tiles * Bn > INT32_MAX) return SSM_ERR_UNSUPPORTED;
         plan.grid = (int)(tiles * Bn);
         plan.sw_pairs = 0;
-        if (const char* e = std::getenv("SSM_SCAN_SW_PAIRS")) {
-            const int v = std::atoi(e);
-            if (v >= 0 && v <= 3) plan.sw_pairs = v;
-        }
+        long long v = 0;
+        if (env_int("SSM_SCAN_SW_PAIRS", &v) && v >= 0 && v <= 3) plan.sw_pairs = (int)v;
         fill_info(a->info, plan.kernel, plan.grid, plan.block, 0, scan_vec_channels_per_cta(),
                   tiles * Bn);
         if (a->flags & SSM_FLAG_DRY_RUN) return SSM_OK;

@@ -366,6 +366,25 @@ def test_conv_error_paths(lib):
     _expect(lib, fn, a, EALIAS)
 
 
+def test_oversized_tensors_are_rejected_before_any_arithmetic(lib):
+    """Element counts, offsets and byte spans past 2^56 would overflow the
+    int64 extent and alias arithmetic: such tensors are refused up front."""
+    m = FakeMem()
+    big = 1 << 30
+    _expect(lib, "ssm_selective_scan_fwd", scan_args(m, x=m(F16, (big, big, 1 << 10))), EUNSUP)  # count
+    _expect(lib, "ssm_selective_scan_fwd",
+            scan_args(m, out=m(F16, (4, 5120, 2048), (1 << 62, 2048, 1))), EUNSUP)          # offset
+    _expect(lib, "ssm_causal_conv1d_fwd", conv_args(m, x=m(F32, (1, 1, 1 << 55))), EUNSUP)  # bytes
+    _expect(lib, "ssm_selective_state_update",
+            ssu_m2_args(m, state=m(F16, (8, 80, 64, 128), (1 << 60, 8192, 128, 1))), EUNSUP)
+    # an empty tensor touches no memory, whatever its other sizes and strides
+    a = conv_args(m, Bn=0, x=m(F16, (0, 64, 100), (1 << 62, 100, 1)))
+    a.out = m(F16, (0, 64, 100))
+    a.conv_state = m(F32, (0, 64, 4))
+    st, info = call(lib, "ssm_causal_conv1d_fwd", a)
+    assert st == OK and info.kernel == 0
+
+
 def test_binding_rejects_cpu_tensors():
     torch = pytest.importorskip("torch")
     x = torch.zeros(1, 2, 3)
