@@ -2,7 +2,8 @@
 
 Argument marshalling only: torch tensors are described by (device pointer,
 dtype, shape, strides) and handed to the C entry points together with the
-current CUDA stream.  Every step of the computation runs in the library's
+current CUDA stream of their device.  All tensors of one call must live on
+one CUDA device; the call runs with that device current.  Every step of the computation runs in the library's
 CUDA kernels; there is no CPU or PyTorch fallback.  If the shared library is
 missing, importing the functions raises instead of degrading silently.
 
@@ -159,12 +160,33 @@ def describe(t) -> Tensor:
                       tuple(t.shape), tuple(t.stride()))
 
 
-def _stream_of(tensors, stream):
-    if stream is not None:
-        return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+def device_of(tensors):
+    """The one CUDA device that every given tensor (None = absent) lives on;
+    a call whose tensors span devices is refused before anything launches."""
+    devs = {(t.device.type, t.device.index) for t in tensors if t is not None}
+    if len(devs) != 1:
+        raise ValueError(f"all tensors of a call must be on one CUDA device, got {sorted(devs)}")
+    return next(t.device for t in tensors if t is not None)
+
+
+def _run(fn, args, tensors, stream):
+    """Call a C entry point on the device of its tensors (switching the
+    current device only when it differs) and on `stream`, else on that
+    device's current stream."""
     import torch
-    dev = next(t.device for t in tensors if t is not None)
-    return torch.cuda.current_stream(dev).cuda_stream
+    dev = device_of(tensors)
+
+    def go():
+        if stream is not None:
+            handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+        else:
+            handle = torch.cuda.current_stream(dev).cuda_stream
+        return fn(ctypes.byref(args), handle)
+
+    if dev.index is not None and dev.index != torch.cuda.current_device():
+        with torch.cuda.device(dev):
+            return go()
+    return go()
 
 
 def _check(status: int, what: str):
@@ -193,7 +215,7 @@ def ssm_causal_conv1d_fwd(x, weight, bias=None, conv_state=None, silu=False, out
     a.x, a.weight, a.bias, a.conv_state, a.out = map(describe, (x, weight, bias, conv_state, out))
     a.silu = int(bool(silu))
     a.info = _info_ptr(info)
-    _check(library().ssm_causal_conv1d_fwd(ctypes.byref(a), _stream_of([x], stream)),
+    _check(_run(library().ssm_causal_conv1d_fwd, a, (x, weight, bias, conv_state, out), stream),
            "ssm_causal_conv1d_fwd")
     return out
 
@@ -212,7 +234,8 @@ def ssm_selective_scan_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, dt_soft
                                           conv_state, ssm_state, out))
     a.dt_softplus = int(bool(dt_softplus))
     a.info = _info_ptr(info)
-    _check(library().ssm_selective_scan_fwd(ctypes.byref(a), _stream_of([x], stream)),
+    _check(_run(library().ssm_selective_scan_fwd, a,
+                (x, dt, A, B, C, D, z, dt_bias, conv_weight, conv_bias, conv_state, ssm_state, out), stream),
            "ssm_selective_scan_fwd")
     return out
 
@@ -233,7 +256,9 @@ def ssm_selective_state_update(state, x, dt, A, B, C, D=None, z=None, dt_bias=No
                    state_batch_indices, out))
     a.dt_softplus = int(bool(dt_softplus))
     a.info = _info_ptr(info)
-    _check(library().ssm_selective_state_update(ctypes.byref(a), _stream_of([x], stream)),
+    _check(_run(library().ssm_selective_state_update, a,
+                (state, x, dt, A, B, C, D, z, dt_bias, conv_weight, conv_bias, conv_state,
+                 state_batch_indices, out), stream),
            "ssm_selective_state_update")
     return out
 

@@ -392,6 +392,70 @@ def test_binding_rejects_cpu_tensors():
         bd.describe(x)
 
 
+def test_binding_refuses_a_call_whose_tensors_span_devices():
+    torch = pytest.importorskip("torch")
+
+    class Stub:  # stands for a CUDA tensor: only its device is read
+        def __init__(self, index):
+            self.device = torch.device("cuda", index)
+
+    a, b, c = Stub(0), Stub(0), Stub(1)
+    assert bd.device_of((a, None, b)) == torch.device("cuda", 0)
+    assert bd.device_of((None, c)) == torch.device("cuda", 1)
+    with pytest.raises(ValueError, match="one CUDA device"):
+        bd.device_of((a, c))
+    with pytest.raises(ValueError, match="one CUDA device"):
+        bd.device_of((None, None))
+
+
+def test_binding_runs_on_the_tensors_device_and_stream(monkeypatch):
+    """The entry point gets the tensors' device's current stream (or the
+    stream given), and the current device is switched only when the tensors
+    live on another one.  torch.cuda is stubbed: nothing touches a GPU."""
+    torch = pytest.importorskip("torch")
+    state = {"current": 0, "switched_to": []}
+
+    class FakeStream:
+        def __init__(self, handle):
+            self.cuda_stream = handle
+
+    class FakeDeviceCtx:
+        def __init__(self, dev):
+            self.dev = dev
+
+        def __enter__(self):
+            state["switched_to"].append(self.dev.index)
+            self.prev, state["current"] = state["current"], self.dev.index
+
+        def __exit__(self, *exc):
+            state["current"] = self.prev
+
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: state["current"])
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda dev: FakeStream(1000 + dev.index))
+    monkeypatch.setattr(torch.cuda, "device", FakeDeviceCtx)
+
+    class Stub:
+        def __init__(self, index):
+            self.device = torch.device("cuda", index)
+
+    seen = []
+
+    def fake_entry(args_ref, handle):
+        seen.append((handle, state["current"]))
+        return 0
+
+    args = bd.ScanArgs()
+    assert bd._run(fake_entry, args, (Stub(0), None, Stub(0)), None) == 0
+    assert seen[-1] == (1000, 0) and state["switched_to"] == []          # same device: no switch
+    assert bd._run(fake_entry, args, (Stub(1), Stub(1)), None) == 0
+    assert seen[-1] == (1001, 1) and state["switched_to"] == [1]          # ran on device 1
+    assert state["current"] == 0                                          # and switched back
+    assert bd._run(fake_entry, args, (Stub(0),), FakeStream(77)) == 0
+    assert seen[-1] == (77, 0)                                            # the given stream
+    assert bd._run(fake_entry, args, (Stub(0),), 88) == 0
+    assert seen[-1] == (88, 0)                                            # a raw handle
+
+
 # ------------------------------------------------- Mamba-2-layout prefill --
 def scan_m2_args(mem, Bn=8, H=80, P=64, N=128, L=2048, G=1, io=F16, time_major=True, **over):
     """x (B, H, P, L) as the view of (B, L, H, P) storage when time_major."""
