@@ -46,6 +46,18 @@ MUTATIONS = [
     ("m2_prefill_bias_dropped", "double v = dt[(b * H + hh) * L + t] + (dt_bias_head ? dt_bias_head[hh] : 0.0);",
      "double v = dt[(b * H + hh) * L + t];"),
     ("m2_prefill_skip_dropped", "if (D_head) acc += D_head[hh] * xv;", "(void)D_head;"),
+    ("m2_prefill_decay_sign", "double decay = exp(delta * A_head[hh]);", "double decay = exp(-delta * A_head[hh]);"),
+    ("m2_prefill_C_for_B_in_update", "delta * Bg[n * L + t] * xv", "delta * Cg[n * L + t] * xv"),
+    ("m2_prefill_h0_ignored", "S[p * N + n] = h0 ? h0[((b * H + hh) * P + p) * N + n] : 0.0;",
+     "S[p * N + n] = 0.0;"),
+    ("m2_prefill_gate_on_x", "if (z) acc *= o_silu(z[at]);", "if (z) acc *= o_silu(x[at]);"),
+    ("m2_prefill_softplus_ignored",
+     "double v = dt[(b * H + hh) * L + t] + (dt_bias_head ? dt_bias_head[hh] : 0.0);\n"
+     "                double delta = dt_softplus ? o_softplus(v) : v;",
+     "double v = dt[(b * H + hh) * L + t] + (dt_bias_head ? dt_bias_head[hh] : 0.0);\n"
+     "                double delta = v;"),
+    ("m2_prefill_time_reversed", "const int64_t at = ((b * H + hh) * P + p) * L + t;",
+     "const int64_t at = ((b * H + hh) * P + p) * L + (L - 1 - t);"),
 ]
 
 # pins exercised against each mutant (all cheap)
