@@ -58,6 +58,14 @@ MUTATIONS = [
      "                double delta = v;"),
     ("m2_prefill_time_reversed", "const int64_t at = ((b * H + hh) * P + p) * L + t;",
      "const int64_t at = ((b * H + hh) * P + p) * L + (L - 1 - t);"),
+    ("conv_bias_dropped", "double acc = bias;", "double acc = 0.0; (void)bias;"),
+    ("conv_silu_skipped", "out[t] = silu ? o_silu(acc) : acc;", "out[t] = acc; (void)silu;"),
+    ("scan_A_transposed", "double a = exp(delta * A[d * N + n]);", "double a = exp(delta * A[n * D + d]);"),
+    ("ssu_conv_silu_skipped", "u = o_silu(acc);", "u = acc;"),
+    ("ssu_dt_bias_dropped", "double v = dt[row] + (dt_bias ? dt_bias[hp] : 0.0);", "double v = dt[row];"),
+    ("ssu_gate_dropped", "y += (Dv ? Dv[hp] : 0.0) * u;\n                if (z) y *= o_silu(z[row]);",
+     "y += (Dv ? Dv[hp] : 0.0) * u;\n                (void)z;"),
+    ("mamba2_decay_of_head_zero", "double dA = exp(delta * A_head[hh]);", "double dA = exp(delta * A_head[0]);"),
 ]
 
 # pins exercised against each mutant (all cheap)
