@@ -10,7 +10,11 @@ shapes:
   * a prefill of the first tokens followed by single-token updates equals
     the whole prefill (Mamba-1 layout with the fused conv);
   * the Mamba-2-layout prefill equals the Mamba-1 scan with its per-head
-    values repeated over the head's rows.
+    values repeated over the head's rows;
+  * both prefills are causal: inputs at later steps leave earlier outputs
+    bit-identical;
+  * Mamba-1 channels are independent: one channel's inputs, parameters and
+    states reach no other channel's outputs or states.
 """
 import numpy as np
 from hypothesis import given, settings
@@ -108,3 +112,70 @@ def test_mamba2_prefill_equals_mamba1_scan_with_heads_repeated(Bt, H, P, N, L, s
                             h0=s.h0.reshape(Bt, D1, N))
     np.testing.assert_allclose(y2, y1.reshape(Bt, H, P, L), rtol=1e-12, atol=1e-13)
     np.testing.assert_allclose(h2, h1.reshape(Bt, H, P, N), rtol=1e-12, atol=1e-13)
+
+
+@settings(**SETTINGS)
+@given(Bt=st.integers(1, 2), D=st.integers(1, 4), L=st.integers(2, 16), N=st.integers(1, 4),
+       W=st.sampled_from([0, 2, 4]), frac=st.floats(0.05, 0.95), seed=st.integers(0, 10**6))
+def test_mamba1_prefill_is_causal(Bt, D, L, N, W, frac, seed):
+    """Changing every input at steps >= t' leaves all outputs before t'
+    bit-identical (the conv looks back only, the scan runs forward)."""
+    cut = max(1, min(L - 1, int(L * frac)))
+    s = gen.scan_inputs(Bt, L, D, N, W=W, io="f32", seed=seed, tag="prop_c", conv_state=W > 0, h0=True)
+    kw = dict(D=s.D, dt_bias=s.dt_bias, conv_weight=s.conv_weight, conv_bias=s.conv_bias,
+              conv_state=s.conv_state, h0=s.h0)
+    y, _, _ = oracle.scan(s.x, s.dt, s.A, s.B, s.C, z=s.z, **kw)
+    late = lambda a, name: np.concatenate(  # noqa: E731
+        [a[..., :cut], gen.normal(a[..., cut:].shape, "prop_c2", seed, name)], -1)
+    y2, _, _ = oracle.scan(late(s.x, "x"), late(s.dt, "dt"), s.A, late(s.B, "B"), late(s.C, "C"),
+                           z=late(s.z, "z"), **kw)
+    np.testing.assert_array_equal(y2[..., :cut], y[..., :cut])
+    assert not np.array_equal(y2[..., cut:], y[..., cut:])
+
+
+@settings(**SETTINGS)
+@given(Bt=st.integers(1, 2), H=st.integers(1, 3), P=st.integers(1, 4), N=st.integers(1, 6),
+       L=st.integers(2, 12), frac=st.floats(0.05, 0.95), seed=st.integers(0, 10**6))
+def test_mamba2_prefill_is_causal(Bt, H, P, N, L, frac, seed):
+    cut = max(1, min(L - 1, int(L * frac)))
+    s = gen.scan_m2_inputs(Bt, H, P, N, L, io="f32", seed=seed, tag="prop_c", h0=True)
+    y, _ = oracle.scan_mamba2(s.x, s.dt, s.A, s.B, s.C, D=s.D, z=s.z, dt_bias=s.dt_bias, h0=s.h0)
+    late = lambda a, name: np.concatenate(  # noqa: E731
+        [a[..., :cut], gen.normal(a[..., cut:].shape, "prop_c2", seed, name)], -1)
+    y2, _ = oracle.scan_mamba2(late(s.x, "x"), late(s.dt, "dt"), s.A, late(s.B, "B"), late(s.C, "C"),
+                               D=s.D, z=late(s.z, "z"), dt_bias=s.dt_bias, h0=s.h0)
+    np.testing.assert_array_equal(y2[..., :cut], y[..., :cut])
+    assert not np.array_equal(y2[..., cut:], y[..., cut:])
+
+
+@settings(**SETTINGS)
+@given(Bt=st.integers(1, 2), D=st.integers(2, 5), L=st.integers(1, 12), N=st.integers(1, 4),
+       W=st.sampled_from([0, 4]), pick=st.integers(0, 10**6), seed=st.integers(0, 10**6))
+def test_mamba1_channels_are_independent(Bt, D, L, N, W, pick, seed):
+    """Channel d's x, dt, z, A row, D, dt_bias, conv weights and states affect
+    channel d's outputs and states only (B and C are shared)."""
+    d = pick % D
+    s = gen.scan_inputs(Bt, L, D, N, W=W, io="f32", seed=seed, tag="prop_i", conv_state=W > 0, h0=True)
+
+    def run(t):
+        return oracle.scan(t.x, t.dt, t.A, t.B, t.C, z=t.z, D=t.D, dt_bias=t.dt_bias,
+                           conv_weight=t.conv_weight, conv_bias=t.conv_bias, conv_state=t.conv_state, h0=t.h0)
+
+    y, hf, csf = run(s)
+    o = gen.scan_inputs(Bt, L, D, N, W=W, io="f32", seed=seed + 1, tag="prop_i", conv_state=W > 0, h0=True)
+    for name, axis in (("x", 1), ("dt", 1), ("z", 1), ("A", 0), ("D", 0), ("dt_bias", 0), ("h0", 1),
+                       ("conv_weight", 0), ("conv_bias", 0), ("conv_state", 1)):
+        a, b = getattr(s, name), getattr(o, name)
+        if a is None:
+            continue
+        a = a.copy()
+        idx = [slice(None)] * a.ndim
+        idx[axis] = d
+        a[tuple(idx)] = b[tuple(idx)]
+        setattr(s, name, a)
+    y2, hf2, csf2 = run(s)
+    keep = [k for k in range(D) if k != d]
+    np.testing.assert_array_equal(y2[:, keep], y[:, keep])
+    np.testing.assert_array_equal(hf2[:, keep], hf[:, keep])
+    if W > 0:
+        np.testing.assert_array_equal(csf2[:, keep], csf[:, keep])
