@@ -14,7 +14,10 @@ shapes:
   * both prefills are causal: inputs at later steps leave earlier outputs
     bit-identical;
   * Mamba-1 channels are independent: one channel's inputs, parameters and
-    states reach no other channel's outputs or states.
+    states reach no other channel's outputs or states;
+  * a Mamba-2-layout prefill cut into pieces scanned from zero states is
+    recovered exactly by composing the pieces' carries and adding the
+    decayed incoming state's readout (the context-parallel decomposition).
 """
 import numpy as np
 from hypothesis import given, settings
@@ -179,3 +182,28 @@ def test_mamba1_channels_are_independent(Bt, D, L, N, W, pick, seed):
     np.testing.assert_array_equal(hf2[:, keep], hf[:, keep])
     if W > 0:
         np.testing.assert_array_equal(csf2[:, keep], csf[:, keep])
+
+
+@settings(**SETTINGS)
+@given(Bt=st.integers(1, 2), H=st.integers(1, 3), P=st.integers(1, 3), N=st.integers(1, 5),
+       L=st.integers(4, 16), R=st.integers(2, 4), seed=st.integers(0, 10**6))
+def test_mamba2_prefill_context_parallel_decomposition(Bt, H, P, N, L, R, seed):
+    """A sequence cut into R pieces, each scanned from a zero state, is put
+    back together by composing the pieces' carries h -> Lambda*h + h_r (Lambda
+    the head's decay over the piece) and adding, at each step t of a piece,
+    silu(z_t) * C_t . (lambda_t * h_in), lambda_t the decay since the piece began."""
+    s = gen.scan_m2_inputs(Bt, H, P, N, L, io="f32", seed=seed, tag="prop_cp", h0=True)
+    full, hfull = oracle.scan_mamba2(s.x, s.dt, s.A, s.B, s.C, D=s.D, z=s.z, dt_bias=s.dt_bias, h0=s.h0)
+    delta = np.vectorize(oracle.softplus)(s.dt + s.dt_bias[None, :, None])  # (B, H, L)
+    cuts = np.linspace(0, L, R + 1).astype(int)
+    h_in = s.h0.copy()  # (B, H, P, N): the true state entering the current piece
+    for r in range(R):
+        sl = slice(cuts[r], cuts[r + 1])
+        y0, h_r = oracle.scan_mamba2(s.x[..., sl], s.dt[..., sl], s.A, s.B[..., sl], s.C[..., sl], D=s.D,
+                                     z=s.z[..., sl], dt_bias=s.dt_bias, h0=None)
+        lam = np.exp(np.cumsum(delta[..., sl], -1) * s.A[None, :, None])  # (B, H, Lr)
+        carry = np.einsum("bnt,bhpn->bhpt", s.C[:, 0, :, sl], h_in) * lam[:, :, None, :]  # one group
+        silu_z = s.z[..., sl] / (1.0 + np.exp(-s.z[..., sl]))
+        np.testing.assert_allclose(y0 + silu_z * carry, full[..., sl], rtol=1e-9, atol=1e-11)
+        h_in = lam[..., -1][:, :, None, None] * h_in + h_r
+    np.testing.assert_allclose(h_in, hfull, rtol=1e-9, atol=1e-11)
