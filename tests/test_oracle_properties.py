@@ -15,9 +15,9 @@ shapes:
     bit-identical;
   * Mamba-1 channels are independent: one channel's inputs, parameters and
     states reach no other channel's outputs or states;
-  * a Mamba-2-layout prefill cut into pieces scanned from zero states is
-    recovered exactly by composing the pieces' carries and adding the
-    decayed incoming state's readout (the context-parallel decomposition).
+  * a prefill cut into pieces scanned from zero states is recovered exactly
+    by composing the pieces' carries and adding the decayed incoming state's
+    readout (the context-parallel decomposition), in both layouts.
 """
 import numpy as np
 from hypothesis import given, settings
@@ -206,4 +206,30 @@ def test_mamba2_prefill_context_parallel_decomposition(Bt, H, P, N, L, R, seed):
         silu_z = s.z[..., sl] / (1.0 + np.exp(-s.z[..., sl]))
         np.testing.assert_allclose(y0 + silu_z * carry, full[..., sl], rtol=1e-9, atol=1e-11)
         h_in = lam[..., -1][:, :, None, None] * h_in + h_r
+    np.testing.assert_allclose(h_in, hfull, rtol=1e-9, atol=1e-11)
+
+
+@settings(**SETTINGS)
+@given(Bt=st.integers(1, 2), D=st.integers(1, 4), N=st.integers(1, 5), L=st.integers(4, 16),
+       R=st.integers(2, 4), W=st.sampled_from([0, 4]), seed=st.integers(0, 10**6))
+def test_mamba1_prefill_context_parallel_decomposition(Bt, D, N, L, R, W, seed):
+    """The same decomposition in the Mamba-1 layout: the decay is per (d, n)
+    element, and a piece's conv history is the W raw inputs before it."""
+    s = gen.scan_inputs(Bt, L, D, N, W=W, io="f32", seed=seed, tag="prop_cp1", conv_state=W > 0, h0=True)
+    kw = dict(D=s.D, dt_bias=s.dt_bias, conv_weight=s.conv_weight, conv_bias=s.conv_bias)
+    full, hfull, _ = oracle.scan(s.x, s.dt, s.A, s.B, s.C, z=s.z, conv_state=s.conv_state, h0=s.h0, **kw)
+    delta = np.vectorize(oracle.softplus)(s.dt + s.dt_bias[None, :, None])  # (B, D, L)
+    raw = np.concatenate([s.conv_state, s.x], -1) if W else None  # W history entries, then x
+    cuts = np.linspace(0, L, R + 1).astype(int)
+    h_in = s.h0.copy()  # (B, D, N)
+    for r in range(R):
+        sl = slice(cuts[r], cuts[r + 1])
+        cs = raw[..., cuts[r]:cuts[r] + W].copy() if W else None
+        y0, h_r, _ = oracle.scan(s.x[..., sl], s.dt[..., sl], s.A, s.B[..., sl], s.C[..., sl], z=s.z[..., sl],
+                                 conv_state=cs, h0=None, **kw)
+        lam = np.exp(np.cumsum(delta[..., sl], -1)[:, :, None, :] * s.A[None, :, :, None])  # (B, D, N, Lr)
+        carry = np.einsum("bnt,bdnt,bdn->bdt", s.C[:, 0, :, sl], lam, h_in)  # one group
+        silu_z = s.z[..., sl] / (1.0 + np.exp(-s.z[..., sl]))
+        np.testing.assert_allclose(y0 + silu_z * carry, full[..., sl], rtol=1e-9, atol=1e-11)
+        h_in = lam[..., -1] * h_in + h_r
     np.testing.assert_allclose(h_in, hfull, rtol=1e-9, atol=1e-11)
