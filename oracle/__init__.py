@@ -21,6 +21,11 @@ Functions (see the header comment of ``oracle.c`` for the definitions):
   SSU configs for Intel Arc Pro B70", section 关键源码片段.
 * :func:`ssu_mamba2` -- the same update in the Mamba-2 notation (scalar A,
   dt, D and dt_bias per head, ngroups), written separately in C.
+* :func:`round_cache` -- a state rounded to its cache dtype (fp32, fp16, bf16;
+  nearest, ties to even); :func:`ssu` and :func:`ssu_mamba2` apply it to the
+  updated state when given ``cache_dtype``, after the step's readout has used
+  the unrounded state, so that several consecutive decode steps can be
+  compared with a GPU cache kept in that dtype.
 """
 from __future__ import annotations
 
@@ -54,6 +59,8 @@ def build(force: bool = False) -> str:
 
 def configure(lib):
     """Declare the C signatures on a loaded oracle library and return it."""
+    lib.oracle_round_cache.restype = ctypes.c_int
+    lib.oracle_round_cache.argtypes = [_dp, _i64, ctypes.c_int]
     lib.oracle_silu.restype = ctypes.c_double
     lib.oracle_silu.argtypes = [ctypes.c_double]
     lib.oracle_softplus.restype = ctypes.c_double
@@ -163,14 +170,28 @@ def scan(x, dt, A, B, C, D=None, z=None, dt_bias=None, dt_softplus=True,
     return out, hf, cso
 
 
+_CACHE_CODES = {None: 0, "f64": 0, "f32": 1, "f16": 2, "bf16": 3}
+
+
+def round_cache(a, dtype):
+    """Values of ``a`` rounded to ``dtype`` ("f32", "f16", "bf16"; None or
+    "f64" keeps them), nearest with ties to even, returned as float64."""
+    out = np.array(a, dtype=np.float64, copy=True, order="C")
+    rc = _load().oracle_round_cache(out.ctypes.data_as(_dp), out.size, _CACHE_CODES[dtype])
+    if rc != 0:
+        raise ValueError("oracle_round_cache rejected its arguments")
+    return out
+
+
 def ssu(state, x, dt, A, B, C, D=None, z=None, dt_bias=None, dt_softplus=True,
-        conv_weight=None, conv_bias=None, conv_state=None):
+        conv_weight=None, conv_bias=None, conv_state=None, cache_dtype=None):
     """General single-token update.  state (Bt, H, P, N); x, z (Bt, H, P);
     dt broadcastable to (Bt, H, P); A broadcastable to (H, P, N);
     B, C (Bt, G, N); D, dt_bias broadcastable to (H, P); conv_weight (H*P, W);
     conv_bias (H*P); conv_state (Bt, H*P, W).
 
     Returns (out, new_state, new_conv_state or None); inputs are not modified.
+    cache_dtype rounds the returned state to that dtype (see round_cache).
     """
     lib = _load()
     st = np.array(state, dtype=np.float64, copy=True, order="C")
@@ -205,12 +226,16 @@ def ssu(state, x, dt, A, B, C, D=None, z=None, dt_bias=None, dt_softplus=True,
                         int(bool(dt_softplus)), pcw, pcb, pcs, po)
     if rc != 0:
         raise ValueError("oracle_ssu rejected its arguments")
+    if _CACHE_CODES[cache_dtype]:
+        st = round_cache(st, cache_dtype)
     return out, st, cs
 
 
-def ssu_mamba2(state, x, dt, A, B, C, D=None, z=None, dt_bias=None, dt_softplus=True):
+def ssu_mamba2(state, x, dt, A, B, C, D=None, z=None, dt_bias=None, dt_softplus=True,
+               cache_dtype=None):
     """Mamba-2 notation.  state (Bt, H, P, N); x, z (Bt, H, P); dt (Bt, H);
-    A, D, dt_bias (H); B, C (Bt, G, N).  Returns (out, new_state)."""
+    A, D, dt_bias (H); B, C (Bt, G, N).  Returns (out, new_state); cache_dtype
+    rounds the returned state to that dtype (see round_cache)."""
     lib = _load()
     st = np.array(state, dtype=np.float64, copy=True, order="C")
     Bt, H, P, N = st.shape
@@ -235,6 +260,8 @@ def ssu_mamba2(state, x, dt, A, B, C, D=None, z=None, dt_bias=None, dt_softplus=
                                int(bool(dt_softplus)), po)
     if rc != 0:
         raise ValueError("oracle_ssu_mamba2 rejected its arguments")
+    if _CACHE_CODES[cache_dtype]:
+        st = round_cache(st, cache_dtype)
     return out, st
 
 

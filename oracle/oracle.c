@@ -304,3 +304,43 @@ int oracle_scan_mamba2(int64_t B, int64_t H, int64_t P, int64_t N, int64_t G, in
     }
     return 0;
 }
+
+/* ---------------------------------------------------------------------------
+ * Rounding of a state cache to its storage dtype, for comparisons of several
+ * consecutive decode steps against a GPU cache kept in fp32, fp16 or bf16:
+ * after each step the stored state is the updated value rounded to nearest,
+ * ties to even (the readout of that step has already used the unrounded
+ * value).  dtype: 0 = keep fp64, 1 = fp32, 2 = fp16, 3 = bf16.
+ *
+ * fp16 keeps 11 significant bits for |v| >= 2^-14 and a fixed quantum of
+ * 2^-24 below (subnormals); bf16 keeps 8 significant bits for |v| >= 2^-126
+ * and a quantum of 2^-133 below.  Values past the largest finite value round
+ * to infinity (65504 for fp16; bf16 shares fp32's exponent range).
+ * ------------------------------------------------------------------------- */
+static double o_round_bits(double v, int sig_bits, int min_exp, double max_finite, double max_half_ulp) {
+    if (v == 0.0 || !isfinite(v)) return v;
+    int e = ilogb(v);                      /* 2^e <= |v| < 2^(e+1) */
+    if (e < min_exp) e = min_exp;          /* subnormal range: fixed quantum */
+    const double q = ldexp(1.0, e - (sig_bits - 1));
+    const double r = nearbyint(v / q) * q; /* default rounding mode: to nearest even */
+    if (fabs(r) > max_finite) {
+        /* values at or beyond max + half an ulp overflow */
+        return fabs(v) >= max_finite + max_half_ulp ? copysign(INFINITY, v) : copysign(max_finite, v);
+    }
+    return r;
+}
+
+int oracle_round_cache(double* v, int64_t n, int dtype) {
+    int64_t i;
+    if (n < 0 || dtype < 0 || dtype > 3) return -1;
+    for (i = 0; i < n; ++i) {
+        if (dtype == 1) {
+            v[i] = (double)(float)v[i];
+        } else if (dtype == 2) {
+            v[i] = o_round_bits(v[i], 11, -14, 65504.0, 16.0);
+        } else if (dtype == 3) {
+            v[i] = o_round_bits(v[i], 8, -126, 3.3895313892515355e38, ldexp(1.0, 127 - 8));
+        }
+    }
+    return 0;
+}

@@ -66,6 +66,12 @@ MUTATIONS = [
     ("ssu_gate_dropped", "y += (Dv ? Dv[hp] : 0.0) * u;\n                if (z) y *= o_silu(z[row]);",
      "y += (Dv ? Dv[hp] : 0.0) * u;\n                (void)z;"),
     ("mamba2_decay_of_head_zero", "double dA = exp(delta * A_head[hh]);", "double dA = exp(delta * A_head[0]);"),
+    ("round_ties_away_from_zero", "const double r = nearbyint(v / q) * q;", "const double r = round(v / q) * q;"),
+    ("round_f16_one_bit_short", "v[i] = o_round_bits(v[i], 11, -14, 65504.0, 16.0);",
+     "v[i] = o_round_bits(v[i], 10, -14, 65504.0, 16.0);"),
+    ("round_bf16_one_bit_long", "v[i] = o_round_bits(v[i], 8, -126,", "v[i] = o_round_bits(v[i], 9, -126,"),
+    ("round_f16_subnormal_quantum", "v[i] = o_round_bits(v[i], 11, -14, 65504.0, 16.0);",
+     "v[i] = o_round_bits(v[i], 11, -15, 65504.0, 16.0);"),
 ]
 
 # pins exercised against each mutant (all cheap)
@@ -86,6 +92,8 @@ PIN_CALLS = [
     lambda: pins.test_mamba2_prefill_matches_mamba1_scan_with_heads_expanded(2),
     lambda: pins.test_mamba2_prefill_equals_repeated_decode(),
     lambda: pins.test_mamba2_prefill_two_steps_by_hand(),
+    lambda: pins.test_round_cache_matches_library_conversions(),
+    lambda: pins.test_round_cache_ties_go_to_even(),
 ]
 
 

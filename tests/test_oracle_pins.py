@@ -402,3 +402,49 @@ def test_activation_special_values():
         # silu(v) - silu(-v) = v and softplus(v) - softplus(-v) = v
         assert oracle.silu(v) - oracle.silu(-v) == pytest.approx(v, rel=1e-14)
         assert oracle.softplus(v) - oracle.softplus(-v) == pytest.approx(v, rel=1e-14)
+
+
+# ------------------------------------------------------- cache-dtype rounding --
+def test_round_cache_matches_library_conversions():
+    """The oracle's rounding of a state to its cache dtype equals numpy's
+    float64 -> float16 conversion, torch's float32 -> bfloat16 conversion (on
+    values exact in float32, so that no double rounding is involved) and the
+    float64 -> float32 cast, including subnormals, ties and overflow."""
+    import torch
+    r = np.random.default_rng(0)
+    v = r.standard_normal(20000) * 10.0 ** r.integers(-9, 6, 20000)
+    edge = np.array([0.0, -0.0, 65504.0, 65519.99, 65520.0, -65520.0, 2.0 ** -24, 2.0 ** -25,
+                     3 * 2.0 ** -26, 1 + 2.0 ** -11, 1 + 3 * 2.0 ** -11, 1e300])
+    v = np.concatenate([v, edge])
+    with np.errstate(over="ignore"):
+        np.testing.assert_array_equal(oracle.round_cache(v, "f16"), v.astype(np.float16).astype(np.float64))
+        np.testing.assert_array_equal(oracle.round_cache(v, "f32"), v.astype(np.float32).astype(np.float64))
+    f = (r.standard_normal(20000) * 10.0 ** r.integers(-40, 38, 20000)).astype(np.float32)
+    f = np.concatenate([f[np.isfinite(f)], np.float32([1 + 2.0 ** -8, 1 + 3 * 2.0 ** -8, 2.0 ** -130])])
+    f = f.astype(np.float64)
+    np.testing.assert_array_equal(oracle.round_cache(f, "bf16"),
+                                  torch.from_numpy(f).float().bfloat16().double().numpy())
+    np.testing.assert_array_equal(oracle.round_cache(v, None), v)
+
+
+def test_round_cache_ties_go_to_even():
+    """Hand values at exact ties: 1 + 2^-11 lies halfway between the fp16
+    neighbours 1 and 1 + 2^-10 and goes to 1 (even last bit); 1 + 3 * 2^-11
+    goes up to 1 + 2^-9; the same for bf16 one exponent step of 2^-8."""
+    got = oracle.round_cache([1 + 2.0 ** -11, 1 + 3 * 2.0 ** -11, -(1 + 2.0 ** -11)], "f16")
+    assert list(got) == [1.0, 1 + 2.0 ** -9, -1.0]
+    got = oracle.round_cache([1 + 2.0 ** -8, 1 + 3 * 2.0 ** -8, 2 + 2.0 ** -7], "bf16")
+    assert list(got) == [1.0, 1 + 2.0 ** -6, 2.0]
+
+
+def test_ssu_cache_dtype_rounds_the_state_after_the_readout():
+    """With cache_dtype the step's output is that of the unrounded update and
+    the returned state is the unrounded state rounded to the cache dtype."""
+    s = gen.ssu_mamba2_inputs(2, 4, 8, 16, io="f32", state="f32", seed=31, tag="round")
+    o, st = oracle.ssu_mamba2(s.state, s.x, s.dt, s.A, s.B, s.C, D=s.D, dt_bias=s.dt_bias)
+    for dt_ in ("f16", "bf16"):
+        o2, st2 = oracle.ssu_mamba2(s.state, s.x, s.dt, s.A, s.B, s.C, D=s.D, dt_bias=s.dt_bias,
+                                    cache_dtype=dt_)
+        np.testing.assert_array_equal(o2, o)
+        np.testing.assert_array_equal(st2, oracle.round_cache(st, dt_))
+        assert not np.array_equal(st2, st)
