@@ -44,16 +44,19 @@
  * kernel; 16-bit inputs are widened on load and 16-bit outputs and caches are
  * rounded to nearest even on store.
  *
- * Ownership and threading.  The caller owns every buffer.  The library never
- * allocates or frees device memory, keeps no pointer after a call returns,
- * never synchronises the stream (except ssm_device_error) and holds no mutable
- * host-side state: every entry point is reentrant.  The only state it keeps is
- * on the device, one error word that the kernels set when they give up a bounded
- * wait (see ssm_device_error).  Environment variables SSM_SCAN_SW_PAIRS,
- * SSM_SSU_ROWS_PER_ITEM, SSM_SSU_CTAS_PER_SM (tuning sweeps), SSM_TEST_DROP_ITEM
- * and SSM_TEST_WAIT_CYCLES (failure tests of the bounded waits) are read at
- * each call and are never needed in normal use.  Work is enqueued on `stream` (a cudaStream_t; NULL is
- * the legacy default stream) and runs asynchronously.
+ * Ownership and threading.  The caller owns every buffer, including the
+ * prefill's optional workspace.  The library never allocates or frees device
+ * memory, keeps no pointer after a call returns and never synchronises the
+ * stream (except ssm_device_error / ssm_device_error_info).  Every entry point
+ * is reentrant: the only state the library keeps is the device-side error
+ * record that the kernels set when they give up a bounded wait (see
+ * ssm_device_error_info) and per-device values it queries once and caches
+ * (SM count, occupancy of the prefill kernel, the error record's address).  The environment variables
+ * SSM_SCAN_KERNEL, SSM_SCAN_SW, SSM_SCAN_SW_PAIRS, SSM_SSU_ROWS_PER_ITEM and
+ * SSM_SSU_CTAS_PER_SM select launch variants for measurement sweeps; they are
+ * read once, at the first call, and are never needed in normal use.  Work is
+ * enqueued on `stream` (a cudaStream_t; NULL is the legacy default stream) and
+ * runs asynchronously.
  *
  * Errors.  Every argument is checked before anything is launched; on an error
  * nothing is launched and nothing is written, and the status says which check
@@ -71,7 +74,7 @@
 extern "C" {
 #endif
 
-#define SSM_CAUSAL_ABI_VERSION 1
+#define SSM_CAUSAL_ABI_VERSION 2
 #define SSM_MAX_DIMS 5
 
 typedef enum ssm_dtype {
@@ -93,7 +96,9 @@ typedef enum ssm_status {
     SSM_ERR_CUDA = 6,        /* the CUDA launch returned an error */
     SSM_ERR_INTERNAL = 7,    /* a library invariant failed */
     SSM_ERR_VERSION = 8,     /* struct_size does not match this library */
-    SSM_ERR_ALIAS = 9        /* an output overlaps an input */
+    SSM_ERR_ALIAS = 9,       /* an output overlaps an input */
+    SSM_ERR_WORKSPACE = 10   /* the workspace is smaller than required or not
+                                256-byte aligned */
 } ssm_status;
 
 /* Flags for the `flags` field of every args struct. */
@@ -142,7 +147,12 @@ typedef enum ssm_kernel_id {
                                        (headdim x dstate) state per head, staged
                                        16-step chunks; headdim and dstate contiguous,
                                        dstate 64, 128 or 256, headdim % 8 == 0 */
-    SSM_KERNEL_SCAN_M2_GENERIC = 12 /* Mamba-2-layout prefill, any strides, warp per row */
+    SSM_KERNEL_SCAN_M2_GENERIC = 12, /* Mamba-2-layout prefill, any strides, warp per row */
+    SSM_KERNEL_SCAN_BAL = 13        /* fused prefill, persistent warps that each take an
+                                       equal slice of the (16-channel unit, 32-step
+                                       chunk) list and hand states over through the
+                                       workspace; d_state <= 16, conv width 0 or 4,
+                                       time contiguous, L % 8 == 0, 16-byte aligned rows */
 } ssm_kernel_id;
 
 /* ------------------------------------------------------------------------ *
@@ -234,9 +244,29 @@ typedef struct ssm_scan_args {
     ssm_tensor ssm_state;
     ssm_tensor out;
     ssm_launch_info* info; /* optional */
+    void* workspace;          /* optional device scratch, see below */
+    uint64_t workspace_bytes; /* its size in bytes */
 } ssm_scan_args;
 
 ssm_status ssm_selective_scan_fwd(const ssm_scan_args* args, void* stream);
+
+/* Workspace of the fast prefill.  On a problem with more (batch entry,
+ * 16-channel) units than the GPU runs warps at once, the fast kernel splits
+ * the work into equal slices per warp; a slice that starts or ends inside a
+ * unit hands its running state to the neighbouring warp through `workspace`.
+ * ssm_selective_scan_workspace_size() returns in *bytes how much workspace a
+ * call with these arguments can use on the current device (0 when it needs
+ * none); it checks the arguments as ssm_selective_scan_fwd does and launches
+ * nothing.  A workspace is a device buffer of at least that size, 256-byte
+ * aligned, ZERO-FILLED BEFORE ITS FIRST USE; every call leaves it in a state
+ * the next call accepts (a generation counter in its first bytes advances per
+ * call), so it is allocated and zeroed once and then reused.  Calls that share
+ * a workspace must be ordered on one stream: two that run at the same time
+ * race.  workspace == NULL runs the prefill without hand-overs (one whole unit
+ * per warp: correct, slower when the units do not divide evenly over the
+ * SMs); a workspace smaller than required, or misaligned, is
+ * SSM_ERR_WORKSPACE.  Returns SSM_ERR_NULL for a NULL `bytes`. */
+ssm_status ssm_selective_scan_workspace_size(const ssm_scan_args* args, uint64_t* bytes);
 
 /* ------------------------------------------------------------------------ *
  * ssm_selective_state_update -- one decode token, caches updated in place.
@@ -299,13 +329,43 @@ typedef struct ssm_ssu_args {
 
 ssm_status ssm_selective_state_update(const ssm_ssu_args* args, void* stream);
 
-/* Waits for the work enqueued on `stream` so far, then reports in *code the
- * device-side error word of the library's kernels and clears it: 0 = none,
- * 1 = a kernel gave up a bounded wait on one of its bulk copies and exited
- * early (its outputs for that call are incomplete).  No kernel ever traps or
- * hangs instead.  Returns SSM_ERR_NULL for a NULL code, SSM_ERR_CUDA if the
- * stream or the copy fails. */
+/* Device-side error record.  Every kernel wait that can only end when
+ * something else happens (a bulk copy landing in shared memory, a hand-over
+ * published by another warp) is bounded; when one runs out the kernel records
+ * it here instead of trapping or hanging:
+ *
+ *   ssm_selective_state_update (bulk-copy kernels SSM_KERNEL_SSU_TMA and
+ *     SSM_KERNEL_SSU_ROW_TMA): the CTA or warp that gave up exits; the work
+ *     items it had not finished are left as they were (their cache rows not
+ *     advanced, their outputs not written), every item it finished before is
+ *     complete.  first_item is the lowest work item any giving-up CTA or warp
+ *     had not finished; work items are numbered as in ssm_launch_info
+ *     (rows_per_item rows each): for SSU_TMA batch-major, then head, then row
+ *     block; for SSU_ROW_TMA channel-block-major, then batch row.
+ *   ssm_selective_scan_fwd (SSM_KERNEL_SCAN_BAL): a warp that waited in vain
+ *     for its predecessor's hand-over scans its piece of that unit from a
+ *     zero state instead; first_item is the lowest such unit
+ *     (batch * ceil(D / 16) + channel / 16); that unit's later outputs and
+ *     final state are wrong, all other units are complete.
+ *
+ * The record belongs to the CURRENT device: call these with that device
+ * current and a stream of that device.  Both wait for the work enqueued on
+ * `stream` so far, then read and clear the record in one step on the device
+ * (a report landing meanwhile is kept for the next read, never lost).
+ * ssm_device_error() stores only the code (0 = none, 1 = a wait ran out) in
+ * *code; ssm_device_error_info() fills a report (set its struct_size).  They
+ * return SSM_ERR_NULL for a NULL pointer, SSM_ERR_VERSION for a wrong
+ * struct_size, SSM_ERR_CUDA if the stream or the copy fails. */
+typedef struct ssm_device_error_report {
+    uint32_t struct_size; /* = sizeof(ssm_device_error_report) */
+    int32_t code;         /* 0 = none, 1 = a bounded wait ran out */
+    int32_t kernel;       /* ssm_kernel_id of the last kernel that reported (0: none) */
+    int32_t reserved;
+    int64_t first_item;   /* lowest unfinished work item as described above (-1: none) */
+} ssm_device_error_report;
+
 ssm_status ssm_device_error(int* code, void* stream);
+ssm_status ssm_device_error_info(ssm_device_error_report* report, void* stream);
 
 /* Human-readable name of a status code (static storage, never NULL). */
 const char* ssm_status_string(int status);
@@ -313,10 +373,19 @@ const char* ssm_status_string(int status);
 /* SSM_CAUSAL_ABI_VERSION of the loaded library. */
 int ssm_abi_version(void);
 
-/* sizeof() of the three args structs and of ssm_tensor / ssm_launch_info as
- * compiled into the library, so that bindings can check their layouts:
- * which = 0 tensor, 1 conv1d args, 2 scan args, 3 ssu args, 4 launch info. */
+/* sizeof() of the three args structs and of ssm_tensor / ssm_launch_info /
+ * ssm_device_error_report as compiled into the library, so that bindings can
+ * check their layouts: which = 0 tensor, 1 conv1d args, 2 scan args, 3 ssu
+ * args, 4 launch info, 5 error report. */
 size_t ssm_struct_size(int which);
+
+/* The wait budget, in cycles, that a failure test's request of `cycles`
+ * becomes: requests below 10^7 cycles are raised to 10^7.  Only the test
+ * build of the library (libssm_causal_testhooks.so, compiled with
+ * SSM_TEST_HOOKS) reads the failure-test switches SSM_TEST_DROP_ITEM and
+ * SSM_TEST_WAIT_CYCLES from the environment; the product library ignores
+ * them and always waits the full budget. */
+long long ssm_test_clamp_wait_budget(long long cycles);
 
 #ifdef __cplusplus
 }

@@ -6,4 +6,5 @@ The functions below are the thin ctypes binding of the three C entry points;
 they raise if the library has not been built (there is no fallback path).
 """
 from .binding import (LaunchInfo, SsmError, library, ssm_causal_conv1d_fwd,  # noqa: F401
-                      ssm_device_error, ssm_selective_scan_fwd, ssm_selective_state_update)
+                      ssm_device_error, ssm_device_error_info, ssm_selective_scan_fwd,
+                      ssm_selective_scan_workspace_size, ssm_selective_state_update)

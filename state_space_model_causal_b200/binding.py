@@ -22,6 +22,8 @@ from typing import Optional, Sequence
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libssm_causal.so")
+# the same library built with the failure-test switches (tests only)
+TESTHOOKS_LIB_PATH = os.path.join(_HERE, "libssm_causal_testhooks.so")
 MAX_DIMS = 5
 
 SSM_F32, SSM_F16, SSM_BF16, SSM_I32 = 0, 1, 2, 3
@@ -30,12 +32,12 @@ SSM_FLAG_DRY_RUN = 0x1
 STATUS = {
     0: "SSM_OK", 1: "SSM_ERR_NULL", 2: "SSM_ERR_SHAPE", 3: "SSM_ERR_DTYPE", 4: "SSM_ERR_STRIDE",
     5: "SSM_ERR_UNSUPPORTED", 6: "SSM_ERR_CUDA", 7: "SSM_ERR_INTERNAL", 8: "SSM_ERR_VERSION",
-    9: "SSM_ERR_ALIAS",
+    9: "SSM_ERR_ALIAS", 10: "SSM_ERR_WORKSPACE",
 }
 KERNELS = {
     0: "none", 1: "conv1d", 2: "conv1d_generic", 3: "scan_chunked", 4: "scan_generic",
     5: "ssu_vec", 6: "ssu_generic", 7: "scan_vec", 8: "ssu_row", 9: "ssu_tma", 10: "ssu_row_tma",
-    11: "scan_m2", 12: "scan_m2_generic",
+    11: "scan_m2", 12: "scan_m2_generic", 13: "scan_bal",
 }
 
 
@@ -63,6 +65,16 @@ class LaunchInfo(ctypes.Structure):
                 "rows_per_item": self.rows_per_item, "work_items": self.work_items}
 
 
+class ErrorReport(ctypes.Structure):
+    _fields_ = [("struct_size", ctypes.c_uint32), ("code", ctypes.c_int32),
+                ("kernel", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("first_item", ctypes.c_int64)]
+
+    def as_dict(self):
+        return {"code": self.code, "kernel": KERNELS.get(self.kernel, self.kernel) if self.code else None,
+                "first_item": self.first_item}
+
+
 class Conv1dArgs(ctypes.Structure):
     _fields_ = [("struct_size", ctypes.c_uint32), ("flags", ctypes.c_uint32),
                 ("x", Tensor), ("weight", Tensor), ("bias", Tensor), ("conv_state", Tensor),
@@ -75,7 +87,8 @@ class ScanArgs(ctypes.Structure):
                 ("x", Tensor), ("dt", Tensor), ("A", Tensor), ("B", Tensor), ("C", Tensor),
                 ("D", Tensor), ("z", Tensor), ("dt_bias", Tensor), ("dt_softplus", ctypes.c_int32),
                 ("conv_weight", Tensor), ("conv_bias", Tensor), ("conv_state", Tensor),
-                ("ssm_state", Tensor), ("out", Tensor), ("info", ctypes.POINTER(LaunchInfo))]
+                ("ssm_state", Tensor), ("out", Tensor), ("info", ctypes.POINTER(LaunchInfo)),
+                ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_uint64)]
 
 
 class SsuArgs(ctypes.Structure):
@@ -89,36 +102,70 @@ class SsuArgs(ctypes.Structure):
 
 _lock = threading.Lock()
 _lib = None
+_override = None  # a library swapped in by using_library() (failure tests)
 
 
 def library():
     """Load libssm_causal.so (raises if it has not been built)."""
     global _lib
+    if _override is not None:
+        return _override
     with _lock:
         if _lib is None:
-            if not os.path.exists(LIB_PATH):
-                raise ImportError(
-                    f"{LIB_PATH} is missing: build it with "
-                    "`python -m state_space_model_causal_b200.build` (there is no fallback)")
-            lib = ctypes.CDLL(LIB_PATH)
-            for name, argt in (("ssm_causal_conv1d_fwd", Conv1dArgs),
-                               ("ssm_selective_scan_fwd", ScanArgs),
-                               ("ssm_selective_state_update", SsuArgs)):
-                fn = getattr(lib, name)
-                fn.restype = ctypes.c_int
-                fn.argtypes = [ctypes.POINTER(argt), ctypes.c_void_p]
-            lib.ssm_status_string.restype = ctypes.c_char_p
-            lib.ssm_status_string.argtypes = [ctypes.c_int]
-            lib.ssm_abi_version.restype = ctypes.c_int
-            lib.ssm_device_error.restype = ctypes.c_int
-            lib.ssm_device_error.argtypes = [ctypes.POINTER(ctypes.c_int), ctypes.c_void_p]
-            lib.ssm_struct_size.restype = ctypes.c_size_t
-            lib.ssm_struct_size.argtypes = [ctypes.c_int]
-            for which, st in enumerate((Tensor, Conv1dArgs, ScanArgs, SsuArgs, LaunchInfo)):
-                if lib.ssm_struct_size(which) != ctypes.sizeof(st):
-                    raise ImportError(f"struct layout mismatch for {st.__name__}")
-            _lib = lib
+            _lib = _open(LIB_PATH)
     return _lib
+
+
+class using_library:
+    """Route every call of this binding to another build of the library (the
+    failure-test build at TESTHOOKS_LIB_PATH) for the duration of the block."""
+
+    def __init__(self, path):
+        self.path = path
+        self.saved = None
+
+    def __enter__(self):
+        global _override
+        self.saved = _override
+        _override = _open(self.path)
+        return _override
+
+    def __exit__(self, *exc):
+        global _override
+        _override = self.saved
+
+
+def _open(path):
+    """Load one build of the library and declare its entry points."""
+    if not os.path.exists(path):
+        raise ImportError(
+            f"{path} is missing: build it with "
+            "`python -m state_space_model_causal_b200.build` (there is no fallback)")
+    lib = ctypes.CDLL(path)
+    for name, argt in (("ssm_causal_conv1d_fwd", Conv1dArgs),
+                       ("ssm_selective_scan_fwd", ScanArgs),
+                       ("ssm_selective_state_update", SsuArgs)):
+        fn = getattr(lib, name)
+        fn.restype = ctypes.c_int
+        fn.argtypes = [ctypes.POINTER(argt), ctypes.c_void_p]
+    lib.ssm_selective_scan_workspace_size.restype = ctypes.c_int
+    lib.ssm_selective_scan_workspace_size.argtypes = [ctypes.POINTER(ScanArgs),
+                                                      ctypes.POINTER(ctypes.c_uint64)]
+    lib.ssm_status_string.restype = ctypes.c_char_p
+    lib.ssm_status_string.argtypes = [ctypes.c_int]
+    lib.ssm_abi_version.restype = ctypes.c_int
+    lib.ssm_device_error.restype = ctypes.c_int
+    lib.ssm_device_error.argtypes = [ctypes.POINTER(ctypes.c_int), ctypes.c_void_p]
+    lib.ssm_device_error_info.restype = ctypes.c_int
+    lib.ssm_device_error_info.argtypes = [ctypes.POINTER(ErrorReport), ctypes.c_void_p]
+    lib.ssm_test_clamp_wait_budget.restype = ctypes.c_longlong
+    lib.ssm_test_clamp_wait_budget.argtypes = [ctypes.c_longlong]
+    lib.ssm_struct_size.restype = ctypes.c_size_t
+    lib.ssm_struct_size.argtypes = [ctypes.c_int]
+    for which, st in enumerate((Tensor, Conv1dArgs, ScanArgs, SsuArgs, LaunchInfo, ErrorReport)):
+        if lib.ssm_struct_size(which) != ctypes.sizeof(st):
+            raise ImportError(f"struct layout mismatch for {st.__name__}")
+    return lib
 
 
 # ------------------------------------------------------------ descriptors --
@@ -203,6 +250,28 @@ def _info_ptr(info: Optional[LaunchInfo]):
 
 
 # ------------------------------------------------------------ entry points --
+def ssm_selective_scan_workspace_size(x, dt, A, B, C, D=None, z=None, dt_bias=None,
+                                      dt_softplus=True, conv_weight=None, conv_bias=None,
+                                      conv_state=None, ssm_state=None, out=None) -> int:
+    """Bytes of workspace ssm_selective_scan_fwd can use for these arguments on
+    their device (0: none)."""
+    import torch
+    if out is None:
+        out = torch.empty_like(x)
+    a = ScanArgs()
+    a.struct_size = ctypes.sizeof(ScanArgs)
+    (a.x, a.dt, a.A, a.B, a.C, a.D, a.z, a.dt_bias, a.conv_weight, a.conv_bias, a.conv_state,
+     a.ssm_state, a.out) = map(describe, (x, dt, A, B, C, D, z, dt_bias, conv_weight, conv_bias,
+                                          conv_state, ssm_state, out))
+    a.dt_softplus = int(bool(dt_softplus))
+    tensors = (x, dt, A, B, C, D, z, dt_bias, conv_weight, conv_bias, conv_state, ssm_state, out)
+    need = ctypes.c_uint64(0)
+    with _on_device(device_of(tensors)):
+        _check(library().ssm_selective_scan_workspace_size(ctypes.byref(a), ctypes.byref(need)),
+               "ssm_selective_scan_workspace_size")
+    return need.value
+
+
 def ssm_causal_conv1d_fwd(x, weight, bias=None, conv_state=None, silu=False, out=None,
                           stream=None, info: Optional[LaunchInfo] = None):
     """Causal depthwise conv1d.  x (B, D, L); weight (D, W) f32; bias (D);
@@ -222,8 +291,14 @@ def ssm_causal_conv1d_fwd(x, weight, bias=None, conv_state=None, silu=False, out
 
 def ssm_selective_scan_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, dt_softplus=True,
                            conv_weight=None, conv_bias=None, conv_state=None, ssm_state=None,
-                           out=None, stream=None, info: Optional[LaunchInfo] = None):
-    """Fused prefill (see include/ssm_causal.h).  Returns out (B, D, L)."""
+                           out=None, stream=None, info: Optional[LaunchInfo] = None,
+                           workspace="auto"):
+    """Fused prefill (see include/ssm_causal.h).  Returns out (B, D, L).
+
+    workspace: "auto" (default) passes a cached zero-initialised workspace of
+    the size the library asks for (one per device and stream); None passes no
+    workspace (the prefill then runs without hand-overs); a uint8 CUDA tensor
+    is passed as given."""
     import torch
     if out is None:
         out = torch.empty_like(x)
@@ -234,10 +309,74 @@ def ssm_selective_scan_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, dt_soft
                                           conv_state, ssm_state, out))
     a.dt_softplus = int(bool(dt_softplus))
     a.info = _info_ptr(info)
-    _check(_run(library().ssm_selective_scan_fwd, a,
-                (x, dt, A, B, C, D, z, dt_bias, conv_weight, conv_bias, conv_state, ssm_state, out), stream),
-           "ssm_selective_scan_fwd")
+    tensors = (x, dt, A, B, C, D, z, dt_bias, conv_weight, conv_bias, conv_state, ssm_state, out)
+    dev = device_of(tensors)
+    with _on_device(dev):
+        if isinstance(workspace, str):
+            if workspace != "auto":
+                raise ValueError(f"workspace must be 'auto', None or a tensor, not {workspace!r}")
+            need = ctypes.c_uint64(0)
+            _check(library().ssm_selective_scan_workspace_size(ctypes.byref(a), ctypes.byref(need)),
+                   "ssm_selective_scan_workspace_size")
+            if need.value:
+                ws = _workspace(dev, stream, need.value)
+                a.workspace, a.workspace_bytes = ws.data_ptr(), ws.numel() * ws.element_size()
+        elif workspace is not None:
+            a.workspace, a.workspace_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+        _check(_run(library().ssm_selective_scan_fwd, a, tensors, stream), "ssm_selective_scan_fwd")
     return out
+
+
+# Prefill workspaces: one per (device, stream), zero-filled when allocated and
+# grown by reallocation; the library keeps it consistent from call to call.
+_ws_lock = threading.Lock()
+_workspaces = {}
+
+
+def _stream_handle(dev, stream):
+    import torch
+    if stream is not None:
+        return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    return torch.cuda.current_stream(dev).cuda_stream
+
+
+def _workspace(dev, stream, nbytes):
+    """The zero-initialised workspace of (dev, stream), at least nbytes long
+    (256-byte aligned: torch's allocator aligns blocks to 512 bytes)."""
+    import torch
+    handle = _stream_handle(dev, stream)
+    key = (dev.index, handle)
+    with _ws_lock:
+        ws = _workspaces.get(key)
+        if ws is None or ws.numel() < nbytes:
+            # allocated and zero-filled on the stream the prefill runs on, so
+            # the fill is ordered before the kernel; a replaced buffer is
+            # recycled by the caching allocator only after that stream's
+            # queued work
+            ext = torch.cuda.ExternalStream(handle, device=dev)
+            with torch.cuda.stream(ext):
+                ws = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+            _workspaces[key] = ws
+        return ws
+
+
+class _on_device:
+    """Make `dev` current for the block (no-op when it already is)."""
+
+    def __init__(self, dev):
+        self.dev = dev
+        self.ctx = None
+
+    def __enter__(self):
+        import torch
+        if self.dev.index is not None and self.dev.index != torch.cuda.current_device():
+            self.ctx = torch.cuda.device(self.dev)
+            self.ctx.__enter__()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ctx is not None:
+            self.ctx.__exit__(*exc)
 
 
 def ssm_selective_state_update(state, x, dt, A, B, C, D=None, z=None, dt_bias=None,
@@ -271,3 +410,16 @@ def ssm_device_error(stream=None) -> int:
     st = stream.cuda_stream if stream is not None else torch.cuda.current_stream().cuda_stream
     _check(library().ssm_device_error(ctypes.byref(code), st), "ssm_device_error")
     return code.value
+
+
+def ssm_device_error_info(stream=None) -> dict:
+    """Wait for the stream, then read and clear the library's device error
+    record: {"code": 0 | 1, "kernel": name of the reporting kernel or None,
+    "first_item": lowest unfinished work item or -1} (see
+    include/ssm_causal.h, ssm_device_error_info)."""
+    import torch
+    rep = ErrorReport()
+    rep.struct_size = ctypes.sizeof(ErrorReport)
+    st = stream.cuda_stream if stream is not None else torch.cuda.current_stream().cuda_stream
+    _check(library().ssm_device_error_info(ctypes.byref(rep), st), "ssm_device_error_info")
+    return rep.as_dict()

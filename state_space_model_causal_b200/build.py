@@ -7,6 +7,11 @@ Each translation unit under ``csrc/`` is compiled to an object in
 ``state_space_model_causal_b200/libssm_causal.so``.  Objects are rebuilt when
 their source or any header is newer.  ``-Xptxas -v`` output (registers,
 spills, shared memory per kernel) is written to ``_build/ptxas.txt``.
+
+A second library, ``libssm_causal_testhooks.so``, is linked from the same
+objects except that the translation units with failure-test switches
+(``TEST_HOOK_SOURCES``) are compiled again with ``-DSSM_TEST_HOOKS``; only the
+GPU failure tests load it.  The product library has no such switches.
 """
 from __future__ import annotations
 
@@ -23,6 +28,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libssm_causal.so")
+TEST_LIB = os.path.join(PKG, "libssm_causal_testhooks.so")
+TEST_HOOK_SOURCES = ("ssu.cu", "api.cpp")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-I", INCLUDE,
@@ -45,42 +52,50 @@ def _headers():
         glob.glob(os.path.join(INCLUDE, "*.h"))
 
 
-def _compile(src: str, force: bool):
-    obj = os.path.join(BUILD, os.path.basename(src) + ".o")
+def _compile(src: str, force: bool, test_hooks: bool = False):
+    obj = os.path.join(BUILD, os.path.basename(src) + (".testhooks.o" if test_hooks else ".o"))
     newest = max([os.path.getmtime(src)] + [os.path.getmtime(h) for h in _headers()])
     if not force and os.path.exists(obj) and os.path.getmtime(obj) >= newest:
         return obj, ""
-    cmd = [_nvcc()] + NVCC_FLAGS + ["-c", src, "-o", obj]
+    extra = ["-DSSM_TEST_HOOKS"] if test_hooks else []
+    cmd = [_nvcc()] + NVCC_FLAGS + extra + ["-c", src, "-o", obj]
     if src.endswith(".cpp"):
-        cmd = [_nvcc()] + ARCH + ["-O3", "-std=c++17", "-Xcompiler", "-fPIC,-Wall", "-I", INCLUDE,
-                                  "-x", "c++", "-c", src, "-o", obj]
+        cmd = [_nvcc()] + ARCH + ["-O3", "-std=c++17", "-Xcompiler", "-fPIC,-Wall", "-I", INCLUDE] + extra + \
+            ["-x", "c++", "-c", src, "-o", obj]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         raise RuntimeError(f"nvcc failed for {src}:\n{res.stdout}\n{res.stderr}")
     return obj, res.stderr
 
 
+def _link(lib: str, objs, force: bool):
+    newest_obj = max(os.path.getmtime(o) for o in objs)
+    if force or not os.path.exists(lib) or os.path.getmtime(lib) < newest_obj:
+        tmp = lib + f".tmp{os.getpid()}"
+        cmd = [_nvcc()] + ARCH + ["-shared", "-o", tmp] + list(objs) + ["-lcudart_static"]
+        res = subprocess.run(cmd, capture_output=True, text=True)
+        if res.returncode != 0:
+            raise RuntimeError(f"link failed:\n{res.stdout}\n{res.stderr}")
+        os.replace(tmp, lib)
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile every CUDA/C++ source and link libssm_causal.so; return its path."""
+    """Compile every CUDA/C++ source, link libssm_causal.so and the failure-test
+    build libssm_causal_testhooks.so; return the product library's path."""
     os.makedirs(BUILD, exist_ok=True)
     srcs = _sources()
-    with cf.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
-        results = list(ex.map(lambda s: _compile(s, force), srcs))
-    objs = [o for o, _ in results]
-    logs = "".join(l for _, l in results if l)
+    jobs = [(s, False) for s in srcs] + [(s, True) for s in srcs if os.path.basename(s) in TEST_HOOK_SOURCES]
+    with cf.ThreadPoolExecutor(max_workers=min(8, len(jobs))) as ex:
+        results = list(ex.map(lambda j: _compile(j[0], force, j[1]), jobs))
+    objs = {j: o for j, (o, _) in zip(jobs, results)}
+    logs = "".join(l for (_, hooks), (_, l) in zip(jobs, results) if l and not hooks)
     if logs:
         with open(os.path.join(BUILD, "ptxas.txt"), "w") as f:
             f.write(logs)
         if verbose:
             sys.stderr.write(logs)
-    newest_obj = max(os.path.getmtime(o) for o in objs)
-    if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < newest_obj:
-        tmp = LIB + f".tmp{os.getpid()}"
-        cmd = [_nvcc()] + ARCH + ["-shared", "-o", tmp] + objs + ["-lcudart_static"]
-        res = subprocess.run(cmd, capture_output=True, text=True)
-        if res.returncode != 0:
-            raise RuntimeError(f"link failed:\n{res.stdout}\n{res.stderr}")
-        os.replace(tmp, LIB)
+    _link(LIB, [objs[(s, False)] for s in srcs], force)
+    _link(TEST_LIB, [objs[(s, os.path.basename(s) in TEST_HOOK_SOURCES)] for s in srcs], force)
     return LIB
 
 

@@ -9,6 +9,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
@@ -155,13 +156,56 @@ bool env_int(const char* name, long long* v) {
     return true;
 }
 
-int sm_count(bool dry_run) {
+// The current device (0 in dry-run mode, which makes no CUDA call).
+int current_device(bool dry_run) {
+    int dev = 0;
+    if (!dry_run && cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+    return dev;
+}
+
+// SM count of a device, queried once per device (dry-run mode assumes a B200).
+int sm_count(bool dry_run, int dev) {
     if (dry_run) return kDefaultSms;
-    int dev = 0, n = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return kDefaultSms;
+    static std::atomic<int> cache[kMaxDevices];
+    if (dev < 0 || dev >= kMaxDevices) return kDefaultSms;
+    int n = cache[dev].load(std::memory_order_acquire);
+    if (n > 0) return n;
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
         return kDefaultSms;
+    cache[dev].store(n, std::memory_order_release);
     return n;
+}
+int sm_count(bool dry_run) { return sm_count(dry_run, current_device(dry_run)); }
+
+// Tuning switches for measurement sweeps, read from the environment once per
+// process (never needed in normal use):
+//   SSM_SCAN_KERNEL=vec    prefill on the whole-unit kernel instead of the balanced one
+//   SSM_SCAN_SW=k          balanced prefill: k of every 8 exponential pairs on the FMA pipe (0..1)
+//   SSM_SCAN_SW_PAIRS=k    whole-unit prefill: k of 4 state pairs on the FMA pipe (0..3)
+//   SSM_SSU_ROWS_PER_ITEM, SSM_SSU_CTAS_PER_SM   Mamba-2 update launch shape
+struct Tuning {
+    bool scan_vec = false;
+    int scan_sw = 0;
+    int scan_vec_sw = 0;
+    long long ssu_rows = 0;
+    int ssu_ctas = 0;
+};
+
+Tuning read_tuning() {
+    Tuning t;
+    const char* k = std::getenv("SSM_SCAN_KERNEL");
+    t.scan_vec = k && std::strcmp(k, "vec") == 0;
+    long long v = 0;
+    if (env_int("SSM_SCAN_SW", &v) && v >= 0 && v <= 1) t.scan_sw = (int)v;
+    if (env_int("SSM_SCAN_SW_PAIRS", &v) && v >= 0 && v <= 3) t.scan_vec_sw = (int)v;
+    if (env_int("SSM_SSU_ROWS_PER_ITEM", &v) && v > 0) t.ssu_rows = v;
+    if (env_int("SSM_SSU_CTAS_PER_SM", &v) && v > 0 && v <= 32) t.ssu_ctas = (int)v;
+    return t;
+}
+
+const Tuning& tuning() {
+    static const Tuning t = read_tuning();  // thread-safe one-time initialisation
+    return t;
 }
 
 void fill_info(ssm_launch_info* info, int kernel, int grid, int block, int smem, int64_t rows,
@@ -252,6 +296,36 @@ ssm_status conv1d_impl(const ssm_conv1d_args* a, cudaStream_t stream) {
     fill_info(a->info, plan.kernel, plan.grid, plan.block, 0, 1, rows);
     if (a->flags & SSM_FLAG_DRY_RUN) return SSM_OK;
     return launch_conv1d(p, plan, stream) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+// ------------------------------------------------------------- workspace --
+// Balanced prefill workspace: a 256-byte header (generation, finished-worker
+// count), one 32-bit flag per worker (rounded up to 256 bytes), then one
+// hand-over state of 16 channels x 16 state entries (1 KB) per worker.
+constexpr long long kWaitBudget = 4000000000LL;  // cycles (~2 s) before a bounded wait gives up
+constexpr long long kMinTestBudget = 10000000LL; // shortest wait a failure test may ask for
+
+// A failure test's wait budget, never below kMinTestBudget.
+long long clamp_test_budget(long long v) { return v < kMinTestBudget ? kMinTestBudget : v; }
+uint64_t bal_flag_bytes(int64_t workers) { return ((uint64_t)workers * 4 + 255) / 256 * 256; }
+uint64_t bal_workspace_bytes(int64_t workers) {
+    return 256 + bal_flag_bytes(workers) + (uint64_t)workers * scan_bal_channels_per_unit() * 16 * 4;
+}
+
+bool present_ws(const ssm_scan_args* a) { return a->workspace != nullptr && a->workspace_bytes > 0; }
+
+// Does the workspace overlap any tensor of the call?
+bool overlaps_any(const ssm_scan_args* a) {
+    const uintptr_t lo = reinterpret_cast<uintptr_t>(a->workspace);
+    const uintptr_t hi = lo + (uintptr_t)a->workspace_bytes;
+    const ssm_tensor* all[] = {&a->x, &a->dt, &a->A, &a->B, &a->C, &a->D, &a->z, &a->dt_bias,
+                               &a->conv_weight, &a->conv_bias, &a->conv_state, &a->ssm_state, &a->out};
+    for (const ssm_tensor* t : all) {
+        uintptr_t tl, th;
+        extent(*t, &tl, &th);
+        if (tl != th && tl < hi && lo < th) return true;
+    }
+    return false;
 }
 
 // -------------------------------------------------------------------- scan --
@@ -372,7 +446,7 @@ ssm_status scan_m2_impl(const ssm_scan_args* a, cudaStream_t stream) {
     return launch_scan_m2(p, kernel, stream) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 
-ssm_status scan_impl(const ssm_scan_args* a, cudaStream_t stream) {
+ssm_status scan_impl(const ssm_scan_args* a, cudaStream_t stream, uint64_t* ws_query) {
     if (!a) return SSM_ERR_NULL;
     if (a->struct_size != sizeof(ssm_scan_args)) return SSM_ERR_VERSION;
     SSM_TRY(info_ok(a->info));
@@ -382,7 +456,18 @@ ssm_status scan_impl(const ssm_scan_args* a, cudaStream_t stream) {
     SSM_TRY(basic(a->B));
     SSM_TRY(basic(a->C));
     SSM_TRY(basic(a->out));
-    if (a->x.ndim == 4) return scan_m2_impl(a, stream);
+    if (a->x.ndim == 4) {
+        if (ws_query) {
+            // the Mamba-2-layout prefill uses no workspace; check the arguments
+            ssm_scan_args dry = *a;
+            dry.flags |= SSM_FLAG_DRY_RUN;
+            dry.info = nullptr;
+            SSM_TRY(scan_m2_impl(&dry, stream));
+            *ws_query = 0;
+            return SSM_OK;
+        }
+        return scan_m2_impl(a, stream);
+    }
     if (a->x.ndim != 3) return SSM_ERR_SHAPE;
     const int64_t Bn = a->x.shape[0], D = a->x.shape[1], L = a->x.shape[2];
     if (a->A.ndim != 2 || a->A.shape[0] != D) return SSM_ERR_SHAPE;
@@ -492,10 +577,17 @@ ssm_status scan_impl(const ssm_scan_args* a, cudaStream_t stream) {
     }
     p.out = a->out.data; p.o_b = sd(a->out, 0); p.o_d = sd(a->out, 1); p.o_t = sd(a->out, 2);
 
+    if (present_ws(a) && overlaps_any(a)) return SSM_ERR_ALIAS;
     if (Bn == 0 || D == 0 || L == 0) {  // nothing to compute, caches unchanged
+        if (ws_query) {
+            *ws_query = 0;
+            return SSM_OK;
+        }
         fill_info(a->info, SSM_KERNEL_NONE, 0, 0, 0, 0, 0);
         return SSM_OK;
     }
+    // a workspace query sizes against the live device unless it is a dry run
+    const bool dry = (a->flags & SSM_FLAG_DRY_RUN) != 0;
     ScanPlan plan{};
     const int es = esize(io);
     auto al16 = [](const void* ptr) { return ptr == nullptr || aligned16(ptr); };
@@ -506,19 +598,72 @@ ssm_status scan_impl(const ssm_scan_args* a, cudaStream_t stream) {
         al16(p.Cm) && al16(p.z) && m16(p.x_b) && m16(p.x_d) && m16(p.dt_b) && m16(p.dt_d) &&
         m16(p.o_b) && m16(p.o_d) && m16(p.B_b) && m16(p.B_g) && m16(p.B_n) && m16(p.C_b) &&
         m16(p.C_g) && m16(p.C_n) && (!p.z || (m16(p.z_b) && m16(p.z_d)));
+    if (vec_layout && scan_bal_supported(p) && !tuning().scan_vec) {
+        // balanced persistent prefill: equal slices of the (unit, chunk) list
+        const int kch = scan_bal_channels_per_unit();
+        const int warps = scan_bal_warps_per_cta();
+        const int dev = current_device(dry);
+        BalPlan bp{};
+        bp.nblk = (D + kch - 1) / kch;
+        bp.units = Bn * bp.nblk;
+        bp.nck = (L + scan_bal_steps_per_chunk() - 1) / scan_bal_steps_per_chunk();
+        bp.sw = tuning().scan_sw;
+        const int smem = scan_bal_smem_bytes(io);
+        // CTAs per SM: the occupancy query when live; in dry-run mode the
+        // shared-memory bound (228 KB per SM, 1 KB reserved per CTA), at most
+        // the 2 that the register budget allows
+        int per_sm = dry ? std::min(2, (228 * 1024) / (smem + 1024)) : scan_bal_ctas_per_sm(p, bp.sw, dev);
+        if (per_sm <= 0) return dry ? SSM_ERR_UNSUPPORTED : SSM_ERR_CUDA;
+        const int64_t slots = (int64_t)sm_count(dry, dev) * per_sm * warps;
+        const bool split = bp.units > slots;
+        const uint64_t need = split ? bal_workspace_bytes(slots) : 0;
+        if (ws_query) {
+            *ws_query = need;
+            return SSM_OK;
+        }
+        // the slice bounds w * units * chunks / workers stay far inside int64
+        if (bp.units > ((int64_t)1 << 40) / std::max<int64_t>(bp.nck, 1)) return SSM_ERR_UNSUPPORTED;
+        if (split && a->workspace) {
+            if (a->workspace_bytes < need || (reinterpret_cast<uintptr_t>(a->workspace) & 255u) != 0)
+                return SSM_ERR_WORKSPACE;
+            bp.workers = slots;
+            bp.cooperative = 1;
+            unsigned char* ws = static_cast<unsigned char*>(a->workspace);
+            bp.ws_head = reinterpret_cast<unsigned*>(ws);
+            bp.ws_flags = reinterpret_cast<unsigned*>(ws + 256);
+            bp.ws_slots = reinterpret_cast<float*>(ws + 256 + bal_flag_bytes(slots));
+        } else {
+            bp.workers = bp.units;  // whole units, no hand-over
+        }
+        const int64_t grid = (bp.workers + warps - 1) / warps;
+        if (grid > INT32_MAX) return SSM_ERR_UNSUPPORTED;
+        bp.grid = (int)grid;
+        bp.wait_budget = kWaitBudget;
+        fill_info(a->info, SSM_KERNEL_SCAN_BAL, bp.grid, 32 * warps, smem, kch, bp.units);
+        if (a->flags & SSM_FLAG_DRY_RUN) return SSM_OK;
+        bp.err = device_error_ptr(dev);
+        if (!bp.err) return SSM_ERR_CUDA;
+        return launch_scan_bal(p, bp, stream, dev) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+    }
     if (vec_layout && scan_vec_supported(p)) {
+        if (ws_query) {
+            *ws_query = 0;
+            return SSM_OK;
+        }
         plan.kernel = SSM_KERNEL_SCAN_VEC;
         plan.block = scan_vec_threads();
         const int64_t tiles = (D + scan_vec_channels_per_cta() - 1) / scan_vec_channels_per_cta();
         if (tiles * Bn > INT32_MAX) return SSM_ERR_UNSUPPORTED;
         plan.grid = (int)(tiles * Bn);
-        plan.sw_pairs = 0;
-        long long v = 0;
-        if (env_int("SSM_SCAN_SW_PAIRS", &v) && v >= 0 && v <= 3) plan.sw_pairs = (int)v;
+        plan.sw_pairs = tuning().scan_vec_sw;
         fill_info(a->info, plan.kernel, plan.grid, plan.block, 0, scan_vec_channels_per_cta(),
                   tiles * Bn);
         if (a->flags & SSM_FLAG_DRY_RUN) return SSM_OK;
         return launch_scan(p, plan, stream) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+    }
+    if (ws_query) {
+        *ws_query = 0;
+        return SSM_OK;
     }
     int ns = 1;
     while (ns * 4 < N) ns *= 2;
@@ -742,14 +887,19 @@ ssm_status ssu_impl(const ssm_ssu_args* a, cudaStream_t stream) {
 
     // ---- plan: streaming kernels when the state rows are 16-byte addressable
     SsuPlan plan{};
-    // bulk-copy waits give up after ~2 s of cycles.  Failure tests can shorten
-    // that and name one work item whose copies are never started, so that its
-    // wait runs out (SSM_TEST_WAIT_CYCLES, SSM_TEST_DROP_ITEM).
-    plan.wait_budget = 4000000000LL;
+    // bulk-copy waits give up after ~2 s of cycles
+    plan.wait_budget = kWaitBudget;
     plan.drop_item = -1;
-    long long v = 0;
-    if (env_int("SSM_TEST_WAIT_CYCLES", &v) && v > 0) plan.wait_budget = v;
-    if (env_int("SSM_TEST_DROP_ITEM", &v) && v >= 0) plan.drop_item = v;
+#ifdef SSM_TEST_HOOKS
+    // Test build only (libssm_causal_testhooks.so): the failure tests name one
+    // work item whose copies are never started, so that its wait runs out,
+    // and shorten the wait (never below kMinTestBudget cycles, ~5 ms).
+    {
+        long long v = 0;
+        if (env_int("SSM_TEST_WAIT_CYCLES", &v) && v > 0) plan.wait_budget = clamp_test_budget(v);
+        if (env_int("SSM_TEST_DROP_ITEM", &v) && v >= 0) plan.drop_item = v;
+    }
+#endif
     const int es = esize(p.state_dt);
     const bool vec_rows = p.st_n == 1 && (N * es) % 16 == 0 && aligned16(p.state) &&
                           (p.st_b * es) % 16 == 0 && (p.st_h * es) % 16 == 0 &&
@@ -796,11 +946,10 @@ ssm_status ssu_impl(const ssm_ssu_args* a, cudaStream_t stream) {
             while (rb > xalign && Bn * H * ((P + rb - 1) / rb) < sms)
                 rb = std::max<int64_t>(xalign, (rb / 2) / xalign * xalign);
             // tuning switches (sweeps): rows per item, CTAs per SM
-            long long t = 0;
-            if (env_int("SSM_SSU_ROWS_PER_ITEM", &t) && t >= xalign && t % xalign == 0 &&
-                t <= rpt * rows_per_pass)
+            const long long t = tuning().ssu_rows;
+            if (t >= xalign && t % xalign == 0 && t <= rpt * rows_per_pass)
                 rb = std::min<int64_t>(t, P / xalign * xalign);
-            if (env_int("SSM_SSU_CTAS_PER_SM", &t) && t > 0 && t <= 32) plan.ctas_per_sm = (int)t;
+            if (tuning().ssu_ctas > 0) plan.ctas_per_sm = tuning().ssu_ctas;
             if (rb <= rpt * rows_per_pass && P % xalign == 0) {
                 plan.kernel = SSM_KERNEL_SSU_TMA;
                 plan.block = 256;
@@ -947,7 +1096,12 @@ ssm_status ssm_causal_conv1d_fwd(const ssm_conv1d_args* args, void* stream) {
 }
 
 ssm_status ssm_selective_scan_fwd(const ssm_scan_args* args, void* stream) {
-    return scan_impl(args, static_cast<cudaStream_t>(stream));
+    return scan_impl(args, static_cast<cudaStream_t>(stream), nullptr);
+}
+
+ssm_status ssm_selective_scan_workspace_size(const ssm_scan_args* args, uint64_t* bytes) {
+    if (!bytes) return SSM_ERR_NULL;
+    return scan_impl(args, nullptr, bytes);
 }
 
 ssm_status ssm_selective_state_update(const ssm_ssu_args* args, void* stream) {
@@ -966,16 +1120,31 @@ const char* ssm_status_string(int status) {
         case SSM_ERR_INTERNAL: return "SSM_ERR_INTERNAL: library invariant failed";
         case SSM_ERR_VERSION: return "SSM_ERR_VERSION: struct_size does not match the library";
         case SSM_ERR_ALIAS: return "SSM_ERR_ALIAS: an output overlaps an input";
+        case SSM_ERR_WORKSPACE: return "SSM_ERR_WORKSPACE: workspace too small or not 256-byte aligned";
         default: return "unknown ssm_status";
     }
 }
 
+ssm_status ssm_device_error_info(ssm_device_error_report* report, void* stream) {
+    if (!report) return SSM_ERR_NULL;
+    if (report->struct_size != sizeof(ssm_device_error_report)) return SSM_ERR_VERSION;
+    DeviceError e{};
+    if (read_and_clear_device_error(&e, static_cast<cudaStream_t>(stream)) != cudaSuccess) return SSM_ERR_CUDA;
+    report->code = e.code;
+    report->kernel = e.code ? e.kernel : 0;
+    report->first_item = e.code ? e.first_item : -1;
+    return SSM_OK;
+}
+
 ssm_status ssm_device_error(int* code, void* stream) {
     if (!code) return SSM_ERR_NULL;
-    return read_and_clear_device_error(code, static_cast<cudaStream_t>(stream)) == cudaSuccess
-               ? SSM_OK
-               : SSM_ERR_CUDA;
+    DeviceError e{};
+    if (read_and_clear_device_error(&e, static_cast<cudaStream_t>(stream)) != cudaSuccess) return SSM_ERR_CUDA;
+    *code = e.code;
+    return SSM_OK;
 }
+
+long long ssm_test_clamp_wait_budget(long long cycles) { return clamp_test_budget(cycles); }
 
 int ssm_abi_version(void) { return SSM_CAUSAL_ABI_VERSION; }
 
@@ -986,6 +1155,7 @@ size_t ssm_struct_size(int which) {
         case 2: return sizeof(ssm_scan_args);
         case 3: return sizeof(ssm_ssu_args);
         case 4: return sizeof(ssm_launch_info);
+        case 5: return sizeof(ssm_device_error_report);
         default: return 0;
     }
 }

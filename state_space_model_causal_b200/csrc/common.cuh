@@ -14,6 +14,15 @@ namespace ssm {
 
 enum : int { kF32 = 0, kF16 = 1, kBF16 = 2, kI32 = 3 };
 
+// Record that a bounded wait ran out: code 1, the reporting kernel, and the
+// lowest work item that did not complete (see DeviceError in problem.h).
+template <typename E>
+__device__ __forceinline__ void report_device_error(E* err, int kernel, long long first_item) {
+    atomicExch(&err->code, 1);
+    atomicExch(&err->kernel, kernel);
+    atomicMin(&err->first_item, first_item);
+}
+
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -117,6 +126,28 @@ __device__ __forceinline__ void st_stream16(void* p, const uint4& v) {
     __stcs(static_cast<uint4*>(p), v);
 }
 
+// ------------------------------------------------------ cp.async staging --
+// 16-byte asynchronous copy global -> shared (zero-filled when !valid)
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
+    const unsigned d = static_cast<unsigned>(__cvta_generic_to_shared(dst));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src),
+                 "r"(valid ? 16 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+template <typename IoT>
+__device__ __forceinline__ void store8(IoT* p, const float* f) {
+    if constexpr (sizeof(IoT) == 2) {
+        __stcs(reinterpret_cast<uint4*>(p), Vec16<IoT>::pack(f));
+    } else {
+        __stcs(reinterpret_cast<uint4*>(p), Vec16<float>::pack(f));
+        __stcs(reinterpret_cast<uint4*>(p) + 1, Vec16<float>::pack(f + 4));
+    }
+}
+
 // ------------------------------------------------------- packed f32x2 math --
 // Two fp32 lanes in one 64-bit register pair; sm_100 executes add/mul/fma on
 // both halves with one instruction.
@@ -157,6 +188,41 @@ __device__ __forceinline__ float ex2_approx(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// 2^x for a pair, on the FMA pipe.  Cody-Waite split x = j + f with j the
+// nearest integer (via the 1.5*2^23 rounding constant) and f in [-1/2, 1/2];
+// 2^f from the degree-5 minimax polynomial for relative error on that
+// interval (coefficients fitted for this kernel by a Remez exchange, max
+// relative error 7.5e-8 before rounding); 2^j applied by adding j to the
+// exponent field.  x is clamped to [-125, 126] so the result stays normal.
+__device__ __forceinline__ u64 exp2_pair_fma(u64 x) {
+    float x0, x1;
+    upk(x, x0, x1);
+    x0 = fminf(fmaxf(x0, -125.0f), 126.0f);
+    x1 = fminf(fmaxf(x1, -125.0f), 126.0f);
+    const u64 xc = pk(x0, x1);
+    const u64 magic = pk(12582912.0f, 12582912.0f);
+    const u64 t = fadd2(xc, magic);
+    const u64 f = fsub2(xc, fsub2(t, magic));
+    u64 p = ffma2(pk(0.0013276472454890609f, 0.0013276472454890609f), f,
+                  pk(0.009675540961325169f, 0.009675540961325169f));
+    p = ffma2(p, f, pk(0.05550713092088699f, 0.05550713092088699f));
+    p = ffma2(p, f, pk(0.24022120237350464f, 0.24022120237350464f));
+    p = ffma2(p, f, pk(0.6931469440460205f, 0.6931469440460205f));
+    p = ffma2(p, f, pk(1.0000001192092896f, 1.0000001192092896f));
+    float p0, p1, t0, t1;
+    upk(p, p0, p1);
+    upk(t, t0, t1);
+    const float r0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+    const float r1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+    return pk(r0, r1);
+}
+
+__device__ __forceinline__ u64 exp2_pair_sfu(u64 x) {
+    float x0, x1;
+    upk(x, x0, x1);
+    return pk(ex2_approx(x0), ex2_approx(x1));
 }
 
 __device__ __forceinline__ float exp_fast(float x) { return ex2_approx(x * kLog2e); }

@@ -8,6 +8,20 @@
 
 namespace ssm {
 
+constexpr int kMaxDevices = 64;  // per-device host caches hold this many devices
+
+// The library's device-side error record (one per device).  code: 0 = none,
+// 1 = a bounded wait ran out; kernel: the ssm_kernel_id that reported last;
+// first_item: the lowest work item (in the reporting kernel's numbering) that
+// did not complete.  Kernels set it with atomics; ssm_device_error_info()
+// reads and clears every field with atomic exchanges.
+struct DeviceError {
+    int code;
+    int kernel;
+    long long first_item;
+};
+constexpr long long kNoItem = 0x7fffffffffffffffLL;
+
 // Single-token state update in the normalised (B, H, P, N) form.  A Mamba-1
 // problem (d_inner channels) is mapped to H = d_inner heads of headdim P = 1,
 // so that channel c = h * P + p and group g = h / (H / G) hold in both layouts.
@@ -83,6 +97,26 @@ struct ScanPlan {
     int sw_pairs;   // vector kernel: state-entry pairs per thread whose exp runs on the FMA pipe
 };
 
+// Launch of the load-balanced prefill (scan_bal.cu).  Units are (batch entry,
+// 16-channel block) x the whole sequence in 32-step chunks; `workers` warps
+// split the flattened (unit, chunk) list into equal contiguous slices.  With
+// more units than workers the slices hand states over through the workspace
+// (ws_* non-NULL, cooperative launch); otherwise workers == units.
+struct BalPlan {
+    int64_t units;       // batch entries x channel blocks
+    int64_t nblk;        // channel blocks per batch entry
+    int64_t nck;         // chunks per unit (ceil(L / 32))
+    int64_t workers;     // warps that take work
+    int grid;            // CTAs
+    int sw;              // exponentials per 8 evaluated on the FMA pipe
+    int cooperative;     // all CTAs co-resident (required when slices hand over)
+    unsigned* ws_head;   // workspace header: generation, finished-worker count
+    unsigned* ws_flags;  // one flag per worker: its hand-over is published
+    float* ws_slots;     // one hand-over state per worker (16 x 16 floats)
+    DeviceError* err;    // device error record
+    long long wait_budget;  // cycles before a hand-over wait gives up
+};
+
 // Prefill in the Mamba-2 layout: x, z, out (Bn, H, P, L); dt (Bn, H, L);
 // A, D, dt_bias (H); B, C (Bn, G, N, L); ssm_state (Bn, H, P, N).  Strides in
 // elements; head h reads group h / (H / G).
@@ -123,7 +157,15 @@ cudaError_t launch_ssu(const SsuProblem& p, const SsuPlan& plan, cudaStream_t s)
 int ssu_tma_max_stages();
 int ssu_row_tma_warps();
 int ssu_row_tma_stages();
-cudaError_t read_and_clear_device_error(int* code, cudaStream_t s);
+cudaError_t read_and_clear_device_error(DeviceError* out, cudaStream_t s);
+DeviceError* device_error_ptr(int dev);
+bool scan_bal_supported(const ScanProblem& p);
+int scan_bal_channels_per_unit();
+int scan_bal_steps_per_chunk();
+int scan_bal_warps_per_cta();
+int scan_bal_smem_bytes(int io_dt);
+int scan_bal_ctas_per_sm(const ScanProblem& p, int sw, int dev);
+cudaError_t launch_scan_bal(const ScanProblem& p, const BalPlan& bp, cudaStream_t s, int dev);
 cudaError_t launch_scan(const ScanProblem& p, const ScanPlan& plan, cudaStream_t s);
 bool scan_vec_supported(const ScanProblem& p);
 int scan_vec_threads();

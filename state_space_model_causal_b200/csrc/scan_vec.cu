@@ -46,62 +46,6 @@ constexpr int kThreads = 32;  // one warp: 8 channel pairs x 4 threads
 constexpr int kV = 8;         // time steps per thread per chunk (one 16-byte vector of 16-bit I/O)
 constexpr int kYStride = kT + 4;
 
-// 2^x for a pair, on the FMA pipe.  Cody-Waite split x = j + f with j the
-// nearest integer (via the 1.5*2^23 rounding constant) and f in [-1/2, 1/2];
-// 2^f from the degree-5 minimax polynomial for relative error on that
-// interval (coefficients fitted for this kernel by a Remez exchange, max
-// relative error 7.5e-8 before rounding); 2^j applied by adding j to the
-// exponent field.  x is clamped to [-125, 126] so the result stays normal.
-__device__ __forceinline__ u64 exp2_pair_fma(u64 x) {
-    float x0, x1;
-    upk(x, x0, x1);
-    x0 = fminf(fmaxf(x0, -125.0f), 126.0f);
-    x1 = fminf(fmaxf(x1, -125.0f), 126.0f);
-    const u64 xc = pk(x0, x1);
-    const u64 magic = pk(12582912.0f, 12582912.0f);
-    const u64 t = fadd2(xc, magic);
-    const u64 f = fsub2(xc, fsub2(t, magic));
-    u64 p = ffma2(pk(0.0013276472454890609f, 0.0013276472454890609f), f,
-                  pk(0.009675540961325169f, 0.009675540961325169f));
-    p = ffma2(p, f, pk(0.05550713092088699f, 0.05550713092088699f));
-    p = ffma2(p, f, pk(0.24022120237350464f, 0.24022120237350464f));
-    p = ffma2(p, f, pk(0.6931469440460205f, 0.6931469440460205f));
-    p = ffma2(p, f, pk(1.0000001192092896f, 1.0000001192092896f));
-    float p0, p1, t0, t1;
-    upk(p, p0, p1);
-    upk(t, t0, t1);
-    const float r0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
-    const float r1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
-    return pk(r0, r1);
-}
-
-__device__ __forceinline__ u64 exp2_pair_sfu(u64 x) {
-    float x0, x1;
-    upk(x, x0, x1);
-    return pk(ex2_approx(x0), ex2_approx(x1));
-}
-
-// 16-byte asynchronous copy global -> shared (zero-filled when !valid)
-__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
-    const unsigned d = static_cast<unsigned>(__cvta_generic_to_shared(dst));
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src),
-                 "r"(valid ? 16 : 0)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
-template <typename IoT>
-__device__ __forceinline__ void store8(IoT* p, const float* f) {
-    if constexpr (sizeof(IoT) == 2) {
-        __stcs(reinterpret_cast<uint4*>(p), Vec16<IoT>::pack(f));
-    } else {
-        __stcs(reinterpret_cast<uint4*>(p), Vec16<float>::pack(f));
-        __stcs(reinterpret_cast<uint4*>(p) + 1, Vec16<float>::pack(f + 4));
-    }
-}
-
 // x, dt, z of one chunk as staged by cp.async: [channel][32 steps].  Each
 // thread copies, and later reads back, only its own 8-step vectors.
 template <typename IoT> struct __align__(16) RawXZ {

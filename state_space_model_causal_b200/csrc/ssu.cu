@@ -22,12 +22,22 @@
 #include "problem.h"
 #include "tma.cuh"
 
+#include <atomic>
+
 namespace ssm {
 
-// Error word shared by the kernels of this file: 0 = none, 1 = a bounded wait
-// on a bulk copy timed out (the kernel then exited early).  Read and cleared
-// by ssm_device_error() through the host helpers at the end of this file.
-__device__ int g_ssm_device_error = 0;
+// The device error record of the library (DeviceError in problem.h): set by
+// a kernel whose bounded wait on a bulk copy (or a hand-over) ran out, read
+// and cleared by ssm_device_error() / ssm_device_error_info() through the
+// host helpers at the end of this file.  Kernels in other files are handed
+// its address (device_error_ptr).
+__device__ DeviceError g_ssm_device_error = {0, 0, kNoItem};
+__device__ DeviceError g_ssm_device_error_snap = {0, 0, kNoItem};
+
+// Budget of the wait for copies still in flight after a stage wait gave up:
+// always the full one, whatever the stage budget, so that a CTA never exits
+// while bulk copies still write into its shared memory.
+constexpr long long kCleanupBudget = 4000000000LL;
 
 namespace {
 
@@ -310,7 +320,9 @@ __global__ void __launch_bounds__(256, 3) ssu_head_tma_kernel(const SsuProblem p
     // padding row completes the stage's phase without data
     auto issue = [&](unsigned k, const Pos& q) {
         uint64_t* bar = &full[k % S];
+#ifdef SSM_TEST_HOOKS
         if ((int64_t)(i0 + k) == plan.drop_item) return;  // failure test: never completes
+#endif
         const int64_t slot = slot_of(q.b);
         if (slot < 0) {
             mbar_arrive(bar);
@@ -381,11 +393,16 @@ __global__ void __launch_bounds__(256, 3) ssu_head_tma_kernel(const SsuProblem p
         }
         const bool ok = mbar_wait_bounded(&full[stage], parity, plan.wait_budget);
         if (__syncthreads_or(!ok)) {
-            // give up: wait (bounded) for this CTA's copies still in flight, flag, exit
+            // give up: wait for this CTA's copies still in flight (items k ..
+            // k+S-1 were issued, all but a dropped one), record, exit
             if (tid == 0) {
-                for (unsigned kk = k; kk < min(cnt, k + S); ++kk)
-                    mbar_wait_bounded(&full[kk % S], (kk / S) & 1u, plan.wait_budget);
-                atomicExch(&g_ssm_device_error, 1);
+                for (unsigned kk = k; kk < min(cnt, k + S); ++kk) {
+#ifdef SSM_TEST_HOOKS
+                    if ((int64_t)(i0 + kk) == plan.drop_item) continue;  // never issued
+#endif
+                    mbar_wait_bounded(&full[kk % S], (kk / S) & 1u, kCleanupBudget);
+                }
+                report_device_error(&g_ssm_device_error, SSM_KERNEL_SSU_TMA, (long long)(i0 + k));
             }
             return;
         }
@@ -540,7 +557,9 @@ __global__ void __launch_bounds__(32 * kRowWarps, kRowMinBlocks) ssu_row_tma_ker
     // stage's phase without data
     auto issue = [&](unsigned k) {
         const unsigned item = i0 + k;
+#ifdef SSM_TEST_HOOKS
         if ((int64_t)item == plan.drop_item) return;  // failure test: never completes
+#endif
         const unsigned cb = item / Bn, b = item - cb * Bn;
         uint64_t* bar = &bars[k % kWarpStages];
         const int64_t slot = slot_of(b);
@@ -610,10 +629,14 @@ __global__ void __launch_bounds__(32 * kRowWarps, kRowMinBlocks) ssu_row_tma_ker
                 // items issued so far: up to k + kWarpStages - 2 (the first
                 // kWarpStages before the loop, one refill per later step)
                 const unsigned hi = min(cnt, k == 0 ? (unsigned)kWarpStages : k + kWarpStages - 1);
-                for (unsigned kk = k; kk < hi; ++kk)
-                    mbar_wait_bounded(&bars[kk % kWarpStages], (kk / kWarpStages) & 1u, plan.wait_budget);
+                for (unsigned kk = k; kk < hi; ++kk) {
+#ifdef SSM_TEST_HOOKS
+                    if ((int64_t)(i0 + kk) == plan.drop_item) continue;  // never issued
+#endif
+                    mbar_wait_bounded(&bars[kk % kWarpStages], (kk / kWarpStages) & 1u, kCleanupBudget);
+                }
                 bulk_wait_all();
-                atomicExch(&g_ssm_device_error, 1);
+                report_device_error(&g_ssm_device_error, SSM_KERNEL_SSU_ROW_TMA, (long long)(i0 + k));
             }
             return;
         }
@@ -1006,23 +1029,48 @@ int ssu_tma_max_stages() { return kTmaStagesMax; }
 int ssu_row_tma_warps() { return kRowWarps; }
 int ssu_row_tma_stages() { return kWarpStages; }
 
-// Read the device error word into *code (after the stream's work so far) and
-// clear it.
-cudaError_t read_and_clear_device_error(int* code, cudaStream_t s) {
-    int v = 0;
-    cudaError_t e = cudaMemcpyFromSymbolAsync(&v, g_ssm_device_error, sizeof(int), 0,
-                                              cudaMemcpyDeviceToHost, s);
+// Device address of the error record on device `dev` (the current device),
+// looked up once per device so that kernels in other translation units can
+// be handed it.  NULL if the lookup fails.
+DeviceError* device_error_ptr(int dev) {
+    static std::atomic<DeviceError*> cache[kMaxDevices];
+    if (dev < 0 || dev >= kMaxDevices) return nullptr;
+    DeviceError* ptr = cache[dev].load(std::memory_order_acquire);
+    if (ptr) return ptr;
+    void* addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_ssm_device_error) != cudaSuccess) return nullptr;
+    ptr = static_cast<DeviceError*>(addr);
+    cache[dev].store(ptr, std::memory_order_release);
+    return ptr;
+}
+
+namespace {
+// Moves the error record into the snapshot and clears it, field by field
+// with atomic exchanges: a report that lands while this runs is either in
+// the snapshot or left for the next read, never lost.
+__global__ void take_device_error_kernel() {
+    g_ssm_device_error_snap.code = atomicExch(&g_ssm_device_error.code, 0);
+    g_ssm_device_error_snap.kernel = atomicExch(&g_ssm_device_error.kernel, 0);
+    g_ssm_device_error_snap.first_item =
+        (long long)atomicExch(reinterpret_cast<unsigned long long*>(&g_ssm_device_error.first_item),
+                              (unsigned long long)kNoItem);
+}
+}  // namespace
+
+// After the work enqueued on `s`, take the current device's error record
+// (read and clear in one step on the device) and copy it to *out.
+cudaError_t read_and_clear_device_error(DeviceError* out, cudaStream_t s) {
+    take_device_error_kernel<<<1, 1, 0, s>>>();
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    DeviceError v{};
+    e = cudaMemcpyFromSymbolAsync(&v, g_ssm_device_error_snap, sizeof(DeviceError), 0,
+                                  cudaMemcpyDeviceToHost, s);
     if (e != cudaSuccess) return e;
     e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) return e;
-    *code = v;
-    if (v != 0) {
-        const int zero = 0;
-        e = cudaMemcpyToSymbolAsync(g_ssm_device_error, &zero, sizeof(int), 0,
-                                    cudaMemcpyHostToDevice, s);
-        if (e == cudaSuccess) e = cudaStreamSynchronize(s);
-    }
-    return e;
+    *out = v;
+    return cudaSuccess;
 }
 
 }  // namespace ssm

@@ -51,7 +51,23 @@ int main(void) {
     a.info = &info;
     int st = ssm_selective_scan_fwd(&a, NULL);
     printf("scan %s kernel %d grid %d\n", ssm_status_string(st), info.kernel, info.grid);
-    if (st != SSM_OK || info.kernel != SSM_KERNEL_SCAN_VEC) ++fails;
+    if (st != SSM_OK || info.kernel != SSM_KERNEL_SCAN_BAL) ++fails;
+
+    /* the workspace the balanced prefill asks for, then the plan that uses it */
+    uint64_t need = 0;
+    st = ssm_selective_scan_workspace_size(&a, &need);
+    printf("scan workspace %s %llu bytes\n", ssm_status_string(st), (unsigned long long)need);
+    if (st != SSM_OK || need == 0) ++fails;
+    a.workspace = (void*)next_addr;
+    next_addr += (uintptr_t)1 << 36;
+    a.workspace_bytes = need;
+    st = ssm_selective_scan_fwd(&a, NULL);
+    printf("scan with workspace %s grid %d\n", ssm_status_string(st), info.grid);
+    if (st != SSM_OK || info.kernel != SSM_KERNEL_SCAN_BAL) ++fails;
+    a.workspace_bytes = need - 1;
+    if (ssm_selective_scan_fwd(&a, NULL) != SSM_ERR_WORKSPACE) ++fails;
+    a.workspace = NULL;
+    a.workspace_bytes = 0;
 
     /* error paths: wrong struct size, NULL args, output aliasing an input */
     a.struct_size = sizeof a - 8;

@@ -21,12 +21,49 @@ def rel_l2(got, ref) -> float:
     return float(num / den) if den > 0 else float(num)
 
 
-def assert_close(got, ref, tol, what=""):
+# significand bits (with the implicit one) and smallest normal exponent of
+# the storage dtypes an output can come back in
+_FORMATS = (("bf16", 8, -126), ("f16", 11, -14), ("f32", 24, -126))
+
+
+def storage_ulp(got, ref):
+    """A unit in the last place, at |ref|, of the coarsest storage dtype in
+    which every value of `got` is exactly representable (bf16, fp16 or fp32;
+    0 for anything finer)."""
+    g = np.asarray(got, np.float64)
+    for name, bits, emin in _FORMATS:
+        if np.array_equal(gen.round_to(g, name), g, equal_nan=True):
+            e = np.floor(np.log2(np.maximum(np.abs(np.asarray(ref, np.float64)), 2.0 ** emin)))
+            return 2.0 ** (e - (bits - 1))
+    return 0.0
+
+
+def assert_close(got, ref, tol, what="", ulps=0.5):
+    """rel-L2 over the whole tensor <= tol (the acceptance bound), and every
+    element within tol * (|ref| + rms(ref)) plus `ulps` units in the last place
+    of the dtype the output is stored in, so that a wrong tile or tail cannot
+    hide in the norm of a large tensor.  One stored rounding is half an ulp;
+    a cache that both sides round to its dtype after each of k steps can
+    drift apart by up to one ulp per step (each step adds one rounding on
+    either side to the decayed earlier difference), so such comparisons pass
+    ulps=k."""
     err = rel_l2(got, ref)
+    g = np.asarray(got, np.float64)
+    r = np.asarray(ref, np.float64)
+    diff = np.abs(g - r)
     if not err <= tol:
-        diff = np.abs(np.asarray(got, np.float64) - np.asarray(ref, np.float64))
         i = np.unravel_index(np.argmax(diff), diff.shape)
         raise AssertionError(f"{what}: rel-L2 {err:.3e} > {tol:.1e}; max |diff| {diff[i]:.3e} at {i}")
+    if r.size:
+        rms = float(np.sqrt(np.mean(r * r)))
+        bound = tol * (np.abs(r) + rms) + ulps * storage_ulp(g, r)
+        bad = ~(diff <= bound)
+        if bad.any():
+            ratio = np.where(bad, diff / np.maximum(bound, 1e-300), 0.0)
+            i = np.unravel_index(np.argmax(ratio), ratio.shape)
+            raise AssertionError(f"{what}: element {i} off by {diff[i]:.3e} > {bound[i]:.3e} "
+                                 f"(= tol * (|ref| + rms) + {ulps} ulp), got {g[i]!r} want {r[i]!r}; "
+                                 f"{int(bad.sum())} such elements; rel-L2 {err:.3e}")
     return err
 
 

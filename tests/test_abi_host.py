@@ -18,7 +18,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "ssm_causal.h")
 
 F32, F16, BF16, I32 = bd.SSM_F32, bd.SSM_F16, bd.SSM_BF16, bd.SSM_I32
-OK, ENULL, ESHAPE, EDTYPE, ESTRIDE, EUNSUP, ECUDA, EINT, EVER, EALIAS = range(10)
+OK, ENULL, ESHAPE, EDTYPE, ESTRIDE, EUNSUP, ECUDA, EINT, EVER, EALIAS, EWORKSPACE = range(11)
 
 
 @pytest.fixture(scope="module")
@@ -45,10 +45,29 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_struct_layouts(lib):
-    assert lib.ssm_abi_version() == 1
-    for which, st in enumerate((bd.Tensor, bd.Conv1dArgs, bd.ScanArgs, bd.SsuArgs, bd.LaunchInfo)):
+    assert lib.ssm_abi_version() == 2
+    for which, st in enumerate((bd.Tensor, bd.Conv1dArgs, bd.ScanArgs, bd.SsuArgs, bd.LaunchInfo,
+                                bd.ErrorReport)):
         assert lib.ssm_struct_size(which) == ctypes.sizeof(st)
     assert lib.ssm_struct_size(99) == 0
+
+
+def test_failure_test_wait_budget_has_a_floor(lib):
+    """A failure test may shorten the bounded waits, never below 10^7 cycles
+    (~5 ms), so a wait for copies still in flight cannot be cut short; the
+    clean-up wait after a give-up always uses the full budget."""
+    assert lib.ssm_test_clamp_wait_budget(1) == 10_000_000
+    assert lib.ssm_test_clamp_wait_budget(0) == 10_000_000
+    assert lib.ssm_test_clamp_wait_budget(20_000_000) == 20_000_000
+    test_lib = bd._open(bd.TESTHOOKS_LIB_PATH)
+    assert test_lib.ssm_test_clamp_wait_budget(5) == 10_000_000
+
+
+def test_error_report_checks_its_arguments(lib):
+    assert lib.ssm_device_error_info(None, None) == ENULL
+    rep = bd.ErrorReport()
+    rep.struct_size = 3
+    assert lib.ssm_device_error_info(ctypes.byref(rep), None) == EVER
 
 
 def test_status_strings(lib):
@@ -163,11 +182,63 @@ def call(lib, fn, args):
 
 # ------------------------------------------------------------- valid plans --
 def test_prefill_2p8b_plan(lib):
+    """Without a workspace every warp takes whole (batch, 16-channel) units:
+    1280 units, 4 warps per CTA."""
     st, info = call(lib, "ssm_selective_scan_fwd", scan_args(FakeMem()))
     assert st == OK
-    assert bd.KERNELS[info.kernel] == "scan_vec"
-    assert info.block == 32 and info.rows_per_item == 16
-    assert info.grid == 4 * 5120 // 16
+    assert bd.KERNELS[info.kernel] == "scan_bal"
+    assert info.block == 128 and info.rows_per_item == 16
+    assert info.work_items == 4 * 5120 // 16
+    assert info.grid == 4 * 5120 // 16 // 4
+
+
+def ws_bytes(workers):
+    """256-byte header, one 32-bit flag per worker rounded up to 256 bytes,
+    one 1 KB hand-over state (16 channels x 16 state entries) per worker."""
+    return 256 + (workers * 4 + 255) // 256 * 256 + workers * 1024
+
+
+def test_prefill_workspace_size_and_balanced_plan(lib):
+    """1280 units > 148 SMs x 2 CTAs x 4 warps = 1184 resident warps: the
+    dry-run plan asks for the hand-over workspace and, given one, runs
+    exactly one persistent wave of 296 CTAs."""
+    mem = FakeMem()
+    a = scan_args(mem)
+    need = ctypes.c_uint64(0)
+    assert lib.ssm_selective_scan_workspace_size(ctypes.byref(a), ctypes.byref(need)) == OK
+    assert need.value == ws_bytes(1184)
+    a.workspace, a.workspace_bytes = mem.next, need.value
+    mem.next += 1 << 36
+    st, info = call(lib, "ssm_selective_scan_fwd", a)
+    assert st == OK and bd.KERNELS[info.kernel] == "scan_bal"
+    assert info.grid == 148 * 2 and info.work_items == 1280
+    assert lib.ssm_selective_scan_workspace_size(ctypes.byref(a), None) == ENULL
+
+
+def test_prefill_small_problem_needs_no_workspace(lib):
+    mem = FakeMem()
+    a = scan_args(mem, Bn=1, D=5120)  # 320 units fit in one wave
+    need = ctypes.c_uint64(123)
+    assert lib.ssm_selective_scan_workspace_size(ctypes.byref(a), ctypes.byref(need)) == OK
+    assert need.value == 0
+    a = scan_args(mem, Bn=2, D=64, L=100)  # chunked kernel
+    assert lib.ssm_selective_scan_workspace_size(ctypes.byref(a), ctypes.byref(need)) == OK
+    assert need.value == 0
+
+
+def test_prefill_workspace_errors(lib):
+    mem = FakeMem()
+    need = ws_bytes(1184)
+    a = scan_args(mem)
+    a.workspace, a.workspace_bytes = mem.next, need - 1
+    mem.next += 1 << 36
+    assert call(lib, "ssm_selective_scan_fwd", a)[0] == EWORKSPACE   # too small
+    a.workspace, a.workspace_bytes = mem.next + 16, need
+    assert call(lib, "ssm_selective_scan_fwd", a)[0] == EWORKSPACE   # not 256-byte aligned
+    a.workspace, a.workspace_bytes = a.out.data, need
+    assert call(lib, "ssm_selective_scan_fwd", a)[0] == EALIAS       # overlaps the output
+    a.workspace, a.workspace_bytes = a.A.data - 256, need
+    assert call(lib, "ssm_selective_scan_fwd", a)[0] == EALIAS       # overlaps A
 
 
 def test_unaligned_or_odd_prefill_layouts_use_the_chunked_kernel(lib):
@@ -187,7 +258,7 @@ def test_unaligned_or_odd_prefill_layouts_use_the_chunked_kernel(lib):
 def test_small_scan_plan_and_generic_for_large_state(lib):
     mem = FakeMem()
     st, info = call(lib, "ssm_selective_scan_fwd", scan_args(mem, Bn=1, D=64, L=128, W=0, io=F32))
-    assert st == OK and bd.KERNELS[info.kernel] == "scan_vec"
+    assert st == OK and bd.KERNELS[info.kernel] == "scan_bal"
     st, info = call(lib, "ssm_selective_scan_fwd", scan_args(mem, Bn=1, D=8, L=16, N=128, W=0))
     assert st == OK and bd.KERNELS[info.kernel] == "scan_generic"
 
@@ -195,7 +266,7 @@ def test_small_scan_plan_and_generic_for_large_state(lib):
 def test_scan_groups_choose_generic_when_tile_straddles_groups(lib):
     mem = FakeMem()
     st, info = call(lib, "ssm_selective_scan_fwd", scan_args(mem, Bn=1, D=64, L=8, G=4))
-    assert st == OK and bd.KERNELS[info.kernel] == "scan_vec"  # 16 channels per group
+    assert st == OK and bd.KERNELS[info.kernel] == "scan_bal"  # 16 channels per group
     st, info = call(lib, "ssm_selective_scan_fwd", scan_args(mem, Bn=1, D=24, L=8, G=3))
     assert st == OK and bd.KERNELS[info.kernel] == "scan_generic"  # 8 channels per group
 

@@ -1,13 +1,17 @@
 """Failure detection on the GPU without a GPU fault.
 
 The bulk-copy state-update kernels give up a wait on a shared-memory stage
-after a cycle budget, set the library's device error word and exit; the host
-reads the word with ssm_device_error().  These tests make one wait run out
-on purpose: SSM_TEST_DROP_ITEM names a work item whose copies are never
+after a cycle budget, record it in the library's device error record and
+exit; the host reads it with ssm_device_error() / ssm_device_error_info().
+These tests make one wait run out on purpose, through the failure-test build
+of the library (libssm_causal_testhooks.so, the only build that reads the
+switches): SSM_TEST_DROP_ITEM names a work item whose copies are never
 started (a flag that nothing sets) and SSM_TEST_WAIT_CYCLES shortens the
-budget to about 10 ms.  The call must return without a CUDA error, the error
-word must read 1 once and then 0, and the context must stay usable: the next
-call, without the switches, matches the oracle."""
+budget to about 10 ms.  The call must return without a CUDA error, the record
+must name the kernel and the dropped item as the first unfinished one, read
+once and then clear, and the context must stay usable: the next call,
+without the switches, matches the oracle.  The product library, given the
+same switches, ignores them."""
 import os
 
 import numpy as np
@@ -37,18 +41,20 @@ class _env:
                 os.environ[k] = v
 
 
-def _expect_timeout_then_clean(run_dropped, run_clean, check):
+def _expect_timeout_then_clean(run_dropped, run_clean, check, kernel):
     import torch
-    from state_space_model_causal_b200 import LaunchInfo, ssm_device_error
-    assert ssm_device_error() == 0
+    from state_space_model_causal_b200 import LaunchInfo, binding, ssm_device_error, ssm_device_error_info
     info = LaunchInfo()
-    with _env(SSM_TEST_DROP_ITEM="5", SSM_TEST_WAIT_CYCLES="20000000"):
-        run_dropped(info)
-        torch.cuda.synchronize()  # no CUDA error: the kernel returned
-    assert ssm_device_error() == 1
-    assert ssm_device_error() == 0  # read and cleared
-    check(run_clean())
-    assert ssm_device_error() == 0
+    with binding.using_library(binding.TESTHOOKS_LIB_PATH):
+        assert ssm_device_error() == 0
+        with _env(SSM_TEST_DROP_ITEM="5", SSM_TEST_WAIT_CYCLES="20000000"):
+            run_dropped(info)
+            torch.cuda.synchronize()  # no CUDA error: the kernel returned
+        rep = ssm_device_error_info()
+        assert rep == {"code": 1, "kernel": kernel, "first_item": 5}, rep
+        assert ssm_device_error() == 0  # read and cleared
+        check(run_clean())
+        assert ssm_device_error() == 0
     return info
 
 
@@ -62,7 +68,7 @@ def test_mamba1_bulk_copy_wait_runs_out_and_is_reported():
         assert_close(N(st), sref, TOL["f16"], "state")
         np.testing.assert_array_equal(N(cs), csref)
 
-    info = _expect_timeout_then_clean(lambda info: _m1_gpu(s), lambda: _m1_gpu(s), check)
+    info = _expect_timeout_then_clean(lambda info: _m1_gpu(s), lambda: _m1_gpu(s), check, "ssu_row_tma")
     assert info is not None
 
 
@@ -75,7 +81,22 @@ def test_mamba2_bulk_copy_wait_runs_out_and_is_reported():
         assert_close(N(out), o, TOL["f16"], "out")
         assert_close(N(st), sref, TOL["f16"], "state")
 
-    _expect_timeout_then_clean(lambda info: _m2_gpu(s), lambda: _m2_gpu(s), check)
+    _expect_timeout_then_clean(lambda info: _m2_gpu(s), lambda: _m2_gpu(s), check, "ssu_tma")
+
+
+def test_product_library_ignores_the_failure_test_switches():
+    """The shipped library never reads SSM_TEST_*: with the switches set the
+    update completes, matches the oracle and leaves the record clear."""
+    import torch
+    from state_space_model_causal_b200 import ssm_device_error
+    s = gen.ssu_mamba2_inputs(16, 8, 64, 128, io="f16", state="f16", seed=23, tag="fail3")
+    with _env(SSM_TEST_DROP_ITEM="5", SSM_TEST_WAIT_CYCLES="20000000"):
+        out, st = _m2_gpu(s)
+        torch.cuda.synchronize()
+    assert ssm_device_error() == 0
+    o, sref = _m2_oracle(s)
+    assert_close(N(out), o, TOL["f16"], "out")
+    assert_close(N(st), sref, TOL["f16"], "state")
 
 
 def test_the_kernels_under_test_are_the_bulk_copy_ones():

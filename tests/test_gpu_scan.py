@@ -120,26 +120,24 @@ def test_scan_empty_sequence_leaves_caches_unchanged():
     np.testing.assert_array_equal(N(cs), s.conv_state)
 
 
-def test_prefill_2p8b_full_size_sampled_channels():
+def test_prefill_2p8b_full_size_every_channel():
     """Full 2.8B-shaped prefill (B=4, L=2048, D=5120, N=16, W=4, fp16) in the
-    launch configuration the benchmark times; 48 sampled channels are checked
-    against the oracle one by one."""
+    launch configuration the benchmark times (balanced slices with hand-overs
+    through the workspace); every one of the 20480 channels is compared with
+    the oracle: outputs and final states by rel-L2 and element by element,
+    final conv states exactly."""
     import torch
     s = gen.prefill_2p8b(seed=0)
     out, h, cs = run_scan_gpu(s)
-    rng = np.random.default_rng(123)
-    picks = [(int(b), int(d)) for b, d in zip(rng.integers(0, 4, 48), rng.integers(0, 5120, 48))]
-    picks += [(0, 0), (3, 5119)]
-    for b, d in picks:
-        sub = gen.ScanInputs(s.x[b:b + 1, d:d + 1], s.dt[b:b + 1, d:d + 1], s.A[d:d + 1],
-                             s.B[b:b + 1], s.C[b:b + 1], s.D[d:d + 1], s.z[b:b + 1, d:d + 1],
-                             s.dt_bias[d:d + 1], s.conv_weight[d:d + 1], s.conv_bias[d:d + 1],
-                             None, None, io="f16")
-        ref, href, csref = run_scan_oracle(sub)
-        assert_close(out[b:b + 1, d:d + 1], ref, TOL["f16"], f"out[{b},{d}]")
-        assert_close(h[b:b + 1, d:d + 1], href, TOL["f16"], f"state[{b},{d}]")
-        np.testing.assert_array_equal(cs[b, d], csref[0, 0])
-    assert np.isfinite(out).all()
+    ref, href, csref = run_scan_oracle(s)
+    assert_close(out, ref, TOL["f16"], "out")
+    assert_close(h, href, TOL["f16"], "ssm_state")
+    np.testing.assert_array_equal(cs, csref)
+    # per channel too, so that one bad unit cannot hide in the whole tensor
+    num = np.linalg.norm((out - ref).reshape(4 * 5120, -1), axis=1)
+    den = np.linalg.norm(ref.reshape(4 * 5120, -1), axis=1)
+    worst = int(np.argmax(num / den))
+    assert (num / den).max() <= TOL["f16"], f"channel {divmod(worst, 5120)}: {(num / den).max():.3e}"
     torch.cuda.empty_cache()
 
 

@@ -333,3 +333,58 @@ def test_mamba1_slot_indices_with_padding_rows():
     for slot in (1, 2, 4):
         np.testing.assert_array_equal(got_st[slot], pool.state[slot])
         np.testing.assert_array_equal(got_cs[slot], pool.conv_state[slot])
+
+
+# ------------------------------------------------- several steps, 16-bit caches --
+@pytest.mark.parametrize("cache,io,P,N_", [("f16", "f16", 64, 128), ("bf16", "bf16", 128, 256)])
+def test_mamba2_multi_step_decode_16bit_cache(cache, io, P, N_):
+    """Eight consecutive decode steps on one fp16 / bf16 cache.  The GPU stores
+    the state rounded to the cache dtype after every step; the oracle rounds
+    its fp64 state the same way (cache_dtype), so outputs and the cache stay
+    comparable step after step."""
+    import torch
+    s = gen.ssu_mamba2_inputs(4, 8, P, N_, io=io, state=cache, seed=41, tag=f"steps{cache}", with_z=True)
+    st = T(s.state, cache)
+    sref = s.state
+    for k in range(8):
+        tg = ("steps16", cache, k)
+        x = gen.round_to(gen.normal((4, 8, P), *tg, "x"), io)
+        dt = gen.round_to(gen.uniform((4, 8), -4.0, -1.0, *tg, "dt"), io)
+        Bm = gen.round_to(gen.normal((4, 1, N_), *tg, "B"), io)
+        Cm = gen.round_to(gen.normal((4, 1, N_), *tg, "C"), io)
+        z = gen.round_to(gen.normal((4, 8, P), *tg, "z"), io)
+        out = _ssu(state=st, x=T(x, io), dt=T(dt, io), A=T(s.A, "f32"), B=T(Bm, io), C=T(Cm, io),
+                   D=T(s.D, "f32"), z=T(z, io), dt_bias=T(s.dt_bias, "f32"))
+        torch.cuda.synchronize()
+        o, sref = oracle.ssu_mamba2(sref, x, dt, s.A, Bm, Cm, D=s.D, z=z, dt_bias=s.dt_bias,
+                                    cache_dtype=cache)
+        assert_close(N(out), o, TOL[io], f"out step {k}")
+        assert_close(N(st), sref, TOL[io], f"cache after step {k}", ulps=k + 1)
+
+
+@pytest.mark.parametrize("cache", ["f16", "bf16"])
+def test_mamba1_multi_step_decode_16bit_cache(cache):
+    """Six consecutive Mamba-1 decode steps (fused conv roll) on a 16-bit ssm
+    cache, compared step by step with the oracle rounding its state the same way."""
+    import torch
+    io = cache
+    s = gen.ssu_mamba1_inputs(9, 64, 16, W=4, io=io, state=cache, seed=42, tag=f"m1steps{cache}")
+    st = T(s.state, cache)
+    cs = T(s.conv_state, "f32")
+    sref, csref = s.state, s.conv_state
+    for k in range(6):
+        tg = ("m1steps16", cache, k)
+        x = gen.round_to(gen.normal((9, 64), *tg, "x"), io)
+        dt = gen.round_to(gen.uniform((9, 64), -4.0, -1.0, *tg, "dt"), io)
+        out = _ssu(state=st, x=T(x, io), dt=T(dt, io), A=T(s.A, "f32"), B=T(s.B, io), C=T(s.C, io),
+                   D=T(s.D, "f32"), z=T(s.z, io), dt_bias=T(s.dt_bias, "f32"),
+                   conv_weight=T(s.conv_weight, "f32"), conv_bias=T(s.conv_bias, "f32"), conv_state=cs)
+        torch.cuda.synchronize()
+        o, st_ref, cs_ref = oracle.ssu(sref[:, :, None, :], x[:, :, None], dt[:, :, None], s.A[:, None, :],
+                                       s.B, s.C, D=s.D[:, None], z=s.z[:, :, None],
+                                       dt_bias=s.dt_bias[:, None], conv_weight=s.conv_weight,
+                                       conv_bias=s.conv_bias, conv_state=csref, cache_dtype=cache)
+        sref, csref = st_ref[:, :, 0], cs_ref.reshape(9, 64, -1)
+        assert_close(N(out), o[:, :, 0], TOL[io], f"out step {k}")
+        assert_close(N(st), sref, TOL[io], f"cache after step {k}", ulps=k + 1)
+    np.testing.assert_array_equal(N(cs), csref)
