@@ -268,6 +268,32 @@ ssm_status ssm_selective_scan_fwd(const ssm_scan_args* args, void* stream);
  * SSM_ERR_WORKSPACE.  Returns SSM_ERR_NULL for a NULL `bytes`. */
 ssm_status ssm_selective_scan_workspace_size(const ssm_scan_args* args, uint64_t* bytes);
 
+/* ssm_selective_scan_fwd_noalloc -- the same prefill as ssm_selective_scan_fwd
+ * for callers that cannot allocate device memory.  It has no counterpart in
+ * the method's description: it exists for callers such as a plugin or
+ * custom-operator interface that is handed its input and output tensors but
+ * no allocator, or a serving loop that must not allocate once it is running
+ * (an allocation there can synchronise the device, fail under memory
+ * pressure, or is simply not permitted).  Such callers cannot provide the
+ * hand-over workspace of the fast prefill.
+ *
+ * The call takes the same arguments as ssm_selective_scan_fwd, with workspace
+ * NULL and workspace_bytes 0 (else SSM_ERR_WORKSPACE), and computes the same
+ * results.  The scratch it needs comes from a fixed 2 MiB device array inside
+ * the library, which every GPU that loads the library holds until the
+ * process exits; a problem that would need more than 2 MiB of scratch is
+ * rejected with SSM_ERR_WORKSPACE before anything is launched (the prefill
+ * needs 256 bytes + 1 KB and 4 bytes per resident warp: about 1.2 MB on a
+ * B200).  It calls no allocating routine: the first call on a device looks
+ * up that array's device address (once per device, kept for later calls), so
+ * make that first call before any stream capture; every call then clears the
+ * array's header and flags with an asynchronous memset on `stream` before
+ * the prefill kernel.  All calls on a device share the one array and find it
+ * as the previous call left it, so two calls whose work overlaps on the GPU
+ * (for example on two streams) race and their results are undefined: order
+ * them on one stream. */
+ssm_status ssm_selective_scan_fwd_noalloc(const ssm_scan_args* args, void* stream);
+
 /* ------------------------------------------------------------------------ *
  * ssm_selective_state_update -- one decode token, caches updated in place.
  *

@@ -7,4 +7,5 @@ they raise if the library has not been built (there is no fallback path).
 """
 from .binding import (LaunchInfo, SsmError, library, ssm_causal_conv1d_fwd,  # noqa: F401
                       ssm_device_error, ssm_device_error_info, ssm_selective_scan_fwd,
+                      ssm_selective_scan_fwd_noalloc,
                       ssm_selective_scan_workspace_size, ssm_selective_state_update)

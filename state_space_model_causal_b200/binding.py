@@ -148,6 +148,8 @@ def _open(path):
         fn = getattr(lib, name)
         fn.restype = ctypes.c_int
         fn.argtypes = [ctypes.POINTER(argt), ctypes.c_void_p]
+    lib.ssm_selective_scan_fwd_noalloc.restype = ctypes.c_int
+    lib.ssm_selective_scan_fwd_noalloc.argtypes = [ctypes.POINTER(ScanArgs), ctypes.c_void_p]
     lib.ssm_selective_scan_workspace_size.restype = ctypes.c_int
     lib.ssm_selective_scan_workspace_size.argtypes = [ctypes.POINTER(ScanArgs),
                                                       ctypes.POINTER(ctypes.c_uint64)]
@@ -250,6 +252,28 @@ def _info_ptr(info: Optional[LaunchInfo]):
 
 
 # ------------------------------------------------------------ entry points --
+def ssm_selective_scan_fwd_noalloc(x, dt, A, B, C, D=None, z=None, dt_bias=None, dt_softplus=True,
+                                   conv_weight=None, conv_bias=None, conv_state=None, ssm_state=None,
+                                   out=None, stream=None, info: Optional[LaunchInfo] = None):
+    """The prefill of ssm_selective_scan_fwd for callers that cannot allocate
+    device memory: the scratch comes from the library's fixed device array
+    (see include/ssm_causal.h).  `out` must be given: this call allocates
+    nothing, not even its output."""
+    if out is None:
+        raise ValueError("ssm_selective_scan_fwd_noalloc allocates nothing: pass `out`")
+    a = ScanArgs()
+    a.struct_size = ctypes.sizeof(ScanArgs)
+    (a.x, a.dt, a.A, a.B, a.C, a.D, a.z, a.dt_bias, a.conv_weight, a.conv_bias, a.conv_state,
+     a.ssm_state, a.out) = map(describe, (x, dt, A, B, C, D, z, dt_bias, conv_weight, conv_bias,
+                                          conv_state, ssm_state, out))
+    a.dt_softplus = int(bool(dt_softplus))
+    a.info = _info_ptr(info)
+    _check(_run(library().ssm_selective_scan_fwd_noalloc, a,
+                (x, dt, A, B, C, D, z, dt_bias, conv_weight, conv_bias, conv_state, ssm_state, out), stream),
+           "ssm_selective_scan_fwd_noalloc")
+    return out
+
+
 def ssm_selective_scan_workspace_size(x, dt, A, B, C, D=None, z=None, dt_bias=None,
                                       dt_softplus=True, conv_weight=None, conv_bias=None,
                                       conv_state=None, ssm_state=None, out=None) -> int:

@@ -1099,6 +1099,33 @@ ssm_status ssm_selective_scan_fwd(const ssm_scan_args* args, void* stream) {
     return scan_impl(args, static_cast<cudaStream_t>(stream), nullptr);
 }
 
+ssm_status ssm_selective_scan_fwd_noalloc(const ssm_scan_args* args, void* stream) {
+    if (!args) return SSM_ERR_NULL;
+    if (args->struct_size != sizeof(ssm_scan_args)) return SSM_ERR_VERSION;
+    // the scratch is the library's own fixed array: no caller workspace
+    if (args->workspace || args->workspace_bytes) return SSM_ERR_WORKSPACE;
+    // check the arguments and size the scratch exactly as the workspace query does
+    uint64_t need = 0;
+    SSM_TRY(scan_impl(args, static_cast<cudaStream_t>(stream), &need));
+    if (need > kStaticWorkspaceBytes) return SSM_ERR_WORKSPACE;
+    ssm_scan_args a = *args;
+    if (need > 0 && !(args->flags & SSM_FLAG_DRY_RUN)) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess) return SSM_ERR_CUDA;
+        void* ws = scan_static_workspace(dev);
+        if (!ws) return SSM_ERR_CUDA;
+        // The array keeps whatever the last call left.  The header and the
+        // hand-over flags must start at zero: clear them on the call's stream
+        // (the hand-over states behind them are written before they are read).
+        const uint64_t flags_max = bal_flag_bytes((int64_t)(kStaticWorkspaceBytes / 1024));
+        if (cudaMemsetAsync(ws, 0, 256 + flags_max, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+            return SSM_ERR_CUDA;
+        a.workspace = ws;
+        a.workspace_bytes = kStaticWorkspaceBytes;
+    }
+    return scan_impl(&a, static_cast<cudaStream_t>(stream), nullptr);
+}
+
 ssm_status ssm_selective_scan_workspace_size(const ssm_scan_args* args, uint64_t* bytes) {
     if (!bytes) return SSM_ERR_NULL;
     return scan_impl(args, nullptr, bytes);

@@ -165,6 +165,10 @@ int scan_bal_steps_per_chunk();
 int scan_bal_warps_per_cta();
 int scan_bal_smem_bytes(int io_dt);
 int scan_bal_ctas_per_sm(const ScanProblem& p, int sw, int dev);
+// Size of the fixed device array behind ssm_selective_scan_fwd_noalloc, and
+// its device address on device `dev` (the current device; NULL on failure).
+constexpr unsigned long long kStaticWorkspaceBytes = 2ull << 20;
+void* scan_static_workspace(int dev);
 cudaError_t launch_scan_bal(const ScanProblem& p, const BalPlan& bp, cudaStream_t s, int dev);
 cudaError_t launch_scan(const ScanProblem& p, const ScanPlan& plan, cudaStream_t s);
 bool scan_vec_supported(const ScanProblem& p);

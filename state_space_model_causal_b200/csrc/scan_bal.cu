@@ -694,6 +694,26 @@ cudaError_t dispatch(const ScanProblem& p, const BalPlan& bp, cudaStream_t s, in
 
 }  // namespace
 
+// ---------------------------------------------------------------------------
+// Allocation-free variant: the hand-over scratch lives in this fixed device
+// array instead of a caller-supplied workspace.  It is zero at module load,
+// every device that loads the library holds its own copy until the process
+// exits, and all calls on a device share it.  Host code may not use the
+// array's name as an address (it names a host-side stand-in): the device
+// address is obtained with cudaGetSymbolAddress, once per device, with that
+// device current.
+static __device__ __align__(256) unsigned char g_scan_static_ws[kStaticWorkspaceBytes];
+
+void* scan_static_workspace(int dev) {
+    static std::atomic<void*> cache[kMaxDevices];
+    if (dev < 0 || dev >= kMaxDevices) return nullptr;
+    void* ptr = cache[dev].load(std::memory_order_acquire);
+    if (ptr) return ptr;
+    if (cudaGetSymbolAddress(&ptr, g_scan_static_ws) != cudaSuccess || !ptr) return nullptr;
+    cache[dev].store(ptr, std::memory_order_release);
+    return ptr;
+}
+
 bool scan_bal_supported(const ScanProblem& p) {
     return p.N <= 16 && (p.W == 0 || p.W == 4) && p.L % 8 == 0 && (p.G == 1 || p.ch_per_group % kCH == 0);
 }
