@@ -225,6 +225,35 @@ __device__ __forceinline__ u64 exp2_pair_sfu(u64 x) {
     return pk(ex2_approx(x0), ex2_approx(x1));
 }
 
+// 1/d for a pair of d >= 1 (up to +inf) on the FMA pipe, so that the SFU
+// keeps its issue slots for the exponentials.  Newton's iteration for the
+// reciprocal, r <- r + r (1 - d r), from the integer-subtraction seed
+// r0 = as_float(K - bits(d)): K = 0x7ef311c2 was chosen here by a search that
+// minimises the seed's relative error over a binade (5.1%); each step squares
+// the relative error, so two steps leave < 7e-6 and three reach fp32 rounding
+// (~1 ulp).  d is clamped to 2^125 first, so the seed stays a normal number
+// and 1/d tends to 0 as d grows.
+template <int STEPS>
+__device__ __forceinline__ u64 rcp_pair_fma(u64 d) {
+    float d0, d1;
+    upk(d, d0, d1);
+    d0 = fminf(d0, 4.2535295865117308e37f);  // 2^125
+    d1 = fminf(d1, 4.2535295865117308e37f);
+    u64 r = pk(__int_as_float(0x7ef311c2 - __float_as_int(d0)), __int_as_float(0x7ef311c2 - __float_as_int(d1)));
+    const u64 nd = pk(-d0, -d1);
+#pragma unroll
+    for (int k = 0; k < STEPS; ++k) r = ffma2(r, ffma2(nd, r, pk(1.0f, 1.0f)), r);
+    return r;
+}
+
+// SiLU on a pair, v / (1 + 2^(-v log2 e)): one SFU exponential per value,
+// the reciprocal on the FMA pipe.
+template <int STEPS>
+__device__ __forceinline__ u64 silu_pair(u64 v) {
+    const u64 den = fadd2(exp2_pair_sfu(fmul2(v, pk(-kLog2e, -kLog2e))), pk(1.0f, 1.0f));
+    return fmul2(v, rcp_pair_fma<STEPS>(den));
+}
+
 __device__ __forceinline__ float exp_fast(float x) { return ex2_approx(x * kLog2e); }
 
 // SiLU(v) = v * sigmoid(v) = v / (1 + e^-v).  For v -> -inf the quotient

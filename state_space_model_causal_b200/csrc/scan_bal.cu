@@ -127,6 +127,13 @@ __device__ __forceinline__ void row8(const IoT* row, int r, int s0, float* f) {
     }
 }
 
+// Four consecutive B or C values of a [t][n] row as two packed fp32 pairs.
+__device__ __forceinline__ void bc4(const float* row, u64* pr) {
+    const float4 v = *reinterpret_cast<const float4*>(row);
+    pr[0] = pk(v.x, v.y);
+    pr[1] = pk(v.z, v.w);
+}
+
 // Parameters of the channel whose prologue a lane computes.
 template <int W> struct BalChan {
     float w[W > 0 ? W : 1];
@@ -138,6 +145,9 @@ template <int W> struct BalChan {
 template <typename IoT, int W, int SW, bool SP, bool HZ>
 __global__ void __launch_bounds__(32 * kWarps, 2) scan_bal_kernel(const ScanProblem p, const BalPlan bp) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
+    // Newton steps of the SiLU reciprocals: 2 (< 7e-6 relative) for 16-bit
+    // outputs, 3 (fp32 rounding) for fp32 outputs
+    constexpr int kRcpSteps = sizeof(IoT) == 2 ? 2 : 3;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int64_t w = (int64_t)blockIdx.x * kWarps + warp;
@@ -409,14 +419,18 @@ __global__ void __launch_bounds__(32 * kWarps, 2) scan_bal_kernel(const ScanProb
                 for (int i = 0; i < W - 1; ++i)
                     ch.hist[i] = __shfl_sync(0xffffffffu, xs[kSPL - (W - 1) + i], lane | 2);
 #pragma unroll
-                for (int i = 0; i < kSPL; ++i) {
-                    float acc = ch.cbias;
+                for (int i = 0; i < kSPL; i += 2) {
+                    float acc[2];
 #pragma unroll
-                    for (int kk = 0; kk < W; ++kk) {
-                        const int j = i - (W - 1) + kk;
-                        acc = fmaf(ch.w[kk], j >= 0 ? xs[j] : prev[W - 1 + j], acc);
+                    for (int s1 = 0; s1 < 2; ++s1) {
+                        acc[s1] = ch.cbias;
+#pragma unroll
+                        for (int kk = 0; kk < W; ++kk) {
+                            const int j = i + s1 - (W - 1) + kk;
+                            acc[s1] = fmaf(ch.w[kk], j >= 0 ? xs[j] : prev[W - 1 + j], acc[s1]);
+                        }
                     }
-                    uu[i] = silu_f(acc);
+                    upk(silu_pair<kRcpSteps>(pk(acc[0], acc[1])), uu[i], uu[i + 1]);
                 }
             } else {
 #pragma unroll
@@ -474,13 +488,7 @@ __global__ void __launch_bounds__(32 * kWarps, 2) scan_bal_kernel(const ScanProb
                 const u64 Du2 = fmul2(pk(ch.dskip, ch.dskip), pk(uu[i], uu[i + 1]));
                 upk(Du2, Du[i], Du[i + 1]);
                 if constexpr (HZ) {
-                    // SiLU(z) = z / (1 + 2^(-z log2 e)) on a pair
-                    const u64 den = fadd2(exp2_pair_sfu(fmul2(pk(zs[i], zs[i + 1]), pk(-kLog2e, -kLog2e))),
-                                          pk(1.0f, 1.0f));
-                    float d0, d1;
-                    upk(den, d0, d1);
-                    const u64 g2 = fmul2(pk(zs[i], zs[i + 1]), pk(__fdividef(1.0f, d0), __fdividef(1.0f, d1)));
-                    upk(g2, gate[i], gate[i + 1]);
+                    upk(silu_pair<kRcpSteps>(pk(zs[i], zs[i + 1])), gate[i], gate[i + 1]);
                 } else {
                     gate[i] = gate[i + 1] = 1.0f;
                 }
@@ -495,17 +503,19 @@ __global__ void __launch_bounds__(32 * kWarps, 2) scan_bal_kernel(const ScanProb
         // this step's partials are stored, so that the loads (and the
         // exponentials behind them) are not held back behind the stores.
         {
+            using RawT = float4;
             float4 d4 = sm.dd[cp][dd_at(0)];  // (dl0, du0, dl1, du1)
-            float4 bq = *reinterpret_cast<const float4*>(&sm.bf[0][4 * q]);
-            float4 cq = *reinterpret_cast<const float4*>(&sm.cf[0][4 * q]);
+            RawT bq = *reinterpret_cast<const RawT*>(&sm.bf[0][4 * q]);
+            RawT cq = *reinterpret_cast<const RawT*>(&sm.cf[0][4 * q]);
 #pragma unroll 4
             for (int t = 0; t < kT; ++t) {
                 const int tn = t + 1 < kT ? t + 1 : t;
                 const float4 d4n = sm.dd[cp][dd_at(tn)];
-                const float4 bqn = *reinterpret_cast<const float4*>(&sm.bf[tn][4 * q]);
-                const float4 cqn = *reinterpret_cast<const float4*>(&sm.cf[tn][4 * q]);
-                const u64 Bp[2] = {pk(bq.x, bq.y), pk(bq.z, bq.w)};
-                const u64 Cp[2] = {pk(cq.x, cq.y), pk(cq.z, cq.w)};
+                const RawT bqn = *reinterpret_cast<const RawT*>(&sm.bf[tn][4 * q]);
+                const RawT cqn = *reinterpret_cast<const RawT*>(&sm.cf[tn][4 * q]);
+                u64 Bp[2], Cp[2];
+                bc4(reinterpret_cast<const float*>(&bq), Bp);
+                bc4(reinterpret_cast<const float*>(&cq), Cp);
                 const float dls[2] = {d4.x, d4.z}, dus[2] = {d4.y, d4.w};
                 float yv[2];
 #pragma unroll
