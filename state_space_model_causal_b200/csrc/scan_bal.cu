@@ -503,40 +503,48 @@ __global__ void __launch_bounds__(32 * kWarps, 2) scan_bal_kernel(const ScanProb
         // this step's partials are stored, so that the loads (and the
         // exponentials behind them) are not held back behind the stores.
         {
-            using RawT = float4;
             float4 d4 = sm.dd[cp][dd_at(0)];  // (dl0, du0, dl1, du1)
-            RawT bq = *reinterpret_cast<const RawT*>(&sm.bf[0][4 * q]);
-            RawT cq = *reinterpret_cast<const RawT*>(&sm.cf[0][4 * q]);
-#pragma unroll 4
-            for (int t = 0; t < kT; ++t) {
-                const int tn = t + 1 < kT ? t + 1 : t;
-                const float4 d4n = sm.dd[cp][dd_at(tn)];
-                const RawT bqn = *reinterpret_cast<const RawT*>(&sm.bf[tn][4 * q]);
-                const RawT cqn = *reinterpret_cast<const RawT*>(&sm.cf[tn][4 * q]);
-                u64 Bp[2], Cp[2];
-                bc4(reinterpret_cast<const float*>(&bq), Bp);
-                bc4(reinterpret_cast<const float*>(&cq), Cp);
-                const float dls[2] = {d4.x, d4.z}, dus[2] = {d4.y, d4.w};
-                float yv[2];
+            float4 bq = *reinterpret_cast<const float4*>(&sm.bf[0][4 * q]);
+            float4 cq = *reinterpret_cast<const float4*>(&sm.cf[0][4 * q]);
+#pragma unroll 2
+            for (int tt = 0; tt < kT; tt += 4) {
+                float yv[2][4];
 #pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    const u64 dl2 = pk(dls[c], dls[c]), du2 = pk(dus[c], dus[c]);
-                    const u64 x0 = fmul2(dl2, A2[c][0]), x1 = fmul2(dl2, A2[c][1]);
-                    const int sidx = (t & 1) * 4 + 2 * c;  // exponential pair index within 2 steps
-                    const u64 a0 = (sidx < SW) ? exp2_pair_fma(x0) : exp2_pair_sfu(x0);
-                    const u64 a1 = (sidx + 1 < SW) ? exp2_pair_fma(x1) : exp2_pair_sfu(x1);
-                    h2[c][0] = ffma2(a0, h2[c][0], fmul2(du2, Bp[0]));
-                    h2[c][1] = ffma2(a1, h2[c][1], fmul2(du2, Bp[1]));
-                    const u64 y2 = ffma2(Cp[1], h2[c][1], fmul2(Cp[0], h2[c][0]));
-                    float lo, hi;
-                    upk(y2, lo, hi);
-                    yv[c] = lo + hi;
+                for (int s4 = 0; s4 < 4; ++s4) {
+                    const int t = tt + s4;
+                    const int tn = t + 1 < kT ? t + 1 : t;
+                    const float4 d4n = sm.dd[cp][dd_at(tn)];
+                    const float4 bqn = *reinterpret_cast<const float4*>(&sm.bf[tn][4 * q]);
+                    const float4 cqn = *reinterpret_cast<const float4*>(&sm.cf[tn][4 * q]);
+                    u64 Bp[2], Cp[2];
+                    bc4(reinterpret_cast<const float*>(&bq), Bp);
+                    bc4(reinterpret_cast<const float*>(&cq), Cp);
+                    const float dls[2] = {d4.x, d4.z}, dus[2] = {d4.y, d4.w};
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        const u64 dl2 = pk(dls[c], dls[c]), du2 = pk(dus[c], dus[c]);
+                        const u64 x0 = fmul2(dl2, A2[c][0]), x1 = fmul2(dl2, A2[c][1]);
+                        const int sidx = (t & 1) * 4 + 2 * c;  // exponential pair index within 2 steps
+                        const u64 a0 = (sidx < SW) ? exp2_pair_fma(x0) : exp2_pair_sfu(x0);
+                        const u64 a1 = (sidx + 1 < SW) ? exp2_pair_fma(x1) : exp2_pair_sfu(x1);
+                        h2[c][0] = ffma2(a0, h2[c][0], fmul2(du2, Bp[0]));
+                        h2[c][1] = ffma2(a1, h2[c][1], fmul2(du2, Bp[1]));
+                        const u64 y2 = ffma2(Cp[1], h2[c][1], fmul2(Cp[0], h2[c][0]));
+                        float lo, hi;
+                        upk(y2, lo, hi);
+                        yv[c][s4] = lo + hi;
+                    }
+                    d4 = d4n;
+                    bq = bqn;
+                    cq = cqn;
                 }
-                reinterpret_cast<float*>(&sm.yp[yp_at(t, 2 * cp)])[q] = yv[0];
-                reinterpret_cast<float*>(&sm.yp[yp_at(t, 2 * cp + 1)])[q] = yv[1];
-                d4 = d4n;
-                bq = bqn;
-                cq = cqn;
+                // the group's partials, stored after the next group's first
+                // operands were loaded
+#pragma unroll
+                for (int s4 = 0; s4 < 4; ++s4) {
+                    reinterpret_cast<float*>(&sm.yp[yp_at(tt + s4, 2 * cp)])[q] = yv[0][s4];
+                    reinterpret_cast<float*>(&sm.yp[yp_at(tt + s4, 2 * cp + 1)])[q] = yv[1][s4];
+                }
             }
         }
         __syncwarp();
