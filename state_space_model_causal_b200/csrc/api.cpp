@@ -308,8 +308,30 @@ constexpr long long kMinTestBudget = 10000000LL; // shortest wait a failure test
 // A failure test's wait budget, never below kMinTestBudget.
 long long clamp_test_budget(long long v) { return v < kMinTestBudget ? kMinTestBudget : v; }
 uint64_t bal_flag_bytes(int64_t workers) { return ((uint64_t)workers * 4 + 255) / 256 * 256; }
+// bytes of one hand-over slot: a unit's 16 x 16 state and 16 partial sums of delta
+uint64_t bal_slot_bytes() { return (uint64_t)scan_bal_channels_per_unit() * 17 * 4; }
 uint64_t bal_workspace_bytes(int64_t workers) {
-    return 256 + bal_flag_bytes(workers) + (uint64_t)workers * scan_bal_channels_per_unit() * 16 * 4;
+    return 256 + bal_flag_bytes(workers) + (uint64_t)workers * bal_slot_bytes();
+}
+// context-parallel records: per (base unit, piece 0..S-2) a 16 x 16 end state
+// and 16 sums of delta
+uint64_t cp_record_bytes(int64_t base_units, int pieces) {
+    return (uint64_t)base_units * (uint64_t)(pieces - 1) * bal_slot_bytes();
+}
+
+// Pieces per sequence for the context-parallel prefill: used when the
+// sequences alone (base units) would fill fewer than 60% of the resident
+// warps.  S - 1 pieces per pass give the warps enough units; a piece is at
+// least 2 chunks and the last one is never empty.  0: off.
+int cp_pieces(int64_t base_units, int64_t slots, int64_t chunks) {
+    if (base_units <= 0 || base_units * 10 >= slots * 6 || chunks < 6) return 0;
+    int64_t per_pass = std::min<int64_t>((slots + base_units - 1) / base_units, 15);
+    for (; per_pass >= 2; --per_pass) {
+        const int64_t S = per_pass + 1;
+        const int64_t pc = (chunks + S - 1) / S;
+        if (pc >= 2 && (S - 1) * pc < chunks) return (int)S;
+    }
+    return 0;
 }
 
 bool present_ws(const ssm_scan_args* a) { return a->workspace != nullptr && a->workspace_bytes > 0; }
@@ -615,25 +637,39 @@ ssm_status scan_impl(const ssm_scan_args* a, cudaStream_t stream, uint64_t* ws_q
         int per_sm = dry ? std::min(2, (228 * 1024) / (smem + 1024)) : scan_bal_ctas_per_sm(p, bp.sw, dev);
         if (per_sm <= 0) return dry ? SSM_ERR_UNSUPPORTED : SSM_ERR_CUDA;
         const int64_t slots = (int64_t)sm_count(dry, dev) * per_sm * warps;
-        const bool split = bp.units > slots;
-        const uint64_t need = split ? bal_workspace_bytes(slots) : 0;
+        const int64_t base_units = bp.units;
+        // context-parallel mode when the sequences alone leave most warps idle
+        const int S = cp_pieces(base_units, slots, bp.nck);
+        const int64_t pass_units = S ? base_units * (S - 1) : base_units;
+        const bool split = pass_units > slots;
+        const uint64_t need = (split || S) ? bal_workspace_bytes(slots) + (S ? cp_record_bytes(base_units, S) : 0) : 0;
         if (ws_query) {
             *ws_query = need;
             return SSM_OK;
         }
         // the slice bounds w * units * chunks / workers stay far inside int64
         if (bp.units > ((int64_t)1 << 40) / std::max<int64_t>(bp.nck, 1)) return SSM_ERR_UNSUPPORTED;
-        if (split && a->workspace) {
+        const bool use_ws = a->workspace && (split || S);
+        if (use_ws) {
             if (a->workspace_bytes < need || (reinterpret_cast<uintptr_t>(a->workspace) & 255u) != 0)
                 return SSM_ERR_WORKSPACE;
-            bp.workers = slots;
-            bp.cooperative = 1;
             unsigned char* ws = static_cast<unsigned char*>(a->workspace);
             bp.ws_head = reinterpret_cast<unsigned*>(ws);
             bp.ws_flags = reinterpret_cast<unsigned*>(ws + 256);
             bp.ws_slots = reinterpret_cast<float*>(ws + 256 + bal_flag_bytes(slots));
+            if (S) {
+                bp.cp_pieces = S;
+                bp.base_units = base_units;
+                bp.piece_chunks = (bp.nck + S - 1) / S;
+                bp.nck = bp.piece_chunks;
+                bp.units = pass_units;
+                bp.carry_h = reinterpret_cast<float*>(ws + bal_workspace_bytes(slots));
+                bp.carry_sdl = bp.carry_h + (size_t)base_units * (S - 1) * scan_bal_channels_per_unit() * 16;
+            }
+            bp.workers = split ? slots : bp.units;
+            bp.cooperative = split ? 1 : 0;
         } else {
-            bp.workers = bp.units;  // whole units, no hand-over
+            bp.workers = bp.units;  // whole units, no hand-over, no pieces
         }
         const int64_t grid = (bp.workers + warps - 1) / warps;
         if (grid > INT32_MAX) return SSM_ERR_UNSUPPORTED;
@@ -643,6 +679,12 @@ ssm_status scan_impl(const ssm_scan_args* a, cudaStream_t stream, uint64_t* ws_q
         if (a->flags & SSM_FLAG_DRY_RUN) return SSM_OK;
         bp.err = device_error_ptr(dev);
         if (!bp.err) return SSM_ERR_CUDA;
+        if (!bp.cp_pieces) return launch_scan_bal(p, bp, stream, dev) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+        // context-parallel: pass 1 (pieces 0..S-2, records), then pass 2
+        // (pieces 1..S-1 from the composed states), in order on the stream
+        bp.cp_pass = 1;
+        if (launch_scan_bal(p, bp, stream, dev) != cudaSuccess) return SSM_ERR_CUDA;
+        bp.cp_pass = 2;
         return launch_scan_bal(p, bp, stream, dev) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
     }
     if (vec_layout && scan_vec_supported(p)) {

@@ -115,6 +115,19 @@ struct BalPlan {
     float* ws_slots;     // one hand-over state per worker (16 x 16 floats)
     DeviceError* err;    // device error record
     long long wait_budget;  // cycles before a hand-over wait gives up
+    // Context-parallel mode (cp_pieces >= 3): every sequence is cut into
+    // cp_pieces pieces of piece_chunks chunks; a unit is (batch entry, channel
+    // block, piece).  Pass 1 runs pieces 0..S-2 -- piece 0 from the initial
+    // state with its outputs, the others from zero states without outputs --
+    // and records each piece's end state and per-channel sum of delta.  Pass
+    // 2 runs pieces 1..S-1 again from the states composed from those records,
+    // with outputs; the last piece writes the final caches.
+    int cp_pieces;       // S (0: off)
+    int cp_pass;         // 1 or 2
+    int64_t base_units;  // batch entries x channel blocks
+    int64_t piece_chunks;
+    float* carry_h;      // [base unit][piece 0..S-2][16 channels][16 state entries]
+    float* carry_sdl;    // [base unit][piece 0..S-2][16 channels]
 };
 
 // Prefill in the Mamba-2 layout: x, z, out (Bn, H, P, L); dt (Bn, H, L);

@@ -59,6 +59,7 @@ constexpr int kSPL = kT / 2;   // prologue / epilogue steps per lane (two lanes 
 constexpr int kWarps = 4;      // independent workers per CTA (one per SM sub-partition)
 constexpr int kDdRow = kT + 2;      // (delta, delta*u) words per channel pair (two pads)
 constexpr int kYpRow = kCH + 1;     // readout words per step (one pad)
+constexpr int kSlot = kCH * 16 + kCH;  // hand-over slot: 16 x 16 state, 16 partial sums of delta
 
 // One warp's shared memory.  Raw tiles are double-buffered (the next chunk's
 // copies fly during the whole current chunk); the widened B/C rows, the
@@ -204,11 +205,26 @@ __global__ void __launch_bounds__(32 * kWarps, 2) scan_bal_kernel(const ScanProb
     int64_t fu_cached = -1;
     const IoT *fx[NXP], *fdt[NXP], *fz[NXP], *fB[NBP], *fC[NBP];
     bool frow[NXP], fn[NBP];
+    // unit -> (base unit: batch entry x channel block, piece, first chunk)
+    auto unit_of = [&](int64_t uu, int64_t& ub, int& piece) -> int64_t {
+        if (bp.cp_pieces > 1) {
+            ub = uu / (bp.cp_pieces - 1);
+            piece = (int)(uu % (bp.cp_pieces - 1)) + (bp.cp_pass == 2 ? 1 : 0);
+            return (int64_t)piece * bp.piece_chunks;
+        }
+        ub = uu;
+        piece = 0;
+        return 0;
+    };
+    int64_t fkc0 = 0;
     auto fetch = [&](int64_t fu, int64_t fk, int fb) {
         if (fu != fu_cached) {
             fu_cached = fu;
-            const int64_t b = fu / bp.nblk;
-            const int64_t d0 = (fu % bp.nblk) * kCH;
+            int64_t ub;
+            int pce;
+            fkc0 = unit_of(fu, ub, pce);
+            const int64_t b = ub / bp.nblk;
+            const int64_t d0 = (ub % bp.nblk) * kCH;
             const int64_t g = d0 / p.ch_per_group;
 #pragma unroll
             for (int j = 0; j < NXP; ++j) {
@@ -228,7 +244,7 @@ __global__ void __launch_bounds__(32 * kWarps, 2) scan_bal_kernel(const ScanProb
                 fC[j] = static_cast<const IoT*>(p.Cm) + b * p.C_b + g * p.C_g + ns * p.C_n;
             }
         }
-        const int64_t t0 = fk * kT;
+        const int64_t t0 = (fkc0 + fk) * kT;
 #pragma unroll
         for (int j = 0; j < NXP; ++j) {
             const int i = lane + 32 * j, row = i / PPR, pcs = i % PPR;
@@ -265,10 +281,18 @@ __global__ void __launch_bounds__(32 * kWarps, 2) scan_bal_kernel(const ScanProb
     u64 A2[2][2], h2[2][2];  // [channel][pair of state entries]
     const IoT* pxrow = nullptr;
     IoT* porow = nullptr;
+    int64_t ub = 0;     // base unit of the segment
+    int piece = 0;      // its piece (context-parallel mode)
+    int64_t kc0 = 0;    // its first chunk in the whole sequence
+    double sdl = 0.0;   // the prologue lane's sum of delta over its steps of the piece so far
+                        // (fp64: exp(A * sum) must match the product of the steps' decays)
+    bool store_out = true;
 
     auto setup = [&]() {
-        b = u / bp.nblk;
-        const int64_t d0 = (u % bp.nblk) * kCH;
+        kc0 = unit_of(u, ub, piece);
+        store_out = !(bp.cp_pass == 1 && piece > 0);  // pass 1 keeps only piece 0's outputs
+        b = ub / bp.nblk;
+        const int64_t d0 = (ub % bp.nblk) * kCH;
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
             const int64_t d = d0 + 2 * cp + c;
@@ -312,25 +336,55 @@ __global__ void __launch_bounds__(32 * kWarps, 2) scan_bal_kernel(const ScanProb
                     __nanosleep(128);
                 }
             }
+            sdl = 0.0;
             if (got) {
+                const float* slot = bp.ws_slots + (w - 1) * kSlot;
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
-                    const float4 v = __ldcg(reinterpret_cast<const float4*>(
-                        bp.ws_slots + ((w - 1) * kCH + 2 * cp + c) * 16 + 4 * q));
+                    const float4 v = __ldcg(reinterpret_cast<const float4*>(slot + (2 * cp + c) * 16 + 4 * q));
                     h[c][0] = v.x; h[c][1] = v.y; h[c][2] = v.z; h[c][3] = v.w;
                 }
+                if (ph == 0) sdl = (double)__ldcg(slot + kCH * 16 + pc);
             } else if (lane == 0) {
                 // the tail of unit u starts from a zero state instead
                 report_device_error(bp.err, SSM_KERNEL_SCAN_BAL, (long long)u);
             }
-        } else if (p.ssm_state) {
+        } else {
+            sdl = 0.0;
+            if (piece == 0) {
+                if (p.ssm_state) {
 #pragma unroll
-            for (int c = 0; c < 2; ++c)
+                    for (int c = 0; c < 2; ++c)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int n = 4 * q + j;
-                    if (sok[c] && n < p.N) h[c][j] = p.ssm_state[b * p.ss_b + sd[c] * p.ss_d + n * p.ss_n];
+                        for (int j = 0; j < 4; ++j) {
+                            const int n = 4 * q + j;
+                            if (sok[c] && n < p.N) h[c][j] = p.ssm_state[b * p.ss_b + sd[c] * p.ss_d + n * p.ss_n];
+                        }
                 }
+            } else if (bp.cp_pass == 2) {
+                // the state at the piece's start, composed from the pass-1
+                // records: h_in(1) = h_end(0); h_in(j+1) = exp(A * sum delta(j)) * h_in(j) + h_end(j)
+                const int64_t rec0 = ub * (bp.cp_pieces - 1);
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    const int ch_ = 2 * cp + c;
+                    const float4 v = __ldcg(reinterpret_cast<const float4*>(bp.carry_h + (rec0 * kCH + ch_) * 16 + 4 * q));
+                    h[c][0] = v.x; h[c][1] = v.y; h[c][2] = v.z; h[c][3] = v.w;
+                    for (int j = 1; j < piece; ++j) {
+                        const float sj = __ldcg(bp.carry_sdl + (rec0 + j) * kCH + ch_);
+                        const float4 e = __ldcg(reinterpret_cast<const float4*>(
+                            bp.carry_h + ((rec0 + j) * kCH + ch_) * 16 + 4 * q));
+                        float a[4];
+                        upk(A2[c][0], a[0], a[1]);
+                        upk(A2[c][1], a[2], a[3]);
+                        h[c][0] = fmaf(ex2_approx(a[0] * sj), h[c][0], e.x);
+                        h[c][1] = fmaf(ex2_approx(a[1] * sj), h[c][1], e.y);
+                        h[c][2] = fmaf(ex2_approx(a[2] * sj), h[c][2], e.z);
+                        h[c][3] = fmaf(ex2_approx(a[3] * sj), h[c][3], e.w);
+                    }
+                }
+            }
+            // pass 1, pieces >= 1: zero state
         }
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
@@ -342,10 +396,10 @@ __global__ void __launch_bounds__(32 * kWarps, 2) scan_bal_kernel(const ScanProb
         for (int i = 0; i < W - 1; ++i) {
             float v = 0.0f;
             if (pok) {
-                if (k0 == 0) {
+                if (kc0 + k0 == 0) {
                     if (p.conv_state) v = ld_f(p.conv_state, b * p.cs_b + pd * p.cs_d + (1 + i) * p.cs_k, p.cs_dt);
                 } else {
-                    v = to_f(pxrow[k0 * kT - (W - 1) + i]);
+                    v = to_f(pxrow[(kc0 + k0) * kT - (W - 1) + i]);
                 }
             }
             ch.hist[i] = v;
@@ -374,7 +428,7 @@ __global__ void __launch_bounds__(32 * kWarps, 2) scan_bal_kernel(const ScanProb
         __syncwarp();  // this chunk's tiles are visible; the other buffer is free
         if (more) fetch(nu, nk, buf ^ 1);
 
-        const int64_t t0 = k * kT;
+        const int64_t t0 = (kc0 + k) * kT;
         // ---- widen B/C into [t][n] rows: lane (row n, half hh) converts 16
         // steps; the two halves write rows of opposite parity at each store so
         // that the 32 lanes hit 32 distinct banks
@@ -478,6 +532,7 @@ __global__ void __launch_bounds__(32 * kWarps, 2) scan_bal_kernel(const ScanProb
             for (int i = 0; i < kSPL; i += 2) {
                 const bool vo = vv[i / 8];
                 const float dl0 = vo ? dl[i] : 0.0f, dl1 = vo ? dl[i + 1] : 0.0f;
+                sdl += (double)dl0 + (double)dl1;
                 const u64 du2 = fmul2(pk(dl0, dl1), pk(uu[i], uu[i + 1]));
                 float du0, du1;
                 upk(du2, du0, du1);
@@ -553,7 +608,7 @@ __global__ void __launch_bounds__(32 * kWarps, 2) scan_bal_kernel(const ScanProb
         // 16ph .. 16ph+15 of channel pc
 #pragma unroll
         for (int v = 0; v < 2; ++v) {
-            if (vv[v]) {
+            if (vv[v] && store_out) {
                 float o[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
@@ -566,19 +621,35 @@ __global__ void __launch_bounds__(32 * kWarps, 2) scan_bal_kernel(const ScanProb
 
         // ---- end of a segment: hand the state over, or write the final caches
         if (k + 1 == k1) {
+            // the channel's sum of delta over the piece so far (both halves)
+            const float sdl_ch = (float)(sdl + __shfl_xor_sync(0xffffffffu, sdl, 2));
             if (kind == 2) {
+                float* slot = bp.ws_slots + w * kSlot;
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
                     float hv[4];
                     upk(h2[c][0], hv[0], hv[1]);
                     upk(h2[c][1], hv[2], hv[3]);
-                    __stcg(reinterpret_cast<float4*>(bp.ws_slots + (w * kCH + 2 * cp + c) * 16 + 4 * q),
+                    __stcg(reinterpret_cast<float4*>(slot + (2 * cp + c) * 16 + 4 * q),
                            make_float4(hv[0], hv[1], hv[2], hv[3]));
                 }
+                if (ph == 0) __stcg(slot + kCH * 16 + pc, sdl_ch);
                 __threadfence();
                 __syncwarp();
                 if (lane == 0) st_release_u32(bp.ws_flags + w, gen + 1u);
-            } else {
+            } else if (bp.cp_pass == 1) {
+                // the piece's end state and sum of delta, for pass 2
+                const int64_t rec = ub * (bp.cp_pieces - 1) + piece;
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    float hv[4];
+                    upk(h2[c][0], hv[0], hv[1]);
+                    upk(h2[c][1], hv[2], hv[3]);
+                    __stcg(reinterpret_cast<float4*>(bp.carry_h + (rec * kCH + 2 * cp + c) * 16 + 4 * q),
+                           make_float4(hv[0], hv[1], hv[2], hv[3]));
+                }
+                if (ph == 0) __stcg(bp.carry_sdl + rec * kCH + pc, sdl_ch);
+            } else if (bp.cp_pass == 0 || piece == bp.cp_pieces - 1) {
                 if (p.ssm_state) {
 #pragma unroll
                     for (int c = 0; c < 2; ++c) {

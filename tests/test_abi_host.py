@@ -194,8 +194,8 @@ def test_prefill_2p8b_plan(lib):
 
 def ws_bytes(workers):
     """256-byte header, one 32-bit flag per worker rounded up to 256 bytes,
-    one 1 KB hand-over state (16 channels x 16 state entries) per worker."""
-    return 256 + (workers * 4 + 255) // 256 * 256 + workers * 1024
+    one 1088-byte hand-over slot (16 x 16 state, 16 sums of delta) per worker."""
+    return 256 + (workers * 4 + 255) // 256 * 256 + workers * 1088
 
 
 def test_prefill_workspace_size_and_balanced_plan(lib):
@@ -215,12 +215,27 @@ def test_prefill_workspace_size_and_balanced_plan(lib):
     assert lib.ssm_selective_scan_workspace_size(ctypes.byref(a), None) == ENULL
 
 
-def test_prefill_small_problem_needs_no_workspace(lib):
+def test_prefill_context_parallel_plan(lib):
+    """B=1: 320 units fill under 60% of the 1184 resident warps, so the
+    sequence is cut into 5 pieces of 13 chunks (the last one 12): each of the
+    two passes runs 4 pieces per unit, 1280 piece-units (more than the
+    warps, so the passes hand over too).  The workspace adds one record
+    (16 x 16 state + 16 sums of delta) per unit and piece 0..3."""
     mem = FakeMem()
-    a = scan_args(mem, Bn=1, D=5120)  # 320 units fit in one wave
+    a = scan_args(mem, Bn=1, D=5120)
     need = ctypes.c_uint64(123)
     assert lib.ssm_selective_scan_workspace_size(ctypes.byref(a), ctypes.byref(need)) == OK
-    assert need.value == 0
+    assert need.value == ws_bytes(1184) + 320 * 4 * 1088
+    a.workspace, a.workspace_bytes = mem.next, need.value
+    mem.next += 1 << 36
+    st, info = call(lib, "ssm_selective_scan_fwd", a)
+    assert st == OK and bd.KERNELS[info.kernel] == "scan_bal"
+    assert info.work_items == 1280 and info.grid == 296
+
+
+def test_prefill_small_problem_needs_no_workspace(lib):
+    mem = FakeMem()
+    need = ctypes.c_uint64(123)
     a = scan_args(mem, Bn=2, D=64, L=100)  # chunked kernel
     assert lib.ssm_selective_scan_workspace_size(ctypes.byref(a), ctypes.byref(need)) == OK
     assert need.value == 0
