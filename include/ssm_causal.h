@@ -254,6 +254,11 @@ ssm_status ssm_selective_scan_fwd(const ssm_scan_args* args, void* stream);
  * 16-channel) units than the GPU runs warps at once, the fast kernel splits
  * the work into equal slices per warp; a slice that starts or ends inside a
  * unit hands its running state to the neighbouring warp through `workspace`.
+ * With few units (under 60% of the warps) it instead cuts every sequence into
+ * pieces scanned in two passes, and the workspace also holds each piece's end
+ * state and sum of delta.  The fast Mamba-2-layout prefill likewise splits
+ * its (batch, head, row block) units over its CTAs, handing 32 KB state tiles
+ * over through the workspace.
  * ssm_selective_scan_workspace_size() returns in *bytes how much workspace a
  * call with these arguments can use on the current device (0 when it needs
  * none); it checks the arguments as ssm_selective_scan_fwd does and launches
@@ -279,7 +284,8 @@ ssm_status ssm_selective_scan_workspace_size(const ssm_scan_args* args, uint64_t
  *
  * The call takes the same arguments as ssm_selective_scan_fwd, with workspace
  * NULL and workspace_bytes 0 (else SSM_ERR_WORKSPACE), and computes the same
- * results.  The scratch it needs comes from a fixed 2 MiB device array inside
+ * results.  (The Mamba-2-layout prefill, x of rank 4, needs no scratch for
+ * its results: it runs here as it does without a workspace.)  The scratch it needs comes from a fixed 2 MiB device array inside
  * the library, which every GPU that loads the library holds until the
  * process exits; a problem that would need more than 2 MiB of scratch is
  * rejected with SSM_ERR_WORKSPACE before anything is launched (the prefill

@@ -353,7 +353,7 @@ bool overlaps_any(const ssm_scan_args* a) {
 // -------------------------------------------------------------------- scan --
 // Prefill in the Mamba-2 layout (x of rank 4); arguments past the common
 // checks of scan_impl.
-ssm_status scan_m2_impl(const ssm_scan_args* a, cudaStream_t stream) {
+ssm_status scan_m2_impl(const ssm_scan_args* a, cudaStream_t stream, uint64_t* ws_query) {
     const int64_t Bn = a->x.shape[0], H = a->x.shape[1], P = a->x.shape[2], L = a->x.shape[3];
     const int io = a->x.dtype;
     if (!is_float(io)) return SSM_ERR_DTYPE;
@@ -429,10 +429,16 @@ ssm_status scan_m2_impl(const ssm_scan_args* a, cudaStream_t stream) {
         p.ss_n = sd(a->ssm_state, 3);
     }
     p.out = a->out.data; p.o_b = sd(a->out, 0); p.o_h = sd(a->out, 1); p.o_p = sd(a->out, 2); p.o_t = sd(a->out, 3);
+    if (present_ws(a) && overlaps_any(a)) return SSM_ERR_ALIAS;
     if (Bn == 0 || H == 0 || P == 0 || L == 0) {  // nothing to compute, caches unchanged
+        if (ws_query) {
+            *ws_query = 0;
+            return SSM_OK;
+        }
         fill_info(a->info, SSM_KERNEL_NONE, 0, 0, 0, 0, 0);
         return SSM_OK;
     }
+    const bool dry = (a->flags & SSM_FLAG_DRY_RUN) != 0;
     // fast kernel: headdim / dstate contiguous, 16-byte aligned rows and steps
     const int es = esize(io);
     const int64_t rpc = scan_m2_rows_per_cta(N);
@@ -446,15 +452,55 @@ ssm_status scan_m2_impl(const ssm_scan_args* a, cudaStream_t stream) {
                       m16(p.B_t) && m16(p.C_b) && m16(p.C_g) && m16(p.C_t) && H <= 65535 && Bn <= 65535;
     int kernel, grid, block, smem;
     int64_t items;
+    M2Plan mp{};
     if (fast) {
         kernel = SSM_KERNEL_SCAN_M2;
         const int64_t blocks = (P + rpc - 1) / rpc;
         if (blocks * H * Bn > INT32_MAX) return SSM_ERR_UNSUPPORTED;
-        grid = (int)(blocks * H * Bn);
         block = scan_m2_threads();
         smem = scan_m2_smem_bytes(io, N);
         items = blocks * H * Bn;
+        // balanced slices when there are more units than resident CTAs
+        const int dev = current_device(dry);
+        const int per_sm = dry ? std::min(3, (228 * 1024) / (smem + 1024)) : scan_m2_ctas_per_sm(p, dev);
+        if (per_sm <= 0) return dry ? SSM_ERR_UNSUPPORTED : SSM_ERR_CUDA;
+        const int64_t slots = (int64_t)sm_count(dry, dev) * per_sm;
+        mp.units = items;
+        mp.nblk = blocks;
+        mp.nck = (L + 15) / 16;
+        mp.dev = dev;
+        const bool split = items > slots;
+        const uint64_t tile = (uint64_t)rpc * N * 4;  // one CTA's state tile
+        const uint64_t need = split ? 256 + bal_flag_bytes(slots) + (uint64_t)slots * tile : 0;
+        if (ws_query) {
+            *ws_query = need;
+            return SSM_OK;
+        }
+        if (mp.units > ((int64_t)1 << 40) / std::max<int64_t>(mp.nck, 1)) return SSM_ERR_UNSUPPORTED;
+        if (split && a->workspace) {
+            if (a->workspace_bytes < need || (reinterpret_cast<uintptr_t>(a->workspace) & 255u) != 0)
+                return SSM_ERR_WORKSPACE;
+            unsigned char* ws = static_cast<unsigned char*>(a->workspace);
+            mp.ws_head = reinterpret_cast<unsigned*>(ws);
+            mp.ws_flags = reinterpret_cast<unsigned*>(ws + 256);
+            mp.ws_slots = reinterpret_cast<float*>(ws + 256 + bal_flag_bytes(slots));
+            mp.workers = slots;
+            mp.cooperative = 1;
+        } else {
+            mp.workers = items;  // one whole unit per CTA
+        }
+        grid = (int)mp.workers;
+        mp.grid = grid;
+        mp.wait_budget = kWaitBudget;
+        if (!dry) {
+            mp.err = device_error_ptr(dev);
+            if (!mp.err) return SSM_ERR_CUDA;
+        }
     } else {
+        if (ws_query) {
+            *ws_query = 0;
+            return SSM_OK;
+        }
         kernel = SSM_KERNEL_SCAN_M2_GENERIC;
         const int64_t rows = Bn * H * P;
         if ((rows + 3) / 4 > INT32_MAX) return SSM_ERR_UNSUPPORTED;
@@ -465,7 +511,7 @@ ssm_status scan_m2_impl(const ssm_scan_args* a, cudaStream_t stream) {
     }
     fill_info(a->info, kernel, grid, block, smem, fast ? rpc : 1, items);
     if (a->flags & SSM_FLAG_DRY_RUN) return SSM_OK;
-    return launch_scan_m2(p, kernel, stream) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+    return launch_scan_m2(p, kernel, mp, stream) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 
 ssm_status scan_impl(const ssm_scan_args* a, cudaStream_t stream, uint64_t* ws_query) {
@@ -478,18 +524,7 @@ ssm_status scan_impl(const ssm_scan_args* a, cudaStream_t stream, uint64_t* ws_q
     SSM_TRY(basic(a->B));
     SSM_TRY(basic(a->C));
     SSM_TRY(basic(a->out));
-    if (a->x.ndim == 4) {
-        if (ws_query) {
-            // the Mamba-2-layout prefill uses no workspace; check the arguments
-            ssm_scan_args dry = *a;
-            dry.flags |= SSM_FLAG_DRY_RUN;
-            dry.info = nullptr;
-            SSM_TRY(scan_m2_impl(&dry, stream));
-            *ws_query = 0;
-            return SSM_OK;
-        }
-        return scan_m2_impl(a, stream);
-    }
+    if (a->x.ndim == 4) return scan_m2_impl(a, stream, ws_query);
     if (a->x.ndim != 3) return SSM_ERR_SHAPE;
     const int64_t Bn = a->x.shape[0], D = a->x.shape[1], L = a->x.shape[2];
     if (a->A.ndim != 2 || a->A.shape[0] != D) return SSM_ERR_SHAPE;
@@ -1146,6 +1181,10 @@ ssm_status ssm_selective_scan_fwd_noalloc(const ssm_scan_args* args, void* strea
     if (args->struct_size != sizeof(ssm_scan_args)) return SSM_ERR_VERSION;
     // the scratch is the library's own fixed array: no caller workspace
     if (args->workspace || args->workspace_bytes) return SSM_ERR_WORKSPACE;
+    // The Mamba-2-layout prefill needs no scratch for its results (its
+    // hand-overs only balance the GPU, with 32 KB per CTA, more than the
+    // array): it runs here with one whole unit per CTA.
+    if (args->x.ndim == 4) return scan_impl(args, static_cast<cudaStream_t>(stream), nullptr);
     // check the arguments and size the scratch exactly as the workspace query does
     uint64_t need = 0;
     SSM_TRY(scan_impl(args, static_cast<cudaStream_t>(stream), &need));

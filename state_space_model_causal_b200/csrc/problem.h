@@ -149,6 +149,21 @@ struct ScanM2Problem {
     void* out; int64_t o_b, o_h, o_p, o_t;
 };
 
+// Launch of the fast Mamba-2-layout prefill: units are (b, h, row block) over
+// the whole sequence in 16-step chunks; `workers` CTAs split the flattened
+// (unit, chunk) list into equal slices, handing 32 KB state tiles over
+// through the workspace when there are more units than resident CTAs
+// (ws_* non-NULL, cooperative launch); otherwise workers == units.
+struct M2Plan {
+    int64_t units, nblk, nck, workers;
+    int grid, cooperative, dev;
+    unsigned* ws_head;
+    unsigned* ws_flags;
+    float* ws_slots;     // one state tile (rows per CTA x dstate floats) per worker
+    DeviceError* err;
+    long long wait_budget;
+};
+
 struct Conv1dProblem {
     int64_t Bn, D, L, W;
     int io_dt;
@@ -192,6 +207,7 @@ cudaError_t launch_conv1d(const Conv1dProblem& p, const Conv1dPlan& plan, cudaSt
 int scan_m2_rows_per_cta(int64_t N);
 int scan_m2_threads();
 int scan_m2_smem_bytes(int io_dt, int64_t N);
-cudaError_t launch_scan_m2(const ScanM2Problem& p, int kernel, cudaStream_t s);
+cudaError_t launch_scan_m2(const ScanM2Problem& p, int kernel, const M2Plan& mp, cudaStream_t s);
+int scan_m2_ctas_per_sm(const ScanM2Problem& p, int dev);
 
 }  // namespace ssm

@@ -37,6 +37,8 @@
 #include "common.cuh"
 #include "problem.h"
 
+#include <atomic>
+
 namespace ssm {
 namespace {
 
@@ -81,99 +83,241 @@ __device__ __forceinline__ void cp_async16_m2(void* dst, const void* src, bool v
 }
 
 template <typename IoT, int NG>
-__global__ void __launch_bounds__(kM2Threads, kM2MinCtas) scan_m2_kernel(const ScanM2Problem p) {
+__global__ void __launch_bounds__(kM2Threads, kM2MinCtas) scan_m2_kernel(const ScanM2Problem p, const M2Plan mp);
+
+// Per device: the shared-memory attributes of the fast kernel, set once, and
+// the CTAs that fit on one SM (0 = not queried yet, else count + 1).
+template <typename IoT, int NG>
+int m2_ctas_per_sm(int dev) {
+    static std::atomic<int> cache[kMaxDevices];
+    if (dev < 0 || dev >= kMaxDevices) return 0;
+    int v = cache[dev].load(std::memory_order_acquire);
+    if (v == 0) {
+        auto kern = scan_m2_kernel<IoT, NG>;
+        const int smem = (int)sizeof(M2Smem<IoT, NG>);
+        int n = 0;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+            cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared) != cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kM2Threads, smem) != cudaSuccess)
+            return 0;
+        v = n + 1;
+        cache[dev].store(v, std::memory_order_release);
+    }
+    return v - 1;
+}
+
+__device__ __forceinline__ unsigned m2_ld_acquire(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void m2_st_release(unsigned* p, unsigned v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ unsigned m2_atom_inc(unsigned* p, unsigned lim) {
+    unsigned old;
+    asm volatile("atom.acq_rel.gpu.global.inc.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(lim) : "memory");
+    return old;
+}
+
+// A unit is one (b, h, row block) over the whole sequence in 16-step chunks.
+// CTA w takes the slice [w * total / workers, (w + 1) * total / workers) of
+// the flattened (unit, chunk) list: the head of the unit the slice ends in
+// first (its state handed to CTA w + 1 through the workspace), then whole
+// units, then the tail of the unit the slice starts in (from the state CTA
+// w - 1 handed over).  Without a workspace, workers == units and every CTA
+// runs one whole unit.
+template <typename IoT, int NG>
+__global__ void __launch_bounds__(kM2Threads, kM2MinCtas) scan_m2_kernel(const ScanM2Problem p, const M2Plan mp) {
     using S = M2Smem<IoT, NG>;
     constexpr int RPC = S::RPC;
     constexpr int N = S::N;
     constexpr int E = 16 / (int)sizeof(IoT);  // elements per 16-byte copy
-    constexpr int PG = kM2Threads / NG;       // row groups of 4
     extern __shared__ __align__(16) unsigned char m2_smem[];
     S& sm = *reinterpret_cast<S*>(m2_smem);
+    __shared__ unsigned s_gen;
+    __shared__ int s_got;
 
     const int tid = threadIdx.x;
     const int ng = tid % NG;
     const int pg = tid / NG;
-    const int64_t b = blockIdx.z;
-    const int64_t h = blockIdx.y;
-    const int64_t p0 = (int64_t)blockIdx.x * RPC;  // first headdim row of the CTA
-    const int64_t g = h / (p.H / p.G);
+    const int64_t w = blockIdx.x;
     const int64_t L = p.L;
-    const IoT* xg = static_cast<const IoT*>(p.x) + b * p.x_b + h * p.x_h + p0;
-    const IoT* zg = p.z ? static_cast<const IoT*>(p.z) + b * p.z_b + h * p.z_h + p0 : nullptr;
-    const IoT* Bg = static_cast<const IoT*>(p.Bm) + b * p.B_b + g * p.B_g;
-    const IoT* Cg = static_cast<const IoT*>(p.Cm) + b * p.C_b + g * p.C_g;
-    const IoT* dtg = static_cast<const IoT*>(p.dt) + b * p.dt_b + h * p.dt_h;
-    IoT* og = static_cast<IoT*>(p.out) + b * p.o_b + h * p.o_h + p0;
-    const float A2 = p.A[h * p.A_h] * kLog2e;
-    const float dbias = p.dt_bias ? p.dt_bias[h * p.db_h] : 0.0f;
-    const float dskip = p.Dp ? p.Dp[h * p.D_h] : 0.0f;
-    const int rows = (int)(p.P - p0 < RPC ? p.P - p0 : RPC);  // valid rows of the block
-
-    // state tile: rows 4pg + r, entries 16ng + 2j, 16ng + 2j + 1 as pairs
-    u64 hs[4][8];
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-        const int row = 4 * pg + r;
-        const bool v = row < rows;
-        const float* src = p.ssm_state
-                               ? p.ssm_state + b * p.ss_b + h * p.ss_h + (p0 + (v ? row : 0)) * p.ss_p +
-                                     16 * ng * p.ss_n
-                               : nullptr;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            float a = 0.0f, c = 0.0f;
-            if (src && v) {
-                a = src[(2 * j) * p.ss_n];
-                c = src[(2 * j + 1) * p.ss_n];
+    const int64_t nck = mp.nck;
+    const int64_t total = mp.units * nck;
+    const int64_t s0 = w * total / mp.workers;
+    const int64_t e0 = (w + 1) * total / mp.workers;
+    const bool has_head = (e0 % nck) != 0;
+    const bool has_tail = (s0 % nck) != 0;
+    const int64_t first_full = (s0 + nck - 1) / nck;
+    const int64_t n_full = e0 / nck - first_full;
+    const int64_t nseg = (has_head ? 1 : 0) + n_full + (has_tail ? 1 : 0);
+    auto seg_of = [&](int64_t i, int64_t& u, int64_t& k0, int64_t& k1) -> int {
+        if (has_head) {
+            if (i == 0) {
+                u = e0 / nck; k0 = 0; k1 = e0 % nck;
+                return 2;  // emits a hand-over
             }
-            hs[r][j] = pk(a, c);
+            --i;
         }
+        if (i < n_full) {
+            u = first_full + i; k0 = 0; k1 = nck;
+            return 0;
+        }
+        u = s0 / nck; k0 = s0 % nck; k1 = nck;
+        return 1;  // receives a hand-over
+    };
+    if (mp.ws_head) {
+        if (tid == 0) s_gen = *reinterpret_cast<volatile unsigned*>(mp.ws_head);
+        __syncthreads();
     }
-    // this thread's B/C pieces: u = 4ng + k, stored at m2_swz(u)
-    int boff[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) boff[k] = m2_swz(4 * ng + k) * 4;
+    const unsigned gen = mp.ws_head ? s_gen : 0u;
 
-    const int nchunks = (int)((L + kM2T - 1) / kM2T);
-    // x, z of chunk ci: kM2T x RPC elements each, into raw[ci & 1]
-    auto fetch_xz = [&](int ci) {
-        typename S::RawXZ& rw = sm.raw[ci & 1];
-        const int64_t t0 = (int64_t)ci * kM2T;
+    // unit -> (b, h, first row); per-unit base pointers
+    struct Unit {
+        int64_t b, h, p0;
+        int rows;
+        const IoT *xg, *zg, *Bg, *Cg, *dtg;
+        IoT* og;
+    };
+    auto unit = [&](int64_t uu) {
+        Unit r;
+        const int64_t pb = uu % mp.nblk;
+        const int64_t bh = uu / mp.nblk;
+        r.h = bh % p.H;
+        r.b = bh / p.H;
+        r.p0 = pb * RPC;
+        const int64_t g = r.h / (p.H / p.G);
+        r.rows = (int)(p.P - r.p0 < RPC ? p.P - r.p0 : RPC);
+        r.xg = static_cast<const IoT*>(p.x) + r.b * p.x_b + r.h * p.x_h + r.p0;
+        r.zg = p.z ? static_cast<const IoT*>(p.z) + r.b * p.z_b + r.h * p.z_h + r.p0 : nullptr;
+        r.Bg = static_cast<const IoT*>(p.Bm) + r.b * p.B_b + g * p.B_g;
+        r.Cg = static_cast<const IoT*>(p.Cm) + r.b * p.C_b + g * p.C_g;
+        r.dtg = static_cast<const IoT*>(p.dt) + r.b * p.dt_b + r.h * p.dt_h;
+        r.og = static_cast<IoT*>(p.out) + r.b * p.o_b + r.h * p.o_h + r.p0;
+        return r;
+    };
+
+    // x, z of chunk ck of unit U: kM2T x RPC elements each, into raw[bi]
+    auto fetch_xz = [&](const Unit& U, int64_t ck, int bi) {
+        typename S::RawXZ& rw = sm.raw[bi];
+        const int64_t t0 = ck * kM2T;
         constexpr int XC = kM2T * RPC / E;
         for (int i = tid; i < XC; i += kM2Threads) {
             const int t = i / (RPC / E), e = (i % (RPC / E)) * E;
-            const bool v = t0 + t < L && e < rows;
+            const bool v = t0 + t < L && e < U.rows;
             const int64_t ts = v ? t0 + t : 0;
-            cp_async16_m2(&rw.x[t][e], xg + ts * p.x_t + (v ? e : 0), v);
-            cp_async16_m2(&rw.z[t][e], (zg ? zg : xg) + ts * (zg ? p.z_t : p.x_t) + (v ? e : 0), v && zg);
+            cp_async16_m2(&rw.x[t][e], U.xg + ts * p.x_t + (v ? e : 0), v);
+            cp_async16_m2(&rw.z[t][e], (U.zg ? U.zg : U.xg) + ts * (U.zg ? p.z_t : p.x_t) + (v ? e : 0), v && U.zg);
         }
     };
-    // B, C of chunk ci: kM2T x N elements each
-    auto fetch_bc = [&](int ci) {
-        const int64_t t0 = (int64_t)ci * kM2T;
+    // B, C of chunk ck: kM2T x N elements each
+    auto fetch_bc = [&](const Unit& U, int64_t ck) {
+        const int64_t t0 = ck * kM2T;
         constexpr int BC = kM2T * N / E;
         for (int i = tid; i < BC; i += kM2Threads) {
             const int t = i / (N / E), e = (i % (N / E)) * E;
             const bool v = t0 + t < L;
             const int64_t ts = v ? t0 + t : 0;
-            cp_async16_m2(&sm.rawB[t][e], Bg + ts * p.B_t + e, v);
-            cp_async16_m2(&sm.rawC[t][e], Cg + ts * p.C_t + e, v);
+            cp_async16_m2(&sm.rawB[t][e], U.Bg + ts * p.B_t + e, v);
+            cp_async16_m2(&sm.rawC[t][e], U.Cg + ts * p.C_t + e, v);
         }
     };
     auto commit = []() { asm volatile("cp.async.commit_group;" ::: "memory"); };
-    // dt of the next chunk, one step per thread of the first warp
-    float dt_next = 0.0f;
-    auto load_dt = [&](int ci) {
-        const int64_t t = (int64_t)ci * kM2T + tid;
-        dt_next = (tid < kM2T && t < L) ? to_f(dtg[t * p.dt_t]) : 0.0f;
+    // dt of a chunk, one step per thread of the first warp
+    auto load_dt = [&](const Unit& U, int64_t ck) -> float {
+        const int64_t t = ck * kM2T + tid;
+        return (tid < kM2T && t < L) ? to_f(U.dtg[t * p.dt_t]) : 0.0f;
     };
-    fetch_xz(0);
-    fetch_bc(0);
-    commit();
-    load_dt(0);
 
-    for (int ci = 0; ci < nchunks; ++ci) {
-        const int64_t t0 = (int64_t)ci * kM2T;
+    // this thread's B/C pieces: u = 4ng + k, stored at m2_swz(u)
+    int boff[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) boff[k] = m2_swz(4 * ng + k) * 4;
+
+    int64_t seg = 0, u = 0, k0 = 0, k1 = 0;
+    int kind = seg_of(0, u, k0, k1);
+    Unit cu = unit(u);
+    float A2 = 0.0f, dbias = 0.0f, dskip = 0.0f;
+    u64 hs[4][8];
+    // state tile of a segment's start: rows 4pg + r, entries 16ng + 2j, 16ng + 2j + 1 as pairs
+    auto setup = [&]() {
+        A2 = p.A[cu.h * p.A_h] * kLog2e;
+        dbias = p.dt_bias ? p.dt_bias[cu.h * p.db_h] : 0.0f;
+        dskip = p.Dp ? p.Dp[cu.h * p.D_h] : 0.0f;
+        if (kind == 1) {
+            if (tid == 0) {
+                int got = 1;
+                if (mp.ws_flags) {
+                    const unsigned* flag = mp.ws_flags + (w - 1);
+                    const long long t_start = clock64();
+                    while (m2_ld_acquire(flag) != gen + 1u) {
+                        if (clock64() - t_start > mp.wait_budget) {
+                            got = 0;
+                            break;
+                        }
+                        __nanosleep(128);
+                    }
+                }
+                if (!got) report_device_error(mp.err, SSM_KERNEL_SCAN_M2, (long long)u);
+                s_got = got;
+            }
+            __syncthreads();
+            const bool got = s_got != 0;
+            const float* slot = mp.ws_slots + (w - 1) * (int64_t)(RPC * N);
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    float2 v = make_float2(0.0f, 0.0f);
+                    if (got) v = __ldcg(reinterpret_cast<const float2*>(slot + (4 * pg + r) * N + 16 * ng + 2 * j));
+                    hs[r][j] = pk(v.x, v.y);
+                }
+        } else {
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const int row = 4 * pg + r;
+                const bool v = row < cu.rows;
+                const float* src = p.ssm_state ? p.ssm_state + cu.b * p.ss_b + cu.h * p.ss_h +
+                                                     (cu.p0 + (v ? row : 0)) * p.ss_p + 16 * ng * p.ss_n
+                                               : nullptr;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    float a = 0.0f, c = 0.0f;
+                    if (src && v) {
+                        a = src[(2 * j) * p.ss_n];
+                        c = src[(2 * j + 1) * p.ss_n];
+                    }
+                    hs[r][j] = pk(a, c);
+                }
+            }
+        }
+    };
+    setup();
+
+    int bi = 0;
+    fetch_xz(cu, k0, bi);
+    fetch_bc(cu, k0);
+    commit();
+    float dt_next = load_dt(cu, k0);
+    int64_t k = k0;
+    for (;;) {
+        // the chunk after this one, possibly in the next segment
+        int64_t nu = u, nk = k + 1, nk0 = k0, nk1 = k1;
+        int nkind = kind;
+        bool more = true, newseg = false;
+        if (nk >= k1) {
+            if (seg + 1 < nseg) {
+                nkind = seg_of(seg + 1, nu, nk0, nk1);
+                nk = nk0;
+                newseg = true;
+            } else {
+                more = false;
+            }
+        }
+        const Unit nuu = newseg ? unit(nu) : cu;
+        const int64_t t0 = k * kM2T;
         const int steps = (int)(L - t0 < kM2T ? L - t0 : kM2T);
         asm volatile("cp.async.wait_group 0;" ::: "memory");
         // ---- per step: delta and the decay (steps past L keep the state)
@@ -187,11 +331,11 @@ __global__ void __launch_bounds__(kM2Threads, kM2MinCtas) scan_m2_kernel(const S
             sm.dd[tid] = make_float2(decay, delta);
         }
         __syncthreads();  // dd and this chunk's staged rows visible to all
-        if (ci + 1 < nchunks) {
-            fetch_xz(ci + 1);
-            load_dt(ci + 1);
+        if (more) {
+            fetch_xz(nuu, nk, bi ^ 1);
+            dt_next = load_dt(nuu, nk);
         }
-        const typename S::RawXZ& rw = sm.raw[ci & 1];
+        const typename S::RawXZ& rw = sm.raw[bi];
         // ---- widen: delta * x per (step, row), fp32 B / C rows (swizzled)
         for (int i = tid; i < kM2T * RPC / 8; i += kM2Threads) {
             const int t = i / (RPC / 8), e = (i % (RPC / 8)) * 8;
@@ -207,29 +351,29 @@ __global__ void __launch_bounds__(kM2Threads, kM2MinCtas) scan_m2_kernel(const S
             *reinterpret_cast<float4*>(&sm.dx[t][e + 4]) = make_float4(dl * xv[4], dl * xv[5], dl * xv[6], dl * xv[7]);
         }
         for (int i = tid; i < kM2T * N / 4; i += kM2Threads) {
-            const int t = i / (N / 4), u = i % (N / 4);  // 16-byte fp32 piece u of row t
+            const int t = i / (N / 4), uq = i % (N / 4);  // 16-byte fp32 piece uq of row t
             float bv[4], cv[4];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                bv[k] = to_f(sm.rawB[t][4 * u + k]);
-                cv[k] = to_f(sm.rawC[t][4 * u + k]);
+            for (int q = 0; q < 4; ++q) {
+                bv[q] = to_f(sm.rawB[t][4 * uq + q]);
+                cv[q] = to_f(sm.rawC[t][4 * uq + q]);
             }
-            const int su = m2_swz(u) * 4;
+            const int su = m2_swz(uq) * 4;
             *reinterpret_cast<float4*>(&sm.B[t][su]) = make_float4(bv[0], bv[1], bv[2], bv[3]);
             *reinterpret_cast<float4*>(&sm.C[t][su]) = make_float4(cv[0], cv[1], cv[2], cv[3]);
         }
         __syncthreads();
         // the raw B/C rows are widened: the next chunk's may land now
-        if (ci + 1 < nchunks) fetch_bc(ci + 1);
+        if (more) fetch_bc(nuu, nk);
         commit();
 
         // ---- scan: 4 groups of 4 steps
 #pragma unroll 1
         for (int tt = 0; tt < kM2T; tt += 4) {
-            float v[16];  // v[4r + k]: partial readout of row r at step tt + k
+            float v[16];  // v[4r + kk]: partial readout of row r at step tt + kk
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int t = tt + k;
+            for (int kk = 0; kk < 4; ++kk) {
+                const int t = tt + kk;
                 const float decay = sm.dd[t].x;
                 const u64 dA2 = pk(decay, decay);
                 const float4 dx4 = *reinterpret_cast<const float4*>(&sm.dx[t][4 * pg]);
@@ -256,7 +400,7 @@ __global__ void __launch_bounds__(kM2Threads, kM2MinCtas) scan_m2_kernel(const S
                 for (int r = 0; r < 4; ++r) {
                     float lo, hi;
                     upk(y2[r], lo, hi);
-                    v[4 * r + k] = lo + hi;
+                    v[4 * r + kk] = lo + hi;
                 }
             }
             // butterfly reduce-scatter over the NG threads of the row group:
@@ -282,7 +426,7 @@ __global__ void __launch_bounds__(kM2Threads, kM2MinCtas) scan_m2_kernel(const S
         // ---- epilogue: D skip and gate on 8 consecutive rows, 16-byte stores
         for (int i = tid; i < kM2T * RPC / 8; i += kM2Threads) {
             const int t = i / (RPC / 8), e = (i % (RPC / 8)) * 8;
-            if (t >= steps || e >= rows) continue;
+            if (t >= steps || e >= cu.rows) continue;
             float xv[8], zv[8], o[8];
             if constexpr (sizeof(IoT) == 2) {
                 Vec16<IoT>::unpack(*reinterpret_cast<const uint4*>(&rw.x[t][e]), xv);
@@ -297,11 +441,11 @@ __global__ void __launch_bounds__(kM2Threads, kM2MinCtas) scan_m2_kernel(const S
             const float4 y1 = *reinterpret_cast<const float4*>(&sm.y[t][e + 4]);
             const float ys[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                o[k] = fmaf(dskip, xv[k], ys[k]);
-                if (zg) o[k] *= silu_f(zv[k]);
+            for (int q = 0; q < 8; ++q) {
+                o[q] = fmaf(dskip, xv[q], ys[q]);
+                if (cu.zg) o[q] *= silu_f(zv[q]);
             }
-            IoT* dst = og + (t0 + t) * p.o_t + e;
+            IoT* dst = cu.og + (t0 + t) * p.o_t + e;
             if constexpr (sizeof(IoT) == 2) {
                 __stcs(reinterpret_cast<uint4*>(dst), Vec16<IoT>::pack(o));
             } else {
@@ -311,22 +455,60 @@ __global__ void __launch_bounds__(kM2Threads, kM2MinCtas) scan_m2_kernel(const S
         }
         // the next chunk overwrites dd / dx / B / C / y only after its own
         // first barrier, which every thread reaches after this epilogue
+
+        // ---- end of a segment: hand the tile over, or write the final state
+        if (k + 1 == k1) {
+            if (kind == 2) {
+                float* slot = mp.ws_slots + w * (int64_t)(RPC * N);
+#pragma unroll
+                for (int r = 0; r < 4; ++r)
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        float a, c;
+                        upk(hs[r][j], a, c);
+                        __stcg(reinterpret_cast<float2*>(slot + (4 * pg + r) * N + 16 * ng + 2 * j), make_float2(a, c));
+                    }
+                __threadfence();
+                __syncthreads();
+                if (tid == 0) m2_st_release(mp.ws_flags + w, gen + 1u);
+            } else if (p.ssm_state) {
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    const int row = 4 * pg + r;
+                    if (row >= cu.rows) continue;
+                    float* dst = p.ssm_state + cu.b * p.ss_b + cu.h * p.ss_h + (cu.p0 + row) * p.ss_p + 16 * ng * p.ss_n;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        float a, c;
+                        upk(hs[r][j], a, c);
+                        dst[(2 * j) * p.ss_n] = a;
+                        dst[(2 * j + 1) * p.ss_n] = c;
+                    }
+                }
+            }
+        }
+        if (!more) break;
+        if (newseg) {
+            ++seg;
+            u = nu;
+            k0 = nk0;
+            k1 = nk1;
+            kind = nkind;
+            cu = nuu;
+            __syncthreads();  // every thread is done with this segment's tile
+            setup();
+        }
+        k = nk;
+        bi ^= 1;
     }
 
-    // ---- final state
-    if (p.ssm_state) {
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            const int row = 4 * pg + r;
-            if (row >= rows) continue;
-            float* dst = p.ssm_state + b * p.ss_b + h * p.ss_h + (p0 + row) * p.ss_p + 16 * ng * p.ss_n;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                float a, c;
-                upk(hs[r][j], a, c);
-                dst[(2 * j) * p.ss_n] = a;
-                dst[(2 * j + 1) * p.ss_n] = c;
-            }
+    // ---- the last CTA to finish advances the workspace generation
+    if (mp.ws_head) {
+        __syncthreads();
+        if (tid == 0) {
+            __threadfence();
+            const unsigned old = m2_atom_inc(mp.ws_head + 1, (unsigned)(mp.workers - 1));
+            if (old == (unsigned)(mp.workers - 1)) atomicAdd(mp.ws_head, 1u);
         }
     }
 }
@@ -384,27 +566,38 @@ __global__ void __launch_bounds__(128) scan_m2_generic_kernel(const ScanM2Proble
 }
 
 template <typename IoT, int NG>
-cudaError_t launch_m2_ng(const ScanM2Problem& p, cudaStream_t s) {
+cudaError_t launch_m2_ng(const ScanM2Problem& p, const M2Plan& mp, cudaStream_t s) {
     using Sm = M2Smem<IoT, NG>;
     auto kern = scan_m2_kernel<IoT, NG>;
     const int smem = (int)sizeof(Sm);
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
-    if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)((p.P + Sm::RPC - 1) / Sm::RPC), (unsigned)p.H, (unsigned)p.Bn);
-    kern<<<grid, kM2Threads, smem, s>>>(p);
-    return cudaGetLastError();
+    if (m2_ctas_per_sm<IoT, NG>(mp.dev) <= 0) return cudaErrorInvalidConfiguration;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)mp.grid);
+    cfg.blockDim = dim3(kM2Threads);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = mp.cooperative ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, p, mp);
 }
 
 template <typename IoT>
-cudaError_t launch_m2_io(const ScanM2Problem& p, cudaStream_t s) {
+cudaError_t launch_m2_io(const ScanM2Problem& p, const M2Plan& mp, cudaStream_t s, int* ctas) {
     switch (p.N / 16) {
-        case 1: return launch_m2_ng<IoT, 1>(p, s);
-        case 2: return launch_m2_ng<IoT, 2>(p, s);
-        case 4: return launch_m2_ng<IoT, 4>(p, s);
-        case 8: return launch_m2_ng<IoT, 8>(p, s);
-        case 16: return launch_m2_ng<IoT, 16>(p, s);
+#define SSM_M2_CASE(ng)                                              \
+    case ng:                                                         \
+        if (ctas) {                                                  \
+            *ctas = m2_ctas_per_sm<IoT, ng>(mp.dev);                 \
+            return cudaSuccess;                                      \
+        }                                                            \
+        return launch_m2_ng<IoT, ng>(p, mp, s);
+        SSM_M2_CASE(4)
+        SSM_M2_CASE(8)
+        SSM_M2_CASE(16)
+#undef SSM_M2_CASE
         default: return cudaErrorInvalidValue;
     }
 }
@@ -434,12 +627,26 @@ int scan_m2_smem_bytes(int io_dt, int64_t N) {
     return pick(__nv_bfloat16{});
 }
 
-cudaError_t launch_scan_m2(const ScanM2Problem& p, int kernel, cudaStream_t s) {
+int scan_m2_ctas_per_sm(const ScanM2Problem& p, int dev) {
+    M2Plan mp{};
+    mp.dev = dev;
+    int n = 0;
+    cudaError_t e = cudaErrorInvalidValue;
+    switch (p.io_dt) {
+        case kF32: e = launch_m2_io<float>(p, mp, nullptr, &n); break;
+        case kF16: e = launch_m2_io<__half>(p, mp, nullptr, &n); break;
+        case kBF16: e = launch_m2_io<__nv_bfloat16>(p, mp, nullptr, &n); break;
+        default: break;
+    }
+    return e == cudaSuccess ? n : 0;
+}
+
+cudaError_t launch_scan_m2(const ScanM2Problem& p, int kernel, const M2Plan& mp, cudaStream_t s) {
     if (kernel == SSM_KERNEL_SCAN_M2) {
         switch (p.io_dt) {
-            case kF32: return launch_m2_io<float>(p, s);
-            case kF16: return launch_m2_io<__half>(p, s);
-            case kBF16: return launch_m2_io<__nv_bfloat16>(p, s);
+            case kF32: return launch_m2_io<float>(p, mp, s, nullptr);
+            case kF16: return launch_m2_io<__half>(p, mp, s, nullptr);
+            case kBF16: return launch_m2_io<__nv_bfloat16>(p, mp, s, nullptr);
             default: return cudaErrorInvalidValue;
         }
     }

@@ -178,3 +178,47 @@ def test_m2_prefill_full_size_sampled_heads():
         assert_close(N(h[b:b + 1, hh:hh + 1]), href, TOL["f16"], f"state[{b},{hh}]")
     del xs, zs, outs
     torch.cuda.empty_cache()
+
+
+# ------------------------------------------- balanced slices with hand-overs --
+def _m2_slots(N_):
+    import torch
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    return sms * 3  # resident CTAs of the fast kernel (3 per SM)
+
+
+@pytest.mark.parametrize("io,N_,P,L", [("f16", 128, 64, 200), ("bf16", 256, 128, 72), ("f32", 64, 64, 56)])
+def test_m2_prefill_balanced_slices_match_oracle_and_whole_units(io, N_, P, L):
+    """More (batch, head, row block) units than resident CTAs: CTAs take equal
+    slices of the (unit, 16-step chunk) list and hand 32 KB state tiles over
+    through the workspace.  Results match the oracle and equal the run
+    without a workspace (one whole unit per CTA) bit for bit."""
+    from state_space_model_causal_b200 import ssm_selective_scan_workspace_size
+    rpc = 512 // (N_ // 16)
+    blocks = -(-P // rpc)
+    H = 8
+    Bt = -(-(_m2_slots(N_) + 31) // (H * blocks))
+    s = gen.scan_m2_inputs(Bt, H, P, N_, L, io=io, seed=5, tag=f"m2bal{io}{N_}", h0=True,
+                           with_z=True)
+    x = _time_major(s.x, io, (0, 3, 1, 2))
+    assert ssm_selective_scan_workspace_size(
+        x, _time_major(s.dt, io, (0, 2, 1)), T(s.A, "f32"), _time_major(s.B, io, (0, 3, 1, 2)),
+        _time_major(s.C, io, (0, 3, 1, 2))) > 0, "problem too small to split"
+    _check(s, kernel="scan_m2")
+    # the same call without a workspace runs whole units: identical results
+    import torch
+    from state_space_model_causal_b200 import ssm_selective_scan_fwd
+
+    def run(workspace):
+        out = _time_major(np.zeros(s.x.shape), io, (0, 3, 1, 2))
+        h = T(s.h0, "f32")
+        ssm_selective_scan_fwd(x, _time_major(s.dt, io, (0, 2, 1)), T(s.A, "f32"),
+                               _time_major(s.B, io, (0, 3, 1, 2)), _time_major(s.C, io, (0, 3, 1, 2)),
+                               D=T(s.D, "f32"), z=_time_major(s.z, io, (0, 3, 1, 2)),
+                               dt_bias=T(s.dt_bias, "f32"), ssm_state=h, out=out, workspace=workspace)
+        torch.cuda.synchronize()
+        return N(out), N(h)
+
+    a, b = run("auto"), run(None)
+    np.testing.assert_array_equal(a[0], b[0])
+    np.testing.assert_array_equal(a[1], b[1])
