@@ -42,7 +42,11 @@ METRIC = "scan Gelem/s (B·L·D·N) prefill; SSU decode HBM GB/s vs B200 peak, p
 WORKLOAD = "mamba1-2.8b-prefill: conv1d(W=4)+SiLU+selective-scan+gate, B=4 L=2048 D=5120 N=16, fp16 I/O"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
-SFU_EX2_PER_CLK_PER_SM = 16  # MUFU ex2 throughput per SM per clock
+SFU_EX2_PER_CLK_PER_SM = 16  # nominal SFU ex2 throughput per SM per clock
+# SFU operations per (b, t, d, n) element of the fused prefill: the decay
+# exp(delta*A), plus per (b, t, d) the exponentials of the conv SiLU, the
+# softplus and the gate (their reciprocals run on the FMA pipe), over N = 16
+PREFILL_SFU_PER_ELEM = 1.0 + 3.0 / 16
 NUM_SMS = 148
 SM_MAX_MHZ = 1965.0
 
@@ -56,6 +60,66 @@ def peaks():
         return float(p["hbm_gbs"]), float(p.get("sm_max_mhz", SM_MAX_MHZ)), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, SM_MAX_MHZ, "fallback"
+
+
+def sfu_rate():
+    """ex2 operations per clock per SM: the rate `python bench.py --peaks`
+    measured on this machine's B200s (recorded in profiles/sfu_pipe_rates.txt),
+    else the nominal 16."""
+    try:
+        for line in open(os.path.join(ROOT, "profiles", "sfu_pipe_rates.txt")):
+            if line.startswith("ex2_per_clk_per_sm:"):
+                return float(line.split(":", 1)[1]), "measured (bench.py --peaks)"
+    except OSError:
+        pass
+    return float(SFU_EX2_PER_CLK_PER_SM), "nominal"
+
+
+# Microbenchmark of the SFU: 16 independent chains per thread, inputs changed
+# by an FMA every iteration, 8 warps per SM sub-partition.
+PEAKS_SRC = r"""
+#include <cstdio>
+#include <cuda_runtime.h>
+__device__ __forceinline__ float ex2(float x) { float y; asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x)); return y; }
+__device__ __forceinline__ float rcp(float x) { float y; asm volatile("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x)); return y; }
+template <int OP> __global__ void k(float* out, int iters) {
+  float x[16], acc[16];
+  for (int j = 0; j < 16; ++j) { x[j] = -0.01f * (threadIdx.x + j); acc[j] = 0.f; }
+  for (int it = 0; it < iters; ++it) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) { x[j] = fmaf(x[j], 0.9999f, -1e-4f); acc[j] += OP == 0 ? ex2(x[j]) : rcp(x[j] - 3.0f); }
+  }
+  float s = 0; for (int j = 0; j < 16; ++j) s += acc[j];
+  if (s == 1234.5f) out[0] = s;
+}
+int main() {
+  float* d; if (cudaMalloc(&d, 4) != cudaSuccess) return 1;
+  int sms, clk; cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, 0); cudaDeviceGetAttribute(&clk, cudaDevAttrClockRate, 0);
+  cudaEvent_t a, b; cudaEventCreate(&a); cudaEventCreate(&b);
+  for (int op = 0; op < 2; ++op) {
+    const int iters = 4096, blocks = sms * 8;
+    auto L = [&] { if (op == 0) k<0><<<blocks, 128>>>(d, iters); else k<1><<<blocks, 128>>>(d, iters); };
+    L(); cudaDeviceSynchronize(); cudaEventRecord(a); L(); cudaEventRecord(b); cudaEventSynchronize(b);
+    float ms; cudaEventElapsedTime(&ms, a, b);
+    printf("%s_per_clk_per_sm: %.3f\n", op == 0 ? "ex2" : "rcp", (double)blocks * 128 * 16 * iters / (ms * 1e-3) / sms / (clk * 1e3));
+  }
+  return cudaGetLastError() == cudaSuccess ? 0 : 1;
+}
+"""
+
+
+def run_peaks():
+    """Compile and run the SFU microbenchmark; print its rates at the max SM clock."""
+    import tempfile
+    with tempfile.TemporaryDirectory() as tmp:
+        src = os.path.join(tmp, "sfu.cu")
+        exe = os.path.join(tmp, "sfu")
+        with open(src, "w") as f:
+            f.write(PEAKS_SRC)
+        subprocess.check_call(["nvcc", "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-o", exe, src])
+        out = subprocess.run([exe], capture_output=True, text=True, check=True).stdout
+    print(out, end="", flush=True)
+    return 0
 
 
 def src_hash(*names):
@@ -385,15 +449,26 @@ def decode_mamba1_2p8b(dev, hbm_peak, slabs=64, replays=20):
             "l2": "each call on a different 100 MB slab", "gpu_launches_per_replay": slabs}
 
 
-def decode_mamba2(dev, hbm_peak, H, P, N, R, cache, io, replays=10, calls_per_graph=5):
-    """Mamba-2 SSU at effective batch R; slabs rotate so every call of the
-    graph touches state that is not resident in L2."""
+def decode_mamba2(dev, hbm_peak, H, P, N, R, cache, io, method="cold", replays=10, calls_per_graph=5):
+    """Mamba-2 SSU at effective batch R, timed one of two ways:
+
+    * "cold": the calls of the graph rotate over ceil(2 * L2 / slab) state
+      slabs (at least `calls_per_graph` calls, one per slab when there are
+      more slabs), so no call finds its state in L2;
+    * "pages": the timing method of the vLLM SSU benchmark -- 20 eager warm-up
+      calls, a graph of 10 calls on the same buffers, 5 warm replays, 100
+      timed replays; at small R the state stays in L2.
+    """
     import torch
     from state_space_model_causal_b200 import inputs as gen, ssm_selective_state_update
     Bt, Hr = gen.effective_batch_shape(R, H)
     es = 4 if cache == "f32" else 2
     state_bytes = Bt * Hr * P * N * es
-    nslab = max(1, min(calls_per_graph, math.ceil(2 * L2_BYTES / state_bytes)))
+    if method == "pages":
+        nslab, ncalls, warm_eager, replays = 1, 10, 20, 100
+    else:
+        nslab = max(1, math.ceil(2 * L2_BYTES / state_bytes))
+        ncalls, warm_eager = max(calls_per_graph, nslab), 3
     tag = ("bench", "mamba2", H, P, N, R, cache)
     A = -torch.from_numpy(gen.uniform((Hr,), 1.0, 16.0, *tag, "A").astype(np.float32)).to(dev)
     db = torch.from_numpy(gen.dt_bias_draw((Hr,), *tag, "db").astype(np.float32)).to(dev)
@@ -408,11 +483,11 @@ def decode_mamba2(dev, hbm_peak, H, P, N, R, cache, io, replays=10, calls_per_gr
         out = torch.empty_like(x)
         b = (st, x, dt, Bm, Cm, out)
         bufs.append(b)
-    for i in range(calls_per_graph):
+    for i in range(ncalls):
         b = bufs[i % nslab]
         calls.append(lambda b=b: ssm_selective_state_update(
             b[0], b[1], b[2], A, b[3], b[4], D=Dv, dt_bias=db, out=b[5]))
-    us, med = graph_time(calls, replays, dev)
+    us, med = graph_time(calls, replays, dev, warm_eager=warm_eager)
     rows = Bt * Hr * P
     nbytes = rows * N * es * 2 + rows * 2 * 2 + Bt * Hr * 2 + Bt * N * 2 * 2 + Hr * 4 * 3
     gbs = nbytes / (us * 1e-6) / 1e9
@@ -420,13 +495,62 @@ def decode_mamba2(dev, hbm_peak, H, P, N, R, cache, io, replays=10, calls_per_gr
     torch.cuda.empty_cache()
     traffic = profiled_traffic(f"ssu_head_tma_mamba2_{P}x{N}_{cache}_R{R}.txt",
                                ["ssu.cu", "common.cuh", "tma.cuh"])
+    l2 = (f"{nslab} state slabs rotated ({nslab * state_bytes / 2**20:.0f} MiB, >= 2 x L2 or one slab larger)"
+          if method == "cold" else f"same buffers, {state_bytes / 2**20:.1f} MiB of state")
     return {"workload": f"mamba2-ssu: H={H} P={P} N={N} G=1, {io} io, {cache} cache",
+            "method": method,
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
                          "frac": round(gbs / hbm_peak, 4), "traffic": traffic},
-            "effective_batch": R, "batch": Bt, "heads": Hr, "P": P, "N": N, "us_per_call": round(us, 3),
-            "us_median": round(med, 3), "bytes_per_call": nbytes, "GBps": round(gbs, 1),
-            "frac_of_hbm_peak": round(gbs / hbm_peak, 4),
-            "l2": f"{nslab} state slabs rotated ({nslab * state_bytes / 2**20:.0f} MiB)"}
+            "requested_R": R, "effective_batch": Bt * Hr, "batch": Bt, "heads": Hr, "P": P, "N": N,
+            "us_per_call": round(us, 3), "us_median": round(med, 3), "bytes_per_call": nbytes,
+            "GBps": round(gbs, 1), "frac_of_hbm_peak": round(gbs / hbm_peak, 4), "l2": l2,
+            "calls_per_graph": ncalls}
+
+
+def eager_latency(dev, R, calls=300):
+    """Host cost of one eager ssm_selective_state_update call (Mamba-2 layout,
+    H=80 P=64 N=128, fp16): the wall time per call of `calls` back-to-back
+    calls of the C entry point with its argument struct built once (library
+    checks, planning and launch), and through the Python binding (argument
+    marshalling included).  The GPU work of these sizes is shorter than the
+    host path, so the host path is what is timed."""
+    import ctypes
+
+    import torch
+    from state_space_model_causal_b200 import binding, inputs as gen, ssm_selective_state_update
+    H, P, N = 80, 64, 128
+    Bt, Hr = gen.effective_batch_shape(R, H)
+    tag = ("bench", "eager", R)
+    st = gen.device_normal((Bt, Hr, P, N), "f16", *tag, "state", device=dev)
+    x = gen.device_normal((Bt, Hr, P), "f16", *tag, "x", device=dev)
+    dt = gen.device_uniform((Bt, Hr), -4.0, -1.0, "f16", *tag, "dt", device=dev)
+    Bm = gen.device_normal((Bt, 1, N), "f16", *tag, "B", device=dev)
+    Cm = gen.device_normal((Bt, 1, N), "f16", *tag, "C", device=dev)
+    A = -torch.linspace(1.0, 16.0, Hr, device=dev)
+    Dv, db = torch.ones(Hr, device=dev), torch.full((Hr,), -3.0, device=dev)
+    out = torch.empty_like(x)
+    a = binding.SsuArgs()
+    a.struct_size = ctypes.sizeof(binding.SsuArgs)
+    a.state, a.x, a.dt, a.A, a.B, a.C, a.D, a.dt_bias, a.out = map(binding.describe, (st, x, dt, A, Bm, Cm, Dv, db, out))
+    a.dt_softplus = 1
+    lib = binding.library()
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    for _ in range(20):
+        if lib.ssm_selective_state_update(ctypes.byref(a), stream) != 0:
+            raise RuntimeError("ssm_selective_state_update refused the eager-latency case")
+    torch.cuda.synchronize(dev)
+    t0 = time.perf_counter()
+    for _ in range(calls):
+        lib.ssm_selective_state_update(ctypes.byref(a), stream)
+    t_c = (time.perf_counter() - t0) / calls
+    torch.cuda.synchronize(dev)
+    t0 = time.perf_counter()
+    for _ in range(calls):
+        ssm_selective_state_update(st, x, dt, A, Bm, Cm, D=Dv, dt_bias=db, out=out)
+    t_py = (time.perf_counter() - t0) / calls
+    torch.cuda.synchronize(dev)
+    return {"requested_R": R, "effective_batch": Bt * Hr, "c_call_us": round(t_c * 1e6, 2),
+            "python_call_us": round(t_py * 1e6, 2)}
 
 
 # ------------------------------------------------------------- reference --
@@ -488,16 +612,50 @@ def oracle_beside(entry, kind, rows=None):
             "sample": f"{sample}; fp64 sequential C on one host thread, {dt:.2f} s"}
 
 
+def oracle_prefill_threads(channels, threads, seed=0):
+    """The oracle on `channels` channels of the prefill recipe split into
+    `threads` contiguous channel ranges, one host thread each (the C oracle
+    runs with the GIL released, and channels are independent); returns
+    (wall seconds, elements)."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    import oracle
+    from state_space_model_causal_b200 import inputs as gen
+    channels = max(threads, min(4 * 5120, channels))
+    Bt = -(-channels // 5120)
+    s = gen.prefill_2p8b(seed=seed, Bt=Bt, D=-(-channels // Bt))
+    Dd = s.x.shape[1]
+    cuts = [Dd * i // threads for i in range(threads + 1)]
+    parts = [slice(cuts[i], cuts[i + 1]) for i in range(threads) if cuts[i + 1] > cuts[i]]
+
+    def one(sl):
+        oracle.scan(s.x[:, sl], s.dt[:, sl], s.A[sl], s.B, s.C, D=s.D[sl], z=s.z[:, sl],
+                    dt_bias=s.dt_bias[sl], conv_weight=s.conv_weight[sl], conv_bias=s.conv_bias[sl])
+
+    with ThreadPoolExecutor(len(parts)) as pool:
+        t0 = time.perf_counter()
+        list(pool.map(one, parts))
+        dt = time.perf_counter() - t0
+    return dt, s.x.shape[0] * Dd * s.x.shape[2] * s.A.shape[1]
+
+
 def cpu_baseline(target_s=10.0):
+    """The fp64 oracle timed on the host: on every core the process may use
+    (one channel range per thread), plus the one-thread figure beside it."""
     import oracle
     oracle.build()
-    t, e = oracle_prefill_sample(64)
-    ch = int(64 * target_s / max(t, 1e-3))
-    t, e = oracle_prefill_sample(ch)
+    t1, e1 = oracle_prefill_sample(64)
+    one_thread = e1 / t1 / 1e9
+    cores = max(1, min(64, len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity")
+                       else (os.cpu_count() or 1)))
+    ch = max(cores, min(4 * 5120, int(64 * cores * target_s / max(t1, 1e-3))))
+    t, e = oracle_prefill_threads(ch, cores)
     ch = e // (2048 * 16)
-    return {"value": round(e / t / 1e9, 6), "unit": "Gelem/s", "cores": 1, "kind": "oracle",
+    return {"value": round(e / t / 1e9, 6), "unit": "Gelem/s", "cores": cores, "kind": "oracle",
+            "single_thread_value": round(one_thread, 6),
             "sample": f"{ch} of the 20480 (b,d) channels of the 2.8B-shaped prefill, full "
-                      f"L=2048, fp64 sequential C on one thread, {t:.1f} s"}
+                      f"L=2048, fp64 C over {cores} host threads (one channel range each), "
+                      f"{t:.1f} s; one thread: 64 channels in {t1:.3f} s"}
 
 
 # ------------------------------------------------------- multi-rank host --
@@ -524,15 +682,19 @@ def run_reference(args):
         return 0
     import oracle
     oracle.build()
+    cores = max(1, min(64, len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity")
+                       else (os.cpu_count() or 1)))
     t, _ = oracle_prefill_sample(64)
-    ch = max(64, min(5120, int(64 * 5.0 / max(t, 1e-3))))  # ~5 s of CPU work per step
+    # about 5 s of CPU work per step, over every host core
+    ch = max(64, min(4 * 5120, int(64 * cores * 5.0 / max(t, 1e-3))))
     for _ in range(args.warmup):
-        oracle_prefill_sample(ch)
+        oracle_prefill_threads(ch, cores)
     times, elems = [], 0
     for _ in range(args.steps):
-        t, e = oracle_prefill_sample(ch)
+        t, e = oracle_prefill_threads(ch, cores)
         times.append(t)
         elems = e
+    ch = elems // (2048 * 16)
     ms = 1000.0 * statistics.mean(times)
     value = elems / (ms / 1000.0) / 1e9
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "Gelem/s",
@@ -541,8 +703,9 @@ def run_reference(args):
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": WORKLOAD, "sample": f"{ch} channels x L=2048 per step",
                        "l2": "n/a (host)"},
-            "cpu_baseline": {"value": round(value, 6), "unit": "Gelem/s", "cores": 1,
-                             "kind": "oracle", "sample": f"{ch} (b,d) channels per step"},
+            "cpu_baseline": {"value": round(value, 6), "unit": "Gelem/s", "cores": cores,
+                             "kind": "oracle",
+                             "sample": f"{ch} (b,d) channels x L=2048 per step over {cores} threads"},
             "e2e": {"value": round(value, 6), "unit": "Gelem/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -551,17 +714,24 @@ def run_reference(args):
 
 # ---------------------------------------------------------------- sweep --
 def run_sweep(dev, hbm_peak):
+    """Mamba-2 SSU per effective batch, both timing methods, both cache dtypes
+    of both configs; then the eager host latency per call."""
     out = []
-    for cache in ("f16", "f32"):
-        for R in (8, 16, 32, 64, 128, 256, 512, 1024, 2048, 4096, 8192, 16384, 32768, 65536, 131072):
-            r = decode_mamba2(dev, hbm_peak, 80, 64, 128, R, cache, "f16", replays=20)
-            print(json.dumps(r), flush=True)
-            out.append(r)
-    for cache in ("bf16", "f32"):
-        for R in (8, 16, 32, 64, 128, 256, 512, 1024, 2048, 4096, 8192, 16384, 32768, 65536):
-            r = decode_mamba2(dev, hbm_peak, 32, 128, 256, R, cache, "bf16", replays=20)
-            print(json.dumps(r), flush=True)
-            out.append(r)
+    grids = ((80, 64, 128, ("f16", "f32"), "f16",
+              (8, 16, 32, 64, 128, 256, 512, 1024, 2048, 4096, 8192, 16384, 32768, 65536, 131072)),
+             (32, 128, 256, ("bf16", "f32"), "bf16",
+              (8, 16, 32, 64, 128, 256, 512, 1024, 2048, 4096, 8192, 16384, 32768, 65536)))
+    for H, P, N, caches, io, Rs in grids:
+        for cache in caches:
+            for R in Rs:
+                for method in (("pages", "cold") if R <= 2048 else ("cold",)):
+                    r = decode_mamba2(dev, hbm_peak, H, P, N, R, cache, io, method=method, replays=20)
+                    print(json.dumps(r), flush=True)
+                    out.append(r)
+    for R in (8, 64, 256, 1024):
+        r = eager_latency(dev, R)
+        print(json.dumps({"eager_host_latency": r}), flush=True)
+        out.append(r)
     return out
 
 
@@ -629,6 +799,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--sweep", action="store_true", help="per-effective-batch decode sweep lines")
+    ap.add_argument("--peaks", action="store_true", help="measure the SFU ex2 / rcp rates and exit")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--only", choices=["prefill", "prefill_m2", "decode_m1", "m2_f16", "m2_f32",
@@ -643,6 +814,8 @@ def main():
 
     if args.impl == "reference":
         return run_reference(args)
+    if args.peaks:
+        return run_peaks()
 
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -686,14 +859,19 @@ def main():
     value = job_throughput(world, pf.elems, ms_step)
 
     # roofline of the prefill kernel: one exp(delta*A) per element on the SFU
-    sfu_peak = NUM_SMS * SFU_EX2_PER_CLK_PER_SM * sm_max * 1e6 / 1e9  # Gelem/s
+    ex2_rate, ex2_kind = sfu_rate()
+    sfu_peak = NUM_SMS * ex2_rate * sm_max * 1e6 / 1e9  # Gelem/s
     alg_bytes = pf.algorithmic_bytes()
     hbm_gbs = alg_bytes / (ms_step * 1e-3) / 1e9
-    traffic = profiled_traffic("scan_vec_prefill_2p8b.txt", ["scan_vec.cu", "common.cuh"])
-    roofline = {"bound": "alu", "achieved": round(pf.elems / (ms_step * 1e-3) / 1e9, 2),
+    traffic = profiled_traffic("scan_bal_prefill_2p8b.txt", ["scan_bal.cu", "common.cuh"])
+    achieved = pf.elems / (ms_step * 1e-3) / 1e9
+    roofline = {"bound": "alu", "achieved": round(achieved, 2),
                 "peak": round(sfu_peak, 1), "unit": "Gelem/s",
-                "frac": round(pf.elems / (ms_step * 1e-3) / 1e9 / sfu_peak, 4),
-                "traffic": traffic, "peak_kind": "SFU ex2 16/clk/SM x 148 SMs x max SM clock",
+                "frac": round(achieved / sfu_peak, 4),
+                "traffic": traffic,
+                "peak_kind": f"SFU ex2 {ex2_rate:g}/clk/SM ({ex2_kind}) x {NUM_SMS} SMs x max SM clock",
+                "sfu_ops_per_elem": PREFILL_SFU_PER_ELEM,
+                "frac_all_sfu_ops": round(achieved * PREFILL_SFU_PER_ELEM / sfu_peak, 4),
                 "hbm_achieved_gbs": round(hbm_gbs, 1), "hbm_peak_gbs": hbm_peak,
                 "hbm_frac": round(hbm_gbs / hbm_peak, 4), "hbm_peak_kind": peak_src,
                 "algorithmic_bytes_per_launch": alg_bytes}

@@ -11,38 +11,44 @@
 //   out   = (sum_n C[n,t] * h[n] + D[d] * u) * silu(z[t])
 //
 // What bounds it: the SFU.  Every (b, t, d, n) element needs one
-// exp(delta * A) and every (b, t, d) five more transcendentals; the four FP32
-// operations per element and the HBM traffic (8 bytes per (b, t, d)) are far
-// below their own ceilings.  The design keeps the SFU fed evenly on every SM
-// sub-partition:
+// exp(delta * A) and every (b, t, d) three more SFU operations (the
+// exponentials of the conv SiLU, the softplus and the gate; their reciprocals
+// run on the FMA pipe); the four FP32 operations per element and the HBM
+// traffic (8 bytes per (b, t, d)) are far below their own ceilings.  The
+// design keeps the SFU fed evenly on every SM sub-partition:
 //
 //   * Work is split into units (batch entry, 16 channels) x the whole
 //     sequence, each cut into 32-step chunks.  A warp is a worker; the workers
-//     are persistent and each takes an equal, contiguous slice of the
-//     flattened (unit, chunk) list, so every sub-partition gets the same
-//     number of chunks to within one -- whole units per warp would leave some
-//     sub-partitions with one unit more than others for the whole kernel.
-//     A slice is [tail of unit U][whole units][head of unit V]; the worker
-//     runs the head first and publishes the state it reaches (1 KB) to its
-//     successor, then its whole units, then the tail, which starts from the
-//     state its predecessor published at the very beginning of its own run.
-//     The hand-over needs a caller-supplied workspace; without one every
-//     worker takes whole units.  All waits are bounded.
-//   * In a warp, lane (c, q) owns channel c and state entries 8q .. 8q+7; the
-//     packed f32x2 operations run across state entries, so B[n], B[n+1] form
-//     one operand straight from shared memory with no widening or duplication.
-//   * Per chunk, B and C rows (16-bit, [n][t]) are widened once into fp32
-//     [t][n] rows: one broadcast 16-byte load gives four state entries of a
-//     step.  (delta, delta, delta*u, delta*u) of a (channel, step) is one
-//     16-byte word written by the lane that computed the prologue.
+//     are persistent (two per sub-partition) and each takes an equal,
+//     contiguous slice of the flattened (unit, chunk) list, so every
+//     sub-partition gets the same number of chunks to within one -- whole
+//     units per warp would leave some sub-partitions with one unit more than
+//     others for the whole kernel.  A slice is [tail of unit U][whole units]
+//     [head of unit V]; the worker runs the head first and publishes the state
+//     it reaches (1 KB) to its successor, then its whole units, then the tail,
+//     which starts from the state its predecessor published at the very
+//     beginning of its own run.  The hand-over needs a caller-supplied
+//     workspace; without one every worker takes whole units.  All waits are
+//     bounded.
+//   * With few units (short batches) the sequence is cut into pieces run in
+//     two passes (context-parallel mode, see BalPlan): pieces from zero states
+//     with end-state records, then re-scans from the states the records
+//     compose to.
+//   * In a warp, lane (cp, q) holds channels 2cp, 2cp+1 x state entries
+//     4q..4q+3; the packed f32x2 operations run across state entries, so
+//     B[n], B[n+1] form one operand straight from the widened fp32 [t][n] rows.
 //   * The lane that stages 16 steps of a channel computes their conv, SiLU,
-//     softplus, D*u and gate in registers (history by shuffle) and later
-//     applies D*u and the gate to the same steps.
-//   * The readout of a step is summed over the two lanes of a channel by one
-//     shuffle per two steps.
+//     softplus, D*u and gate in registers (history by shuffle), writes
+//     (delta, delta*u) for the scan lanes and later applies D*u and the gate
+//     to the same steps.
+//   * Readout partials go to shared memory once per 4-step group, after the
+//     next group's first operands are loaded (a store ahead of the loads
+//     would hold them back); the epilogue lane sums the four partials of a
+//     (step, channel).  Padded and swizzled layouts keep every shared-memory
+//     access conflict-free.
 //   * The next chunk's x/dt/z/B/C tiles are copied by cp.async while the
 //     current one is computed (double buffer).
-//   * Optionally SW of every eight exponentials take their value from the
+//   * Optionally SW of every eight exponential pairs take their value from the
 //     Cody-Waite + minimax polynomial on the FMA pipe instead of the SFU.
 #include "../../include/ssm_causal.h"
 #include "common.cuh"
