@@ -231,9 +231,20 @@ __global__ void __launch_bounds__(256, 3) ssu_head_kernel(const SsuProblem p, co
 // new state back with 16-byte stores.  `lpr` lanes share a row, each owning
 // CPL 16-byte chunks; a thread owns RPT rows of an item, and the RPT partial
 // readouts of a thread are summed over the row's lanes by a butterfly
-// reduce-scatter.  I/O dtype IoT is a template parameter.
+// reduce-scatter.  I/O dtype IoT is a template parameter.  With one dt per
+// head, the items' scalars (Delta, exp(Delta*A), D, the B/C group) are
+// computed 32 items at a time, one item per lane of the CTA's last warp, into
+// a ring in shared memory that the per-item barrier publishes; the other
+// threads only read them.  The warp loads a batch's inputs 32 items before it
+// computes them, so no barrier waits on those loads.
 // ------------------------------------------------------------------------
 constexpr int kTmaStagesMax = 4;
+constexpr int kScBatch = 32;  // items per batch of scalars (one per lane)
+
+struct ItemScalars {
+    float delta, dA, dskip;
+    int g;
+};
 
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
@@ -264,6 +275,7 @@ __global__ void __launch_bounds__(256, 3) ssu_head_tma_kernel(const SsuProblem p
     constexpr int VE = V::VE;
     extern __shared__ __align__(128) unsigned char tma_stage[];
     __shared__ __align__(8) uint64_t full[kTmaStagesMax];
+    __shared__ __align__(16) ItemScalars item_sc[2 * kScBatch];  // two batches
 
     const unsigned tid = threadIdx.x;
     const unsigned lpr = (unsigned)plan.lpr;
@@ -316,10 +328,11 @@ __global__ void __launch_bounds__(256, 3) ssu_head_tma_kernel(const SsuProblem p
         const int64_t sl = p.slot_idx[b * p.si_b];
         return (sl < 0 || sl >= p.n_slots) ? -1 : sl;
     };
-    // thread 0: start the copies of the item at `q` into stage k % S; a
-    // padding row completes the stage's phase without data
-    auto issue = [&](unsigned k, const Pos& q) {
-        uint64_t* bar = &full[k % S];
+    // thread 0: start the copies of local item k (at `q`) into stage `sg`,
+    // with the item's scalars (one dt per head); a padding row completes the
+    // stage's phase without data
+    auto issue = [&](unsigned k, unsigned sg, const Pos& q) {
+        uint64_t* bar = &full[sg];
 #ifdef SSM_TEST_HOOKS
         if ((int64_t)(i0 + k) == plan.drop_item) return;  // failure test: never completes
 #endif
@@ -335,12 +348,48 @@ __global__ void __launch_bounds__(256, 3) ssu_head_tma_kernel(const SsuProblem p
         const IoT* xs = xg + q.b * p.x_b + (int64_t)q.h * p.x_h + p0;
         const uint32_t sbytes = nr * row_bytes;
         const uint32_t xbytes = (nr * (unsigned)sizeof(IoT) + 15u) & ~15u;
-        unsigned char* dst = tma_stage + (k % S) * stage_bytes;
+        unsigned char* dst = tma_stage + sg * stage_bytes;
         mbar_arrive_expect_tx(bar, sbytes + xbytes);
         tma_load_1d(dst, src, sbytes, bar);
         tma_load_1d(dst + x_off, xs, xbytes, bar);
     };
 
+    // last warp: the inputs of local items 32*j .. 32*j+31 (one per lane) are
+    // loaded into registers by sc_load(j) and turned into ring entries
+    // (item & 63) by sc_store(j).  Padding rows get entries too (x and dt are
+    // indexed by batch row, not by cache slot); nobody reads them.
+    // (measured: the ring pays for 16-bit caches, whose kernels are
+    // issue-bound; fp32-cache items keep per-thread scalars, loaded before the
+    // stage wait)
+    const bool ring = sizeof(ST) == 2 && !dt_row;
+    const bool sc_lane = ring && tid / 32 == blockDim.x / 32 - 1;
+    float sc_v = 0.0f, sc_a = 0.0f, sc_d = 0.0f;
+    int sc_g = 0;
+    auto sc_load = [&](unsigned j) {
+        const unsigned k = j * kScBatch + (tid & 31u);
+        if (k >= cnt) return;
+        const Pos q = first(i0 + k);
+        sc_v = to_f(dtg[q.b * p.dt_b + q.h * p.dt_h]);
+        if (p.dt_bias) sc_v += p.dt_bias[q.h * p.db_h];
+        sc_a = p.A[q.h * p.A_h] * kLog2e;
+        sc_d = p.Dp ? p.Dp[q.h * p.D_h] : 0.0f;
+        sc_g = p.G == 1 ? 0 : (int)(q.h / (unsigned)p.heads_per_group);
+    };
+    auto sc_store = [&](unsigned j) {
+        const unsigned k = j * kScBatch + (tid & 31u);
+        if (k >= cnt) return;
+        ItemScalars sc;
+        sc.delta = p.softplus ? softplus_f(sc_v) : sc_v;
+        sc.dA = ex2_approx(sc.delta * sc_a);
+        sc.dskip = sc_d;
+        sc.g = sc_g;
+        item_sc[k & (2 * kScBatch - 1)] = sc;
+    };
+    if (sc_lane) {
+        sc_load(0);
+        sc_store(0);
+        sc_load(1);
+    }
     if (tid == 0) {
         for (unsigned s2 = 0; s2 < S; ++s2) mbar_init(&full[s2], 1);
         mbar_fence_init();
@@ -350,38 +399,44 @@ __global__ void __launch_bounds__(256, 3) ssu_head_tma_kernel(const SsuProblem p
     if (tid == 0) {
         Pos q = cur;
         for (unsigned k = 0; k < min(cnt, S); ++k) {
-            issue(k, q);
+            issue(k, k, q);
             next(q);
         }
     }
     Pos ahead = cur;  // position of item k + S (thread 0's refill cursor)
     for (unsigned k = 0; k < S; ++k) next(ahead);
+    // lpr and RPT are powers of two: the epilogue lanes by shift and mask
+    const unsigned group = lpr / RPT;
+    const unsigned gshift = __ffs(group) - 1;
 
     int64_t cached_key = -1;
     float Bv[CPL][VE], Cv[CPL][VE];
+    // B and C of (b, group g) into registers, when they change
+    auto load_bc = [&](unsigned b, unsigned g) {
+        const int64_t key = (int64_t)b * p.G + g;
+        if (key == cached_key) return;
+        cached_key = key;
+#pragma unroll
+        for (int j = 0; j < CPL; ++j) {
+#pragma unroll
+            for (int e = 0; e < VE; ++e) {
+                const int64_t n = (int64_t)(lane_r + lpr * j) * VE + e;
+                Bv[j][e] = to_f(Bg[b * p.B_b + g * p.B_g + n * p.B_n]);
+                Cv[j][e] = to_f(Cg[b * p.C_b + g * p.C_g + n * p.C_n]);
+            }
+        }
+    };
+    unsigned stage = 0;
+    uint32_t parity = 0;
     for (unsigned k = 0; k < cnt; ++k, next(cur)) {
         const unsigned b = cur.b, h = cur.h;
         const unsigned p0 = cur.pb * rb;
         const unsigned p1 = min(p0 + rb, P);
         const int64_t slot = slot_of(b);
-        const unsigned stage = k % S;
-        const uint32_t parity = (k / S) & 1u;
         float delta = 0.0f, dA = 0.0f, a2 = 0.0f, dskip = 0.0f;
-        if (slot >= 0) {
-            const unsigned g = h / (unsigned)p.heads_per_group;
-            const int64_t key = (int64_t)b * p.G + g;
-            if (key != cached_key) {
-                cached_key = key;
-#pragma unroll
-                for (int j = 0; j < CPL; ++j) {
-#pragma unroll
-                    for (int e = 0; e < VE; ++e) {
-                        const int64_t n = (int64_t)(lane_r + lpr * j) * VE + e;
-                        Bv[j][e] = to_f(Bg[b * p.B_b + g * p.B_g + n * p.B_n]);
-                        Cv[j][e] = to_f(Cg[b * p.C_b + g * p.C_g + n * p.C_n]);
-                    }
-                }
-            }
+        if (slot >= 0 && !ring) {
+            // per-thread scalars and B/C, loaded before the wait
+            load_bc(b, p.G == 1 ? 0u : h / (unsigned)p.heads_per_group);
             a2 = p.A[h * p.A_h] * kLog2e;
             dskip = p.Dp ? p.Dp[h * p.D_h] : 0.0f;
             if (!dt_row) {
@@ -407,6 +462,13 @@ __global__ void __launch_bounds__(256, 3) ssu_head_tma_kernel(const SsuProblem p
             return;
         }
         if (slot >= 0) {
+            if (ring) {
+                const ItemScalars sc = item_sc[k & (2 * kScBatch - 1)];
+                delta = sc.delta;
+                dA = sc.dA;
+                dskip = sc.dskip;
+                load_bc(b, (unsigned)sc.g);
+            }
             const unsigned char* st = tma_stage + stage * stage_bytes;
             const IoT* xsm = reinterpret_cast<const IoT*>(st + x_off);
             char* gbase = static_cast<char*>(p.state) +
@@ -450,9 +512,8 @@ __global__ void __launch_bounds__(256, 3) ssu_head_tma_kernel(const SsuProblem p
                 acc[r] = a0 + a1;
             }
             row_reduce_scatter<RPT>(acc, lane_r, lpr);
-            const unsigned group = lpr / RPT;
-            if (lane_r % group == 0) {
-                const unsigned r = lane_r / group;
+            if ((lane_r & (group - 1)) == 0) {
+                const unsigned r = lane_r >> gshift;
                 const unsigned pl = row_slot + r * rows_per_pass;
                 const unsigned pp = p0 + pl;
                 if (pp < p1) {
@@ -466,12 +527,23 @@ __global__ void __launch_bounds__(256, 3) ssu_head_tma_kernel(const SsuProblem p
                 }
             }
         }
+        // halfway through batch j: batch j + 1 into the ring (its entries were
+        // last read by batch j - 1, and 16 barriers publish it before its first
+        // item), then the loads of batch j + 2
+        if (sc_lane && (k & (kScBatch - 1)) == kScBatch / 2) {
+            sc_store(k / kScBatch + 1);
+            sc_load(k / kScBatch + 2);
+        }
         __syncthreads();  // every thread is done reading this stage
         if (tid == 0 && k + S < cnt) {
             fence_proxy_async_smem();
-            issue(k + S, ahead);
+            issue(k + S, stage, ahead);
         }
         next(ahead);
+        if (++stage == S) {
+            stage = 0;
+            parity ^= 1u;
+        }
     }
 }
 

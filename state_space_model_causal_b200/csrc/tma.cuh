@@ -30,11 +30,13 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                  : "memory");
 }
 
-__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+// One potentially blocking probe of the barrier's phase: the thread is
+// suspended until the phase completes or a hardware time limit passes.
+__device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
     uint32_t done;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(done)
         : "r"(smem_u32(bar)), "r"(parity)
@@ -42,14 +44,14 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
     return done != 0;
 }
 
-// Poll the barrier's phase with a back-off; give up after `budget` cycles.
+// Wait for the barrier's phase (woken by its completion, not by polling);
+// give up after `budget` cycles.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
                                                   long long budget) {
-    if (mbar_test(bar, parity)) return true;
+    if (mbar_try(bar, parity)) return true;
     const long long t0 = clock64();
     for (;;) {
-        __nanosleep(32);
-        if (mbar_test(bar, parity)) return true;
+        if (mbar_try(bar, parity)) return true;
         if (clock64() - t0 > budget) return false;
     }
 }
