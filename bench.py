@@ -221,11 +221,11 @@ def device_uuid(dev):
 class Prefill:
     """Device-resident inputs and the call of the 2.8B-shaped prefill."""
 
-    def __init__(self, dev, seed=0):
+    def __init__(self, dev, seed=0, Bt=4):
         import torch
         from state_space_model_causal_b200 import inputs as gen
         self.gen = gen
-        s = gen.prefill_2p8b(seed=seed)
+        s = gen.prefill_2p8b(seed=seed, Bt=Bt)
         self.s = s
         self.Bt, self.D, self.L = s.x.shape
         self.N = s.A.shape[1]
@@ -316,6 +316,30 @@ def prefill_mamba2(dev, hbm_peak, sm_max, steps=20, warmup=3):
                          "hbm_achieved_gbs": round(gbs, 1), "hbm_peak_gbs": hbm_peak,
                          "hbm_frac": round(gbs / hbm_peak, 4), "algorithmic_bytes_per_launch": alg},
             "l2": "flushed (256 MiB write) before every step", "gpu_launches": steps}
+
+
+def prefill_single_sequence(dev, sfu_peak, hbm_peak, steps=20, warmup=3):
+    """The 2.8B-shaped prefill at batch 1 (320 units of 16 channels, fewer
+    than the 1184 worker warps): the context-parallel mode, two launches per
+    call (pieces from zero states with carry records, then the re-scan from
+    the composed states).  CUDA events per call, L2 flushed before each."""
+    import torch
+    pf = Prefill(dev, Bt=1)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    ms = time_prefill(pf, steps, warmup, dev, flush)
+    mean = statistics.mean(ms)
+    gel = pf.elems / (mean * 1e-3) / 1e9
+    alg = pf.algorithmic_bytes()
+    del pf
+    torch.cuda.empty_cache()
+    return {"workload": "mamba1-2.8b-prefill, one sequence: B=1 L=2048 D=5120 N=16 W=4, fp16 I/O "
+                        "(context-parallel pieces, two launches per call)",
+            "us_per_call": round(mean * 1e3, 2), "Gelem_s": round(gel, 1),
+            "roofline": {"bound": "alu", "achieved": round(gel, 1), "peak": round(sfu_peak, 1),
+                         "unit": "Gelem/s", "frac": round(gel / sfu_peak, 4), "traffic": None,
+                         "peak_kind": "SFU ex2 rate x 148 SMs x max SM clock (one exp per element)",
+                         "hbm_achieved_gbs": round(alg / (mean * 1e-3) / 1e9, 1), "hbm_peak_gbs": hbm_peak},
+            "l2": "flushed (256 MiB write) before every step", "gpu_launches": 2 * steps}
 
 
 def time_prefill(pf, steps, warmup, dev, flush):
@@ -880,6 +904,7 @@ def main():
     e2e_val = world * pf.elems / (statistics.mean(e2e_ms) * 1e-3) / 1e9
 
     prefill_m2 = prefill_mamba2(dev, hbm_peak, sm_max) if not args.no_decode else None
+    prefill_b1 = prefill_single_sequence(dev, sfu_peak, hbm_peak) if not args.no_decode else None
 
     decode = []
     if not args.no_decode:
@@ -895,6 +920,9 @@ def main():
         # the oracle timed beside every other measured kernel, in its line's unit
         if prefill_m2:
             prefill_m2["oracle"] = oracle_beside(prefill_m2, "m2_prefill")
+        if prefill_b1:  # the same per-channel work as the headline's sample
+            prefill_b1["oracle"] = dict(cpu, sample="the headline's cpu_baseline (same recipe, per channel): "
+                                                    + cpu["sample"])
         for i, entry in enumerate(decode):
             entry["oracle"] = oracle_beside(entry, "m1_decode" if i == 0 else "m2_decode")
 
@@ -915,6 +943,7 @@ def main():
             "e2e": {"value": round(e2e_val, 3), "unit": "Gelem/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": args.steps, "clocks": clk.summary(), "prefill_mamba2": prefill_m2,
+            "prefill_one_sequence": prefill_b1,
             "decode": decode}
     print(json.dumps(line), flush=True)
     return 0

@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 namespace ssm {
 
 constexpr int kMaxDevices = 64;  // per-device host caches hold this many devices
@@ -209,5 +211,36 @@ int scan_m2_threads();
 int scan_m2_smem_bytes(int io_dt, int64_t N);
 cudaError_t launch_scan_m2(const ScanM2Problem& p, int kernel, const M2Plan& mp, cudaStream_t s);
 int scan_m2_ctas_per_sm(const ScanM2Problem& p, int dev);
+
+// Launch preparation done once per (kernel, device, dynamic shared memory,
+// block): the attributes a launch needs are set by `prepare` (which returns
+// the CTAs per SM, or a negative number on failure) the first time, and the
+// result is remembered.  Thread-safe; the table holds far more entries than
+// the library has kernel instances.
+template <typename F>
+cudaError_t prepared_launch(const void* fn, int smem, int block, int* per_sm, F prepare) {
+    struct Entry { const void* fn; int dev, smem, block, per_sm; };
+    static std::mutex mu;
+    static Entry tab[1024];
+    static int n = 0;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    {
+        std::lock_guard<std::mutex> g(mu);
+        for (int i = 0; i < n; ++i)
+            if (tab[i].fn == fn && tab[i].dev == dev && tab[i].smem == smem && tab[i].block == block) {
+                *per_sm = tab[i].per_sm;
+                return cudaSuccess;
+            }
+    }
+    int v = 0;
+    e = prepare(&v);
+    if (e != cudaSuccess) return e;
+    *per_sm = v;
+    std::lock_guard<std::mutex> g(mu);
+    if (n < 1024) tab[n++] = Entry{fn, dev, smem, block, v};
+    return cudaSuccess;
+}
 
 }  // namespace ssm

@@ -421,8 +421,12 @@ cudaError_t launch_w(const ScanProblem& p, int sw, cudaStream_t s) {
     dim3 grid((unsigned)((p.D + kDT - 1) / kDT), (unsigned)p.Bn);
     auto run = [&](auto kern) -> cudaError_t {
         // many small CTAs per SM: ask for the largest shared-memory carveout
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                             cudaSharedmemCarveoutMaxShared);
+        // (once per kernel and device)
+        int unused = 0;
+        cudaError_t e = prepared_launch(reinterpret_cast<const void*>(kern), 0, kThreads, &unused, [&](int*) {
+            return cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                        cudaSharedmemCarveoutMaxShared);
+        });
         if (e != cudaSuccess) return e;
         kern<<<grid, kThreads, 0, s>>>(p);
         return cudaGetLastError();
