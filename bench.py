@@ -299,9 +299,13 @@ def prefill_mamba2(dev, hbm_peak, sm_max, steps=20, warmup=3):
     ms = time_prefill(pm, steps, warmup, dev, flush)
     mean = statistics.mean(ms)
     gel = pm.elems / (mean * 1e-3) / 1e9
-    # FP32 pipe: 128 lanes per SM; per state element and step the method needs
-    # delta*x*B (1 mul), the decay FMA and the readout FMA: 3 FP32 operations
-    fp32_peak = NUM_SMS * 128 * sm_max * 1e6 / 3 / 1e9  # Gelem/s
+    # FP32 pipe: 128 lanes per SM.  Per state element and step the recurrence
+    # needs at least two FP32 operations (the state update and the readout,
+    # as the kernel's rescaled form does them); written directly it needs
+    # three (delta*x*B, the decay FMA, the readout FMA).  The peak is the
+    # two-operation floor; the three-operation figure is reported beside it.
+    fp32_peak = NUM_SMS * 128 * sm_max * 1e6 / 2 / 1e9  # Gelem/s
+    fp32_peak_direct = fp32_peak * 2 / 3
     alg = pm.algorithmic_bytes()
     gbs = alg / (mean * 1e-3) / 1e9
     traffic = profiled_traffic("scan_m2_prefill_2p7b.txt", ["scan_m2.cu", "common.cuh"])
@@ -312,7 +316,8 @@ def prefill_mamba2(dev, hbm_peak, sm_max, steps=20, warmup=3):
             "us_per_call": round(mean * 1e3, 2), "Gelem_s": round(gel, 1),
             "roofline": {"bound": "alu", "achieved": round(gel, 1), "peak": round(fp32_peak, 1),
                          "unit": "Gelem/s", "frac": round(gel / fp32_peak, 4), "traffic": traffic,
-                         "peak_kind": "FP32 pipe 128 lanes/SM x 148 SMs x max SM clock / 3 ops per element",
+                         "peak_kind": "FP32 pipe 128 lanes/SM x 148 SMs x max SM clock / 2 ops per element",
+                         "frac_of_direct_form_bound": round(gel / fp32_peak_direct, 4),
                          "hbm_achieved_gbs": round(gbs, 1), "hbm_peak_gbs": hbm_peak,
                          "hbm_frac": round(gbs / hbm_peak, 4), "algorithmic_bytes_per_launch": alg},
             "l2": "flushed (256 MiB write) before every step", "gpu_launches": steps}

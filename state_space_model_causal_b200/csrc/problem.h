@@ -212,34 +212,47 @@ int scan_m2_smem_bytes(int io_dt, int64_t N);
 cudaError_t launch_scan_m2(const ScanM2Problem& p, int kernel, const M2Plan& mp, cudaStream_t s);
 int scan_m2_ctas_per_sm(const ScanM2Problem& p, int dev);
 
-// Launch preparation done once per (kernel, device, dynamic shared memory,
-// block): the attributes a launch needs are set by `prepare` (which returns
-// the CTAs per SM, or a negative number on failure) the first time, and the
-// result is remembered.  Thread-safe; the table holds far more entries than
-// the library has kernel instances.
-template <typename F>
-cudaError_t prepared_launch(const void* fn, int smem, int block, int* per_sm, F prepare) {
-    struct Entry { const void* fn; int dev, smem, block, per_sm; };
+// Launch preparation, done once and remembered (thread-safe):
+//   * per (kernel, device), `attrs(smem)` opts the kernel into `smem` bytes of
+//     dynamic shared memory (and any other attribute it needs).  The limit
+//     only ever grows -- it is raised when a launch needs more than any
+//     before -- so that a launch never meets a limit set for a smaller one;
+//   * per (kernel, device, shared memory, block), `occupancy(&n)` gives the
+//     CTAs per SM.
+// The tables hold far more entries than the library has kernel instances.
+template <typename Attrs, typename Occupancy>
+cudaError_t prepared_launch(const void* fn, int smem, int block, int* per_sm, Attrs attrs,
+                            Occupancy occupancy) {
+    struct Limit { const void* fn; int dev, smem; };
+    struct Fit { const void* fn; int dev, smem, block, per_sm; };
     static std::mutex mu;
-    static Entry tab[1024];
-    static int n = 0;
+    static Limit limits[1024];
+    static Fit fits[1024];
+    static int n_limits = 0, n_fits = 0;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    {
-        std::lock_guard<std::mutex> g(mu);
-        for (int i = 0; i < n; ++i)
-            if (tab[i].fn == fn && tab[i].dev == dev && tab[i].smem == smem && tab[i].block == block) {
-                *per_sm = tab[i].per_sm;
-                return cudaSuccess;
-            }
+    std::lock_guard<std::mutex> g(mu);
+    int li = -1;
+    for (int i = 0; i < n_limits; ++i)
+        if (limits[i].fn == fn && limits[i].dev == dev) li = i;
+    if (li < 0 || limits[li].smem < smem) {
+        e = attrs(smem);
+        if (e != cudaSuccess) return e;
+        if (li >= 0) limits[li].smem = smem;
+        else if (n_limits < 1024) limits[n_limits++] = Limit{fn, dev, smem};
+        else return cudaErrorUnknown;  // never: more kernels than the table
     }
+    for (int i = 0; i < n_fits; ++i)
+        if (fits[i].fn == fn && fits[i].dev == dev && fits[i].smem == smem && fits[i].block == block) {
+            *per_sm = fits[i].per_sm;
+            return cudaSuccess;
+        }
     int v = 0;
-    e = prepare(&v);
+    e = occupancy(&v);
     if (e != cudaSuccess) return e;
     *per_sm = v;
-    std::lock_guard<std::mutex> g(mu);
-    if (n < 1024) tab[n++] = Entry{fn, dev, smem, block, v};
+    if (n_fits < 1024) fits[n_fits++] = Fit{fn, dev, smem, block, v};
     return cudaSuccess;
 }
 

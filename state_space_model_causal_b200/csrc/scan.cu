@@ -280,9 +280,13 @@ cudaError_t launch_chunked_t(const ScanProblem& p, const ScanPlan& plan, cudaStr
     auto kern = scan_chunked_kernel<IoT, NS, DT, T>;
     if (S::BYTES > 48 * 1024) {
         int unused = 0;
-        cudaError_t e = prepared_launch(reinterpret_cast<const void*>(kern), S::BYTES, DT * NS, &unused, [&](int*) {
-            return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::BYTES);
-        });
+        cudaError_t e = prepared_launch(
+            reinterpret_cast<const void*>(kern), S::BYTES, DT * NS, &unused,
+            [&](int limit) { return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, limit); },
+            [](int* n) {
+                *n = 0;
+                return cudaSuccess;
+            });
         if (e != cudaSuccess) return e;
     }
     dim3 grid((unsigned)((p.D + DT - 1) / DT), (unsigned)p.Bn);

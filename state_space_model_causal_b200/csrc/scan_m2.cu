@@ -10,8 +10,13 @@
 //   out     = (sum_n C[b,g,n,t] * s[p,n] + D[h] * x[b,h,p,t]) * silu(z[b,h,p,t])
 //
 // with g = h / (H / G).  The decay is one exponential per (b, h, t), so the
-// work is two FMAs per state element and step: the kernel is FMA-bound, not
-// SFU-bound like the Mamba-1 prefill.
+// work is FP32 arithmetic per state element and step: the kernel is bound by
+// the FMA pipe, not by the SFU like the Mamba-1 prefill.  Because the decay
+// is one scalar per (b, h, t), a chunk can run in a rescaled form: with P_t
+// the product of the chunk's decays up to step t, g = s / P_t obeys
+// g += (delta x / P_t) B, one FMA per element instead of a multiply and an
+// FMA, and the readout is P_t (C . g).  Chunks whose decay product would
+// leave the safe fp32 range run the direct recurrence.
 //
 // Fast kernel (time-major rows: headdim contiguous in x, z, out, and a
 // multiple of 8; dstate 64, 128 or 256, contiguous in B, C; 16-byte aligned
@@ -26,9 +31,11 @@
 //     the previous chunk is scanned (x, z double-buffered for the epilogue;
 //     B, C single-buffered, refilled once widened); dt is prefetched into a
 //     register one chunk ahead;
-//   * per chunk the CTA computes once (delta, decay) per step, delta * x per
-//     (step, row) and the fp32 B, C rows (16-byte pieces XOR-swizzled so the NG
-//     groups of a quarter-warp read distinct banks);
+//   * per chunk the CTA computes once per step delta and the decay (the
+//     chunk's decay prefix products P_t by a warp prefix scan of delta * A, in
+//     log2), delta * x per (step, row) -- divided by P_t in the rescaled form --
+//     and the fp32 B, C rows (16-byte pieces XOR-swizzled so the NG groups of a
+//     quarter-warp read distinct banks);
 //   * the readout partials of 4 steps x 4 rows are summed over the NG threads
 //     of a row block by a butterfly reduce-scatter; the epilogue applies the D
 //     skip and the gate to 8 consecutive rows per thread and stores 16 bytes.
@@ -38,6 +45,7 @@
 #include "problem.h"
 
 #include <atomic>
+#include <type_traits>
 
 namespace ssm {
 namespace {
@@ -54,6 +62,10 @@ namespace {
 constexpr int kM2Threads = SSM_M2_THREADS;  // threads per CTA
 constexpr int kM2T = SSM_M2_STEPS;          // steps per chunk
 constexpr int kM2MinCtas = SSM_M2_MIN_CTAS; // register budget: CTAs resident per SM
+// A chunk runs in the rescaled form while every partial decay product P of
+// the chunk lies within 2^+-64 (so that P and 1 / P stay far inside the fp32
+// range); otherwise directly.
+constexpr float kRescaleLog2 = 64.0f;
 
 // (16-byte piece u of a B/C row) -> stored piece: the pieces a quarter-warp's
 // NG groups read at once (u = 4 ng + k) land in distinct banks
@@ -69,7 +81,7 @@ template <typename IoT, int NG> struct M2Smem {
     RawXZ raw[2];      // x, z: read again by the epilogue, so double-buffered
     IoT rawB[kM2T][N];  // B, C: widened right after arrival, single buffer
     IoT rawC[kM2T][N];
-    float2 dd[kM2T];           // (decay, delta) per step
+    float2 dd[kM2T];           // per step: (decay, delta), or rescaled (P_t, delta / P_t)
     float dx[kM2T][RPC];       // delta * x
     float B[kM2T][N];          // swizzled fp32 rows
     float C[kM2T][N];
@@ -138,6 +150,7 @@ __global__ void __launch_bounds__(kM2Threads, kM2MinCtas) scan_m2_kernel(const S
     S& sm = *reinterpret_cast<S*>(m2_smem);
     __shared__ unsigned s_gen;
     __shared__ int s_got;
+    __shared__ int s_rescale;
 
     const int tid = threadIdx.x;
     const int ng = tid % NG;
@@ -320,17 +333,39 @@ __global__ void __launch_bounds__(kM2Threads, kM2MinCtas) scan_m2_kernel(const S
         const int64_t t0 = k * kM2T;
         const int steps = (int)(L - t0 < kM2T ? L - t0 : kM2T);
         asm volatile("cp.async.wait_group 0;" ::: "memory");
-        // ---- per step: delta and the decay (steps past L keep the state)
-        if (tid < kM2T) {
-            float delta = 0.0f, decay = 1.0f;
+        // ---- per step (first warp, one step per lane): delta and the decay,
+        // steps past L keep the state.  The chunk's log2 decays are summed by
+        // a prefix scan: P_t = 2^cum_t is the decay from the chunk start to
+        // the end of step t.
+        if (tid < 32) {
+            float delta = 0.0f, l2 = 0.0f;
             if (tid < steps) {
                 const float v = dt_next + dbias;
                 delta = p.softplus ? softplus_f(v) : v;
-                decay = ex2_approx(delta * A2);
+                l2 = delta * A2;
             }
-            sm.dd[tid] = make_float2(decay, delta);
+            float cum = l2;
+#pragma unroll
+            for (int o = 1; o < kM2T; o <<= 1) {
+                const float up = __shfl_up_sync(0xffffffffu, cum, o);
+                if (tid >= o) cum += up;
+            }
+            // rescaled only while every P_t and 1 / P_t stays within 2^+-64
+            // (delta * A can be positive without the softplus)
+            float lo = tid < kM2T ? cum : 0.0f, hi = lo;
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) {
+                lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+                hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+            }
+            const bool rs = lo >= -kRescaleLog2 && hi <= kRescaleLog2;
+            if (tid < kM2T)
+                sm.dd[tid] = rs ? make_float2(ex2_approx(cum), delta * ex2_approx(-cum))
+                                : make_float2(ex2_approx(l2), delta);
+            if (tid == 0) s_rescale = rs;
         }
         __syncthreads();  // dd and this chunk's staged rows visible to all
+        const bool rescale = s_rescale != 0;
         if (more) {
             fetch_xz(nuu, nk, bi ^ 1);
             dt_next = load_dt(nuu, nk);
@@ -367,60 +402,83 @@ __global__ void __launch_bounds__(kM2Threads, kM2MinCtas) scan_m2_kernel(const S
         if (more) fetch_bc(nuu, nk);
         commit();
 
-        // ---- scan: 4 groups of 4 steps
+        // ---- scan: 4 groups of 4 steps.  Direct form: s = decay * s + dx * B.
+        // Rescaled form: the tile holds g = s / P_t, updated by g += (dx / P_t) * B
+        // (dd carries delta / P_t, so dx does too); the readout C . g is scaled by
+        // P_t, and at the chunk's end the tile is scaled back, s = P_end * g.
+        // Both give s_t = sum_{u<=t} (P_t / P_u) dx_u B_u + P_t s_start; the
+        // rescaled one in two FP32 operations per element and step instead of
+        // three.
+        auto scan_chunk = [&](auto rescaled) {
+            constexpr bool RS = decltype(rescaled)::value;
 #pragma unroll 1
-        for (int tt = 0; tt < kM2T; tt += 4) {
-            float v[16];  // v[4r + kk]: partial readout of row r at step tt + kk
+            for (int tt = 0; tt < kM2T; tt += 4) {
+                float v[16];  // v[4r + kk]: partial readout of row r at step tt + kk
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const int t = tt + kk;
-                const float decay = sm.dd[t].x;
-                const u64 dA2 = pk(decay, decay);
-                const float4 dx4 = *reinterpret_cast<const float4*>(&sm.dx[t][4 * pg]);
-                const u64 dx2[4] = {pk(dx4.x, dx4.x), pk(dx4.y, dx4.y), pk(dx4.z, dx4.z), pk(dx4.w, dx4.w)};
-                u64 y2[4];
-                // one 16-byte piece of B and C at a time (short live ranges)
+                for (int kk = 0; kk < 4; ++kk) {
+                    const int t = tt + kk;
+                    const float decay = sm.dd[t].x;
+                    const u64 dA2 = pk(decay, decay);
+                    const float4 dx4 = *reinterpret_cast<const float4*>(&sm.dx[t][4 * pg]);
+                    const u64 dx2[4] = {pk(dx4.x, dx4.x), pk(dx4.y, dx4.y), pk(dx4.z, dx4.z), pk(dx4.w, dx4.w)};
+                    u64 y2[4];
+                    // one 16-byte piece of B and C at a time (short live ranges)
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float4 bq = *reinterpret_cast<const float4*>(&sm.B[t][boff[q]]);
-                    const float4 cq = *reinterpret_cast<const float4*>(&sm.C[t][boff[q]]);
-                    const u64 b2[2] = {pk(bq.x, bq.y), pk(bq.z, bq.w)};
-                    const u64 c2[2] = {pk(cq.x, cq.y), pk(cq.z, cq.w)};
+                    for (int q = 0; q < 4; ++q) {
+                        const float4 bq = *reinterpret_cast<const float4*>(&sm.B[t][boff[q]]);
+                        const float4 cq = *reinterpret_cast<const float4*>(&sm.C[t][boff[q]]);
+                        const u64 b2[2] = {pk(bq.x, bq.y), pk(bq.z, bq.w)};
+                        const u64 c2[2] = {pk(cq.x, cq.y), pk(cq.z, cq.w)};
+#pragma unroll
+                        for (int r = 0; r < 4; ++r) {
+#pragma unroll
+                            for (int jj = 0; jj < 2; ++jj) {
+                                const int j = 2 * q + jj;
+                                if constexpr (RS)
+                                    hs[r][j] = ffma2(dx2[r], b2[jj], hs[r][j]);
+                                else
+                                    hs[r][j] = ffma2(dA2, hs[r][j], fmul2(dx2[r], b2[jj]));
+                                y2[r] = j == 0 ? fmul2(c2[jj], hs[r][j]) : ffma2(c2[jj], hs[r][j], y2[r]);
+                            }
+                        }
+                    }
 #pragma unroll
                     for (int r = 0; r < 4; ++r) {
+                        float lo, hi;
+                        upk(y2[r], lo, hi);
+                        v[4 * r + kk] = RS ? (lo + hi) * decay : lo + hi;  // decay holds P_t
+                    }
+                }
+                // butterfly reduce-scatter over the NG threads of the row group:
+                // thread ng ends with v[i], i = ng * (16 / NG) + local
 #pragma unroll
-                        for (int jj = 0; jj < 2; ++jj) {
-                            const int j = 2 * q + jj;
-                            hs[r][j] = ffma2(dA2, hs[r][j], fmul2(dx2[r], b2[jj]));
-                            y2[r] = j == 0 ? fmul2(c2[jj], hs[r][j]) : ffma2(c2[jj], hs[r][j], y2[r]);
-                        }
+                for (int m = NG / 2, S2 = 8; m >= 1; m >>= 1, S2 >>= 1) {
+                    const bool up = (ng & m) != 0;
+#pragma unroll
+                    for (int i = 0; i < S2; ++i) {
+                        const float send = up ? v[i] : v[i + S2];
+                        const float keep = up ? v[i + S2] : v[i];
+                        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
                     }
                 }
 #pragma unroll
-                for (int r = 0; r < 4; ++r) {
-                    float lo, hi;
-                    upk(y2[r], lo, hi);
-                    v[4 * r + kk] = lo + hi;
+                for (int l = 0; l < 16 / NG; ++l) {
+                    const int i = ng * (16 / NG) + l;
+                    sm.y[tt + (i & 3)][4 * pg + (i >> 2)] = v[l];
                 }
             }
-            // butterfly reduce-scatter over the NG threads of the row group:
-            // thread ng ends with v[i], i = ng * (16 / NG) + local
+            if constexpr (RS) {
+                const u64 pe = pk(sm.dd[kM2T - 1].x, sm.dd[kM2T - 1].x);  // P at the chunk's end
 #pragma unroll
-            for (int m = NG / 2, S2 = 8; m >= 1; m >>= 1, S2 >>= 1) {
-                const bool up = (ng & m) != 0;
+                for (int r = 0; r < 4; ++r)
 #pragma unroll
-                for (int i = 0; i < S2; ++i) {
-                    const float send = up ? v[i] : v[i + S2];
-                    const float keep = up ? v[i + S2] : v[i];
-                    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
-                }
+                    for (int j = 0; j < 8; ++j) hs[r][j] = fmul2(pe, hs[r][j]);
             }
-#pragma unroll
-            for (int l = 0; l < 16 / NG; ++l) {
-                const int i = ng * (16 / NG) + l;
-                sm.y[tt + (i & 3)][4 * pg + (i >> 2)] = v[l];
-            }
-        }
+        };
+        if (rescale)
+            scan_chunk(std::true_type{});
+        else
+            scan_chunk(std::false_type{});
         __syncthreads();
 
         // ---- epilogue: D skip and gate on 8 consecutive rows, 16-byte stores

@@ -423,10 +423,16 @@ cudaError_t launch_w(const ScanProblem& p, int sw, cudaStream_t s) {
         // many small CTAs per SM: ask for the largest shared-memory carveout
         // (once per kernel and device)
         int unused = 0;
-        cudaError_t e = prepared_launch(reinterpret_cast<const void*>(kern), 0, kThreads, &unused, [&](int*) {
-            return cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                        cudaSharedmemCarveoutMaxShared);
-        });
+        cudaError_t e = prepared_launch(
+            reinterpret_cast<const void*>(kern), 0, kThreads, &unused,
+            [&](int) {
+                return cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                            cudaSharedmemCarveoutMaxShared);
+            },
+            [](int* n) {
+                *n = 0;
+                return cudaSuccess;
+            });
         if (e != cudaSuccess) return e;
         kern<<<grid, kThreads, 0, s>>>(p);
         return cudaGetLastError();

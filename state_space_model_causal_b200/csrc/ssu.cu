@@ -966,17 +966,18 @@ cudaError_t launch_head(const SsuProblem& p, const SsuPlan& plan, cudaStream_t s
 
 // Opt the kernel into its dynamic shared memory and the largest shared-memory
 // carveout, and return how many of its CTAs fit on one SM.
-// Done once per kernel, device and shared-memory size (prepared_launch).
+// Done once per kernel, device and size (prepared_launch).
 template <typename K>
 cudaError_t prepare_tma_kernel(K kern, int block, int smem, int* per_sm) {
-    return prepared_launch(reinterpret_cast<const void*>(kern), smem, block, per_sm, [&](int* n) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                 cudaSharedmemCarveoutMaxShared);
-        if (e != cudaSuccess) return e;
-        return cudaOccupancyMaxActiveBlocksPerMultiprocessor(n, kern, block, smem);
-    });
+    return prepared_launch(
+        reinterpret_cast<const void*>(kern), smem, block, per_sm,
+        [&](int limit) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, limit);
+            if (e != cudaSuccess) return e;
+            return cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                        cudaSharedmemCarveoutMaxShared);
+        },
+        [&](int* n) { return cudaOccupancyMaxActiveBlocksPerMultiprocessor(n, kern, block, smem); });
 }
 
 template <typename ST, typename IoT>

@@ -222,3 +222,33 @@ def test_m2_prefill_balanced_slices_match_oracle_and_whole_units(io, N_, P, L):
     a, b = run("auto"), run(None)
     np.testing.assert_array_equal(a[0], b[0])
     np.testing.assert_array_equal(a[1], b[1])
+
+
+@pytest.mark.parametrize("io", ["f32", "f16"])
+def test_m2_prefill_rescaled_and_direct_chunks(io):
+    """The kernel runs a 16-step chunk in the rescaled form (state divided by
+    the running decay product) while every partial decay product of the chunk
+    stays within 2^+-64, else in the direct form.  dt is raised on alternate 24-step spans,
+    so that chunks are mild, strong or mixed: with dt_bias = 0 a strong step
+    has delta = softplus(0.5) = 0.97, a decay of 2^-22.5 per step at A = -16
+    (direct form) and 2^-1.4 at A = -1 (rescaled form even when strong).
+    Both forms must match the oracle, state included."""
+    s = gen.scan_m2_inputs(2, 3, 64, 128, 100, io=io, seed=9, tag=f"m2rs{io}", h0=True)
+    s.A = np.array([-16.0, -4.0, -1.0])
+    s.dt_bias = np.zeros(3)
+    strong = (np.arange(100) // 24) % 2 == 1
+    dt = np.array(s.dt, dtype=np.float64)
+    dt[:, :, strong] = 0.5
+    s.dt = gen.round_to(dt, io)
+    _check(s, kernel="scan_m2")
+
+
+def test_m2_prefill_rescaled_form_long_mild_decay():
+    """Weak decay over a long sequence (delta * A ~ -0.02 per step): every
+    chunk runs in the rescaled form and the state builds up over hundreds of
+    steps; fp32 I/O at the fp32 bound."""
+    s = gen.scan_m2_inputs(1, 2, 64, 64, 640, io="f32", seed=10, tag="m2mild", h0=True)
+    s.A = np.array([-1.0, -2.0])
+    s.dt = gen.round_to(np.full(s.dt.shape, -3.9), "f32")
+    s.dt_bias = np.array([-0.05, -0.05])
+    _check(s, kernel="scan_m2")

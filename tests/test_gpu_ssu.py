@@ -128,6 +128,21 @@ def test_mamba2_64x128_effective_batch(cache, R):
     assert_close(N(st), sref, TOL["f16"], "state")
 
 
+def test_mamba2_launch_sizes_in_any_order():
+    """The library opts each kernel into its shared memory once and remembers
+    it; launches of one kernel with stages of different sizes, largest first,
+    then smaller, then between, then the largest again, must all run and
+    match the oracle (a remembered size must never meet a lower limit)."""
+    import torch
+    for R in (1024, 8, 80, 1024, 16):
+        s = gen.mamba2_64x128(R, cache="f16")
+        out, st = _m2_gpu(s)
+        torch.cuda.synchronize()
+        o, sref = _m2_oracle(s)
+        assert_close(N(out), o, TOL["f16"], f"out R={R}")
+        assert_close(N(st), sref, TOL["f16"], f"state R={R}")
+
+
 @pytest.mark.parametrize("cache", ["bf16", "f32"])
 @pytest.mark.parametrize("R", [8, 32, 512, 2048])
 def test_mamba2_128x256_effective_batch(cache, R):
