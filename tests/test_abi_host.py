@@ -233,6 +233,23 @@ def test_prefill_context_parallel_plan(lib):
     assert info.work_items == 1280 and info.grid == 296
 
 
+def test_prefill_context_parallel_plan_short_batch(lib):
+    """B=1, D=64, L=512 (4 units of 16 channels, 16 chunks): as many pieces as
+    leave at least two chunks each with the last piece shorter -- 8 pieces of
+    2 chunks, 7 per pass -- so 28 piece-units per pass, no hand-overs between
+    warps (28 < 1184), and one record per unit and piece 0..6."""
+    mem = FakeMem()
+    a = scan_args(mem, Bn=1, D=64, L=512)
+    need = ctypes.c_uint64(123)
+    assert lib.ssm_selective_scan_workspace_size(ctypes.byref(a), ctypes.byref(need)) == OK
+    assert need.value == ws_bytes(1184) + 4 * 7 * 1088
+    a.workspace, a.workspace_bytes = mem.next, need.value
+    mem.next += 1 << 36
+    st, info = call(lib, "ssm_selective_scan_fwd", a)
+    assert st == OK and bd.KERNELS[info.kernel] == "scan_bal"
+    assert info.work_items == 28
+
+
 def test_prefill_small_problem_needs_no_workspace(lib):
     mem = FakeMem()
     need = ctypes.c_uint64(123)
