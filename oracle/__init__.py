@@ -21,6 +21,11 @@ Functions (see the header comment of ``oracle.c`` for the definitions):
   SSU configs for Intel Arc Pro B70", section 关键源码片段.
 * :func:`ssu_mamba2` -- the same update in the Mamba-2 notation (scalar A,
   dt, D and dt_bias per head, ngroups), written separately in C.
+* :func:`delta_sum` and :func:`carry_fold` -- a prefill cut into sequence
+  pieces: the sum of a piece's steps delta, and the state entering the next
+  piece, exp(A * sum delta) * h_in + h_end (the pieces of a context-parallel
+  prefill; the long-context claim of "feat(llama.cu): 适配 mamba 模型" section
+  6.1).
 * :func:`round_cache` -- a state rounded to its cache dtype (fp32, fp16, bf16;
   nearest, ties to even); :func:`ssu` and :func:`ssu_mamba2` apply it to the
   updated state when given ``cache_dtype``, after the step's readout has used
@@ -75,6 +80,10 @@ def configure(lib):
     lib.oracle_ssu_mamba2.argtypes = [_i64] * 5 + [_dp] * 8 + [_dp] + [ctypes.c_int] + [_dp]
     lib.oracle_scan_mamba2.restype = ctypes.c_int
     lib.oracle_scan_mamba2.argtypes = [_i64] * 6 + [_dp] * 8 + [ctypes.c_int] + [_dp] * 3
+    lib.oracle_delta_sum.restype = ctypes.c_int
+    lib.oracle_delta_sum.argtypes = [_i64] * 3 + [_dp] * 2 + [ctypes.c_int] + [_dp]
+    lib.oracle_carry_fold.restype = ctypes.c_int
+    lib.oracle_carry_fold.argtypes = [_i64] * 3 + [_dp] * 4
     return lib
 
 
@@ -293,3 +302,32 @@ def scan_mamba2(x, dt, A, B, C, D=None, z=None, dt_bias=None, dt_softplus=True, 
     if rc != 0:
         raise ValueError("oracle_scan_mamba2 rejected its arguments")
     return out, hf
+
+
+def delta_sum(dt, dt_bias=None, dt_softplus=True):
+    """S (Bt, Dd): the sum over t of delta = softplus(dt + dt_bias) (dt + dt_bias
+    without the softplus); dt (Bt, Dd, L), dt_bias (Dd)."""
+    lib = _load()
+    dt_, pdt = _in(dt)
+    Bt, Dd, L = dt_.shape
+    _, pdb = _in(dt_bias, (Dd,)) if dt_bias is not None else (None, None)
+    out, po = _out((Bt, Dd))
+    if lib.oracle_delta_sum(Bt, Dd, L, pdt, pdb, int(bool(dt_softplus)), po) != 0:
+        raise ValueError("oracle_delta_sum rejected its arguments")
+    return out
+
+
+def carry_fold(state, A, S, h_end):
+    """exp(A * S) * state + h_end: the state entering the next sequence piece,
+    from the state entering this one (state), the piece's sum of delta (S) and
+    its end state from a zero start (h_end).  state, h_end (Bt, Dd, N); A (Dd, N);
+    S (Bt, Dd).  Returns a new array."""
+    lib = _load()
+    st = np.array(state, dtype=np.float64, copy=True, order="C")
+    Bt, Dd, N = st.shape
+    _, pA = _in(A, (Dd, N))
+    _, pS = _in(S, (Bt, Dd))
+    _, ph = _in(h_end, (Bt, Dd, N))
+    if lib.oracle_carry_fold(Bt, Dd, N, pA, pS, ph, st.ctypes.data_as(_dp)) != 0:
+        raise ValueError("oracle_carry_fold rejected its arguments")
+    return st

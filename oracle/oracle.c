@@ -344,3 +344,50 @@ int oracle_round_cache(double* v, int64_t n, int dtype) {
     }
     return 0;
 }
+
+/* ---------------------------------------------------------------------------
+ * Sequence pieces.  A prefill over a sequence cut into consecutive pieces
+ * equals the prefills of the pieces, each started from the state that the
+ * earlier pieces leave (the scan is a first-order linear recurrence in h).
+ * Started from a zero state, piece j ends in h_end(j); the state entering
+ * piece j+1 is
+ *     h_in(j+1)[b,d,n] = exp(A[d,n] * S(j)[b,d]) * h_in(j)[b,d,n] + h_end(j)[b,d,n]
+ * where S(j)[b,d] is the sum over the piece's steps of delta (softplus(dt +
+ * dt_bias), or dt + dt_bias without the softplus): the product of the piece's
+ * per-step decays exp(delta*A) is exp(A * sum delta).  Pages: the long-context
+ * claim of "feat(llama.cu): 适配 mamba 模型" section 6.1 (the scan is linear in
+ * the sequence length); the decomposition itself is the recurrence's algebra.
+ *
+ *   oracle_delta_sum   S[b,d] = sum_t delta(dt[b,d,t] + dt_bias[d])   dt (B, D, L)
+ *   oracle_carry_fold  state[b,d,n] <- exp(A[d,n] * S[b,d]) * state[b,d,n] + h_end[b,d,n]
+ *                      A (D, N); S (B, D); h_end, state (B, D, N)
+ * ------------------------------------------------------------------------- */
+int oracle_delta_sum(int64_t B, int64_t D, int64_t L, const double* dt, const double* dt_bias,
+                     int dt_softplus, double* out) {
+    int64_t b, d, t;
+    if (B < 0 || D < 0 || L < 0 || !dt || !out) return -1;
+    for (b = 0; b < B; ++b) {
+        for (d = 0; d < D; ++d) {
+            double sum = 0.0;
+            for (t = 0; t < L; ++t) {
+                const double v = dt[(b * D + d) * L + t] + (dt_bias ? dt_bias[d] : 0.0);
+                sum += dt_softplus ? o_softplus(v) : v;
+            }
+            out[b * D + d] = sum;
+        }
+    }
+    return 0;
+}
+
+int oracle_carry_fold(int64_t B, int64_t D, int64_t N, const double* A, const double* S,
+                      const double* h_end, double* state) {
+    int64_t b, d, n;
+    if (B < 0 || D < 0 || N < 0 || !A || !S || !h_end || !state) return -1;
+    for (b = 0; b < B; ++b)
+        for (d = 0; d < D; ++d)
+            for (n = 0; n < N; ++n) {
+                const int64_t i = (b * D + d) * N + n;
+                state[i] = exp(A[d * N + n] * S[b * D + d]) * state[i] + h_end[i];
+            }
+    return 0;
+}

@@ -72,6 +72,15 @@ MUTATIONS = [
     ("round_bf16_one_bit_long", "v[i] = o_round_bits(v[i], 8, -126,", "v[i] = o_round_bits(v[i], 9, -126,"),
     ("round_f16_subnormal_quantum", "v[i] = o_round_bits(v[i], 11, -14, 65504.0, 16.0);",
      "v[i] = o_round_bits(v[i], 11, -15, 65504.0, 16.0);"),
+    ("delta_sum_bias_dropped", "const double v = dt[(b * D + d) * L + t] + (dt_bias ? dt_bias[d] : 0.0);",
+     "const double v = dt[(b * D + d) * L + t];"),
+    ("delta_sum_softplus_skipped", "sum += dt_softplus ? o_softplus(v) : v;", "sum += v;"),
+    ("carry_fold_decay_sign", "state[i] = exp(A[d * N + n] * S[b * D + d]) * state[i] + h_end[i];",
+     "state[i] = exp(-A[d * N + n] * S[b * D + d]) * state[i] + h_end[i];"),
+    ("carry_fold_end_state_dropped", "state[i] = exp(A[d * N + n] * S[b * D + d]) * state[i] + h_end[i];",
+     "state[i] = exp(A[d * N + n] * S[b * D + d]) * state[i];"),
+    ("carry_fold_A_transposed", "state[i] = exp(A[d * N + n] * S[b * D + d]) * state[i] + h_end[i];",
+     "state[i] = exp(A[n * D + d] * S[b * D + d]) * state[i] + h_end[i];"),
 ]
 
 # pins exercised against each mutant (all cheap)
@@ -94,6 +103,8 @@ PIN_CALLS = [
     lambda: pins.test_mamba2_prefill_two_steps_by_hand(),
     lambda: pins.test_round_cache_matches_library_conversions(),
     lambda: pins.test_round_cache_ties_go_to_even(),
+    lambda: pins.test_delta_sum_is_the_decay_exponent_of_the_scan(True),
+    lambda: pins.test_carry_fold_composes_sequence_pieces((3, 8)),
 ]
 
 

@@ -448,3 +448,61 @@ def test_ssu_cache_dtype_rounds_the_state_after_the_readout():
         np.testing.assert_array_equal(o2, o)
         np.testing.assert_array_equal(st2, oracle.round_cache(st, dt_))
         assert not np.array_equal(st2, st)
+
+
+# ----------------------------------------------------------- sequence pieces --
+@pytest.mark.parametrize("softplus", [True, False])
+def test_delta_sum_is_the_decay_exponent_of_the_scan(softplus):
+    """With B = 0 the scan only decays its initial state, h_L = exp(A * S) h0
+    with S the sum of the steps' delta: oracle.delta_sum must give that S (the
+    scan is pinned to a recurrence-free brute force above)."""
+    s = gen.scan_inputs(2, 9, 3, 2, io="f32", seed=11, tag="dsum", h0=True)
+    dt = s.dt if softplus else np.abs(s.dt) * 0.05  # delta must stay positive without the softplus
+    A = np.array([[-0.5, -1.0], [-0.25, -2.0], [-1.5, -0.75]])
+    h0 = np.ones((2, 3, 2))
+    _, hL, _ = oracle.scan(s.x, dt, A, np.zeros_like(s.B), s.C, D=s.D, z=s.z, dt_bias=s.dt_bias,
+                           dt_softplus=softplus, h0=h0)
+    S = oracle.delta_sum(dt, s.dt_bias, dt_softplus=softplus)
+    np.testing.assert_allclose(hL, np.exp(A[None] * S[:, :, None]), rtol=1e-12, atol=0)
+    assert oracle.delta_sum(dt[..., :0], s.dt_bias).tolist() == [[0.0] * 3] * 2
+
+
+@pytest.mark.parametrize("cuts", [(5,), (3, 8), (1, 6, 11)])
+def test_carry_fold_composes_sequence_pieces(cuts):
+    """A prefill cut into consecutive pieces: each piece scanned from a zero
+    state (conv history: the raw inputs just before it) ends in h_end(j).
+    Folding h_in(j+1) = carry_fold(h_in(j), A, delta_sum(piece j), h_end(j))
+    from h_in(0) = h0 must give the state the whole scan reaches at every cut,
+    and each piece re-scanned from h_in(j) the whole scan's outputs."""
+    L = 14
+    s = gen.scan_inputs(2, L, 3, 4, W=4, io="f32", seed=12, tag="fold", conv_state=True, h0=True)
+    kw = dict(D=s.D, dt_bias=s.dt_bias, conv_weight=s.conv_weight, conv_bias=s.conv_bias)
+    piece = lambda a, t0, t1: a[..., t0:t1]  # noqa: E731
+    full, hf, _ = oracle.scan(s.x, s.dt, s.A, s.B, s.C, z=s.z, conv_state=s.conv_state, h0=s.h0, **kw)
+    bounds = (0,) + tuple(cuts) + (L,)
+    h_in = s.h0
+    cs = s.conv_state
+    for j in range(len(bounds) - 1):
+        t0, t1 = bounds[j], bounds[j + 1]
+        args = [piece(a, t0, t1) for a in (s.x, s.dt)] + [s.A] + [piece(a, t0, t1) for a in (s.B, s.C)]
+        out_j, _, cs_next = oracle.scan(*args, z=piece(s.z, t0, t1), conv_state=cs, h0=h_in, **kw)
+        np.testing.assert_allclose(out_j, full[..., t0:t1], rtol=1e-11, atol=1e-12)
+        _, h_end, _ = oracle.scan(*args, z=piece(s.z, t0, t1), conv_state=cs, h0=None, **kw)
+        h_in = oracle.carry_fold(h_in, s.A, oracle.delta_sum(piece(s.dt, t0, t1), s.dt_bias), h_end)
+        _, h_cut, _ = oracle.scan(*[piece(a, 0, t1) for a in (s.x, s.dt)], s.A,
+                                  *[piece(a, 0, t1) for a in (s.B, s.C)], z=piece(s.z, 0, t1),
+                                  conv_state=s.conv_state, h0=s.h0, **kw)
+        np.testing.assert_allclose(h_in, h_cut, rtol=1e-11, atol=1e-12)
+        cs = cs_next
+    np.testing.assert_allclose(h_in, hf, rtol=1e-11, atol=1e-12)
+
+
+def test_carry_fold_special_cases():
+    """A = 0: no decay, the states add; S = 0: the same; a decay far below
+    the smallest double: the earlier state is forgotten."""
+    rng = np.random.default_rng(13)
+    st, he = rng.standard_normal((2, 3, 4)), rng.standard_normal((2, 3, 4))
+    A = -rng.uniform(0.5, 2.0, (3, 4))
+    np.testing.assert_array_equal(oracle.carry_fold(st, np.zeros((3, 4)), np.ones((2, 3)), he), st + he)
+    np.testing.assert_array_equal(oracle.carry_fold(st, A, np.zeros((2, 3)), he), st + he)
+    np.testing.assert_array_equal(oracle.carry_fold(st, A, np.full((2, 3), 1e6), he), he)
