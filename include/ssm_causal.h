@@ -74,7 +74,7 @@
 extern "C" {
 #endif
 
-#define SSM_CAUSAL_ABI_VERSION 2
+#define SSM_CAUSAL_ABI_VERSION 3
 #define SSM_MAX_DIMS 5
 
 typedef enum ssm_dtype {
@@ -148,11 +148,13 @@ typedef enum ssm_kernel_id {
                                        16-step chunks; headdim and dstate contiguous,
                                        dstate 64, 128 or 256, headdim % 8 == 0 */
     SSM_KERNEL_SCAN_M2_GENERIC = 12, /* Mamba-2-layout prefill, any strides, warp per row */
-    SSM_KERNEL_SCAN_BAL = 13        /* fused prefill, persistent warps that each take an
+    SSM_KERNEL_SCAN_BAL = 13,       /* fused prefill, persistent warps that each take an
                                        equal slice of the (16-channel unit, 32-step
                                        chunk) list and hand states over through the
                                        workspace; d_state <= 16, conv width 0 or 4,
                                        time contiguous, L % 8 == 0, 16-byte aligned rows */
+    SSM_KERNEL_DELTA_SUM = 14,      /* sum of a sequence piece's delta, warp per (b, d) */
+    SSM_KERNEL_CARRY_FOLD = 15      /* state entering the next sequence piece, elementwise */
 } ssm_kernel_id;
 
 /* ------------------------------------------------------------------------ *
@@ -301,6 +303,60 @@ ssm_status ssm_selective_scan_workspace_size(const ssm_scan_args* args, uint64_t
 ssm_status ssm_selective_scan_fwd_noalloc(const ssm_scan_args* args, void* stream);
 
 /* ------------------------------------------------------------------------ *
+ * Sequence pieces: a prefill split along L across calls, devices or ranks
+ * (context parallelism; the scan is linear in the sequence length, the
+ * long-context point of "feat(llama.cu): 适配 mamba 模型" section 6.1).
+ *
+ * The scan is a first-order linear recurrence in h, so a sequence cut into
+ * consecutive pieces j = 0, 1, ... composes: run piece j from a zero ssm
+ * state (conv_state = the raw inputs just before it) with
+ * ssm_selective_scan_fwd to get its end state h_end(j), and its sum of steps
+ * S(j) with ssm_scan_delta_sum; then the state entering piece j+1 is
+ *
+ *     h_in(j+1)[b,d,n] = exp(A[d,n] * S(j)[b,d]) * h_in(j)[b,d,n] + h_end(j)[b,d,n]
+ *
+ * from h_in(0) = the sequence's initial state (ssm_scan_carry_fold applies
+ * one such step), and piece j run from h_in(j) gives the whole prefill's
+ * outputs over its steps.  Mamba-1 layout (x of rank 3) only.
+ *
+ * ssm_scan_delta_sum
+ *   dt          (B, D, L)  f32 | f16 | bf16
+ *   dt_bias     (D)        f32, optional (absent = 0)
+ *   dt_softplus nonzero: delta = softplus(dt + dt_bias), else dt + dt_bias
+ *   out         (B, D)     f32: sum over t of delta, accumulated in double
+ *                          (the prefill kernels' delta, rounded once)
+ * L = 0 writes zeros.
+ *
+ * ssm_scan_carry_fold
+ *   state       (B, D, N)  f32, in/out: h_in(j) in, h_in(j+1) out
+ *   A           (D, N)     f32
+ *   delta_sum   (B, D)     f32: S(j)
+ *   h_end       (B, D, N)  f32: h_end(j); may not overlap state
+ * ------------------------------------------------------------------------ */
+typedef struct ssm_delta_sum_args {
+    uint32_t struct_size; /* = sizeof(ssm_delta_sum_args) */
+    uint32_t flags;       /* SSM_FLAG_* */
+    ssm_tensor dt;
+    ssm_tensor dt_bias;
+    int32_t dt_softplus;
+    ssm_tensor out;
+    ssm_launch_info* info; /* optional */
+} ssm_delta_sum_args;
+
+typedef struct ssm_carry_fold_args {
+    uint32_t struct_size; /* = sizeof(ssm_carry_fold_args) */
+    uint32_t flags;       /* SSM_FLAG_* */
+    ssm_tensor state;
+    ssm_tensor A;
+    ssm_tensor delta_sum;
+    ssm_tensor h_end;
+    ssm_launch_info* info; /* optional */
+} ssm_carry_fold_args;
+
+ssm_status ssm_scan_delta_sum(const ssm_delta_sum_args* args, void* stream);
+ssm_status ssm_scan_carry_fold(const ssm_carry_fold_args* args, void* stream);
+
+/* ------------------------------------------------------------------------ *
  * ssm_selective_state_update -- one decode token, caches updated in place.
  *
  * Mamba-1 layout (state rank 3):
@@ -405,10 +461,10 @@ const char* ssm_status_string(int status);
 /* SSM_CAUSAL_ABI_VERSION of the loaded library. */
 int ssm_abi_version(void);
 
-/* sizeof() of the three args structs and of ssm_tensor / ssm_launch_info /
+/* sizeof() of the args structs and of ssm_tensor / ssm_launch_info /
  * ssm_device_error_report as compiled into the library, so that bindings can
  * check their layouts: which = 0 tensor, 1 conv1d args, 2 scan args, 3 ssu
- * args, 4 launch info, 5 error report. */
+ * args, 4 launch info, 5 error report, 6 delta-sum args, 7 carry-fold args. */
 size_t ssm_struct_size(int which);
 
 /* The wait budget, in cycles, that a failure test's request of `cycles`

@@ -2,10 +2,10 @@
 single-token selective_state_update, behind the C-ABI library
 ``libssm_causal.so`` (declared in ``include/ssm_causal.h``).
 
-The functions below are the thin ctypes binding of the three C entry points;
-they raise if the library has not been built (there is no fallback path).
+The functions below are the thin ctypes binding of the C entry points; they
+raise if the library has not been built (there is no fallback path).
 """
 from .binding import (LaunchInfo, SsmError, library, ssm_causal_conv1d_fwd,  # noqa: F401
-                      ssm_device_error, ssm_device_error_info, ssm_selective_scan_fwd,
-                      ssm_selective_scan_fwd_noalloc,
+                      ssm_device_error, ssm_device_error_info, ssm_scan_carry_fold,
+                      ssm_scan_delta_sum, ssm_selective_scan_fwd, ssm_selective_scan_fwd_noalloc,
                       ssm_selective_scan_workspace_size, ssm_selective_state_update)

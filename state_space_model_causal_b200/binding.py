@@ -37,7 +37,7 @@ STATUS = {
 KERNELS = {
     0: "none", 1: "conv1d", 2: "conv1d_generic", 3: "scan_chunked", 4: "scan_generic",
     5: "ssu_vec", 6: "ssu_generic", 7: "scan_vec", 8: "ssu_row", 9: "ssu_tma", 10: "ssu_row_tma",
-    11: "scan_m2", 12: "scan_m2_generic", 13: "scan_bal",
+    11: "scan_m2", 12: "scan_m2_generic", 13: "scan_bal", 14: "delta_sum", 15: "carry_fold",
 }
 
 
@@ -100,6 +100,18 @@ class SsuArgs(ctypes.Structure):
                 ("info", ctypes.POINTER(LaunchInfo))]
 
 
+class DeltaSumArgs(ctypes.Structure):
+    _fields_ = [("struct_size", ctypes.c_uint32), ("flags", ctypes.c_uint32),
+                ("dt", Tensor), ("dt_bias", Tensor), ("dt_softplus", ctypes.c_int32), ("out", Tensor),
+                ("info", ctypes.POINTER(LaunchInfo))]
+
+
+class CarryFoldArgs(ctypes.Structure):
+    _fields_ = [("struct_size", ctypes.c_uint32), ("flags", ctypes.c_uint32),
+                ("state", Tensor), ("A", Tensor), ("delta_sum", Tensor), ("h_end", Tensor),
+                ("info", ctypes.POINTER(LaunchInfo))]
+
+
 _lock = threading.Lock()
 _lib = None
 _override = None  # a library swapped in by using_library() (failure tests)
@@ -144,7 +156,9 @@ def _open(path):
     lib = ctypes.CDLL(path)
     for name, argt in (("ssm_causal_conv1d_fwd", Conv1dArgs),
                        ("ssm_selective_scan_fwd", ScanArgs),
-                       ("ssm_selective_state_update", SsuArgs)):
+                       ("ssm_selective_state_update", SsuArgs),
+                       ("ssm_scan_delta_sum", DeltaSumArgs),
+                       ("ssm_scan_carry_fold", CarryFoldArgs)):
         fn = getattr(lib, name)
         fn.restype = ctypes.c_int
         fn.argtypes = [ctypes.POINTER(argt), ctypes.c_void_p]
@@ -164,7 +178,8 @@ def _open(path):
     lib.ssm_test_clamp_wait_budget.argtypes = [ctypes.c_longlong]
     lib.ssm_struct_size.restype = ctypes.c_size_t
     lib.ssm_struct_size.argtypes = [ctypes.c_int]
-    for which, st in enumerate((Tensor, Conv1dArgs, ScanArgs, SsuArgs, LaunchInfo, ErrorReport)):
+    for which, st in enumerate((Tensor, Conv1dArgs, ScanArgs, SsuArgs, LaunchInfo, ErrorReport,
+                                DeltaSumArgs, CarryFoldArgs)):
         if lib.ssm_struct_size(which) != ctypes.sizeof(st):
             raise ImportError(f"struct layout mismatch for {st.__name__}")
     return lib
@@ -424,6 +439,34 @@ def ssm_selective_state_update(state, x, dt, A, B, C, D=None, z=None, dt_bias=No
                  state_batch_indices, out), stream),
            "ssm_selective_state_update")
     return out
+
+
+def ssm_scan_delta_sum(dt, dt_bias=None, dt_softplus=True, out=None, stream=None,
+                       info: Optional[LaunchInfo] = None):
+    """Sum over t of a sequence piece's delta (see include/ssm_causal.h):
+    dt (B, D, L) -> (B, D) float32."""
+    import torch
+    if out is None:
+        out = torch.empty(dt.shape[0], dt.shape[1], dtype=torch.float32, device=dt.device)
+    a = DeltaSumArgs()
+    a.struct_size = ctypes.sizeof(DeltaSumArgs)
+    a.dt, a.dt_bias, a.out = map(describe, (dt, dt_bias, out))
+    a.dt_softplus = int(bool(dt_softplus))
+    a.info = _info_ptr(info)
+    _check(_run(library().ssm_scan_delta_sum, a, (dt, dt_bias, out), stream), "ssm_scan_delta_sum")
+    return out
+
+
+def ssm_scan_carry_fold(state, A, delta_sum, h_end, stream=None, info: Optional[LaunchInfo] = None):
+    """state <- exp(A * delta_sum) * state + h_end in place: the state entering
+    the next sequence piece (see include/ssm_causal.h).  Returns state."""
+    a = CarryFoldArgs()
+    a.struct_size = ctypes.sizeof(CarryFoldArgs)
+    a.state, a.A, a.delta_sum, a.h_end = map(describe, (state, A, delta_sum, h_end))
+    a.info = _info_ptr(info)
+    _check(_run(library().ssm_scan_carry_fold, a, (state, A, delta_sum, h_end), stream),
+           "ssm_scan_carry_fold")
+    return state
 
 
 def ssm_device_error(stream=None) -> int:

@@ -298,6 +298,86 @@ ssm_status conv1d_impl(const ssm_conv1d_args* a, cudaStream_t stream) {
     return launch_conv1d(p, plan, stream) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 
+// --------------------------------------------------------- sequence pieces --
+ssm_status delta_sum_impl(const ssm_delta_sum_args* a, cudaStream_t stream) {
+    if (!a) return SSM_ERR_NULL;
+    if (a->struct_size != sizeof(ssm_delta_sum_args)) return SSM_ERR_VERSION;
+    SSM_TRY(info_ok(a->info));
+    SSM_TRY(basic(a->dt));
+    SSM_TRY(basic(a->out));
+    if (a->dt.ndim != 3) return SSM_ERR_SHAPE;
+    const int64_t B = a->dt.shape[0], D = a->dt.shape[1], L = a->dt.shape[2];
+    if (!is_float(a->dt.dtype) || a->out.dtype != SSM_F32) return SSM_ERR_DTYPE;
+    SSM_TRY(want(a->out, {B, D}));
+    if (!non_overlapping(a->out)) return SSM_ERR_STRIDE;
+    if (present(a->dt_bias)) {
+        SSM_TRY(basic(a->dt_bias));
+        SSM_TRY(want(a->dt_bias, {D}));
+        if (a->dt_bias.dtype != SSM_F32) return SSM_ERR_DTYPE;
+    }
+    if (overlap(a->out, a->dt) || overlap(a->out, a->dt_bias)) return SSM_ERR_ALIAS;
+    const int64_t rows = B * D;
+    if (rows == 0) {
+        fill_info(a->info, SSM_KERNEL_NONE, 0, 0, 0, 0, 0);
+        return SSM_OK;
+    }
+    constexpr int kBlock = 256;
+    const int64_t grid = (rows + kBlock / 32 - 1) / (kBlock / 32);  // one warp per row
+    if (grid > INT32_MAX) return SSM_ERR_UNSUPPORTED;
+    fill_info(a->info, SSM_KERNEL_DELTA_SUM, (int)grid, kBlock, 0, 1, rows);
+    if (a->flags & SSM_FLAG_DRY_RUN) return SSM_OK;
+    DeltaSumProblem p{};
+    p.Bn = B; p.D = D; p.L = L; p.dt_dt = a->dt.dtype;
+    p.dt = a->dt.data; p.dt_b = sd(a->dt, 0); p.dt_d = sd(a->dt, 1); p.dt_t = sd(a->dt, 2);
+    p.dt_bias = static_cast<const float*>(a->dt_bias.data);
+    p.db_d = present(a->dt_bias) ? sd(a->dt_bias, 0) : 0;
+    p.softplus = a->dt_softplus != 0;
+    p.out = static_cast<float*>(a->out.data); p.o_b = sd(a->out, 0); p.o_d = sd(a->out, 1);
+    return launch_delta_sum(p, (int)grid, kBlock, stream) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+ssm_status carry_fold_impl(const ssm_carry_fold_args* a, cudaStream_t stream) {
+    if (!a) return SSM_ERR_NULL;
+    if (a->struct_size != sizeof(ssm_carry_fold_args)) return SSM_ERR_VERSION;
+    SSM_TRY(info_ok(a->info));
+    SSM_TRY(basic(a->state));
+    SSM_TRY(basic(a->A));
+    SSM_TRY(basic(a->delta_sum));
+    SSM_TRY(basic(a->h_end));
+    if (a->state.ndim != 3) return SSM_ERR_SHAPE;
+    const int64_t B = a->state.shape[0], D = a->state.shape[1], N = a->state.shape[2];
+    SSM_TRY(want(a->A, {D, N}));
+    SSM_TRY(want(a->delta_sum, {B, D}));
+    SSM_TRY(want(a->h_end, {B, D, N}));
+    const ssm_tensor* all[] = {&a->state, &a->A, &a->delta_sum, &a->h_end};
+    for (const ssm_tensor* t : all)
+        if (t->dtype != SSM_F32) return SSM_ERR_DTYPE;
+    if (!non_overlapping(a->state)) return SSM_ERR_STRIDE;
+    if (overlap(a->state, a->A) || overlap(a->state, a->delta_sum) || overlap(a->state, a->h_end))
+        return SSM_ERR_ALIAS;
+    const int64_t total = B * D * N;
+    if (total == 0) {
+        fill_info(a->info, SSM_KERNEL_NONE, 0, 0, 0, 0, 0);
+        return SSM_OK;
+    }
+    constexpr int kBlock = 256;
+    const bool dry = (a->flags & SSM_FLAG_DRY_RUN) != 0;
+    // grid-stride: at most 16 CTAs of 256 threads per SM
+    const int64_t grid = std::min<int64_t>((total + kBlock - 1) / kBlock, (int64_t)sm_count(dry) * 16);
+    fill_info(a->info, SSM_KERNEL_CARRY_FOLD, (int)grid, kBlock, 0, N, B * D);
+    if (dry) return SSM_OK;
+    CarryFoldProblem p{};
+    p.Bn = B; p.D = D; p.N = N;
+    p.state = static_cast<float*>(a->state.data);
+    p.s_b = sd(a->state, 0); p.s_d = sd(a->state, 1); p.s_n = sd(a->state, 2);
+    p.A = static_cast<const float*>(a->A.data); p.A_d = sd(a->A, 0); p.A_n = sd(a->A, 1);
+    p.S = static_cast<const float*>(a->delta_sum.data);
+    p.S_b = sd(a->delta_sum, 0); p.S_d = sd(a->delta_sum, 1);
+    p.h_end = static_cast<const float*>(a->h_end.data);
+    p.h_b = sd(a->h_end, 0); p.h_d = sd(a->h_end, 1); p.h_n = sd(a->h_end, 2);
+    return launch_carry_fold(p, (int)grid, kBlock, stream) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
 // ------------------------------------------------------------- workspace --
 // Balanced prefill workspace: a 256-byte header (generation, finished-worker
 // count), one 32-bit flag per worker (rounded up to 256 bytes), then one
@@ -1219,6 +1299,14 @@ ssm_status ssm_selective_state_update(const ssm_ssu_args* args, void* stream) {
     return ssu_impl(args, static_cast<cudaStream_t>(stream));
 }
 
+ssm_status ssm_scan_delta_sum(const ssm_delta_sum_args* args, void* stream) {
+    return delta_sum_impl(args, static_cast<cudaStream_t>(stream));
+}
+
+ssm_status ssm_scan_carry_fold(const ssm_carry_fold_args* args, void* stream) {
+    return carry_fold_impl(args, static_cast<cudaStream_t>(stream));
+}
+
 const char* ssm_status_string(int status) {
     switch (status) {
         case SSM_OK: return "SSM_OK";
@@ -1267,6 +1355,8 @@ size_t ssm_struct_size(int which) {
         case 3: return sizeof(ssm_ssu_args);
         case 4: return sizeof(ssm_launch_info);
         case 5: return sizeof(ssm_device_error_report);
+        case 6: return sizeof(ssm_delta_sum_args);
+        case 7: return sizeof(ssm_carry_fold_args);
         default: return 0;
     }
 }

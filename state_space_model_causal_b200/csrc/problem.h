@@ -177,6 +177,26 @@ struct Conv1dProblem {
     void* out; int64_t o_b, o_d, o_t;
 };
 
+// Sum of a sequence piece's delta: dt (Bn, D, L) any strides; out (Bn, D) f32.
+struct DeltaSumProblem {
+    int64_t Bn, D, L;
+    int dt_dt;
+    const void* dt; int64_t dt_b, dt_d, dt_t;
+    const float* dt_bias; int64_t db_d;
+    int softplus;
+    float* out; int64_t o_b, o_d;
+};
+
+// State entering the next sequence piece: state, h_end (Bn, D, N); A (D, N);
+// S (Bn, D); all f32, any strides.
+struct CarryFoldProblem {
+    int64_t Bn, D, N;
+    float* state; int64_t s_b, s_d, s_n;
+    const float* A; int64_t A_d, A_n;
+    const float* S; int64_t S_b, S_d;
+    const float* h_end; int64_t h_b, h_d, h_n;
+};
+
 struct Conv1dPlan {
     int kernel;
     int block;
@@ -206,6 +226,8 @@ int scan_vec_threads();
 int scan_vec_channels_per_cta();
 cudaError_t launch_scan_vec(const ScanProblem& p, int sw_pairs, cudaStream_t s);
 cudaError_t launch_conv1d(const Conv1dProblem& p, const Conv1dPlan& plan, cudaStream_t s);
+cudaError_t launch_delta_sum(const DeltaSumProblem& p, int grid, int block, cudaStream_t s);
+cudaError_t launch_carry_fold(const CarryFoldProblem& p, int grid, int block, cudaStream_t s);
 int scan_m2_rows_per_cta(int64_t N);
 int scan_m2_threads();
 int scan_m2_smem_bytes(int io_dt, int64_t N);

@@ -35,6 +35,7 @@ def declared_functions():
 def test_header_declares_the_three_entry_points():
     fns = declared_functions()
     for name in ("ssm_causal_conv1d_fwd", "ssm_selective_scan_fwd", "ssm_selective_state_update",
+                 "ssm_scan_delta_sum", "ssm_scan_carry_fold",
                  "ssm_status_string", "ssm_abi_version", "ssm_struct_size"):
         assert name in fns
 
@@ -45,9 +46,9 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_struct_layouts(lib):
-    assert lib.ssm_abi_version() == 2
+    assert lib.ssm_abi_version() == 3
     for which, st in enumerate((bd.Tensor, bd.Conv1dArgs, bd.ScanArgs, bd.SsuArgs, bd.LaunchInfo,
-                                bd.ErrorReport)):
+                                bd.ErrorReport, bd.DeltaSumArgs, bd.CarryFoldArgs)):
         assert lib.ssm_struct_size(which) == ctypes.sizeof(st)
     assert lib.ssm_struct_size(99) == 0
 
@@ -643,3 +644,76 @@ def test_plain_c_client_links_and_runs(tmp_path, lib):
     res = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert res.returncode == 0, res.stdout + res.stderr
     assert "fails 0" in res.stdout
+
+
+# ----------------------------------------------------------- sequence pieces --
+def delta_sum_args(mem, Bn=2, D=64, L=300, io=F16, **over):
+    a = bd.DeltaSumArgs()
+    a.struct_size = ctypes.sizeof(bd.DeltaSumArgs)
+    a.flags = bd.SSM_FLAG_DRY_RUN
+    a.dt = mem(io, (Bn, D, L))
+    a.dt_bias = mem(F32, (D,))
+    a.dt_softplus = 1
+    a.out = mem(F32, (Bn, D))
+    for k, v in over.items():
+        setattr(a, k, v)
+    return a
+
+
+def carry_fold_args(mem, Bn=2, D=64, N=16, **over):
+    a = bd.CarryFoldArgs()
+    a.struct_size = ctypes.sizeof(bd.CarryFoldArgs)
+    a.flags = bd.SSM_FLAG_DRY_RUN
+    a.state = mem(F32, (Bn, D, N))
+    a.A = mem(F32, (D, N))
+    a.delta_sum = mem(F32, (Bn, D))
+    a.h_end = mem(F32, (Bn, D, N))
+    for k, v in over.items():
+        setattr(a, k, v)
+    return a
+
+
+def test_delta_sum_plan_and_checks(lib):
+    """One warp per (b, d) row, 8 rows per 256-thread CTA; fp32 output of
+    shape (B, D); dt of any float dtype; bias optional; empty rows launch
+    nothing; an output over dt is refused."""
+    mem = FakeMem()
+    st, info = call(lib, "ssm_scan_delta_sum", delta_sum_args(mem))
+    assert st == OK and bd.KERNELS[info.kernel] == "delta_sum"
+    assert info.grid == 2 * 64 // 8 and info.block == 256 and info.work_items == 128
+    st, _ = call(lib, "ssm_scan_delta_sum", delta_sum_args(mem, io=F32, dt_bias=bd.Tensor()))
+    assert st == OK
+    st, _ = call(lib, "ssm_scan_delta_sum", delta_sum_args(mem, L=0))  # writes zeros
+    assert st == OK
+    st, info = call(lib, "ssm_scan_delta_sum", delta_sum_args(mem, Bn=0, out=mem(F32, (0, 64))))
+    assert st == OK and bd.KERNELS[info.kernel] == "none"
+    assert call(lib, "ssm_scan_delta_sum", delta_sum_args(mem, out=mem(F16, (2, 64))))[0] == EDTYPE
+    assert call(lib, "ssm_scan_delta_sum", delta_sum_args(mem, out=mem(F32, (2, 63))))[0] == ESHAPE
+    assert call(lib, "ssm_scan_delta_sum", delta_sum_args(mem, dt_bias=mem(F32, (65,))))[0] == ESHAPE
+    a = delta_sum_args(mem)
+    a.out = bd.raw_tensor(a.dt.data, F32, (2, 64))
+    assert call(lib, "ssm_scan_delta_sum", a)[0] == EALIAS
+    a = delta_sum_args(mem)
+    a.struct_size -= 8
+    assert call(lib, "ssm_scan_delta_sum", a)[0] == EVER
+
+
+def test_carry_fold_plan_and_checks(lib):
+    """Elementwise over B*D*N with a grid-stride loop of at most 16 CTAs per
+    SM; every tensor fp32 with matching shapes; the state may not overlap an
+    input."""
+    mem = FakeMem()
+    st, info = call(lib, "ssm_scan_carry_fold", carry_fold_args(mem))
+    assert st == OK and bd.KERNELS[info.kernel] == "carry_fold"
+    assert info.grid == 2 * 64 * 16 // 256 and info.rows_per_item == 16 and info.work_items == 128
+    st, info = call(lib, "ssm_scan_carry_fold", carry_fold_args(mem, Bn=64, D=5120, N=16))
+    assert st == OK and info.grid == 148 * 16
+    assert call(lib, "ssm_scan_carry_fold", carry_fold_args(mem, A=mem(F32, (64, 15))))[0] == ESHAPE
+    assert call(lib, "ssm_scan_carry_fold", carry_fold_args(mem, delta_sum=mem(F16, (2, 64))))[0] == EDTYPE
+    a = carry_fold_args(mem)
+    a.h_end = bd.raw_tensor(a.state.data, F32, (2, 64, 16))
+    assert call(lib, "ssm_scan_carry_fold", a)[0] == EALIAS
+    st, info = call(lib, "ssm_scan_carry_fold", carry_fold_args(mem, Bn=0, state=mem(F32, (0, 64, 16)),
+                                                                  delta_sum=mem(F32, (0, 64)),
+                                                                  h_end=mem(F32, (0, 64, 16))))
+    assert st == OK and bd.KERNELS[info.kernel] == "none"
