@@ -433,8 +433,13 @@ ssm_status ssm_selective_state_update(const ssm_ssu_args* args, void* stream);
  *   ssm_selective_scan_fwd (SSM_KERNEL_SCAN_BAL): a warp that waited in vain
  *     for its predecessor's hand-over scans its piece of that unit from a
  *     zero state instead; first_item is the lowest such unit
- *     (batch * ceil(D / 16) + channel / 16); that unit's later outputs and
- *     final state are wrong, all other units are complete.
+ *     (batch * ceil(D / 16) + channel / 16); in the context-parallel mode
+ *     it is unit * (pieces - 1) + piece, less 1 in the second pass.  That
+ *     unit's later outputs and final state are wrong, all other units are
+ *     complete.
+ *   ssm_selective_scan_fwd, x of rank 4 (SSM_KERNEL_SCAN_M2): the same for a
+ *     CTA that waited in vain for its predecessor's state tile; first_item is
+ *     the unit (b * H + h) * ceil(P / rows per CTA) + row block.
  *
  * The record belongs to the CURRENT device: call these with that device
  * current and a stream of that device.  Both wait for the work enqueued on
