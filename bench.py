@@ -62,6 +62,23 @@ def peaks():
         return FALLBACK_HBM_GBS, SM_MAX_MHZ, "fallback"
 
 
+def probe_rates():
+    """Every `name: value` line of profiles/sfu_pipe_rates.txt (the figures
+    `python bench.py --peaks` printed on this machine's B200s)."""
+    rec = {}
+    try:
+        for line in open(os.path.join(ROOT, "profiles", "sfu_pipe_rates.txt")):
+            if ":" in line and not line.startswith("#"):
+                k, v = line.split(":", 1)
+                try:
+                    rec[k.strip()] = float(v)
+                except ValueError:
+                    pass
+    except OSError:
+        pass
+    return rec
+
+
 def sfu_rate():
     """ex2 operations per clock per SM: the rate `python bench.py --peaks`
     measured on this machine's B200s (recorded in profiles/sfu_pipe_rates.txt),
@@ -92,6 +109,17 @@ template <int OP> __global__ void k(float* out, int iters) {
   float s = 0; for (int j = 0; j < 16; ++j) s += acc[j];
   if (s == 1234.5f) out[0] = s;
 }
+// STREAM-style copy: four 16-byte loads in flight per thread, then the stores
+__global__ void copy16(const float4* __restrict__ a, float4* __restrict__ b, size_t n) {
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += 4 * stride) {
+    float4 v[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) if (i + k * stride < n) v[k] = a[i + k * stride];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) if (i + k * stride < n) b[i + k * stride] = v[k];
+  }
+}
 int main() {
   float* d; if (cudaMalloc(&d, 4) != cudaSuccess) return 1;
   int sms, clk; cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, 0); cudaDeviceGetAttribute(&clk, cudaDevAttrClockRate, 0);
@@ -102,6 +130,25 @@ int main() {
     L(); cudaDeviceSynchronize(); cudaEventRecord(a); L(); cudaEventRecord(b); cudaEventSynchronize(b);
     float ms; cudaEventElapsedTime(&ms, a, b);
     printf("%s_per_clk_per_sm: %.3f\n", op == 0 ? "ex2" : "rcp", (double)blocks * 128 * 16 * iters / (ms * 1e-3) / sms / (clk * 1e3));
+  }
+  {
+    const size_t bytes = (size_t)2 << 30;  // 2 GiB each way, far beyond L2
+    float4 *x, *y;
+    if (cudaMalloc(&x, bytes) != cudaSuccess || cudaMalloc(&y, bytes) != cudaSuccess) return 1;
+    cudaMemset(x, 0, bytes);
+    const size_t n = bytes / 16;
+    float best = 1e30f;
+    for (int rep = 0; rep < 12; ++rep) {  // kernel copies, then the runtime's device-to-device copy
+      cudaEventRecord(a);
+      if (rep < 6) copy16<<<sms * 4, 512>>>(x, y, n);
+      else cudaMemcpyAsync(y, x, bytes, cudaMemcpyDeviceToDevice, 0);
+      cudaEventRecord(b);
+      cudaEventSynchronize(b);
+      float ms; cudaEventElapsedTime(&ms, a, b);
+      if (rep != 0 && rep != 6 && ms < best) best = ms;  // the first of each kind warms up
+    }
+    printf("hbm_copy_gbs: %.1f\n", 2.0 * bytes / (best * 1e-3) / 1e9);
+    cudaFree(x); cudaFree(y);
   }
   return cudaGetLastError() == cudaSuccess ? 0 : 1;
 }
@@ -947,7 +994,13 @@ def main():
             "roofline": roofline, "cpu_baseline": cpu,
             "e2e": {"value": round(e2e_val, 3), "unit": "Gelem/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
-            "gpu_launches": args.steps, "clocks": clk.summary(), "prefill_mamba2": prefill_m2,
+            "gpu_launches": args.steps, "clocks": clk.summary(),
+            "peaks": {"hbm_gbs": hbm_peak, "hbm_kind": peak_src,
+                      "hbm_copy_probe_gbs": probe_rates().get("hbm_copy_gbs"),
+                      "ex2_per_clk_per_sm": ex2_rate, "ex2_kind": ex2_kind,
+                      "note": "roofline fractions use hbm_gbs (MEASURED_PEAKS.json, else the fallback "
+                              "figure); the copy probe of bench.py --peaks is context"},
+            "prefill_mamba2": prefill_m2,
             "prefill_one_sequence": prefill_b1,
             "decode": decode}
     print(json.dumps(line), flush=True)
