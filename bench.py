@@ -447,6 +447,67 @@ def time_prefill_e2e(pf, steps, warmup, dev):
     return ms, h2d, d2h
 
 
+def time_prefill_e2e_pipelined(pf, steps, warmup, dev):
+    """The end-to-end metric with the steps pipelined the way a stream of
+    prefills runs: two sets of device buffers; step i's inputs go up on a
+    copy stream while step i-1 computes on a second stream and step i-2's
+    results come down on a third (the two copy directions use separate copy
+    engines).  Every step still copies all its inputs from pinned host memory
+    and reads its results back.  Returns (ms per step, H2D bytes, D2H bytes)
+    from events around the whole run: the first upload to the last download."""
+    import torch
+    from state_space_model_causal_b200 import ssm_selective_scan_fwd
+    names_in, names_out = ("x", "dt", "z", "B", "C"), ("out", "h", "cs")
+    host = {k: getattr(pf, k).cpu().pin_memory() for k in names_in}
+    back = [{k: torch.empty_like(getattr(pf, k), device="cpu").pin_memory() for k in names_out}
+            for _ in range(2)]
+    sets = [{k: getattr(pf, k) for k in names_in + names_out}]
+    sets.append({k: torch.empty_like(v) for k, v in sets[0].items()})
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = sum(v.numel() * v.element_size() for v in back[0].values())
+    up, comp, down = (torch.cuda.Stream(dev) for _ in range(3))
+    done_comp = [torch.cuda.Event() for _ in range(2)]   # set j's inputs consumed
+    done_down = [torch.cuda.Event() for _ in range(2)]   # set j's results read back
+    ready = [torch.cuda.Event() for _ in range(2)]       # set j's inputs uploaded
+    for j in range(2):  # nothing pending yet
+        done_comp[j].record(comp)
+        done_down[j].record(down)
+
+    def step(i):
+        j = i % 2
+        S, hb = sets[j], back[j]
+        with torch.cuda.stream(up):
+            up.wait_event(done_comp[j])
+            for k in names_in:
+                S[k].copy_(host[k], non_blocking=True)
+            ready[j].record(up)
+        with torch.cuda.stream(comp):
+            comp.wait_event(ready[j])
+            comp.wait_event(done_down[j])
+            S["h"].zero_()
+            S["cs"].zero_()
+            ssm_selective_scan_fwd(S["x"], S["dt"], pf.A, S["B"], S["C"], D=pf.Dv, z=S["z"],
+                                   dt_bias=pf.db, conv_weight=pf.cw, conv_bias=pf.cb,
+                                   conv_state=S["cs"], ssm_state=S["h"], out=S["out"], stream=comp)
+            done_comp[j].record(comp)
+        with torch.cuda.stream(down):
+            down.wait_event(done_comp[j])
+            for k in names_out:
+                hb[k].copy_(S[k], non_blocking=True)
+            done_down[j].record(down)
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(up)
+    for i in range(steps):
+        step(i)
+    b.record(down)
+    torch.cuda.synchronize(dev)
+    return a.elapsed_time(b) / steps, h2d, d2h
+
+
 # ---------------------------------------------------------------- decode --
 def graph_time(calls, replays, dev, warm_eager=3):
     """Per-call microseconds: `calls` (a list of closures) captured in one
@@ -953,7 +1014,9 @@ def main():
                 "algorithmic_bytes_per_launch": alg_bytes}
 
     e2e_ms, h2d, d2h = time_prefill_e2e(pf, max(3, args.steps // 4), 3, dev)
-    e2e_val = world * pf.elems / (statistics.mean(e2e_ms) * 1e-3) / 1e9
+    e2e_serial = world * pf.elems / (statistics.mean(e2e_ms) * 1e-3) / 1e9
+    e2e_pipe_ms, _, _ = time_prefill_e2e_pipelined(pf, max(6, args.steps // 4), 3, dev)
+    e2e_val = world * pf.elems / (e2e_pipe_ms * 1e-3) / 1e9
 
     prefill_m2 = prefill_mamba2(dev, hbm_peak, sm_max) if not args.no_decode else None
     prefill_b1 = prefill_single_sequence(dev, sfu_peak, hbm_peak) if not args.no_decode else None
@@ -993,7 +1056,12 @@ def main():
                        "l2": "flushed (256 MiB write) before every step; inputs 338 MB > 126 MB L2"},
             "roofline": roofline, "cpu_baseline": cpu,
             "e2e": {"value": round(e2e_val, 3), "unit": "Gelem/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h},
+                    "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_pipe_ms, 3),
+                    "method": "pipelined: step i's inputs upload while step i-1 computes and step i-2's "
+                              "results download (two device buffer sets, three streams), events from "
+                              "the first upload to the last download",
+                    "serial_value": round(e2e_serial, 3),
+                    "serial_method": "one step at a time: upload, call, download inside each step's events"},
             "gpu_launches": args.steps, "clocks": clk.summary(),
             "peaks": {"hbm_gbs": hbm_peak, "hbm_kind": peak_src,
                       "hbm_copy_probe_gbs": probe_rates().get("hbm_copy_gbs"),
