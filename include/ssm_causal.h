@@ -317,7 +317,9 @@ ssm_status ssm_selective_scan_fwd_noalloc(const ssm_scan_args* args, void* strea
  *
  * from h_in(0) = the sequence's initial state (ssm_scan_carry_fold applies
  * one such step), and piece j run from h_in(j) gives the whole prefill's
- * outputs over its steps.  Mamba-1 layout (x of rank 3) only.
+ * outputs over its steps.  In the Mamba-2 layout (x of rank 4) the same holds
+ * per head: S(j)[b,h] from dt (B, H, L), and
+ * h_in(j+1)[b,h,p,n] = exp(A[h] * S(j)[b,h]) * h_in(j)[b,h,p,n] + h_end(j)[b,h,p,n].
  *
  * ssm_scan_delta_sum
  *   dt          (B, D, L)  f32 | f16 | bf16
@@ -328,10 +330,10 @@ ssm_status ssm_selective_scan_fwd_noalloc(const ssm_scan_args* args, void* strea
  * L = 0 writes zeros.
  *
  * ssm_scan_carry_fold
- *   state       (B, D, N)  f32, in/out: h_in(j) in, h_in(j+1) out
- *   A           (D, N)     f32
- *   delta_sum   (B, D)     f32: S(j)
- *   h_end       (B, D, N)  f32: h_end(j); may not overlap state
+ *   state       (B, D, N) or (B, H, P, N)  f32, in/out: h_in(j) in, h_in(j+1) out
+ *   A           (D, N)    or (H)           f32
+ *   delta_sum   (B, D)    or (B, H)        f32: S(j)
+ *   h_end       like state                 f32: h_end(j); may not overlap state
  * ------------------------------------------------------------------------ */
 typedef struct ssm_delta_sum_args {
     uint32_t struct_size; /* = sizeof(ssm_delta_sum_args) */

@@ -344,18 +344,38 @@ ssm_status carry_fold_impl(const ssm_carry_fold_args* a, cudaStream_t stream) {
     SSM_TRY(basic(a->A));
     SSM_TRY(basic(a->delta_sum));
     SSM_TRY(basic(a->h_end));
-    if (a->state.ndim != 3) return SSM_ERR_SHAPE;
-    const int64_t B = a->state.shape[0], D = a->state.shape[1], N = a->state.shape[2];
-    SSM_TRY(want(a->A, {D, N}));
-    SSM_TRY(want(a->delta_sum, {B, D}));
-    SSM_TRY(want(a->h_end, {B, D, N}));
+    CarryFoldProblem p{};
+    if (a->state.ndim == 3) {
+        // Mamba-1 layout: (B, D, N), A (D, N), S (B, D)
+        const int64_t B = a->state.shape[0], D = a->state.shape[1], N = a->state.shape[2];
+        SSM_TRY(want(a->A, {D, N}));
+        SSM_TRY(want(a->delta_sum, {B, D}));
+        SSM_TRY(want(a->h_end, {B, D, N}));
+        p.Bn = B; p.H = D; p.P = 1; p.N = N;
+        p.s_b = sd(a->state, 0); p.s_h = sd(a->state, 1); p.s_p = 0; p.s_n = sd(a->state, 2);
+        p.A_h = sd(a->A, 0); p.A_p = 0; p.A_n = sd(a->A, 1);
+        p.h_b = sd(a->h_end, 0); p.h_h = sd(a->h_end, 1); p.h_p = 0; p.h_n = sd(a->h_end, 2);
+    } else if (a->state.ndim == 4) {
+        // Mamba-2 layout: (B, H, P, N), A (H) per head, S (B, H)
+        const int64_t B = a->state.shape[0], H = a->state.shape[1], P = a->state.shape[2],
+                      N = a->state.shape[3];
+        SSM_TRY(want(a->A, {H}));
+        SSM_TRY(want(a->delta_sum, {B, H}));
+        SSM_TRY(want(a->h_end, {B, H, P, N}));
+        p.Bn = B; p.H = H; p.P = P; p.N = N;
+        p.s_b = sd(a->state, 0); p.s_h = sd(a->state, 1); p.s_p = sd(a->state, 2); p.s_n = sd(a->state, 3);
+        p.A_h = sd(a->A, 0); p.A_p = 0; p.A_n = 0;
+        p.h_b = sd(a->h_end, 0); p.h_h = sd(a->h_end, 1); p.h_p = sd(a->h_end, 2); p.h_n = sd(a->h_end, 3);
+    } else {
+        return SSM_ERR_SHAPE;
+    }
     const ssm_tensor* all[] = {&a->state, &a->A, &a->delta_sum, &a->h_end};
     for (const ssm_tensor* t : all)
         if (t->dtype != SSM_F32) return SSM_ERR_DTYPE;
     if (!non_overlapping(a->state)) return SSM_ERR_STRIDE;
     if (overlap(a->state, a->A) || overlap(a->state, a->delta_sum) || overlap(a->state, a->h_end))
         return SSM_ERR_ALIAS;
-    const int64_t total = B * D * N;
+    const int64_t total = p.Bn * p.H * p.P * p.N;
     if (total == 0) {
         fill_info(a->info, SSM_KERNEL_NONE, 0, 0, 0, 0, 0);
         return SSM_OK;
@@ -364,17 +384,13 @@ ssm_status carry_fold_impl(const ssm_carry_fold_args* a, cudaStream_t stream) {
     const bool dry = (a->flags & SSM_FLAG_DRY_RUN) != 0;
     // grid-stride: at most 16 CTAs of 256 threads per SM
     const int64_t grid = std::min<int64_t>((total + kBlock - 1) / kBlock, (int64_t)sm_count(dry) * 16);
-    fill_info(a->info, SSM_KERNEL_CARRY_FOLD, (int)grid, kBlock, 0, N, B * D);
+    fill_info(a->info, SSM_KERNEL_CARRY_FOLD, (int)grid, kBlock, 0, p.P * p.N, p.Bn * p.H);
     if (dry) return SSM_OK;
-    CarryFoldProblem p{};
-    p.Bn = B; p.D = D; p.N = N;
     p.state = static_cast<float*>(a->state.data);
-    p.s_b = sd(a->state, 0); p.s_d = sd(a->state, 1); p.s_n = sd(a->state, 2);
-    p.A = static_cast<const float*>(a->A.data); p.A_d = sd(a->A, 0); p.A_n = sd(a->A, 1);
+    p.A = static_cast<const float*>(a->A.data);
     p.S = static_cast<const float*>(a->delta_sum.data);
-    p.S_b = sd(a->delta_sum, 0); p.S_d = sd(a->delta_sum, 1);
+    p.S_b = sd(a->delta_sum, 0); p.S_h = sd(a->delta_sum, 1);
     p.h_end = static_cast<const float*>(a->h_end.data);
-    p.h_b = sd(a->h_end, 0); p.h_d = sd(a->h_end, 1); p.h_n = sd(a->h_end, 2);
     return launch_carry_fold(p, (int)grid, kBlock, stream) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 

@@ -13,7 +13,9 @@
 //   delta_sum_kernel   S[b,d] = sum_t delta(dt[b,d,t] + dt_bias[d]); one warp per
 //                      (b, d) row, lanes over t, the sum in double; delta is the
 //                      prefill kernels' own softplus
-//   carry_fold_kernel  state <- exp(A * S) * state + h_end, elementwise, grid-stride
+//   carry_fold_kernel  state <- exp(A * S) * state + h_end, elementwise, grid-stride;
+//                      the Mamba-1 layout (A per channel and state entry, S per
+//                      channel) or the Mamba-2 layout (A and S per head)
 //
 // Both are tiny next to the prefill (B*D*L reads of dt; 3 * B*D*N floats),
 // HBM-bound, and run once per piece.
@@ -42,15 +44,19 @@ __global__ void __launch_bounds__(256) delta_sum_kernel(const DeltaSumProblem p)
 }
 
 __global__ void __launch_bounds__(256) carry_fold_kernel(const CarryFoldProblem p) {
-    const int64_t total = p.Bn * p.D * p.N;
+    const int64_t total = p.Bn * p.H * p.P * p.N;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
          i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t n = i % p.N, bd = i / p.N;
-        const int64_t d = bd % p.D, b = bd / p.D;
-        const float a = p.A[d * p.A_d + n * p.A_n] * kLog2e;
-        const float S = p.S[b * p.S_b + d * p.S_d];
-        float* st = p.state + b * p.s_b + d * p.s_d + n * p.s_n;
-        *st = fmaf(ex2_approx(a * S), *st, p.h_end[b * p.h_b + d * p.h_d + n * p.h_n]);
+        int64_t r = i;
+        const int64_t n = r % p.N;
+        r /= p.N;
+        const int64_t pp = r % p.P;
+        r /= p.P;
+        const int64_t h = r % p.H, b = r / p.H;
+        const float a = p.A[h * p.A_h + pp * p.A_p + n * p.A_n] * kLog2e;
+        const float S = p.S[b * p.S_b + h * p.S_h];
+        float* st = p.state + b * p.s_b + h * p.s_h + pp * p.s_p + n * p.s_n;
+        *st = fmaf(ex2_approx(a * S), *st, p.h_end[b * p.h_b + h * p.h_h + pp * p.h_p + n * p.h_n]);
     }
 }
 

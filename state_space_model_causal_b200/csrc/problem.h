@@ -187,14 +187,15 @@ struct DeltaSumProblem {
     float* out; int64_t o_b, o_d;
 };
 
-// State entering the next sequence piece: state, h_end (Bn, D, N); A (D, N);
-// S (Bn, D); all f32, any strides.
+// State entering the next sequence piece: state, h_end (Bn, H, P, N); A
+// indexed (H, P, N) by strides (Mamba-1 layout: H channels, P = 1; Mamba-2
+// layout: A per head, strides 0 over P and N); S (Bn, H); all f32.
 struct CarryFoldProblem {
-    int64_t Bn, D, N;
-    float* state; int64_t s_b, s_d, s_n;
-    const float* A; int64_t A_d, A_n;
-    const float* S; int64_t S_b, S_d;
-    const float* h_end; int64_t h_b, h_d, h_n;
+    int64_t Bn, H, P, N;
+    float* state; int64_t s_b, s_h, s_p, s_n;
+    const float* A; int64_t A_h, A_p, A_n;
+    const float* S; int64_t S_b, S_h;
+    const float* h_end; int64_t h_b, h_h, h_p, h_n;
 };
 
 struct Conv1dPlan {

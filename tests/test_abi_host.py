@@ -717,3 +717,19 @@ def test_carry_fold_plan_and_checks(lib):
                                                                   delta_sum=mem(F32, (0, 64)),
                                                                   h_end=mem(F32, (0, 64, 16))))
     assert st == OK and bd.KERNELS[info.kernel] == "none"
+
+
+def test_carry_fold_mamba2_layout_plan(lib):
+    """Rank-4 state (B, H, P, N) with A and the sums per head."""
+    mem = FakeMem()
+    a = carry_fold_args(mem, state=mem(F32, (2, 8, 64, 128)), A=mem(F32, (8,)), delta_sum=mem(F32, (2, 8)),
+                        h_end=mem(F32, (2, 8, 64, 128)))
+    st, info = call(lib, "ssm_scan_carry_fold", a)
+    assert st == OK and bd.KERNELS[info.kernel] == "carry_fold"
+    assert info.rows_per_item == 64 * 128 and info.work_items == 16
+    a = carry_fold_args(mem, state=mem(F32, (2, 8, 64, 128)), A=mem(F32, (8, 64)), delta_sum=mem(F32, (2, 8)),
+                        h_end=mem(F32, (2, 8, 64, 128)))
+    assert call(lib, "ssm_scan_carry_fold", a)[0] == ESHAPE
+    a = carry_fold_args(mem, state=mem(F32, (2, 8, 64)), A=mem(F32, (8,)), delta_sum=mem(F32, (2, 8)),
+                        h_end=mem(F32, (2, 8, 64)))
+    assert call(lib, "ssm_scan_carry_fold", a)[0] == ESHAPE  # rank 3 needs A (D, N)

@@ -163,3 +163,75 @@ def test_context_parallel_driver_with_emulated_ranks(io, lengths):
     assert_close(np.concatenate([res[0] for res in results], -1), ref, tol, "out")
     assert_close(results[-1][1], href, tol, "final ssm state")
     np.testing.assert_array_equal(results[-1][2], gen.round_to(csref, "f32"))
+
+
+def test_carry_fold_mamba2_layout_matches_oracle():
+    """Rank-4 state, A and the sums per head: the oracle's fold with A and S
+    repeated over the head's rows."""
+    import torch
+    from state_space_model_causal_b200 import ssm_scan_carry_fold
+    rng = np.random.default_rng(33)
+    st = gen.round_to(rng.standard_normal((2, 3, 8, 32)), "f32")
+    he = gen.round_to(rng.standard_normal((2, 3, 8, 32)), "f32")
+    A = gen.round_to(-rng.uniform(1.0, 16.0, 3), "f32")
+    S = gen.round_to(rng.uniform(0.0, 0.3, (2, 3)), "f32")
+    g = T(st, "f32")
+    ssm_scan_carry_fold(g, T(A, "f32"), T(S, "f32"), T(he, "f32"))
+    torch.cuda.synchronize()
+    rows = lambda a: a.reshape(2, 24, 32)  # noqa: E731
+    ref = oracle.carry_fold(rows(st), np.repeat(A, 8)[:, None].repeat(32, 1), np.repeat(S, 8, axis=1), rows(he))
+    assert_close(N(g).reshape(2, 24, 32), ref, 1e-5, "carry fold (Mamba-2 layout)")
+
+
+def _time_major(a, dtype, perm):
+    import torch  # noqa: F401
+    store = T(np.ascontiguousarray(np.transpose(a, perm)), dtype)
+    return store.permute(*[int(i) for i in np.argsort(perm)])
+
+
+@pytest.mark.parametrize("io,lengths", [("f16", (64, 48)), ("f32", (32, 40, 56))])
+def test_context_parallel_driver_mamba2_layout_with_emulated_ranks(io, lengths):
+    """The driver on Mamba-2-layout pieces (time-major rows, as the model
+    stores them), one host thread per rank on one GPU, against the oracle's
+    whole-sequence Mamba-2-layout prefill."""
+    import torch
+    from state_space_model_causal_b200.context_parallel import prefill_context_parallel
+    L = sum(lengths)
+    s = gen.scan_m2_inputs(2, 3, 64, 128, L, io=io, seed=34, tag="cpm2", h0=True)
+    ref, href = oracle.scan_mamba2(s.x, s.dt, s.A, s.B, s.C, D=s.D, z=s.z, dt_bias=s.dt_bias, h0=s.h0)
+    R = len(lengths)
+    bounds = np.cumsum((0,) + tuple(lengths))
+    shared = {"slots": [None] * R, "barrier": threading.Barrier(R, timeout=120)}
+    results, errors = [None] * R, []
+    dev = torch.device("cuda", 0)
+
+    def rank_main(r):
+        try:
+            torch.cuda.set_device(dev)
+            t0, t1 = int(bounds[r]), int(bounds[r + 1])
+            sl = lambda a: np.ascontiguousarray(a[..., t0:t1])  # noqa: E731
+            x = _time_major(sl(s.x), io, (0, 3, 1, 2))
+            z = _time_major(sl(s.z), io, (0, 3, 1, 2))
+            dt = _time_major(sl(s.dt), io, (0, 2, 1))
+            Bm = _time_major(sl(s.B), io, (0, 3, 1, 2))
+            Cm = _time_major(sl(s.C), io, (0, 3, 1, 2))
+            out = _time_major(np.zeros(x.shape), io, (0, 3, 1, 2))
+            h = T(s.h0, "f32") if r == 0 else torch.zeros(2, 3, 64, 128, device=dev)
+            prefill_context_parallel(x, dt, T(s.A, "f32"), Bm, Cm, D=T(s.D, "f32"), z=z,
+                                     dt_bias=T(s.dt_bias, "f32"), ssm_state=h, out=out,
+                                     comm=_ThreadComm(r, R, shared))
+            torch.cuda.synchronize()
+            results[r] = (N(out), N(h))
+        except Exception as e:
+            errors.append(repr(e))
+            shared["barrier"].abort()
+
+    threads = [threading.Thread(target=rank_main, args=(r,)) for r in range(R)]
+    for th in threads:
+        th.start()
+    for th in threads:
+        th.join(timeout=300)
+    assert not errors, errors
+    tol = 2 * (1e-5 if io == "f32" else TOL[io])
+    assert_close(np.concatenate([res[0] for res in results], -1), ref, tol, "out")
+    assert_close(results[-1][1], href, tol, "final ssm state")
