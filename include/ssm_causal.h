@@ -477,9 +477,12 @@ size_t ssm_struct_size(int which);
 /* The wait budget, in cycles, that a failure test's request of `cycles`
  * becomes: requests below 10^7 cycles are raised to 10^7.  Only the test
  * build of the library (libssm_causal_testhooks.so, compiled with
- * SSM_TEST_HOOKS) reads the failure-test switches SSM_TEST_DROP_ITEM and
- * SSM_TEST_WAIT_CYCLES from the environment; the product library ignores
- * them and always waits the full budget. */
+ * SSM_TEST_HOOKS) reads the failure-test switches from the environment:
+ * SSM_TEST_DROP_ITEM (a state-update work item whose copies are never
+ * started), SSM_TEST_DROP_WORKER (a prefill worker whose hand-over is never
+ * published) and SSM_TEST_WAIT_CYCLES (the budget of the waits they leave
+ * unanswered); the product library ignores them and always waits the full
+ * budget. */
 long long ssm_test_clamp_wait_budget(long long cycles);
 
 #ifdef __cplusplus

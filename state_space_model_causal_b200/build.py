@@ -29,7 +29,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libssm_causal.so")
 TEST_LIB = os.path.join(PKG, "libssm_causal_testhooks.so")
-TEST_HOOK_SOURCES = ("ssu.cu", "api.cpp")
+TEST_HOOK_SOURCES = ("ssu.cu", "scan_bal.cu", "api.cpp")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-I", INCLUDE,

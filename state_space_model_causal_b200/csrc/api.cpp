@@ -806,6 +806,16 @@ ssm_status scan_impl(const ssm_scan_args* a, cudaStream_t stream, uint64_t* ws_q
         if (grid > INT32_MAX) return SSM_ERR_UNSUPPORTED;
         bp.grid = (int)grid;
         bp.wait_budget = kWaitBudget;
+        bp.drop_worker = -1;
+#ifdef SSM_TEST_HOOKS
+        // Test build only: a worker whose hand-over is never published, and a
+        // shorter wait (never below kMinTestBudget cycles)
+        {
+            long long v = 0;
+            if (env_int("SSM_TEST_WAIT_CYCLES", &v) && v > 0) bp.wait_budget = clamp_test_budget(v);
+            if (env_int("SSM_TEST_DROP_WORKER", &v) && v >= 0) bp.drop_worker = v;
+        }
+#endif
         fill_info(a->info, SSM_KERNEL_SCAN_BAL, bp.grid, 32 * warps, smem, kch, bp.units);
         if (a->flags & SSM_FLAG_DRY_RUN) return SSM_OK;
         bp.err = device_error_ptr(dev);

@@ -117,6 +117,8 @@ struct BalPlan {
     float* ws_slots;     // one hand-over state per worker (16 x 16 floats)
     DeviceError* err;    // device error record
     long long wait_budget;  // cycles before a hand-over wait gives up
+    int64_t drop_worker;    // failure tests only: worker whose hand-over is never
+                            // published, so its successor's wait runs out (-1: none)
     // Context-parallel mode (cp_pieces >= 3): every sequence is cut into
     // cp_pieces pieces of piece_chunks chunks; a unit is (batch entry, channel
     // block, piece).  Pass 1 runs pieces 0..S-2 -- piece 0 from the initial

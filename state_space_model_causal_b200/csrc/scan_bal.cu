@@ -642,7 +642,12 @@ __global__ void __launch_bounds__(32 * kWarps, 2) scan_bal_kernel(const ScanProb
                 if (ph == 0) __stcg(slot + kCH * 16 + pc, sdl_ch);
                 __threadfence();
                 __syncwarp();
+#ifdef SSM_TEST_HOOKS
+                if (lane == 0 && (int64_t)w != bp.drop_worker)  // failure test: never published
+                    st_release_u32(bp.ws_flags + w, gen + 1u);
+#else
                 if (lane == 0) st_release_u32(bp.ws_flags + w, gen + 1u);
+#endif
             } else if (bp.cp_pass == 1) {
                 // the piece's end state and sum of delta, for pass 2
                 const int64_t rec = ub * (bp.cp_pieces - 1) + piece;

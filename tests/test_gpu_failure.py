@@ -117,3 +117,59 @@ def test_the_kernels_under_test_are_the_bulk_copy_ones():
                                T(s2.B, "f16"), T(s2.C, "f16"), D=T(s2.D, "f32"), dt_bias=T(s2.dt_bias, "f32"),
                                info=info)
     assert info.as_dict()["kernel"] == "ssu_tma" and info.work_items > 5
+
+
+def test_prefill_hand_over_wait_runs_out_and_is_reported():
+    """The balanced prefill: worker w never publishes the state it hands to
+    worker w + 1 (SSM_TEST_DROP_WORKER, test build only).  w + 1 gives up its
+    bounded wait, scans its piece of that unit from a zero state, and the
+    record names the prefill kernel and that unit; every other unit's outputs
+    are complete, and the next call without the switch matches the oracle.
+    The product library ignores the switch."""
+    import torch
+    from state_space_model_causal_b200 import (LaunchInfo, binding, ssm_device_error, ssm_device_error_info,
+                                               ssm_selective_scan_fwd)
+    from tests.parity import T, run_scan_oracle
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    Bt, L = 3, 72
+    units_wanted = sms * 2 * 4 + 29  # more 16-channel units than resident warps: slices hand over
+    D = 16 * -(-units_wanted // Bt)
+    s = gen.scan_inputs(Bt, L, D, 16, W=4, io="f16", seed=50, tag="dropworker", conv_state=True, h0=True)
+    ref, href, _ = run_scan_oracle(s)
+
+    def call():
+        info = LaunchInfo()
+        out = ssm_selective_scan_fwd(T(s.x, "f16"), T(s.dt, "f16"), T(s.A, "f32"), T(s.B, "f16"),
+                                     T(s.C, "f16"), D=T(s.D, "f32"), z=T(s.z, "f16"),
+                                     dt_bias=T(s.dt_bias, "f32"), conv_weight=T(s.conv_weight, "f32"),
+                                     conv_bias=T(s.conv_bias, "f32"), conv_state=T(s.conv_state, "f32"),
+                                     ssm_state=T(s.h0, "f32"), info=info)
+        torch.cuda.synchronize()
+        return N(out), info
+
+    out, info = call()  # product library: plan of the split
+    assert binding.KERNELS[info.kernel] == "scan_bal"
+    workers, units, nck = info.grid * 4, info.work_items, -(-L // 32)
+    total = units * nck
+    # a worker whose slice ends inside a unit: it hands that unit's state over
+    w = next(v for v in range(workers - 1) if ((v + 1) * total // workers) % nck != 0)
+    lost = ((w + 1) * total // workers) // nck  # the unit its successor continues
+    with binding.using_library(binding.TESTHOOKS_LIB_PATH):
+        assert ssm_device_error() == 0
+        with _env(SSM_TEST_DROP_WORKER=str(w), SSM_TEST_WAIT_CYCLES="20000000"):
+            out_d, _ = call()
+        rep = ssm_device_error_info()
+        assert rep == {"code": 1, "kernel": "scan_bal", "first_item": lost}, rep
+        assert ssm_device_error() == 0  # read and cleared
+        # every other unit (batch entry b, channels 16c .. 16c+15) is complete
+        nblk = D // 16
+        keep = np.ones((Bt, D), dtype=bool)
+        keep[lost // nblk, 16 * (lost % nblk):16 * (lost % nblk + 1)] = False
+        assert_close(out_d[keep], ref[keep], TOL["f16"], "outputs of the other units")
+        out_c, _ = call()  # the switch gone: complete again
+        assert_close(out_c, ref, TOL["f16"], "out after the failure")
+        assert ssm_device_error() == 0
+    with _env(SSM_TEST_DROP_WORKER=str(w), SSM_TEST_WAIT_CYCLES="20000000"):
+        out_p, _ = call()  # product library: the switch has no effect
+    assert_close(out_p, ref, TOL["f16"], "out (product library)")
+    assert ssm_device_error() == 0
