@@ -26,6 +26,10 @@ Functions (see the header comment of ``oracle.c`` for the definitions):
   piece, exp(A * sum delta) * h_in + h_end (the pieces of a context-parallel
   prefill; the long-context claim of "feat(llama.cu): 适配 mamba 模型" section
   6.1).
+* :func:`gated_conv1d` -- the double-gated short causal conv of the
+  "double-gated LIV convolution blocks" named in "LFM2.5-1.2B-Thinking性能优化
+  CUDA核心编程技巧" section 2.1, on the reading out = Cg * conv(Bg * x) (the
+  page prints no equation; see ``oracle.c``).
 * :func:`round_cache` -- a state rounded to its cache dtype (fp32, fp16, bf16;
   nearest, ties to even); :func:`ssu` and :func:`ssu_mamba2` apply it to the
   updated state when given ``cache_dtype``, after the step's readout has used
@@ -84,6 +88,8 @@ def configure(lib):
     lib.oracle_delta_sum.argtypes = [_i64] * 3 + [_dp] * 2 + [ctypes.c_int] + [_dp]
     lib.oracle_carry_fold.restype = ctypes.c_int
     lib.oracle_carry_fold.argtypes = [_i64] * 3 + [_dp] * 4
+    lib.oracle_gated_conv1d.restype = ctypes.c_int
+    lib.oracle_gated_conv1d.argtypes = [_i64] * 4 + [_dp] * 8
     return lib
 
 
@@ -331,3 +337,23 @@ def carry_fold(state, A, S, h_end):
     if lib.oracle_carry_fold(Bt, Dd, N, pA, pS, ph, st.ctypes.data_as(_dp)) != 0:
         raise ValueError("oracle_carry_fold rejected its arguments")
     return st
+
+
+def gated_conv1d(x, Bg, Cg, weight, bias=None, conv_state=None):
+    """out = Cg * (bias + causal conv of Bg * x).  x, Bg, Cg (B, D, L); weight
+    (D, W); bias (D); conv_state (B, D, W), the last W gated inputs before x.
+    Returns (out (B, D, L), conv_state_out (B, D, W))."""
+    lib = _load()
+    x_, px = _in(x)
+    B, D, L = x_.shape
+    _, pB = _in(Bg, (B, D, L))
+    _, pC = _in(Cg, (B, D, L))
+    w_, pw = _in(weight)
+    W = w_.shape[1]
+    _, pb = _in(bias, (D,)) if bias is not None else (None, None)
+    _, pcs = _in(conv_state, (B, D, W)) if conv_state is not None else (None, None)
+    out, po = _out((B, D, L))
+    cso, pcso = _out((B, D, W))
+    if lib.oracle_gated_conv1d(B, D, L, W, px, pB, pC, pw, pb, pcs, po, pcso) != 0:
+        raise ValueError("oracle_gated_conv1d rejected its arguments")
+    return out, cso

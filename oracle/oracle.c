@@ -391,3 +391,47 @@ int oracle_carry_fold(int64_t B, int64_t D, int64_t N, const double* A, const do
             }
     return 0;
 }
+
+/* ---------------------------------------------------------------------------
+ * Double-gated short causal conv: the convolution of the "double-gated LIV
+ * convolution blocks" that "LFM2.5-1.2B-Thinking性能优化CUDA核心编程技巧"
+ * (section 2.1) names next to the GQA blocks.  The page prints no equation;
+ * the reading taken here is the plainest one the name supports: two
+ * input-dependent multiplicative gates around a depthwise causal conv, one
+ * before it (Bg) and one after it (Cg), with no activation:
+ *
+ *   v[t]   = Bg[t] * x[t]
+ *   c[t]   = bias + sum_{k=0}^{W-1} w[k] * v[t-(W-1)+k]
+ *   out[t] = Cg[t] * c[t]
+ *
+ * v at t < 0 comes from the incoming conv_state, whose W entries are the last
+ * W gated inputs v, oldest first (zeros for a fresh sequence); conv_state_out
+ * holds the last W entries of (incoming state ++ v).
+ *
+ * Layouts: x, Bg, Cg, out (B, D, L); weight (D, W); bias (D);
+ * conv_state (B, D, W).
+ * ------------------------------------------------------------------------- */
+int oracle_gated_conv1d(int64_t B, int64_t D, int64_t L, int64_t W,
+                        const double* x, const double* Bg, const double* Cg,
+                        const double* weight, const double* bias, const double* conv_state_in,
+                        double* out, double* conv_state_out) {
+    int64_t b, d, t;
+    if (B < 0 || D < 0 || L < 0 || W < 1 || !x || !Bg || !Cg || !weight || !out) return -1;
+    double* v = (double*)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
+    double* c = (double*)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
+    for (b = 0; b < B; ++b) {
+        for (d = 0; d < D; ++d) {
+            const int64_t row = b * D + d;
+            /* the input gate */
+            for (t = 0; t < L; ++t) v[t] = Bg[row * L + t] * x[row * L + t];
+            /* the causal conv of the gated input, no activation */
+            o_conv_channel(L, W, conv_state_in ? conv_state_in + row * W : NULL, v, weight + d * W,
+                           bias ? bias[d] : 0.0, 0, c, conv_state_out ? conv_state_out + row * W : NULL);
+            /* the output gate */
+            for (t = 0; t < L; ++t) out[row * L + t] = Cg[row * L + t] * c[t];
+        }
+    }
+    free(v);
+    free(c);
+    return 0;
+}

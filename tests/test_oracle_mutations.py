@@ -81,6 +81,17 @@ MUTATIONS = [
      "state[i] = exp(A[d * N + n] * S[b * D + d]) * state[i];"),
     ("carry_fold_A_transposed", "state[i] = exp(A[d * N + n] * S[b * D + d]) * state[i] + h_end[i];",
      "state[i] = exp(A[n * D + d] * S[b * D + d]) * state[i] + h_end[i];"),
+    ("gated_conv_gates_swapped", "for (t = 0; t < L; ++t) v[t] = Bg[row * L + t] * x[row * L + t];",
+     "for (t = 0; t < L; ++t) v[t] = Cg[row * L + t] * x[row * L + t];"),
+    ("gated_conv_output_gate_dropped", "for (t = 0; t < L; ++t) out[row * L + t] = Cg[row * L + t] * c[t];",
+     "for (t = 0; t < L; ++t) out[row * L + t] = c[t];"),
+    ("gated_conv_input_gate_after_conv", "for (t = 0; t < L; ++t) v[t] = Bg[row * L + t] * x[row * L + t];",
+     "for (t = 0; t < L; ++t) v[t] = x[row * L + t];"),
+    ("gated_conv_bias_dropped", "bias ? bias[d] : 0.0, 0, c,", "0.0, 0, c,"),
+    ("gated_conv_output_gate_one_step_late", "out[row * L + t] = Cg[row * L + t] * c[t];",
+     "out[row * L + t] = Cg[row * L + (t > 0 ? t - 1 : 0)] * c[t];"),
+    ("gated_conv_state_ignored", "o_conv_channel(L, W, conv_state_in ? conv_state_in + row * W : NULL, v,",
+     "o_conv_channel(L, W, NULL, v,"),
 ]
 
 # pins exercised against each mutant (all cheap)
@@ -105,6 +116,8 @@ PIN_CALLS = [
     lambda: pins.test_round_cache_ties_go_to_even(),
     lambda: pins.test_delta_sum_is_the_decay_exponent_of_the_scan(True),
     lambda: pins.test_carry_fold_composes_sequence_pieces((3, 8)),
+    lambda: pins.test_gated_conv_matches_numpy_convolve_and_state(5, 3),
+    lambda: pins.test_gated_conv_impulse_response(3),
 ]
 
 

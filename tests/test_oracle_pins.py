@@ -506,3 +506,92 @@ def test_carry_fold_special_cases():
     np.testing.assert_array_equal(oracle.carry_fold(st, np.zeros((3, 4)), np.ones((2, 3)), he), st + he)
     np.testing.assert_array_equal(oracle.carry_fold(st, A, np.zeros((2, 3)), he), st + he)
     np.testing.assert_array_equal(oracle.carry_fold(st, A, np.full((2, 3), 1e6), he), he)
+
+
+# ---- double-gated short causal conv ("LFM2.5-1.2B-Thinking性能优化CUDA核心编程技巧"
+# section 2.1 names the block; the reading out = Cg * conv(Bg * x) is the oracle's)
+
+@pytest.mark.parametrize("L,W", [(0, 3), (1, 3), (2, 1), (3, 4), (5, 3), (9, 2), (11, 4)])
+def test_gated_conv_matches_numpy_convolve_and_state(L, W):
+    """The conv of the gated input through numpy.convolve, times the output
+    gate; the outgoing state is the last W gated inputs."""
+    Bt, Dd = 2, 3
+    x, bg, cg = (_rand((Bt, Dd, L), 40, n) for n in ("x", "bg", "cg"))
+    w = _rand((Dd, W), 40, "w")
+    b = _rand((Dd,), 40, "b")
+    cs = _rand((Bt, Dd, W), 40, "cs")
+    out, cso = oracle.gated_conv1d(x, bg, cg, w, bias=b, conv_state=cs)
+    for bb in range(Bt):
+        for d in range(Dd):
+            v = bg[bb, d] * x[bb, d]
+            np.testing.assert_allclose(out[bb, d], cg[bb, d] * _conv_ref(v, w[d], b[d], cs[bb, d]),
+                                       rtol=1e-13, atol=1e-14)
+            np.testing.assert_array_equal(cso[bb, d], np.concatenate([cs[bb, d], v])[-W:])
+
+
+def test_gated_conv_unit_gates_is_the_plain_conv():
+    x = _rand((2, 4, 13), 41, "x")
+    w, b = _rand((4, 3), 41, "w"), _rand((4,), 41, "b")
+    cs = _rand((2, 4, 3), 41, "cs")
+    one = np.ones_like(x)
+    out, cso = oracle.gated_conv1d(x, one, one, w, bias=b, conv_state=cs)
+    ref, csr = oracle.conv1d(x, w, bias=b, conv_state=cs, silu=False)
+    np.testing.assert_array_equal(out, ref)
+    np.testing.assert_array_equal(cso, csr)
+
+
+@pytest.mark.parametrize("W", [1, 3, 4])
+def test_gated_conv_impulse_response(W):
+    """x = impulse at t0: out[t0 + j] = Cg[t0 + j] * (bias + w[W-1-j] * Bg[t0])."""
+    L, t0 = 12, 3
+    x = np.zeros((1, 1, L))
+    x[0, 0, t0] = 1.0
+    bg, cg = _rand((1, 1, L), 42, "bg"), _rand((1, 1, L), 42, "cg")
+    w = _rand((1, W), 42, "w")
+    out, _ = oracle.gated_conv1d(x, bg, cg, w, bias=np.array([0.25]))
+    c = np.full(L, 0.25)
+    for j in range(W):
+        c[t0 + j] += w[0, W - 1 - j] * bg[0, 0, t0]
+    np.testing.assert_allclose(out[0, 0], cg[0, 0] * c, rtol=1e-15, atol=1e-16)
+
+
+def test_gated_conv_gates_act_before_and_after():
+    """Changing the input gate at step t moves outputs t .. t+W-1; changing the
+    output gate at step t moves output t alone; a zero input gate leaves
+    Cg * bias."""
+    L, W, t = 10, 4, 4
+    x, bg, cg = (_rand((1, 2, L), 43, n) for n in ("x", "bg", "cg"))
+    w, b = _rand((2, W), 43, "w"), _rand((2,), 43, "b")
+    out, _ = oracle.gated_conv1d(x, bg, cg, w, bias=b)
+    bg2 = bg.copy()
+    bg2[..., t] += 1.0
+    moved = np.abs(oracle.gated_conv1d(x, bg2, cg, w, bias=b)[0] - out) > 0
+    assert moved[..., t:t + W].all() and not moved[..., :t].any() and not moved[..., t + W:].any()
+    cg2 = cg.copy()
+    cg2[..., t] += 1.0
+    moved = np.abs(oracle.gated_conv1d(x, bg, cg2, w, bias=b)[0] - out) > 0
+    assert moved[..., t].all() and moved.sum() == 2
+    out0, cs0 = oracle.gated_conv1d(x, np.zeros_like(bg), cg, w, bias=b)
+    np.testing.assert_array_equal(out0, cg * b[None, :, None])
+    np.testing.assert_array_equal(cs0, np.zeros((1, 2, W)))
+
+
+@pytest.mark.parametrize("k", [0, 1, 3, 7, 12])
+def test_gated_conv_split_and_token_steps_equal_one_call(k):
+    """The sequence cut at k with the state carried, and token-by-token
+    decoding, equal one call over the whole sequence."""
+    L, W = 12, 3
+    x, bg, cg = (_rand((2, 3, L), 44, n) for n in ("x", "bg", "cg"))
+    w, b = _rand((3, W), 44, "w"), _rand((3,), 44, "b")
+    cs = _rand((2, 3, W), 44, "cs")
+    full, csf = oracle.gated_conv1d(x, bg, cg, w, bias=b, conv_state=cs)
+    o1, cs1 = oracle.gated_conv1d(x[..., :k], bg[..., :k], cg[..., :k], w, bias=b, conv_state=cs)
+    o2, cs2 = oracle.gated_conv1d(x[..., k:], bg[..., k:], cg[..., k:], w, bias=b, conv_state=cs1)
+    np.testing.assert_allclose(np.concatenate([o1, o2], -1), full, rtol=1e-14, atol=1e-15)
+    np.testing.assert_array_equal(cs2, csf)
+    st, steps = cs, []
+    for t in range(L):
+        o, st = oracle.gated_conv1d(x[..., t:t + 1], bg[..., t:t + 1], cg[..., t:t + 1], w, bias=b, conv_state=st)
+        steps.append(o)
+    np.testing.assert_allclose(np.concatenate(steps, -1), full, rtol=1e-14, atol=1e-15)
+    np.testing.assert_array_equal(st, csf)
