@@ -12,7 +12,8 @@ flushed before every step and only the kernel is inside each step's event
 pair.  The same line carries the decode updates (ssm_selective_state_update)
 measured in the same run: HBM GB/s and fraction of the measured copy peak for
 the Mamba-1 2.8B-shaped decode step (64 layer slabs) and the Mamba-2 layouts at
-their largest effective batch.
+their largest effective batch, and the double-gated short conv of an
+LFM2-style conv block (HBM GB/s).
 
 Multi-GPU: the work does not need an exchange between GPUs (every (b, d)
 recurrence is independent), so N ranks run independent replicas (weak
@@ -394,8 +395,67 @@ def prefill_single_sequence(dev, sfu_peak, hbm_peak, steps=20, warmup=3):
             "l2": "flushed (256 MiB write) before every step", "gpu_launches": 2 * steps}
 
 
+class GatedConv:
+    """The double-gated short conv of an LFM2-style conv block, B=4, L=2048,
+    D=2048, W=3, fp16: x and both gates are the three D-wide slices of one
+    token-major (B, L, 3D) projection output (drawn on the device), the output
+    is token-major (B, L, D), the conv state fp32."""
+
+    def __init__(self, dev, Bt=4, L=2048, D=2048, W=3):
+        import torch
+        from state_space_model_causal_b200 import inputs as gen
+        tag = ("bench", "gated_conv")
+        self.Bt, self.L, self.D, self.W = Bt, L, D, W
+        self.proj = gen.device_normal((Bt, L, 3 * D), "f16", *tag, "proj", device=dev)
+        self.bg, self.cg, self.x = (self.proj[:, :, i * D:(i + 1) * D].transpose(1, 2) for i in range(3))
+        self.w = gen.device_normal((D, W), "f32", *tag, "w", std=0.2, device=dev)
+        self.b = gen.device_normal((D,), "f32", *tag, "b", std=0.1, device=dev)
+        self.cs = torch.zeros(Bt, D, W, device=dev)
+        self.out = torch.empty(Bt, L, D, dtype=torch.float16, device=dev).transpose(1, 2)
+        self.elems = Bt * L * D
+
+    def algorithmic_bytes(self):
+        io = 4 * self.Bt * self.L * self.D * 2            # x, b_gate, c_gate in, out
+        params = self.D * (self.W + 1) * 4
+        state = self.Bt * self.D * (2 * self.W - 1) * 4   # W-1 entries read, W written
+        return io + params + state
+
+    def run(self):
+        from state_space_model_causal_b200 import ssm_gated_conv1d_fwd
+        ssm_gated_conv1d_fwd(self.x, self.bg, self.cg, self.w, bias=self.b, conv_state=self.cs, out=self.out)
+
+
+def gated_conv_lfm(dev, hbm_peak, steps=20, warmup=3):
+    """The double-gated conv: CUDA events per call, L2 flushed before each."""
+    import torch
+    gc = GatedConv(dev)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    ms = time_prefill(gc, steps, warmup, dev, flush)
+    mean = statistics.mean(ms)
+    alg = gc.algorithmic_bytes()
+    gbs = alg / (mean * 1e-3) / 1e9
+    traffic = profiled_traffic("gated_conv_lfm.txt", ["gconv.cu", "common.cuh"])
+    entry = {"workload": "double-gated short conv (LFM2-style conv block): B=4 L=2048 D=2048 W=3, fp16 "
+                         "x/gates (slices of one token-major projection), token-major out, fp32 state",
+             "us_per_call": round(mean * 1e3, 2), "Gelem_s": round(gc.elems / (mean * 1e-3) / 1e9, 1),
+             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+                          "frac": round(gbs / hbm_peak, 4), "traffic": traffic,
+                          "algorithmic_bytes_per_launch": alg},
+             "l2": "flushed (256 MiB write) before every step", "gpu_launches": steps}
+    del gc
+    torch.cuda.empty_cache()
+    return entry
+
+
+LEAD_CYCLES = 200_000  # ~0.1 ms of device time queued ahead of each timed call
+
+
 def time_prefill(pf, steps, warmup, dev, flush):
-    """Per-step CUDA events around the kernel only, L2 flushed before each step."""
+    """Per-step CUDA events around the kernel only, L2 flushed before each
+    step.  A short device-side sleep follows the flush, so that the host has
+    already queued the call (whose Python marshalling takes tens of
+    microseconds) when the start event fires: the pair then brackets device
+    work only, which matters for kernels of a few tens of microseconds."""
     import torch
     stream = torch.cuda.current_stream(dev)
     for _ in range(warmup):
@@ -406,6 +466,7 @@ def time_prefill(pf, steps, warmup, dev, flush):
           for _ in range(steps)]
     for a, b in ev:
         flush.zero_()
+        torch.cuda._sleep(LEAD_CYCLES)
         a.record(stream)
         pf.run()
         b.record(stream)
@@ -710,8 +771,8 @@ def oracle_prefill_sample(channels, seed=0):
 def oracle_beside(entry, kind, rows=None):
     """Time the fp64 oracle (one host thread) on a bounded sample of a sub-line's
     workload and express it in that line's unit, so that every measured kernel
-    has the oracle timed beside it.  kind: "m1_decode", "m2_decode" or
-    "m2_prefill"; rows overrides the sample size (tests)."""
+    has the oracle timed beside it.  kind: "m1_decode", "m2_decode",
+    "m2_prefill" or "gated_conv"; rows overrides the sample size (tests)."""
     import oracle
     from state_space_model_causal_b200 import inputs as gen
     if kind == "m1_decode":
@@ -735,6 +796,15 @@ def oracle_beside(entry, kind, rows=None):
         per_b = entry["bytes_per_call"] / entry["batch"]
         value, unit = Bt * per_b / dt / 1e9, "GB/s"
         sample = f"{Bt} batch rows x {H} heads, one decode step"
+    elif kind == "gated_conv":
+        Bt = rows or 1
+        s = gen.gated_conv_inputs(Bt, 2048, 2048, 3, io="f16", seed=0, tag="oracle_beside")
+        t0 = time.perf_counter()
+        oracle.gated_conv1d(s.x, s.bg, s.cg, s.weight, bias=s.bias)
+        dt = time.perf_counter() - t0
+        per_elem = entry["roofline"]["algorithmic_bytes_per_launch"] / (4 * 2048 * 2048)
+        value, unit = Bt * 2048 * 2048 * per_elem / dt / 1e9, "GB/s"
+        sample = f"{Bt} of the 4 batch entries, all 2048 channels, full L=2048"
     elif kind == "m2_prefill":
         heads = rows or 8
         s = gen.scan_m2_inputs(1, heads, 64, 128, 2048, io="f16", seed=0, tag="oracle_beside")
@@ -883,6 +953,9 @@ def run_only(args, dev):
     elif args.only == "prefill_m2":
         pm = PrefillM2(dev)
         fn = pm.run
+    elif args.only == "gated_conv":
+        gc = GatedConv(dev)
+        fn = gc.run
     elif args.only == "decode_m1":
         Bt, D, N, W = args.B, 5120, 16, 4  # default: two layers' worth of rows, 200 MB of state
         tag = ("only", "decode_m1")
@@ -940,7 +1013,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--only", choices=["prefill", "prefill_m2", "decode_m1", "m2_f16", "m2_f32",
-                                       "m2_bf16", "m2_f32_256"],
+                                       "m2_bf16", "m2_f32_256", "gated_conv"],
                     help="run --warmup then --steps launches of one case and exit "
                          "(for profiler captures; prints no JSON line)")
     ap.add_argument("--R", type=int, default=16384, help="effective batch for --only m2_*")
@@ -1020,6 +1093,7 @@ def main():
 
     prefill_m2 = prefill_mamba2(dev, hbm_peak, sm_max) if not args.no_decode else None
     prefill_b1 = prefill_single_sequence(dev, sfu_peak, hbm_peak) if not args.no_decode else None
+    gated_conv = gated_conv_lfm(dev, hbm_peak) if not args.no_decode else None
 
     decode = []
     if not args.no_decode:
@@ -1040,6 +1114,8 @@ def main():
                                                     + cpu["sample"])
         for i, entry in enumerate(decode):
             entry["oracle"] = oracle_beside(entry, "m1_decode" if i == 0 else "m2_decode")
+        if gated_conv:
+            gated_conv["oracle"] = oracle_beside(gated_conv, "gated_conv")
 
     if pg:
         pg.barrier()
@@ -1070,6 +1146,7 @@ def main():
                               "figure); the copy probe of bench.py --peaks is context"},
             "prefill_mamba2": prefill_m2,
             "prefill_one_sequence": prefill_b1,
+            "gated_conv": gated_conv,
             "decode": decode}
     print(json.dumps(line), flush=True)
     return 0

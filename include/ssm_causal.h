@@ -13,6 +13,10 @@
  *                               conv-state roll) and Mamba-2 layout (nheads x
  *                               headdim x dstate, scalar A per head, ngroups).
  *
+ * Beside them: ssm_scan_delta_sum and ssm_scan_carry_fold join a prefill split
+ * along the sequence, and ssm_gated_conv1d_fwd is the double-gated short causal
+ * conv of an LFM2-style conv block (prefill or one decode step).
+ *
  * Sources.  The operators "causal-conv1d, selective-scan, silu, element-mul"
  * and the Mamba state cache that is read and updated by capturing the conv and
  * scan operators come from "feat(llama.cu): 适配 mamba 模型" (InfiniLM-Rust PR
@@ -74,7 +78,7 @@
 extern "C" {
 #endif
 
-#define SSM_CAUSAL_ABI_VERSION 3
+#define SSM_CAUSAL_ABI_VERSION 4
 #define SSM_MAX_DIMS 5
 
 typedef enum ssm_dtype {
@@ -154,7 +158,10 @@ typedef enum ssm_kernel_id {
                                        workspace; d_state <= 16, conv width 0 or 4,
                                        time contiguous, L % 8 == 0, 16-byte aligned rows */
     SSM_KERNEL_DELTA_SUM = 14,      /* sum of a sequence piece's delta, warp per (b, d) */
-    SSM_KERNEL_CARRY_FOLD = 15      /* state entering the next sequence piece, elementwise */
+    SSM_KERNEL_CARRY_FOLD = 15,     /* state entering the next sequence piece, elementwise */
+    SSM_KERNEL_GATED_CONV = 16,     /* double-gated conv, 16-byte vectors of channels that
+                                       are contiguous in memory */
+    SSM_KERNEL_GATED_CONV_GENERIC = 17 /* double-gated conv, any strides */
 } ssm_kernel_id;
 
 /* ------------------------------------------------------------------------ *
@@ -359,6 +366,49 @@ ssm_status ssm_scan_delta_sum(const ssm_delta_sum_args* args, void* stream);
 ssm_status ssm_scan_carry_fold(const ssm_carry_fold_args* args, void* stream);
 
 /* ------------------------------------------------------------------------ *
+ * ssm_gated_conv1d_fwd -- double-gated short causal conv, the convolution of
+ * the "double-gated LIV convolution blocks" that "LFM2.5-1.2B-Thinking性能优化
+ * CUDA核心编程技巧" (section 2.1) names next to its GQA blocks.  The page
+ * prints no equation; the definition taken is two input-dependent gates
+ * around a depthwise causal conv, with no activation:
+ *
+ *   v[b,d,t]   = b_gate[b,d,t] * x[b,d,t]
+ *   out[b,d,t] = c_gate[b,d,t] * (bias[d] + sum_{k<W} weight[d,k] * v[b,d,t-(W-1)+k])
+ *
+ *   x, b_gate, c_gate (B, D, L)  f32 | f16 | bf16, one dtype   inputs
+ *   weight     (D, W)     f32, 1 <= W <= 8                      required
+ *   bias       (D)        f32                                   optional
+ *   conv_state (B, D, W)  f32 or x's dtype, in/out              optional:
+ *              read as the W gated inputs v preceding step 0 (oldest first),
+ *              then overwritten with the last W entries of (state ++ v).
+ *              Absent: zeros are used and nothing is written.
+ *   out        (B, D, L)  x's dtype                             output
+ *
+ * L = 1 with a conv state is one decode step.  L = 0 leaves the state
+ * unchanged.  Any strides; the fast kernel (SSM_KERNEL_GATED_CONV) takes the
+ * layout a token-major projection writes: x, b_gate, c_gate and out with unit
+ * channel stride, D a multiple of 8 (16-bit) or 4 (fp32), 16-byte aligned
+ * data pointers, and batch and step strides that keep every 16 bytes aligned
+ * (for example the three D-wide slices of one (B, L, 3D) projection output).
+ * Other layouts run on SSM_KERNEL_GATED_CONV_GENERIC.  out may not overlap an
+ * input or the state.
+ * ------------------------------------------------------------------------ */
+typedef struct ssm_gated_conv1d_args {
+    uint32_t struct_size; /* = sizeof(ssm_gated_conv1d_args) */
+    uint32_t flags;       /* SSM_FLAG_* */
+    ssm_tensor x;
+    ssm_tensor b_gate;
+    ssm_tensor c_gate;
+    ssm_tensor weight;
+    ssm_tensor bias;
+    ssm_tensor conv_state;
+    ssm_tensor out;
+    ssm_launch_info* info; /* optional */
+} ssm_gated_conv1d_args;
+
+ssm_status ssm_gated_conv1d_fwd(const ssm_gated_conv1d_args* args, void* stream);
+
+/* ------------------------------------------------------------------------ *
  * ssm_selective_state_update -- one decode token, caches updated in place.
  *
  * Mamba-1 layout (state rank 3):
@@ -471,7 +521,8 @@ int ssm_abi_version(void);
 /* sizeof() of the args structs and of ssm_tensor / ssm_launch_info /
  * ssm_device_error_report as compiled into the library, so that bindings can
  * check their layouts: which = 0 tensor, 1 conv1d args, 2 scan args, 3 ssu
- * args, 4 launch info, 5 error report, 6 delta-sum args, 7 carry-fold args. */
+ * args, 4 launch info, 5 error report, 6 delta-sum args, 7 carry-fold args,
+ * 8 gated-conv args. */
 size_t ssm_struct_size(int which);
 
 /* The wait budget, in cycles, that a failure test's request of `cycles`

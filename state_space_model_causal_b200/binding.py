@@ -7,11 +7,13 @@ one CUDA device; the call runs with that device current.  Every step of the comp
 CUDA kernels; there is no CPU or PyTorch fallback.  If the shared library is
 missing, importing the functions raises instead of degrading silently.
 
-The three entry points keep the C names:
+The entry points keep the C names:
 
 * :func:`ssm_causal_conv1d_fwd`
 * :func:`ssm_selective_scan_fwd`
 * :func:`ssm_selective_state_update`
+* :func:`ssm_scan_delta_sum`, :func:`ssm_scan_carry_fold` (sequence pieces)
+* :func:`ssm_gated_conv1d_fwd` (double-gated short causal conv)
 """
 from __future__ import annotations
 
@@ -38,6 +40,7 @@ KERNELS = {
     0: "none", 1: "conv1d", 2: "conv1d_generic", 3: "scan_chunked", 4: "scan_generic",
     5: "ssu_vec", 6: "ssu_generic", 7: "scan_vec", 8: "ssu_row", 9: "ssu_tma", 10: "ssu_row_tma",
     11: "scan_m2", 12: "scan_m2_generic", 13: "scan_bal", 14: "delta_sum", 15: "carry_fold",
+    16: "gated_conv", 17: "gated_conv_generic",
 }
 
 
@@ -112,6 +115,13 @@ class CarryFoldArgs(ctypes.Structure):
                 ("info", ctypes.POINTER(LaunchInfo))]
 
 
+class GatedConvArgs(ctypes.Structure):
+    _fields_ = [("struct_size", ctypes.c_uint32), ("flags", ctypes.c_uint32),
+                ("x", Tensor), ("b_gate", Tensor), ("c_gate", Tensor), ("weight", Tensor),
+                ("bias", Tensor), ("conv_state", Tensor), ("out", Tensor),
+                ("info", ctypes.POINTER(LaunchInfo))]
+
+
 _lock = threading.Lock()
 _lib = None
 _override = None  # a library swapped in by using_library() (failure tests)
@@ -158,7 +168,8 @@ def _open(path):
                        ("ssm_selective_scan_fwd", ScanArgs),
                        ("ssm_selective_state_update", SsuArgs),
                        ("ssm_scan_delta_sum", DeltaSumArgs),
-                       ("ssm_scan_carry_fold", CarryFoldArgs)):
+                       ("ssm_scan_carry_fold", CarryFoldArgs),
+                       ("ssm_gated_conv1d_fwd", GatedConvArgs)):
         fn = getattr(lib, name)
         fn.restype = ctypes.c_int
         fn.argtypes = [ctypes.POINTER(argt), ctypes.c_void_p]
@@ -179,7 +190,7 @@ def _open(path):
     lib.ssm_struct_size.restype = ctypes.c_size_t
     lib.ssm_struct_size.argtypes = [ctypes.c_int]
     for which, st in enumerate((Tensor, Conv1dArgs, ScanArgs, SsuArgs, LaunchInfo, ErrorReport,
-                                DeltaSumArgs, CarryFoldArgs)):
+                                DeltaSumArgs, CarryFoldArgs, GatedConvArgs)):
         if lib.ssm_struct_size(which) != ctypes.sizeof(st):
             raise ImportError(f"struct layout mismatch for {st.__name__}")
     return lib
@@ -467,6 +478,30 @@ def ssm_scan_carry_fold(state, A, delta_sum, h_end, stream=None, info: Optional[
     _check(_run(library().ssm_scan_carry_fold, a, (state, A, delta_sum, h_end), stream),
            "ssm_scan_carry_fold")
     return state
+
+
+def ssm_gated_conv1d_fwd(x, b_gate, c_gate, weight, bias=None, conv_state=None, out=None,
+                         stream=None, info: Optional[LaunchInfo] = None):
+    """Double-gated short causal conv: out = c_gate * (bias + causal conv of
+    b_gate * x) (see include/ssm_causal.h).  x, b_gate, c_gate (B, D, L);
+    weight (D, W) f32; bias (D); conv_state (B, D, W) in/out, the last W gated
+    inputs.  Without ``out``, the output takes x's layout: channels contiguous
+    (B, L, D storage) when x has unit channel stride, else (B, D, L).  Returns out."""
+    import torch
+    if out is None:
+        if x.dim() == 3 and x.stride(1) == 1 and x.shape[1] > 1:
+            out = torch.empty((x.shape[0], x.shape[2], x.shape[1]), dtype=x.dtype,
+                              device=x.device).transpose(1, 2)
+        else:
+            out = torch.empty(x.shape, dtype=x.dtype, device=x.device)
+    a = GatedConvArgs()
+    a.struct_size = ctypes.sizeof(GatedConvArgs)
+    a.x, a.b_gate, a.c_gate, a.weight, a.bias, a.conv_state, a.out = map(
+        describe, (x, b_gate, c_gate, weight, bias, conv_state, out))
+    a.info = _info_ptr(info)
+    _check(_run(library().ssm_gated_conv1d_fwd, a, (x, b_gate, c_gate, weight, bias, conv_state, out), stream),
+           "ssm_gated_conv1d_fwd")
+    return out
 
 
 def ssm_device_error(stream=None) -> int:

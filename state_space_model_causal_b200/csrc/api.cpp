@@ -394,6 +394,100 @@ ssm_status carry_fold_impl(const ssm_carry_fold_args* a, cudaStream_t stream) {
     return launch_carry_fold(p, (int)grid, kBlock, stream) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 
+// ------------------------------------------------------------ gated conv --
+ssm_status gated_conv_impl(const ssm_gated_conv1d_args* a, cudaStream_t stream) {
+    if (!a) return SSM_ERR_NULL;
+    if (a->struct_size != sizeof(ssm_gated_conv1d_args)) return SSM_ERR_VERSION;
+    SSM_TRY(info_ok(a->info));
+    SSM_TRY(basic(a->x));
+    SSM_TRY(basic(a->b_gate));
+    SSM_TRY(basic(a->c_gate));
+    SSM_TRY(basic(a->weight));
+    SSM_TRY(basic(a->out));
+    if (a->x.ndim != 3) return SSM_ERR_SHAPE;
+    const int64_t B = a->x.shape[0], D = a->x.shape[1], L = a->x.shape[2];
+    SSM_TRY(want(a->b_gate, {B, D, L}));
+    SSM_TRY(want(a->c_gate, {B, D, L}));
+    SSM_TRY(want(a->out, {B, D, L}));
+    if (a->weight.ndim != 2 || a->weight.shape[0] != D) return SSM_ERR_SHAPE;
+    const int64_t W = a->weight.shape[1];
+    if (W < 1) return SSM_ERR_SHAPE;
+    if (W > kMaxConvW) return SSM_ERR_UNSUPPORTED;
+    const int io = a->x.dtype;
+    if (!is_float(io) || a->b_gate.dtype != io || a->c_gate.dtype != io || a->out.dtype != io)
+        return SSM_ERR_DTYPE;
+    if (a->weight.dtype != SSM_F32) return SSM_ERR_DTYPE;
+    if (present(a->bias)) {
+        SSM_TRY(basic(a->bias));
+        SSM_TRY(want(a->bias, {D}));
+        if (a->bias.dtype != SSM_F32) return SSM_ERR_DTYPE;
+    }
+    const bool has_cs = present(a->conv_state);
+    if (has_cs) {
+        SSM_TRY(basic(a->conv_state));
+        SSM_TRY(want(a->conv_state, {B, D, W}));
+        if (a->conv_state.dtype != SSM_F32 && a->conv_state.dtype != io) return SSM_ERR_DTYPE;
+        if (!non_overlapping(a->conv_state)) return SSM_ERR_STRIDE;
+    }
+    if (!non_overlapping(a->out)) return SSM_ERR_STRIDE;
+    const ssm_tensor* ins[] = {&a->x, &a->b_gate, &a->c_gate, &a->weight, &a->bias};
+    for (const ssm_tensor* t : ins) {
+        if (overlap(a->out, *t)) return SSM_ERR_ALIAS;
+        if (has_cs && overlap(a->conv_state, *t)) return SSM_ERR_ALIAS;
+    }
+    if (has_cs && overlap(a->out, a->conv_state)) return SSM_ERR_ALIAS;
+    if (B * D == 0 || L == 0) {  // nothing to compute; a conv state stays as it is
+        fill_info(a->info, SSM_KERNEL_NONE, 0, 0, 0, 0, 0);
+        return SSM_OK;
+    }
+
+    // the vector kernel: 16-byte vectors of V channels with unit channel stride
+    const int es = esize(io);
+    const int V = 16 / es;
+    bool vec = D % V == 0;
+    const ssm_tensor* io_t[] = {&a->x, &a->b_gate, &a->c_gate, &a->out};
+    for (const ssm_tensor* t : io_t) {
+        vec = vec && t->stride[1] == 1 && aligned16(t->data) && (sd(*t, 0) * es) % 16 == 0 &&
+              (sd(*t, 2) * es) % 16 == 0;
+    }
+    const int64_t nv = vec ? D / V : D;
+    // segments of S >= 8 steps (so >= W - 1): as many as make one wave of the
+    // vector kernel (2 CTAs of 256 threads per SM), or about 1024 threads per
+    // SM for the generic one
+    const bool dry = (a->flags & SSM_FLAG_DRY_RUN) != 0;
+    const int block = gated_conv_block();
+    const int64_t wave = (int64_t)sm_count(dry) * (vec ? gated_conv_ctas_per_sm() * block : 1024);
+    int64_t nseg = std::min<int64_t>(std::max<int64_t>((wave + B * nv - 1) / (B * nv), 1), (L + 7) / 8);
+    int64_t S = L;
+    if (nseg > 1) {
+        S = (L + nseg - 1) / nseg;
+        nseg = (L + S - 1) / S;
+    }
+    const int64_t threads = B * nv * nseg;
+    const int64_t grid = (threads + block - 1) / block;
+    if (grid > INT32_MAX) return SSM_ERR_UNSUPPORTED;
+    const int kernel = vec ? SSM_KERNEL_GATED_CONV : SSM_KERNEL_GATED_CONV_GENERIC;
+    fill_info(a->info, kernel, (int)grid, block, vec ? gated_conv_ring_smem_bytes() : 0, vec ? V : 1, threads);
+    if (dry) return SSM_OK;
+
+    GatedConvProblem p{};
+    p.Bn = B; p.D = D; p.L = L; p.W = W; p.io_dt = io;
+    p.x = a->x.data; p.x_b = sd(a->x, 0); p.x_d = sd(a->x, 1); p.x_t = sd(a->x, 2);
+    p.bg = a->b_gate.data; p.bg_b = sd(a->b_gate, 0); p.bg_d = sd(a->b_gate, 1); p.bg_t = sd(a->b_gate, 2);
+    p.cg = a->c_gate.data; p.cg_b = sd(a->c_gate, 0); p.cg_d = sd(a->c_gate, 1); p.cg_t = sd(a->c_gate, 2);
+    p.w = static_cast<const float*>(a->weight.data); p.w_d = sd(a->weight, 0); p.w_k = sd(a->weight, 1);
+    p.bias = static_cast<const float*>(a->bias.data);
+    p.b_d = present(a->bias) ? sd(a->bias, 0) : 0;
+    p.conv_state = a->conv_state.data;
+    if (has_cs) {
+        p.cs_dt = a->conv_state.dtype;
+        p.cs_b = sd(a->conv_state, 0); p.cs_d = sd(a->conv_state, 1); p.cs_k = sd(a->conv_state, 2);
+    }
+    p.out = a->out.data; p.o_b = sd(a->out, 0); p.o_d = sd(a->out, 1); p.o_t = sd(a->out, 2);
+    p.S = S; p.nseg = nseg;
+    return launch_gated_conv(p, kernel, (int)grid, block, stream) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
 // ------------------------------------------------------------- workspace --
 // Balanced prefill workspace: a 256-byte header (generation, finished-worker
 // count), one 32-bit flag per worker (rounded up to 256 bytes), then one
@@ -1333,6 +1427,10 @@ ssm_status ssm_scan_carry_fold(const ssm_carry_fold_args* args, void* stream) {
     return carry_fold_impl(args, static_cast<cudaStream_t>(stream));
 }
 
+ssm_status ssm_gated_conv1d_fwd(const ssm_gated_conv1d_args* args, void* stream) {
+    return gated_conv_impl(args, static_cast<cudaStream_t>(stream));
+}
+
 const char* ssm_status_string(int status) {
     switch (status) {
         case SSM_OK: return "SSM_OK";
@@ -1383,6 +1481,7 @@ size_t ssm_struct_size(int which) {
         case 5: return sizeof(ssm_device_error_report);
         case 6: return sizeof(ssm_delta_sum_args);
         case 7: return sizeof(ssm_carry_fold_args);
+        case 8: return sizeof(ssm_gated_conv1d_args);
         default: return 0;
     }
 }

@@ -179,6 +179,22 @@ struct Conv1dProblem {
     void* out; int64_t o_b, o_d, o_t;
 };
 
+// Double-gated short causal conv: x, bg, cg, out (Bn, D, L) any strides (the
+// vector kernel needs unit channel strides); the rows are cut into nseg
+// segments of S steps (S >= W - 1 when nseg > 1).
+struct GatedConvProblem {
+    int64_t Bn, D, L, W;
+    int io_dt;
+    const void* x;  int64_t x_b, x_d, x_t;
+    const void* bg; int64_t bg_b, bg_d, bg_t;
+    const void* cg; int64_t cg_b, cg_d, cg_t;
+    const float* w; int64_t w_d, w_k;
+    const float* bias; int64_t b_d;
+    void* conv_state; int cs_dt; int64_t cs_b, cs_d, cs_k;
+    void* out; int64_t o_b, o_d, o_t;
+    int64_t S, nseg;
+};
+
 // Sum of a sequence piece's delta: dt (Bn, D, L) any strides; out (Bn, D) f32.
 struct DeltaSumProblem {
     int64_t Bn, D, L;
@@ -229,6 +245,10 @@ int scan_vec_threads();
 int scan_vec_channels_per_cta();
 cudaError_t launch_scan_vec(const ScanProblem& p, int sw_pairs, cudaStream_t s);
 cudaError_t launch_conv1d(const Conv1dProblem& p, const Conv1dPlan& plan, cudaStream_t s);
+cudaError_t launch_gated_conv(const GatedConvProblem& p, int kernel, int grid, int block, cudaStream_t s);
+int gated_conv_ring_smem_bytes();  // dynamic shared memory of the vector kernel's CTA
+int gated_conv_ctas_per_sm();      // CTAs of the vector kernel resident per SM
+int gated_conv_block();            // threads per CTA of both kernels
 cudaError_t launch_delta_sum(const DeltaSumProblem& p, int grid, int block, cudaStream_t s);
 cudaError_t launch_carry_fold(const CarryFoldProblem& p, int grid, int block, cudaStream_t s);
 int scan_m2_rows_per_cta(int64_t N);

@@ -17,11 +17,15 @@ these seeded tensors stand in for them -- no dataset items, no weights):
   fp16 x/dt/z/B/C, one independent slab per layer.
 * ``mamba2_64x128`` H=80, P=64, N=128, G=1, fp16 inputs, fp16/fp32 state.
 * ``mamba2_128x256`` H=32, P=128, N=256, G=1, bf16 inputs, bf16/fp32 state.
+* ``gated_conv_lfm``  double-gated short conv: B=4, L=2048, D=2048, W=3, fp16
+  x and gates, fp32 weights and state (the LFM2.5 page gives only the model's
+  size; the width and the conv width are choices, stated as such).
 
 Distributions: x, z, B, C ~ N(0, 1); dt ~ U(-4, -1); dt_bias = the inverse of
 softplus applied to U(1e-3, 0.1), i.e. log(expm1(u)); Mamba-1 A[d, n] = -(n+1);
 Mamba-2 A[h] = -U(1, 16); D = 1; conv weight ~ N(0, sigma=0.2), conv bias 0;
-states ~ N(0, 1) where a state is given.
+states ~ N(0, 1) where a state is given.  Gated conv: x and both gates ~ N(0, 1),
+weight ~ N(0, sigma=0.2), bias ~ N(0, sigma=0.1).
 """
 from __future__ import annotations
 
@@ -288,6 +292,37 @@ def mamba2_128x256(R, cache="bf16", seed=0) -> SsuInputs:
     Bt, Hr = effective_batch_shape(R, 32)
     return ssu_mamba2_inputs(Bt, Hr, 128, 256, io="bf16", state=cache, seed=seed,
                              tag=f"mamba2_128x256/R{R}")
+
+
+# --------------------------------------------------------------------------
+# double-gated short causal conv
+# --------------------------------------------------------------------------
+@dataclasses.dataclass
+class GatedConvInputs:
+    x: np.ndarray                     # (B, D, L)
+    bg: np.ndarray                    # (B, D, L) input gate
+    cg: np.ndarray                    # (B, D, L) output gate
+    weight: np.ndarray                # (D, W) fp32 values
+    bias: Optional[np.ndarray]        # (D,)
+    conv_state: Optional[np.ndarray]  # (B, D, W)
+    io: str
+
+
+def gated_conv_inputs(Bt, L, D, W, *, io="f16", seed=0, tag="gated_conv", bias=True,
+                      conv_state=False, state_dtype="f32") -> GatedConvInputs:
+    t = (seed, tag)
+    x = round_to(normal((Bt, D, L), *t, "x"), io)
+    bg = round_to(normal((Bt, D, L), *t, "bg"), io)
+    cg = round_to(normal((Bt, D, L), *t, "cg"), io)
+    w = round_to(normal((D, W), *t, "w", std=0.2), "f32")
+    b = round_to(normal((D,), *t, "b", std=0.1), "f32") if bias else None
+    cs = round_to(normal((Bt, D, W), *t, "conv_state"), state_dtype) if conv_state else None
+    return GatedConvInputs(x, bg, cg, w, b, cs, io)
+
+
+def gated_conv_lfm(seed=0, Bt=4, L=2048, D=2048, W=3) -> GatedConvInputs:
+    """The double-gated conv workload: fp16 x and gates, a 3-wide conv."""
+    return gated_conv_inputs(Bt, L, D, W, io="f16", seed=seed, tag="gated_conv_lfm")
 
 
 # --------------------------------------------------------------------------

@@ -35,7 +35,7 @@ def declared_functions():
 def test_header_declares_the_three_entry_points():
     fns = declared_functions()
     for name in ("ssm_causal_conv1d_fwd", "ssm_selective_scan_fwd", "ssm_selective_state_update",
-                 "ssm_scan_delta_sum", "ssm_scan_carry_fold",
+                 "ssm_scan_delta_sum", "ssm_scan_carry_fold", "ssm_gated_conv1d_fwd",
                  "ssm_status_string", "ssm_abi_version", "ssm_struct_size"):
         assert name in fns
 
@@ -46,9 +46,9 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_struct_layouts(lib):
-    assert lib.ssm_abi_version() == 3
+    assert lib.ssm_abi_version() == 4
     for which, st in enumerate((bd.Tensor, bd.Conv1dArgs, bd.ScanArgs, bd.SsuArgs, bd.LaunchInfo,
-                                bd.ErrorReport, bd.DeltaSumArgs, bd.CarryFoldArgs)):
+                                bd.ErrorReport, bd.DeltaSumArgs, bd.CarryFoldArgs, bd.GatedConvArgs)):
         assert lib.ssm_struct_size(which) == ctypes.sizeof(st)
     assert lib.ssm_struct_size(99) == 0
 
@@ -733,3 +733,88 @@ def test_carry_fold_mamba2_layout_plan(lib):
     a = carry_fold_args(mem, state=mem(F32, (2, 8, 64)), A=mem(F32, (8,)), delta_sum=mem(F32, (2, 8)),
                         h_end=mem(F32, (2, 8, 64)))
     assert call(lib, "ssm_scan_carry_fold", a)[0] == ESHAPE  # rank 3 needs A (D, N)
+
+
+# ------------------------------------------------------------- gated conv --
+def gconv_args(mem, Bn=4, D=2048, L=2048, W=3, io=F16, layout="tokens", **over):
+    """layout "tokens": x, b_gate, c_gate are the three D-wide slices of one
+    (B, L, 3D) projection output and out is (B, L, D) storage, all viewed as
+    (B, D, L); "rows": every tensor (B, D, L) contiguous."""
+    a = bd.GatedConvArgs()
+    a.struct_size = ctypes.sizeof(bd.GatedConvArgs)
+    a.flags = bd.SSM_FLAG_DRY_RUN
+    es = 4 if io == F32 else 2
+    if layout == "tokens":
+        proj = mem(io, (Bn, L, 3 * D))
+        st = (L * 3 * D, 1, 3 * D)
+        a.b_gate, a.c_gate, a.x = (bd.raw_tensor(proj.data + i * D * es, io, (Bn, D, L), st) for i in range(3))
+        a.out = mem(io, (Bn, D, L), (L * D, 1, D))
+    else:
+        a.x, a.b_gate, a.c_gate, a.out = (mem(io, (Bn, D, L)) for _ in range(4))
+    a.weight = mem(F32, (D, W))
+    a.bias = mem(F32, (D,))
+    a.conv_state = mem(F32, (Bn, D, W))
+    for k, v in over.items():
+        setattr(a, k, v)
+    return a
+
+
+def test_gated_conv_plan_token_major_layout(lib):
+    """The three slices of a (B, L, 3D) projection: 16-byte vectors of 8
+    channels; segments sized to one wave of 2 CTAs of 256 threads per SM
+    (4 x 256 vectors x 74 segments of 28 steps = 296 CTAs), a 96 KB ring of
+    8 steps x 3 vectors per thread."""
+    st, info = call(lib, "ssm_gated_conv1d_fwd", gconv_args(FakeMem()))
+    assert st == OK and bd.KERNELS[info.kernel] == "gated_conv"
+    assert info.block == 256 and info.rows_per_item == 8 and info.smem_bytes == 8 * 3 * 256 * 16
+    assert info.work_items == 4 * 256 * 74 and info.grid == 2 * 148
+    st, info = call(lib, "ssm_gated_conv1d_fwd", gconv_args(FakeMem(), io=F32))
+    assert st == OK and bd.KERNELS[info.kernel] == "gated_conv" and info.rows_per_item == 4
+    # one decode step: one segment of one step per vector
+    st, info = call(lib, "ssm_gated_conv1d_fwd", gconv_args(FakeMem(), Bn=245, L=1))
+    assert st == OK and bd.KERNELS[info.kernel] == "gated_conv" and info.work_items == 245 * 256
+    # a long, narrow problem keeps segments of at least 8 steps
+    st, info = call(lib, "ssm_gated_conv1d_fwd", gconv_args(FakeMem(), Bn=1, D=8, L=20))
+    assert st == OK and info.work_items == 3
+
+
+def test_gated_conv_other_layouts_use_the_generic_kernel(lib):
+    m = FakeMem()
+    st, info = call(lib, "ssm_gated_conv1d_fwd", gconv_args(m, layout="rows"))
+    assert st == OK and bd.KERNELS[info.kernel] == "gated_conv_generic" and info.rows_per_item == 1
+    assert info.smem_bytes == 0
+    st, info = call(lib, "ssm_gated_conv1d_fwd", gconv_args(m, D=2044))  # D not a multiple of 8
+    assert st == OK and bd.KERNELS[info.kernel] == "gated_conv_generic"
+    a = gconv_args(m)
+    a.x = bd.raw_tensor(a.x.data + 2, F16, (4, 2048, 2048), (2048 * 3 * 2048, 1, 3 * 2048))  # 2-byte offset
+    st, info = call(lib, "ssm_gated_conv1d_fwd", a)
+    assert st == OK and bd.KERNELS[info.kernel] == "gated_conv_generic"
+
+
+def test_gated_conv_error_paths(lib):
+    fn = "ssm_gated_conv1d_fwd"
+    m = FakeMem()
+    assert lib.ssm_gated_conv1d_fwd(None, None) == ENULL
+    _expect(lib, fn, gconv_args(m, weight=bd.Tensor()), ENULL)
+    _expect(lib, fn, gconv_args(m, c_gate=bd.Tensor()), ENULL)
+    _expect(lib, fn, gconv_args(m, weight=m(F32, (2048, 9))), EUNSUP)
+    _expect(lib, fn, gconv_args(m, weight=m(F32, (2048, 0))), ESHAPE)
+    _expect(lib, fn, gconv_args(m, b_gate=m(F16, (4, 2048, 2047))), ESHAPE)
+    _expect(lib, fn, gconv_args(m, b_gate=m(BF16, (4, 2048, 2048))), EDTYPE)
+    _expect(lib, fn, gconv_args(m, out=m(F32, (4, 2048, 2048))), EDTYPE)
+    _expect(lib, fn, gconv_args(m, bias=m(F16, (2048,))), EDTYPE)
+    _expect(lib, fn, gconv_args(m, conv_state=m(F32, (4, 2048, 4))), ESHAPE)
+    _expect(lib, fn, gconv_args(m, conv_state=m(BF16, (4, 2048, 3))), EDTYPE)
+    a = gconv_args(m)
+    a.out = a.c_gate
+    _expect(lib, fn, a, EALIAS)
+    a = gconv_args(m)
+    a.conv_state = bd.raw_tensor(a.out.data, F32, (4, 2048, 3))
+    _expect(lib, fn, a, EALIAS)
+    a = gconv_args(m)
+    a.struct_size -= 8
+    _expect(lib, fn, a, EVER)
+    st, info = call(lib, fn, gconv_args(m, L=0))  # the state is left as it is
+    assert st == OK and bd.KERNELS[info.kernel] == "none"
+    st, info = call(lib, fn, gconv_args(m, Bn=0, conv_state=m(F32, (0, 2048, 3))))
+    assert st == OK and bd.KERNELS[info.kernel] == "none"
