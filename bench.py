@@ -343,7 +343,7 @@ def prefill_mamba2(dev, hbm_peak, sm_max, steps=20, warmup=3):
     """Mamba-2-layout prefill: CUDA events per step, L2 flushed before each."""
     import torch
     pm = PrefillM2(dev)
-    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    flush = L2Flush(dev)
     ms = time_prefill(pm, steps, warmup, dev, flush)
     mean = statistics.mean(ms)
     gel = pm.elems / (mean * 1e-3) / 1e9
@@ -368,7 +368,7 @@ def prefill_mamba2(dev, hbm_peak, sm_max, steps=20, warmup=3):
                          "frac_of_direct_form_bound": round(gel / fp32_peak_direct, 4),
                          "hbm_achieved_gbs": round(gbs, 1), "hbm_peak_gbs": hbm_peak,
                          "hbm_frac": round(gbs / hbm_peak, 4), "algorithmic_bytes_per_launch": alg},
-            "l2": "flushed (256 MiB write) before every step", "gpu_launches": steps}
+            "l2": "flushed before every step (256 MiB write, then a 256 MiB read of another buffer, so no dirty line is left to write back)", "gpu_launches": steps}
 
 
 def prefill_single_sequence(dev, sfu_peak, hbm_peak, steps=20, warmup=3):
@@ -378,7 +378,7 @@ def prefill_single_sequence(dev, sfu_peak, hbm_peak, steps=20, warmup=3):
     the composed states).  CUDA events per call, L2 flushed before each."""
     import torch
     pf = Prefill(dev, Bt=1)
-    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    flush = L2Flush(dev)
     ms = time_prefill(pf, steps, warmup, dev, flush)
     mean = statistics.mean(ms)
     gel = pf.elems / (mean * 1e-3) / 1e9
@@ -392,7 +392,7 @@ def prefill_single_sequence(dev, sfu_peak, hbm_peak, steps=20, warmup=3):
                          "unit": "Gelem/s", "frac": round(gel / sfu_peak, 4), "traffic": None,
                          "peak_kind": "SFU ex2 rate x 148 SMs x max SM clock (one exp per element)",
                          "hbm_achieved_gbs": round(alg / (mean * 1e-3) / 1e9, 1), "hbm_peak_gbs": hbm_peak},
-            "l2": "flushed (256 MiB write) before every step", "gpu_launches": 2 * steps}
+            "l2": "flushed before every step (256 MiB write, then a 256 MiB read of another buffer, so no dirty line is left to write back)", "gpu_launches": 2 * steps}
 
 
 class GatedConv:
@@ -429,7 +429,7 @@ def gated_conv_lfm(dev, hbm_peak, steps=20, warmup=3):
     """The double-gated conv: CUDA events per call, L2 flushed before each."""
     import torch
     gc = GatedConv(dev)
-    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    flush = L2Flush(dev)
     ms = time_prefill(gc, steps, warmup, dev, flush)
     mean = statistics.mean(ms)
     alg = gc.algorithmic_bytes()
@@ -441,13 +441,32 @@ def gated_conv_lfm(dev, hbm_peak, steps=20, warmup=3):
              "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
                           "frac": round(gbs / hbm_peak, 4), "traffic": traffic,
                           "algorithmic_bytes_per_launch": alg},
-             "l2": "flushed (256 MiB write) before every step", "gpu_launches": steps}
+             "l2": "flushed before every step (256 MiB write, then a 256 MiB read of another buffer, so no dirty line is left to write back)", "gpu_launches": steps}
     del gc
     torch.cuda.empty_cache()
     return entry
 
 
 LEAD_CYCLES = 200_000  # ~0.1 ms of device time queued ahead of each timed call
+
+
+class L2Flush:
+    """Empties L2 between timed steps: writes a buffer twice the L2 size,
+    then reads another one as large.  The read evicts the dirty lines of the
+    write (and of the previous step's outputs) before the timed call starts,
+    so the call neither finds its inputs in L2 nor pays for write-backs that
+    are not its own."""
+
+    def __init__(self, dev):
+        import torch
+        self.w = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+        self.r = torch.zeros(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+        self.out = torch.empty((), dtype=torch.float32, device=dev)
+
+    def __call__(self):
+        import torch
+        self.w.zero_()
+        torch.sum(self.r, 0, out=self.out)
 
 
 def time_prefill(pf, steps, warmup, dev, flush):
@@ -459,13 +478,13 @@ def time_prefill(pf, steps, warmup, dev, flush):
     import torch
     stream = torch.cuda.current_stream(dev)
     for _ in range(warmup):
-        flush.zero_()
+        flush()
         pf.run()
     torch.cuda.synchronize(dev)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(steps)]
     for a, b in ev:
-        flush.zero_()
+        flush()
         torch.cuda._sleep(LEAD_CYCLES)
         a.record(stream)
         pf.run()
@@ -1055,7 +1074,7 @@ def main():
         return run_only(args, dev)
 
     pf = Prefill(dev)
-    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    flush = L2Flush(dev)
 
     if pg:
         pg.barrier()
@@ -1129,7 +1148,8 @@ def main():
             "config": {"workload": WORKLOAD, "global_batch": 4 * world, "seq_len": 2048,
                        "d_inner": 5120, "d_state": 16, "conv_width": 4, "io_dtype": "f16",
                        "parallelism": f"replicas x{world}",
-                       "l2": "flushed (256 MiB write) before every step; inputs 338 MB > 126 MB L2"},
+                       "l2": "flushed before every step (256 MiB write, then a 256 MiB read of another "
+                             "buffer, so no dirty line is left to write back); inputs 338 MB > 126 MB L2"},
             "roofline": roofline, "cpu_baseline": cpu,
             "e2e": {"value": round(e2e_val, 3), "unit": "Gelem/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_pipe_ms, 3),
