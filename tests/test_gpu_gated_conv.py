@@ -64,6 +64,22 @@ def test_gated_conv_matches_oracle(layout, io, Bt, L, D, W):
     np.testing.assert_array_equal(cs, gen.round_to(csref, "f32"))
 
 
+@pytest.mark.parametrize("io", ["f32", "f16", "bf16"])
+@pytest.mark.parametrize("Bt,L,W", [(2, 1, 3), (3, 5, 4), (1, 37, 3), (2, 300, 4), (2, 129, 1), (1, 64, 8),
+                                    (2, 2100, 3)])
+def test_gated_conv_whole_warp_rows_match_oracle(io, Bt, L, W):
+    """Rows of exactly 32 channel vectors (D = 256 at 16-bit, 128 at fp32),
+    so that every warp's threads share one (batch, segment) row; ragged
+    segment lengths, widths 1..8, an incoming state."""
+    D = 128 if io == "f32" else 256
+    s = gen.gated_conv_inputs(Bt, L, D, W, io=io, seed=7, tag=f"gcw/{L}/{W}", conv_state=True)
+    got, cs, kern = _run(s, "tokens")
+    assert kern == "gated_conv"
+    ref, csref = oracle.gated_conv1d(s.x, s.bg, s.cg, s.weight, bias=s.bias, conv_state=s.conv_state)
+    assert_close(got, ref, TOL[io], "out")
+    np.testing.assert_array_equal(cs, gen.round_to(csref, "f32"))
+
+
 @pytest.mark.parametrize("io", ["f16", "bf16"])
 def test_gated_conv_state_in_the_io_dtype_and_no_bias(io):
     s = gen.gated_conv_inputs(2, 50, 32, 3, io=io, seed=2, tag="gc/io_state", bias=False, conv_state=True,
@@ -84,12 +100,13 @@ def test_gated_conv_without_state_starts_from_zeros(layout):
     assert_close(got, ref, TOL["f16"], "out")
 
 
-def test_gated_conv_decode_steps_equal_one_prefill():
+@pytest.mark.parametrize("D", [64, 256])
+def test_gated_conv_decode_steps_equal_one_prefill(D):
     """Token-by-token calls (L = 1) through the conv state give the prefill's
     outputs and final state; each step also matches the oracle's step."""
     import torch
     from state_space_model_causal_b200 import ssm_gated_conv1d_fwd
-    Bt, L, D, W = 3, 12, 64, 3
+    Bt, L, W = 3, 12, 3
     s = gen.gated_conv_inputs(Bt, L, D, W, io="f16", seed=4, tag="gc/decode", conv_state=True)
     x, bg, cg, _, cs = _device(s, "tokens")
     w, b = T(s.weight, "f32"), T(s.bias, "f32")
