@@ -377,7 +377,20 @@ def prefill_single_sequence(dev, sfu_peak, hbm_peak, steps=20, warmup=3):
     call (pieces from zero states with carry records, then the re-scan from
     the composed states).  CUDA events per call, L2 flushed before each."""
     import torch
+    from state_space_model_causal_b200 import LaunchInfo, ssm_selective_scan_fwd
     pf = Prefill(dev, Bt=1)
+    # the plan: work_items = base units x (pieces - 1) per pass; pieces of
+    # ceil(chunks / pieces) 32-step chunks; pass 1 runs pieces 0 .. S-2 and
+    # pass 2 pieces 1 .. S-1, so per base unit (S-2) * piece + all chunks run
+    info = LaunchInfo()
+    ssm_selective_scan_fwd(pf.x, pf.dt, pf.A, pf.B, pf.C, D=pf.Dv, z=pf.z, dt_bias=pf.db,
+                           conv_weight=pf.cw, conv_bias=pf.cb, conv_state=pf.cs, ssm_state=pf.h,
+                           out=pf.out, info=info)
+    nck = -(-pf.L // 32)
+    base_units = pf.Bt * pf.D // 16
+    pieces = info.work_items // base_units + 1
+    piece = -(-nck // pieces)
+    work_factor = ((pieces - 2) * piece + nck) / nck
     flush = L2Flush(dev)
     ms = time_prefill(pf, steps, warmup, dev, flush)
     mean = statistics.mean(ms)
@@ -391,6 +404,8 @@ def prefill_single_sequence(dev, sfu_peak, hbm_peak, steps=20, warmup=3):
             "roofline": {"bound": "alu", "achieved": round(gel, 1), "peak": round(sfu_peak, 1),
                          "unit": "Gelem/s", "frac": round(gel / sfu_peak, 4), "traffic": None,
                          "peak_kind": "SFU ex2 rate x 148 SMs x max SM clock (one exp per element)",
+                         "pieces": pieces, "executed_work_factor": round(work_factor, 4),
+                         "frac_of_executed_work": round(gel * work_factor / sfu_peak, 4),
                          "hbm_achieved_gbs": round(alg / (mean * 1e-3) / 1e9, 1), "hbm_peak_gbs": hbm_peak},
             "l2": "flushed before every step (256 MiB write, then a 256 MiB read of another buffer, so no dirty line is left to write back)", "gpu_launches": 2 * steps}
 

@@ -457,7 +457,11 @@ ssm_status gated_conv_impl(const ssm_gated_conv1d_args* a, cudaStream_t stream) 
     const bool dry = (a->flags & SSM_FLAG_DRY_RUN) != 0;
     const int block = gated_conv_block();
     const int64_t wave = (int64_t)sm_count(dry) * (vec ? gated_conv_ctas_per_sm() * block : 1024);
-    int64_t nseg = std::min<int64_t>(std::max<int64_t>((wave + B * nv - 1) / (B * nv), 1), (L + 7) / 8);
+    // at most L / 8 segments, so that S = ceil(L / nseg) >= 8 >= W - 1: only the
+    // first segment of a row reads the incoming state, which its own thread
+    // then overwrites
+    int64_t nseg = std::min<int64_t>(std::max<int64_t>((wave + B * nv - 1) / (B * nv), 1),
+                                     std::max<int64_t>(L / 8, 1));
     int64_t S = L;
     if (nseg > 1) {
         S = (L + nseg - 1) / nseg;

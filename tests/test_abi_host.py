@@ -773,9 +773,11 @@ def test_gated_conv_plan_token_major_layout(lib):
     # one decode step: one segment of one step per vector
     st, info = call(lib, "ssm_gated_conv1d_fwd", gconv_args(FakeMem(), Bn=245, L=1))
     assert st == OK and bd.KERNELS[info.kernel] == "gated_conv" and info.work_items == 245 * 256
-    # a long, narrow problem keeps segments of at least 8 steps
-    st, info = call(lib, "ssm_gated_conv1d_fwd", gconv_args(FakeMem(), Bn=1, D=8, L=20))
-    assert st == OK and info.work_items == 3
+    # a long, narrow problem keeps segments of at least 8 steps (>= W - 1, so
+    # only a row's first segment reads the state it later overwrites)
+    for L, segs in ((20, 2), (17, 2), (15, 1), (8, 1), (64, 8), (65, 8)):
+        st, info = call(lib, "ssm_gated_conv1d_fwd", gconv_args(FakeMem(), Bn=1, D=8, L=L, W=8))
+        assert st == OK and info.work_items == segs, (L, info.work_items)
 
 
 def test_gated_conv_other_layouts_use_the_generic_kernel(lib):

@@ -51,7 +51,8 @@ KERNEL_OF = {"tokens": "gated_conv", "rows": "gated_conv_generic"}
 @pytest.mark.parametrize("layout", ["tokens", "rows"])
 @pytest.mark.parametrize("io", ["f32", "f16", "bf16"])
 @pytest.mark.parametrize("Bt,L,D,W", [(2, 1, 16, 3), (2, 5, 16, 4), (1, 37, 24, 3), (3, 300, 32, 4),
-                                      (2, 129, 8, 1), (1, 64, 16, 8), (2, 7, 16, 8)])
+                                      (2, 129, 8, 1), (1, 64, 16, 8), (2, 7, 16, 8), (1, 17, 8, 8),
+                                      (1, 23, 8, 8), (2, 65, 8, 7)])
 def test_gated_conv_matches_oracle(layout, io, Bt, L, D, W):
     """Ragged lengths, lengths below the conv width, widths 1..8, many
     segments per row (few channel vectors), with bias and an incoming state."""
