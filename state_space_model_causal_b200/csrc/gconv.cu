@@ -83,12 +83,13 @@ constexpr int kBlock = 256;     // threads per CTA
 constexpr int kP = 8;           // steps in flight per thread (vector kernel)
 constexpr int kCtasPerSm = 2;   // vector kernel: 96 KB of ring per CTA, <= 128 registers
 
-// any strides: one channel per thread (V = 1), or the vector layout without
-// the ring (V > 1, kept for the generic launcher's template)
-template <typename IoT, int V, int W>
+// any strides: one channel per thread, scalar loads, U steps of loads issued
+// together
+template <typename IoT, int W>
 __global__ void __launch_bounds__(kBlock) gconv_kernel(const GatedConvProblem p) {
+    constexpr int V = 1;
     using LN = Lane<IoT, V>;
-    constexpr int U = V == 1 ? 8 : 4;  // steps whose loads are issued together
+    constexpr int U = 8;
     const int64_t nv = p.D / V;
     const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= p.Bn * p.nseg * nv) return;
@@ -100,7 +101,6 @@ __global__ void __launch_bounds__(kBlock) gconv_kernel(const GatedConvProblem p)
     const int64_t t0 = seg * p.S;
     const int64_t t1 = t0 + p.S < p.L ? t0 + p.S : p.L;
 
-    // channel c of the vector sits at d0 + c (V > 1: unit channel stride)
     const int64_t xo = b * p.x_b + d0 * p.x_d, bo = b * p.bg_b + d0 * p.bg_d;
     const int64_t co = b * p.cg_b + d0 * p.cg_d, oo = b * p.o_b + d0 * p.o_d;
     const IoT* __restrict__ xp = static_cast<const IoT*>(p.x);
@@ -321,17 +321,17 @@ cudaError_t launch_ring(const GatedConvProblem& p, int grid, cudaStream_t s) {
     }
 }
 
-template <typename IoT, int V>
-cudaError_t launch_w(const GatedConvProblem& p, int grid, int block, cudaStream_t s) {
+template <typename IoT>
+cudaError_t launch_generic(const GatedConvProblem& p, int grid, int block, cudaStream_t s) {
     switch (p.W) {
-        case 1: gconv_kernel<IoT, V, 1><<<grid, block, 0, s>>>(p); break;
-        case 2: gconv_kernel<IoT, V, 2><<<grid, block, 0, s>>>(p); break;
-        case 3: gconv_kernel<IoT, V, 3><<<grid, block, 0, s>>>(p); break;
-        case 4: gconv_kernel<IoT, V, 4><<<grid, block, 0, s>>>(p); break;
-        case 5: gconv_kernel<IoT, V, 5><<<grid, block, 0, s>>>(p); break;
-        case 6: gconv_kernel<IoT, V, 6><<<grid, block, 0, s>>>(p); break;
-        case 7: gconv_kernel<IoT, V, 7><<<grid, block, 0, s>>>(p); break;
-        case 8: gconv_kernel<IoT, V, 8><<<grid, block, 0, s>>>(p); break;
+        case 1: gconv_kernel<IoT, 1><<<grid, block, 0, s>>>(p); break;
+        case 2: gconv_kernel<IoT, 2><<<grid, block, 0, s>>>(p); break;
+        case 3: gconv_kernel<IoT, 3><<<grid, block, 0, s>>>(p); break;
+        case 4: gconv_kernel<IoT, 4><<<grid, block, 0, s>>>(p); break;
+        case 5: gconv_kernel<IoT, 5><<<grid, block, 0, s>>>(p); break;
+        case 6: gconv_kernel<IoT, 6><<<grid, block, 0, s>>>(p); break;
+        case 7: gconv_kernel<IoT, 7><<<grid, block, 0, s>>>(p); break;
+        case 8: gconv_kernel<IoT, 8><<<grid, block, 0, s>>>(p); break;
         default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();
@@ -339,7 +339,7 @@ cudaError_t launch_w(const GatedConvProblem& p, int grid, int block, cudaStream_
 
 template <typename IoT>
 cudaError_t launch_io(const GatedConvProblem& p, bool vec, int grid, int block, cudaStream_t s) {
-    return vec ? launch_ring<IoT>(p, grid, s) : launch_w<IoT, 1>(p, grid, block, s);
+    return vec ? launch_ring<IoT>(p, grid, s) : launch_generic<IoT>(p, grid, block, s);
 }
 
 }  // namespace
