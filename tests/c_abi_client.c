@@ -99,6 +99,42 @@ int main(void) {
     printf("ssu %s kernel %d grid %d\n", ssm_status_string(st), info.kernel, info.grid);
     if (st != SSM_OK || info.kernel != SSM_KERNEL_SSU_TMA) ++fails;
 
+    /* double-gated short conv, token-major: x, b_gate, c_gate are the three
+       D-wide slices of one (B, L, 3D) projection output, out is (B, L, D) */
+    {
+        const int64_t Bn = 4, L = 2048, D = 2048, W = 3;
+        const int64_t proj_shape[3] = {Bn, L, 3 * D}, out_shape[3] = {Bn, L, D}, wshape[2] = {D, W},
+                      dshape[1] = {D}, csshape[3] = {Bn, D, W};
+        const ssm_tensor proj = dense(SSM_F16, 3, proj_shape), outs = dense(SSM_F16, 3, out_shape);
+        ssm_gated_conv1d_args g;
+        memset(&g, 0, sizeof g);
+        g.struct_size = sizeof g;
+        g.flags = SSM_FLAG_DRY_RUN;
+        ssm_tensor* views[3] = {&g.b_gate, &g.c_gate, &g.x};
+        for (int i = 0; i < 3; ++i) {
+            ssm_tensor v = proj;  /* (B, D, L) view: channel stride 1, step stride 3D */
+            v.data = (char*)proj.data + (size_t)(i * D) * 2;
+            v.shape[0] = Bn; v.shape[1] = D; v.shape[2] = L;
+            v.stride[0] = L * 3 * D; v.stride[1] = 1; v.stride[2] = 3 * D;
+            *views[i] = v;
+        }
+        g.out = outs;
+        g.out.shape[0] = Bn; g.out.shape[1] = D; g.out.shape[2] = L;
+        g.out.stride[0] = L * D; g.out.stride[1] = 1; g.out.stride[2] = D;
+        g.weight = dense(SSM_F32, 2, wshape);
+        g.bias = dense(SSM_F32, 1, dshape);
+        g.conv_state = dense(SSM_F32, 3, csshape);
+        memset(&info, 0, sizeof info);
+        info.struct_size = sizeof info;
+        g.info = &info;
+        st = ssm_gated_conv1d_fwd(&g, NULL);
+        printf("gated conv %s kernel %d grid %d\n", ssm_status_string(st), info.kernel, info.grid);
+        if (st != SSM_OK || info.kernel != SSM_KERNEL_GATED_CONV) ++fails;
+        if (ssm_struct_size(8) != sizeof(ssm_gated_conv1d_args)) ++fails;
+        g.out = g.x;  /* an output over an input */
+        if (ssm_gated_conv1d_fwd(&g, NULL) != SSM_ERR_ALIAS) ++fails;
+    }
+
     printf("fails %d\n", fails);
     return fails == 0 ? 0 : 1;
 }
