@@ -79,17 +79,18 @@ template <typename IoT> struct __align__(16) BalSmem {
     float bf[kT][16];     // B widened, [t][n]
     float cf[kT][16];     // C widened
     float4 dd[kCH / 2][kDdRow];  // (delta, delta*u) of channels 2cp and 2cp+1 per step
-    float4 yp[kT * kYpRow + 1];  // readout partials of the four lanes q per (step, channel)
+    float4 yp[kT * kYpRow + 4];  // readout partials of the four lanes q per (step, channel)
 };
 
 // (delta, delta*u) row of a channel pair: steps 16..31 sit one word further
 // on, so that the two prologue halves of a pair write distinct banks.
 __device__ __forceinline__ int dd_at(int t) { return t + (t >> 4); }
-// Readout partials of (step t, channel c): one row of kYpRow words per step,
-// channels 8..15 one word further on (the 32 lanes of a store hit 32 distinct
-// banks) and steps 16..31 one word further on (the epilogue's two halves read
-// distinct banks).
-__device__ __forceinline__ int yp_at(int t, int c) { return t * kYpRow + (t >> 4) + c + (c >> 3); }
+// Readout partials of (step t, channel c), one 16-byte word each: one row of
+// kYpRow words per step, channels 8..15 one word further on (the 32 lanes of
+// a store hit 32 distinct banks), and steps 16..31 four words further on, so
+// that the two halves of an epilogue quarter-warp (steps t and t + 16, four
+// channels each) read eight distinct 16-byte bank groups.
+__device__ __forceinline__ int yp_at(int t, int c) { return t * kYpRow + (t >> 4) * 4 + c + (c >> 3); }
 // Raw tiles hold 16-byte pieces of each row XOR-swizzled by row, so that the
 // pieces the prologue (and the B/C widening) read at once fall in distinct
 // banks: rows are 4 pieces (16-bit) or 8 pieces (fp32) long.
