@@ -926,8 +926,10 @@ def run_reference(args):
     cores = max(1, min(64, len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity")
                        else (os.cpu_count() or 1)))
     t, _ = oracle_prefill_sample(64)
-    # about 5 s of CPU work per step, over every host core
-    ch = max(64, min(4 * 5120, int(64 * cores * 5.0 / max(t, 1e-3))))
+    # up to 5 s of CPU work per step over every host core, less when there
+    # are many steps, so that the whole run stays near two and a half minutes
+    per_step_s = max(0.5, min(5.0, 150.0 / max(1, args.steps + args.warmup)))
+    ch = max(64, min(4 * 5120, int(64 * cores * per_step_s / max(t, 1e-3))))
     for _ in range(args.warmup):
         oracle_prefill_threads(ch, cores)
     times, elems = [], 0
