@@ -17,7 +17,10 @@ shapes:
     states reach no other channel's outputs or states;
   * a prefill cut into pieces scanned from zero states is recovered exactly
     by composing the pieces' carries and adding the decayed incoming state's
-    readout (the context-parallel decomposition), in both layouts.
+    readout (the context-parallel decomposition), in both layouts;
+  * the double-gated short conv: a split anywhere equals one call, the
+    output is linear in x for fixed gates, and it is causal with a window of
+    W steps for the input gate.
 """
 import numpy as np
 from hypothesis import given, settings
@@ -233,3 +236,54 @@ def test_mamba1_prefill_context_parallel_decomposition(Bt, D, N, L, R, W, seed):
         np.testing.assert_allclose(y0 + silu_z * carry, full[..., sl], rtol=1e-9, atol=1e-11)
         h_in = lam[..., -1] * h_in + h_r
     np.testing.assert_allclose(h_in, hfull, rtol=1e-9, atol=1e-11)
+
+
+# ---- double-gated short causal conv (reading: out = Cg * conv(Bg * x))
+@settings(**SETTINGS)
+@given(Bt=st.integers(1, 2), D=st.integers(1, 5), L=st.integers(2, 24), W=st.integers(1, 8),
+       frac=st.floats(0.05, 0.95), seed=st.integers(0, 10**6))
+def test_gated_conv_split_anywhere(Bt, D, L, W, frac, seed):
+    """A sequence cut anywhere, the conv state carried across, equals one call."""
+    split = max(1, min(L - 1, int(L * frac)))
+    s = gen.gated_conv_inputs(Bt, L, D, W, io="f32", seed=seed, tag="prop_gc", conv_state=True)
+    full, csf = oracle.gated_conv1d(s.x, s.bg, s.cg, s.weight, bias=s.bias, conv_state=s.conv_state)
+    a, b = slice(0, split), slice(split, L)
+    o1, cs1 = oracle.gated_conv1d(s.x[..., a], s.bg[..., a], s.cg[..., a], s.weight, bias=s.bias,
+                                  conv_state=s.conv_state)
+    o2, cs2 = oracle.gated_conv1d(s.x[..., b], s.bg[..., b], s.cg[..., b], s.weight, bias=s.bias, conv_state=cs1)
+    np.testing.assert_allclose(np.concatenate([o1, o2], -1), full, rtol=1e-13, atol=1e-14)
+    np.testing.assert_array_equal(cs2, csf)
+
+
+@settings(**SETTINGS)
+@given(D=st.integers(1, 5), L=st.integers(1, 16), W=st.integers(1, 6), alpha=st.floats(-3, 3),
+       seed=st.integers(0, 10**6))
+def test_gated_conv_linear_in_x_with_the_gates_fixed(D, L, W, alpha, seed):
+    """Without bias and state, x -> out is linear for fixed gates."""
+    s = gen.gated_conv_inputs(1, L, D, W, io="f32", seed=seed, tag="prop_gc_lin", bias=False)
+    x2 = gen.normal(s.x.shape, seed, "prop_gc_lin", "x2")
+    f = lambda x: oracle.gated_conv1d(x, s.bg, s.cg, s.weight)[0]  # noqa: E731
+    np.testing.assert_allclose(f(s.x + alpha * x2), f(s.x) + alpha * f(x2), rtol=1e-11, atol=1e-12)
+
+
+@settings(**SETTINGS)
+@given(Bt=st.integers(1, 2), D=st.integers(1, 4), L=st.integers(2, 16), W=st.integers(1, 8),
+       frac=st.floats(0.05, 0.95), seed=st.integers(0, 10**6))
+def test_gated_conv_is_causal_with_a_window_of_W(Bt, D, L, W, frac, seed):
+    """Changing x, Bg and Cg from step t on leaves outputs before t
+    bit-identical; changing only the input gate at step t moves outputs t ..
+    t+W-1 at most."""
+    t = max(1, min(L - 1, int(L * frac)))
+    s = gen.gated_conv_inputs(Bt, L, D, W, io="f32", seed=seed, tag="prop_gc_causal", conv_state=True)
+    base, _ = oracle.gated_conv1d(s.x, s.bg, s.cg, s.weight, bias=s.bias, conv_state=s.conv_state)
+    x2, bg2, cg2 = s.x.copy(), s.bg.copy(), s.cg.copy()
+    x2[..., t:] += 1.0
+    bg2[..., t:] -= 0.5
+    cg2[..., t:] *= 2.0
+    moved, _ = oracle.gated_conv1d(x2, bg2, cg2, s.weight, bias=s.bias, conv_state=s.conv_state)
+    np.testing.assert_array_equal(moved[..., :t], base[..., :t])
+    bg3 = s.bg.copy()
+    bg3[..., t] += 1.0
+    only, _ = oracle.gated_conv1d(s.x, bg3, s.cg, s.weight, bias=s.bias, conv_state=s.conv_state)
+    np.testing.assert_array_equal(only[..., :t], base[..., :t])
+    np.testing.assert_array_equal(only[..., t + W:], base[..., t + W:])
