@@ -45,6 +45,13 @@ def cases():
                 "(inputs.scan_m2_inputs(1, 2, 8, 64, 40, io='f32', seed=0, tag='golden', h0=True)); "
                 "out[0, h, p, :] for (h, p) = (0, 0), (1, 7), and the final state [0, 1, 3, :8]",
                 {"out": np.stack([y2[0, 0, 0], y2[0, 1, 7]]), "h_final": h2[0, 1, 3, :8][None]}))
+    g = gen.gated_conv_inputs(2, 24, 8, 3, io="f32", seed=0, tag="golden", conv_state=True)
+    yg, csg = oracle.gated_conv1d(g.x, g.bg, g.cg, g.weight, bias=g.bias, conv_state=g.conv_state)
+    out.append(("gated_conv_seed0.txt",
+                "double-gated short conv: B=2 L=24 D=8 W=3 fp32, seed 0, tag 'golden', incoming conv state "
+                "(inputs.gated_conv_inputs(2, 24, 8, 3, io='f32', seed=0, tag='golden', conv_state=True)); "
+                "out[b, d, :] for (b, d) = (0, 0), (1, 7), and the outgoing conv state [1, 3, :]",
+                {"out": np.stack([yg[0, 0], yg[1, 7]]), "conv_state": csg[1, 3][None]}))
     return out
 
 
