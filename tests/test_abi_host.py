@@ -816,6 +816,12 @@ def test_gated_conv_error_paths(lib):
     a = gconv_args(m)
     a.struct_size -= 8
     _expect(lib, fn, a, EVER)
+    # outputs and the in/out state may not broadcast (stride 0)
+    _expect(lib, fn, gconv_args(m, out=m(F16, (4, 2048, 2048), (2048 * 2048, 0, 2048))), ESTRIDE)
+    _expect(lib, fn, gconv_args(m, conv_state=m(F32, (4, 2048, 3), (3 * 2048, 3, 0))), ESTRIDE)
+    # inputs may: one gate shared by every batch entry
+    st, info = call(lib, fn, gconv_args(m, layout="rows", b_gate=m(F16, (4, 2048, 2048), (0, 2048, 1))))
+    assert st == OK and bd.KERNELS[info.kernel] == "gated_conv_generic"
     st, info = call(lib, fn, gconv_args(m, L=0))  # the state is left as it is
     assert st == OK and bd.KERNELS[info.kernel] == "none"
     st, info = call(lib, fn, gconv_args(m, Bn=0, conv_state=m(F32, (0, 2048, 3))))
