@@ -146,3 +146,20 @@ def test_gated_conv_empty_and_zero_length():
     torch.cuda.synchronize()
     assert binding.KERNELS[info.kernel] == "none"
     np.testing.assert_array_equal(N(cs), before)
+
+
+def test_gated_conv_input_gate_broadcast_over_the_batch():
+    """One input gate for every batch entry (batch stride 0), rows layout."""
+    import torch
+    from state_space_model_causal_b200 import ssm_gated_conv1d_fwd
+    s = gen.gated_conv_inputs(3, 40, 16, 4, io="f16", seed=8, tag="gc/bcast", conv_state=True)
+    bg1 = s.bg[:1]
+    bgt = T(bg1, "f16").expand(3, -1, -1)
+    cs = T(s.conv_state, "f32")
+    out = ssm_gated_conv1d_fwd(T(s.x, "f16"), bgt, T(s.cg, "f16"), T(s.weight, "f32"), bias=T(s.bias, "f32"),
+                               conv_state=cs)
+    torch.cuda.synchronize()
+    bg_full = np.broadcast_to(bg1, s.bg.shape)
+    ref, csref = oracle.gated_conv1d(s.x, bg_full, s.cg, s.weight, bias=s.bias, conv_state=s.conv_state)
+    assert_close(N(out), ref, TOL["f16"], "out")
+    np.testing.assert_array_equal(N(cs), gen.round_to(csref, "f32"))
