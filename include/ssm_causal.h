@@ -161,7 +161,9 @@ typedef enum ssm_kernel_id {
     SSM_KERNEL_CARRY_FOLD = 15,     /* state entering the next sequence piece, elementwise */
     SSM_KERNEL_GATED_CONV = 16,     /* double-gated conv, 16-byte vectors of channels that
                                        are contiguous in memory */
-    SSM_KERNEL_GATED_CONV_GENERIC = 17 /* double-gated conv, any strides */
+    SSM_KERNEL_GATED_CONV_GENERIC = 17, /* double-gated conv, any strides */
+    SSM_KERNEL_GATED_CONV_ROWS = 18 /* double-gated conv, (B, D, L) rows with contiguous time:
+                                       16-byte vectors of steps, history by shuffle */
 } ssm_kernel_id;
 
 /* ------------------------------------------------------------------------ *
@@ -390,7 +392,10 @@ ssm_status ssm_scan_carry_fold(const ssm_carry_fold_args* args, void* stream);
  * channel stride, D a multiple of 8 (16-bit) or 4 (fp32), 16-byte aligned
  * data pointers, and batch and step strides that keep every 16 bytes aligned
  * (for example the three D-wide slices of one (B, L, 3D) projection output).
- * Other layouts run on SSM_KERNEL_GATED_CONV_GENERIC.  out may not overlap an
+ * The time-contiguous layout ((B, D, L) rows with unit step stride, 16-byte
+ * aligned rows, L a multiple of 8 at 16-bit or 4 at fp32, W - 1 at most that
+ * multiple) runs on SSM_KERNEL_GATED_CONV_ROWS.  Other layouts run on
+ * SSM_KERNEL_GATED_CONV_GENERIC.  out may not overlap an
  * input or the state.
  * ------------------------------------------------------------------------ */
 typedef struct ssm_gated_conv1d_args {

@@ -40,7 +40,7 @@ KERNELS = {
     0: "none", 1: "conv1d", 2: "conv1d_generic", 3: "scan_chunked", 4: "scan_generic",
     5: "ssu_vec", 6: "ssu_generic", 7: "scan_vec", 8: "ssu_row", 9: "ssu_tma", 10: "ssu_row_tma",
     11: "scan_m2", 12: "scan_m2_generic", 13: "scan_bal", 14: "delta_sum", 15: "carry_fold",
-    16: "gated_conv", 17: "gated_conv_generic",
+    16: "gated_conv", 17: "gated_conv_generic", 18: "gated_conv_rows",
 }
 
 

@@ -450,6 +450,45 @@ ssm_status gated_conv_impl(const ssm_gated_conv1d_args* a, cudaStream_t stream) 
         vec = vec && t->stride[1] == 1 && aligned16(t->data) && (sd(*t, 0) * es) % 16 == 0 &&
               (sd(*t, 2) * es) % 16 == 0;
     }
+    // else the time-contiguous kernel: rows of L contiguous steps, 16-byte
+    // aligned, L a multiple of V, the history within one lane below
+    bool rows_vec = !vec && L % V == 0 && W - 1 <= V;
+    for (const ssm_tensor* t : io_t) {
+        rows_vec = rows_vec && t->stride[2] == 1 && aligned16(t->data) && (sd(*t, 0) * es) % 16 == 0 &&
+                   (sd(*t, 1) * es) % 16 == 0;
+    }
+    if (rows_vec) {
+        // one warp per (row, segment of whole 32-lane blocks), about 32 warps per SM
+        const bool dry_r = (a->flags & SSM_FLAG_DRY_RUN) != 0;
+        const int64_t rows = B * D, blk = 32 * (int64_t)V;
+        const int64_t want = (int64_t)sm_count(dry_r) * 32;
+        int64_t nseg = std::min<int64_t>(std::max<int64_t>((want + rows - 1) / rows, 1), (L + blk - 1) / blk);
+        int64_t S = ((L + nseg - 1) / nseg + blk - 1) / blk * blk;
+        nseg = (L + S - 1) / S;
+        const int block = gated_conv_block();
+        const int64_t warps = rows * nseg;
+        const int64_t grid = (warps + block / 32 - 1) / (block / 32);
+        if (grid > INT32_MAX) return SSM_ERR_UNSUPPORTED;
+        fill_info(a->info, SSM_KERNEL_GATED_CONV_ROWS, (int)grid, block, 0, 1, warps);
+        if (dry_r) return SSM_OK;
+        GatedConvProblem p{};
+        p.Bn = B; p.D = D; p.L = L; p.W = W; p.io_dt = io;
+        p.x = a->x.data; p.x_b = sd(a->x, 0); p.x_d = sd(a->x, 1); p.x_t = 1;
+        p.bg = a->b_gate.data; p.bg_b = sd(a->b_gate, 0); p.bg_d = sd(a->b_gate, 1); p.bg_t = 1;
+        p.cg = a->c_gate.data; p.cg_b = sd(a->c_gate, 0); p.cg_d = sd(a->c_gate, 1); p.cg_t = 1;
+        p.w = static_cast<const float*>(a->weight.data); p.w_d = sd(a->weight, 0); p.w_k = sd(a->weight, 1);
+        p.bias = static_cast<const float*>(a->bias.data);
+        p.b_d = present(a->bias) ? sd(a->bias, 0) : 0;
+        p.conv_state = a->conv_state.data;
+        if (has_cs) {
+            p.cs_dt = a->conv_state.dtype;
+            p.cs_b = sd(a->conv_state, 0); p.cs_d = sd(a->conv_state, 1); p.cs_k = sd(a->conv_state, 2);
+        }
+        p.out = a->out.data; p.o_b = sd(a->out, 0); p.o_d = sd(a->out, 1); p.o_t = 1;
+        p.S = S; p.nseg = nseg;
+        return launch_gated_conv(p, SSM_KERNEL_GATED_CONV_ROWS, (int)grid, block, stream) == cudaSuccess
+                   ? SSM_OK : SSM_ERR_CUDA;
+    }
     const int64_t nv = vec ? D / V : D;
     // segments of S >= 8 steps (so >= W - 1): as many as make one wave of the
     // vector kernel (2 CTAs of 256 threads per SM), or about 1024 threads per

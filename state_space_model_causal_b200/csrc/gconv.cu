@@ -33,6 +33,10 @@
 //     writes the outgoing state, after its reads, in ascending entry order:
 //     new entry k reads old entry L + k > k, so nothing it still needs is
 //     overwritten, and no other thread touches the state.
+//   * In the time-contiguous layout ((B, D, L) rows, as the Mamba tensors
+//     are laid out) a warp takes a segment of one row and a lane 16-byte
+//     vectors of consecutive steps, the history passed between lanes by
+//     shuffle (gconv_rows_kernel).
 //   * Any other layout runs a plain kernel (one channel per thread, scalar
 //     loads at any strides, U steps of loads issued together).
 #include "../../include/ssm_causal.h"
@@ -337,9 +341,130 @@ cudaError_t launch_generic(const GatedConvProblem& p, int grid, int block, cudaS
     return cudaGetLastError();
 }
 
+// the time-contiguous layout: x, b_gate, c_gate and out rows of L contiguous
+// steps (16-byte aligned, L a multiple of V).  A warp takes a segment of S
+// steps of one (b, d) row, a lane 16-byte vectors of V consecutive steps; the
+// W-1 gated inputs before a lane's first step come from the lane below by
+// shuffle (W - 1 <= V), before lane 0's from the previous block's lane 31, or
+// at the segment start from the row itself (or the incoming state).  The
+// next block's loads are issued before the current one is computed.
+template <typename IoT, int W>
+__global__ void __launch_bounds__(kBlock) gconv_rows_kernel(const GatedConvProblem p) {
+    constexpr int V = 16 / (int)sizeof(IoT);
+    constexpr int H = W > 1 ? W - 1 : 1;
+    static_assert(W - 1 <= V, "the history must come from one lane below");
+    using LN = Lane<IoT, V>;
+    const int lane = threadIdx.x & 31;
+    const int64_t gw = (int64_t)blockIdx.x * (kBlock / 32) + (threadIdx.x >> 5);
+    if (gw >= p.Bn * p.D * p.nseg) return;  // whole warps
+    const int64_t row = gw / p.nseg, seg = gw % p.nseg;
+    const int64_t b = row / p.D, d = row - b * p.D;
+    const int64_t t0 = seg * p.S;
+    const int64_t t1 = t0 + p.S < p.L ? t0 + p.S : p.L;
+    const IoT* __restrict__ xr = static_cast<const IoT*>(p.x) + b * p.x_b + d * p.x_d;
+    const IoT* __restrict__ br = static_cast<const IoT*>(p.bg) + b * p.bg_b + d * p.bg_d;
+    const IoT* __restrict__ cr = static_cast<const IoT*>(p.cg) + b * p.cg_b + d * p.cg_d;
+    IoT* __restrict__ orow = static_cast<IoT*>(p.out) + b * p.o_b + d * p.o_d;
+    const int64_t cs0 = b * p.cs_b + d * p.cs_d;
+
+    float w[W];
+#pragma unroll
+    for (int k = 0; k < W; ++k) w[k] = p.w[d * p.w_d + k * p.w_k];
+    const float bias = p.bias ? p.bias[d * p.b_d] : 0.0f;
+    // carry[i] = gated input at step (block start) - (W-1) + i
+    float carry[H];
+#pragma unroll
+    for (int i = 0; i < W - 1; ++i) {
+        const int64_t t = t0 - (W - 1) + i;
+        carry[i] = t >= 0 ? to_f(br[t]) * to_f(xr[t])
+                          : (p.conv_state ? ld_f(p.conv_state, cs0 + (W + t) * p.cs_k, p.cs_dt) : 0.0f);
+    }
+
+    uint4 nx = make_uint4(0, 0, 0, 0), nb = nx, nc = nx;
+    {
+        const int64_t t = t0 + lane * V;
+        if (t < t1) {
+            nx = LN::load(xr, t);
+            nb = LN::load(br, t);
+            nc = LN::load(cr, t);
+        }
+    }
+    for (int64_t tb = t0; tb < t1; tb += 32 * V) {
+        const int64_t t = tb + lane * V;
+        const bool valid = t < t1;
+        const uint4 cx = nx, cb = nb, cc = nc;
+        const int64_t tn = t + 32 * V;  // the next block, in flight while this one is computed
+        if (tn < t1) {
+            nx = LN::load(xr, tn);
+            nb = LN::load(br, tn);
+            nc = LN::load(cr, tn);
+        }
+        float xf[V], bf[V], cf[V], v[V], o[V];
+        LN::widen(cx, xf);
+        LN::widen(cb, bf);
+        LN::widen(cc, cf);
+#pragma unroll
+        for (int j = 0; j < V; ++j) v[j] = valid ? bf[j] * xf[j] : 0.0f;
+        float prev[H];
+#pragma unroll
+        for (int i = 0; i < W - 1; ++i) {
+            const float up = __shfl_up_sync(0xffffffffu, v[V - (W - 1) + i], 1);
+            prev[i] = lane == 0 ? carry[i] : up;
+        }
+#pragma unroll
+        for (int i = 0; i < W - 1; ++i) carry[i] = __shfl_sync(0xffffffffu, v[V - (W - 1) + i], 31);
+#pragma unroll
+        for (int j = 0; j < V; ++j) {
+            float acc = bias;
+#pragma unroll
+            for (int k = 0; k < W; ++k) {
+                const int idx = j - (W - 1) + k;
+                acc = fmaf(w[k], idx >= 0 ? v[idx] : prev[W - 1 + idx], acc);
+            }
+            o[j] = cf[j] * acc;
+        }
+        if (valid) LN::store(orow, t, o);
+    }
+
+    // outgoing state, by the first segment's warp: lane k < W computes entry k
+    // (the gated input at step L - W + k, or old entry L + k), all lanes read
+    // before any writes
+    if (p.conv_state && seg == 0) {
+        float nv = 0.0f;
+        if (lane < W) {
+            const int64_t t = p.L - W + lane;
+            nv = t >= 0 ? to_f(br[t]) * to_f(xr[t]) : ld_f(p.conv_state, cs0 + (p.L + lane) * p.cs_k, p.cs_dt);
+        }
+        __syncwarp();
+        if (lane < W) st_f(p.conv_state, cs0 + lane * p.cs_k, p.cs_dt, nv);
+    }
+}
+
 template <typename IoT>
-cudaError_t launch_io(const GatedConvProblem& p, bool vec, int grid, int block, cudaStream_t s) {
-    return vec ? launch_ring<IoT>(p, grid, s) : launch_generic<IoT>(p, grid, block, s);
+cudaError_t launch_rows(const GatedConvProblem& p, int grid, cudaStream_t s) {
+    constexpr int V = 16 / (int)sizeof(IoT);
+    switch (p.W) {
+        case 1: gconv_rows_kernel<IoT, 1><<<grid, kBlock, 0, s>>>(p); break;
+        case 2: gconv_rows_kernel<IoT, 2><<<grid, kBlock, 0, s>>>(p); break;
+        case 3: gconv_rows_kernel<IoT, 3><<<grid, kBlock, 0, s>>>(p); break;
+        case 4: gconv_rows_kernel<IoT, 4><<<grid, kBlock, 0, s>>>(p); break;
+        case 5: gconv_rows_kernel<IoT, 5><<<grid, kBlock, 0, s>>>(p); break;
+        case 6: if constexpr (V >= 5) { gconv_rows_kernel<IoT, (V >= 5 ? 6 : 1)><<<grid, kBlock, 0, s>>>(p); break; }
+                return cudaErrorInvalidValue;
+        case 7: if constexpr (V >= 6) { gconv_rows_kernel<IoT, (V >= 6 ? 7 : 1)><<<grid, kBlock, 0, s>>>(p); break; }
+                return cudaErrorInvalidValue;
+        case 8: if constexpr (V >= 7) { gconv_rows_kernel<IoT, (V >= 7 ? 8 : 1)><<<grid, kBlock, 0, s>>>(p); break; }
+                return cudaErrorInvalidValue;
+        default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+template <typename IoT>
+cudaError_t launch_io(const GatedConvProblem& p, int kernel, int grid, int block, cudaStream_t s) {
+    if (kernel == SSM_KERNEL_GATED_CONV) return launch_ring<IoT>(p, grid, s);
+    if (kernel == SSM_KERNEL_GATED_CONV_ROWS) return launch_rows<IoT>(p, grid, s);
+    return launch_generic<IoT>(p, grid, block, s);
 }
 
 }  // namespace
@@ -349,13 +474,14 @@ int gated_conv_ctas_per_sm() { return kCtasPerSm; }
 int gated_conv_block() { return kBlock; }
 
 cudaError_t launch_gated_conv(const GatedConvProblem& p, int kernel, int grid, int block, cudaStream_t s) {
-    const bool vec = kernel == SSM_KERNEL_GATED_CONV;
-    if (!vec && kernel != SSM_KERNEL_GATED_CONV_GENERIC) return cudaErrorInvalidValue;
+    if (kernel != SSM_KERNEL_GATED_CONV && kernel != SSM_KERNEL_GATED_CONV_ROWS &&
+        kernel != SSM_KERNEL_GATED_CONV_GENERIC)
+        return cudaErrorInvalidValue;
     if (block != kBlock) return cudaErrorInvalidValue;
     switch (p.io_dt) {
-        case kF32: return launch_io<float>(p, vec, grid, block, s);
-        case kF16: return launch_io<__half>(p, vec, grid, block, s);
-        case kBF16: return launch_io<__nv_bfloat16>(p, vec, grid, block, s);
+        case kF32: return launch_io<float>(p, kernel, grid, block, s);
+        case kF16: return launch_io<__half>(p, kernel, grid, block, s);
+        case kBF16: return launch_io<__nv_bfloat16>(p, kernel, grid, block, s);
         default: return cudaErrorInvalidValue;
     }
 }

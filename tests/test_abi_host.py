@@ -780,9 +780,26 @@ def test_gated_conv_plan_token_major_layout(lib):
         assert st == OK and info.work_items == segs, (L, info.work_items)
 
 
-def test_gated_conv_other_layouts_use_the_generic_kernel(lib):
+def test_gated_conv_time_contiguous_rows_plan(lib):
+    """(B, D, L) rows with unit step stride: one warp per (row, segment of
+    whole 256-step blocks), about 32 warps per SM (8192 rows: one segment)."""
     m = FakeMem()
     st, info = call(lib, "ssm_gated_conv1d_fwd", gconv_args(m, layout="rows"))
+    assert st == OK and bd.KERNELS[info.kernel] == "gated_conv_rows" and info.smem_bytes == 0
+    assert info.work_items == 4 * 2048 and info.grid == 4 * 2048 // 8 and info.block == 256
+    # few rows: segments of whole blocks (one row of 2048 steps -> 8 segments of 256)
+    st, info = call(lib, "ssm_gated_conv1d_fwd", gconv_args(m, layout="rows", Bn=1, D=1))
+    assert st == OK and bd.KERNELS[info.kernel] == "gated_conv_rows" and info.work_items == 8
+    # fp32: vectors of 4 steps, so W - 1 <= 4
+    st, info = call(lib, "ssm_gated_conv1d_fwd", gconv_args(m, layout="rows", io=F32, W=5))
+    assert st == OK and bd.KERNELS[info.kernel] == "gated_conv_rows"
+    st, info = call(lib, "ssm_gated_conv1d_fwd", gconv_args(m, layout="rows", io=F32, W=6))
+    assert st == OK and bd.KERNELS[info.kernel] == "gated_conv_generic"
+
+
+def test_gated_conv_other_layouts_use_the_generic_kernel(lib):
+    m = FakeMem()
+    st, info = call(lib, "ssm_gated_conv1d_fwd", gconv_args(m, layout="rows", L=2044))  # L not a multiple of 8
     assert st == OK and bd.KERNELS[info.kernel] == "gated_conv_generic" and info.rows_per_item == 1
     assert info.smem_bytes == 0
     st, info = call(lib, "ssm_gated_conv1d_fwd", gconv_args(m, D=2044))  # D not a multiple of 8
@@ -821,7 +838,7 @@ def test_gated_conv_error_paths(lib):
     _expect(lib, fn, gconv_args(m, conv_state=m(F32, (4, 2048, 3), (3 * 2048, 3, 0))), ESTRIDE)
     # inputs may: one gate shared by every batch entry
     st, info = call(lib, fn, gconv_args(m, layout="rows", b_gate=m(F16, (4, 2048, 2048), (0, 2048, 1))))
-    assert st == OK and bd.KERNELS[info.kernel] == "gated_conv_generic"
+    assert st == OK and bd.KERNELS[info.kernel] == "gated_conv_rows"
     st, info = call(lib, fn, gconv_args(m, L=0))  # the state is left as it is
     assert st == OK and bd.KERNELS[info.kernel] == "none"
     st, info = call(lib, fn, gconv_args(m, Bn=0, conv_state=m(F32, (0, 2048, 3))))

@@ -5,7 +5,8 @@ reading of the "double-gated LIV convolution blocks" of
 
 Both layouts: "tokens" (x, Bg, Cg the three D-wide slices of one (B, L, 3D)
 projection output, out (B, L, D) storage: the 16-byte vector kernel) and
-"rows" (every tensor (B, D, L): the generic kernel).  The outgoing conv state
+"rows" (every tensor (B, D, L): the time-contiguous kernel when L is a
+multiple of the vector width, else the generic one).  The outgoing conv state
 holds gated inputs, which are exact in fp32 for 16-bit inputs and correctly
 rounded for fp32 inputs, so it is compared bit for bit."""
 import numpy as np
@@ -45,7 +46,12 @@ def _run(s, layout, state_dtype="f32"):
     return N(out), N(cs), binding.KERNELS[info.kernel]
 
 
-KERNEL_OF = {"tokens": "gated_conv", "rows": "gated_conv_generic"}
+def expected_kernel(layout, io, L, W):
+    """The kernel the planner picks for contiguous test tensors."""
+    V = 4 if io == "f32" else 8
+    if layout == "tokens" or L == 1:
+        return "gated_conv"
+    return "gated_conv_rows" if L % V == 0 and W - 1 <= V else "gated_conv_generic"
 
 
 @pytest.mark.parametrize("layout", ["tokens", "rows"])
@@ -58,8 +64,7 @@ def test_gated_conv_matches_oracle(layout, io, Bt, L, D, W):
     segments per row (few channel vectors), with bias and an incoming state."""
     s = gen.gated_conv_inputs(Bt, L, D, W, io=io, seed=1, tag=f"gc/{L}/{D}/{W}", conv_state=True)
     got, cs, kern = _run(s, layout)
-    # at L = 1 the rows layout has unit channel stride too: the vector kernel
-    assert kern == ("gated_conv" if L == 1 else KERNEL_OF[layout])
+    assert kern == expected_kernel(layout, io, L, W)
     ref, csref = oracle.gated_conv1d(s.x, s.bg, s.cg, s.weight, bias=s.bias, conv_state=s.conv_state)
     assert_close(got, ref, TOL[io], "out")
     np.testing.assert_array_equal(cs, gen.round_to(csref, "f32"))
@@ -81,6 +86,21 @@ def test_gated_conv_whole_warp_rows_match_oracle(io, Bt, L, W):
     np.testing.assert_array_equal(cs, gen.round_to(csref, "f32"))
 
 
+@pytest.mark.parametrize("io", ["f32", "f16", "bf16"])
+@pytest.mark.parametrize("Bt,L,D,W", [(2, 256, 4, 3), (1, 264, 3, 4), (1, 2048, 2, 4), (3, 520, 5, 1),
+                                      (1, 8, 2, 5), (2, 776, 3, 8)])
+def test_gated_conv_time_contiguous_rows_match_oracle(io, Bt, L, D, W):
+    """(B, D, L) rows: one block of 256 steps exactly, a ragged last block,
+    rows cut into segments (few rows), L = 8, widths 1..8 (fp32 takes the
+    strided kernel above W = 5), with an incoming state."""
+    s = gen.gated_conv_inputs(Bt, L, D, W, io=io, seed=9, tag=f"gcr/{L}/{D}/{W}", conv_state=True)
+    got, cs, kern = _run(s, "rows")
+    assert kern == expected_kernel("rows", io, L, W)
+    ref, csref = oracle.gated_conv1d(s.x, s.bg, s.cg, s.weight, bias=s.bias, conv_state=s.conv_state)
+    assert_close(got, ref, TOL[io], "out")
+    np.testing.assert_array_equal(cs, gen.round_to(csref, "f32"))
+
+
 @pytest.mark.parametrize("io", ["f16", "bf16"])
 def test_gated_conv_state_in_the_io_dtype_and_no_bias(io):
     s = gen.gated_conv_inputs(2, 50, 32, 3, io=io, seed=2, tag="gc/io_state", bias=False, conv_state=True,
@@ -92,9 +112,9 @@ def test_gated_conv_state_in_the_io_dtype_and_no_bias(io):
     np.testing.assert_array_equal(cs, gen.round_to(csref, io))
 
 
-@pytest.mark.parametrize("layout", ["tokens", "rows"])
-def test_gated_conv_without_state_starts_from_zeros(layout):
-    s = gen.gated_conv_inputs(2, 40, 16, 4, io="f16", seed=3, tag="gc/nostate")
+@pytest.mark.parametrize("layout,L", [("tokens", 40), ("rows", 40), ("rows", 300)])
+def test_gated_conv_without_state_starts_from_zeros(layout, L):
+    s = gen.gated_conv_inputs(2, L, 16, 4, io="f16", seed=3, tag="gc/nostate")
     got, cs, _ = _run(s, layout)
     assert cs is None
     ref, _ = oracle.gated_conv1d(s.x, s.bg, s.cg, s.weight, bias=s.bias)
