@@ -130,8 +130,9 @@ typedef struct ssm_launch_info {
 
 typedef enum ssm_kernel_id {
     SSM_KERNEL_NONE = 0,            /* empty problem: nothing launched */
-    SSM_KERNEL_CONV1D = 1,          /* vectorised conv1d, L contiguous */
-    SSM_KERNEL_CONV1D_GENERIC = 2,  /* any strides */
+    SSM_KERNEL_CONV1D = 1,          /* conv1d, 16-byte vectors of steps: L contiguous, 16-byte aligned
+                                       rows, L a multiple of 8 (16-bit) or 4 (fp32), W - 1 at most that */
+    SSM_KERNEL_CONV1D_GENERIC = 2,  /* conv1d, any strides: a warp per row */
     SSM_KERNEL_SCAN_CHUNKED = 3,    /* fused prefill, smem-staged chunks of L */
     SSM_KERNEL_SCAN_GENERIC = 4,    /* fused prefill, any strides / group layout */
     SSM_KERNEL_SSU_VEC = 5,         /* 128-bit streaming state update, one decay per

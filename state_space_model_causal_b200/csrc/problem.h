@@ -220,6 +220,9 @@ struct Conv1dPlan {
     int kernel;
     int block;
     int grid;
+    int64_t seg_steps;  // vector kernel: steps per row segment (a multiple of 32 vectors)
+    int64_t nseg;       // vector kernel: segments per row
+    int depth;          // vector kernel: blocks of loads in flight ahead of the arithmetic (1 or 2)
 };
 
 cudaError_t launch_ssu(const SsuProblem& p, const SsuPlan& plan, cudaStream_t s);

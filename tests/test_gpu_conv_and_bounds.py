@@ -31,13 +31,94 @@ def test_conv1d_matches_oracle(io, L, W, silu):
     np.testing.assert_array_equal(N(csg), csref)
 
 
-def test_conv1d_without_state_and_full_size():
+def _conv_kernel(io, L, W):
+    """The kernel the planner picks for contiguous (B, D, L) tensors."""
+    V = 4 if io == "f32" else 8
+    return "conv1d" if L % V == 0 and W - 1 <= V else "conv1d_generic"
+
+
+@pytest.mark.parametrize("io", ["f32", "f16", "bf16"])
+@pytest.mark.parametrize("Bt,D,L,W", [(2, 3, 8, 4), (1, 2, 256, 4), (1, 2, 264, 4), (1, 1, 4096, 4),
+                                      (3, 5, 776, 1), (2, 3, 520, 5), (1, 4, 1032, 8), (2, 2, 2048, 7)])
+@pytest.mark.parametrize("silu", [False, True])
+def test_conv1d_vector_rows_match_oracle(io, Bt, D, L, W, silu):
+    """The 16-byte vector kernel: L = 8 (less than one block), one block of
+    256 steps exactly, a ragged last block, long rows cut into many segments
+    (few rows), widths 1..8 (fp32 takes the warp-per-row kernel above W = 5),
+    with an incoming state."""
+    import torch
+    from state_space_model_causal_b200 import LaunchInfo, binding, ssm_causal_conv1d_fwd
+    tag = ("convv", Bt, D, L, W)
+    x = gen.round_to(gen.normal((Bt, D, L), *tag, "x"), io)
+    w = gen.round_to(gen.normal((D, W), *tag, "w", std=0.2), "f32")
+    b = gen.round_to(gen.normal((D,), *tag, "b"), "f32")
+    cs = gen.round_to(gen.normal((Bt, D, W), *tag, "cs"), "f32")
+    csg = T(cs, "f32")
+    info = LaunchInfo()
+    out = ssm_causal_conv1d_fwd(T(x, io), T(w, "f32"), bias=T(b, "f32"), conv_state=csg, silu=silu, info=info)
+    torch.cuda.synchronize()
+    assert binding.KERNELS[info.kernel] == _conv_kernel(io, L, W)
+    ref, csref = oracle.conv1d(x, w, bias=b, conv_state=cs, silu=silu)
+    assert_close(N(out), ref, TOL[io], "out")
+    np.testing.assert_array_equal(N(csg), csref)
+
+
+@pytest.mark.parametrize("io", ["f16", "bf16"])
+def test_conv1d_vector_state_in_io_dtype_and_padded_rows(io):
+    """A conv state in the io dtype, no bias, and x / out rows that sit in a
+    wider (B, D, L + 16) buffer (aligned, not contiguous)."""
+    import torch
+    from state_space_model_causal_b200 import LaunchInfo, binding, ssm_causal_conv1d_fwd
+    Bt, D, L, W = 2, 7, 512, 4
+    x = gen.round_to(gen.normal((Bt, D, L), "convp", "x"), io)
+    w = gen.round_to(gen.normal((D, W), "convp", "w", std=0.2), "f32")
+    cs = gen.round_to(gen.normal((Bt, D, W), "convp", "cs"), io)
+    xb = torch.zeros((Bt, D, L + 16), dtype=T(x, io).dtype, device="cuda")
+    xb[:, :, :L] = T(x, io)
+    ob = torch.full_like(xb, 7.0)
+    csg = T(cs, io)
+    info = LaunchInfo()
+    ssm_causal_conv1d_fwd(xb[:, :, :L], T(w, "f32"), conv_state=csg, silu=True, out=ob[:, :, :L], info=info)
+    torch.cuda.synchronize()
+    assert binding.KERNELS[info.kernel] == "conv1d"
+    ref, csref = oracle.conv1d(x, w, conv_state=cs, silu=True)
+    assert_close(N(ob[:, :, :L]), ref, TOL[io], "out")
+    assert bool(torch.all(ob[:, :, L:] == 7.0))
+    np.testing.assert_array_equal(N(csg), gen.round_to(csref, io))
+
+
+def test_conv1d_vector_decode_after_prefill():
+    """A vector-kernel prefill's outgoing state feeds token-by-token calls
+    (the warp-per-row kernel at L = 1); together they equal one oracle call."""
     import torch
     from state_space_model_causal_b200 import ssm_causal_conv1d_fwd
-    s = gen.prefill_2p8b(seed=0)
-    out = ssm_causal_conv1d_fwd(T(s.x, "f16"), T(s.conv_weight, "f32"),
-                                bias=T(s.conv_bias, "f32"), silu=True)
+    Bt, D, L, W, extra = 2, 5, 256, 4, 6
+    x = gen.round_to(gen.normal((Bt, D, L + extra), "convd", "x"), "f16")
+    w = gen.round_to(gen.normal((D, W), "convd", "w", std=0.2), "f32")
+    cs = gen.round_to(gen.normal((Bt, D, W), "convd", "cs"), "f32")
+    csg = T(cs, "f32")
+    xt = T(x, "f16")
+    outs = [N(ssm_causal_conv1d_fwd(xt[:, :, :L].contiguous(), T(w, "f32"), conv_state=csg, silu=True))]
+    for t in range(L, L + extra):
+        outs.append(N(ssm_causal_conv1d_fwd(xt[:, :, t:t + 1].contiguous(), T(w, "f32"), conv_state=csg,
+                                            silu=True)))
     torch.cuda.synchronize()
+    ref, csref = oracle.conv1d(x, w, conv_state=cs, silu=True)
+    assert_close(np.concatenate(outs, -1), ref, TOL["f16"], "out")
+    np.testing.assert_array_equal(N(csg), csref)
+
+
+def test_conv1d_without_state_and_full_size():
+    """The 2.8B prefill's conv (B=4, D=5120, L=2048, W=4, fp16, SiLU) on the
+    vector kernel; 16 sampled rows against the oracle."""
+    import torch
+    from state_space_model_causal_b200 import LaunchInfo, binding, ssm_causal_conv1d_fwd
+    s = gen.prefill_2p8b(seed=0)
+    info = LaunchInfo()
+    out = ssm_causal_conv1d_fwd(T(s.x, "f16"), T(s.conv_weight, "f32"),
+                                bias=T(s.conv_bias, "f32"), silu=True, info=info)
+    torch.cuda.synchronize()
+    assert binding.KERNELS[info.kernel] == "conv1d"
     got = N(out)
     rng = np.random.default_rng(3)
     for b, d in zip(rng.integers(0, 4, 16), rng.integers(0, 5120, 16)):
