@@ -462,6 +462,56 @@ def gated_conv_lfm(dev, hbm_peak, steps=20, warmup=3):
     return entry
 
 
+class Conv1d:
+    """The standalone causal conv1d of one Mamba-1 2.8B layer: x (B=4,
+    D=5120, L=2048) fp16 time-contiguous, W=4, bias, SiLU, an fp32 conv state
+    read and written."""
+
+    def __init__(self, dev, Bt=4, D=5120, L=2048, W=4):
+        import torch
+        from state_space_model_causal_b200 import inputs as gen
+        tag = ("bench", "conv1d")
+        self.Bt, self.D, self.L, self.W = Bt, D, L, W
+        self.x = gen.device_normal((Bt, D, L), "f16", *tag, "x", device=dev)
+        self.w = gen.device_normal((D, W), "f32", *tag, "w", std=0.2, device=dev)
+        self.b = gen.device_normal((D,), "f32", *tag, "b", std=0.1, device=dev)
+        self.cs = gen.device_normal((Bt, D, W), "f32", *tag, "cs", device=dev)
+        self.out = torch.empty_like(self.x)
+        self.elems = Bt * D * L
+
+    def algorithmic_bytes(self):
+        io = 2 * self.Bt * self.D * self.L * 2            # x in, out
+        params = self.D * (self.W + 1) * 4
+        state = self.Bt * self.D * (2 * self.W - 1) * 4   # W-1 entries read, W written
+        return io + params + state
+
+    def run(self):
+        from state_space_model_causal_b200 import ssm_causal_conv1d_fwd
+        ssm_causal_conv1d_fwd(self.x, self.w, bias=self.b, conv_state=self.cs, silu=True, out=self.out)
+
+
+def conv1d_2p8b(dev, hbm_peak, steps=20, warmup=3):
+    """The standalone conv1d: CUDA events per call, L2 flushed before each."""
+    import torch
+    cv = Conv1d(dev)
+    flush = L2Flush(dev)
+    ms = time_prefill(cv, steps, warmup, dev, flush)
+    mean = statistics.mean(ms)
+    alg = cv.algorithmic_bytes()
+    gbs = alg / (mean * 1e-3) / 1e9
+    traffic = profiled_traffic("conv1d_2p8b.txt", ["conv1d.cu", "common.cuh"])
+    entry = {"workload": "mamba1-2.8b conv1d: B=4 D=5120 L=2048 W=4, fp16 time-contiguous x/out, bias, "
+                         "SiLU, fp32 conv state",
+             "us_per_call": round(mean * 1e3, 2), "Gelem_s": round(cv.elems / (mean * 1e-3) / 1e9, 1),
+             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+                          "frac": round(gbs / hbm_peak, 4), "traffic": traffic,
+                          "algorithmic_bytes_per_launch": alg},
+             "l2": "flushed before every step (256 MiB write, then a 256 MiB read of another buffer, so no dirty line is left to write back)", "gpu_launches": steps}
+    del cv
+    torch.cuda.empty_cache()
+    return entry
+
+
 LEAD_CYCLES = 200_000  # ~0.1 ms of device time queued ahead of each timed call
 
 
@@ -806,7 +856,8 @@ def oracle_beside(entry, kind, rows=None):
     """Time the fp64 oracle (one host thread) on a bounded sample of a sub-line's
     workload and express it in that line's unit, so that every measured kernel
     has the oracle timed beside it.  kind: "m1_decode", "m2_decode",
-    "m2_prefill" or "gated_conv"; rows overrides the sample size (tests)."""
+    "m2_prefill", "gated_conv" or "conv1d"; rows overrides the sample size
+    (tests)."""
     import oracle
     from state_space_model_causal_b200 import inputs as gen
     if kind == "m1_decode":
@@ -839,6 +890,18 @@ def oracle_beside(entry, kind, rows=None):
         per_elem = entry["roofline"]["algorithmic_bytes_per_launch"] / (4 * 2048 * 2048)
         value, unit = Bt * 2048 * 2048 * per_elem / dt / 1e9, "GB/s"
         sample = f"{Bt} of the 4 batch entries, all 2048 channels, full L=2048"
+    elif kind == "conv1d":
+        chans = rows or 5120
+        s = gen.normal((1, chans, 2048), "oracle_beside", "conv1d", "x")
+        w = gen.normal((chans, 4), "oracle_beside", "conv1d", "w", std=0.2)
+        b = gen.normal((chans,), "oracle_beside", "conv1d", "b", std=0.1)
+        cs = gen.normal((1, chans, 4), "oracle_beside", "conv1d", "cs")
+        t0 = time.perf_counter()
+        oracle.conv1d(s, w, bias=b, conv_state=cs, silu=True)
+        dt = time.perf_counter() - t0
+        per_elem = entry["roofline"]["algorithmic_bytes_per_launch"] / (4 * 5120 * 2048)
+        value, unit = chans * 2048 * per_elem / dt / 1e9, "GB/s"
+        sample = f"{chans} of the 20480 (b, d) rows, full L=2048"
     elif kind == "m2_prefill":
         heads = rows or 8
         s = gen.scan_m2_inputs(1, heads, 64, 128, 2048, io="f16", seed=0, tag="oracle_beside")
@@ -992,6 +1055,9 @@ def run_only(args, dev):
     elif args.only == "gated_conv":
         gc = GatedConv(dev)
         fn = gc.run
+    elif args.only == "conv1d":
+        cv = Conv1d(dev)
+        fn = cv.run
     elif args.only == "decode_m1":
         Bt, D, N, W = args.B, 5120, 16, 4  # default: two layers' worth of rows, 200 MB of state
         tag = ("only", "decode_m1")
@@ -1049,7 +1115,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--only", choices=["prefill", "prefill_m2", "decode_m1", "m2_f16", "m2_f32",
-                                       "m2_bf16", "m2_f32_256", "gated_conv"],
+                                       "m2_bf16", "m2_f32_256", "gated_conv", "conv1d"],
                     help="run --warmup then --steps launches of one case and exit "
                          "(for profiler captures; prints no JSON line)")
     ap.add_argument("--R", type=int, default=16384, help="effective batch for --only m2_*")
@@ -1130,6 +1196,7 @@ def main():
     prefill_m2 = prefill_mamba2(dev, hbm_peak, sm_max) if not args.no_decode else None
     prefill_b1 = prefill_single_sequence(dev, sfu_peak, hbm_peak) if not args.no_decode else None
     gated_conv = gated_conv_lfm(dev, hbm_peak) if not args.no_decode else None
+    conv1d = conv1d_2p8b(dev, hbm_peak) if not args.no_decode else None
 
     decode = []
     if not args.no_decode:
@@ -1152,6 +1219,8 @@ def main():
             entry["oracle"] = oracle_beside(entry, "m1_decode" if i == 0 else "m2_decode")
         if gated_conv:
             gated_conv["oracle"] = oracle_beside(gated_conv, "gated_conv")
+        if conv1d:
+            conv1d["oracle"] = oracle_beside(conv1d, "conv1d")
 
     if pg:
         pg.barrier()
@@ -1184,6 +1253,7 @@ def main():
             "prefill_mamba2": prefill_m2,
             "prefill_one_sequence": prefill_b1,
             "gated_conv": gated_conv,
+            "conv1d": conv1d,
             "decode": decode}
     print(json.dumps(line), flush=True)
     return 0

@@ -183,16 +183,12 @@ int sm_count(bool dry_run) { return sm_count(dry_run, current_device(dry_run)); 
 //   SSM_SCAN_SW=k          balanced prefill: k of every 8 exponential pairs on the FMA pipe (0..1)
 //   SSM_SCAN_SW_PAIRS=k    whole-unit prefill: k of 4 state pairs on the FMA pipe (0..3)
 //   SSM_SSU_ROWS_PER_ITEM, SSM_SSU_CTAS_PER_SM   Mamba-2 update launch shape
-//   SSM_CONV_DEPTH=1|2, SSM_CONV_WARPS_PER_SM=n   time-contiguous conv1d: loads in
-//                          flight per warp, and the warps per SM the row segments target
 struct Tuning {
     bool scan_vec = false;
     int scan_sw = 0;
     int scan_vec_sw = 0;
     long long ssu_rows = 0;
     int ssu_ctas = 0;
-    int conv_depth = 0;
-    int conv_warps = 0;
 };
 
 Tuning read_tuning() {
@@ -204,8 +200,6 @@ Tuning read_tuning() {
     if (env_int("SSM_SCAN_SW_PAIRS", &v) && v >= 0 && v <= 3) t.scan_vec_sw = (int)v;
     if (env_int("SSM_SSU_ROWS_PER_ITEM", &v) && v > 0) t.ssu_rows = v;
     if (env_int("SSM_SSU_CTAS_PER_SM", &v) && v > 0 && v <= 32) t.ssu_ctas = (int)v;
-    if (env_int("SSM_CONV_DEPTH", &v) && (v == 1 || v == 2)) t.conv_depth = (int)v;
-    if (env_int("SSM_CONV_WARPS_PER_SM", &v) && v > 0 && v <= 1024) t.conv_warps = (int)v;
     return t;
 }
 
@@ -303,23 +297,20 @@ ssm_status conv1d_impl(const ssm_conv1d_args* a, cudaStream_t stream) {
         vec = vec && t->stride[2] == 1 && aligned16(t->data) && (sd(*t, 0) * es) % 16 == 0 &&
               (sd(*t, 1) * es) % 16 == 0;
     if (vec) {
-        // one warp per (row, segment of whole 32-lane blocks), about 32 warps per SM
-        const int64_t blk = 32 * (int64_t)V;
-        const int warps = tuning().conv_warps > 0 ? tuning().conv_warps : 32;
-        const int64_t want = (int64_t)sm_count((a->flags & SSM_FLAG_DRY_RUN) != 0) * warps;
-        int64_t nseg = std::min<int64_t>(std::max<int64_t>((want + rows - 1) / rows, 1), (L + blk - 1) / blk);
-        const int64_t S = ((L + nseg - 1) / nseg + blk - 1) / blk * blk;
-        nseg = (L + S - 1) / S;
+        // units of U 32-vector blocks of a row; persistent CTAs of 8 warps
+        const bool dry = (a->flags & SSM_FLAG_DRY_RUN) != 0;
+        const int U = conv1d_vec_unroll();
+        const int64_t nb = (L + 32 * V - 1) / (32 * V);
+        const int64_t nbs = (nb + U - 1) / U;
+        const int64_t units = rows * nbs;
+        const int64_t grid = std::min<int64_t>((units + 7) / 8, (int64_t)sm_count(dry) * conv1d_vec_ctas_per_sm());
         plan.kernel = SSM_KERNEL_CONV1D;
         plan.block = 256;
-        plan.seg_steps = S;
-        plan.nseg = nseg;
-        plan.depth = tuning().conv_depth > 0 ? tuning().conv_depth : 1;
-        const int64_t grid = (rows * nseg + 7) / 8;
-        if (grid > INT32_MAX) return SSM_ERR_UNSUPPORTED;
         plan.grid = (int)grid;
-        fill_info(a->info, plan.kernel, plan.grid, plan.block, 0, 1, rows * nseg);
-        if (a->flags & SSM_FLAG_DRY_RUN) return SSM_OK;
+        plan.units_per_row = nbs;
+        plan.units = units;
+        fill_info(a->info, plan.kernel, plan.grid, plan.block, 0, 1, units);
+        if (dry) return SSM_OK;
         return launch_conv1d(p, plan, stream) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
     }
     plan.kernel = SSM_KERNEL_CONV1D_GENERIC;

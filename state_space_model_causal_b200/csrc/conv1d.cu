@@ -9,14 +9,14 @@
 // outgoing conv state is the last W raw inputs of (incoming state ++ x).
 //
 // Two kernels.  conv1d_vec_kernel takes the time-contiguous layout with
-// 16-byte aligned rows (a lane holds one 16-byte vector of steps; below).
+// 16-byte aligned rows (units of one 512-byte block of a row; below).
 // conv1d_kernel takes any strides: one warp owns one (b, d) row for the whole
 // sequence, so the incoming state is read before the outgoing state is
-// written with no cross-CTA ordering.
-// Each lane handles kVPT consecutive steps per segment; the W-1 history values
-// a lane needs come from its left neighbour by shuffle, and lane 0 takes them
-// from the previous segment's last lane.  The op is HBM-bound (2 or 4 bytes in
-// and out per element, W FMAs).
+// written with no cross-CTA ordering; each lane handles kVPT consecutive
+// steps per segment, the W-1 history values a lane needs come from its left
+// neighbour by shuffle, and lane 0 takes them from the previous segment's
+// last lane.  The op is HBM-bound (2 or 4 bytes in and out per element, W
+// FMAs).
 #include "../../include/ssm_causal.h"
 #include "common.cuh"
 #include "problem.h"
@@ -113,106 +113,138 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta) conv1d_kernel(const Conv1dP
 }
 
 // The time-contiguous layout with 16-byte aligned rows and L a multiple of V
-// (V = 8 steps at 16-bit, 4 at fp32), W - 1 <= V: a warp takes a segment of
-// whole 32V-step blocks of one (b, d) row, a lane one 16-byte vector of V
-// consecutive steps.  The W-1 inputs before a lane's steps come from the lane
-// below by shuffle, before lane 0's from the previous block's lane 31, or at
-// a segment start from the row itself (or the incoming state); the next
-// block's load (or the next two blocks') is issued before the current one is
-// computed.  Only the first
-// segment of a row reads the incoming state (a segment is >= 32V > W-1
-// steps), and its warp writes the outgoing state after all its lanes read.
-template <typename IoT, int W, int Depth>
-__global__ void __launch_bounds__(256) conv1d_vec_kernel(const Conv1dProblem p, int64_t S, int64_t nseg) {
+// (V = 8 steps at 16-bit, 4 at fp32), W - 1 <= V.  The work is cut into units
+// of U consecutive 32V-step blocks (U x 512 bytes) of one (b, d) row,
+// numbered row-major, and the persistent warps take units gw, gw + nw, ...
+// (nw warps in the grid): at any moment neighbouring warps read and write
+// neighbouring stretches of memory, one contiguous front through the tensor
+// as in a copy, not one front per row.  A lane holds one
+// 16-byte vector of V steps per block; the W-1 inputs before a lane's steps
+// come from the lane below by shuffle, before lane 0's from the previous
+// block's lane 31, and at the unit's start from the 16-byte vector ahead of it
+// (or, at a row's start, the incoming state).  A warp issues all U block
+// loads of its unit at once, then computes the blocks in order.  A row's
+// incoming state is read
+// only by the warp on its first unit, and that warp writes the outgoing state
+// (the last W raw inputs, read back from the row) after its lanes have read.
+// U = 4 blocks per unit (2 KB of loads in flight per warp); 3 CTAs of 256
+// threads per SM (the launch bounds' register cap).  Measured at the 2.8B
+// conv shape: 2 blocks per unit at 4 CTAs per SM was 13% slower, 8 blocks
+// 3% faster but spilling at the larger widths.
+constexpr int kUnroll = 4;
+constexpr int kVecCtasPerSm = 3;
+
+template <typename IoT, int W, int U = kUnroll>
+__global__ void __launch_bounds__(256, kVecCtasPerSm) conv1d_vec_kernel(const Conv1dProblem p, int64_t nbs, int64_t units) {
     constexpr int V = 16 / (int)sizeof(IoT);
     constexpr int H = W > 1 ? W - 1 : 1;
+    constexpr int64_t kSeg = (int64_t)U * 32 * V;  // steps per unit
     static_assert(W - 1 <= V, "the history must come from one lane below");
     const int lane = threadIdx.x & 31;
-    const int64_t gw = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-    if (gw >= p.Bn * p.D * nseg) return;  // whole warps
-    const int64_t row = gw / nseg, seg = gw % nseg;
-    const int64_t b = row / p.D, d = row - b * p.D;
-    const int64_t t0 = seg * S;
-    const int64_t t1 = t0 + S < p.L ? t0 + S : p.L;
-    const IoT* __restrict__ xr = static_cast<const IoT*>(p.x) + b * p.x_b + d * p.x_d;
-    IoT* __restrict__ orow = static_cast<IoT*>(p.out) + b * p.o_b + d * p.o_d;
-    const int64_t cs0 = b * p.cs_b + d * p.cs_d;
+    const int64_t nw = (int64_t)gridDim.x * 8;
+    const uint4 zero = make_uint4(0, 0, 0, 0);
 
-    float w[W];
+    int64_t u = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (u >= units) return;  // whole warps
+    // the unit's (b, d, segment), advanced by nw units per step without
+    // division: nw = q nbs + rs units, q = qd D + qr rows
+    const int64_t q = nw / nbs, rs = nw - q * nbs;
+    const int64_t qd = q / p.D, qr = q - qd * p.D;
+    int64_t sg = u % nbs, d = (u / nbs) % p.D, b = (u / nbs) / p.D;
+    for (; u < units; u += nw) {
+        const IoT* __restrict__ xr = static_cast<const IoT*>(p.x) + b * p.x_b + d * p.x_d;
+        IoT* __restrict__ orow = static_cast<IoT*>(p.out) + b * p.o_b + d * p.o_d;
+        const int64_t cs0 = b * p.cs_b + d * p.cs_d;
+        const int64_t t0 = sg * kSeg;
+        uint4 xv[U];
 #pragma unroll
-    for (int k = 0; k < W; ++k) w[k] = p.w[d * p.w_d + k * p.w_k];
-    const float bias = p.bias ? p.bias[d * p.b_d] : 0.0f;
-    float carry[H];  // raw input at (block start) - (W-1) + i
+        for (int i = 0; i < U; ++i) {
+            const int64_t t = t0 + i * 32 * V + lane * V;
+            xv[i] = t < p.L ? *reinterpret_cast<const uint4*>(xr + t) : zero;
+        }
+        float w[W];
 #pragma unroll
-    for (int i = 0; i < W - 1; ++i) {
-        const int64_t t = t0 - (W - 1) + i;
-        carry[i] = t >= 0 ? to_f(xr[t])
-                          : (p.conv_state ? ld_f(p.conv_state, cs0 + (W + t) * p.cs_k, p.cs_dt) : 0.0f);
-    }
-    // loads run Depth blocks ahead of the arithmetic
-    uint4 nx[Depth];
+        for (int k = 0; k < W; ++k) w[k] = p.w[d * p.w_d + k * p.w_k];
+        const float bias = p.bias ? p.bias[d * p.b_d] : 0.0f;
+        // carry[k] = input at t0 - (W-1) + k (lane 0's history), then the
+        // previous block's last W-1 inputs
+        float carry[H];
+        if (sg > 0) {
+            float hv[V];
+            Vec16<IoT>::unpack(*reinterpret_cast<const uint4*>(xr + t0 - V), hv);
 #pragma unroll
-    for (int i = 0; i < Depth; ++i) {
-        const int64_t t = t0 + lane * V + i * 32 * V;
-        nx[i] = t < t1 ? *reinterpret_cast<const uint4*>(xr + t) : make_uint4(0, 0, 0, 0);
-    }
-    for (int64_t tb = t0; tb < t1; tb += 32 * V) {
-        const int64_t t = tb + lane * V;
-        const bool valid = t < t1;
-        const uint4 cx = nx[0];
+            for (int k = 0; k < W - 1; ++k) carry[k] = hv[V - (W - 1) + k];
+        } else {
 #pragma unroll
-        for (int i = 0; i + 1 < Depth; ++i) nx[i] = nx[i + 1];
-        if (t + Depth * 32 * V < t1) nx[Depth - 1] = *reinterpret_cast<const uint4*>(xr + t + Depth * 32 * V);
-        float v[V], o[V];
-        Vec16<IoT>::unpack(cx, v);
-#pragma unroll
-        for (int j = 0; j < V; ++j) v[j] = valid ? v[j] : 0.0f;
-        float prev[H];
-#pragma unroll
-        for (int i = 0; i < W - 1; ++i) {
-            const float up = __shfl_up_sync(0xffffffffu, v[V - (W - 1) + i], 1);
-            prev[i] = lane == 0 ? carry[i] : up;
+            for (int k = 0; k < W - 1; ++k)
+                carry[k] = p.conv_state ? ld_f(p.conv_state, cs0 + (k + 1) * p.cs_k, p.cs_dt) : 0.0f;
         }
 #pragma unroll
-        for (int i = 0; i < W - 1; ++i) carry[i] = __shfl_sync(0xffffffffu, v[V - (W - 1) + i], 31);
+        for (int i = 0; i < U; ++i) {
+            if (t0 + i * 32 * V >= p.L) break;  // uniform: the row ends before this block
+            const int64_t t = t0 + i * 32 * V + lane * V;
+            float v[V], o[V];
+            Vec16<IoT>::unpack(xv[i], v);  // zero past the row's end
+            float prev[H];
 #pragma unroll
-        for (int j = 0; j < V; ++j) {
-            float acc = bias;
-#pragma unroll
-            for (int k = 0; k < W; ++k) {
-                const int idx = j - (W - 1) + k;
-                acc = fmaf(w[k], idx >= 0 ? v[idx] : prev[W - 1 + idx], acc);
+            for (int k = 0; k < W - 1; ++k) {
+                const float up = __shfl_up_sync(0xffffffffu, v[V - (W - 1) + k], 1);
+                prev[k] = lane == 0 ? carry[k] : up;
             }
-            o[j] = p.silu ? silu_f(acc) : acc;
+#pragma unroll
+            for (int k = 0; k < W - 1; ++k) carry[k] = __shfl_sync(0xffffffffu, v[V - (W - 1) + k], 31);
+#pragma unroll
+            for (int j = 0; j < V; ++j) {
+                float acc = bias;
+#pragma unroll
+                for (int k = 0; k < W; ++k) {
+                    const int idx = j - (W - 1) + k;
+                    acc = fmaf(w[k], idx >= 0 ? v[idx] : prev[W - 1 + idx], acc);
+                }
+                o[j] = p.silu ? silu_f(acc) : acc;
+            }
+            if (t < p.L) *reinterpret_cast<uint4*>(orow + t) = Vec16<IoT>::pack(o);
         }
-        if (valid) *reinterpret_cast<uint4*>(orow + t) = Vec16<IoT>::pack(o);
-    }
-    if (p.conv_state && seg == 0) {
-        float nv = 0.0f;
-        if (lane < W) {
-            const int64_t t = p.L - W + lane;
-            nv = t >= 0 ? to_f(xr[t]) : ld_f(p.conv_state, cs0 + (p.L + lane) * p.cs_k, p.cs_dt);
+        if (sg == 0 && p.conv_state) {
+            float nv = 0.0f;
+            if (lane < W) {
+                const int64_t tt = p.L - W + lane;
+                nv = tt >= 0 ? to_f(xr[tt]) : ld_f(p.conv_state, cs0 + (p.L + lane) * p.cs_k, p.cs_dt);
+            }
+            __syncwarp();
+            if (lane < W) st_f(p.conv_state, cs0 + lane * p.cs_k, p.cs_dt, nv);
         }
-        __syncwarp();
-        if (lane < W) st_f(p.conv_state, cs0 + lane * p.cs_k, p.cs_dt, nv);
+        // next unit
+        sg += rs;
+        int64_t c = 0;
+        if (sg >= nbs) {
+            sg -= nbs;
+            c = 1;
+        }
+        d += qr + c;
+        b += qd;
+        if (d >= p.D) {
+            d -= p.D;
+            ++b;
+        }
     }
 }
 
-template <typename IoT, int D>
+template <typename IoT>
 cudaError_t launch_vec(const Conv1dProblem& p, const Conv1dPlan& plan, cudaStream_t s) {
     constexpr int V = 16 / (int)sizeof(IoT);
-    const int64_t S = plan.seg_steps, nseg = plan.nseg;
+    const int64_t nbs = plan.units_per_row, units = plan.units;
     switch (p.W) {
-        case 1: conv1d_vec_kernel<IoT, 1, D><<<plan.grid, plan.block, 0, s>>>(p, S, nseg); break;
-        case 2: conv1d_vec_kernel<IoT, 2, D><<<plan.grid, plan.block, 0, s>>>(p, S, nseg); break;
-        case 3: conv1d_vec_kernel<IoT, 3, D><<<plan.grid, plan.block, 0, s>>>(p, S, nseg); break;
-        case 4: conv1d_vec_kernel<IoT, 4, D><<<plan.grid, plan.block, 0, s>>>(p, S, nseg); break;
-        case 5: conv1d_vec_kernel<IoT, 5, D><<<plan.grid, plan.block, 0, s>>>(p, S, nseg); break;
-        case 6: if constexpr (V >= 5) { conv1d_vec_kernel<IoT, (V >= 5 ? 6 : 1), D><<<plan.grid, plan.block, 0, s>>>(p, S, nseg); break; }
+        case 1: conv1d_vec_kernel<IoT, 1><<<plan.grid, plan.block, 0, s>>>(p, nbs, units); break;
+        case 2: conv1d_vec_kernel<IoT, 2><<<plan.grid, plan.block, 0, s>>>(p, nbs, units); break;
+        case 3: conv1d_vec_kernel<IoT, 3><<<plan.grid, plan.block, 0, s>>>(p, nbs, units); break;
+        case 4: conv1d_vec_kernel<IoT, 4><<<plan.grid, plan.block, 0, s>>>(p, nbs, units); break;
+        case 5: conv1d_vec_kernel<IoT, 5><<<plan.grid, plan.block, 0, s>>>(p, nbs, units); break;
+        case 6: if constexpr (V >= 5) { conv1d_vec_kernel<IoT, (V >= 5 ? 6 : 1)><<<plan.grid, plan.block, 0, s>>>(p, nbs, units); break; }
                 return cudaErrorInvalidValue;
-        case 7: if constexpr (V >= 6) { conv1d_vec_kernel<IoT, (V >= 6 ? 7 : 1), D><<<plan.grid, plan.block, 0, s>>>(p, S, nseg); break; }
+        case 7: if constexpr (V >= 6) { conv1d_vec_kernel<IoT, (V >= 6 ? 7 : 1)><<<plan.grid, plan.block, 0, s>>>(p, nbs, units); break; }
                 return cudaErrorInvalidValue;
-        case 8: if constexpr (V >= 7) { conv1d_vec_kernel<IoT, (V >= 7 ? 8 : 1), D><<<plan.grid, plan.block, 0, s>>>(p, S, nseg); break; }
+        case 8: if constexpr (V >= 7) { conv1d_vec_kernel<IoT, (V >= 7 ? 8 : 1)><<<plan.grid, plan.block, 0, s>>>(p, nbs, units); break; }
                 return cudaErrorInvalidValue;
         default: return cudaErrorInvalidValue;
     }
@@ -221,14 +253,15 @@ cudaError_t launch_vec(const Conv1dProblem& p, const Conv1dPlan& plan, cudaStrea
 
 }  // namespace
 
+int conv1d_vec_ctas_per_sm() { return kVecCtasPerSm; }
+int conv1d_vec_unroll() { return kUnroll; }
+
 cudaError_t launch_conv1d(const Conv1dProblem& p, const Conv1dPlan& plan, cudaStream_t s) {
     if (plan.kernel == SSM_KERNEL_CONV1D) {
-        const bool d2 = plan.depth == 2;
         switch (p.io_dt) {
-            case kF32: return d2 ? launch_vec<float, 2>(p, plan, s) : launch_vec<float, 1>(p, plan, s);
-            case kF16: return d2 ? launch_vec<__half, 2>(p, plan, s) : launch_vec<__half, 1>(p, plan, s);
-            case kBF16:
-                return d2 ? launch_vec<__nv_bfloat16, 2>(p, plan, s) : launch_vec<__nv_bfloat16, 1>(p, plan, s);
+            case kF32: return launch_vec<float>(p, plan, s);
+            case kF16: return launch_vec<__half>(p, plan, s);
+            case kBF16: return launch_vec<__nv_bfloat16>(p, plan, s);
             default: return cudaErrorInvalidValue;
         }
     }

@@ -220,10 +220,11 @@ struct Conv1dPlan {
     int kernel;
     int block;
     int grid;
-    int64_t seg_steps;  // vector kernel: steps per row segment (a multiple of 32 vectors)
-    int64_t nseg;       // vector kernel: segments per row
-    int depth;          // vector kernel: blocks of loads in flight ahead of the arithmetic (1 or 2)
+    int64_t units_per_row;   // vector kernel: ceil(32-vector blocks per row / conv1d_vec_unroll())
+    int64_t units;           // vector kernel: rows x units_per_row
 };
+int conv1d_vec_ctas_per_sm();
+int conv1d_vec_unroll();
 
 cudaError_t launch_ssu(const SsuProblem& p, const SsuPlan& plan, cudaStream_t s);
 int ssu_tma_max_stages();

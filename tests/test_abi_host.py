@@ -373,19 +373,23 @@ def test_empty_problems_launch_nothing(lib):
 
 
 def test_conv_plan(lib):
-    """L a multiple of the vector width: the 16-byte vector kernel, one warp
-    per (row, segment of 256-step blocks), about 32 warps per SM of the
-    dry-run B200; otherwise (or W - 1 above the vector width, or unit time
-    stride missing) the warp-per-row kernel."""
+    """L a multiple of the vector width: the 16-byte vector kernel, units of
+    four 256-step blocks (fp16) of a row, persistent CTAs of 8 warps (at most
+    3 per SM of the dry-run B200); otherwise (or W - 1 above the vector
+    width, or unit time stride missing) the warp-per-row kernel."""
     st, info = call(lib, "ssm_causal_conv1d_fwd", conv_args(FakeMem()))
     assert st == OK and bd.KERNELS[info.kernel] == "conv1d_generic" and info.grid == 2 * 64 // 4
-    # 128 rows x ceil(148 * 32 / 128) = 37 segments, capped at 2048 / 256 = 8
+    # 128 rows x 2 units of 4 blocks: one unit per warp
     st, info = call(lib, "ssm_causal_conv1d_fwd", conv_args(FakeMem(), L=2048))
     assert st == OK and bd.KERNELS[info.kernel] == "conv1d" and info.block == 256
-    assert info.grid == 2 * 64 * 8 // 8 and info.work_items == 2 * 64 * 8
-    # many rows: one segment per row
+    assert info.grid == 2 * 64 * 2 // 8 and info.work_items == 2 * 64 * 2
+    # many units: the grid stops at 148 SMs x 3 CTAs
     st, info = call(lib, "ssm_causal_conv1d_fwd", conv_args(FakeMem(), Bn=4, D=5120, L=2048))
-    assert st == OK and bd.KERNELS[info.kernel] == "conv1d" and info.grid == 4 * 5120 // 8
+    assert st == OK and bd.KERNELS[info.kernel] == "conv1d" and info.grid == 148 * 3
+    assert info.work_items == 4 * 5120 * 2
+    # a ragged last block: ceil(264 / 256) = 2 blocks, one unit per row
+    st, info = call(lib, "ssm_causal_conv1d_fwd", conv_args(FakeMem(), Bn=1, D=3, L=264))
+    assert st == OK and bd.KERNELS[info.kernel] == "conv1d" and info.work_items == 3 and info.grid == 1
     # fp32: 4 steps per vector, so W = 6 needs the generic kernel; W = 5 does not
     st, info = call(lib, "ssm_causal_conv1d_fwd", conv_args(FakeMem(), L=64, W=6, io=F32))
     assert st == OK and bd.KERNELS[info.kernel] == "conv1d_generic"

@@ -63,13 +63,39 @@ def test_conv1d_vector_rows_match_oracle(io, Bt, D, L, W, silu):
     np.testing.assert_array_equal(N(csg), csref)
 
 
+@pytest.mark.parametrize("io", ["f32", "f16", "bf16"])
+@pytest.mark.parametrize("Bt,D,L,W", [(1, 3600, 8, 4), (2, 1800, 1032, 4), (1, 4000, 264, 1), (1, 3560, 520, 5),
+                                      (1, 3600, 16, 8), (1, 3600, 4, 5), (3, 1500, 2048, 3), (2, 1800, 4096, 4)])
+def test_conv1d_vector_many_rows_match_oracle(io, Bt, D, L, W):
+    """More units than the persistent grid's warps (148 SMs x 4 CTAs x 8),
+    so each warp takes several units across row ends: rows of one short
+    block, rows of several blocks with a ragged last one, L below the width
+    (fp32, L = 4, W = 5), widths 1..8, SiLU, bias and an incoming state."""
+    import torch
+    from state_space_model_causal_b200 import LaunchInfo, binding, ssm_causal_conv1d_fwd
+    tag = ("convm", Bt, D, L, W)
+    x = gen.round_to(gen.normal((Bt, D, L), *tag, "x"), io)
+    w = gen.round_to(gen.normal((D, W), *tag, "w", std=0.2), "f32")
+    b = gen.round_to(gen.normal((D,), *tag, "b"), "f32")
+    cs = gen.round_to(gen.normal((Bt, D, W), *tag, "cs"), "f32")
+    csg = T(cs, "f32")
+    info = LaunchInfo()
+    out = ssm_causal_conv1d_fwd(T(x, io), T(w, "f32"), bias=T(b, "f32"), conv_state=csg, silu=True, info=info)
+    torch.cuda.synchronize()
+    assert binding.KERNELS[info.kernel] == _conv_kernel(io, L, W)
+    ref, csref = oracle.conv1d(x, w, bias=b, conv_state=cs, silu=True)
+    assert_close(N(out), ref, TOL[io], "out")
+    np.testing.assert_array_equal(N(csg), csref)
+
+
 @pytest.mark.parametrize("io", ["f16", "bf16"])
-def test_conv1d_vector_state_in_io_dtype_and_padded_rows(io):
+@pytest.mark.parametrize("D", [7, 3600])
+def test_conv1d_vector_state_in_io_dtype_and_padded_rows(io, D):
     """A conv state in the io dtype, no bias, and x / out rows that sit in a
     wider (B, D, L + 16) buffer (aligned, not contiguous)."""
     import torch
     from state_space_model_causal_b200 import LaunchInfo, binding, ssm_causal_conv1d_fwd
-    Bt, D, L, W = 2, 7, 512, 4
+    Bt, L, W = 2, 512, 4
     x = gen.round_to(gen.normal((Bt, D, L), "convp", "x"), io)
     w = gen.round_to(gen.normal((D, W), "convp", "w", std=0.2), "f32")
     cs = gen.round_to(gen.normal((Bt, D, W), "convp", "cs"), io)
@@ -80,19 +106,21 @@ def test_conv1d_vector_state_in_io_dtype_and_padded_rows(io):
     info = LaunchInfo()
     ssm_causal_conv1d_fwd(xb[:, :, :L], T(w, "f32"), conv_state=csg, silu=True, out=ob[:, :, :L], info=info)
     torch.cuda.synchronize()
-    assert binding.KERNELS[info.kernel] == "conv1d"
+    assert binding.KERNELS[info.kernel] == _conv_kernel(io, L, W)
     ref, csref = oracle.conv1d(x, w, conv_state=cs, silu=True)
     assert_close(N(ob[:, :, :L]), ref, TOL[io], "out")
     assert bool(torch.all(ob[:, :, L:] == 7.0))
     np.testing.assert_array_equal(N(csg), gen.round_to(csref, io))
 
 
-def test_conv1d_vector_decode_after_prefill():
-    """A vector-kernel prefill's outgoing state feeds token-by-token calls
-    (the warp-per-row kernel at L = 1); together they equal one oracle call."""
+@pytest.mark.parametrize("D", [5, 1800])
+def test_conv1d_vector_decode_after_prefill(D):
+    """A vector-kernel prefill's outgoing state (few rows, or more rows than
+    the grid has warps) feeds token-by-token calls (the warp-per-row kernel
+    at L = 1); together they equal one oracle call."""
     import torch
     from state_space_model_causal_b200 import ssm_causal_conv1d_fwd
-    Bt, D, L, W, extra = 2, 5, 256, 4, 6
+    Bt, L, W, extra = 2, 256, 4, 6
     x = gen.round_to(gen.normal((Bt, D, L + extra), "convd", "x"), "f16")
     w = gen.round_to(gen.normal((D, W), "convd", "w", std=0.2), "f32")
     cs = gen.round_to(gen.normal((Bt, D, W), "convd", "cs"), "f32")

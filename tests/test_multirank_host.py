@@ -75,6 +75,7 @@ def test_reference_arm_runs_on_rank_zero_only():
     ("m2_decode", {"bytes_per_call": 4331209248, "batch": 1639, "heads": 80, "P": 64, "N": 128}, 1),
     ("m2_prefill", {}, 1),
     ("gated_conv", {"roofline": {"algorithmic_bytes_per_launch": 134414336}}, 1),
+    ("conv1d", {"roofline": {"algorithmic_bytes_per_launch": 168448000}}, 8),
 ])
 def test_oracle_beside_each_sub_line_runs_on_the_host(kind, entry, rows):
     """The oracle timings attached to the bench's sub-lines run on the host
