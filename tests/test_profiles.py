@@ -33,7 +33,7 @@ def test_there_are_traffic_summaries_for_every_bench_kernel():
     for need in ("scan_bal_prefill_2p8b.txt", "scan_m2_prefill_2p7b.txt", "ssu_row_tma_decode_2p8b.txt",
                  "ssu_head_tma_mamba2_64x128_f16_R131072.txt", "ssu_head_tma_mamba2_64x128_f32_R131072.txt",
                  "ssu_head_tma_mamba2_128x256_bf16_R65536.txt", "ssu_head_tma_mamba2_128x256_f32_R65536.txt",
-                 "gated_conv_lfm.txt"):
+                 "gated_conv_lfm.txt", "conv1d_2p8b.txt"):
         assert need in names
 
 
