@@ -180,8 +180,18 @@ typedef enum ssm_kernel_id {
  *   silu       nonzero: apply SiLU to the conv output
  *   out        (B, D, L)  x's dtype                               output
  *
- * out[b,d,t] = act(bias[d] + sum_k weight[d,k] * x[b,d,t-(W-1)+k]).
- * L = 0 leaves conv_state unchanged.
+ * out[b,d,t] = act(bias[d] + sum_k weight[d,k] * x[b,d,t-(W-1)+k]): the
+ * "causal-conv1d" operator of "feat(llama.cu): 适配 mamba 模型" (section 2.1),
+ * with the conv-state cache of its section 3.1 read before and written after
+ * the sequence.  L = 0 leaves conv_state unchanged.
+ *
+ * Any strides.  Time-contiguous rows (unit step stride, 16-byte aligned data
+ * and row strides for x and out, L a multiple of 8 at 16-bit or 4 at fp32,
+ * W - 1 at most that multiple) run on SSM_KERNEL_CONV1D; other layouts on
+ * SSM_KERNEL_CONV1D_GENERIC.  out may not overlap x, weight, bias or the
+ * state, nor the state x, weight or bias (SSM_ERR_ALIAS); an out or
+ * conv_state whose elements overlap one another (a broadcast view) is
+ * SSM_ERR_STRIDE.
  * ------------------------------------------------------------------------ */
 typedef struct ssm_conv1d_args {
     uint32_t struct_size; /* = sizeof(ssm_conv1d_args) */

@@ -488,6 +488,15 @@ def test_conv_error_paths(lib):
     a = conv_args(m)
     a.out = a.x
     _expect(lib, fn, a, EALIAS)
+    a = conv_args(m)                      # the state inside x
+    a.conv_state = bd.raw_tensor(a.x.data, F32, (2, 64, 4), None)
+    _expect(lib, fn, a, EALIAS)
+    a = conv_args(m)                      # the state inside out
+    a.conv_state = bd.raw_tensor(a.out.data + 256, F32, (2, 64, 4), None)
+    _expect(lib, fn, a, EALIAS)
+    # broadcast (self-overlapping) out or state: refused, not raced
+    _expect(lib, fn, conv_args(m, out=m(F16, (2, 64, 100), (0, 100, 1))), ESTRIDE)
+    _expect(lib, fn, conv_args(m, conv_state=m(F32, (2, 64, 4), (4 * 64, 0, 1))), ESTRIDE)
 
 
 def test_oversized_tensors_are_rejected_before_any_arithmetic(lib):
