@@ -136,9 +136,9 @@ def test_conv1d_vector_decode_after_prefill(D):
     np.testing.assert_array_equal(N(csg), csref)
 
 
-def test_conv1d_without_state_and_full_size():
-    """The 2.8B prefill's conv (B=4, D=5120, L=2048, W=4, fp16, SiLU) on the
-    vector kernel; 16 sampled rows against the oracle."""
+def test_conv1d_without_state_at_the_prefill_shape():
+    """No conv state: zeros before t = 0 and nothing written; 16 sampled rows
+    of the 2.8B prefill's x against the oracle."""
     import torch
     from state_space_model_causal_b200 import LaunchInfo, binding, ssm_causal_conv1d_fwd
     s = gen.prefill_2p8b(seed=0)
@@ -153,6 +153,27 @@ def test_conv1d_without_state_and_full_size():
         ref, _ = oracle.conv1d(s.x[b:b + 1, d:d + 1], s.conv_weight[d:d + 1],
                                bias=s.conv_bias[d:d + 1], silu=True)
         assert_close(got[b:b + 1, d:d + 1], ref, TOL["f16"], f"row ({b},{d})")
+
+
+def test_conv1d_full_size_every_element():
+    """The benchmark's launch (B=4, D=5120, L=2048, W=4, fp16, bias, SiLU, an
+    fp32 conv state read and written) against the oracle on every output
+    element and every state entry."""
+    import torch
+    from state_space_model_causal_b200 import LaunchInfo, binding, ssm_causal_conv1d_fwd
+    tag = ("convfull",)
+    x = gen.round_to(gen.normal((4, 5120, 2048), *tag, "x"), "f16")
+    w = gen.round_to(gen.normal((5120, 4), *tag, "w", std=0.2), "f32")
+    b = gen.round_to(gen.normal((5120,), *tag, "b", std=0.1), "f32")
+    cs = gen.round_to(gen.normal((4, 5120, 4), *tag, "cs"), "f32")
+    csg = T(cs, "f32")
+    info = LaunchInfo()
+    out = ssm_causal_conv1d_fwd(T(x, "f16"), T(w, "f32"), bias=T(b, "f32"), conv_state=csg, silu=True, info=info)
+    torch.cuda.synchronize()
+    assert binding.KERNELS[info.kernel] == "conv1d"
+    ref, csref = oracle.conv1d(x, w, bias=b, conv_state=cs, silu=True)
+    assert_close(N(out), ref, TOL["f16"], "out")
+    np.testing.assert_array_equal(N(csg), csref)
 
 
 # ------------------------------------------------------------ canary bands --
