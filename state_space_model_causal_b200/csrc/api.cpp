@@ -297,9 +297,10 @@ ssm_status conv1d_impl(const ssm_conv1d_args* a, cudaStream_t stream) {
         vec = vec && t->stride[2] == 1 && aligned16(t->data) && (sd(*t, 0) * es) % 16 == 0 &&
               (sd(*t, 1) * es) % 16 == 0;
     if (vec) {
-        // units of U 32-vector blocks of a row; persistent CTAs of 8 warps
+        // units of U 32-vector blocks of a row (U = 8 or 4 by dtype and
+        // width); persistent CTAs of 8 warps
         const bool dry = (a->flags & SSM_FLAG_DRY_RUN) != 0;
-        const int U = conv1d_vec_unroll();
+        const int U = conv1d_vec_unroll(p.io_dt, W);
         const int64_t nb = (L + 32 * V - 1) / (32 * V);
         const int64_t nbs = (nb + U - 1) / U;
         const int64_t units = rows * nbs;

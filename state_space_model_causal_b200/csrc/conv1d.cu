@@ -21,6 +21,8 @@
 #include "common.cuh"
 #include "problem.h"
 
+#include <type_traits>
+
 namespace ssm {
 namespace {
 
@@ -127,14 +129,18 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta) conv1d_kernel(const Conv1dP
 // incoming state is read
 // only by the warp on its first unit, and that warp writes the outgoing state
 // (the last W raw inputs, read back from the row) after its lanes have read.
-// U = 4 blocks per unit (2 KB of loads in flight per warp); 3 CTAs of 256
-// threads per SM (the launch bounds' register cap).  Measured at the 2.8B
-// conv shape: 2 blocks per unit at 4 CTAs per SM was 13% slower, 8 blocks
-// 3% faster but spilling at the larger widths.
-constexpr int kUnroll = 4;
+// U blocks per unit (U x 512 bytes of loads in flight per warp): 8 for fp16
+// and fp32 up to W = 4, 4 otherwise (at 8, bf16 and the larger widths spill);
+// 3 CTAs of 256 threads per SM (the launch bounds' register cap).  Measured at
+// the 2.8B conv shape: 8 blocks 41.0-41.5 us, 4 blocks 42.4-43.1 us, 2 blocks
+// (at 4 CTAs per SM) 47.9 us.
+template <typename IoT>
+constexpr int unroll_of(int W) {
+    return (sizeof(IoT) == 4 || std::is_same<IoT, __half>::value) && W <= 4 ? 8 : 4;
+}
 constexpr int kVecCtasPerSm = 3;
 
-template <typename IoT, int W, int U = kUnroll>
+template <typename IoT, int W, int U = unroll_of<IoT>(W)>
 __global__ void __launch_bounds__(256, kVecCtasPerSm) conv1d_vec_kernel(const Conv1dProblem p, int64_t nbs, int64_t units) {
     constexpr int V = 16 / (int)sizeof(IoT);
     constexpr int H = W > 1 ? W - 1 : 1;
@@ -254,7 +260,11 @@ cudaError_t launch_vec(const Conv1dProblem& p, const Conv1dPlan& plan, cudaStrea
 }  // namespace
 
 int conv1d_vec_ctas_per_sm() { return kVecCtasPerSm; }
-int conv1d_vec_unroll() { return kUnroll; }
+int conv1d_vec_unroll(int io_dt, int64_t W) {
+    if (W < 1 || W > 8) return 4;
+    const int w = (int)W;
+    return io_dt == kF32 ? unroll_of<float>(w) : io_dt == kF16 ? unroll_of<__half>(w) : unroll_of<__nv_bfloat16>(w);
+}
 
 cudaError_t launch_conv1d(const Conv1dProblem& p, const Conv1dPlan& plan, cudaStream_t s) {
     if (plan.kernel == SSM_KERNEL_CONV1D) {

@@ -220,11 +220,11 @@ struct Conv1dPlan {
     int kernel;
     int block;
     int grid;
-    int64_t units_per_row;   // vector kernel: ceil(32-vector blocks per row / conv1d_vec_unroll())
+    int64_t units_per_row;   // vector kernel: ceil(32-vector blocks per row / conv1d_vec_unroll(io, W))
     int64_t units;           // vector kernel: rows x units_per_row
 };
 int conv1d_vec_ctas_per_sm();
-int conv1d_vec_unroll();
+int conv1d_vec_unroll(int io_dt, int64_t W);  // 32-vector blocks per unit of the vector kernel
 
 cudaError_t launch_ssu(const SsuProblem& p, const SsuPlan& plan, cudaStream_t s);
 int ssu_tma_max_stages();

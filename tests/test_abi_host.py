@@ -374,19 +374,26 @@ def test_empty_problems_launch_nothing(lib):
 
 def test_conv_plan(lib):
     """L a multiple of the vector width: the 16-byte vector kernel, units of
-    four 256-step blocks (fp16) of a row, persistent CTAs of 8 warps (at most
-    3 per SM of the dry-run B200); otherwise (or W - 1 above the vector
-    width, or unit time stride missing) the warp-per-row kernel."""
+    U 256-step blocks (fp16) of a row -- U = 8 for fp16 and fp32 up to W = 4,
+    else 4 -- on persistent CTAs of 8 warps (at most 3 per SM of the dry-run
+    B200); otherwise (or W - 1 above the vector width, or unit time stride
+    missing) the warp-per-row kernel."""
     st, info = call(lib, "ssm_causal_conv1d_fwd", conv_args(FakeMem()))
     assert st == OK and bd.KERNELS[info.kernel] == "conv1d_generic" and info.grid == 2 * 64 // 4
-    # 128 rows x 2 units of 4 blocks: one unit per warp
+    # 128 rows of 8 blocks, fp16, W = 4: one unit of 8 blocks per row
     st, info = call(lib, "ssm_causal_conv1d_fwd", conv_args(FakeMem(), L=2048))
     assert st == OK and bd.KERNELS[info.kernel] == "conv1d" and info.block == 256
-    assert info.grid == 2 * 64 * 2 // 8 and info.work_items == 2 * 64 * 2
+    assert info.grid == 2 * 64 // 8 and info.work_items == 2 * 64
+    # bf16: units of 4 blocks, two per row
+    st, info = call(lib, "ssm_causal_conv1d_fwd", conv_args(FakeMem(), L=2048, io=BF16))
+    assert st == OK and bd.KERNELS[info.kernel] == "conv1d" and info.work_items == 2 * 64 * 2
+    # fp16, W = 5: units of 4 blocks
+    st, info = call(lib, "ssm_causal_conv1d_fwd", conv_args(FakeMem(), L=2048, W=5))
+    assert st == OK and bd.KERNELS[info.kernel] == "conv1d" and info.work_items == 2 * 64 * 2
     # many units: the grid stops at 148 SMs x 3 CTAs
     st, info = call(lib, "ssm_causal_conv1d_fwd", conv_args(FakeMem(), Bn=4, D=5120, L=2048))
     assert st == OK and bd.KERNELS[info.kernel] == "conv1d" and info.grid == 148 * 3
-    assert info.work_items == 4 * 5120 * 2
+    assert info.work_items == 4 * 5120
     # a ragged last block: ceil(264 / 256) = 2 blocks, one unit per row
     st, info = call(lib, "ssm_causal_conv1d_fwd", conv_args(FakeMem(), Bn=1, D=3, L=264))
     assert st == OK and bd.KERNELS[info.kernel] == "conv1d" and info.work_items == 3 and info.grid == 1
