@@ -9,7 +9,7 @@
 // outgoing conv state is the last W raw inputs of (incoming state ++ x).
 //
 // Two kernels.  conv1d_vec_kernel takes the time-contiguous layout with
-// 16-byte aligned rows (units of one 512-byte block of a row; below).
+// 16-byte aligned rows (units of 4 or 8 512-byte blocks of a row; below).
 // conv1d_kernel takes any strides: one warp owns one (b, d) row for the whole
 // sequence, so the incoming state is read before the outgoing state is
 // written with no cross-CTA ordering; each lane handles kVPT consecutive
@@ -116,24 +116,24 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta) conv1d_kernel(const Conv1dP
 
 // The time-contiguous layout with 16-byte aligned rows and L a multiple of V
 // (V = 8 steps at 16-bit, 4 at fp32), W - 1 <= V.  The work is cut into units
-// of U consecutive 32V-step blocks (U x 512 bytes) of one (b, d) row,
-// numbered row-major, and the persistent warps take units gw, gw + nw, ...
-// (nw warps in the grid): at any moment neighbouring warps read and write
-// neighbouring stretches of memory, one contiguous front through the tensor
-// as in a copy, not one front per row.  A lane holds one
-// 16-byte vector of V steps per block; the W-1 inputs before a lane's steps
-// come from the lane below by shuffle, before lane 0's from the previous
-// block's lane 31, and at the unit's start from the 16-byte vector ahead of it
-// (or, at a row's start, the incoming state).  A warp issues all U block
-// loads of its unit at once, then computes the blocks in order.  A row's
-// incoming state is read
-// only by the warp on its first unit, and that warp writes the outgoing state
-// (the last W raw inputs, read back from the row) after its lanes have read.
-// U blocks per unit (U x 512 bytes of loads in flight per warp): 8 for fp16
-// and fp32 up to W = 4, 4 otherwise (at 8, bf16 and the larger widths spill);
-// 3 CTAs of 256 threads per SM (the launch bounds' register cap).  Measured at
-// the 2.8B conv shape: 8 blocks 41.0-41.5 us, 4 blocks 42.4-43.1 us, 2 blocks
-// (at 4 CTAs per SM) 47.9 us.
+// of U consecutive 32V-step blocks (U x 512 bytes) of one (b, d) row, numbered
+// row-major, and the persistent warps take units gw, gw + nw, ... (nw warps in
+// the grid): at any moment neighbouring warps read and write neighbouring
+// stretches of memory, one contiguous front through the tensor as in a copy,
+// not one front per row.  A warp issues all U block loads of its unit at
+// once, then computes the blocks in order.  A lane holds one 16-byte vector
+// of V steps per block; the W-1 inputs before a lane's steps come from the
+// lane below by shuffle, before lane 0's from the previous block's lane 31,
+// and at the unit's start from the 16-byte vector ahead of it (or, at a row's
+// start, the incoming state).  A row's incoming state is read only by the warp
+// on its first unit, and that warp writes the outgoing state (the last W raw
+// inputs, read back from the row) after its lanes have read.
+//
+// U (U x 512 bytes of loads in flight per warp) is 8 for fp16 and fp32 up to
+// W = 4 and 4 otherwise (at 8, bf16 and the larger widths spill); 3 CTAs of
+// 256 threads per SM (the launch bounds' register cap).  Measured at the 2.8B
+// conv shape: 8 blocks 40.9-41.5 us, 4 blocks 42.4-43.1 us, 2 blocks (at 4
+// CTAs per SM) 47.9 us.
 template <typename IoT>
 constexpr int unroll_of(int W) {
     return (sizeof(IoT) == 4 || std::is_same<IoT, __half>::value) && W <= 4 ? 8 : 4;
