@@ -404,6 +404,31 @@ def test_conv_plan(lib):
     assert st == OK and bd.KERNELS[info.kernel] == "conv1d"
 
 
+def test_conv_plan_matches_its_rules_on_random_shapes(lib):
+    """The planner's choice, unroll, unit count and grid for 300 random
+    contiguous shapes, against the rules stated plainly: the vector kernel
+    when L is a multiple of V and W - 1 <= V; U = 8 for fp16 and fp32 up to
+    W = 4, else 4; units = rows x ceil(ceil(L / 32V) / U); grid =
+    min(ceil(units / 8), 148 x 3)."""
+    import numpy as np
+    rng = np.random.default_rng(11)
+    for _ in range(300):
+        io = [F32, F16, BF16][rng.integers(3)]
+        Bn, D = int(rng.integers(1, 5)), int(rng.integers(1, 300))
+        L, W = int(rng.integers(1, 5000)), int(rng.integers(1, 9))
+        st, info = call(lib, "ssm_causal_conv1d_fwd", conv_args(FakeMem(), Bn=Bn, D=D, L=L, W=W, io=io))
+        assert st == OK
+        V = 4 if io == F32 else 8
+        rows = Bn * D
+        if L % V or W - 1 > V:
+            assert bd.KERNELS[info.kernel] == "conv1d_generic", (io, Bn, D, L, W)
+            continue
+        U = 8 if io in (F32, F16) and W <= 4 else 4
+        units = rows * (-(-(-(-L // (32 * V))) // U))
+        assert bd.KERNELS[info.kernel] == "conv1d", (io, Bn, D, L, W)
+        assert info.work_items == units and info.grid == min(-(-units // 8), 148 * 3), (io, Bn, D, L, W)
+
+
 # ------------------------------------------------------------ error paths --
 def test_null_args_and_version(lib):
     for fn in ("ssm_causal_conv1d_fwd", "ssm_selective_scan_fwd", "ssm_selective_state_update"):
